@@ -1,0 +1,509 @@
+#!/usr/bin/env python
+"""Benchmark of the CSA/HCA attention layer on B200 (one JSON line on rank 0).
+
+Headline: CSA prefill of one layer at n = 65536 tokens (c = 512, m = 4,
+64 indexer heads x 128, top-k 512, 64 query heads, window 128, bf16), one
+step = compress (KV) + compress (index keys) + indexer/top-k + sparse
+attention, reported as query-tokens/s.  The same line carries the HCA
+prefill layer (n = 16384, m = 128) and the two decode workloads (batch 64 at
+context 131072; batch 4 at context 1048576 with one CSA and one HCA layer)
+under "workloads", each with its roofline.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
+
+--impl reference times the fp64 CPU oracle on the host cores on a bounded
+sample of the same workload.  Several GPUs run independent replicas (the
+layer is run on one GPU; no data-path collective), timed as the max over
+ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import torch  # noqa: E402
+
+import csa_inputs as G  # noqa: E402
+
+METRIC = "CSA prefill query-tokens/s (n=65536, c=512, top-k 512)"
+UNIT = "tokens/s"
+
+
+# ----------------------------------------------------------------- helpers ---
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return dict(hbm_gbs=d["hbm_gbs"], bf16=d["bf16_tflops"],
+                    bf16_sustained=d["bf16_tflops_sustained"], source="measured")
+    return dict(hbm_gbs=6650.0, bf16=1590.0, bf16_sustained=1400.0, source="fallback")
+
+
+def sum_visible(n, m, E=None):
+    """sum over t < n of min(floor((t+1)/m), E)."""
+    E = n // m if E is None else E
+    return sum(min((t + 1) // m, E) for t in range(n))
+
+
+def sum_entry_sets(n, m, k, window):
+    """sum over t of |E_t| = min(k, V(t)) + min(t+1, W) (k=None: dense)."""
+    tot = 0
+    for t in range(n):
+        V = (t + 1) // m
+        tot += (V if k is None else min(k, V)) + min(t + 1, window)
+    return tot
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle-reason samples during a timed region."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device):
+        self.device = device
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        try:
+            uuid = str(torch.cuda.get_device_properties(self.device).uuid)
+            sel = ["-i", uuid if uuid.startswith("GPU-") else "GPU-" + uuid]
+        except Exception:
+            sel = []
+        fd, self.path = tempfile.mkstemp(suffix=".csv")
+        os.close(fd)
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", *sel, f"--query-gpu={self.FIELDS}", "--format=csv,noheader",
+                 "-lms", "100"], stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+        time.sleep(0.3)
+
+    def stop(self):
+        if self.proc is None:
+            return {"error": "nvidia-smi unavailable"}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        rows = []
+        with open(self.path) as f:
+            for line in f:
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) >= 9:
+                    rows.append(parts)
+        os.unlink(self.path)
+        if not rows:
+            return {"error": "no samples"}
+        sm = [float(r[1].split()[0]) for r in rows if r[1].split()[0].replace(".", "").isdigit()]
+        mx = [float(r[2].split()[0]) for r in rows if r[2].split()[0].replace(".", "").isdigit()]
+        names = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i] == "Active"})
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(mx) if mx else None, "reasons": reasons,
+                "samples": len(rows)}
+
+
+def dist_setup():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                device_id=torch.device("cuda", local))
+    else:
+        torch.cuda.set_device(local)
+    return rank, world, local
+
+
+def max_over_ranks(x: float, world: int) -> float:
+    if world == 1:
+        return x
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+    torch.cuda.synchronize()
+
+
+# ------------------------------------------------------- CSA prefill layer ---
+
+class CsaPrefill:
+    """All device buffers of one CSA prefill layer call; step() runs it."""
+
+    def __init__(self, w: G.Prefill, dev):
+        import compressed_sparse_attention_11_b200 as csa
+        self.csa, self.w, self.dev = csa, w, dev
+        self.host = G.prefill_inputs(w)
+        self.d = {k: v.to(dev) for k, v in self.host.items()}
+        B, n, E = w.batch, w.n, w.n // w.m
+        self.kv = torch.empty((B, E, w.c), dtype=w.dtype, device=dev)
+        self.ki = torch.empty((B, E, w.c_i), dtype=w.dtype, device=dev)
+        self.idx = torch.empty((B, n, w.k), dtype=torch.int32, device=dev)
+        self.out = torch.empty_like(self.d["q"])
+        nb = csa.csa_index_topk_workspace(B, n, w.nh_i, w.c_i, w.m, w.k)
+        self.ws = torch.empty(max(nb, 16), dtype=torch.uint8, device=dev)
+        self.calls = ("compress_kv", "compress_index_keys", "index_topk", "sparse_attn")
+        self.launches_per_step = 5   # compress x2, index scores, top-k rows, attention
+
+    def step(self, ev=None):
+        c, d, w = self.csa, self.d, self.w
+        if ev: ev[0].record()
+        c.csa_compress(d["ca"], d["cb"], d["za"], d["zb"], d["ba"], d["bb"], w.m, out=self.kv)
+        if ev: ev[1].record()
+        c.csa_compress(d["ica"], d["icb"], d["iza"], d["izb"], d["iba"], d["ibb"], w.m,
+                       out=self.ki)
+        if ev: ev[2].record()
+        c.csa_index_topk(d["q_i"], d["w_i"], self.ki, w.m, w.k, ws=self.ws, out=self.idx)
+        if ev: ev[3].record()
+        c.csa_sparse_attn(d["q"], self.kv, self.idx, d["kv_win"], w.window, d["sink"], w.scale,
+                          w.m, out=self.out)
+        if ev: ev[4].record()
+
+    def work(self):
+        """Algorithmic work per call: (kind, amount) with kind bytes or flops."""
+        w = self.w
+        elt = 2 if w.dtype == torch.bfloat16 else 4
+        n, E = w.n, w.n // w.m
+        sv = sum_visible(n, w.m)
+        se = sum_entry_sets(n, w.m, w.k, w.window)
+        return {
+            "compress_kv": ("bytes", 4 * n * w.c * elt + E * w.c * elt + 2 * w.m * w.c * 4),
+            "compress_index_keys": ("bytes", 4 * n * w.c_i * elt + E * w.c_i * elt),
+            "index_topk": ("flops", 2 * w.nh_i * w.c_i * sv),
+            "sparse_attn": ("flops", 4 * w.nh * w.c * se),
+        }
+
+    def h2d_inputs(self, pinned):
+        for k, v in pinned.items():
+            self.d[k].copy_(v, non_blocking=True)
+
+
+def time_steps(step_fn, ncalls, K, world, dev):
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(ncalls + 1)] for _ in range(K)]
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier(world)
+    start.record()
+    for i in range(K):
+        step_fn(evs[i])
+    end.record()
+    torch.cuda.synchronize()
+    total = start.elapsed_time(end)
+    per_call = [sum(evs[i][j].elapsed_time(evs[i][j + 1]) for i in range(K)) / K
+                for j in range(ncalls)]
+    return total, per_call
+
+
+def roofline(kind, amount, ms, peaks):
+    if kind == "bytes":
+        ach = amount / (ms * 1e-3) / 1e9
+        return {"bound": "hbm", "achieved": round(ach, 1), "peak": peaks["hbm_gbs"],
+                "unit": "GB/s", "frac": round(ach / peaks["hbm_gbs"], 4),
+                "algorithmic": amount, "peak_source": peaks["source"] + " hbm_gbs"}
+    ach = amount / (ms * 1e-3) / 1e12
+    pk = peaks["bf16_sustained"]
+    return {"bound": "tensor", "achieved": round(ach, 2), "peak": pk, "unit": "TFLOP/s",
+            "frac": round(ach / pk, 4), "algorithmic": amount,
+            "peak_source": peaks["source"] + " bf16_tflops_sustained"}
+
+
+# ------------------------------------------------------------ other layers ---
+
+def bench_hca_prefill(dev, K, W, peaks):
+    import compressed_sparse_attention_11_b200 as csa
+    w = G.HCA_PREFILL
+    h = G.prefill_inputs(w)
+    d = {k: v.to(dev) for k, v in h.items()}
+    kv = torch.empty((w.batch, w.n // w.m, w.c), dtype=w.dtype, device=dev)
+    out = torch.empty_like(d["q"])
+
+    def step(ev):
+        ev[0].record()
+        csa.csa_compress(d["ca"], None, d["za"], None, d["ba"], None, w.m, out=kv)
+        ev[1].record()
+        csa.hca_attn(d["q"], kv, d["kv_win"], w.window, d["sink"], w.scale, w.m, out=out)
+        ev[2].record()
+
+    for _ in range(W):
+        step([torch.cuda.Event(enable_timing=True) for _ in range(3)])
+    total, per = time_steps(step, 2, K, 1, dev)
+    ms = total / K
+    elt = 2
+    comp_bytes = 2 * w.n * w.c * elt + (w.n // w.m) * w.c * elt
+    attn_flops = 4 * w.nh * w.c * sum_entry_sets(w.n, w.m, None, w.window)
+    return {"workload": w.name, "metric": "query-tokens/s", "value": round(w.n / (ms * 1e-3), 1),
+            "ms_per_step": round(ms, 4), "calls_ms": {"compress": round(per[0], 4),
+                                                      "hca_attn": round(per[1], 4)},
+            "roofline": {"compress": roofline("bytes", comp_bytes, per[0], peaks),
+                         "hca_attn": roofline("flops", attn_flops, per[1], peaks)}}
+
+
+def _decode_layer(w: G.Decode, dev, steps):
+    import compressed_sparse_attention_11_b200 as csa
+    inp = G.decode_inputs(w, steps=steps)
+    E = w.t // w.m
+    cache = csa.CsaCache(w.batch, E + steps // w.m + 2, w.c, w.rope_dims, w.m, w.window, w.nh,
+                         w.is_hca, c_i=w.c_i, nh_i=w.nh_i, k=w.k, device=dev)
+    cache.store_entries(0, inp["cache_kv"].to(dev),
+                        None if w.is_hca else inp["cache_ikey"].to(dev))
+    names = ("ca", "za", "kv_win") if w.is_hca else \
+        ("ca", "cb", "za", "zb", "ica", "icb", "iza", "izb", "kv_win")
+    tail = w.window + 2 * w.m
+    cache.write_rows(w.t - tail, {nm: inp["rows_" + nm][:, :tail].contiguous().to(dev)
+                                  for nm in names})
+    bias_keys = ("ba",) if w.is_hca else ("ba", "bb", "iba", "ibb")
+    per_step = []
+    for s in range(steps):
+        per_step.append(dict(
+            pos=torch.full((w.batch,), w.t + s, dtype=torch.int64, device=dev),
+            rows={nm: inp["rows_" + nm][:, tail + s].contiguous().to(dev) for nm in names},
+            q=inp["q"][s].to(dev),
+            q_i=None if w.is_hca else inp["q_i"][s].to(dev),
+            w_i=None if w.is_hca else inp["w_i"][s].to(dev)))
+    biases = {k: inp[k].to(dev) for k in bias_keys}
+    sink = inp["sink"].to(dev)
+    out = torch.empty((w.batch, w.nh, w.c), dtype=torch.bfloat16, device=dev)
+    del inp
+    return cache, per_step, biases, sink, out
+
+
+def decode_bytes(w: G.Decode, t: int):
+    """Algorithmic HBM bytes of one decode step at position t (all sequences)."""
+    B, c, rope = w.batch, w.c, w.rope_dims
+    V = (t + 1) // w.m
+    entry = (c - rope) + 4 + 2 * rope
+    win = min(t + 1, w.window) * c * 2
+    qo = 2 * w.nh * c * 2
+    rows = (2 if w.is_hca else 4) * c * 2 + c * 2
+    if w.is_hca:
+        return B * (V * entry + win + qo + rows)
+    ikey = w.c_i + 4
+    return B * (V * ikey + min(w.k, V) * entry + win + qo + rows + w.nh_i * (w.c_i * 2 + 4)
+                + 4 * w.c_i * 2)
+
+
+def bench_decode(layers, dev, K, W, peaks, name):
+    """Times `steps` consecutive decode positions (the last one emits), L2 flushed."""
+    steps = 4
+    built = [_decode_layer(w, dev, steps) for w in layers]
+    flush = torch.empty(512 << 20, dtype=torch.uint8, device=dev)
+    times = []
+    for it in range(W + K):
+        for s in range(steps):
+            flush.zero_()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            for w, (cache, ps, biases, sink, out) in zip(layers, built):
+                st = ps[s]
+                cache.decode_step(st["pos"], st["rows"], biases, sink, w.scale, st["q"],
+                                  st["q_i"], st["w_i"], out=out)
+            e1.record()
+            torch.cuda.synchronize()
+            if it >= W:
+                times.append(e0.elapsed_time(e1))
+    us = [1000 * t for t in times]
+    mean_us = statistics.mean(us)
+    nbytes = statistics.mean(sum(decode_bytes(w, w.t + s) for w in layers)
+                             for s in range(steps))
+    rl = roofline("bytes", nbytes, mean_us / 1000, peaks)
+    return {"workload": name, "metric": "decode us/step", "value": round(mean_us, 2),
+            "max_us": round(max(us), 2), "steps_timed": len(us), "l2": "flushed before each step",
+            "roofline": rl}
+
+
+# -------------------------------------------------------------- CPU oracle ---
+
+def oracle_sample(budget_s=12.0):
+    """Times the fp64 oracle on a bounded sample of the CSA prefill workload.
+
+    Compresses the whole sequence (KV and index keys), then runs index
+    scores, top-k and attention for strided query rows until the budget is
+    spent.  Returns seconds per query token extrapolated to the workload."""
+    import numpy as np
+    import oracle as O
+    try:
+        from threadpoolctl import threadpool_info
+        threads = max([p.get("num_threads", 1) for p in threadpool_info()] or [1])
+    except Exception:
+        threads = os.cpu_count() or 1
+    w = G.CSA_PREFILL
+    inp = G.prefill_inputs(w)
+    b = 0
+    t0 = time.perf_counter()
+    kv = O.csa_compress(inp["ca"][b], inp["cb"][b], inp["za"][b], inp["zb"][b], inp["ba"],
+                        inp["bb"], w.m)
+    ki = O.csa_compress(inp["ica"][b], inp["icb"][b], inp["iza"][b], inp["izb"][b], inp["iba"],
+                        inp["ibb"], w.m)
+    t_comp = time.perf_counter() - t0
+    rows = list(range(w.n - 1, 0, -(w.n // 64)))    # strided, from the longest row down
+    order = [rows[i] for i in np.random.default_rng(0).permutation(len(rows))]
+    done, t1 = [], time.perf_counter()
+    for t in order:
+        V = O.visible(t, w.m)
+        sc = O.index_scores_row(inp["q_i"][b, t], inp["w_i"][b, t], ki, V)
+        sel = O.topk_row(sc, w.k)
+        Et = O.sparse_entry_set(kv, sel, inp["kv_win"][b], t, w.m, w.window)
+        O.attend(inp["q"][b, t], Et, inp["sink"], w.scale)
+        done.append(t)
+        if time.perf_counter() - t1 > budget_s and len(done) >= 8:
+            break
+    t_rows = time.perf_counter() - t1
+    # rows are sampled uniformly over positions, so their mean cost estimates
+    # the mean over all n rows
+    per_token = t_comp / w.n + t_rows / len(done)
+    return {"value": round(1.0 / per_token, 3), "unit": UNIT, "cores": threads,
+            "kind": "oracle",
+            "sample": f"full compression of both streams ({t_comp:.1f} s) + index/top-k/"
+                      f"attention of {len(done)} strided query rows ({t_rows:.1f} s), "
+                      f"extrapolated to n={w.n}"}
+
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    t0 = time.perf_counter()
+    cb = oracle_sample(budget_s=max(5.0, 20.0 / max(1, args.steps)))
+    elapsed = time.perf_counter() - t0
+    line = {"impl": "reference", "metric": METRIC, "value": cb["value"], "unit": UNIT,
+            "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": round(G.CSA_PREFILL.n / cb["value"] * 1000, 1),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic", "config": {"workload": G.CSA_PREFILL.name,
+                                            "seq_len": G.CSA_PREFILL.n, "batch": 1},
+            "cpu_baseline": cb,
+            "e2e": {"value": cb["value"], "unit": UNIT, "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0},
+            "wall_s": round(elapsed, 1)}
+    print(json.dumps(line), flush=True)
+
+
+# -------------------------------------------------------------------- main ---
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=5)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", default="ours", choices=("ours", "reference"))
+    ap.add_argument("--skip-extras", action="store_true", help="headline workload only")
+    ap.add_argument("--skip-cpu", action="store_true", help="no oracle timing")
+    args = ap.parse_args()
+    if args.impl == "reference":
+        run_reference(args)
+        return
+    rank, world, local = dist_setup()
+    dev = torch.device("cuda", local)
+    import compressed_sparse_attention_11_b200 as csa
+    csa.lib()
+    peaks = load_peaks()
+    w = G.CSA_PREFILL
+    L = CsaPrefill(w, dev)
+    ncalls = len(L.calls)
+    for _ in range(args.warmup):
+        L.step()
+    torch.cuda.synchronize()
+    clk = ClockSampler(dev)
+    clk.start()
+    total, per_call = time_steps(L.step, ncalls, args.steps, world, dev)
+    clocks = clk.stop()
+    total = max_over_ranks(total, world)
+    ms = total / args.steps
+    value = w.n * w.batch * world / (ms * 1e-3)
+    work = L.work()
+    calls = {name: round(t, 4) for name, t in zip(L.calls, per_call)}
+    roof = {name: roofline(*work[name], per_call[i], peaks) for i, name in enumerate(L.calls)}
+    dom = max(range(ncalls), key=lambda i: per_call[i])
+    dominant = dict(roof[L.calls[dom]])
+    dominant["kernel"] = L.calls[dom]
+    dominant["traffic"] = None
+
+    # end to end: pinned host inputs -> device, layer, output -> host, every step
+    pinned = {k: v.pin_memory() for k, v in L.host.items()}
+    out_host = torch.empty(L.out.shape, dtype=L.out.dtype, pin_memory=True)
+    h2d = sum(v.numel() * v.element_size() for v in pinned.values())
+    d2h = out_host.numel() * out_host.element_size()
+
+    def e2e_step(ev=None):
+        L.h2d_inputs(pinned)
+        L.step()
+        out_host.copy_(L.out, non_blocking=True)
+
+    e2e_step()
+    torch.cuda.synchronize()
+    e2e_total, _ = time_steps(lambda ev: e2e_step(), 0, max(2, args.steps // 2), world, dev)
+    e2e_total = max_over_ranks(e2e_total, world)
+    e2e_ms = e2e_total / max(2, args.steps // 2)
+    del pinned, out_host
+
+    workloads = {}
+    if not args.skip_extras:
+        del L
+        torch.cuda.empty_cache()
+        workloads["hca_prefill"] = bench_hca_prefill(dev, args.steps, args.warmup, peaks)
+        torch.cuda.empty_cache()
+        workloads["csa_decode"] = bench_decode([G.CSA_DECODE], dev, max(2, args.steps // 2),
+                                               1, peaks, G.CSA_DECODE.name)
+        torch.cuda.empty_cache()
+        workloads["mixed_decode"] = bench_decode([G.MIXED_DECODE_CSA, G.MIXED_DECODE_HCA], dev,
+                                                 max(2, args.steps // 2), 1, peaks,
+                                                 "mixed_decode_b4_ctx1048576_csa+hca")
+    cpu = None
+    if rank == 0 and not args.skip_cpu:
+        cpu = oracle_sample()
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": round(value, 1), "unit": UNIT, "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 4),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic",
+            "config": {"workload": w.name, "seq_len": w.n, "batch": w.batch, "c": w.c,
+                       "m": w.m, "top_k": w.k, "heads": w.nh, "index_heads": w.nh_i,
+                       "index_dim": w.c_i, "window": w.window,
+                       "parallelism": f"replicas x{world}",
+                       "l2": "inputs (5.8 GB) larger than L2"},
+            "calls_ms": calls,
+            "roofline": dominant,
+            "roofline_per_call": roof,
+            "gpu_launches": 5 * args.steps,
+            "e2e": {"value": round(w.n * w.batch * world / (e2e_ms * 1e-3), 1), "unit": UNIT,
+                    "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                    "ms_per_step": round(e2e_ms, 3)},
+            "clocks": clocks,
+            "cpu_baseline": cpu,
+            "workloads": workloads,
+            "peaks": peaks,
+        }
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,266 @@
+"""Python binding of libcsa.so, the CSA/HCA attention layer for one B200.
+
+Argument marshalling only: every function here checks tensor shapes, dtypes
+and devices, passes raw device pointers and the current CUDA stream to the C
+ABI declared in ``include/csa.h`` and raises ``CsaError`` on a non-OK status.
+All arithmetic runs in the library's CUDA kernels; there is no fallback.
+
+The functions carry the C names: ``csa_compress``, ``csa_index_topk``,
+``csa_sparse_attn``, ``hca_attn`` and the decode-cache calls
+(``CsaCache`` wraps ``csa_cache_layout`` / ``csa_cache_store_entries`` /
+``csa_cache_write_rows`` / ``csa_decode_step``).
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libcsa.so")
+
+CSA_OK, CSA_ERR_INVALID_ARG, CSA_ERR_UNSUPPORTED, CSA_ERR_WORKSPACE, CSA_ERR_CUDA, \
+    CSA_ERR_TIMEOUT = 0, -1, -2, -3, -4, -5
+CSA_F32, CSA_BF16 = 0, 1
+
+EXPORTED = (
+    "csa_status_string", "csa_last_error", "csa_abi_version", "csa_compress",
+    "csa_index_topk_workspace", "csa_index_topk", "csa_sparse_attn", "hca_attn",
+    "csa_cache_layout", "csa_cache_store_entries", "csa_cache_write_rows",
+    "csa_decode_workspace", "csa_decode_step",
+)
+
+
+class CsaError(RuntimeError):
+    def __init__(self, status: int, detail: str):
+        self.status = status
+        super().__init__(f"{status_string(status)}: {detail}")
+
+
+class CacheDesc(ctypes.Structure):
+    _fields_ = [("batch", ctypes.c_int64), ("capacity", ctypes.c_int64), ("c", ctypes.c_int32),
+                ("rope_dims", ctypes.c_int32), ("c_i", ctypes.c_int32), ("m", ctypes.c_int32),
+                ("window", ctypes.c_int32), ("nh", ctypes.c_int32), ("nh_i", ctypes.c_int32),
+                ("k", ctypes.c_int32), ("is_hca", ctypes.c_int32)]
+
+
+class CacheLayout(ctypes.Structure):
+    _fields_ = [(nm, ctypes.c_size_t) for nm in (
+        "entry_fp8", "entry_scale", "entry_rope", "ikey_fp8", "ikey_scale", "window", "state",
+        "istate", "total_bytes")]
+
+
+class Rows(ctypes.Structure):
+    _fields_ = [(nm, ctypes.c_void_p) for nm in (
+        "ca", "cb", "za", "zb", "ica", "icb", "iza", "izb", "kv_win")]
+
+
+class DecodeParams(ctypes.Structure):
+    _fields_ = [("ba", ctypes.c_void_p), ("bb", ctypes.c_void_p), ("iba", ctypes.c_void_p),
+                ("ibb", ctypes.c_void_p), ("sink", ctypes.c_void_p), ("scale", ctypes.c_float)]
+
+
+_lib = None
+
+
+def lib() -> ctypes.CDLL:
+    """The loaded libcsa.so (raises if it has not been built)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(f"{LIB_PATH} is missing: build it with "
+                          "`python -m compressed_sparse_attention_11_b200.build`")
+    L = ctypes.CDLL(LIB_PATH)
+    vp, i64, i32, sz, f32 = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int, ctypes.c_size_t, \
+        ctypes.c_float
+    sig = {
+        "csa_status_string": (ctypes.c_char_p, [i32]),
+        "csa_last_error": (ctypes.c_char_p, []),
+        "csa_abi_version": (i32, []),
+        "csa_compress": (i32, [vp, vp, vp, vp, vp, vp, i64, i64, i32, i32, i32, i32, vp, vp]),
+        "csa_index_topk_workspace": (sz, [i64, i64, i32, i32, i32, i32]),
+        "csa_index_topk": (i32, [vp, vp, vp, i64, i64, i32, i32, i32, i32, i32, vp, vp, sz, vp]),
+        "csa_sparse_attn": (i32, [vp, vp, vp, i32, vp, i32, vp, f32, i64, i64, i32, i32, i32,
+                                  i32, vp, vp]),
+        "hca_attn": (i32, [vp, vp, vp, i32, vp, f32, i64, i64, i32, i32, i32, i32, vp, vp]),
+        "csa_cache_layout": (i32, [ctypes.POINTER(CacheDesc), ctypes.POINTER(CacheLayout)]),
+        "csa_cache_store_entries": (i32, [ctypes.POINTER(CacheDesc), vp, i64, i64, vp, vp, i32,
+                                          vp]),
+        "csa_cache_write_rows": (i32, [ctypes.POINTER(CacheDesc), vp, i64, i64,
+                                       ctypes.POINTER(Rows), vp]),
+        "csa_decode_workspace": (sz, [ctypes.POINTER(CacheDesc)]),
+        "csa_decode_step": (i32, [ctypes.POINTER(CacheDesc), vp, vp, ctypes.POINTER(Rows),
+                                  ctypes.POINTER(DecodeParams), vp, vp, vp, vp, vp, sz, vp]),
+    }
+    for name, (res, args) in sig.items():
+        fn = getattr(L, name)
+        fn.restype = res
+        fn.argtypes = args
+    _lib = L
+    return L
+
+
+def status_string(status: int) -> str:
+    return lib().csa_status_string(int(status)).decode()
+
+
+def _check(status: int):
+    if status != CSA_OK:
+        raise CsaError(status, lib().csa_last_error().decode())
+
+
+def _dt(t: torch.Tensor) -> int:
+    if t.dtype == torch.float32:
+        return CSA_F32
+    if t.dtype == torch.bfloat16:
+        return CSA_BF16
+    raise ValueError(f"unsupported dtype {t.dtype}; use float32 or bfloat16")
+
+
+def _ptr(t: Optional[torch.Tensor]) -> Optional[int]:
+    if t is None:
+        return None
+    if not t.is_cuda:
+        raise ValueError("tensors must live on a CUDA device")
+    if not t.is_contiguous():
+        raise ValueError("tensors must be contiguous")
+    return t.data_ptr()
+
+
+def _stream(t: torch.Tensor) -> int:
+    return torch.cuda.current_stream(t.device).cuda_stream
+
+
+# ------------------------------------------------------------------ prefill ---
+
+def csa_compress(ca, cb, za, zb, ba, bb, m: int, out: Optional[torch.Tensor] = None):
+    """Compress [B, n, c] streams into [B, n//m, c] entries.
+
+    CSA (overlapped) when ``cb`` is given, HCA (single stream) when ``cb``,
+    ``zb`` and ``bb`` are None.
+    """
+    overlap = 1 if cb is not None else 0
+    B, n, c = ca.shape
+    if out is None:
+        out = torch.empty((B, n // m, c), dtype=ca.dtype, device=ca.device)
+    _check(lib().csa_compress(_ptr(ca), _ptr(cb), _ptr(za), _ptr(zb), _ptr(ba), _ptr(bb), B, n,
+                              c, m, overlap, _dt(ca), _ptr(out), _stream(ca)))
+    return out
+
+
+def csa_index_topk_workspace(batch: int, n: int, nh_i: int, c_i: int, m: int, k: int) -> int:
+    return int(lib().csa_index_topk_workspace(batch, n, nh_i, c_i, m, k))
+
+
+def csa_index_topk(q_i, w_i, k_i, m: int, k: int, ws: Optional[torch.Tensor] = None,
+                   out: Optional[torch.Tensor] = None):
+    """Top-k entry indices [B, n, k] int32 (ascending, -1 padded)."""
+    B, n, H, ci = q_i.shape
+    need = csa_index_topk_workspace(B, n, H, ci, m, k)
+    if ws is None:
+        ws = torch.empty(max(need, 16), dtype=torch.uint8, device=q_i.device)
+    if out is None:
+        out = torch.empty((B, n, k), dtype=torch.int32, device=q_i.device)
+    _check(lib().csa_index_topk(_ptr(q_i), _ptr(w_i), _ptr(k_i), B, n, H, ci, m, k, _dt(q_i),
+                                _ptr(out), _ptr(ws), ws.numel() * ws.element_size(),
+                                _stream(q_i)))
+    return out
+
+
+def csa_sparse_attn(q, kv_comp, idx, kv_win, window: int, sink, scale: float, m: int,
+                    out: Optional[torch.Tensor] = None):
+    B, n, nh, c = q.shape
+    if out is None:
+        out = torch.empty_like(q)
+    _check(lib().csa_sparse_attn(_ptr(q), _ptr(kv_comp), _ptr(idx), idx.shape[-1], _ptr(kv_win),
+                                 window, _ptr(sink), float(scale), B, n, nh, c, m, _dt(q),
+                                 _ptr(out), _stream(q)))
+    return out
+
+
+def hca_attn(q, kv_comp, kv_win, window: int, sink, scale: float, m_heavy: int,
+             out: Optional[torch.Tensor] = None):
+    B, n, nh, c = q.shape
+    if out is None:
+        out = torch.empty_like(q)
+    _check(lib().hca_attn(_ptr(q), _ptr(kv_comp), _ptr(kv_win), window, _ptr(sink), float(scale),
+                          B, n, nh, c, m_heavy, _dt(q), _ptr(out), _stream(q)))
+    return out
+
+
+# ------------------------------------------------------------------- decode ---
+
+class CsaCache:
+    """A caller-owned decode cache (one layer, ``batch`` sequences)."""
+
+    def __init__(self, batch: int, capacity: int, c: int, rope_dims: int, m: int, window: int,
+                 nh: int, is_hca: bool, c_i: int = 0, nh_i: int = 0, k: int = 0,
+                 device="cuda"):
+        self.desc = CacheDesc(batch, capacity, c, rope_dims, c_i, m, window, nh, nh_i, k,
+                              1 if is_hca else 0)
+        self.layout = CacheLayout()
+        _check(lib().csa_cache_layout(ctypes.byref(self.desc), ctypes.byref(self.layout)))
+        self.buffer = torch.zeros(self.layout.total_bytes, dtype=torch.uint8, device=device)
+        ws = int(lib().csa_decode_workspace(ctypes.byref(self.desc)))
+        self.workspace = torch.empty(max(ws, 16), dtype=torch.uint8, device=device)
+
+    # views of the regions (for tests and inspection)
+    def region(self, name: str, dtype, shape):
+        off = getattr(self.layout, name)
+        nbytes = int(torch.tensor(shape).prod().item()) * torch.empty((), dtype=dtype).element_size()
+        return self.buffer[off:off + nbytes].view(dtype).view(*shape)
+
+    def entries(self):
+        d = self.desc
+        B, cap = d.batch, d.capacity
+        out = dict(codes=self.region("entry_fp8", torch.uint8, (B, cap, d.c - d.rope_dims)),
+                   scale=self.region("entry_scale", torch.float32, (B, cap)),
+                   rope=self.region("entry_rope", torch.bfloat16, (B, cap, d.rope_dims)))
+        if not d.is_hca:
+            out["icodes"] = self.region("ikey_fp8", torch.uint8, (B, cap, d.c_i))
+            out["iscale"] = self.region("ikey_scale", torch.float32, (B, cap))
+        return out
+
+    def store_entries(self, first: int, kv, ikey=None):
+        count = kv.shape[1]
+        _check(lib().csa_cache_store_entries(ctypes.byref(self.desc), _ptr(self.buffer), first,
+                                             count, _ptr(kv), _ptr(ikey), _dt(kv),
+                                             _stream(self.buffer)))
+
+    @staticmethod
+    def _rows(rows: dict) -> Rows:
+        r = Rows()
+        for nm in ("ca", "cb", "za", "zb", "ica", "icb", "iza", "izb", "kv_win"):
+            t = rows.get(nm)
+            if t is not None and t.dtype != torch.bfloat16:
+                raise ValueError(f"row stream {nm} must be bfloat16")
+            setattr(r, nm, _ptr(t))
+        return r
+
+    def write_rows(self, first_pos: int, rows: dict):
+        count = rows["kv_win"].shape[1]
+        r = self._rows(rows)
+        _check(lib().csa_cache_write_rows(ctypes.byref(self.desc), _ptr(self.buffer), first_pos,
+                                          count, ctypes.byref(r), _stream(self.buffer)))
+
+    def decode_step(self, pos, rows: dict, biases: dict, sink, scale: float, q, q_i=None,
+                    w_i=None, out: Optional[torch.Tensor] = None):
+        """One token per sequence at positions ``pos`` (int64 [B] on device).
+
+        ``rows``: per-stream [B, dim] bf16 tensors; ``biases``: ba, bb, iba, ibb
+        fp32; returns out [B, nh, c] bf16."""
+        if out is None:
+            out = torch.empty_like(q)
+        r = self._rows({k: v for k, v in rows.items()})
+        p = DecodeParams(_ptr(biases.get("ba")), _ptr(biases.get("bb")), _ptr(biases.get("iba")),
+                         _ptr(biases.get("ibb")), _ptr(sink), float(scale))
+        if pos.dtype != torch.int64:
+            raise ValueError("pos must be int64")
+        _check(lib().csa_decode_step(ctypes.byref(self.desc), _ptr(self.buffer), _ptr(pos),
+                                     ctypes.byref(r), ctypes.byref(p), _ptr(q), _ptr(q_i),
+                                     _ptr(w_i), _ptr(out), _ptr(self.workspace),
+                                     self.workspace.numel(), _stream(q)))
+        return out

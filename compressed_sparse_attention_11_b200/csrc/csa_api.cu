@@ -1,0 +1,297 @@
+// C ABI of the CSA/HCA attention layer: argument checks, then launches.
+// Every entry point validates before enqueuing anything on the stream and
+// never allocates, frees or synchronises.
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+
+#include "common.cuh"
+#include "launch.h"
+
+using namespace csa;
+
+namespace {
+
+thread_local char g_err[512] = "";
+
+csa_status fail(csa_status st, const char* fmt, ...) {
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(g_err, sizeof(g_err), fmt, ap);
+  va_end(ap);
+  return st;
+}
+
+csa_status ok() {
+  g_err[0] = '\0';
+  return CSA_OK;
+}
+
+csa_status cuda_status(cudaError_t e, const char* where) {
+  if (e == cudaSuccess) return ok();
+  return fail(CSA_ERR_CUDA, "%s: %s", where, cudaGetErrorString(e));
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+#define REQUIRE(cond, ...) \
+  do { if (!(cond)) return fail(CSA_ERR_INVALID_ARG, __VA_ARGS__); } while (0)
+#define REQUIRE_PTR(p) \
+  do { \
+    if ((p) == nullptr) return fail(CSA_ERR_INVALID_ARG, "%s is NULL", #p); \
+    if (!aligned16(p)) return fail(CSA_ERR_INVALID_ARG, "%s is not 16-byte aligned", #p); \
+  } while (0)
+#define REQUIRE_OPT_PTR(p) \
+  do { \
+    if ((p) != nullptr && !aligned16(p)) \
+      return fail(CSA_ERR_INVALID_ARG, "%s is not 16-byte aligned", #p); \
+  } while (0)
+
+bool valid_dt(csa_dtype dt) { return dt == CSA_F32 || dt == CSA_BF16; }
+
+constexpr size_t kMaxSmem = 227 * 1024;
+
+csa_status check_attn_common(const void* q, const void* kv_comp, const void* kv_win, int window,
+                             float scale, int64_t batch, int64_t n, int nh, int c, int m,
+                             csa_dtype dt, const void* out, const float* sink) {
+  REQUIRE(valid_dt(dt), "dt must be CSA_F32 or CSA_BF16");
+  REQUIRE(batch >= 0 && n >= 0, "batch and n must be >= 0");
+  REQUIRE(nh >= 1, "nh must be >= 1");
+  REQUIRE(c >= 8 && c % 8 == 0, "c must be a positive multiple of 8");
+  REQUIRE(m >= 1, "m must be >= 1");
+  REQUIRE(window >= 1, "window must be >= 1");
+  REQUIRE(scale == scale && scale > -3.4e38f && scale < 3.4e38f, "scale must be finite");
+  if (batch == 0 || n == 0) return ok();
+  REQUIRE_PTR(q);
+  REQUIRE_PTR(kv_win);
+  REQUIRE_PTR(out);
+  REQUIRE_OPT_PTR(sink);
+  if (n / m > 0) REQUIRE_PTR(kv_comp);
+  if (c % 32 != 0 || c > 512) return fail(CSA_ERR_UNSUPPORTED, "attention needs c %% 32 == 0 and c <= 512");
+  return ok();
+}
+
+csa_status check_desc(const csa_cache_desc* d) {
+  REQUIRE(d != nullptr, "desc is NULL");
+  REQUIRE(d->batch >= 1 && d->capacity >= 1, "batch and capacity must be >= 1");
+  REQUIRE(d->c >= 32 && d->c % 32 == 0, "c must be a positive multiple of 32");
+  REQUIRE(d->rope_dims >= 0 && d->rope_dims < d->c && d->rope_dims % 8 == 0,
+          "rope_dims must be in [0, c) and a multiple of 8");
+  REQUIRE((d->c - d->rope_dims) % 16 == 0, "c - rope_dims must be a multiple of 16");
+  REQUIRE(d->m >= 1, "m must be >= 1");
+  REQUIRE(d->window >= 1, "window must be >= 1");
+  REQUIRE(d->nh >= 1, "nh must be >= 1");
+  REQUIRE(d->is_hca == 0 || d->is_hca == 1, "is_hca must be 0 or 1");
+  if (!d->is_hca) {
+    REQUIRE(d->c_i >= 16 && d->c_i % 16 == 0, "c_i must be a positive multiple of 16");
+    REQUIRE(d->nh_i >= 1, "nh_i must be >= 1");
+    REQUIRE(d->k >= 1, "k must be >= 1");
+  }
+  if (d->c > 512) return fail(CSA_ERR_UNSUPPORTED, "decode attention needs c <= 512");
+  return ok();
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* csa_status_string(int status) {
+  switch (status) {
+    case CSA_OK: return "CSA_OK";
+    case CSA_ERR_INVALID_ARG: return "CSA_ERR_INVALID_ARG";
+    case CSA_ERR_UNSUPPORTED: return "CSA_ERR_UNSUPPORTED";
+    case CSA_ERR_WORKSPACE: return "CSA_ERR_WORKSPACE";
+    case CSA_ERR_CUDA: return "CSA_ERR_CUDA";
+    case CSA_ERR_TIMEOUT: return "CSA_ERR_TIMEOUT";
+    default: return "CSA_ERR_UNKNOWN";
+  }
+}
+
+const char* csa_last_error(void) { return g_err; }
+
+int csa_abi_version(void) { return 1; }
+
+csa_status csa_compress(const void* ca, const void* cb, const void* za, const void* zb,
+                        const float* ba, const float* bb, int64_t batch, int64_t n, int c,
+                        int m, int overlap, csa_dtype dt, void* out, void* stream) {
+  REQUIRE(valid_dt(dt), "dt must be CSA_F32 or CSA_BF16");
+  REQUIRE(batch >= 0 && n >= 0, "batch and n must be >= 0");
+  REQUIRE(c >= 8 && c % 8 == 0, "c must be a positive multiple of 8");
+  REQUIRE(m >= 1, "m must be >= 1");
+  REQUIRE(overlap == 0 || overlap == 1, "overlap must be 0 or 1");
+  if (!overlap)
+    REQUIRE(cb == nullptr && zb == nullptr && bb == nullptr,
+            "cb, zb and bb must be NULL when overlap == 0");
+  if (batch == 0 || n / m == 0) return ok();
+  REQUIRE_PTR(ca);
+  REQUIRE_PTR(za);
+  REQUIRE_PTR(ba);
+  REQUIRE_PTR(out);
+  if (overlap) {
+    REQUIRE_PTR(cb);
+    REQUIRE_PTR(zb);
+    REQUIRE_PTR(bb);
+  }
+  return cuda_status(launch_compress(ca, cb, za, zb, ba, bb, batch, n, c, m, overlap, dt, out,
+                                     (cudaStream_t)stream),
+                     "csa_compress");
+}
+
+size_t csa_index_topk_workspace(int64_t batch, int64_t n, int nh_i, int c_i, int m, int k) {
+  (void)nh_i; (void)c_i; (void)k;
+  if (batch <= 0 || n <= 0 || m <= 0) return 0;
+  const int64_t E = n / m;
+  return (size_t)batch * (size_t)n * (size_t)E * sizeof(float);
+}
+
+csa_status csa_index_topk(const void* q_i, const float* w_i, const void* k_i, int64_t batch,
+                          int64_t n, int nh_i, int c_i, int m, int k, csa_dtype dt,
+                          int32_t* idx, void* ws, size_t ws_bytes, void* stream) {
+  REQUIRE(valid_dt(dt), "dt must be CSA_F32 or CSA_BF16");
+  REQUIRE(batch >= 0 && n >= 0, "batch and n must be >= 0");
+  REQUIRE(nh_i >= 1, "nh_i must be >= 1");
+  REQUIRE(c_i >= 8 && c_i % 8 == 0, "c_i must be a positive multiple of 8");
+  REQUIRE(m >= 1, "m must be >= 1");
+  REQUIRE(k >= 1, "k must be >= 1");
+  if (batch == 0 || n == 0) return ok();
+  REQUIRE_PTR(idx);
+  const int64_t E = n / m;
+  if (E > 0) {
+    REQUIRE_PTR(q_i);
+    REQUIRE_PTR(w_i);
+    REQUIRE_PTR(k_i);
+    const int nh_pad = (nh_i + 31) / 32 * 32;
+    if ((size_t)c_i * (128 + nh_pad) * 4 > kMaxSmem)
+      return fail(CSA_ERR_UNSUPPORTED, "indexer tile for c_i=%d, nh_i=%d exceeds shared memory",
+                  c_i, nh_i);
+    const size_t need = csa_index_topk_workspace(batch, n, nh_i, c_i, m, k);
+    if (ws_bytes < need || ws == nullptr)
+      return fail(CSA_ERR_WORKSPACE, "workspace %zu bytes < required %zu", ws_bytes, need);
+    REQUIRE_PTR(ws);
+  }
+  cudaStream_t s = (cudaStream_t)stream;
+  float* scores = static_cast<float*>(ws);
+  if (E > 0) {
+    cudaError_t e = launch_index_scores(q_i, w_i, k_i, batch, n, nh_i, c_i, m, dt, scores, E, s);
+    if (e != cudaSuccess) return cuda_status(e, "csa_index_topk (scores)");
+  }
+  return cuda_status(launch_topk_rows(scores, E, batch, n, m, E, k, idx, s),
+                     "csa_index_topk (top-k)");
+}
+
+csa_status csa_sparse_attn(const void* q, const void* kv_comp, const int32_t* idx, int k,
+                           const void* kv_win, int window, const float* sink, float scale,
+                           int64_t batch, int64_t n, int nh, int c, int m, csa_dtype dt,
+                           void* out, void* stream) {
+  REQUIRE(k >= 1, "k must be >= 1");
+  csa_status st = check_attn_common(q, kv_comp, kv_win, window, scale, batch, n, nh, c, m, dt,
+                                    out, sink);
+  if (st != CSA_OK || batch == 0 || n == 0) return st;
+  REQUIRE_PTR(idx);
+  return cuda_status(launch_attn(q, kv_comp, idx, k, kv_win, window, sink, scale, batch, n, nh,
+                                 c, m, dt, out, (cudaStream_t)stream),
+                     "csa_sparse_attn");
+}
+
+csa_status hca_attn(const void* q, const void* kv_comp, const void* kv_win, int window,
+                    const float* sink, float scale, int64_t batch, int64_t n, int nh, int c,
+                    int m_heavy, csa_dtype dt, void* out, void* stream) {
+  csa_status st = check_attn_common(q, kv_comp, kv_win, window, scale, batch, n, nh, c, m_heavy,
+                                    dt, out, sink);
+  if (st != CSA_OK || batch == 0 || n == 0) return st;
+  return cuda_status(launch_attn(q, kv_comp, nullptr, 0, kv_win, window, sink, scale, batch, n,
+                                 nh, c, m_heavy, dt, out, (cudaStream_t)stream),
+                     "hca_attn");
+}
+
+csa_status csa_cache_layout(const csa_cache_desc* desc, csa_cache_layout_t* layout) {
+  csa_status st = check_desc(desc);
+  if (st != CSA_OK) return st;
+  REQUIRE(layout != nullptr, "layout is NULL");
+  cache_layout(*desc, layout);
+  return ok();
+}
+
+csa_status csa_cache_store_entries(const csa_cache_desc* desc, void* cache, int64_t first,
+                                   int64_t count, const void* kv, const void* ikey,
+                                   csa_dtype dt, void* stream) {
+  csa_status st = check_desc(desc);
+  if (st != CSA_OK) return st;
+  REQUIRE(valid_dt(dt), "dt must be CSA_F32 or CSA_BF16");
+  REQUIRE(first >= 0 && count >= 0 && first + count <= desc->capacity,
+          "entries [first, first+count) must lie within [0, capacity)");
+  if (count == 0) return ok();
+  REQUIRE_PTR(cache);
+  REQUIRE_PTR(kv);
+  if (!desc->is_hca) REQUIRE_PTR(ikey);
+  return cuda_status(launch_store_entries(*desc, cache_view(*desc, cache), first, count, kv,
+                                          ikey, dt, (cudaStream_t)stream),
+                     "csa_cache_store_entries");
+}
+
+static csa_status check_rows(const csa_cache_desc* d, const csa_rows* rows) {
+  REQUIRE(rows != nullptr, "rows is NULL");
+  REQUIRE_PTR(rows->ca);
+  REQUIRE_PTR(rows->za);
+  REQUIRE_PTR(rows->kv_win);
+  if (!d->is_hca) {
+    REQUIRE_PTR(rows->cb);
+    REQUIRE_PTR(rows->zb);
+    REQUIRE_PTR(rows->ica);
+    REQUIRE_PTR(rows->icb);
+    REQUIRE_PTR(rows->iza);
+    REQUIRE_PTR(rows->izb);
+  }
+  return ok();
+}
+
+csa_status csa_cache_write_rows(const csa_cache_desc* desc, void* cache, int64_t first_pos,
+                                int64_t count, const csa_rows* rows, void* stream) {
+  csa_status st = check_desc(desc);
+  if (st != CSA_OK) return st;
+  REQUIRE(first_pos >= 0 && count >= 0, "first_pos and count must be >= 0");
+  if (count == 0) return ok();
+  REQUIRE_PTR(cache);
+  if ((st = check_rows(desc, rows)) != CSA_OK) return st;
+  return cuda_status(launch_write_rows(*desc, cache_view(*desc, cache), first_pos, count, *rows,
+                                       (cudaStream_t)stream),
+                     "csa_cache_write_rows");
+}
+
+size_t csa_decode_workspace(const csa_cache_desc* desc) {
+  if (check_desc(desc) != CSA_OK) return 0;
+  return decode_workspace(*desc);
+}
+
+csa_status csa_decode_step(const csa_cache_desc* desc, void* cache, const int64_t* pos,
+                           const csa_rows* rows, const csa_decode_params* params,
+                           const void* q, const void* q_i, const float* w_i, void* out,
+                           void* ws, size_t ws_bytes, void* stream) {
+  csa_status st = check_desc(desc);
+  if (st != CSA_OK) return st;
+  REQUIRE_PTR(cache);
+  REQUIRE_PTR(pos);
+  if ((st = check_rows(desc, rows)) != CSA_OK) return st;
+  REQUIRE(params != nullptr, "params is NULL");
+  REQUIRE_PTR(params->ba);
+  REQUIRE_OPT_PTR(params->sink);
+  REQUIRE(params->scale == params->scale, "scale must not be NaN");
+  REQUIRE_PTR(q);
+  REQUIRE_PTR(out);
+  if (!desc->is_hca) {
+    REQUIRE_PTR(params->bb);
+    REQUIRE_PTR(params->iba);
+    REQUIRE_PTR(params->ibb);
+    REQUIRE_PTR(q_i);
+    REQUIRE_PTR(w_i);
+  }
+  const size_t need = decode_workspace(*desc);
+  if (ws == nullptr || ws_bytes < need)
+    return fail(CSA_ERR_WORKSPACE, "workspace %zu bytes < required %zu", ws_bytes, need);
+  REQUIRE_PTR(ws);
+  return cuda_status(launch_decode_step(*desc, cache_view(*desc, cache), pos, *rows, *params, q,
+                                        q_i, w_i, out, ws, (cudaStream_t)stream),
+                     "csa_decode_step");
+}
+
+}  // extern "C"

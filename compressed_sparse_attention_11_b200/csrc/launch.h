@@ -1,0 +1,57 @@
+// Host-side launch functions, one per kernel family.  Arguments are already
+// validated by the C ABI layer (csa_api.cu); these only size grids and launch.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <cuda_bf16.h>
+#include <stdint.h>
+
+#include "../../include/csa.h"
+
+namespace csa {
+
+cudaError_t launch_compress(const void* ca, const void* cb, const void* za, const void* zb,
+                            const float* ba, const float* bb, int64_t batch, int64_t n, int c,
+                            int m, int overlap, csa_dtype dt, void* out, cudaStream_t s);
+
+// fp32 scores[b][t][s] (row stride `ld`) for s < V(t); entries beyond V(t) untouched.
+cudaError_t launch_index_scores(const void* q_i, const float* w_i, const void* k_i,
+                                int64_t batch, int64_t n, int nh_i, int c_i, int m,
+                                csa_dtype dt, float* scores, int64_t ld, cudaStream_t s);
+
+// Top-k rows: row r of `rows` has V(r) candidates; writes idx[r][0..k).
+cudaError_t launch_topk_rows(const float* scores, int64_t ld, int64_t batch, int64_t n,
+                             int m, int64_t E, int k, int32_t* idx, cudaStream_t s);
+
+cudaError_t launch_attn(const void* q, const void* kv_comp, const int32_t* idx, int k,
+                        const void* kv_win, int window, const float* sink, float scale,
+                        int64_t batch, int64_t n, int nh, int c, int m, csa_dtype dt,
+                        void* out, cudaStream_t s);
+
+// ---- decode --------------------------------------------------------------
+struct CacheView {
+  uint8_t* entry_fp8;
+  float* entry_scale;
+  __nv_bfloat16* entry_rope;
+  uint8_t* ikey_fp8;
+  float* ikey_scale;
+  __nv_bfloat16* window;
+  __nv_bfloat16* state;
+  __nv_bfloat16* istate;
+};
+
+CacheView cache_view(const csa_cache_desc& d, void* cache);
+void cache_layout(const csa_cache_desc& d, csa_cache_layout_t* L);
+
+cudaError_t launch_store_entries(const csa_cache_desc& d, const CacheView& cv, int64_t first,
+                                 int64_t count, const void* kv, const void* ikey, csa_dtype dt,
+                                 cudaStream_t s);
+cudaError_t launch_write_rows(const csa_cache_desc& d, const CacheView& cv, int64_t first_pos,
+                              int64_t count, const csa_rows& rows, cudaStream_t s);
+size_t decode_workspace(const csa_cache_desc& d);
+cudaError_t launch_decode_step(const csa_cache_desc& d, const CacheView& cv, const int64_t* pos,
+                               const csa_rows& rows, const csa_decode_params& p, const void* q,
+                               const void* q_i, const float* w_i, void* out, void* ws,
+                               cudaStream_t s);
+
+}  // namespace csa

@@ -315,34 +315,27 @@ _E4M3_POS = np.array([e4m3_value(c) for c in range(0x7F)])  # codes 0x00..0x7E, 
 
 
 def e4m3_encode(x) -> np.ndarray:
-    """Round each value to E4M3, nearest with ties to even code, saturating.
+    """Round each value to E4M3, nearest with ties to the even code, saturating.
 
     Works on the exact value of x (float32 inputs widen exactly).  The
-    candidates are the 127 finite non-negative codes, which are increasing in
-    value; ties pick the code with an even mantissa.  NaN maps to 0x7F.
+    candidates are the 127 finite non-negative codes, whose values increase
+    with the code; a tie between two neighbours picks the even code (the one
+    whose mantissa ends in 0).  NaN maps to 0x7F.
     """
     x = np.asarray(x, dtype=np.float64)
-    flat = x.reshape(-1)
-    out = np.zeros(flat.shape[0], dtype=np.uint8)
-    for i, v in enumerate(flat):
-        if np.isnan(v):
-            out[i] = 0x7F
-            continue
-        a = min(abs(v), E4M3_MAX)
-        hi = int(np.searchsorted(_E4M3_POS, a, side="left"))   # first code >= a
-        if hi < len(_E4M3_POS) and _E4M3_POS[hi] == a:
-            code = hi
-        else:
-            lo = hi - 1
-            dlo, dhi = a - _E4M3_POS[lo], _E4M3_POS[hi] - a
-            if dlo < dhi:
-                code = lo
-            elif dhi < dlo:
-                code = hi
-            else:
-                code = lo if lo % 2 == 0 else hi
-        out[i] = code | (0x80 if (v < 0 or (v == 0 and np.signbit(v))) else 0)
-    return out.reshape(x.shape)
+    a = np.minimum(np.abs(x), E4M3_MAX)
+    hi = np.searchsorted(_E4M3_POS, a, side="left")           # first code with value >= a
+    hi = np.minimum(hi, len(_E4M3_POS) - 1)
+    lo = np.maximum(hi - 1, 0)
+    dlo = a - _E4M3_POS[lo]
+    dhi = _E4M3_POS[hi] - a
+    code = np.where(dlo < dhi, lo, hi)
+    code = np.where(dlo == dhi, np.where(lo % 2 == 0, lo, hi), code)
+    code = np.where(_E4M3_POS[hi] == a, hi, code)             # exact hit
+    neg = (x < 0) | ((x == 0) & np.signbit(x))
+    out = (code.astype(np.uint8) | np.where(neg, 0x80, 0).astype(np.uint8))
+    out = np.where(np.isnan(x), np.uint8(0x7F), out).astype(np.uint8)
+    return out
 
 
 def e4m3_decode(codes) -> np.ndarray:

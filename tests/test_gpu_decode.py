@@ -1,0 +1,165 @@
+"""GPU parity of the decode entry points (cache store, row hand-off, decode
+step) against the oracle's incremental decode sequence."""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import compressed_sparse_attention_11_b200 as csa
+import csa_inputs as G
+import oracle as O
+from _util import check_close, host
+
+pytestmark = pytest.mark.gpu
+
+DEV = "cuda"
+CSA_STREAMS = ("ca", "cb", "za", "zb", "ica", "icb", "iza", "izb", "kv_win")
+HCA_STREAMS = ("ca", "za", "kv_win")
+
+
+def _quantize_all(x, rope):
+    """Oracle cache form of every entry in x [E, c] (fp32)."""
+    q = [O.quantize_entry(np.asarray(x[e], dtype=np.float32), rope) for e in range(x.shape[0])]
+    return q
+
+
+def code_distance(a, b):
+    """|ordinal distance| between E4M3 codes of the same sign (sign flips count large)."""
+    a = a.astype(np.int64)
+    b = b.astype(np.int64)
+    same_sign = (a & 0x80) == (b & 0x80)
+    return np.where(same_sign, np.abs((a & 0x7F) - (b & 0x7F)), 1000)
+
+
+@pytest.mark.parametrize("dt", [torch.float32, torch.bfloat16])
+def test_store_entries_bit_exact(dt):
+    B, E, c, rope, ci = 3, 50, 128, 32, 64
+    kv = G.normal((B, E, c), 5, 20, dtype=dt)
+    ik = G.normal((B, E, ci), 5, 21, dtype=dt)
+    kv[0, 3] = 0.0                                   # amax 0: scale 1, codes 0
+    kv[1, 4, 7] = 1e4                                # one huge element
+    cache = csa.CsaCache(B, E + 5, c, rope, 4, 16, 8, False, c_i=ci, nh_i=4, k=8)
+    cache.store_entries(2, kv.to(DEV), ik.to(DEV))
+    torch.cuda.synchronize()
+    got = {k: host(v) for k, v in cache.entries().items()}
+    for b in range(B):
+        for e in range(E):
+            codes, scale, rp = O.quantize_entry(kv[b, e].float().numpy(), rope)
+            assert np.array_equal(got["codes"][b, 2 + e].numpy(), codes), (b, e)
+            assert got["scale"][b, 2 + e].item() == scale, (b, e)
+            assert np.array_equal(got["rope"][b, 2 + e].double().numpy(), rp), (b, e)
+            icodes, iscale, _ = O.quantize_entry(ik[b, e].float().numpy(), 0)
+            assert np.array_equal(got["icodes"][b, 2 + e].numpy(), icodes), (b, e)
+            assert got["iscale"][b, 2 + e].item() == iscale
+
+
+def _setup(w, B, E, steps, seed):
+    """Cache with E stored entries and raw rows up to position t0-1 (t0 = m*E)."""
+    t0 = w.m * E
+    inp = G.decode_inputs(w, entries=E, batch=B, t=t0, steps=steps, seed=seed)
+    first = int(inp["first_pos"])
+    cap = E + steps // w.m + 2
+    cache = csa.CsaCache(B, cap, w.c, w.rope_dims, w.m, w.window, w.nh, w.is_hca, c_i=w.c_i,
+                         nh_i=w.nh_i, k=w.k)
+    cache.store_entries(0, inp["cache_kv"].to(DEV),
+                        None if w.is_hca else inp["cache_ikey"].to(DEV))
+    tail = w.window + 2 * w.m
+    skip = max(0, -first)             # short histories start at position 0
+    names = HCA_STREAMS if w.is_hca else CSA_STREAMS
+    cache.write_rows(first + skip, {nm: inp["rows_" + nm][:, skip:tail].contiguous().to(DEV)
+                                    for nm in names})
+    return inp, cache, t0, first, tail, names
+
+
+def _oracle_sequence(w, inp, b, E, first, tail, names):
+    seq = O.DecodeSequence(w.c, w.rope_dims, w.m, w.window, w.is_hca, w.c_i)
+    for e in range(E):
+        seq.store_entry(inp["cache_kv"][b, e].numpy(),
+                        None if w.is_hca else inp["cache_ikey"][b, e].numpy())
+    for r in range(max(0, -first), tail):
+        for nm in names:
+            seq.put_row(nm, first + r, inp["rows_" + nm][b, r])
+    return seq
+
+
+def _biases(inp, w):
+    keys = ("ba",) if w.is_hca else ("ba", "bb", "iba", "ibb")
+    return {k: inp[k] for k in keys}
+
+
+def _run_and_compare(w, B, E, steps, seed, check_seqs=None):
+    inp, cache, t0, first, tail, names = _setup(w, B, E, steps, seed)
+    biases = _biases(inp, w)
+    dbias = {k: v.to(DEV) for k, v in biases.items()}
+    sink = inp["sink"].to(DEV)
+    check_seqs = range(B) if check_seqs is None else check_seqs
+    seqs = {b: _oracle_sequence(w, inp, b, E, first, tail, names) for b in check_seqs}
+    for s in range(steps):
+        t = t0 + s
+        r = tail + s
+        rows = {nm: inp["rows_" + nm][:, r].contiguous().to(DEV) for nm in names}
+        pos = torch.full((B,), t, dtype=torch.int64, device=DEV)
+        q = inp["q"][s].to(DEV)
+        qi = None if w.is_hca else inp["q_i"][s].to(DEV)
+        wi = None if w.is_hca else inp["w_i"][s].to(DEV)
+        out = host(cache.decode_step(pos, rows, dbias, sink, w.scale, q, qi, wi))
+        for b in check_seqs:
+            ref, _ = seqs[b].step(t, {nm: inp["rows_" + nm][b, r] for nm in names}, biases,
+                                  inp["q"][s, b], None if w.is_hca else inp["q_i"][s, b],
+                                  None if w.is_hca else inp["w_i"][s, b], inp["sink"], w.scale,
+                                  w.k)
+            check_close(out[b], ref, torch.bfloat16, f"step t={t} b={b}")
+    # emitted entries agree with the oracle's from-scratch compression
+    got = {k: host(v) for k, v in cache.entries().items()}
+    n_emit = (t0 + steps) // w.m - E
+    for b in check_seqs:
+        for i in range(E, E + n_emit):
+            codes, scale, rope = seqs[b].entries[i]
+            assert abs(got["scale"][b, i].item() / scale - 1) < 1e-5
+            dist = code_distance(got["codes"][b, i].numpy(), codes)
+            assert dist.max() <= 1 and (dist > 0).mean() < 0.02, (b, i, dist.max())
+            assert np.abs(got["rope"][b, i].double().numpy() - rope).max() <= \
+                np.abs(rope).max() * 2 ** -7
+            if not w.is_hca:
+                icodes, iscale, _ = seqs[b].ikeys[i]
+                assert abs(got["iscale"][b, i].item() / iscale - 1) < 1e-5
+                assert code_distance(got["icodes"][b, i].numpy(), icodes).max() <= 1
+    return cache
+
+
+SMALL_CSA = G.Decode("small_csa_decode", 3, 0, 128, 32, 4, 8, 16, False, nh_i=4, c_i=64, k=12,
+                     seed=101)
+SMALL_HCA = G.Decode("small_hca_decode", 2, 0, 128, 32, 16, 8, 16, True, seed=102)
+
+
+def test_decode_csa_small_crosses_emissions():
+    _run_and_compare(SMALL_CSA, B=3, E=100, steps=9, seed=7)
+
+
+def test_decode_csa_fewer_entries_than_k():
+    _run_and_compare(SMALL_CSA, B=2, E=5, steps=6, seed=8)    # V <= k: every entry selected
+
+
+def test_decode_hca_small_crosses_emission():
+    _run_and_compare(SMALL_HCA, B=2, E=20, steps=18, seed=9)
+
+
+def test_decode_csa_realistic_dims_two_chunks():
+    w = G.Decode("csa_decode_dims", 2, 0, 512, 64, 4, 64, 128, False, nh_i=64, c_i=128, k=512,
+                 seed=103)
+    _run_and_compare(w, B=2, E=2500, steps=4, seed=10)
+
+
+def test_write_rows_fills_ring_and_state():
+    w = SMALL_CSA
+    B, E = 2, 10
+    inp, cache, t0, first, tail, names = _setup(w, B, E, 1, seed=4)
+    win = cache.region("window", torch.bfloat16, (B, w.window, w.c))
+    st = cache.region("state", torch.bfloat16, (B, 2, 4, w.m, w.c))
+    for u in range(t0 - w.window, t0):
+        assert torch.equal(host(win)[:, u % w.window], inp["rows_kv_win"][:, u - first])
+    for u in range(t0 - 2 * w.m, t0):
+        par, row = (u // w.m) % 2, u % w.m
+        for si, nm in enumerate(("ca", "cb", "za", "zb")):
+            assert torch.equal(host(st)[:, par, si, row], inp["rows_" + nm][:, u - first])
