@@ -27,7 +27,8 @@ CSA_F32, CSA_BF16 = 0, 1
 
 EXPORTED = (
     "csa_status_string", "csa_last_error", "csa_abi_version", "csa_compress",
-    "csa_index_topk_workspace", "csa_index_topk", "csa_sparse_attn", "hca_attn",
+    "csa_index_topk_workspace", "csa_index_topk", "csa_index_topk_noalloc", "csa_sparse_attn",
+    "hca_attn",
     "csa_cache_layout", "csa_cache_store_entries", "csa_cache_write_rows",
     "csa_decode_workspace", "csa_decode_step",
 )
@@ -83,6 +84,7 @@ def lib() -> ctypes.CDLL:
         "csa_compress": (i32, [vp, vp, vp, vp, vp, vp, i64, i64, i32, i32, i32, i32, vp, vp]),
         "csa_index_topk_workspace": (sz, [i64, i64, i32, i32, i32, i32]),
         "csa_index_topk": (i32, [vp, vp, vp, i64, i64, i32, i32, i32, i32, i32, vp, vp, sz, vp]),
+        "csa_index_topk_noalloc": (i32, [vp, vp, vp, i64, i64, i32, i32, i32, i32, i32, vp, vp]),
         "csa_sparse_attn": (i32, [vp, vp, vp, i32, vp, i32, vp, f32, i64, i64, i32, i32, i32,
                                   i32, vp, vp]),
         "hca_attn": (i32, [vp, vp, vp, i32, vp, f32, i64, i64, i32, i32, i32, i32, vp, vp]),
@@ -167,6 +169,19 @@ def csa_index_topk(q_i, w_i, k_i, m: int, k: int, ws: Optional[torch.Tensor] = N
     _check(lib().csa_index_topk(_ptr(q_i), _ptr(w_i), _ptr(k_i), B, n, H, ci, m, k, _dt(q_i),
                                 _ptr(out), _ptr(ws), ws.numel() * ws.element_size(),
                                 _stream(q_i)))
+    return out
+
+
+def csa_index_topk_noalloc(q_i, w_i, k_i, m: int, k: int, out: Optional[torch.Tensor] = None):
+    """csa_index_topk using the library's built-in score scratch (no workspace).
+
+    For callers that cannot allocate device memory; limited to
+    batch * n * (n // m) <= 2**21 scores, and concurrent calls race."""
+    B, n, H, ci = q_i.shape
+    if out is None:
+        out = torch.empty((B, n, k), dtype=torch.int32, device=q_i.device)
+    _check(lib().csa_index_topk_noalloc(_ptr(q_i), _ptr(w_i), _ptr(k_i), B, n, H, ci, m, k,
+                                        _dt(q_i), _ptr(out), _stream(q_i)))
     return out
 
 

@@ -93,6 +93,14 @@ csa_status check_desc(const csa_cache_desc* d) {
 
 }  // namespace
 
+csa_status csa::set_last_error(csa_status st, const char* fmt, ...) {
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(g_err, sizeof(g_err), fmt, ap);
+  va_end(ap);
+  return st;
+}
+
 extern "C" {
 
 const char* csa_status_string(int status) {

@@ -10,6 +10,9 @@
 
 namespace csa {
 
+// Records a one-line reason for `st` (read back by csa_last_error) and returns st.
+csa_status set_last_error(csa_status st, const char* fmt, ...);
+
 cudaError_t launch_compress(const void* ca, const void* cb, const void* za, const void* zb,
                             const float* ba, const float* bb, int64_t batch, int64_t n, int c,
                             int m, int overlap, csa_dtype dt, void* out, cudaStream_t s);

@@ -109,6 +109,23 @@ csa_status csa_index_topk(const void* q_i, const float* w_i, const void* k_i, in
                           int32_t* idx, void* ws, size_t ws_bytes, void* stream);
 
 /* ------------------------------------------------------------------------
+ * csa_index_topk_noalloc -- csa_index_topk for callers that cannot allocate
+ * device memory (no counterpart on the pages; a library convenience).
+ *
+ * Same arguments, results and errors as csa_index_topk, without `ws`: the
+ * score scratch is a fixed array inside the library (8 MiB per device, held
+ * by every GPU that loads the library until the process exits).  Calls that
+ * need more than 2^21 fp32 scores (batch * n * floor(n/m)) return
+ * CSA_ERR_UNSUPPORTED.  All calls share that array, so calls whose work
+ * overlaps on the GPU race on it.  The first call on a device looks up the
+ * array's address (cudaGetSymbolAddress with that device current); make it
+ * before any stream capture.  Never allocates.
+ * ------------------------------------------------------------------------ */
+csa_status csa_index_topk_noalloc(const void* q_i, const float* w_i, const void* k_i,
+                                  int64_t batch, int64_t n, int nh_i, int c_i, int m, int k,
+                                  csa_dtype dt, int32_t* idx, void* stream);
+
+/* ------------------------------------------------------------------------
  * csa_sparse_attn -- CSA core attention: shared-KV MQA over the selected
  * compressed entries plus the sliding window, with the sink in the same
  * denominator ([Walk-through] 4.3 shared-KV MQA, 4.5 sliding window and
