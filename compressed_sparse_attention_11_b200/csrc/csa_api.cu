@@ -4,6 +4,7 @@
 #include <cstdarg>
 #include <cstdio>
 #include <cstring>
+#include <mutex>
 
 #include "common.cuh"
 #include "launch.h"
@@ -93,6 +94,26 @@ csa_status check_desc(const csa_cache_desc* d) {
 
 }  // namespace
 
+namespace {
+// Set (bit OR) by kernels whose bounded waits expired; read by csa_check.
+static __device__ unsigned int g_timeout_flag;
+constexpr int kMaxDev = 64;
+std::mutex g_flag_mu;
+unsigned int* g_flag_ptr[kMaxDev] = {};
+}  // namespace
+
+unsigned int* csa::device_timeout_flag() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDev) return nullptr;
+  std::lock_guard<std::mutex> lock(g_flag_mu);
+  if (g_flag_ptr[dev] == nullptr) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_timeout_flag) != cudaSuccess) return nullptr;
+    g_flag_ptr[dev] = static_cast<unsigned int*>(p);
+  }
+  return g_flag_ptr[dev];
+}
+
 csa_status csa::set_last_error(csa_status st, const char* fmt, ...) {
   va_list ap;
   va_start(ap, fmt);
@@ -118,6 +139,22 @@ const char* csa_status_string(int status) {
 const char* csa_last_error(void) { return g_err; }
 
 int csa_abi_version(void) { return 1; }
+
+csa_status csa_check(void* stream) {
+  cudaError_t e = cudaStreamSynchronize((cudaStream_t)stream);
+  if (e != cudaSuccess) return cuda_status(e, "csa_check");
+  unsigned int* flag = device_timeout_flag();
+  if (flag == nullptr) return fail(CSA_ERR_CUDA, "csa_check: no device flag");
+  unsigned int v = 0;
+  e = cudaMemcpy(&v, flag, sizeof(v), cudaMemcpyDeviceToHost);
+  if (e != cudaSuccess) return cuda_status(e, "csa_check");
+  if (v != 0) {
+    const unsigned int zero = 0;
+    cudaMemcpy(flag, &zero, sizeof(zero), cudaMemcpyHostToDevice);
+    return fail(CSA_ERR_TIMEOUT, "a kernel gave up a bounded wait; its outputs are invalid");
+  }
+  return ok();
+}
 
 csa_status csa_compress(const void* ca, const void* cb, const void* za, const void* zb,
                         const float* ba, const float* bb, int64_t batch, int64_t n, int c,

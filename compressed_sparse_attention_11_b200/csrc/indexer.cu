@@ -1,4 +1,5 @@
-// Lightning-indexer scores on CUDA cores (fp32 path and general shapes).
+// Lightning-indexer scores on CUDA cores (fp32 path and shapes the tcgen05
+// kernel in indexer_tc.cu does not take).
 //
 // I[t, s] = sum_h w[t, h] * ReLU(q_i[t, h, :] . K_i[s, :]) for s < V(t),
 // V(t) = floor((t+1)/m)  (B9 indexer equation of the "Core formulas chapter";
@@ -89,6 +90,11 @@ cudaError_t launch_index_scores(const void* q_i, const float* w_i, const void* k
                                 csa_dtype dt, float* scores, int64_t ld, cudaStream_t s) {
   const int64_t E = n / m;
   if (E == 0) return cudaSuccess;
+  if (index_scores_tc_supported(nh_i, c_i, dt, q_i, k_i)) {
+    unsigned int* err = device_timeout_flag();
+    if (err == nullptr) return cudaErrorUnknown;
+    return launch_index_scores_tc(q_i, w_i, k_i, batch, n, nh_i, c_i, m, scores, ld, err, s);
+  }
   const int nh_pad = (nh_i + kIdxHG - 1) / kIdxHG * kIdxHG;
   const size_t smem = sizeof(float) * ((size_t)c_i * kIdxKeys + (size_t)c_i * nh_pad);
   dim3 grid((unsigned)((E + kIdxKeys - 1) / kIdxKeys),

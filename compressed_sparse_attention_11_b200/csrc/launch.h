@@ -13,6 +13,16 @@ namespace csa {
 // Records a one-line reason for `st` (read back by csa_last_error) and returns st.
 csa_status set_last_error(csa_status st, const char* fmt, ...);
 
+// Device word that kernels with bounded waits OR a bit into when a wait
+// expires (per current device; csa_check reads and clears it).
+unsigned int* device_timeout_flag();
+
+// tcgen05 indexer (bf16, c_i in {64, 128}, nh_i in {16, 32, 64, 128}).
+bool index_scores_tc_supported(int nh_i, int c_i, csa_dtype dt, const void* q_i, const void* k_i);
+cudaError_t launch_index_scores_tc(const void* q_i, const float* w_i, const void* k_i,
+                                   int64_t batch, int64_t n, int nh_i, int c_i, int m,
+                                   float* scores, int64_t ld, unsigned int* err, cudaStream_t s);
+
 cudaError_t launch_compress(const void* ca, const void* cb, const void* za, const void* zb,
                             const float* ba, const float* bb, int64_t batch, int64_t n, int c,
                             int m, int overlap, csa_dtype dt, void* out, cudaStream_t s);

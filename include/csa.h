@@ -62,6 +62,11 @@ const char* csa_status_string(int status);
 const char* csa_last_error(void);
 /* ABI version, bumped on any signature or layout change. */
 int csa_abi_version(void);
+/* Synchronises `stream`, then returns CSA_ERR_TIMEOUT if any kernel of this
+ * library on the current device gave up a bounded wait since the last check
+ * (the outputs of that launch are invalid), and clears that record.  The one
+ * entry point that synchronises. */
+csa_status csa_check(void* stream);
 
 /* ------------------------------------------------------------------------
  * csa_compress -- token-level KV compressor ([Formulas B9] CSA and HCA

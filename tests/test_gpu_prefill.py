@@ -85,10 +85,17 @@ def _index_inputs(B, n, H, ci, m, dt, seed):
     (2, 1030, 4, 64, 4, 32, torch.float32, None),          # ragged, batch 2
     (1, 4096, 64, 128, 4, 512, torch.bfloat16, "sample"),  # V up to 1024 > k
     (1, 300, 3, 24, 4, 5, torch.bfloat16, None),           # odd head count and dim
+    # tensor-core indexer shapes (bf16, c_i in {64, 128}, nh_i in {16..128})
+    (2, 1000, 64, 128, 4, 64, torch.bfloat16, "sample"),   # ragged query tile, batch 2
+    (1, 2100, 16, 64, 4, 100, torch.bfloat16, "sample"),
+    (1, 1500, 32, 128, 4, 33, torch.bfloat16, "sample"),
+    (1, 1100, 128, 64, 4, 20, torch.bfloat16, "sample"),
+    (1, 600, 64, 128, 1, 200, torch.bfloat16, "sample"),   # m = 1 (token-level selection)
 ])
 def test_index_topk_parity(B, n, H, ci, m, k, dt, rows):
     q, w, kk = _index_inputs(B, n, H, ci, m, dt, seed=17)
     idx = csa.csa_index_topk(q.to(DEV), w.to(DEV), kk.to(DEV), m, k)
+    csa.csa_check()
     g = host(idx).numpy()
     rr = range(n) if rows is None else sorted(set(list(range(0, 12)) + list(range(n - 40, n)) +
                                                  list(range(3, n, 97))))
@@ -101,12 +108,14 @@ def test_index_topk_parity(B, n, H, ci, m, k, dt, rows):
     assert exact > 0.9 * B * len(rr)
 
 
-@pytest.mark.parametrize("dt", [torch.float32, torch.bfloat16])
-def test_index_topk_integer_scores_bit_exact(dt):
-    """One head, w = 1, q = (256, 1, 0..), key s = (hi_s, lo_s, 0..): every score
-    is the integer 256*hi + lo, exact in bf16 inputs and fp32 sums, with
-    deliberate ties (repeated pairs) that must resolve to the smaller index."""
-    n, m, k, ci = 2048, 4, 37, 16
+@pytest.mark.parametrize("dt,H,ci", [(torch.float32, 1, 16), (torch.bfloat16, 1, 16),
+                                     (torch.bfloat16, 16, 64), (torch.bfloat16, 64, 128)])
+def test_index_topk_integer_scores_bit_exact(dt, H, ci):
+    """Head 0 has q = (256, 1, 0..) and w = 1, the other heads q = 0; key s is
+    (hi_s, lo_s, 0..): every score is the integer 256*hi + lo, exact in bf16
+    inputs and fp32 sums, with deliberate ties (repeated pairs) that must
+    resolve to the smaller index.  H > 1 runs the tensor-core indexer."""
+    n, m, k = 2048, 4, 37
     E = n // m
     r = np.random.default_rng(3)
     hi = r.integers(0, 200, E)
@@ -115,11 +124,12 @@ def test_index_topk_integer_scores_bit_exact(dt):
     hi[dup[:30]], lo[dup[:30]] = hi[dup[30:]], lo[dup[30:]]
     keys = np.zeros((1, E, ci))
     keys[0, :, 0], keys[0, :, 1] = hi, lo
-    q = np.zeros((1, n, 1, ci))
-    q[..., 0], q[..., 1] = 256.0, 1.0
-    w = np.ones((1, n, 1), dtype=np.float32)
+    q = np.zeros((1, n, H, ci))
+    q[:, :, 0, 0], q[:, :, 0, 1] = 256.0, 1.0
+    w = np.ones((1, n, H), dtype=np.float32)
     qt, kt = torch.tensor(q, dtype=dt), torch.tensor(keys, dtype=dt)
     idx = host(csa.csa_index_topk(qt.to(DEV), torch.tensor(w).to(DEV), kt.to(DEV), m, k)).numpy()
+    csa.csa_check()
     scores = 256.0 * hi + lo
     for t in range(n):
         V = O.visible(t, m)
