@@ -1,5 +1,6 @@
 // Core attention on CUDA cores: shared-KV MQA over an explicit entry set with
-// the attention sink in the softmax denominator (fp32 path, general shapes).
+// the attention sink in the softmax denominator (fp32 path and the shapes the
+// tcgen05 kernel in attn_tc.cu does not take).
 //
 // For query t and head h, E_t is (CSA) the selected compressed entries
 // idx[t, :] that are visible (0 <= s < floor((t+1)/m)), or (HCA) every
@@ -136,6 +137,12 @@ cudaError_t launch_attn(const void* q, const void* kv_comp, const int32_t* idx, 
                         int64_t batch, int64_t n, int nh, int c, int m, csa_dtype dt,
                         void* out, cudaStream_t s) {
   const int64_t E = n / m;
+  if (attn_tc_supported(nh, c, idx ? k : 0, dt, q, kv_comp ? kv_comp : q, kv_win)) {
+    unsigned int* err = device_timeout_flag();
+    if (err == nullptr) return cudaErrorUnknown;
+    return launch_attn_tc(q, kv_comp, idx, k, kv_win, window, sink, scale, batch, n, m, out,
+                          err, s);
+  }
   const size_t smem = sizeof(float) * ((size_t)kAttnTE * (c + 1) + (size_t)kAttnHG * c +
                                        kAttnHG * kAttnTE) + sizeof(int64_t) * kAttnTE;
   dim3 grid((unsigned)n, (unsigned)((nh + kAttnHG - 1) / kAttnHG), (unsigned)batch);

@@ -1,0 +1,508 @@
+// Core attention on the tcgen05 tensor cores: shared-KV MQA over a per-query
+// entry set with the attention sink in the softmax denominator (bf16 in/out,
+// fp32 accumulation), for 64 query heads of dim 512.
+//
+// E_t is (CSA) the selected compressed entries idx[t, :] with 0 <= s < V(t)
+// or (HCA) every visible compressed entry, followed by the raw window rows
+// max(0, t-W+1) .. t; each entry is both key and value, and
+//   o_h = sum_j exp(l_hj) e_j / (exp(sink_h) + sum_j exp(l_hj)),
+// l_hj = scale q_h . e_j  (sections 4.3 and 4.5 of "DeepSeek-V4: million-token
+// context"; B9 of the "Core formulas chapter"; one softmax shared by the
+// window, the compressed entries and the sink).
+//
+// Every query reads its own gathered entries, so the 64 heads of ONE query
+// are the whole reuse available; the contractions therefore run "swapped":
+//   S^T[e, h] = K[e, :] . Q[h, :]           M = 128 entries, N = 64 heads
+//   O^T[d, h] += sum_e V[e, d] P^T[e, h]     M = 128 dims (x4), N = 64 heads
+// The gathered 128 x 512 entry tile is stored once (eight 64-dim slabs,
+// 128-byte swizzle) and read as the K-major A operand of Q.K and as the
+// MN-major A operand (V^T) of P.V.  S^T lands one entry per TMEM lane, so the
+// per-head softmax statistics need cross-lane reductions (a 31-shuffle
+// transpose-reduce per warp, then 4 warps through shared memory); the
+// running max is only moved -- and O^T rescaled in TMEM -- when a tile's max
+// exceeds it by more than 2^8.
+//
+// Persistent CTAs (one per SM) walk the queries.  Every wait is bounded
+// (including the warp-group exchanges, which use mbarriers rather than
+// named barriers), so a fault upstream ends the kernel with the timeout flag
+// set instead of a hang.  Warp roles: warps 0-7
+// softmax + epilogue (warp w: TMEM lanes 32*(w%4), heads 32*(w/4)), warps
+// 8-10 gather (cp.async, zero-filled past the end of E_t; they also compact
+// the query's valid selected indices), warp 11 issues the MMAs.
+#include "common.cuh"
+#include "launch.h"
+#include "sm100.cuh"
+
+#include <algorithm>
+
+namespace csa {
+
+namespace {
+
+constexpr int kNH = 64;                  // query heads (MMA N)
+constexpr int kC = 512;                  // entry dim
+constexpr int kTE = 128;                 // entries per tile
+constexpr int kSlabs = kC / 64;          // 64-dim slabs
+constexpr int kSlabBytes = kTE * 128;    // 16 KB
+constexpr int kQSlabBytes = kNH * 128;   // 8 KB
+constexpr int kSoftWarps = 8, kProdWarps = 3;
+constexpr int kProdThreads = kProdWarps * 32;
+constexpr int kMmaWarp = kSoftWarps + kProdWarps;
+constexpr int kThreads = (kMmaWarp + 1) * 32;  // 384: 3 warps per SM sub-partition
+constexpr int kRowsPerPass = kProdThreads / 8;  // 12 rows x 8 16-byte chunks per pass
+constexpr int kPasses = (kTE + kRowsPerPass - 1) / kRowsPerPass;  // 11
+constexpr int kMaxSel = 2048;                  // selected entries per query
+constexpr float kRescaleLog2 = 8.f;            // move the running max only past 2^8
+
+constexpr uint32_t kColS = 0;    // S^T, double-buffered: 2 x 64 columns
+constexpr uint32_t kColO = 128;  // O^T: 4 chunks x 64 columns
+
+struct __align__(16) AttnMeta {
+  int ntiles, nrows;
+  int64_t t, b;
+};
+
+struct __align__(8) AttnBars {
+  uint64_t slab_full[kSlabs], slab_empty[kSlabs];
+  uint64_t s_full[2], s_empty[2], p_full, p_empty, q_full, q_empty, o_empty, meta_full[2], drain;
+  uint64_t grp_soft[2], grp_prod;  // bounded group barriers (one arrive per warp)
+  uint32_t tmem_base;
+};
+
+constexpr int OFF_Q = 0;
+constexpr int OFF_KV = OFF_Q + kSlabs * kQSlabBytes;        // 65536
+constexpr int OFF_P = OFF_KV + kSlabs * kSlabBytes;         // 196608
+constexpr int OFF_LIST = OFF_P + kTE * 128;                 // 212992
+constexpr int OFF_RED = OFF_LIST + kMaxSel * 4;             // [3][2 hh][4 quad][32] floats
+constexpr int OFF_META = OFF_RED + 3 * 2 * 4 * 32 * 4;
+constexpr int OFF_SCAN = OFF_META + 2 * (int)sizeof(AttnMeta);
+constexpr int OFF_BAR = OFF_SCAN + 64;
+constexpr int SMEM = OFF_BAR + (int)sizeof(AttnBars) + 1024;
+static_assert(SMEM <= 232448, "shared memory budget");
+
+// Bounded barrier among the 4 warps that share `bar` (one arrive per warp).
+__device__ __forceinline__ bool group_sync(uint64_t* bar, uint32_t& phase, unsigned int* err) {
+  __syncwarp();
+  if ((threadIdx.x & 31) == 0) sm100::mbar_arrive(bar);
+  const bool ok = sm100::mbar_wait(bar, phase & 1, err);
+  ++phase;
+  return ok;
+}
+
+// Lane i ends with the reduction (max or sum) of element i over the 32 lanes.
+template <bool kMax>
+__device__ __forceinline__ float transpose_reduce(float (&v)[32]) {
+  const int lane = threadIdx.x & 31;
+#pragma unroll
+  for (int half = 16; half >= 1; half >>= 1) {
+    const bool upper = (lane & half) != 0;
+#pragma unroll
+    for (int i = 0; i < half; ++i) {
+      const float send = upper ? v[i] : v[i + half];
+      const float keep = upper ? v[i + half] : v[i];
+      const float recv = __shfl_xor_sync(0xffffffffu, send, half);
+      v[i] = kMax ? fmaxf(keep, recv) : keep + recv;
+    }
+  }
+  return v[0];
+}
+
+__global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(
+    const __grid_constant__ CUtensorMap tm_q, const __nv_bfloat16* __restrict__ kv_comp,
+    const int32_t* __restrict__ idx, int k, const __nv_bfloat16* __restrict__ kv_win,
+    int window, const float* __restrict__ sink, float scale, int64_t n, int m, int64_t E,
+    int64_t total, __nv_bfloat16* __restrict__ out, unsigned int* __restrict__ err) {
+  using namespace sm100;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = smem_raw + ((1024 - (smem_u32(smem_raw) & 1023)) & 1023);
+  uint8_t* sQ = smem + OFF_Q;
+  uint8_t* sKV = smem + OFF_KV;
+  uint8_t* sP = smem + OFF_P;
+  int32_t* list = reinterpret_cast<int32_t*>(smem + OFF_LIST);
+  float* red = reinterpret_cast<float*>(smem + OFF_RED);
+  AttnMeta* meta = reinterpret_cast<AttnMeta*>(smem + OFF_META);
+  int* pscan = reinterpret_cast<int*>(smem + OFF_SCAN);
+  AttnBars* bar = reinterpret_cast<AttnBars*>(smem + OFF_BAR);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if ((int64_t)blockIdx.x >= total) return;
+  if (flag_value(err) != 0) return;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kSlabs; ++s) {
+      mbar_init(&bar->slab_full[s], kProdThreads);
+      mbar_init(&bar->slab_empty[s], 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&bar->s_full[i], 1);
+      mbar_init(&bar->s_empty[i], kSoftWarps);
+      mbar_init(&bar->meta_full[i], 1);
+    }
+    mbar_init(&bar->p_full, kSoftWarps);
+    mbar_init(&bar->p_empty, 1);
+    mbar_init(&bar->q_full, 1);
+    mbar_init(&bar->q_empty, 1);
+    mbar_init(&bar->o_empty, kSoftWarps);
+    mbar_init(&bar->drain, 1);
+    mbar_init(&bar->grp_soft[0], 4);
+    mbar_init(&bar->grp_soft[1], 4);
+    mbar_init(&bar->grp_prod, kProdWarps);
+    fence_mbar_init();
+  }
+  if (warp == kMmaWarp) {
+    tmem_alloc(&bar->tmem_base, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = bar->tmem_base;
+
+  if (warp >= kSoftWarps && warp < kMmaWarp) {
+    // ======================= gather producer (128 threads) =====================
+    const int ptid = threadIdx.x - kSoftWarps * 32;
+    const int pw = ptid >> 5;
+    const int chunk = ptid & 7;
+    int g = 0;
+    uint32_t gphase = 0;
+    int64_t q_issued = -1;  // last query whose Q load was issued
+    bool ok = true;
+    for (int64_t kq = 0; ok; ++kq) {
+      const int64_t qi = blockIdx.x + kq * gridDim.x;
+      if (qi >= total) break;
+      const int64_t b = qi / n, t = qi % n;
+      const int64_t V = min((t + 1) / m, E);
+      const int64_t w0 = max((int64_t)0, t - window + 1);
+      const int nwin = (int)(t - w0 + 1);
+      // the previous query's list is no longer read
+      if (!group_sync(&bar->grp_prod, gphase, err)) break;
+      int nsel;
+      if (idx != nullptr) {
+        // compact the valid selections, keeping their order
+        const int per = (k + kProdThreads - 1) / kProdThreads;
+        const int lo = min(k, ptid * per), hi = min(k, lo + per);
+        const int32_t* row = idx + (b * n + t) * k;
+        int cnt = 0;
+        for (int j = lo; j < hi; ++j) {
+          const int s = row[j];
+          cnt += (s >= 0 && s < V) ? 1 : 0;
+        }
+        int inc = cnt;
+#pragma unroll
+        for (int off = 1; off < 32; off <<= 1) {
+          const int v = __shfl_up_sync(0xffffffffu, inc, off);
+          if (lane >= off) inc += v;
+        }
+        if (lane == 31) pscan[pw] = inc;
+        if (!group_sync(&bar->grp_prod, gphase, err)) break;
+        int base = 0;
+        nsel = 0;
+        for (int w = 0; w < kProdWarps; ++w) {
+          if (w < pw) base += pscan[w];
+          nsel += pscan[w];
+        }
+        int pos = base + inc - cnt;
+        for (int j = lo; j < hi; ++j) {
+          const int s = row[j];
+          if (s >= 0 && s < V) list[pos++] = s;
+        }
+        if (!group_sync(&bar->grp_prod, gphase, err)) break;
+      } else {
+        nsel = (int)V;
+      }
+      const int N = nsel + nwin;
+      const int T = (N + kTE - 1) / kTE;
+      if (ptid == 0) {
+        AttnMeta& mt = meta[kq & 1];
+        mt.ntiles = T;
+        mt.nrows = N;
+        mt.t = t;
+        mt.b = b;
+        mbar_arrive(&bar->meta_full[kq & 1]);
+        // the query's 64 heads, once the previous query's Q.K has finished
+        if (kq >= 1 && !mbar_wait(&bar->q_empty, (uint32_t)((kq - 1) & 1), err)) ok = false;
+        if (ok) {
+          mbar_arrive_expect_tx(&bar->q_full, kSlabs * kQSlabBytes);
+          for (int s = 0; s < kSlabs; ++s)
+            tma_load_3d(sQ + s * kQSlabBytes, &tm_q, &bar->q_full, s * 64, (int)(t * kNH), (int)b);
+          q_issued = kq;
+        }
+      }
+      for (int tt = 0; tt < T && ok; ++tt, ++g) {
+        // this thread's rows of the tile: global row pointers (nullptr = zero fill)
+        const __nv_bfloat16* src[kPasses];
+#pragma unroll
+        for (int rr = 0; rr < kPasses; ++rr) {
+          const int slot = tt * kTE + (ptid >> 3) + kRowsPerPass * rr;
+          const __nv_bfloat16* p = nullptr;
+          if (slot < nsel) {
+            const int64_t e = idx != nullptr ? (int64_t)list[slot] : (int64_t)slot;
+            p = kv_comp + (b * E + e) * kC;
+          } else if (slot < N) {
+            p = kv_win + (b * n + w0 + (slot - nsel)) * kC;
+          }
+          src[rr] = p;
+        }
+        for (int s = 0; s < kSlabs; ++s) {
+          if (g >= 1 && !mbar_wait(&bar->slab_empty[s], (uint32_t)((g - 1) & 1), err)) {
+            ok = false;
+            break;
+          }
+          uint8_t* dst = sKV + s * kSlabBytes;
+#pragma unroll
+          for (int rr = 0; rr < kPasses; ++rr) {
+            const int row = (ptid >> 3) + kRowsPerPass * rr;
+            if (row >= kTE) continue;
+            const __nv_bfloat16* p = src[rr] != nullptr ? src[rr] + s * 64 + chunk * 8 : kv_win;
+            cp_async_16(dst + row * 128 + ((chunk ^ (row & 7)) * 16), p,
+                        src[rr] != nullptr ? 16u : 0u);
+          }
+          cp_async_arrive_noinc(&bar->slab_full[s]);
+        }
+      }
+    }
+    asm volatile("cp.async.wait_all;" ::: "memory");
+    if (ptid == 0 && q_issued >= 0)  // the last Q load has landed before exit
+      mbar_wait(&bar->q_full, (uint32_t)(q_issued & 1), err, false);
+  } else if (warp == kMmaWarp) {
+    // ======================= MMA issuer (one lane) =============================
+    constexpr uint32_t kIdQK = idesc_bf16(kTE, kNH, 0, 0);
+    constexpr uint32_t kIdPV = idesc_bf16(128, kNH, 1, 1);
+    const uint32_t kv0 = smem_u32(sKV), q0 = smem_u32(sQ), p0 = smem_u32(sP);
+    int g = 0;
+    bool ok = true;
+    for (int64_t kq = 0; ok; ++kq) {
+      const int64_t qi = blockIdx.x + kq * gridDim.x;
+      if (qi >= total) break;
+      if (!mbar_wait(&bar->meta_full[kq & 1], (uint32_t)((kq >> 1) & 1), err)) break;
+      const int T = meta[kq & 1].ntiles;
+      if (!mbar_wait(&bar->q_full, (uint32_t)(kq & 1), err)) break;
+      for (int tt = 0; tt < T; ++tt, ++g) {
+        const int sb = g & 1;
+        if (g >= 2 && !mbar_wait(&bar->s_empty[sb], (uint32_t)(((g >> 1) - 1) & 1), err)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        for (int s = 0; s < kSlabs && ok; ++s) {
+          if (!mbar_wait(&bar->slab_full[s], (uint32_t)(g & 1), err)) { ok = false; break; }
+          fence_proxy_async();
+          tc_fence_after();
+          if (lane == 0) {
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk)
+              mma_bf16(tmem + kColS + sb * kNH, desc_sw128(kv0 + s * kSlabBytes + kk * 32),
+                       desc_sw128(q0 + s * kQSlabBytes + kk * 32), kIdQK,
+                       (s | kk) != 0 ? 1u : 0u);
+          }
+          __syncwarp();
+        }
+        if (!ok) break;
+        if (lane == 0) {
+          mma_commit(&bar->s_full[sb]);
+          if (tt == T - 1) mma_commit(&bar->q_empty);
+        }
+        __syncwarp();
+        if (!mbar_wait(&bar->p_full, (uint32_t)(g & 1), err)) { ok = false; break; }
+        if (tt == 0 && kq >= 1 && !mbar_wait(&bar->o_empty, (uint32_t)((kq - 1) & 1), err)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        if (lane == 0) {
+          for (int c = 0; c < 4; ++c) {
+#pragma unroll
+            for (int kk = 0; kk < kTE / 16; ++kk)
+              mma_bf16(tmem + kColO + c * kNH,
+                       desc_sw128_mn(kv0 + 2 * c * kSlabBytes + kk * 2048, kSlabBytes, 1024),
+                       desc_sw128_mn(p0 + kk * 2048, 1024, 1024), kIdPV,
+                       (tt == 0 && kk == 0) ? 0u : 1u);
+            mma_commit(&bar->slab_empty[2 * c]);
+            mma_commit(&bar->slab_empty[2 * c + 1]);
+          }
+          mma_commit(&bar->p_empty);
+        }
+        __syncwarp();
+      }
+    }
+    if (lane == 0) mma_commit(&bar->drain);
+    __syncwarp();
+    mbar_wait(&bar->drain, 0, err, false);
+  } else {
+    // ======================= softmax + epilogue (8 warps) ======================
+    const int quad = warp & 3, hh = warp >> 2;
+    const uint32_t lane_base = tmem + ((uint32_t)(quad * 32) << 16);
+    const float qscale = scale * kLog2e;
+    const int row = quad * 32 + lane;  // entry row within a tile / dim within a chunk
+    uint32_t gphase = 0;
+    int g = 0;
+    for (int64_t kq = 0;; ++kq) {
+      const int64_t qi = blockIdx.x + kq * gridDim.x;
+      if (qi >= total) break;
+      if (!mbar_wait(&bar->meta_full[kq & 1], (uint32_t)((kq >> 1) & 1), err)) break;
+      const AttnMeta mt = meta[kq & 1];
+      float m_run = kNegInf;  // lane i: running max (log2 units) of head hh*32+i
+      float psum[32];
+#pragma unroll
+      for (int i = 0; i < 32; ++i) psum[i] = 0.f;
+      bool ok = true;
+      for (int tt = 0; tt < mt.ntiles; ++tt, ++g) {
+        const int sb = g & 1;
+        if (!mbar_wait(&bar->s_full[sb], (uint32_t)((g >> 1) & 1), err)) { ok = false; break; }
+        tc_fence_after();
+        const uint32_t s_addr = lane_base + kColS + sb * kNH + hh * 32;
+        const bool valid = tt * kTE + row < mt.nrows;
+        float v[32];
+        {
+          uint32_t r[32];
+          tmem_ld32(s_addr, r);
+          tmem_ld_wait();
+#pragma unroll
+          for (int i = 0; i < 32; ++i) v[i] = valid ? __uint_as_float(r[i]) * qscale : kNegInf;
+        }
+        float* rmax = red + ((sb * 2 + hh) * 4) * 32;
+        rmax[quad * 32 + lane] = transpose_reduce<true>(v);
+        if (!group_sync(&bar->grp_soft[hh], gphase, err)) { ok = false; break; }
+        const float mtile = fmaxf(fmaxf(rmax[lane], rmax[32 + lane]),
+                                  fmaxf(rmax[64 + lane], rmax[96 + lane]));
+        float m_new, f_lane = 1.f;
+        bool resc = false;
+        if (tt == 0) {
+          m_new = mtile;
+        } else {
+          resc = mtile > m_run + kRescaleLog2;
+          m_new = resc ? mtile : m_run;
+          f_lane = resc ? ex2(m_run - m_new) : 1.f;
+        }
+        m_run = m_new;
+        // the P^T buffer (and, for a rescale, O^T) is free once the previous P.V is done
+        if (g >= 1 && !mbar_wait(&bar->p_empty, (uint32_t)((g - 1) & 1), err)) { ok = false; break; }
+        tc_fence_after();
+        if (__any_sync(0xffffffffu, resc)) {
+          float f[32];
+#pragma unroll
+          for (int i = 0; i < 32; ++i) {
+            f[i] = __shfl_sync(0xffffffffu, f_lane, i);
+            psum[i] *= f[i];
+          }
+          for (int c = 0; c < 4; ++c) {
+            uint32_t o[32];
+            tmem_ld32(lane_base + kColO + c * kNH + hh * 32, o);
+            tmem_ld_wait();
+#pragma unroll
+            for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * f[i]);
+            tmem_st32(lane_base + kColO + c * kNH + hh * 32, o);
+          }
+          tmem_st_wait();
+        }
+        // the logits again (cheaper than holding them across the reductions)
+        uint32_t r[32];
+        tmem_ld32(s_addr, r);
+        tmem_ld_wait();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bar->s_empty[sb]);
+        uint32_t pk[16];
+#pragma unroll
+        for (int i = 0; i < 32; i += 2) {
+          float ma = __shfl_sync(0xffffffffu, m_run, i);
+          float mb = __shfl_sync(0xffffffffu, m_run, i + 1);
+          ma = ma == kNegInf ? 0.f : ma;
+          mb = mb == kNegInf ? 0.f : mb;
+          const float la = valid ? __uint_as_float(r[i]) * qscale : kNegInf;
+          const float lb = valid ? __uint_as_float(r[i + 1]) * qscale : kNegInf;
+          const float pa = ex2(la - ma), pb = ex2(lb - mb);
+          psum[i] += pa;
+          psum[i + 1] += pb;
+          pk[i >> 1] = pack_bf16x2(pa, pb);
+        }
+        uint8_t* prow = sP + row * 128;
+#pragma unroll
+        for (int j = 0; j < 4; ++j)
+          *reinterpret_cast<uint4*>(prow + (((hh * 4 + j) ^ (row & 7)) * 16)) =
+              make_uint4(pk[4 * j], pk[4 * j + 1], pk[4 * j + 2], pk[4 * j + 3]);
+        fence_proxy_async();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bar->p_full);
+      }
+      if (!ok) break;
+      // ---- epilogue: o = O^T / (sum_j p_j + 2^(sink - m)) ----------------------
+      if (!mbar_wait(&bar->p_empty, (uint32_t)((g - 1) & 1), err)) break;
+      tc_fence_after();
+      float* rsum = red + (2 * 2 * 4 + hh * 4) * 32;
+      rsum[quad * 32 + lane] = transpose_reduce<false>(psum);
+      if (!group_sync(&bar->grp_soft[hh], gphase, err)) break;
+      const int h_lane = hh * 32 + lane;
+      const float tot = rsum[lane] + rsum[32 + lane] + rsum[64 + lane] + rsum[96 + lane];
+      const float mref = m_run == kNegInf ? 0.f : m_run;
+      const float z = sink != nullptr ? sink[h_lane] * kLog2e : kNegInf;
+      const float den = tot + (z == kNegInf ? 0.f : ex2(z - mref));
+      const float inv = 1.f / den;
+      __nv_bfloat16* ob = out + ((mt.b * n + mt.t) * kNH) * kC;
+      for (int c = 0; c < 4; ++c) {
+        uint32_t o[32];
+        tmem_ld32(lane_base + kColO + c * kNH + hh * 32, o);
+        tmem_ld_wait();
+        const int d = c * 128 + row;
+#pragma unroll
+        for (int i = 0; i < 32; ++i) {
+          const float iv = __shfl_sync(0xffffffffu, inv, i);
+          ob[(int64_t)(hh * 32 + i) * kC + d] = __float2bfloat16_rn(__uint_as_float(o[i]) * iv);
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bar->o_empty);
+      if (!group_sync(&bar->grp_soft[hh], gphase, err)) break;  // rsum is reused next query
+    }
+  }
+  __syncwarp();
+  tc_fence_before();
+  __syncthreads();
+  if (warp == kMmaWarp) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+int sm_count() {
+  static int count = 0;
+  if (count == 0) {
+    int dev = 0;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&count, cudaDevAttrMultiProcessorCount, dev);
+    if (count <= 0) count = 148;
+  }
+  return count;
+}
+
+}  // namespace
+
+bool attn_tc_supported(int nh, int c, int k, csa_dtype dt, const void* q, const void* kv_comp,
+                       const void* kv_win) {
+  if (dt != CSA_BF16 || nh != kNH || c != kC || k > kMaxSel) return false;
+  return ((reinterpret_cast<uintptr_t>(q) | reinterpret_cast<uintptr_t>(kv_comp) |
+           reinterpret_cast<uintptr_t>(kv_win)) & 15) == 0;
+}
+
+cudaError_t launch_attn_tc(const void* q, const void* kv_comp, const int32_t* idx, int k,
+                           const void* kv_win, int window, const float* sink, float scale,
+                           int64_t batch, int64_t n, int m, void* out, unsigned int* err,
+                           cudaStream_t s) {
+  CUtensorMap tq;
+  if (!make_tmap_bf16_3d(&tq, q, kC, (uint64_t)n * kNH, batch, kC * 2ull,
+                         (uint64_t)n * kNH * kC * 2, 64, kNH))
+    return cudaErrorInvalidValue;
+  cudaError_t e = cudaFuncSetAttribute(attn_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       SMEM);
+  if (e != cudaSuccess) return e;
+  const int64_t total = batch * n;
+  const int64_t grid = std::min<int64_t>(total, sm_count());
+  attn_tc_kernel<<<(unsigned)grid, kThreads, SMEM, s>>>(
+      tq, (const __nv_bfloat16*)kv_comp, idx, k, (const __nv_bfloat16*)kv_win, window, sink,
+      scale, n, m, n / m, total, (__nv_bfloat16*)out, err);
+  return cudaGetLastError();
+}
+
+}  // namespace csa

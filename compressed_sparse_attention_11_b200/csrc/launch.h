@@ -23,6 +23,14 @@ cudaError_t launch_index_scores_tc(const void* q_i, const float* w_i, const void
                                    int64_t batch, int64_t n, int nh_i, int c_i, int m,
                                    float* scores, int64_t ld, unsigned int* err, cudaStream_t s);
 
+// tcgen05 attention (bf16, 64 heads of dim 512, up to 2048 selected entries).
+bool attn_tc_supported(int nh, int c, int k, csa_dtype dt, const void* q, const void* kv_comp,
+                       const void* kv_win);
+cudaError_t launch_attn_tc(const void* q, const void* kv_comp, const int32_t* idx, int k,
+                           const void* kv_win, int window, const float* sink, float scale,
+                           int64_t batch, int64_t n, int m, void* out, unsigned int* err,
+                           cudaStream_t s);
+
 cudaError_t launch_compress(const void* ca, const void* cb, const void* za, const void* zb,
                             const float* ba, const float* bb, int64_t batch, int64_t n, int c,
                             int m, int overlap, csa_dtype dt, void* out, cudaStream_t s);

@@ -169,6 +169,7 @@ def test_sparse_attn_parity(B, n, nh, c, m, k, W, dt, rows):
     idx = _random_selection(B, n, m, k, seed=5)
     out = csa.csa_sparse_attn(q.to(DEV), kv.to(DEV), torch.tensor(idx).to(DEV), win.to(DEV), W,
                               sink.to(DEV), 1 / math.sqrt(c), m)
+    csa.csa_check()
     g = host(out)
     rr = list(range(n)) if rows is None else sorted(set(list(range(0, 8)) + list(range(n - 8, n)) +
                                                         list(range(5, n, 61))))
@@ -177,14 +178,53 @@ def test_sparse_attn_parity(B, n, nh, c, m, k, W, dt, rows):
         check_close(g[b, rr], ref, dt, f"sparse attn b={b}")
 
 
+def _messy_selection(B, n, m, k, seed):
+    """Valid entries in ascending order with -1, negative and future (>= V)
+    indices sprinkled between them; only the valid ones may be attended."""
+    r = np.random.default_rng(seed)
+    idx = np.full((B, n, k), -1, dtype=np.int32)
+    for b in range(B):
+        for t in range(n):
+            V = O.visible(t, m)
+            cnt = int(r.integers(0, min(k, V) + 1)) if V else 0
+            ch = np.sort(r.choice(V, size=cnt, replace=False)) if cnt else np.zeros(0, int)
+            slots = np.sort(r.choice(k, size=cnt, replace=False))
+            row = r.choice([-1, -5, V, V + 3, 10 ** 6], size=k).astype(np.int32)
+            row[slots] = ch
+            idx[b, t] = row
+    return idx
+
+
+@pytest.mark.parametrize("B,n,k,W,sink_none", [
+    (2, 700, 96, 200, False),    # window longer than a tile boundary, batch 2
+    (1, 300, 2048, 7, True),     # the largest selection, tiny window, no sink
+])
+def test_sparse_attn_tensor_core_messy_selection(B, n, k, W, sink_none):
+    nh, c, m = 64, 512, 4
+    q, kv, win, sink = _attn_inputs(B, n, nh, c, m, torch.bfloat16, seed=41)
+    idx = _messy_selection(B, n, m, k, seed=6)
+    s_dev = None if sink_none else sink.to(DEV)
+    out = csa.csa_sparse_attn(q.to(DEV), kv.to(DEV), torch.tensor(idx).to(DEV), win.to(DEV), W,
+                              s_dev, 1 / math.sqrt(c), m)
+    csa.csa_check()
+    g = host(out)
+    rr = sorted(set(list(range(0, 12)) + list(range(n - 12, n)) + list(range(5, n, 23))))
+    for b in range(B):
+        ref = O.sparse_attn(q[b], kv[b], idx[b], win[b], W, None if sink_none else sink,
+                            1 / math.sqrt(c), m, rows=rr)
+        check_close(g[b, rr], ref, torch.bfloat16, f"sparse attn b={b}")
+
+
 @pytest.mark.parametrize("B,n,nh,c,m,W,dt,rows", [
     (1, 2048, 64, 512, 128, 128, torch.bfloat16, "sample"),
+    (2, 1100, 64, 512, 16, 64, torch.bfloat16, "sample"),   # more entries than a tile
     (2, 700, 16, 128, 32, 50, torch.float32, None),
     (1, 64, 4, 32, 128, 128, torch.float32, None),    # no entry complete: window only
 ])
 def test_hca_attn_parity(B, n, nh, c, m, W, dt, rows):
     q, kv, win, sink = _attn_inputs(B, n, nh, c, m, dt, seed=23)
     out = csa.hca_attn(q.to(DEV), kv.to(DEV), win.to(DEV), W, sink.to(DEV), 1 / math.sqrt(c), m)
+    csa.csa_check()
     g = host(out)
     rr = list(range(n)) if rows is None else sorted(set(list(range(0, 8)) + list(range(n - 8, n)) +
                                                         list(range(120, 140)) +
