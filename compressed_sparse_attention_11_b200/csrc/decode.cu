@@ -26,6 +26,11 @@
 
 namespace csa {
 
+constexpr int kSelThreads = 512;          // CUDA-core chunk top-k / merge blocks
+constexpr int kDecSelThreads = 1024;      // one selection block per sequence
+constexpr int kDecSelCap = 8192;          // candidates kept above the sampled threshold
+constexpr int kDecSelSample = 4096;       // sample size of the threshold estimate
+
 static inline size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
 
 void cache_layout(const csa_cache_desc& d, csa_cache_layout_t* L) {
@@ -240,8 +245,8 @@ __global__ void __launch_bounds__(kSelThreads) index_chunk_kernel(
     const __nv_bfloat16* __restrict__ q_i, const float* __restrict__ w_i, int nchunks,
     float* __restrict__ cand_score, int32_t* __restrict__ cand_idx) {
   extern __shared__ __align__(16) unsigned char smem_raw[];
-  SelectShared& sh = *reinterpret_cast<SelectShared*>(smem_raw);
-  uint32_t* keys = reinterpret_cast<uint32_t*>(smem_raw + sizeof(SelectShared));  // [kDecChunk]
+  SelectShared<kSelThreads>& sh = *reinterpret_cast<SelectShared<kSelThreads>*>(smem_raw);
+  uint32_t* keys = reinterpret_cast<uint32_t*>(smem_raw + sizeof(SelectShared<kSelThreads>));
   float* sc = reinterpret_cast<float*>(keys + kDecChunk);                          // [kDecChunk]
   int32_t* pick = reinterpret_cast<int32_t*>(sc + kDecChunk);                      // [k]
   float* qs = reinterpret_cast<float*>(pick + ((d.k + 3) & ~3));  // [c_i][nh_i]
@@ -301,7 +306,7 @@ __global__ void __launch_bounds__(kSelThreads) index_chunk_kernel(
     }
     return;
   }
-  block_select_topk(KeysInSmem{keys}, Vc, d.k, pick, nullptr, sh);
+  block_select_topk<kSelThreads>(KeysInSmem{keys}, Vc, d.k, pick, nullptr, sh);
   for (int j = threadIdx.x; j < d.k; j += blockDim.x) {
     const int32_t pp = pick[j];
     oid[j] = (int32_t)(c0 + pp);
@@ -314,7 +319,7 @@ __global__ void __launch_bounds__(kSelThreads) topk_merge_kernel(
     csa_cache_desc d, const int64_t* __restrict__ pos, int nchunks,
     const float* __restrict__ cand_score, const int32_t* __restrict__ cand_idx,
     int32_t* __restrict__ sel) {
-  __shared__ SelectShared sh;
+  __shared__ SelectShared<kSelThreads> sh;
   const int64_t b = blockIdx.x;
   const int64_t t = pos[b];
   const int64_t V = min((t + 1) / d.m, d.capacity);
@@ -326,7 +331,27 @@ __global__ void __launch_bounds__(kSelThreads) topk_merge_kernel(
   const int64_t N = (int64_t)nchunks * d.k;
   const float* s = cand_score + b * N;
   const int32_t* id = cand_idx + b * N;
-  block_select_topk(CandidatesInGlobal{s, id}, N, d.k, out, id, sh);
+  block_select_topk<kSelThreads>(CandidatesInGlobal{s, id}, N, d.k, out, id, sh);
+}
+
+// Step 3' (CSA, tensor-core indexer): top-k over one sequence's score array.
+__global__ void __launch_bounds__(kDecSelThreads) decode_select_kernel(
+    csa_cache_desc d, const int64_t* __restrict__ pos, const float* __restrict__ scores,
+    int32_t* __restrict__ sel) {
+  extern __shared__ __align__(16) unsigned char smem_raw[];
+  SelectShared<kDecSelThreads>& sh = *reinterpret_cast<SelectShared<kDecSelThreads>*>(smem_raw);
+  int32_t* cand = reinterpret_cast<int32_t*>(smem_raw + sizeof(SelectShared<kDecSelThreads>));
+  uint32_t* sample = reinterpret_cast<uint32_t*>(cand + kDecSelCap);
+  const int64_t b = blockIdx.x;
+  const int64_t t = pos[b];
+  const int64_t V = t < 0 ? 0 : min((t + 1) / d.m, d.capacity);
+  int32_t* out = sel + b * d.k;
+  if (V <= d.k) {
+    for (int j = threadIdx.x; j < d.k; j += blockDim.x) out[j] = j < V ? j : -1;
+    return;
+  }
+  block_select_topk_sampled<kDecSelThreads>(ScoresIn{scores + b * d.capacity}, V, d.k, out, sh,
+                                            cand, kDecSelCap, sample, kDecSelSample);
 }
 
 // ---------------------------------------------------------------------------
@@ -488,18 +513,23 @@ __global__ void __launch_bounds__(256) attn_combine_kernel(
 // ---------------------------------------------------------------------------
 struct DecodeWs {
   int nchunks, nsplit;
-  size_t cand_score, cand_idx, sel, part_o, part_ms, total;
+  bool tc_index, tc_attn;
+  size_t cand_score, cand_idx, scores, sel, part_o, part_ms, total;
 };
 
 static DecodeWs decode_ws_layout(const csa_cache_desc& d) {
   DecodeWs w;
-  w.nchunks = d.is_hca ? 0 : (int)((d.capacity + kDecChunk - 1) / kDecChunk);
+  w.tc_index = decode_index_tc_supported(d);
+  w.nchunks = (d.is_hca || w.tc_index) ? 0 : (int)((d.capacity + kDecChunk - 1) / kDecChunk);
   const int64_t max_slots = (d.is_hca ? d.capacity : (int64_t)d.k) + d.window;
-  w.nsplit = (int)std::min<int64_t>(128, std::max<int64_t>(1, (max_slots + 63) / 64));
+  w.tc_attn = decode_attn_tc_supported(d);
+  w.nsplit = w.tc_attn ? decode_attn_splits(d)
+                       : (int)std::min<int64_t>(128, std::max<int64_t>(1, (max_slots + 63) / 64));
   const size_t B = (size_t)d.batch;
   size_t off = 0;
   w.cand_score = off; off = align256(off + B * w.nchunks * d.k * 4);
   w.cand_idx = off;   off = align256(off + B * w.nchunks * d.k * 4);
+  w.scores = off;     off = align256(off + (w.tc_index ? B * (size_t)d.capacity * 4 : 0));
   w.sel = off;        off = align256(off + B * (d.is_hca ? 0 : d.k) * 4);
   w.part_o = off;     off = align256(off + B * w.nsplit * d.nh * (size_t)d.c * 4);
   w.part_ms = off;    off = align256(off + B * w.nsplit * d.nh * 2 * 4);
@@ -525,8 +555,20 @@ cudaError_t launch_decode_step(const csa_cache_desc& d, const CacheView& cv, con
   append_emit_kernel<<<(unsigned)d.batch, 256, emit_smem, s>>>(d, cv, pos, rows, p);
   cudaError_t err = cudaGetLastError();
   if (err != cudaSuccess) return err;
-  if (!d.is_hca) {
-    const size_t smem = sizeof(SelectShared) + (size_t)kDecChunk * 8 +
+  if (!d.is_hca && w.tc_index) {
+    float* scores = reinterpret_cast<float*>(wb + w.scores);
+    unsigned int* flag = device_timeout_flag();
+    if (flag == nullptr) return cudaErrorUnknown;
+    err = launch_decode_index_tc(d, cv, pos, q_i, w_i, scores, flag, s);
+    if (err != cudaSuccess) return err;
+    const size_t smem = sizeof(SelectShared<kDecSelThreads>) + (size_t)kDecSelCap * 4 +
+                        (size_t)kDecSelSample * 4;
+    cudaFuncSetAttribute(decode_select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                         (int)smem);
+    decode_select_kernel<<<(unsigned)d.batch, kDecSelThreads, smem, s>>>(d, pos, scores, sel);
+    if ((err = cudaGetLastError()) != cudaSuccess) return err;
+  } else if (!d.is_hca) {
+    const size_t smem = sizeof(SelectShared<kSelThreads>) + (size_t)kDecChunk * 8 +
                         (size_t)((d.k + 3) & ~3) * 4 + (size_t)d.c_i * d.nh_i * 4 +
                         (size_t)d.nh_i * 4;
     cudaFuncSetAttribute(index_chunk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -538,11 +580,21 @@ cudaError_t launch_decode_step(const csa_cache_desc& d, const CacheView& cv, con
                                                                 cand_idx, sel);
     if ((err = cudaGetLastError()) != cudaSuccess) return err;
   }
+  const unsigned hgroups = (unsigned)((d.nh + kDecHG - 1) / kDecHG);
+  if (w.tc_attn) {
+    unsigned int* flag = device_timeout_flag();
+    if (flag == nullptr) return cudaErrorUnknown;
+    err = launch_decode_attn_tc(d, cv, pos, q, sel, p.sink, p.scale, w.nsplit, out, part_o,
+                                part_ms, flag, s);
+    if (err != cudaSuccess || w.nsplit == 1) return err;
+    attn_combine_kernel<<<dim3((unsigned)d.batch, hgroups), 256, 0, s>>>(
+        d, p.sink, w.nsplit, part_o, part_ms, (__nv_bfloat16*)out);
+    return cudaGetLastError();
+  }
   const size_t asmem = sizeof(float) * ((size_t)kDecTE * (d.c + 1) + (size_t)kDecHG * d.c +
                                         kDecHG * kDecTE) + sizeof(int64_t) * kDecTE;
   cudaFuncSetAttribute(attn_split_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                        (int)asmem);
-  const unsigned hgroups = (unsigned)((d.nh + kDecHG - 1) / kDecHG);
   attn_split_kernel<<<dim3(w.nsplit, hgroups, (unsigned)d.batch), 256, asmem, s>>>(
       d, cv, pos, (const __nv_bfloat16*)q, sel, p.scale, w.nsplit, part_o, part_ms);
   if ((err = cudaGetLastError()) != cudaSuccess) return err;

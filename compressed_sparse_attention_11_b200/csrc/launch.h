@@ -31,6 +31,22 @@ cudaError_t launch_attn_tc(const void* q, const void* kv_comp, const int32_t* id
                            int64_t batch, int64_t n, int m, void* out, unsigned int* err,
                            cudaStream_t s);
 
+// tcgen05 decode indexer over FP8 keys (c_i = 128, nh_i in {16, 32, 64, 128}).
+struct CacheView;
+bool decode_index_tc_supported(const csa_cache_desc& d);
+cudaError_t launch_decode_index_tc(const csa_cache_desc& d, const CacheView& cv,
+                                   const int64_t* pos, const void* q_i, const float* w_i,
+                                   float* scores, unsigned int* err, cudaStream_t s);
+
+// tcgen05 decode attention (64 heads x 512, FP8/bf16 cache), split-K.
+bool decode_attn_tc_supported(const csa_cache_desc& d);
+int decode_attn_splits(const csa_cache_desc& d);
+cudaError_t launch_decode_attn_tc(const csa_cache_desc& d, const CacheView& cv,
+                                  const int64_t* pos, const void* q, const int32_t* sel,
+                                  const float* sink, float scale, int nsplit, void* out,
+                                  float* part_o, float* part_ms, unsigned int* err,
+                                  cudaStream_t s);
+
 cudaError_t launch_compress(const void* ca, const void* cb, const void* za, const void* zb,
                             const float* ba, const float* bb, int64_t batch, int64_t n, int c,
                             int m, int overlap, csa_dtype dt, void* out, cudaStream_t s);

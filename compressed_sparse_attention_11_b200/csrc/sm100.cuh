@@ -233,10 +233,16 @@ __device__ __forceinline__ void tmem_st_wait() {
 }  // namespace sm100
 
 // ---- host: tensor maps -----------------------------------------------------------
-// Encodes a 3-D bf16 tensor map (x innermost) with the 128-byte swizzle.
-// Returns false if the driver entry point is unavailable or rejects the map.
-bool make_tmap_bf16_3d(CUtensorMap* map, const void* base, uint64_t x, uint64_t y, uint64_t z,
-                       uint64_t stride_y_bytes, uint64_t stride_z_bytes, uint32_t box_x,
-                       uint32_t box_y);
+// Encodes a 3-D tensor map (x innermost) with the 128-byte swizzle; elem_bytes
+// 2 = bf16, 1 = uint8.  Returns false if the driver entry point is
+// unavailable or rejects the map.
+bool make_tmap_3d(CUtensorMap* map, const void* base, int elem_bytes, uint64_t x, uint64_t y,
+                  uint64_t z, uint64_t stride_y_bytes, uint64_t stride_z_bytes, uint32_t box_x,
+                  uint32_t box_y);
+inline bool make_tmap_bf16_3d(CUtensorMap* map, const void* base, uint64_t x, uint64_t y,
+                              uint64_t z, uint64_t stride_y_bytes, uint64_t stride_z_bytes,
+                              uint32_t box_x, uint32_t box_y) {
+  return make_tmap_3d(map, base, 2, x, y, z, stride_y_bytes, stride_z_bytes, box_x, box_y);
+}
 
 }  // namespace csa

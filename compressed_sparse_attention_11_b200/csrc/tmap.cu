@@ -24,16 +24,18 @@ void resolve() {
 }
 }  // namespace
 
-bool make_tmap_bf16_3d(CUtensorMap* map, const void* base, uint64_t x, uint64_t y, uint64_t z,
-                       uint64_t stride_y_bytes, uint64_t stride_z_bytes, uint32_t box_x,
-                       uint32_t box_y) {
+bool make_tmap_3d(CUtensorMap* map, const void* base, int elem_bytes, uint64_t x, uint64_t y,
+                  uint64_t z, uint64_t stride_y_bytes, uint64_t stride_z_bytes, uint32_t box_x,
+                  uint32_t box_y) {
   std::call_once(g_once, resolve);
   if (!g_encode) return false;
   const cuuint64_t dims[3] = {x, y, z};
   const cuuint64_t strides[2] = {stride_y_bytes, stride_z_bytes};
   const cuuint32_t box[3] = {box_x, box_y, 1};
   const cuuint32_t estr[3] = {1, 1, 1};
-  CUresult r = g_encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims,
+  const CUtensorMapDataType dt =
+      elem_bytes == 1 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+  CUresult r = g_encode(map, dt, 3, const_cast<void*>(base), dims,
                         strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
                         CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                         CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);

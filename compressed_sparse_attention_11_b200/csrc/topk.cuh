@@ -1,23 +1,32 @@
 // Block-wide exact top-k select (radix select, no sort), shared by the
-// prefill top-k kernel and the decode candidate merge.
+// prefill top-k kernel and the decode selection.
 //
 // Order: larger score first; among equal scores the earlier position wins.
 // The chosen positions are emitted in ascending position order, which is the
 // order the selection is compacted in, so no sort is needed.
+//
+// Two front ends:
+//   block_select_topk          radix select over all V keys (4 histogram
+//                              passes + 2 compaction passes);
+//   block_select_topk_sampled  estimates a threshold from a strided sample,
+//                              keeps the (few) keys at or above it in order,
+//                              and runs the exact radix select on those only
+//                              -- two passes over V instead of six.  It falls
+//                              back to the full select when the estimate
+//                              keeps fewer than k or more than `cap` keys.
 #pragma once
 
 #include "common.cuh"
 
 namespace csa {
 
-constexpr int kSelThreads = 512;
-constexpr int kSelWarps = kSelThreads / 32;
-
+template <int NT>
 struct SelectShared {
-  uint32_t hist[kSelWarps][256];
+  static constexpr int kWarps = NT / 32;
+  uint32_t hist[kWarps][256];
   uint32_t total[256];
-  uint32_t warp_a[kSelWarps];
-  uint32_t warp_b[kSelWarps];
+  uint32_t warp_a[kWarps];
+  uint32_t warp_b[kWarps];
   uint32_t digit, remaining;
 };
 
@@ -26,7 +35,7 @@ struct KeysInSmem {
   const uint32_t* k;
   __device__ __forceinline__ uint32_t key(int64_t i) const { return k[i]; }
 };
-struct ScoresInGlobal {
+struct ScoresIn {
   const float* s;
   __device__ __forceinline__ uint32_t key(int64_t i) const { return order_key(s[i]); }
 };
@@ -37,20 +46,26 @@ struct CandidatesInGlobal {  // (score, index) pairs; index < 0 is padding
     return id[i] < 0 ? 0u : order_key(s[i]);
   }
 };
-
-// Selects the k largest keys among positions [0, V) (V > k) and writes, in
-// ascending position order, out[j] = map ? map[pos] : pos.  All threads of a
-// kSelThreads block must call it.
 template <class Src>
-__device__ void block_select_topk(const Src& src, int64_t V, int k, int32_t* __restrict__ out,
-                                  const int32_t* __restrict__ map, SelectShared& sh) {
+struct Gathered {  // keys of positions pos[0..)
+  Src src;
+  const int32_t* pos;
+  __device__ __forceinline__ uint32_t key(int64_t i) const { return src.key(pos[i]); }
+};
+
+// Radix search for the key T of the k-th largest element among [0, V)
+// (1 <= k <= V) and the number of elements equal to T inside the top k.
+template <int NT, class Src>
+__device__ void radix_kth(const Src& src, int64_t V, int k, SelectShared<NT>& sh, uint32_t& T,
+                          uint32_t& take_eq) {
+  constexpr int W = NT / 32;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   uint32_t prefix = 0, mask = 0;
   if (tid == 0) sh.remaining = (uint32_t)k;
   for (int shift = 24; shift >= 0; shift -= 8) {
-    for (int i = tid; i < kSelWarps * 256; i += kSelThreads) (&sh.hist[0][0])[i] = 0;
+    for (int i = tid; i < W * 256; i += NT) (&sh.hist[0][0])[i] = 0;
     __syncthreads();
-    for (int64_t i = tid; i < V; i += kSelThreads) {
+    for (int64_t i = tid; i < V; i += NT) {
       const uint32_t u = src.key(i);
       const bool in = (u & mask) == prefix;
       const uint32_t dig = (u >> shift) & 255u;
@@ -62,11 +77,11 @@ __device__ void block_select_topk(const Src& src, int64_t V, int k, int32_t* __r
       }
     }
     __syncthreads();
-    if (tid < 256) {
+    for (int d = tid; d < 256; d += NT) {
       uint32_t s = 0;
 #pragma unroll
-      for (int w = 0; w < kSelWarps; ++w) s += sh.hist[w][tid];
-      sh.total[tid] = s;
+      for (int w = 0; w < W; ++w) s += sh.hist[w][d];
+      sh.total[d] = s;
     }
     __syncthreads();
     if (warp == 0) {
@@ -100,11 +115,20 @@ __device__ void block_select_topk(const Src& src, int64_t V, int k, int32_t* __r
     mask |= 255u << shift;
     __syncthreads();
   }
-  const uint32_t T = prefix;             // key of the k-th largest element
-  const uint32_t take_eq = sh.remaining; // how many elements equal to T are chosen
+  T = prefix;
+  take_eq = sh.remaining;
+  __syncthreads();
+}
 
-  // contiguous segment per warp, a multiple of 32 long
-  const int64_t seg = ((V + kSelWarps - 1) / kSelWarps + 31) / 32 * 32;
+// Writes, in ascending position order, out[j] = map ? map[pos] : pos for the
+// positions whose key is > T, plus the first take_eq positions whose key == T.
+template <int NT, class Src>
+__device__ void emit_selected(const Src& src, int64_t V, uint32_t T, uint32_t take_eq, int k,
+                              int32_t* __restrict__ out, const int32_t* __restrict__ map,
+                              SelectShared<NT>& sh) {
+  constexpr int W = NT / 32;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int64_t seg = ((V + W - 1) / W + 31) / 32 * 32;  // contiguous per warp
   const int64_t lo = (int64_t)warp * seg, hi = min(V, lo + seg);
   uint32_t gt = 0, eq = 0;
   for (int64_t base = lo; base < hi; base += 32) {
@@ -140,6 +164,75 @@ __device__ void block_select_topk(const Src& src, int64_t V, int k, int32_t* __r
     run_sel += __popc(sel_mask);
   }
   __syncthreads();
+}
+
+// Selects the k largest keys among positions [0, V) (V >= k) and writes, in
+// ascending position order, out[j] = map ? map[pos] : pos.  All NT threads
+// of the block must call it.
+template <int NT, class Src>
+__device__ void block_select_topk(const Src& src, int64_t V, int k, int32_t* __restrict__ out,
+                                  const int32_t* __restrict__ map, SelectShared<NT>& sh) {
+  uint32_t T, take_eq;
+  radix_kth<NT>(src, V, k, sh, T, take_eq);
+  emit_selected<NT>(src, V, T, take_eq, k, out, map, sh);
+}
+
+// Same result as block_select_topk (positions, no map).  `cand` is scratch
+// for up to `cap` positions and `sample` for `nsample` keys, both owned by
+// the block (shared or global memory).
+template <int NT, class Src>
+__device__ void block_select_topk_sampled(const Src& src, int64_t V, int k,
+                                          int32_t* __restrict__ out, SelectShared<NT>& sh,
+                                          int32_t* __restrict__ cand, int cap,
+                                          uint32_t* __restrict__ sample, int nsample) {
+  constexpr int W = NT / 32;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  if (V <= (int64_t)cap || nsample < 64) {
+    block_select_topk<NT>(src, V, k, out, nullptr, sh);
+    return;
+  }
+  // 1. threshold from a strided sample: about 1.5x the wanted share, + 16
+  const int S = nsample;
+  for (int i = tid; i < S; i += NT) sample[i] = src.key((V * (int64_t)i) / S);
+  __syncthreads();
+  const int r = min(S, (int)((1.5 * S * (double)k) / (double)V) + 16);
+  uint32_t T0, unused;
+  radix_kth<NT>(KeysInSmem{sample}, S, r, sh, T0, unused);
+  // 2. count the keys >= T0 (per warp over a contiguous segment)
+  const int64_t seg = ((V + W - 1) / W + 31) / 32 * 32;
+  const int64_t lo = (int64_t)warp * seg, hi = min(V, lo + seg);
+  uint32_t c = 0;
+  for (int64_t base = lo; base < hi; base += 32) {
+    const int64_t i = base + lane;
+    c += __popc(__ballot_sync(0xffffffffu, i < hi && src.key(i) >= T0));
+  }
+  if (lane == 0) sh.warp_a[warp] = c;
+  __syncthreads();
+  uint32_t before = 0, total = 0;
+  for (int w = 0; w < W; ++w) {
+    const uint32_t x = sh.warp_a[w];
+    if (w < warp) before += x;
+    total += x;
+  }
+  __syncthreads();
+  if (total < (uint32_t)k || total > (uint32_t)cap) {  // the estimate missed: exact path
+    block_select_topk<NT>(src, V, k, out, nullptr, sh);
+    return;
+  }
+  // 3. keep those positions in order, then the exact select among them
+  const uint32_t lt_mask = (1u << lane) - 1u;
+  uint32_t run = before;
+  for (int64_t base = lo; base < hi; base += 32) {
+    const int64_t i = base + lane;
+    const bool keep = i < hi && src.key(i) >= T0;
+    const uint32_t msk = __ballot_sync(0xffffffffu, keep);
+    if (keep) cand[run + __popc(msk & lt_mask)] = (int32_t)i;
+    run += __popc(msk);
+  }
+  __syncthreads();
+  // candidates are in ascending position order: emitting the chosen slots in
+  // order and mapping each slot to its position keeps the output ascending
+  block_select_topk<NT>(Gathered<Src>{src, cand}, total, k, out, cand, sh);
 }
 
 }  // namespace csa

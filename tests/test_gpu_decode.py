@@ -104,6 +104,7 @@ def _run_and_compare(w, B, E, steps, seed, check_seqs=None):
         qi = None if w.is_hca else inp["q_i"][s].to(DEV)
         wi = None if w.is_hca else inp["w_i"][s].to(DEV)
         out = host(cache.decode_step(pos, rows, dbias, sink, w.scale, q, qi, wi))
+        csa.csa_check()
         for b in check_seqs:
             ref, _ = seqs[b].step(t, {nm: inp["rows_" + nm][b, r] for nm in names}, biases,
                                   inp["q"][s, b], None if w.is_hca else inp["q_i"][s, b],
@@ -149,6 +150,20 @@ def test_decode_csa_realistic_dims_two_chunks():
     w = G.Decode("csa_decode_dims", 2, 0, 512, 64, 4, 64, 128, False, nh_i=64, c_i=128, k=512,
                  seed=103)
     _run_and_compare(w, B=2, E=2500, steps=4, seed=10)
+
+
+def test_decode_hca_realistic_dims_split_k():
+    """64 heads x 512, FP8/bf16 cache, dense over ~300 entries: the tensor-core
+    attention splits the entry set over several CTAs and a combine kernel."""
+    w = G.Decode("hca_decode_dims", 2, 0, 512, 64, 128, 64, 128, True, seed=104)
+    _run_and_compare(w, B=2, E=300, steps=2, seed=11)
+
+
+def test_decode_csa_many_sequences_one_split():
+    """Enough sequences that each gets a single attention CTA (no combine)."""
+    w = G.Decode("csa_decode_many", 80, 0, 512, 64, 4, 64, 128, False, nh_i=64, c_i=128, k=64,
+                 seed=105)
+    _run_and_compare(w, B=80, E=40, steps=5, seed=12, check_seqs=[0, 37, 79])
 
 
 def test_write_rows_fills_ring_and_state():
