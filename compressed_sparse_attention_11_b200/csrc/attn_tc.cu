@@ -32,6 +32,7 @@
 #include "common.cuh"
 #include "launch.h"
 #include "sm100.cuh"
+#include "tc_attn_util.cuh"
 
 #include <algorithm>
 
@@ -58,34 +59,9 @@ constexpr uint32_t kColS = 0;    // S^T, double-buffered: 2 x 64 columns
 constexpr uint32_t kColO = 128;  // O^T: 4 chunks x 64 columns
 
 struct __align__(16) AttnMeta {
-  int ntiles, nrows, tile_lo, split;
+  int ntiles, nrows;
   int64_t t, b;
 };
-
-// Decode-mode extras: the FP8 cache, split-K partial outputs.
-struct DecodeSide {
-  CacheView cv;
-  const int64_t* pos;  // [batch] position of each sequence's token
-  int nsplit;          // CTAs (work items) per sequence
-  int rope;            // trailing bf16 dims of an entry
-  float* part_o;       // [batch][nsplit][64][512] unnormalised O (nsplit > 1)
-  float* part_ms;      // [batch][nsplit][64][2]   running max (log2), sum
-};
-
-// Work item qi -> (sequence, position, split).
-template <bool kDec>
-__device__ __forceinline__ void query_of(int64_t qi, int64_t n, const DecodeSide& ds, int64_t& b,
-                                         int64_t& t, int& split) {
-  if (kDec) {
-    b = qi / ds.nsplit;
-    split = (int)(qi % ds.nsplit);
-    t = ds.pos[b];
-  } else {
-    b = qi / n;
-    t = qi % n;
-    split = 0;
-  }
-}
 
 struct __align__(8) AttnBars {
   uint64_t slab_full[kSlabs], slab_empty[kSlabs];
@@ -105,45 +81,11 @@ constexpr int OFF_BAR = OFF_SCAN + 64;
 constexpr int SMEM = OFF_BAR + (int)sizeof(AttnBars) + 1024;
 static_assert(SMEM <= 232448, "shared memory budget");
 
-// Bounded barrier among the 4 warps that share `bar` (one arrive per warp).
-__device__ __forceinline__ bool group_sync(uint64_t* bar, uint32_t& phase, unsigned int* err) {
-  __syncwarp();
-  if ((threadIdx.x & 31) == 0) sm100::mbar_arrive(bar);
-  const bool ok = sm100::mbar_wait(bar, phase & 1, err);
-  ++phase;
-  return ok;
-}
-
-// Lane i ends with the reduction (max or sum) of element i over the 32 lanes.
-template <bool kMax>
-__device__ __forceinline__ float transpose_reduce(float (&v)[32]) {
-  const int lane = threadIdx.x & 31;
-#pragma unroll
-  for (int half = 16; half >= 1; half >>= 1) {
-    const bool upper = (lane & half) != 0;
-#pragma unroll
-    for (int i = 0; i < half; ++i) {
-      const float send = upper ? v[i] : v[i + half];
-      const float keep = upper ? v[i + half] : v[i];
-      const float recv = __shfl_xor_sync(0xffffffffu, send, half);
-      v[i] = kMax ? fmaxf(keep, recv) : keep + recv;
-    }
-  }
-  return v[0];
-}
-
-// kDec = false: prefill (q [B][n][64][512], entries kv_comp / kv_win, bf16).
-// kDec = true: one token per sequence over the FP8/bf16 decode cache;
-// idx is then the per-sequence selection [B][k] (nullptr for HCA), E the
-// cache capacity, and with ds.nsplit > 1 each work item covers a slice of
-// the entry set and writes partial (O, max, sum) for the combine kernel.
-template <bool kDec>
 __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(
     const __grid_constant__ CUtensorMap tm_q, const __nv_bfloat16* __restrict__ kv_comp,
     const int32_t* __restrict__ idx, int k, const __nv_bfloat16* __restrict__ kv_win,
     int window, const float* __restrict__ sink, float scale, int64_t n, int m, int64_t E,
-    int64_t total, __nv_bfloat16* __restrict__ out, unsigned int* __restrict__ err,
-    const __grid_constant__ DecodeSide ds) {
+    int64_t total, __nv_bfloat16* __restrict__ out, unsigned int* __restrict__ err) {
   using namespace sm100;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = smem_raw + ((1024 - (smem_u32(smem_raw) & 1023)) & 1023);
@@ -202,12 +144,10 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(
     for (int64_t kq = 0; ok; ++kq) {
       const int64_t qi = blockIdx.x + kq * gridDim.x;
       if (qi >= total) break;
-      int64_t b, t;
-      int split;
-      query_of<kDec>(qi, n, ds, b, t, split);
-      const int64_t V = t < 0 ? 0 : min((t + 1) / m, E);
+      const int64_t b = qi / n, t = qi % n;
+      const int64_t V = min((t + 1) / m, E);
       const int64_t w0 = max((int64_t)0, t - window + 1);
-      const int nwin = t < 0 ? 0 : (int)(t - w0 + 1);
+      const int nwin = (int)(t - w0 + 1);
       // the previous query's list is no longer read
       if (!group_sync(&bar->grp_prod, gphase, err)) break;
       int nsel;
@@ -215,7 +155,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(
         // compact the valid selections, keeping their order
         const int per = (k + kProdThreads - 1) / kProdThreads;
         const int lo = min(k, ptid * per), hi = min(k, lo + per);
-        const int32_t* row = kDec ? idx + b * k : idx + (b * n + t) * k;
+        const int32_t* row = idx + (b * n + t) * k;
         int cnt = 0;
         for (int j = lo; j < hi; ++j) {
           const int s = row[j];
@@ -245,16 +185,11 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(
         nsel = (int)V;
       }
       const int N = nsel + nwin;
-      const int Tall = (N + kTE - 1) / kTE;
-      const int nsp = kDec ? ds.nsplit : 1;
-      const int tlo = (int)(((int64_t)Tall * split) / nsp);
-      const int T = (int)(((int64_t)Tall * (split + 1)) / nsp) - tlo;
+      const int T = (N + kTE - 1) / kTE;
       if (ptid == 0) {
         AttnMeta& mt = meta[kq & 1];
         mt.ntiles = T;
         mt.nrows = N;
-        mt.tile_lo = tlo;
-        mt.split = split;
         mt.t = t;
         mt.b = b;
         mbar_arrive(&bar->meta_full[kq & 1]);
@@ -263,121 +198,40 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(
         if (ok) {
           mbar_arrive_expect_tx(&bar->q_full, kSlabs * kQSlabBytes);
           for (int s = 0; s < kSlabs; ++s)
-            tma_load_3d(sQ + s * kQSlabBytes, &tm_q, &bar->q_full, s * 64,
-                        kDec ? 0 : (int)(t * kNH), (int)b);
+            tma_load_3d(sQ + s * kQSlabBytes, &tm_q, &bar->q_full, s * 64, (int)(t * kNH), (int)b);
           q_issued = kq;
         }
       }
       for (int tt = 0; tt < T && ok; ++tt, ++g) {
-        const int tile = tlo + tt;
-        if constexpr (!kDec) {
-          // this thread's rows of the tile: global row pointers (nullptr = zero fill)
-          const __nv_bfloat16* src[kPasses];
+        // this thread's rows of the tile: global row pointers (nullptr = zero fill)
+        const __nv_bfloat16* src[kPasses];
+#pragma unroll
+        for (int rr = 0; rr < kPasses; ++rr) {
+          const int slot = tt * kTE + (ptid >> 3) + kRowsPerPass * rr;
+          const __nv_bfloat16* p = nullptr;
+          if (slot < nsel) {
+            const int64_t e = idx != nullptr ? (int64_t)list[slot] : (int64_t)slot;
+            p = kv_comp + (b * E + e) * kC;
+          } else if (slot < N) {
+            p = kv_win + (b * n + w0 + (slot - nsel)) * kC;
+          }
+          src[rr] = p;
+        }
+        for (int s = 0; s < kSlabs; ++s) {
+          if (g >= 1 && !mbar_wait(&bar->slab_empty[s], (uint32_t)((g - 1) & 1), err)) {
+            ok = false;
+            break;
+          }
+          uint8_t* dst = sKV + s * kSlabBytes;
 #pragma unroll
           for (int rr = 0; rr < kPasses; ++rr) {
-            const int slot = tile * kTE + (ptid >> 3) + kRowsPerPass * rr;
-            const __nv_bfloat16* p = nullptr;
-            if (slot < nsel) {
-              const int64_t e = idx != nullptr ? (int64_t)list[slot] : (int64_t)slot;
-              p = kv_comp + (b * E + e) * kC;
-            } else if (slot < N) {
-              p = kv_win + (b * n + w0 + (slot - nsel)) * kC;
-            }
-            src[rr] = p;
+            const int row = (ptid >> 3) + kRowsPerPass * rr;
+            if (row >= kTE) continue;
+            const __nv_bfloat16* p = src[rr] != nullptr ? src[rr] + s * 64 + chunk * 8 : kv_win;
+            cp_async_16(dst + row * 128 + ((chunk ^ (row & 7)) * 16), p,
+                        src[rr] != nullptr ? 16u : 0u);
           }
-          for (int s = 0; s < kSlabs; ++s) {
-            if (g >= 1 && !mbar_wait(&bar->slab_empty[s], (uint32_t)((g - 1) & 1), err)) {
-              ok = false;
-              break;
-            }
-            uint8_t* dst = sKV + s * kSlabBytes;
-#pragma unroll
-            for (int rr = 0; rr < kPasses; ++rr) {
-              const int row = (ptid >> 3) + kRowsPerPass * rr;
-              if (row >= kTE) continue;
-              const __nv_bfloat16* p = src[rr] != nullptr ? src[rr] + s * 64 + chunk * 8 : kv_win;
-              cp_async_16(dst + row * 128 + ((chunk ^ (row & 7)) * 16), p,
-                          src[rr] != nullptr ? 16u : 0u);
-            }
-            cp_async_arrive_noinc(&bar->slab_full[s]);
-          }
-        } else {
-          // FP8 entries are dequantised to bf16 (code * scale) on the way in;
-          // RoPE dims and window rows are bf16 already.  Loads of slab s+1 are
-          // in flight while slab s is converted and stored.
-          const int body = kC - ds.rope;
-          const uint8_t* code[kPasses];
-          const __nv_bfloat16* bfp[kPasses];   // rope dims (entries) or the whole row (window)
-          float scl[kPasses];
-#pragma unroll
-          for (int rr = 0; rr < kPasses; ++rr) {
-            const int slot = tile * kTE + (ptid >> 3) + kRowsPerPass * rr;
-            code[rr] = nullptr;
-            bfp[rr] = nullptr;
-            scl[rr] = 0.f;
-            if (slot < nsel) {
-              const int64_t e = b * E + (idx != nullptr ? (int64_t)list[slot] : (int64_t)slot);
-              code[rr] = ds.cv.entry_fp8 + e * body;
-              bfp[rr] = ds.cv.entry_rope + e * ds.rope;
-              scl[rr] = ds.cv.entry_scale[e];
-            } else if (slot < N) {
-              const int64_t u = w0 + (slot - nsel);
-              bfp[rr] = ds.cv.window + (b * window + u % window) * kC;
-            }
-          }
-          uint4 cur[kPasses], nxt[kPasses];
-          auto fetch = [&](int s, uint4(&buf)[kPasses]) {
-            const int d0 = s * 64 + chunk * 8;
-#pragma unroll
-            for (int rr = 0; rr < kPasses; ++rr) {
-              uint4 v = make_uint4(0, 0, 0, 0);
-              if (code[rr] != nullptr) {
-                if (d0 < body) {
-                  const uint2 c8 = *reinterpret_cast<const uint2*>(code[rr] + d0);
-                  v.x = c8.x;
-                  v.y = c8.y;
-                } else {
-                  v = *reinterpret_cast<const uint4*>(bfp[rr] + (d0 - body));
-                }
-              } else if (bfp[rr] != nullptr) {
-                v = *reinterpret_cast<const uint4*>(bfp[rr] + d0);
-              }
-              buf[rr] = v;
-            }
-          };
-          fetch(0, cur);
-#pragma unroll
-          for (int s = 0; s < kSlabs; ++s) {
-            if (s + 1 < kSlabs) fetch(s + 1, nxt);
-            if (ok && g >= 1 && !mbar_wait(&bar->slab_empty[s], (uint32_t)((g - 1) & 1), err))
-              ok = false;
-            if (ok) {
-              const int d0 = s * 64 + chunk * 8;
-              uint8_t* dst = sKV + s * kSlabBytes;
-#pragma unroll
-              for (int rr = 0; rr < kPasses; ++rr) {
-                const int row = (ptid >> 3) + kRowsPerPass * rr;
-                if (row >= kTE) continue;
-                uint4 v = cur[rr];
-                if (code[rr] != nullptr && d0 < body) {
-                  const uint32_t w2[2] = {cur[rr].x, cur[rr].y};
-                  uint32_t o[4];
-#pragma unroll
-                  for (int q = 0; q < 4; ++q) {
-                    const uint32_t pair = (w2[q >> 1] >> ((q & 1) * 16)) & 0xffffu;
-                    o[q] = pack_bf16x2(e4m3_value((uint8_t)(pair & 0xff)) * scl[rr],
-                                       e4m3_value((uint8_t)(pair >> 8)) * scl[rr]);
-                  }
-                  v = make_uint4(o[0], o[1], o[2], o[3]);
-                }
-                *reinterpret_cast<uint4*>(dst + row * 128 + ((chunk ^ (row & 7)) * 16)) = v;
-              }
-              fence_proxy_async();
-              mbar_arrive(&bar->slab_full[s]);
-            }
-#pragma unroll
-            for (int rr = 0; rr < kPasses; ++rr) cur[rr] = nxt[rr];
-          }
+          cp_async_arrive_noinc(&bar->slab_full[s]);
         }
       }
     }
@@ -397,10 +251,6 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(
       if (!mbar_wait(&bar->meta_full[kq & 1], (uint32_t)((kq >> 1) & 1), err)) break;
       const int T = meta[kq & 1].ntiles;
       if (!mbar_wait(&bar->q_full, (uint32_t)(kq & 1), err)) break;
-      if (T == 0) {  // an empty split: nothing to multiply, Q is free again
-        if (lane == 0) mma_commit(&bar->q_empty);
-        __syncwarp();
-      }
       for (int tt = 0; tt < T; ++tt, ++g) {
         const int sb = g & 1;
         if (g >= 2 && !mbar_wait(&bar->s_empty[sb], (uint32_t)(((g >> 1) - 1) & 1), err)) {
@@ -475,7 +325,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(
         if (!mbar_wait(&bar->s_full[sb], (uint32_t)((g >> 1) & 1), err)) { ok = false; break; }
         tc_fence_after();
         const uint32_t s_addr = lane_base + kColS + sb * kNH + hh * 32;
-        const bool valid = (mt.tile_lo + tt) * kTE + row < mt.nrows;
+        const bool valid = tt * kTE + row < mt.nrows;
         float v[32];
         {
           uint32_t r[32];
@@ -552,42 +402,18 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(
       }
       if (!ok) break;
       // ---- epilogue: o = O^T / (sum_j p_j + 2^(sink - m)) ----------------------
-      if (mt.ntiles > 0 && !mbar_wait(&bar->p_empty, (uint32_t)((g - 1) & 1), err)) break;
+      if (!mbar_wait(&bar->p_empty, (uint32_t)((g - 1) & 1), err)) break;
       tc_fence_after();
       float* rsum = red + (2 * 2 * 4 + hh * 4) * 32;
       rsum[quad * 32 + lane] = transpose_reduce<false>(psum);
       if (!group_sync(&bar->grp_soft[hh], gphase, err)) break;
       const int h_lane = hh * 32 + lane;
       const float tot = rsum[lane] + rsum[32 + lane] + rsum[64 + lane] + rsum[96 + lane];
-      if (kDec && ds.nsplit > 1) {
-        // partial result of this slice: unnormalised O, running max, sum
-        const int64_t pbase = (mt.b * ds.nsplit + mt.split) * kNH;
-        if (quad == 0) {
-          ds.part_ms[(pbase + h_lane) * 2 + 0] = mt.ntiles > 0 ? m_run : kNegInf;
-          ds.part_ms[(pbase + h_lane) * 2 + 1] = mt.ntiles > 0 ? tot : 0.f;
-        }
-        if (mt.ntiles > 0) {
-          for (int c = 0; c < 4; ++c) {
-            uint32_t o[32];
-            tmem_ld32(lane_base + kColO + c * kNH + hh * 32, o);
-            tmem_ld_wait();
-            const int d = c * 128 + row;
-#pragma unroll
-            for (int i = 0; i < 32; ++i)
-              ds.part_o[(pbase + hh * 32 + i) * kC + d] = __uint_as_float(o[i]);
-          }
-        }
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&bar->o_empty);
-        if (!group_sync(&bar->grp_soft[hh], gphase, err)) break;
-        continue;
-      }
       const float mref = m_run == kNegInf ? 0.f : m_run;
       const float z = sink != nullptr ? sink[h_lane] * kLog2e : kNegInf;
       const float den = tot + (z == kNegInf ? 0.f : ex2(z - mref));
       const float inv = 1.f / den;
-      __nv_bfloat16* ob = out + ((mt.b * n + (kDec ? 0 : mt.t)) * kNH) * kC;
+      __nv_bfloat16* ob = out + ((mt.b * n + mt.t) * kNH) * kC;
       for (int c = 0; c < 4; ++c) {
         uint32_t o[32];
         tmem_ld32(lane_base + kColO + c * kNH + hh * 32, o);
@@ -642,53 +468,14 @@ cudaError_t launch_attn_tc(const void* q, const void* kv_comp, const int32_t* id
   if (!make_tmap_bf16_3d(&tq, q, kC, (uint64_t)n * kNH, batch, kC * 2ull,
                          (uint64_t)n * kNH * kC * 2, 64, kNH))
     return cudaErrorInvalidValue;
-  auto kern = attn_tc_kernel<false>;
-  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM);
+  cudaError_t e = cudaFuncSetAttribute(attn_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       SMEM);
   if (e != cudaSuccess) return e;
   const int64_t total = batch * n;
   const int64_t grid = std::min<int64_t>(total, sm_count());
-  DecodeSide ds = {};
-  ds.nsplit = 1;
-  kern<<<(unsigned)grid, kThreads, SMEM, s>>>(
+  attn_tc_kernel<<<(unsigned)grid, kThreads, SMEM, s>>>(
       tq, (const __nv_bfloat16*)kv_comp, idx, k, (const __nv_bfloat16*)kv_win, window, sink,
-      scale, n, m, n / m, total, (__nv_bfloat16*)out, err, ds);
-  return cudaGetLastError();
-}
-
-bool decode_attn_tc_supported(const csa_cache_desc& d) {
-  return d.nh == kNH && d.c == kC && (d.is_hca || d.k <= kMaxSel) && d.rope_dims % 8 == 0;
-}
-
-int decode_attn_splits(const csa_cache_desc& d) {
-  const int64_t slots = (d.is_hca ? d.capacity : (int64_t)d.k) + d.window;
-  const int64_t tiles = (slots + kTE - 1) / kTE;
-  const int64_t per_seq = std::max<int64_t>(1, sm_count() / std::max<int64_t>(1, d.batch));
-  return (int)std::max<int64_t>(1, std::min<int64_t>(tiles, per_seq));
-}
-
-cudaError_t launch_decode_attn_tc(const csa_cache_desc& d, const CacheView& cv,
-                                  const int64_t* pos, const void* q, const int32_t* sel,
-                                  const float* sink, float scale, int nsplit, void* out,
-                                  float* part_o, float* part_ms, unsigned int* err,
-                                  cudaStream_t s) {
-  CUtensorMap tq;
-  if (!make_tmap_bf16_3d(&tq, q, kC, kNH, d.batch, kC * 2ull, (uint64_t)kNH * kC * 2, 64, kNH))
-    return cudaErrorInvalidValue;
-  auto kern = attn_tc_kernel<true>;
-  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM);
-  if (e != cudaSuccess) return e;
-  const int64_t total = d.batch * nsplit;
-  const int64_t grid = std::min<int64_t>(total, sm_count());
-  DecodeSide ds;
-  ds.cv = cv;
-  ds.pos = pos;
-  ds.nsplit = nsplit;
-  ds.rope = d.rope_dims;
-  ds.part_o = part_o;
-  ds.part_ms = part_ms;
-  kern<<<(unsigned)grid, kThreads, SMEM, s>>>(tq, nullptr, d.is_hca ? nullptr : sel, d.k,
-                                              nullptr, d.window, sink, scale, 1, d.m,
-                                              d.capacity, total, (__nv_bfloat16*)out, err, ds);
+      scale, n, m, n / m, total, (__nv_bfloat16*)out, err);
   return cudaGetLastError();
 }
 

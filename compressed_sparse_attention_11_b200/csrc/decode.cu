@@ -28,8 +28,7 @@ namespace csa {
 
 constexpr int kSelThreads = 512;          // CUDA-core chunk top-k / merge blocks
 constexpr int kDecSelThreads = 1024;      // one selection block per sequence
-constexpr int kDecSelCap = 8192;          // candidates kept above the sampled threshold
-constexpr int kDecSelSample = 4096;       // sample size of the threshold estimate
+
 
 static inline size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
 
@@ -210,9 +209,14 @@ __device__ float emit_dim(const __nv_bfloat16* st, int64_t b, int64_t i, int m, 
 
 __global__ void __launch_bounds__(256) append_emit_kernel(csa_cache_desc d, CacheView cv,
                                                           const int64_t* __restrict__ pos,
-                                                          csa_rows rows, csa_decode_params p) {
+                                                          csa_rows rows, csa_decode_params p,
+                                                          uint32_t* __restrict__ range) {
   extern __shared__ float sx[];  // [c + c_i] + 32
   const int64_t b = blockIdx.x;
+  if (range != nullptr && threadIdx.x == 0) {  // the indexer's score range starts empty
+    range[b * 2 + 0] = 0u;
+    range[b * 2 + 1] = 0xffffffffu;
+  }
   const int64_t t = pos[b];
   if (t < 0) return;  // no token for this sequence
   put_rows(d, cv, rows, b, 1, 0, t, true, true);
@@ -335,23 +339,205 @@ __global__ void __launch_bounds__(kSelThreads) topk_merge_kernel(
 }
 
 // Step 3' (CSA, tensor-core indexer): top-k over one sequence's score array.
+// The indexer recorded the sequence's score range; scores are bucketed
+// linearly over it (4096 buckets), one histogram pass finds the bucket T of
+// the k-th largest score, one pass keeps the scores in buckets >= T (all of
+// buckets > T are chosen), and the bucket-T scores are ranked among
+// themselves (ties to the smaller index).  Degenerate ranges or crowded
+// buckets fall back to the radix select.
+constexpr int kLinBins = 4096;
+constexpr int kLinCap = 4096;        // scores kept in buckets >= T
+constexpr int kLinBucketMax = 1024;  // bucket-T scores ranked directly
+
+struct LinSelShared {
+  uint32_t bins[kLinBins];
+  uint32_t ckey[kLinCap];
+  int32_t cpos[kLinCap];
+  uint32_t bkey[kLinBucketMax];
+  int32_t bslot[kLinBucketMax];
+  uint8_t take[kLinCap];
+  uint32_t wsum[kDecSelThreads / 32];
+  uint32_t T, G, C;
+};
+
+__device__ __forceinline__ int lin_bucket(float s, float lo, float inv) {
+  const float x = (s - lo) * inv;
+  return x <= 0.f ? 0 : (x >= (float)(kLinBins - 1) ? kLinBins - 1 : (int)x);
+}
+
+// Block-wide exclusive prefix of `v` (in thread order); `total` gets the sum.
+__device__ __forceinline__ uint32_t block_exclusive(uint32_t v, uint32_t* wsum, uint32_t& total) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, W = blockDim.x >> 5;
+  uint32_t inc = v;
+#pragma unroll
+  for (int off = 1; off < 32; off <<= 1) {
+    const uint32_t x = __shfl_up_sync(0xffffffffu, inc, off);
+    if (lane >= off) inc += x;
+  }
+  __syncthreads();
+  if (lane == 31) wsum[warp] = inc;
+  __syncthreads();
+  uint32_t before = inc - v;
+  total = 0;
+  for (int w = 0; w < W; ++w) {
+    if (w < warp) before += wsum[w];
+    total += wsum[w];
+  }
+  return before;
+}
+
 __global__ void __launch_bounds__(kDecSelThreads) decode_select_kernel(
     csa_cache_desc d, const int64_t* __restrict__ pos, const float* __restrict__ scores,
-    int32_t* __restrict__ sel) {
+    const uint32_t* __restrict__ range, int32_t* __restrict__ sel) {
   extern __shared__ __align__(16) unsigned char smem_raw[];
-  SelectShared<kDecSelThreads>& sh = *reinterpret_cast<SelectShared<kDecSelThreads>*>(smem_raw);
-  int32_t* cand = reinterpret_cast<int32_t*>(smem_raw + sizeof(SelectShared<kDecSelThreads>));
-  uint32_t* sample = reinterpret_cast<uint32_t*>(cand + kDecSelCap);
+  LinSelShared& ls = *reinterpret_cast<LinSelShared*>(smem_raw);
+  constexpr int NT = kDecSelThreads;
+  const int tid = threadIdx.x, lane = tid & 31;
   const int64_t b = blockIdx.x;
   const int64_t t = pos[b];
   const int64_t V = t < 0 ? 0 : min((t + 1) / d.m, d.capacity);
-  int32_t* out = sel + b * d.k;
-  if (V <= d.k) {
-    for (int j = threadIdx.x; j < d.k; j += blockDim.x) out[j] = j < V ? j : -1;
+  const int k = d.k;
+  int32_t* out = sel + b * k;
+  if (V <= k) {
+    for (int j = tid; j < k; j += NT) out[j] = j < V ? j : -1;
     return;
   }
-  block_select_topk_sampled<kDecSelThreads>(ScoresIn{scores + b * d.capacity}, V, d.k, out, sh,
-                                            cand, kDecSelCap, sample, kDecSelSample);
+  const float* row = scores + b * d.capacity;
+  const float hi_s = key_to_float(range[b * 2 + 0]), lo_s = key_to_float(range[b * 2 + 1]);
+  bool fallback = !(hi_s > lo_s) || !isfinite(hi_s - lo_s);
+  const float inv = fallback ? 0.f : (float)kLinBins / (hi_s - lo_s);
+  if (!fallback) {
+    // 1. histogram
+    for (int i = tid; i < kLinBins; i += NT) ls.bins[i] = 0;
+    if (tid == 0) { ls.T = 0; ls.G = 0; ls.C = 0xffffffffu; }
+    __syncthreads();
+    constexpr int kBatch = 8;  // loads in flight per thread
+    for (int64_t i0 = tid; i0 < V; i0 += (int64_t)NT * kBatch) {
+      float v[kBatch];
+#pragma unroll
+      for (int u = 0; u < kBatch; ++u) {
+        const int64_t i = i0 + (int64_t)u * NT;
+        v[u] = i < V ? row[i] : 0.f;
+      }
+#pragma unroll
+      for (int u = 0; u < kBatch; ++u)
+        if (i0 + (int64_t)u * NT < V) atomicAdd(&ls.bins[lin_bucket(v[u], lo_s, inv)], 1u);
+    }
+    __syncthreads();
+    // 2. the bucket where the count from the top reaches k (thread tid owns
+    //    buckets 4095-4tid .. 4092-4tid, descending)
+    constexpr int BPT = kLinBins / NT;
+    uint32_t mine[BPT], loc = 0;
+#pragma unroll
+    for (int j = 0; j < BPT; ++j) {
+      mine[j] = ls.bins[kLinBins - 1 - (tid * BPT + j)];
+      loc += mine[j];
+    }
+    uint32_t tot;
+    uint32_t acc = block_exclusive(loc, ls.wsum, tot);
+#pragma unroll
+    for (int j = 0; j < BPT; ++j) {
+      if (acc < (uint32_t)k && acc + mine[j] >= (uint32_t)k) {
+        ls.T = kLinBins - 1 - (tid * BPT + j);
+        ls.G = acc;
+        ls.C = acc + mine[j];
+      }
+      acc += mine[j];
+    }
+    __syncthreads();
+    fallback = ls.C > (uint32_t)kLinCap || ls.C - ls.G > (uint32_t)kLinBucketMax;
+  }
+  if (fallback) {
+    __syncthreads();
+    auto& sh = *reinterpret_cast<SelectShared<NT>*>(smem_raw);
+    block_select_topk<NT>(ScoresIn{row}, V, k, out, nullptr, sh);
+    return;
+  }
+  const int T = (int)ls.T;
+  const uint32_t G = ls.G, C = ls.C, need = (uint32_t)k - G;
+  // 3. keep the scores in buckets >= T in position order (per warp segments)
+  {
+    constexpr int W = NT / 32;
+    const int warp = tid >> 5;
+    const int64_t seg = ((V + W - 1) / W + 31) / 32 * 32;
+    const int64_t lo = (int64_t)warp * seg, hi = min(V, lo + seg);
+    uint32_t c = 0;
+    constexpr int kBatch = 8;  // loads in flight per lane
+    for (int64_t base = lo; base < hi; base += 32 * kBatch) {
+      float v[kBatch];
+#pragma unroll
+      for (int u = 0; u < kBatch; ++u) {
+        const int64_t i = base + u * 32 + lane;
+        v[u] = i < hi ? row[i] : 0.f;
+      }
+#pragma unroll
+      for (int u = 0; u < kBatch; ++u) {
+        const int64_t i = base + u * 32 + lane;
+        c += __popc(__ballot_sync(0xffffffffu, i < hi && lin_bucket(v[u], lo_s, inv) >= T));
+      }
+    }
+    uint32_t all;
+    uint32_t run = block_exclusive(lane == 0 ? c : 0u, ls.wsum, all);
+    run = __shfl_sync(0xffffffffu, run, 0);
+    const uint32_t lt = (1u << lane) - 1u;
+    for (int64_t base = lo; base < hi; base += 32 * kBatch) {
+      float v[kBatch];
+#pragma unroll
+      for (int u = 0; u < kBatch; ++u) {
+        const int64_t i = base + u * 32 + lane;
+        v[u] = i < hi ? row[i] : 0.f;
+      }
+#pragma unroll
+      for (int u = 0; u < kBatch; ++u) {
+        const int64_t i = base + u * 32 + lane;
+        const int bk = i < hi ? lin_bucket(v[u], lo_s, inv) : -1;
+        const bool keep = i < hi && bk >= T;
+        const uint32_t msk = __ballot_sync(0xffffffffu, keep);
+        if (keep) {
+          const uint32_t p = run + __popc(msk & lt);
+          if (p < (uint32_t)kLinCap) {
+            ls.ckey[p] = order_key(v[u]);
+            ls.cpos[p] = (int32_t)i;
+            ls.take[p] = bk > T ? 1 : 0;
+          }
+        }
+        run += __popc(msk);
+      }
+    }
+    __syncthreads();
+  }
+  // 4. rank the bucket-T scores among themselves
+  {
+    const int per = (int)((C + NT - 1) / NT);
+    const int lo = min((int)C, tid * per), hi = min((int)C, lo + per);
+    uint32_t nb = 0;
+    for (int i = lo; i < hi; ++i) nb += ls.take[i] ? 0u : 1u;
+    uint32_t all;
+    uint32_t o = block_exclusive(nb, ls.wsum, all);
+    for (int i = lo; i < hi; ++i)
+      if (!ls.take[i]) {
+        ls.bkey[o] = ls.ckey[i];
+        ls.bslot[o] = i;
+        ++o;
+      }
+    __syncthreads();
+    for (int e = tid; e < (int)all; e += NT) {
+      const uint32_t ke = ls.bkey[e];
+      uint32_t r = 0;
+      for (int f = 0; f < (int)all; ++f) {
+        const uint32_t kf = ls.bkey[f];
+        r += (kf > ke || (kf == ke && f < e)) ? 1u : 0u;
+      }
+      if (r < need) ls.take[ls.bslot[e]] = 1;
+    }
+    __syncthreads();
+    // 5. the chosen positions, ascending
+    uint32_t nt = 0;
+    for (int i = lo; i < hi; ++i) nt += ls.take[i];
+    uint32_t o2 = block_exclusive(nt, ls.wsum, all);
+    for (int i = lo; i < hi; ++i)
+      if (ls.take[i] && o2 < (uint32_t)k) out[o2++] = ls.cpos[i];
+  }
 }
 
 // ---------------------------------------------------------------------------
@@ -514,7 +700,7 @@ __global__ void __launch_bounds__(256) attn_combine_kernel(
 struct DecodeWs {
   int nchunks, nsplit;
   bool tc_index, tc_attn;
-  size_t cand_score, cand_idx, scores, sel, part_o, part_ms, total;
+  size_t cand_score, cand_idx, scores, range, sel, part_o, part_ms, total;
 };
 
 static DecodeWs decode_ws_layout(const csa_cache_desc& d) {
@@ -530,6 +716,7 @@ static DecodeWs decode_ws_layout(const csa_cache_desc& d) {
   w.cand_score = off; off = align256(off + B * w.nchunks * d.k * 4);
   w.cand_idx = off;   off = align256(off + B * w.nchunks * d.k * 4);
   w.scores = off;     off = align256(off + (w.tc_index ? B * (size_t)d.capacity * 4 : 0));
+  w.range = off;      off = align256(off + (w.tc_index ? B * 2 * 4 : 0));
   w.sel = off;        off = align256(off + B * (d.is_hca ? 0 : d.k) * 4);
   w.part_o = off;     off = align256(off + B * w.nsplit * d.nh * (size_t)d.c * 4);
   w.part_ms = off;    off = align256(off + B * w.nsplit * d.nh * 2 * 4);
@@ -551,21 +738,22 @@ cudaError_t launch_decode_step(const csa_cache_desc& d, const CacheView& cv, con
   float* part_o = reinterpret_cast<float*>(wb + w.part_o);
   float* part_ms = reinterpret_cast<float*>(wb + w.part_ms);
 
+  uint32_t* range = w.tc_index ? reinterpret_cast<uint32_t*>(wb + w.range) : nullptr;
   const size_t emit_smem = sizeof(float) * (d.c + (d.is_hca ? 0 : d.c_i) + 32);
-  append_emit_kernel<<<(unsigned)d.batch, 256, emit_smem, s>>>(d, cv, pos, rows, p);
+  append_emit_kernel<<<(unsigned)d.batch, 256, emit_smem, s>>>(d, cv, pos, rows, p, range);
   cudaError_t err = cudaGetLastError();
   if (err != cudaSuccess) return err;
   if (!d.is_hca && w.tc_index) {
     float* scores = reinterpret_cast<float*>(wb + w.scores);
     unsigned int* flag = device_timeout_flag();
     if (flag == nullptr) return cudaErrorUnknown;
-    err = launch_decode_index_tc(d, cv, pos, q_i, w_i, scores, flag, s);
+    err = launch_decode_index_tc(d, cv, pos, q_i, w_i, scores, range, flag, s);
     if (err != cudaSuccess) return err;
-    const size_t smem = sizeof(SelectShared<kDecSelThreads>) + (size_t)kDecSelCap * 4 +
-                        (size_t)kDecSelSample * 4;
+    const size_t smem = std::max(sizeof(LinSelShared), sizeof(SelectShared<kDecSelThreads>));
     cudaFuncSetAttribute(decode_select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                          (int)smem);
-    decode_select_kernel<<<(unsigned)d.batch, kDecSelThreads, smem, s>>>(d, pos, scores, sel);
+    decode_select_kernel<<<(unsigned)d.batch, kDecSelThreads, smem, s>>>(d, pos, scores, range,
+                                                                          sel);
     if ((err = cudaGetLastError()) != cudaSuccess) return err;
   } else if (!d.is_hca) {
     const size_t smem = sizeof(SelectShared<kSelThreads>) + (size_t)kDecChunk * 8 +
@@ -584,12 +772,8 @@ cudaError_t launch_decode_step(const csa_cache_desc& d, const CacheView& cv, con
   if (w.tc_attn) {
     unsigned int* flag = device_timeout_flag();
     if (flag == nullptr) return cudaErrorUnknown;
-    err = launch_decode_attn_tc(d, cv, pos, q, sel, p.sink, p.scale, w.nsplit, out, part_o,
-                                part_ms, flag, s);
-    if (err != cudaSuccess || w.nsplit == 1) return err;
-    attn_combine_kernel<<<dim3((unsigned)d.batch, hgroups), 256, 0, s>>>(
-        d, p.sink, w.nsplit, part_o, part_ms, (__nv_bfloat16*)out);
-    return cudaGetLastError();
+    return launch_decode_attn_tc(d, cv, pos, q, sel, p.sink, p.scale, w.nsplit, out, part_o,
+                                 part_ms, flag, s);
   }
   const size_t asmem = sizeof(float) * ((size_t)kDecTE * (d.c + 1) + (size_t)kDecHG * d.c +
                                         kDecHG * kDecTE) + sizeof(int64_t) * kDecTE;

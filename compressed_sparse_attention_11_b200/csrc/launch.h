@@ -34,11 +34,15 @@ cudaError_t launch_attn_tc(const void* q, const void* kv_comp, const int32_t* id
 // tcgen05 decode indexer over FP8 keys (c_i = 128, nh_i in {16, 32, 64, 128}).
 struct CacheView;
 bool decode_index_tc_supported(const csa_cache_desc& d);
+// scores [batch][capacity] fp32; range [batch][2] receives the largest and
+// smallest order key of each sequence's scores (0 / ~0 on entry).
 cudaError_t launch_decode_index_tc(const csa_cache_desc& d, const CacheView& cv,
                                    const int64_t* pos, const void* q_i, const float* w_i,
-                                   float* scores, unsigned int* err, cudaStream_t s);
+                                   float* scores, unsigned int* range, unsigned int* err,
+                                   cudaStream_t s);
 
-// tcgen05 decode attention (64 heads x 512, FP8/bf16 cache), split-K.
+// tcgen05 decode attention (64 heads x 512, FP8/bf16 cache): one 128-entry
+// tile per CTA (ntile = decode_attn_splits), merged by a combine kernel.
 bool decode_attn_tc_supported(const csa_cache_desc& d);
 int decode_attn_splits(const csa_cache_desc& d);
 cudaError_t launch_decode_attn_tc(const csa_cache_desc& d, const CacheView& cv,

@@ -5,15 +5,18 @@
 // The chosen positions are emitted in ascending position order, which is the
 // order the selection is compacted in, so no sort is needed.
 //
-// Two front ends:
+// Three front ends:
 //   block_select_topk          radix select over all V keys (4 histogram
 //                              passes + 2 compaction passes);
 //   block_select_topk_sampled  estimates a threshold from a strided sample,
 //                              keeps the (few) keys at or above it in order,
 //                              and runs the exact radix select on those only
-//                              -- two passes over V instead of six.  It falls
-//                              back to the full select when the estimate
-//                              keeps fewer than k or more than `cap` keys.
+//                              -- two passes over V instead of six;
+//   block_select_topk_ranked   the same, but the sample and the kept keys are
+//                              ranked by direct comparison counts, which costs
+//                              a few block barriers instead of dozens.
+// The sampled front ends fall back to the full select when the estimate
+// keeps fewer than k or too many keys.
 #pragma once
 
 #include "common.cuh"
@@ -233,6 +236,110 @@ __device__ void block_select_topk_sampled(const Src& src, int64_t V, int k,
   // candidates are in ascending position order: emitting the chosen slots in
   // order and mapping each slot to its position keeps the output ascending
   block_select_topk<NT>(Gathered<Src>{src, cand}, total, k, out, cand, sh);
+}
+
+// Rank of element i among n keys (larger first, ties to the smaller index).
+__device__ __forceinline__ uint32_t rank_in(const uint32_t* __restrict__ keys, int n, int i) {
+  const uint32_t ki = keys[i];
+  uint32_t r = 0;
+  for (int j = 0; j < n; ++j) {
+    const uint32_t kj = keys[j];
+    r += (kj > ki || (kj == ki && j < i)) ? 1u : 0u;
+  }
+  return r;
+}
+
+// Same result as block_select_topk (positions, no map), for k <= V.  A strided
+// sample of S keys is ranked exactly to pick a threshold somewhat below the
+// k-th largest; one pass keeps the keys at or above it (in position order);
+// those are ranked exactly when there are at most `rank_max`, radix-selected
+// otherwise.  Scratch: skey / spos hold `cap` entries (shared memory).
+template <int NT, class Src>
+__device__ void block_select_topk_ranked(const Src& src, int64_t V, int k,
+                                         int32_t* __restrict__ out, SelectShared<NT>& sh,
+                                         uint32_t* __restrict__ skey, int32_t* __restrict__ spos,
+                                         int cap, int rank_max) {
+  constexpr int W = NT / 32;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const uint32_t lt = (1u << lane) - 1u;
+  uint32_t C;
+  if (V <= (int64_t)rank_max) {  // small: every key is a candidate
+    for (int i = tid; i < V; i += NT) {
+      skey[i] = src.key(i);
+      spos[i] = i;
+    }
+    C = (uint32_t)V;
+    __syncthreads();
+  } else {
+    // 1. threshold: the r-th largest of a strided sample
+    const int S = (int)min(V, (int64_t)(V > 65536 ? 2048 : 1024));
+    const int r = (int)min((int64_t)S, (3 * (int64_t)S * k) / (2 * V) + 12);
+    for (int i = tid; i < S; i += NT) skey[i] = src.key((V * (int64_t)i) / S);
+    if (tid == 0) sh.digit = 0;
+    __syncthreads();
+    for (int i = tid; i < S; i += NT)
+      if (rank_in(skey, S, i) == (uint32_t)(r - 1)) sh.digit = skey[i];
+    __syncthreads();
+    const uint32_t T0 = sh.digit;
+    // 2. count and keep the keys >= T0, per warp over a contiguous segment
+    const int64_t seg = ((V + W - 1) / W + 31) / 32 * 32;
+    const int64_t lo = (int64_t)warp * seg, hi = min(V, lo + seg);
+    uint32_t c = 0;
+    for (int64_t base = lo; base < hi; base += 32) {
+      const int64_t i = base + lane;
+      c += __popc(__ballot_sync(0xffffffffu, i < hi && src.key(i) >= T0));
+    }
+    if (lane == 0) sh.warp_a[warp] = c;
+    __syncthreads();
+    uint32_t before = 0;
+    C = 0;
+    for (int w = 0; w < W; ++w) {
+      if (w < warp) before += sh.warp_a[w];
+      C += sh.warp_a[w];
+    }
+    __syncthreads();
+    if (C < (uint32_t)k || C > (uint32_t)cap) {  // the estimate missed: exact path
+      block_select_topk<NT>(src, V, k, out, nullptr, sh);
+      return;
+    }
+    uint32_t run = before;
+    for (int64_t base = lo; base < hi; base += 32) {
+      const int64_t i = base + lane;
+      const uint32_t key = i < hi ? src.key(i) : 0u;
+      const bool keep = i < hi && key >= T0;
+      const uint32_t msk = __ballot_sync(0xffffffffu, keep);
+      if (keep) {
+        const uint32_t p = run + __popc(msk & lt);
+        skey[p] = key;
+        spos[p] = (int32_t)i;
+      }
+      run += __popc(msk);
+    }
+    __syncthreads();
+    if (C > (uint32_t)rank_max) {
+      block_select_topk<NT>(KeysInSmem{skey}, C, k, out, spos, sh);
+      return;
+    }
+  }
+  // 3. exact ranks among the candidates; contiguous candidates per thread
+  //    keep the output in ascending position order
+  const int per = (int)((C + NT - 1) / NT);
+  const int lo = min((int)C, tid * per), hi = min((int)C, lo + per);
+  uint32_t mine = 0;
+  for (int i = lo; i < hi; ++i) mine += rank_in(skey, C, i) < (uint32_t)k ? 1u : 0u;
+  uint32_t inc = mine;
+#pragma unroll
+  for (int off = 1; off < 32; off <<= 1) {
+    const uint32_t v = __shfl_up_sync(0xffffffffu, inc, off);
+    if (lane >= off) inc += v;
+  }
+  if (lane == 31) sh.warp_b[warp] = inc;
+  __syncthreads();
+  uint32_t o = inc - mine;
+  for (int w = 0; w < warp; ++w) o += sh.warp_b[w];
+  for (int i = lo; i < hi; ++i)
+    if (rank_in(skey, C, i) < (uint32_t)k && o < (uint32_t)k) out[o++] = spos[i];
+  __syncthreads();
 }
 
 }  // namespace csa
