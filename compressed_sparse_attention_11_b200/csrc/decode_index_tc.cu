@@ -201,11 +201,24 @@ __global__ void __launch_bounds__(kThreads, 1) decode_index_tc_kernel(
     const int row = quad * 32 + lane;
     const uint32_t lane_addr = tmem + ((uint32_t)(quad * 32) << 16);
     uint32_t kmax = 0u, kmin = 0xffffffffu;  // order keys of this thread's scores
-    for (int j = grp; j < ntiles; j += 2) {
+    // the key scales do not depend on the MMA: all of this thread's loads go
+    // out at once, so one DRAM latency is paid instead of one per tile
+    constexpr int kMine = kChunk / kKeys / 2;
+    float kscale[kMine];
+#pragma unroll
+    for (int i = 0; i < kMine; ++i) {
+      const int64_t s = c0 + (int64_t)(grp + 2 * i) * kKeys + row;
+      kscale[i] = s < V ? __ldcs(key_scale + b * cap + s) : 0.f;
+    }
+#pragma unroll 1
+    for (int i = 0; i < kMine; ++i) {
+      const int j = grp + 2 * i;
+      if (j >= ntiles) break;
       const int p = j % C::DBUFS, v = j / C::DBUFS;
       const int64_t s = c0 + (int64_t)j * kKeys + row;
-      // the key scale is independent of the MMA: load it before waiting
-      const float kscale = s < V ? key_scale[b * cap + s] : 0.f;
+      const float ks = kscale[0];  // shift the queue (registers, not a local array)
+#pragma unroll
+      for (int q = 0; q + 1 < kMine; ++q) kscale[q] = kscale[q + 1];
       if (!mbar_wait(&bar->d_full[p], (uint32_t)(v & 1), err)) break;
       tc_fence_after();
       float acc = 0.f;
@@ -224,7 +237,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_index_tc_kernel(
       __syncwarp();
       if (lane == 0) mbar_arrive(&bar->d_empty[p]);
       if (s < V) {
-        const float sc = acc * kscale;
+        const float sc = acc * ks;
         scores[b * cap + s] = sc;
         const uint32_t ky = order_key(sc);
         kmax = max(kmax, ky);
