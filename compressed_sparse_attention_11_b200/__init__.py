@@ -60,7 +60,8 @@ class Rows(ctypes.Structure):
 
 class DecodeParams(ctypes.Structure):
     _fields_ = [("ba", ctypes.c_void_p), ("bb", ctypes.c_void_p), ("iba", ctypes.c_void_p),
-                ("ibb", ctypes.c_void_p), ("sink", ctypes.c_void_p), ("scale", ctypes.c_float)]
+                ("ibb", ctypes.c_void_p), ("sink", ctypes.c_void_p), ("scale", ctypes.c_float),
+                ("sel_out", ctypes.c_void_p)]
 
 
 _lib = None
@@ -268,16 +269,21 @@ class CsaCache:
                                           count, ctypes.byref(r), _stream(self.buffer)))
 
     def decode_step(self, pos, rows: dict, biases: dict, sink, scale: float, q, q_i=None,
-                    w_i=None, out: Optional[torch.Tensor] = None):
+                    w_i=None, out: Optional[torch.Tensor] = None,
+                    sel_out: Optional[torch.Tensor] = None):
         """One token per sequence at positions ``pos`` (int64 [B] on device).
 
         ``rows``: per-stream [B, dim] bf16 tensors; ``biases``: ba, bb, iba, ibb
-        fp32; returns out [B, nh, c] bf16."""
+        fp32; returns out [B, nh, c] bf16.  ``sel_out`` (CSA, optional, int32
+        [B, k] on device) receives the selected entry indices."""
         if out is None:
             out = torch.empty_like(q)
         r = self._rows({k: v for k, v in rows.items()})
+        if sel_out is not None and (sel_out.dtype != torch.int32 or not sel_out.is_contiguous()
+                                    or sel_out.numel() != self.desc.batch * self.desc.k):
+            raise ValueError("sel_out must be a contiguous int32 [batch, k] tensor")
         p = DecodeParams(_ptr(biases.get("ba")), _ptr(biases.get("bb")), _ptr(biases.get("iba")),
-                         _ptr(biases.get("ibb")), _ptr(sink), float(scale))
+                         _ptr(biases.get("ibb")), _ptr(sink), float(scale), _ptr(sel_out))
         if pos.dtype != torch.int64:
             raise ValueError("pos must be int64")
         _check(lib().csa_decode_step(ctypes.byref(self.desc), _ptr(self.buffer), _ptr(pos),

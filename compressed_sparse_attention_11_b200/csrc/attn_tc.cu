@@ -440,17 +440,6 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(
   }
 }
 
-int sm_count() {
-  static int count = 0;
-  if (count == 0) {
-    int dev = 0;
-    cudaGetDevice(&dev);
-    cudaDeviceGetAttribute(&count, cudaDevAttrMultiProcessorCount, dev);
-    if (count <= 0) count = 148;
-  }
-  return count;
-}
-
 }  // namespace
 
 bool attn_tc_supported(int nh, int c, int k, csa_dtype dt, const void* q, const void* kv_comp,

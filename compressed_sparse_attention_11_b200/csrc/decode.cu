@@ -20,6 +20,7 @@
 //   5. attn_combine  : merge the slices and the sink, write bf16 output
 #include "common.cuh"
 #include "launch.h"
+#include "sm100.cuh"
 #include "topk.cuh"
 
 #include <algorithm>
@@ -183,43 +184,128 @@ cudaError_t launch_write_rows(const csa_cache_desc& d, const CacheView& cv, int6
 // ---------------------------------------------------------------------------
 // Per-dim softmax over the state rows of entry i (dims d of a `dim`-wide
 // stream set).  CSA: own block (parity i%2, streams ca/za) and, for i > 0, the
-// previous block (parity (i-1)%2, streams cb/zb).  HCA: streams C/Z.
+// previous block (parity (i-1)%2, streams cb/zb).  HCA: streams C/Z.  The
+// rows are loaded sixteen at a time (CSA: all 2m at once) before they are
+// folded in, so a block of rows costs one memory latency, not one per row.
 __device__ float emit_dim(const __nv_bfloat16* st, int64_t b, int64_t i, int m, int dim, int d,
                           const float* ba, const float* bb, bool hca) {
   float M = kNegInf, S = 0.f, A = 0.f;
+  if (!hca && m <= 8) {  // CSA: both blocks' 2m rows and biases in flight at once
+    const int64_t pa = i & 1, pb = (i - 1) & 1;
+    auto blk = [&](int64_t par, int s) { return st + ((b * 2 + par) * 4 + s) * (int64_t)m * dim; };
+    const __nv_bfloat16 *ca = blk(pa, 0), *za = blk(pa, 2), *cb = blk(pb, 1), *zb = blk(pb, 3);
+    float cv[16], zv[16];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      cv[j] = cv[8 + j] = 0.f;
+      zv[j] = zv[8 + j] = kNegInf;
+      if (j < m) {
+        cv[j] = __bfloat162float(ca[(int64_t)j * dim + d]);
+        zv[j] = __bfloat162float(za[(int64_t)j * dim + d]) + ba[(int64_t)j * dim + d];
+        if (i > 0) {
+          cv[8 + j] = __bfloat162float(cb[(int64_t)j * dim + d]);
+          zv[8 + j] = __bfloat162float(zb[(int64_t)j * dim + d]) + bb[(int64_t)j * dim + d];
+        }
+      }
+    }
+#pragma unroll
+    for (int j = 0; j < 16; ++j)
+      if ((j & 7) < m && (j < 8 || i > 0)) osm_update(M, S, A, zv[j], cv[j]);
+    return A / S;
+  }
+  auto fold = [&](const __nv_bfloat16* cb, const __nv_bfloat16* zb, const float* bias) {
+    for (int j0 = 0; j0 < m; j0 += 16) {
+      float cval[16], zval[16];
+#pragma unroll
+      for (int q = 0; q < 16; ++q) {
+        const int64_t j = j0 + q;
+        cval[q] = 0.f;
+        zval[q] = kNegInf;
+        if (j < m) {
+          cval[q] = __bfloat162float(cb[j * dim + d]);
+          zval[q] = __bfloat162float(zb[j * dim + d]) + bias[j * dim + d];
+        }
+      }
+#pragma unroll
+      for (int q = 0; q < 16; ++q)
+        if (j0 + q < m) osm_update(M, S, A, zval[q], cval[q]);
+    }
+  };
   if (hca) {
     const __nv_bfloat16* base = st + b * 2 * (int64_t)m * dim;
-    for (int j = 0; j < m; ++j) {
-      const float cval = __bfloat162float(base[(int64_t)j * dim + d]);
-      const float z = __bfloat162float(base[((int64_t)m + j) * dim + d]);
-      osm_update(M, S, A, z + ba[(int64_t)j * dim + d], cval);
-    }
+    fold(base, base + (int64_t)m * dim, ba);
   } else {
     const int64_t pa = i & 1, pb = (i - 1) & 1;
-    auto at = [&](int64_t par, int s, int j) {
-      return __bfloat162float(st[(((b * 2 + par) * 4 + s) * m + j) * dim + d]);
-    };
-    for (int j = 0; j < m; ++j) osm_update(M, S, A, at(pa, 2, j) + ba[(int64_t)j * dim + d], at(pa, 0, j));
-    if (i > 0)
-      for (int j = 0; j < m; ++j)
-        osm_update(M, S, A, at(pb, 3, j) + bb[(int64_t)j * dim + d], at(pb, 1, j));
+    auto blk = [&](int64_t par, int s) { return st + ((b * 2 + par) * 4 + s) * (int64_t)m * dim; };
+    fold(blk(pa, 0), blk(pa, 2), ba);
+    if (i > 0) fold(blk(pb, 1), blk(pb, 3), bb);
   }
   return A / S;
 }
 
-__global__ void __launch_bounds__(256) append_emit_kernel(csa_cache_desc d, CacheView cv,
+// The token's rows -- the window row and the compressor-state rows -- copied
+// into the cache with every load issued before any store.
+__device__ void append_rows(const csa_cache_desc& d, const CacheView& cv, const csa_rows& rows,
+                            int64_t b, int64_t u) {
+  typedef __nv_bfloat16 bf;
+  constexpr int kMaxRows = 9;
+  const int64_t c = d.c, ci = d.c_i, m = d.m, row = u % m;
+  const bf* src[kMaxRows];
+  bf* dst[kMaxRows];
+  int nch[kMaxRows];  // 16-byte chunks per row
+  int nr = 0;
+  auto add = [&](const void* sp, bf* dp, int64_t dim) {
+    src[nr] = (const bf*)sp + b * dim;
+    dst[nr] = dp;
+    nch[nr++] = (int)(dim / 8);
+  };
+  add(rows.kv_win, cv.window + (b * d.window + u % d.window) * c, c);
+  if (d.is_hca) {
+    bf* st = cv.state + b * 2 * m * c;
+    add(rows.ca, st + row * c, c);
+    add(rows.za, st + (m + row) * c, c);
+  } else {
+    const int64_t par = (u / m) & 1;
+    const void* sv[4] = {rows.ca, rows.cb, rows.za, rows.zb};
+    const void* iv[4] = {rows.ica, rows.icb, rows.iza, rows.izb};
+    for (int s = 0; s < 4; ++s) {
+      add(sv[s], cv.state + (((b * 2 + par) * 4 + s) * m + row) * c, c);
+      add(iv[s], cv.istate + (((b * 2 + par) * 4 + s) * m + row) * ci, ci);
+    }
+  }
+  int total = 0;
+  for (int r = 0; r < nr; ++r) total += nch[r];
+  constexpr int kPer = 4;  // chunks per thread per round
+  for (int base = 0; base < total; base += (int)blockDim.x * kPer) {
+    uint4 v[kPer];
+    bf* dp[kPer];
+#pragma unroll
+    for (int q = 0; q < kPer; ++q) {
+      int ch = base + q * (int)blockDim.x + (int)threadIdx.x;
+      dp[q] = nullptr;
+      if (ch >= total) continue;
+      int r = 0;
+      while (ch >= nch[r]) ch -= nch[r++];
+      v[q] = *reinterpret_cast<const uint4*>(src[r] + ch * 8);
+      dp[q] = dst[r] + ch * 8;
+    }
+#pragma unroll
+    for (int q = 0; q < kPer; ++q)
+      if (dp[q] != nullptr) *reinterpret_cast<uint4*>(dp[q]) = v[q];
+  }
+}
+
+__global__ void __launch_bounds__(1024) append_emit_kernel(csa_cache_desc d, CacheView cv,
                                                           const int64_t* __restrict__ pos,
-                                                          csa_rows rows, csa_decode_params p,
-                                                          uint32_t* __restrict__ range) {
+                                                          csa_rows rows, csa_decode_params p) {
   extern __shared__ float sx[];  // [c + c_i] + 32
   const int64_t b = blockIdx.x;
-  if (range != nullptr && threadIdx.x == 0) {  // the indexer's score range starts empty
-    range[b * 2 + 0] = 0u;
-    range[b * 2 + 1] = 0xffffffffu;
-  }
+  // the previous step's kernels read the window slot this token overwrites
+  sm100::pdl_wait();
+  sm100::pdl_trigger();
   const int64_t t = pos[b];
   if (t < 0) return;  // no token for this sequence
-  put_rows(d, cv, rows, b, 1, 0, t, true, true);
+  append_rows(d, cv, rows, b, t);
   if ((t + 1) % d.m != 0) return;  // uniform over the block
   __syncthreads();                 // the rows just written are read back below
   const int64_t i = t / d.m;
@@ -338,206 +424,21 @@ __global__ void __launch_bounds__(kSelThreads) topk_merge_kernel(
   block_select_topk<kSelThreads>(CandidatesInGlobal{s, id}, N, d.k, out, id, sh);
 }
 
-// Step 3' (CSA, tensor-core indexer): top-k over one sequence's score array.
-// The indexer recorded the sequence's score range; scores are bucketed
-// linearly over it (4096 buckets), one histogram pass finds the bucket T of
-// the k-th largest score, one pass keeps the scores in buckets >= T (all of
-// buckets > T are chosen), and the bucket-T scores are ranked among
-// themselves (ties to the smaller index).  Degenerate ranges or crowded
-// buckets fall back to the radix select.
-constexpr int kLinBins = 4096;
-constexpr int kLinCap = 4096;        // scores kept in buckets >= T
-constexpr int kLinBucketMax = 1024;  // bucket-T scores ranked directly
-
-struct LinSelShared {
-  uint32_t bins[kLinBins];
-  uint32_t ckey[kLinCap];
-  int32_t cpos[kLinCap];
-  uint32_t bkey[kLinBucketMax];
-  int32_t bslot[kLinBucketMax];
-  uint8_t take[kLinCap];
-  uint32_t wsum[kDecSelThreads / 32];
-  uint32_t T, G, C;
-};
-
-__device__ __forceinline__ int lin_bucket(float s, float lo, float inv) {
-  const float x = (s - lo) * inv;
-  return x <= 0.f ? 0 : (x >= (float)(kLinBins - 1) ? kLinBins - 1 : (int)x);
-}
-
-// Block-wide exclusive prefix of `v` (in thread order); `total` gets the sum.
-__device__ __forceinline__ uint32_t block_exclusive(uint32_t v, uint32_t* wsum, uint32_t& total) {
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, W = blockDim.x >> 5;
-  uint32_t inc = v;
-#pragma unroll
-  for (int off = 1; off < 32; off <<= 1) {
-    const uint32_t x = __shfl_up_sync(0xffffffffu, inc, off);
-    if (lane >= off) inc += x;
-  }
-  __syncthreads();
-  if (lane == 31) wsum[warp] = inc;
-  __syncthreads();
-  uint32_t before = inc - v;
-  total = 0;
-  for (int w = 0; w < W; ++w) {
-    if (w < warp) before += wsum[w];
-    total += wsum[w];
-  }
-  return before;
-}
-
+// Step 3' (CSA, tensor-core indexer), capacities beyond the cluster top-k:
+// top-k over one sequence's score array in global memory.
 __global__ void __launch_bounds__(kDecSelThreads) decode_select_kernel(
     csa_cache_desc d, const int64_t* __restrict__ pos, const float* __restrict__ scores,
-    const uint32_t* __restrict__ range, int32_t* __restrict__ sel) {
-  extern __shared__ __align__(16) unsigned char smem_raw[];
-  LinSelShared& ls = *reinterpret_cast<LinSelShared*>(smem_raw);
-  constexpr int NT = kDecSelThreads;
-  const int tid = threadIdx.x, lane = tid & 31;
+    int32_t* __restrict__ sel) {
+  __shared__ SelectShared<kDecSelThreads> sh;
   const int64_t b = blockIdx.x;
   const int64_t t = pos[b];
   const int64_t V = t < 0 ? 0 : min((t + 1) / d.m, d.capacity);
-  const int k = d.k;
-  int32_t* out = sel + b * k;
-  if (V <= k) {
-    for (int j = tid; j < k; j += NT) out[j] = j < V ? j : -1;
+  int32_t* out = sel + b * d.k;
+  if (V <= d.k) {
+    for (int j = threadIdx.x; j < d.k; j += kDecSelThreads) out[j] = j < V ? j : -1;
     return;
   }
-  const float* row = scores + b * d.capacity;
-  const float hi_s = key_to_float(range[b * 2 + 0]), lo_s = key_to_float(range[b * 2 + 1]);
-  bool fallback = !(hi_s > lo_s) || !isfinite(hi_s - lo_s);
-  const float inv = fallback ? 0.f : (float)kLinBins / (hi_s - lo_s);
-  if (!fallback) {
-    // 1. histogram
-    for (int i = tid; i < kLinBins; i += NT) ls.bins[i] = 0;
-    if (tid == 0) { ls.T = 0; ls.G = 0; ls.C = 0xffffffffu; }
-    __syncthreads();
-    constexpr int kBatch = 8;  // loads in flight per thread
-    for (int64_t i0 = tid; i0 < V; i0 += (int64_t)NT * kBatch) {
-      float v[kBatch];
-#pragma unroll
-      for (int u = 0; u < kBatch; ++u) {
-        const int64_t i = i0 + (int64_t)u * NT;
-        v[u] = i < V ? row[i] : 0.f;
-      }
-#pragma unroll
-      for (int u = 0; u < kBatch; ++u)
-        if (i0 + (int64_t)u * NT < V) atomicAdd(&ls.bins[lin_bucket(v[u], lo_s, inv)], 1u);
-    }
-    __syncthreads();
-    // 2. the bucket where the count from the top reaches k (thread tid owns
-    //    buckets 4095-4tid .. 4092-4tid, descending)
-    constexpr int BPT = kLinBins / NT;
-    uint32_t mine[BPT], loc = 0;
-#pragma unroll
-    for (int j = 0; j < BPT; ++j) {
-      mine[j] = ls.bins[kLinBins - 1 - (tid * BPT + j)];
-      loc += mine[j];
-    }
-    uint32_t tot;
-    uint32_t acc = block_exclusive(loc, ls.wsum, tot);
-#pragma unroll
-    for (int j = 0; j < BPT; ++j) {
-      if (acc < (uint32_t)k && acc + mine[j] >= (uint32_t)k) {
-        ls.T = kLinBins - 1 - (tid * BPT + j);
-        ls.G = acc;
-        ls.C = acc + mine[j];
-      }
-      acc += mine[j];
-    }
-    __syncthreads();
-    fallback = ls.C > (uint32_t)kLinCap || ls.C - ls.G > (uint32_t)kLinBucketMax;
-  }
-  if (fallback) {
-    __syncthreads();
-    auto& sh = *reinterpret_cast<SelectShared<NT>*>(smem_raw);
-    block_select_topk<NT>(ScoresIn{row}, V, k, out, nullptr, sh);
-    return;
-  }
-  const int T = (int)ls.T;
-  const uint32_t G = ls.G, C = ls.C, need = (uint32_t)k - G;
-  // 3. keep the scores in buckets >= T in position order (per warp segments)
-  {
-    constexpr int W = NT / 32;
-    const int warp = tid >> 5;
-    const int64_t seg = ((V + W - 1) / W + 31) / 32 * 32;
-    const int64_t lo = (int64_t)warp * seg, hi = min(V, lo + seg);
-    uint32_t c = 0;
-    constexpr int kBatch = 8;  // loads in flight per lane
-    for (int64_t base = lo; base < hi; base += 32 * kBatch) {
-      float v[kBatch];
-#pragma unroll
-      for (int u = 0; u < kBatch; ++u) {
-        const int64_t i = base + u * 32 + lane;
-        v[u] = i < hi ? row[i] : 0.f;
-      }
-#pragma unroll
-      for (int u = 0; u < kBatch; ++u) {
-        const int64_t i = base + u * 32 + lane;
-        c += __popc(__ballot_sync(0xffffffffu, i < hi && lin_bucket(v[u], lo_s, inv) >= T));
-      }
-    }
-    uint32_t all;
-    uint32_t run = block_exclusive(lane == 0 ? c : 0u, ls.wsum, all);
-    run = __shfl_sync(0xffffffffu, run, 0);
-    const uint32_t lt = (1u << lane) - 1u;
-    for (int64_t base = lo; base < hi; base += 32 * kBatch) {
-      float v[kBatch];
-#pragma unroll
-      for (int u = 0; u < kBatch; ++u) {
-        const int64_t i = base + u * 32 + lane;
-        v[u] = i < hi ? row[i] : 0.f;
-      }
-#pragma unroll
-      for (int u = 0; u < kBatch; ++u) {
-        const int64_t i = base + u * 32 + lane;
-        const int bk = i < hi ? lin_bucket(v[u], lo_s, inv) : -1;
-        const bool keep = i < hi && bk >= T;
-        const uint32_t msk = __ballot_sync(0xffffffffu, keep);
-        if (keep) {
-          const uint32_t p = run + __popc(msk & lt);
-          if (p < (uint32_t)kLinCap) {
-            ls.ckey[p] = order_key(v[u]);
-            ls.cpos[p] = (int32_t)i;
-            ls.take[p] = bk > T ? 1 : 0;
-          }
-        }
-        run += __popc(msk);
-      }
-    }
-    __syncthreads();
-  }
-  // 4. rank the bucket-T scores among themselves
-  {
-    const int per = (int)((C + NT - 1) / NT);
-    const int lo = min((int)C, tid * per), hi = min((int)C, lo + per);
-    uint32_t nb = 0;
-    for (int i = lo; i < hi; ++i) nb += ls.take[i] ? 0u : 1u;
-    uint32_t all;
-    uint32_t o = block_exclusive(nb, ls.wsum, all);
-    for (int i = lo; i < hi; ++i)
-      if (!ls.take[i]) {
-        ls.bkey[o] = ls.ckey[i];
-        ls.bslot[o] = i;
-        ++o;
-      }
-    __syncthreads();
-    for (int e = tid; e < (int)all; e += NT) {
-      const uint32_t ke = ls.bkey[e];
-      uint32_t r = 0;
-      for (int f = 0; f < (int)all; ++f) {
-        const uint32_t kf = ls.bkey[f];
-        r += (kf > ke || (kf == ke && f < e)) ? 1u : 0u;
-      }
-      if (r < need) ls.take[ls.bslot[e]] = 1;
-    }
-    __syncthreads();
-    // 5. the chosen positions, ascending
-    uint32_t nt = 0;
-    for (int i = lo; i < hi; ++i) nt += ls.take[i];
-    uint32_t o2 = block_exclusive(nt, ls.wsum, all);
-    for (int i = lo; i < hi; ++i)
-      if (ls.take[i] && o2 < (uint32_t)k) out[o2++] = ls.cpos[i];
-  }
+  block_select_topk<kDecSelThreads>(ScoresIn{scores + b * d.capacity}, V, d.k, out, nullptr, sh);
 }
 
 // ---------------------------------------------------------------------------
@@ -700,7 +601,7 @@ __global__ void __launch_bounds__(256) attn_combine_kernel(
 struct DecodeWs {
   int nchunks, nsplit;
   bool tc_index, tc_attn;
-  size_t cand_score, cand_idx, scores, range, sel, part_o, part_ms, total;
+  size_t cand_score, cand_idx, scores, sel, part_o, part_ms, total;
 };
 
 static DecodeWs decode_ws_layout(const csa_cache_desc& d) {
@@ -716,7 +617,6 @@ static DecodeWs decode_ws_layout(const csa_cache_desc& d) {
   w.cand_score = off; off = align256(off + B * w.nchunks * d.k * 4);
   w.cand_idx = off;   off = align256(off + B * w.nchunks * d.k * 4);
   w.scores = off;     off = align256(off + (w.tc_index ? B * (size_t)d.capacity * 4 : 0));
-  w.range = off;      off = align256(off + (w.tc_index ? B * 2 * 4 : 0));
   w.sel = off;        off = align256(off + B * (d.is_hca ? 0 : d.k) * 4);
   w.part_o = off;     off = align256(off + B * w.nsplit * d.nh * (size_t)d.c * 4);
   w.part_ms = off;    off = align256(off + B * w.nsplit * d.nh * 2 * 4);
@@ -734,27 +634,30 @@ cudaError_t launch_decode_step(const csa_cache_desc& d, const CacheView& cv, con
   uint8_t* wb = static_cast<uint8_t*>(ws);
   float* cand_score = reinterpret_cast<float*>(wb + w.cand_score);
   int32_t* cand_idx = reinterpret_cast<int32_t*>(wb + w.cand_idx);
-  int32_t* sel = reinterpret_cast<int32_t*>(wb + w.sel);
+  int32_t* sel = p.sel_out != nullptr ? p.sel_out : reinterpret_cast<int32_t*>(wb + w.sel);
   float* part_o = reinterpret_cast<float*>(wb + w.part_o);
   float* part_ms = reinterpret_cast<float*>(wb + w.part_ms);
 
-  uint32_t* range = w.tc_index ? reinterpret_cast<uint32_t*>(wb + w.range) : nullptr;
-  const size_t emit_smem = sizeof(float) * (d.c + (d.is_hca ? 0 : d.c_i) + 32);
-  append_emit_kernel<<<(unsigned)d.batch, 256, emit_smem, s>>>(d, cv, pos, rows, p, range);
-  cudaError_t err = cudaGetLastError();
+  // one thread per emitted dim (c + c_i of them), 256 to 1024 threads
+  const int dims = d.c + (d.is_hca ? 0 : d.c_i);
+  const unsigned emit_threads = (unsigned)std::min(1024, std::max(256, (dims + 31) / 32 * 32));
+  const size_t emit_smem = sizeof(float) * (dims + 32);
+  cudaError_t err = launch_pdl(append_emit_kernel, dim3((unsigned)d.batch), dim3(emit_threads),
+                               emit_smem, s, d, cv, pos, rows, p);
   if (err != cudaSuccess) return err;
   if (!d.is_hca && w.tc_index) {
     float* scores = reinterpret_cast<float*>(wb + w.scores);
     unsigned int* flag = device_timeout_flag();
     if (flag == nullptr) return cudaErrorUnknown;
-    err = launch_decode_index_tc(d, cv, pos, q_i, w_i, scores, range, flag, s);
+    err = launch_decode_index_tc(d, cv, pos, q_i, w_i, scores, flag, s);
     if (err != cudaSuccess) return err;
-    const size_t smem = std::max(sizeof(LinSelShared), sizeof(SelectShared<kDecSelThreads>));
-    cudaFuncSetAttribute(decode_select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                         (int)smem);
-    decode_select_kernel<<<(unsigned)d.batch, kDecSelThreads, smem, s>>>(d, pos, scores, range,
-                                                                          sel);
-    if ((err = cudaGetLastError()) != cudaSuccess) return err;
+    if (decode_topk_supported(d)) {
+      err = launch_decode_topk(d, pos, scores, sel, s);
+    } else {
+      decode_select_kernel<<<(unsigned)d.batch, kDecSelThreads, 0, s>>>(d, pos, scores, sel);
+      err = cudaGetLastError();
+    }
+    if (err != cudaSuccess) return err;
   } else if (!d.is_hca) {
     const size_t smem = sizeof(SelectShared<kSelThreads>) + (size_t)kDecChunk * 8 +
                         (size_t)((d.k + 3) & ~3) * 4 + (size_t)d.c_i * d.nh_i * 4 +

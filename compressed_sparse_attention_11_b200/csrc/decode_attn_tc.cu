@@ -1,23 +1,31 @@
-// Decode attention on the tcgen05 tensor cores over the FP8/bf16 cache: one
-// 128-entry tile of one sequence's entry set per CTA.
+// Decode attention on the tcgen05 tensor cores over the FP8/bf16 cache.
 //
 // For the decode token of sequence b at position t, E_t is (CSA) the selected
 // entries sel[b, :] with 0 <= s < V = floor((t+1)/m), or (HCA) every visible
 // entry, followed by the window rows max(0, t-W+1) .. t from the ring
 // (sections 4.3 / 4.5 of "DeepSeek-V4: million-token context"; entries stored
-// as FP8 codes with one fp32 scale plus bf16 RoPE dims, section 7.3 of the
-// "DeepSeek paper-feature analysis").  Each CTA takes tile j of E_t:
-//   1. all 384 threads gather the tile -- FP8 codes dequantised to bf16
-//      (code * scale), RoPE dims and window rows copied -- into the same
-//      128-byte-swizzled slab layout as the prefill kernel, with many loads
-//      in flight per thread (a decode step has few queries, so the gather's
-//      memory parallelism decides the time);
-//   2. S^T = K Q^T (M = 128 entries, N = 64 heads) on the tensor core;
-//   3. softmax statistics of the tile (max, then exp2 and row sums);
-//   4. O^T = V^T P^T (four M = 128 dim chunks);
-//   5. the tile's unnormalised O, max and sum go to the partial buffers, and
-//      a combine kernel merges the tiles of each sequence with the sink.
-// With a single tile per sequence the CTA writes the final output itself.
+// as 448 FP8 codes with one fp32 scale plus 64 bf16 RoPE dims, section 7.3 of
+// the "DeepSeek paper-feature analysis"); one softmax over E_t and the sink.
+//
+// E_t is cut into 128-entry tiles and each sequence's tiles into `nsplit`
+// contiguous ranges, one CTA per range (about one CTA per SM over the
+// batch).  In a CTA:
+//   * every warp but the MMA warp gathers: each thread owns one 16-dim
+//     quarter of one 64-dim slab for up to 12 rows of the tile, issues all of
+//     its loads at once (the FP8 codes of a row are 448 contiguous bytes, the
+//     RoPE dims and window rows 1 KB of bf16), then dequantises (code * scale)
+//     into the 128-byte-swizzled bf16 slab once the previous tile's P.V has
+//     released that slab;
+//   * S^T = K Q^T (M = 128 entries, N = 64 heads), the eight softmax warps
+//     keep a running max per head (moved, with O^T rescaled in TMEM, only
+//     when a tile's max exceeds it by more than 2^8) and write P^T in bf16;
+//   * O^T += V^T P^T (four M = 128 dim chunks) accumulates in TMEM across the
+//     CTA's tiles; each chunk's completion frees two slabs for the next
+//     tile's gather.
+// The CTA's unnormalised O, max and sum go to the partial buffers and a
+// combine kernel merges a sequence's ranges with the sink; with one range per
+// sequence the CTA writes the normalised output itself.  Every wait is
+// bounded: a fault upstream ends the kernel with the timeout flag set.
 #include "common.cuh"
 #include "launch.h"
 #include "sm100.cuh"
@@ -28,35 +36,60 @@ namespace csa {
 namespace {
 
 constexpr int kNH = 64, kC = 512, kTE = 128;
-constexpr int kSlabs = kC / 64;
-constexpr int kSlabBytes = kTE * 128;
-constexpr int kQSlabBytes = kNH * 128;
-constexpr int kThreads = 384;  // gather: all; then warps 0-7 softmax/epilogue, warp 8 MMA
-constexpr int kMmaWarp = 8;
+constexpr int kRope = 64, kBody = kC - kRope;  // FP8 dims, then bf16 RoPE dims
+constexpr int kSlabs = kC / 64;                // 64-dim slabs; slab 7 holds the RoPE dims
+constexpr int kSlabBytes = kTE * 128;          // 16 KB
+constexpr int kQSlabBytes = kNH * 128;         // 8 KB
+constexpr int kSoftWarps = 8;
+constexpr int kMmaWarp = 11;
+constexpr int kThreads = (kMmaWarp + 1) * 32;  // 384
+constexpr int kGatherThreads = kMmaWarp * 32;  // 352: every warp but the MMA warp
+constexpr int kRowsPerThread = (kTE + kMmaWarp - 1) / kMmaWarp;  // 12
 constexpr int kMaxSelDec = 1024;
+constexpr float kRescaleLog2 = 8.f;
+static_assert(kGatherThreads % 32 == 0, "a thread keeps one slab quarter for every row");
+
+constexpr uint32_t kColS = 0, kColO = 64;  // S^T: 64 columns; O^T: 4 chunks x 64 columns
 
 struct __align__(8) DecAttnBars {
-  uint64_t q_full, s_full, p_full, o_full, grp[2];
+  uint64_t slab_full[kSlabs], slab_empty[kSlabs];
+  uint64_t q_full, s_full, p_full, p_empty, o_full, grp[2];
   uint32_t tmem_base;
-  int nsel;
+  unsigned int abort;  // the timeout flag as read once for the whole CTA
 };
 
 constexpr int OFF_Q = 0;
-constexpr int OFF_KV = OFF_Q + kSlabs * kQSlabBytes;
-constexpr int OFF_P = OFF_KV + kSlabs * kSlabBytes;
-constexpr int OFF_LIST = OFF_P + kTE * 128;
+constexpr int OFF_KV = OFF_Q + kSlabs * kQSlabBytes;    // 65536
+constexpr int OFF_P = OFF_KV + kSlabs * kSlabBytes;     // 196608
+constexpr int OFF_LIST = OFF_P + kTE * 128;             // 212992
 constexpr int OFF_RED = OFF_LIST + kMaxSelDec * 4;      // [2 (max,sum)][2 hh][4 quad][32]
 constexpr int OFF_SCAN = OFF_RED + 2 * 2 * 4 * 32 * 4;  // [12] warp counts
 constexpr int OFF_BAR = OFF_SCAN + 64;
 constexpr int SMEM = OFF_BAR + (int)sizeof(DecAttnBars) + 1024;
 static_assert(SMEM <= 232448, "shared memory budget");
 
-constexpr uint32_t kColS = 0, kColO = 64;
+// 16 FP8 codes -> 16 bf16 (code * scale), as two 16-byte chunks.
+__device__ __forceinline__ void dequant16(const uint4 c8, float sc, uint4& lo, uint4& hi) {
+  const uint32_t w[4] = {c8.x, c8.y, c8.z, c8.w};
+  uint32_t o[8];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+#pragma unroll
+    for (int hlf = 0; hlf < 2; ++hlf) {
+      const __nv_fp8x2_storage_t pair = (__nv_fp8x2_storage_t)((w[i] >> (16 * hlf)) & 0xffffu);
+      const __half2_raw h2 = __nv_cvt_fp8x2_to_halfraw2(pair, __NV_E4M3);
+      const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&h2));
+      o[2 * i + hlf] = pack_bf16x2(f.x * sc, f.y * sc);
+    }
+  }
+  lo = make_uint4(o[0], o[1], o[2], o[3]);
+  hi = make_uint4(o[4], o[5], o[6], o[7]);
+}
 
-__global__ void __launch_bounds__(kThreads, 1) decode_attn_tile_kernel(
+__global__ void __launch_bounds__(kThreads, 1) decode_attn_tc_kernel(
     const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CacheView cv,
     const int64_t* __restrict__ pos, const int32_t* __restrict__ sel, int k, int window, int m,
-    int64_t cap, int rope, const float* __restrict__ sink, float scale, int ntile_max,
+    int64_t cap, const float* __restrict__ sink, float scale, int nsplit,
     float* __restrict__ part_o, float* __restrict__ part_ms, __nv_bfloat16* __restrict__ out,
     unsigned int* __restrict__ err) {
   using namespace sm100;
@@ -71,15 +104,38 @@ __global__ void __launch_bounds__(kThreads, 1) decode_attn_tile_kernel(
   DecAttnBars* bar = reinterpret_cast<DecAttnBars*>(smem + OFF_BAR);
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int tile = blockIdx.x;
+  const int split = blockIdx.x;
   const int64_t b = blockIdx.y;
+  const bool direct = nsplit == 1;
+  const int64_t pbase = (b * nsplit + split) * kNH;
+
+  if (tid == 0) {
+    for (int s = 0; s < kSlabs; ++s) {
+      mbar_init(&bar->slab_full[s], kGatherThreads / 8);  // 4 lanes per slab in each warp
+      mbar_init(&bar->slab_empty[s], 1);
+    }
+    mbar_init(&bar->q_full, 1);
+    mbar_init(&bar->s_full, 1);
+    mbar_init(&bar->p_full, kSoftWarps);
+    mbar_init(&bar->p_empty, 1);
+    mbar_init(&bar->o_full, 1);
+    mbar_init(&bar->grp[0], 4);
+    mbar_init(&bar->grp[1], 4);
+    fence_mbar_init();
+    tma_prefetch_desc(&tm_q);
+  }
+  if (warp == kMmaWarp) {
+    tmem_alloc(&bar->tmem_base, 512);
+    tmem_relinquish();
+  }
+  // set-up above; the selection and the cache are written by earlier kernels
+  pdl_wait();
+  pdl_trigger();
+  if (tid == 0) bar->abort = flag_value(err);
   const int64_t t = pos[b];
   const int64_t V = t < 0 ? 0 : min((t + 1) / m, cap);
   const int64_t w0 = max((int64_t)0, t - window + 1);
   const int nwin = t < 0 ? 0 : (int)(t - w0 + 1);
-  const bool direct = ntile_max == 1;
-  const int64_t pbase = (b * ntile_max + tile) * kNH;
-  if (flag_value(err) != 0) return;
 
   // -------- the entry list: valid selections in order (CSA) or 0..V-1 (HCA) ----
   int nsel;
@@ -106,214 +162,253 @@ __global__ void __launch_bounds__(kThreads, 1) decode_attn_tile_kernel(
     int p = base + inc - cnt;
     for (int j = lo; j < hi; ++j)
       if (row[j] >= 0 && row[j] < V) list[p++] = row[j];
-    __syncthreads();
   } else {
     nsel = (int)V;
   }
   const int N = nsel + nwin;
   const int T = (N + kTE - 1) / kTE;
-  if (tile >= T) {  // an empty tile: contributes nothing to the combine
-    if (!direct && tid < kNH) {
-      part_ms[(pbase + tid) * 2 + 0] = kNegInf;
-      part_ms[(pbase + tid) * 2 + 1] = 0.f;
-    }
-    return;
-  }
-
-  if (tid == 0) {
-    mbar_init(&bar->q_full, 1);
-    mbar_init(&bar->s_full, 1);
-    mbar_init(&bar->p_full, 8);
-    mbar_init(&bar->o_full, 1);
-    mbar_init(&bar->grp[0], 4);
-    mbar_init(&bar->grp[1], 4);
-    fence_mbar_init();
-  }
-  if (warp == kMmaWarp) {
-    tmem_alloc(&bar->tmem_base, 512);
-    tmem_relinquish();
-  }
+  const int tile0 = (int)((int64_t)T * split / nsplit);
+  const int tile1 = (int)((int64_t)T * (split + 1) / nsplit);
+  const int ntile = tile1 - tile0;
   tc_fence_before();
-  __syncthreads();
+  __syncthreads();  // the list, the barriers and the TMEM address
   tc_fence_after();
   const uint32_t tmem = bar->tmem_base;
-  if (tid == 0) {
-    mbar_arrive_expect_tx(&bar->q_full, kSlabs * kQSlabBytes);
-    for (int s = 0; s < kSlabs; ++s)
-      tma_load_3d(sQ + s * kQSlabBytes, &tm_q, &bar->q_full, s * 64, 0, (int)b);
+  const bool live = ntile > 0 && bar->abort == 0;
+  if (!live && !direct && tid < kNH) {  // an empty range adds nothing to the combine
+    part_ms[(pbase + tid) * 2 + 0] = kNegInf;
+    part_ms[(pbase + tid) * 2 + 1] = 0.f;
   }
 
-  // -------- gather: 128 rows x 64 chunks of 8 dims, 8 loads in flight/thread ----
-  const int body = kC - rope;
-  constexpr int kUnroll = 8;
-  for (int e0 = tid; e0 < kTE * 64; e0 += kThreads * kUnroll) {
-    uint4 v[kUnroll];
-    float sc[kUnroll];
-    bool fp8[kUnroll];
+  // -------- gather of tile jt of the range by one thread -------------------------
+  // Thread tid owns 16-dim quarter q_me of slab s_me for rows warp + 11 i.
+  const int s_me = (tid & 31) >> 2, q_me = tid & 3;
+  auto gather_tile = [&](int jt) -> bool {
+    const int tile = tile0 + jt;
+    // an FP8 row (a selected entry, body slab) keeps its scale in hi.x
+    const bool body = s_me < kBody / 64;
+    uint4 lo[kRowsPerThread], hi[kRowsPerThread];
 #pragma unroll
-    for (int u = 0; u < kUnroll; ++u) {
-      const int e = e0 + u * kThreads;
-      v[u] = make_uint4(0, 0, 0, 0);
-      sc[u] = 0.f;
-      fp8[u] = false;
-      if (e >= kTE * 64) continue;
-      const int r = e >> 6, c = e & 63, d0 = c * 8;
+    for (int i = 0; i < kRowsPerThread; ++i) {  // every load in flight before any use
+      const int r = warp + kMmaWarp * i;
+      lo[i] = make_uint4(0, 0, 0, 0);
+      hi[i] = lo[i];
+      if (r >= kTE) continue;
       const int slot = tile * kTE + r;
       if (slot < nsel) {
         const int64_t es = b * cap + (sel != nullptr ? (int64_t)list[slot] : (int64_t)slot);
-        if (d0 < body) {
-          const uint2 c8 = *reinterpret_cast<const uint2*>(cv.entry_fp8 + es * body + d0);
-          v[u].x = c8.x;
-          v[u].y = c8.y;
-          sc[u] = cv.entry_scale[es];
-          fp8[u] = true;
+        if (body) {
+          lo[i] = __ldcs(reinterpret_cast<const uint4*>(cv.entry_fp8 + es * kBody + s_me * 64 +
+                                                         q_me * 16));
+          hi[i].x = __float_as_uint(__ldcs(cv.entry_scale + es));
         } else {
-          v[u] = *reinterpret_cast<const uint4*>(cv.entry_rope + es * rope + (d0 - body));
+          const uint4* p = reinterpret_cast<const uint4*>(cv.entry_rope + es * kRope + q_me * 16);
+          lo[i] = __ldcs(p);
+          hi[i] = __ldcs(p + 1);
         }
       } else if (slot < N) {
-        const int64_t u_pos = w0 + (slot - nsel);
-        v[u] = *reinterpret_cast<const uint4*>(cv.window + (b * window + u_pos % window) * kC +
-                                               d0);
+        const int64_t u = w0 + (slot - nsel);
+        const uint4* p = reinterpret_cast<const uint4*>(
+            cv.window + (b * window + u % window) * kC + s_me * 64 + q_me * 16);
+        lo[i] = __ldcs(p);
+        hi[i] = __ldcs(p + 1);
       }
     }
+    // the slab is free once the previous tile's P.V chunk that reads it is done
+    if (jt >= 1 && !mbar_wait(&bar->slab_empty[s_me], (uint32_t)((jt - 1) & 1), err)) return false;
+    uint8_t* dst = sKV + s_me * kSlabBytes;
 #pragma unroll
-    for (int u = 0; u < kUnroll; ++u) {
-      const int e = e0 + u * kThreads;
-      if (e >= kTE * 64) continue;
-      const int r = e >> 6, c = e & 63;
-      uint4 o = v[u];
-      if (fp8[u]) {
-        const uint32_t w2[2] = {v[u].x, v[u].y};
-        uint32_t q[4];
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          const uint32_t pair = (w2[i >> 1] >> ((i & 1) * 16)) & 0xffffu;
-          q[i] = pack_bf16x2(e4m3_value((uint8_t)(pair & 0xff)) * sc[u],
-                             e4m3_value((uint8_t)(pair >> 8)) * sc[u]);
-        }
-        o = make_uint4(q[0], q[1], q[2], q[3]);
-      }
-      const int slab = c >> 3, cs = c & 7;
-      *reinterpret_cast<uint4*>(sKV + slab * kSlabBytes + r * 128 + ((cs ^ (r & 7)) * 16)) = o;
+    for (int i = 0; i < kRowsPerThread; ++i) {
+      const int r = warp + kMmaWarp * i;
+      if (r >= kTE) continue;
+      uint4 a = lo[i], c = hi[i];
+      if (body && tile * kTE + r < nsel) dequant16(lo[i], __uint_as_float(hi[i].x), a, c);
+      *reinterpret_cast<uint4*>(dst + r * 128 + (((2 * q_me) ^ (r & 7)) * 16)) = a;
+      *reinterpret_cast<uint4*>(dst + r * 128 + (((2 * q_me + 1) ^ (r & 7)) * 16)) = c;
     }
-  }
-  fence_proxy_async();
-  tc_fence_before();
-  __syncthreads();
-  tc_fence_after();
+    fence_proxy_async();  // generic-proxy writes before the tensor core reads them
+    mbar_arrive(&bar->slab_full[s_me]);
+    return true;
+  };
 
   if (warp == kMmaWarp) {
     // -------------------------------- MMA ----------------------------------------
-    constexpr uint32_t kIdQK = idesc_bf16(kTE, kNH, 0, 0);
-    constexpr uint32_t kIdPV = idesc_bf16(128, kNH, 1, 1);
-    const uint32_t kv0 = smem_u32(sKV), q0 = smem_u32(sQ), p0 = smem_u32(sP);
-    if (mbar_wait(&bar->q_full, 0, err)) {
-      tc_fence_after();
+    if (live) {
+      constexpr uint32_t kIdQK = idesc_bf16(kTE, kNH, 0, 0);
+      constexpr uint32_t kIdPV = idesc_bf16(128, kNH, 1, 1);
+      const uint32_t kv0 = smem_u32(sKV), q0 = smem_u32(sQ), p0 = smem_u32(sP);
       if (lane == 0) {
+        mbar_arrive_expect_tx(&bar->q_full, kSlabs * kQSlabBytes);
         for (int s = 0; s < kSlabs; ++s)
-#pragma unroll
-          for (int kk = 0; kk < 4; ++kk)
-            mma_bf16(tmem + kColS, desc_sw128(kv0 + s * kSlabBytes + kk * 32),
-                     desc_sw128(q0 + s * kQSlabBytes + kk * 32), kIdQK, (s | kk) != 0 ? 1u : 0u);
-        mma_commit(&bar->s_full);
+          tma_load_3d(sQ + s * kQSlabBytes, &tm_q, &bar->q_full, s * 64, 0, (int)b);
       }
       __syncwarp();
-      if (mbar_wait(&bar->p_full, 0, err)) {
+      bool ok = mbar_wait(&bar->q_full, 0, err);
+      int issued = 0;  // tiles whose P.V was issued
+      for (int jt = 0; jt < ntile && ok; ++jt) {
+        for (int s = 0; s < kSlabs && ok; ++s)
+          ok = mbar_wait(&bar->slab_full[s], (uint32_t)(jt & 1), err);
+        if (!ok) break;
         tc_fence_after();
         if (lane == 0) {
-          for (int c = 0; c < 4; ++c)
+          for (int s = 0; s < kSlabs; ++s)
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk)
+              mma_bf16(tmem + kColS, desc_sw128(kv0 + s * kSlabBytes + kk * 32),
+                       desc_sw128(q0 + s * kQSlabBytes + kk * 32), kIdQK, (s | kk) != 0 ? 1u : 0u);
+          mma_commit(&bar->s_full);
+        }
+        __syncwarp();
+        if (!(ok = mbar_wait(&bar->p_full, (uint32_t)(jt & 1), err))) break;
+        tc_fence_after();
+        if (lane == 0) {
+          for (int c = 0; c < 4; ++c) {
 #pragma unroll
             for (int kk = 0; kk < kTE / 16; ++kk)
               mma_bf16(tmem + kColO + c * kNH,
                        desc_sw128_mn(kv0 + 2 * c * kSlabBytes + kk * 2048, kSlabBytes, 1024),
-                       desc_sw128_mn(p0 + kk * 2048, 1024, 1024), kIdPV, kk > 0 ? 1u : 0u);
-          mma_commit(&bar->o_full);
+                       desc_sw128_mn(p0 + kk * 2048, 1024, 1024), kIdPV,
+                       (jt == 0 && kk == 0) ? 0u : 1u);
+            mma_commit(&bar->slab_empty[2 * c]);
+            mma_commit(&bar->slab_empty[2 * c + 1]);
+          }
+          mma_commit(&bar->p_empty);
         }
         __syncwarp();
-        mbar_wait(&bar->o_full, 0, err, false);  // drain before TMEM is released
+        ++issued;
       }
-    } else {
-      mbar_wait(&bar->q_full, 0, err, false);
+      if (lane == 0) mma_commit(&bar->o_full);
+      __syncwarp();
+      mbar_wait(&bar->o_full, 0, err, false);  // every MMA done before TMEM is released
+      if (!ok && issued == 0) mbar_wait(&bar->q_full, 0, err, false);  // the Q load has landed
     }
-  } else if (warp < 8) {
-    // ------------------------- softmax and epilogue --------------------------------
+  } else if (warp >= kSoftWarps) {
+    // ------------------------------ gather only ----------------------------------
+    for (int jt = 0; jt < ntile && live; ++jt)
+      if (!gather_tile(jt)) break;
+  } else if (live) {
+    // ----------------------- gather, softmax and epilogue ---------------------------
     const int quad = warp & 3, hh = warp >> 2;
-    const int row = quad * 32 + lane;
+    const int row = quad * 32 + lane;  // entry row within a tile / dim within a chunk
     const uint32_t lane_base = tmem + ((uint32_t)(quad * 32) << 16);
+    const uint32_t s_addr = lane_base + kColS + hh * 32;
     const float qscale = scale * kLog2e;
     uint32_t gphase = 0;
-    bool ok = mbar_wait(&bar->s_full, 0, err);
-    float m_h = kNegInf, psum[32];
-    if (ok) {
-      tc_fence_after();
-      const bool valid = tile * kTE + row < N;
-      uint32_t r[32];
-      tmem_ld32(lane_base + kColS + hh * 32, r);
-      tmem_ld_wait();
-      float v[32];
+    float m_run = kNegInf;  // lane i: running max (log2 units) of head hh*32+i
+    float psum[32];
 #pragma unroll
-      for (int i = 0; i < 32; ++i) v[i] = valid ? __uint_as_float(r[i]) * qscale : kNegInf;
+    for (int i = 0; i < 32; ++i) psum[i] = 0.f;
+    bool ok = true;
+    for (int jt = 0; jt < ntile && ok; ++jt) {
+      if (!(ok = gather_tile(jt))) break;
+      if (!(ok = mbar_wait(&bar->s_full, (uint32_t)(jt & 1), err))) break;
+      tc_fence_after();
+      const bool valid = (tile0 + jt) * kTE + row < N;
+      float v[32];
+      {
+        uint32_t r[32];
+        tmem_ld32(s_addr, r);
+        tmem_ld_wait();
+#pragma unroll
+        for (int i = 0; i < 32; ++i) v[i] = valid ? __uint_as_float(r[i]) * qscale : kNegInf;
+      }
       float* rmax = red + (hh * 4) * 32;
       rmax[quad * 32 + lane] = transpose_reduce<true>(v);
-      ok = group_sync(&bar->grp[hh], gphase, err);
-      if (ok) {
-        m_h = fmaxf(fmaxf(rmax[lane], rmax[32 + lane]), fmaxf(rmax[64 + lane], rmax[96 + lane]));
-        uint32_t pk[16];
-#pragma unroll
-        for (int i = 0; i < 32; i += 2) {
-          float ma = __shfl_sync(0xffffffffu, m_h, i), mb = __shfl_sync(0xffffffffu, m_h, i + 1);
-          ma = ma == kNegInf ? 0.f : ma;
-          mb = mb == kNegInf ? 0.f : mb;
-          const float la = valid ? __uint_as_float(r[i]) * qscale : kNegInf;
-          const float lb = valid ? __uint_as_float(r[i + 1]) * qscale : kNegInf;
-          const float pa = ex2(la - ma), pb = ex2(lb - mb);
-          psum[i] = pa;
-          psum[i + 1] = pb;
-          pk[i >> 1] = pack_bf16x2(pa, pb);
-        }
-        uint8_t* prow = sP + row * 128;
-#pragma unroll
-        for (int j = 0; j < 4; ++j)
-          *reinterpret_cast<uint4*>(prow + (((hh * 4 + j) ^ (row & 7)) * 16)) =
-              make_uint4(pk[4 * j], pk[4 * j + 1], pk[4 * j + 2], pk[4 * j + 3]);
-        fence_proxy_async();
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&bar->p_full);
+      if (!(ok = group_sync(&bar->grp[hh], gphase, err))) break;
+      const float mtile = fmaxf(fmaxf(rmax[lane], rmax[32 + lane]),
+                                fmaxf(rmax[64 + lane], rmax[96 + lane]));
+      float f_lane = 1.f;
+      bool resc = false;
+      if (jt == 0) {
+        m_run = mtile;
+      } else if (mtile > m_run + kRescaleLog2) {
+        resc = true;
+        f_lane = ex2(m_run - mtile);
+        m_run = mtile;
       }
+      // rmax is rewritten next tile only after every warp of the group has read it
+      if (!(ok = group_sync(&bar->grp[hh], gphase, err))) break;
+      // P^T (and, for a rescale, O^T) is free once the previous P.V is done
+      if (jt >= 1 && !(ok = mbar_wait(&bar->p_empty, (uint32_t)((jt - 1) & 1), err))) break;
+      tc_fence_after();
+      if (__any_sync(0xffffffffu, resc)) {
+        float f[32];
+#pragma unroll
+        for (int i = 0; i < 32; ++i) {
+          f[i] = __shfl_sync(0xffffffffu, f_lane, i);
+          psum[i] *= f[i];
+        }
+        for (int c = 0; c < 4; ++c) {
+          uint32_t o[32];
+          tmem_ld32(lane_base + kColO + c * kNH + hh * 32, o);
+          tmem_ld_wait();
+#pragma unroll
+          for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * f[i]);
+          tmem_st32(lane_base + kColO + c * kNH + hh * 32, o);
+        }
+        tmem_st_wait();
+      }
+      uint32_t r[32];  // the logits again (cheaper than holding them across the reductions)
+      tmem_ld32(s_addr, r);
+      tmem_ld_wait();
+      uint32_t pk[16];
+#pragma unroll
+      for (int i = 0; i < 32; i += 2) {
+        float ma = __shfl_sync(0xffffffffu, m_run, i);
+        float mb = __shfl_sync(0xffffffffu, m_run, i + 1);
+        ma = ma == kNegInf ? 0.f : ma;
+        mb = mb == kNegInf ? 0.f : mb;
+        const float la = valid ? __uint_as_float(r[i]) * qscale : kNegInf;
+        const float lb = valid ? __uint_as_float(r[i + 1]) * qscale : kNegInf;
+        const float pa = ex2(la - ma), pb = ex2(lb - mb);
+        psum[i] += pa;
+        psum[i + 1] += pb;
+        pk[i >> 1] = pack_bf16x2(pa, pb);
+      }
+      uint8_t* prow = sP + row * 128;
+#pragma unroll
+      for (int j = 0; j < 4; ++j)
+        *reinterpret_cast<uint4*>(prow + (((hh * 4 + j) ^ (row & 7)) * 16)) =
+            make_uint4(pk[4 * j], pk[4 * j + 1], pk[4 * j + 2], pk[4 * j + 3]);
+      fence_proxy_async();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bar->p_full);
     }
+    // ---- epilogue: this range's O^T, max and sum (or, alone, the output) ----------
     if (ok) ok = mbar_wait(&bar->o_full, 0, err);
     if (ok) {
       tc_fence_after();
       float* rsum = red + (2 * 4 + hh * 4) * 32;
       rsum[quad * 32 + lane] = transpose_reduce<false>(psum);
       ok = group_sync(&bar->grp[hh], gphase, err);
-      if (ok) {
-        const int h = hh * 32 + lane;
-        const float tot = rsum[lane] + rsum[32 + lane] + rsum[64 + lane] + rsum[96 + lane];
-        float inv = 1.f;
-        if (direct) {
-          const float mref = m_h == kNegInf ? 0.f : m_h;
-          const float z = sink != nullptr ? sink[h] * kLog2e : kNegInf;
-          inv = 1.f / (tot + (z == kNegInf ? 0.f : ex2(z - mref)));
-        } else if (quad == 0) {
-          part_ms[(pbase + h) * 2 + 0] = m_h;
-          part_ms[(pbase + h) * 2 + 1] = tot;
-        }
-        for (int c = 0; c < 4; ++c) {
-          uint32_t o[32];
-          tmem_ld32(lane_base + kColO + c * kNH + hh * 32, o);
-          tmem_ld_wait();
-          const int d = c * 128 + row;
+    }
+    if (ok) {
+      const int h = hh * 32 + lane;
+      const float* rsum = red + (2 * 4 + hh * 4) * 32;
+      const float tot = rsum[lane] + rsum[32 + lane] + rsum[64 + lane] + rsum[96 + lane];
+      float inv = 1.f;
+      if (direct) {
+        const float mref = m_run == kNegInf ? 0.f : m_run;
+        const float z = sink != nullptr ? sink[h] * kLog2e : kNegInf;
+        inv = 1.f / (tot + (z == kNegInf ? 0.f : ex2(z - mref)));
+      } else if (quad == 0) {
+        part_ms[(pbase + h) * 2 + 0] = m_run;
+        part_ms[(pbase + h) * 2 + 1] = tot;
+      }
+      for (int c = 0; c < 4; ++c) {
+        uint32_t o[32];
+        tmem_ld32(lane_base + kColO + c * kNH + hh * 32, o);
+        tmem_ld_wait();
+        const int d = c * 128 + row;
 #pragma unroll
-          for (int i = 0; i < 32; ++i) {
-            const int hd = hh * 32 + i;
-            if (direct)
-              out[(b * kNH + hd) * kC + d] =
-                  __float2bfloat16_rn(__uint_as_float(o[i]) * __shfl_sync(0xffffffffu, inv, i));
-            else
-              part_o[(pbase + hd) * kC + d] = __uint_as_float(o[i]);
-          }
+        for (int i = 0; i < 32; ++i) {
+          const int hd = hh * 32 + i;
+          if (direct)
+            out[(b * kNH + hd) * kC + d] =
+                __float2bfloat16_rn(__uint_as_float(o[i]) * __shfl_sync(0xffffffffu, inv, i));
+          else
+            part_o[(pbase + hd) * kC + d] = __uint_as_float(o[i]);
         }
       }
     }
@@ -327,26 +422,28 @@ __global__ void __launch_bounds__(kThreads, 1) decode_attn_tile_kernel(
   }
 }
 
-// Merges the tiles of each sequence: o = sum_i 2^(m_i - M) O_i /
-// (sum_i 2^(m_i - M) l_i + 2^(sink - M)).  One CTA per (sequence, head).
+// Merges the ranges of each sequence: o = sum_i 2^(m_i - M) O_i /
+// (sum_i 2^(m_i - M) l_i + 2^(sink - M)).  One CTA per (head, sequence).
 __global__ void __launch_bounds__(128) decode_combine_kernel(
     const float* __restrict__ part_o, const float* __restrict__ part_ms,
-    const float* __restrict__ sink, int ntile, __nv_bfloat16* __restrict__ out) {
+    const float* __restrict__ sink, int nsplit, __nv_bfloat16* __restrict__ out) {
+  sm100::pdl_wait();  // the partials come from the previous kernel
+  sm100::pdl_trigger();
   const int64_t b = blockIdx.y;
   const int h = blockIdx.x;
   const float z = sink != nullptr ? sink[h] * kLog2e : kNegInf;
   float M = z;
-  for (int i = 0; i < ntile; ++i) M = fmaxf(M, part_ms[((b * ntile + i) * kNH + h) * 2]);
+  for (int i = 0; i < nsplit; ++i) M = fmaxf(M, part_ms[((b * nsplit + i) * kNH + h) * 2]);
   float den = z == kNegInf ? 0.f : ex2(z - M);
   float acc[4] = {0.f, 0.f, 0.f, 0.f};
   const int d0 = threadIdx.x * 4;
-  for (int i = 0; i < ntile; ++i) {
-    const int64_t base = (b * ntile + i) * kNH + h;
+  for (int i = 0; i < nsplit; ++i) {
+    const int64_t base = (b * nsplit + i) * kNH + h;
     const float mi = part_ms[base * 2];
     if (mi == kNegInf) continue;
     const float wgt = ex2(mi - M);
     den = fmaf(wgt, part_ms[base * 2 + 1], den);
-    const float4 o = *reinterpret_cast<const float4*>(part_o + base * kC + d0);
+    const float4 o = __ldcs(reinterpret_cast<const float4*>(part_o + base * kC + d0));
     acc[0] = fmaf(wgt, o.x, acc[0]);
     acc[1] = fmaf(wgt, o.y, acc[1]);
     acc[2] = fmaf(wgt, o.z, acc[2]);
@@ -361,33 +458,36 @@ __global__ void __launch_bounds__(128) decode_combine_kernel(
 }  // namespace
 
 bool decode_attn_tc_supported(const csa_cache_desc& d) {
-  return d.nh == kNH && d.c == kC && (d.is_hca || d.k <= kMaxSelDec) && d.rope_dims % 8 == 0;
+  return d.nh == kNH && d.c == kC && d.rope_dims == kRope && (d.is_hca || d.k <= kMaxSelDec);
 }
 
 int decode_attn_splits(const csa_cache_desc& d) {
-  const int64_t slots = (d.is_hca ? d.capacity : (int64_t)d.k) + d.window;
-  return (int)((slots + kTE - 1) / kTE);
+  const int64_t slots = (d.is_hca ? d.capacity : (int64_t)std::min<int64_t>(d.k, d.capacity)) +
+                        d.window;
+  const int64_t tmax = (slots + kTE - 1) / kTE;
+  const int64_t per_sm = std::max<int64_t>(1, sm_count() / std::max<int64_t>(1, d.batch));
+  return (int)std::max<int64_t>(1, std::min<int64_t>(tmax, per_sm));
 }
 
 cudaError_t launch_decode_attn_tc(const csa_cache_desc& d, const CacheView& cv,
                                   const int64_t* pos, const void* q, const int32_t* sel,
-                                  const float* sink, float scale, int ntile, void* out,
+                                  const float* sink, float scale, int nsplit, void* out,
                                   float* part_o, float* part_ms, unsigned int* err,
                                   cudaStream_t s) {
   CUtensorMap tq;
   if (!make_tmap_bf16_3d(&tq, q, kC, kNH, d.batch, kC * 2ull, (uint64_t)kNH * kC * 2, 64, kNH))
     return cudaErrorInvalidValue;
-  cudaError_t e = cudaFuncSetAttribute(decode_attn_tile_kernel,
+  cudaError_t e = cudaFuncSetAttribute(decode_attn_tc_kernel,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM);
   if (e != cudaSuccess) return e;
-  decode_attn_tile_kernel<<<dim3((unsigned)ntile, (unsigned)d.batch), kThreads, SMEM, s>>>(
-      tq, cv, pos, d.is_hca ? nullptr : sel, d.k, d.window, d.m, d.capacity, d.rope_dims, sink,
-      scale, ntile, part_o, part_ms, (__nv_bfloat16*)out, err);
-  if ((e = cudaGetLastError()) != cudaSuccess || ntile == 1) return e;
-  decode_combine_kernel<<<dim3(kNH, (unsigned)d.batch), kC / 4, 0, s>>>(part_o, part_ms, sink,
-                                                                        ntile,
-                                                                        (__nv_bfloat16*)out);
-  return cudaGetLastError();
+  e = launch_pdl(decode_attn_tc_kernel, dim3((unsigned)nsplit, (unsigned)d.batch), dim3(kThreads),
+                 (size_t)SMEM, s, tq, cv, pos, d.is_hca ? nullptr : sel, (int)d.k, (int)d.window,
+                 (int)d.m, (int64_t)d.capacity, sink, scale, nsplit, part_o, part_ms,
+                 (__nv_bfloat16*)out, err);
+  if (e != cudaSuccess || nsplit == 1) return e;
+  return launch_pdl(decode_combine_kernel, dim3(kNH, (unsigned)d.batch), dim3(kC / 4), 0, s,
+                    (const float*)part_o, (const float*)part_ms, sink, nsplit,
+                    (__nv_bfloat16*)out);
 }
 
 }  // namespace csa

@@ -1,4 +1,4 @@
-// Decode indexer on the tcgen05 tensor cores, FP8 x FP8.
+// Decode indexer on the tcgen05 tensor cores, FP8 x FP8, persistent.
 //
 // For one decode token per sequence b at position t:
 //   I[s] = sum_h w[h] * ReLU(q_i[h, :] . k_s),  k_s = scale_s * code_s,
@@ -9,20 +9,26 @@
 // the contraction.
 //
 // The keys dominate the bytes of a decode step, so this kernel is an HBM
-// stream with the FP8 tiles fed to the tensor core as they arrive: TMA brings
-// 128-key tiles (16 KB, 128-byte swizzle) into a 12-stage ring and one lane
-// issues M=128 keys x N=2H x K=128 kind::f8f6f4 MMAs straight from the ring.
-// The B operand holds each query head twice: hi = E4M3(q/s_h) and
-// lo = E4M3(q/s_h - hi), s_h a power of two with max|q_h|/s_h <= 448, so
-// s_h (hi + lo) reproduces the bf16 query exactly except for elements below
-// 2^-6 s_h in magnitude (absolute error below 2^-10 s_h there).  Two groups
-// of four epilogue warps (alternate tiles, up to four accumulators in TMEM)
-// add the two halves, apply ReLU, the head weights (with s_h folded in) and
-// the key scale; scores go to a per-sequence fp32 array
-// (L2-resident at these sizes) for the selection kernel, with the largest
-// and smallest score order keys of each sequence (atomicMax / atomicMin into
-// `range`, which must hold 0 / ~0 on entry).  One CTA per SM keeps 12 tiles
-// (192 KB) in flight.
+// stream with the FP8 tiles fed to the tensor core as they arrive.  All
+// sequences' 128-key tiles form one list, cut into equal contiguous ranges,
+// one per CTA (one CTA per SM); each CTA keeps a single TMA ring of 16 KB
+// tiles (128-byte swizzle) full across sequence boundaries, so the stream
+// never drains between sequences.  One lane issues M = 128 keys x N = 2H x
+// K = 128 kind::f8f6f4 MMAs straight from the ring.  The B operand holds each
+// query head twice: hi = E4M3(q/s_h) and lo = E4M3(q/s_h - hi), s_h a power
+// of two with max|q_h|/s_h <= 448, so s_h (hi + lo) reproduces the bf16 query
+// exactly except for elements below 2^-6 s_h in magnitude (absolute error
+// below 2^-10 s_h there); two warps build it for the next sequence of the
+// range while the current one streams (two operand slots, each freed by the
+// MMAs of its sequence's last tile; the head weights sit in a 16-deep ring
+// freed by the epilogue, which trails the MMAs by at most ten tiles, so no
+// phase of its barriers can alias).  Per K step two
+// N = H MMAs accumulate the hi and the lo halves into the same TMEM columns,
+// so the accumulator already holds q . code.  Two warpgroups of epilogue warps
+// take alternate tiles (eight accumulators in TMEM for H = 64) and apply
+// ReLU, the head weights (with s_h folded in) and the key scale; scores go to
+// a per-sequence fp32 array (L2-resident at these sizes) for the selection
+// kernel.
 #include "common.cuh"
 #include "launch.h"
 #include "sm100.cuh"
@@ -31,228 +37,365 @@ namespace csa {
 
 namespace {
 
-constexpr int kKeys = 128;             // keys per tile (MMA M)
-constexpr int kCI = 128;               // index-key dim = bytes per FP8 key
-constexpr int kStages = 12;              // 192 KB of key tiles in flight per SM
+constexpr int kKeys = 128;               // keys per tile (MMA M)
+constexpr int kCI = 128;                 // index-key dim = bytes per FP8 key
 constexpr int kTileBytes = kKeys * kCI;  // 16 KB
-constexpr int kChunk = 2048;           // keys per CTA
-constexpr int kThreads = 384;          // warp 0 TMA, warp 1 MMA, warps 4-11 epilogue
+constexpr int kThreads = 384;  // warp 0 TMA, 1 MMA, 2-3 query split, 4-7 / 8-11 epilogue
+constexpr int kBSlots = 2;               // query operands (sequences) in flight
+constexpr int kWSlots = 16;              // head-weight vectors (sequences) in flight
+constexpr int kSmemLimit = 232448;
 
-constexpr int kDBufs = 4;              // TMEM accumulators (tiles in flight past the MMA)
-
+template <int S>
 struct __align__(8) DecIdxBars {
-  uint64_t full[kStages], empty[kStages], d_full[kDBufs], d_empty[kDBufs], drain;
+  uint64_t full[S], empty[S], d_full[8], d_empty[8], b_full[kBSlots], b_empty[kBSlots], drain;
+  uint64_t w_full[kWSlots], w_empty[kWSlots];
   uint32_t tmem_base;
+  int j0, count;  // the CTA's first tile (within sequence b0) and its number of tiles
+  int64_t b0;
 };
 
 template <int H>
 struct DecIdxCfg {
   static constexpr int N = 2 * H;                  // hi and lo rows per head
+  static constexpr int B_BYTES = N * 128;          // one query operand
+  static constexpr int STAGES =
+      (kSmemLimit - 1024 - kBSlots * B_BYTES - kWSlots * H * 4 - 768) / kTileBytes;
   static constexpr int OFF_RAW = 0;
-  static constexpr int OFF_B = OFF_RAW + kStages * kTileBytes;
-  static constexpr int OFF_W = OFF_B + N * 128;
-  static constexpr int OFF_BAR = OFF_W + H * 4;
-  static constexpr int SMEM = OFF_BAR + (int)sizeof(DecIdxBars) + 1024;
-  static constexpr uint32_t TMEM_COLS = kDBufs * N <= 512 ? kDBufs * N : 512;
-  static constexpr int DBUFS = (int)(TMEM_COLS / N);  // 4 for H = 64, 2 for H = 128
+  static constexpr int OFF_B = OFF_RAW + STAGES * kTileBytes;
+  static constexpr int OFF_W = OFF_B + kBSlots * B_BYTES;
+  static constexpr int OFF_BAR = OFF_W + kWSlots * H * 4;
+  static constexpr int SMEM = OFF_BAR + (int)sizeof(DecIdxBars<STAGES>) + 1024;
+  static constexpr int DBUFS = 512 / H;            // TMEM accumulators: 8 (H = 64), 4 (H = 128)
+  static_assert(SMEM <= kSmemLimit, "shared memory budget");
+  static_assert(DBUFS >= 2 && DBUFS <= 8 && DBUFS % 2 == 0, "TMEM accumulators");
 };
+
+__device__ __forceinline__ int tiles_of(const int64_t* pos, int64_t b, int m, int64_t cap) {
+  const int64_t t = pos[b];
+  const int64_t V = t < 0 ? 0 : min((t + 1) / m, cap);
+  return (int)((V + kKeys - 1) / kKeys);
+}
+
+// Walks the CTA's tiles in order: sequence b, tile j of nt.
+struct TileWalk {
+  int64_t b;
+  int j, nt;
+  __device__ void start(const int64_t* pos, int64_t b0, int j0, int m, int64_t cap) {
+    b = b0;
+    j = j0;
+    nt = tiles_of(pos, b0, m, cap);
+  }
+  __device__ void next(const int64_t* pos, int64_t batch, int m, int64_t cap) {
+    if (++j < nt) return;
+    j = 0;
+    do {
+      ++b;
+      nt = b < batch ? tiles_of(pos, b, m, cap) : 1;
+    } while (nt == 0);
+  }
+};
+
+// Warp 0: this CTA's contiguous share [g0, g1) of the flattened tile list
+// and the sequence / tile where it starts.
+__device__ void locate_range(const int64_t* pos, int64_t batch, int m, int64_t cap,
+                             int64_t& b0, int& j0, int& count) {
+  const int lane = threadIdx.x & 31;
+  int64_t total = 0;
+  for (int64_t base = 0; base < batch; base += 32) {
+    int64_t nt = base + lane < batch ? tiles_of(pos, base + lane, m, cap) : 0;
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) nt += __shfl_xor_sync(0xffffffffu, nt, off);
+    total += nt;
+  }
+  const int64_t g0 = total * blockIdx.x / gridDim.x, g1 = total * (blockIdx.x + 1) / gridDim.x;
+  count = (int)(g1 - g0);
+  b0 = 0;
+  j0 = 0;
+  if (count == 0) return;
+  int64_t run = 0;
+  for (int64_t base = 0; base < batch; base += 32) {
+    const int64_t nt = base + lane < batch ? tiles_of(pos, base + lane, m, cap) : 0;
+    int64_t inc = nt;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+      const int64_t v = __shfl_up_sync(0xffffffffu, inc, off);
+      if (lane >= off) inc += v;
+    }
+    const unsigned hit = __ballot_sync(0xffffffffu, run + inc > g0);
+    if (hit != 0) {
+      const int f = __ffs(hit) - 1;
+      const int64_t before = __shfl_sync(0xffffffffu, run + inc - nt, f);
+      b0 = base + f;
+      j0 = (int)(g0 - before);
+      return;
+    }
+    run += __shfl_sync(0xffffffffu, inc, 31);
+  }
+}
 
 template <int H>
 __global__ void __launch_bounds__(kThreads, 1) decode_index_tc_kernel(
     const __grid_constant__ CUtensorMap tm_keys, const float* __restrict__ key_scale,
     const __nv_bfloat16* __restrict__ q_i, const float* __restrict__ w_i,
-    const int64_t* __restrict__ pos, int64_t cap, int m, float* __restrict__ scores,
-    unsigned int* __restrict__ range, unsigned int* __restrict__ err) {
+    const int64_t* __restrict__ pos, int64_t batch, int64_t cap, int m,
+    float* __restrict__ scores, unsigned int* __restrict__ err) {
   using C = DecIdxCfg<H>;
+  constexpr int S = C::STAGES, DB = C::DBUFS;
   using namespace sm100;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = smem_raw + ((1024 - (smem_u32(smem_raw) & 1023)) & 1023);
   uint8_t* sRaw = smem + C::OFF_RAW;
   uint8_t* sB = smem + C::OFF_B;
   float* sW = reinterpret_cast<float*>(smem + C::OFF_W);
-  DecIdxBars* bar = reinterpret_cast<DecIdxBars*>(smem + C::OFF_BAR);
-
+  DecIdxBars<S>* bar = reinterpret_cast<DecIdxBars<S>*>(smem + C::OFF_BAR);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int64_t b = blockIdx.y;
-  const int64_t t = pos[b];
-  const int64_t V = t < 0 ? 0 : min((t + 1) / m, cap);
-  const int64_t c0 = (int64_t)blockIdx.x * kChunk;
-  const int64_t Vc = max((int64_t)0, min((int64_t)kChunk, V - c0));
-  const int ntiles = (int)((Vc + kKeys - 1) / kKeys);
-  if (ntiles == 0) return;
-  if (flag_value(err) != 0) return;
 
-  if (threadIdx.x == 0) {
-    for (int s = 0; s < kStages; ++s) {
-      mbar_init(&bar->full[s], 1);
-      mbar_init(&bar->empty[s], 1);
+  if (warp == 0) {
+    if (lane == 0) {
+      for (int s = 0; s < S; ++s) {
+        mbar_init(&bar->full[s], 1);
+        mbar_init(&bar->empty[s], 1);
+      }
+      for (int p = 0; p < 8; ++p) {
+        mbar_init(&bar->d_full[p], 1);
+        mbar_init(&bar->d_empty[p], 4);
+      }
+      for (int u = 0; u < kBSlots; ++u) {
+        mbar_init(&bar->b_full[u], 2);
+        mbar_init(&bar->b_empty[u], 1);  // the MMAs of the sequence's last tile
+      }
+      for (int u = 0; u < kWSlots; ++u) {
+        mbar_init(&bar->w_full[u], 2);
+        mbar_init(&bar->w_empty[u], 8);  // every epilogue warp, once per sequence
+      }
+      mbar_init(&bar->drain, 1);
+      fence_mbar_init();
+      tma_prefetch_desc(&tm_keys);
     }
-    for (int p = 0; p < kDBufs; ++p) {
-      mbar_init(&bar->d_full[p], 1);
-      mbar_init(&bar->d_empty[p], 4);
+    int64_t b0;
+    int j0, count;
+    locate_range(pos, batch, m, cap, b0, j0, count);
+    if (lane == 0) {
+      bar->b0 = b0;
+      bar->j0 = j0;
+      bar->count = count;
     }
-    mbar_init(&bar->drain, 1);
-    fence_mbar_init();
-    // the key tiles do not depend on the query: start streaming at once
-    for (int j = 0; j < ntiles && j < kStages; ++j) {
-      mbar_arrive_expect_tx(&bar->full[j], kTileBytes);
-      tma_load_3d(sRaw + j * kTileBytes, &tm_keys, &bar->full[j], 0,
-                  (int)(c0 + (int64_t)j * kKeys), (int)b);
-    }
-  }
-  if (warp == 1) {
-    tmem_alloc(&bar->tmem_base, C::TMEM_COLS);
+  } else if (warp == 1) {
+    tmem_alloc(&bar->tmem_base, 512);
     tmem_relinquish();
   }
-  // B operand: per head a power-of-two scale and the hi / lo E4M3 split
-  constexpr int kWarps = kThreads / 32, kHPW = (H + kWarps - 1) / kWarps;
-  uint2 qraw[kHPW];
-#pragma unroll
-  for (int i = 0; i < kHPW; ++i) {  // all of this warp's loads in flight at once
-    const int h = warp + i * kWarps;
-    if (h < H) qraw[i] = *reinterpret_cast<const uint2*>(q_i + (b * H + h) * kCI + lane * 4);
-  }
-#pragma unroll
-  for (int i = 0; i < kHPW; ++i) {
-    const int h = warp + i * kWarps;
-    if (h >= H) break;
-    float v[4];
-    {
-      const uint2 raw = qraw[i];
-      v[0] = __uint_as_float(raw.x << 16);
-      v[1] = __uint_as_float(raw.x & 0xffff0000u);
-      v[2] = __uint_as_float(raw.y << 16);
-      v[3] = __uint_as_float(raw.y & 0xffff0000u);
-    }
-    float amax = fmaxf(fmaxf(fabsf(v[0]), fabsf(v[1])), fmaxf(fabsf(v[2]), fabsf(v[3])));
-#pragma unroll
-    for (int off = 16; off > 0; off >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, off));
-    float sc = 1.f;
-    if (amax > 0.f) {  // smallest power of two >= amax / 448
-      const uint32_t u = __float_as_uint(amax / 448.f);
-      sc = (u & 0x007fffffu) == 0 ? __uint_as_float(u) : __uint_as_float((u & 0x7f800000u) + 0x00800000u);
-    }
-    uint32_t hi4 = 0, lo4 = 0;
-#pragma unroll
-    for (int e = 0; e < 4; ++e) {
-      const float x = v[e] / sc;  // exact: sc is a power of two
-      const uint8_t hc = e4m3_code(x);
-      const uint8_t lc = e4m3_code(x - e4m3_value(hc));
-      hi4 |= (uint32_t)hc << (8 * e);
-      lo4 |= (uint32_t)lc << (8 * e);
-    }
-    const int d = lane * 4, ch = d >> 4;
-    const int rh = h, rl = H + h;
-    *reinterpret_cast<uint32_t*>(sB + rh * 128 + ((ch ^ (rh & 7)) * 16) + (d & 15)) = hi4;
-    *reinterpret_cast<uint32_t*>(sB + rl * 128 + ((ch ^ (rl & 7)) * 16) + (d & 15)) = lo4;
-    if (lane == 0) sW[h] = w_i[b * H + h] * sc;
-  }
-  fence_proxy_async();
+  // everything above is set-up; the cache (the emitted key) is written by the
+  // previous kernel
+  pdl_wait();
+  pdl_trigger();
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = bar->tmem_base;
+  const int count = bar->count;
+  const int64_t b0 = bar->b0;
+  const int j0 = bar->j0;
+  const bool live = count > 0 && flag_value(err) == 0;
 
-  if (warp == 0) {
+  if (warp == 0 && live) {
     // ------------------------------- TMA producer --------------------------------
-    int issued[kStages];
-#pragma unroll
-    for (int s = 0; s < kStages; ++s) issued[s] = s < ntiles ? 1 : 0;  // prefetched above
-    for (int j = kStages; j < ntiles; ++j) {
-      const int s = j % kStages, u = j / kStages;
-      if (!mbar_wait(&bar->empty[s], (uint32_t)((u - 1) & 1), err)) break;
+    TileWalk it;
+    it.start(pos, b0, j0, m, cap);
+    int i = 0;
+    for (; i < count; ++i, it.next(pos, batch, m, cap)) {
+      const int s = i % S;
+      if (i >= S && !mbar_wait(&bar->empty[s], (uint32_t)(((i / S) - 1) & 1), err)) break;
       if (lane == 0) {
         mbar_arrive_expect_tx(&bar->full[s], kTileBytes);
-        tma_load_3d(sRaw + s * kTileBytes, &tm_keys, &bar->full[s], 0,
-                    (int)(c0 + (int64_t)j * kKeys), (int)b);
+        tma_load_3d(sRaw + s * kTileBytes, &tm_keys, &bar->full[s], 0, it.j * kKeys, (int)it.b);
       }
       __syncwarp();
-      ++issued[s];
     }
-    for (int s = 0; s < kStages; ++s)
-      if (issued[s] > 0) mbar_wait(&bar->full[s], (uint32_t)((issued[s] - 1) & 1), err, false);
-  } else if (warp == 1) {
+    // every issued tile has landed before the CTA exits
+    for (int r = (i > S ? i - S : 0); r < i; ++r)
+      mbar_wait(&bar->full[r % S], (uint32_t)((r / S) & 1), err, false);
+  } else if (warp == 1 && live) {
     // ------------------------------- MMA issuer ----------------------------------
-    constexpr uint32_t kIdesc = idesc_e4m3(kKeys, C::N);
-    const uint32_t a0 = smem_u32(sRaw), b0 = smem_u32(sB);
-    for (int j = 0; j < ntiles; ++j) {
-      const int s = j % kStages, u = j / kStages, p = j % C::DBUFS, v = j / C::DBUFS;
-      if (!mbar_wait(&bar->full[s], (uint32_t)(u & 1), err)) break;
-      if (v >= 1 && !mbar_wait(&bar->d_empty[p], (uint32_t)((v - 1) & 1), err)) break;
+    constexpr uint32_t kIdesc = idesc_e4m3(kKeys, H);
+    const uint32_t a0 = smem_u32(sRaw), bb0 = smem_u32(sB);
+    TileWalk it;
+    it.start(pos, b0, j0, m, cap);
+    int u = -1;  // sequence counter within the range
+    for (int i = 0; i < count; ++i, it.next(pos, batch, m, cap)) {
+      const int s = i % S, p = i % DB;
+      if (i == 0 || it.j == 0) {
+        ++u;
+        if (!mbar_wait(&bar->b_full[u & 1], (uint32_t)((u >> 1) & 1), err)) break;
+      }
+      if (!mbar_wait(&bar->full[s], (uint32_t)((i / S) & 1), err)) break;
+      if (i >= DB && !mbar_wait(&bar->d_empty[p], (uint32_t)(((i / DB) - 1) & 1), err)) break;
       tc_fence_after();
       if (lane == 0) {
+        const uint32_t bslot = bb0 + (u & 1) * C::B_BYTES;
 #pragma unroll
-        for (int kk = 0; kk < kCI / 32; ++kk)  // K = 32 bytes per instruction
-          mma_f8(tmem + p * C::N, desc_sw128(a0 + s * kTileBytes + kk * 32),
-                 desc_sw128(b0 + kk * 32), kIdesc, kk > 0 ? 1u : 0u);
+        for (int kk = 0; kk < kCI / 32; ++kk) {  // K = 32 bytes per instruction
+          const uint64_t a = desc_sw128(a0 + s * kTileBytes + kk * 32);
+          // hi rows 0..H-1, then lo rows H..2H-1 into the same columns
+          mma_f8(tmem + p * H, a, desc_sw128(bslot + kk * 32), kIdesc, kk > 0 ? 1u : 0u);
+          mma_f8(tmem + p * H, a, desc_sw128(bslot + H * 128 + kk * 32), kIdesc, 1u);
+        }
         mma_commit(&bar->d_full[p]);
         mma_commit(&bar->empty[s]);
+        if (i + 1 == count || it.j + 1 == it.nt) mma_commit(&bar->b_empty[u & 1]);
       }
       __syncwarp();
     }
     if (lane == 0) mma_commit(&bar->drain);
     __syncwarp();
     mbar_wait(&bar->drain, 0, err, false);
-  } else if (warp >= 4) {
-    // ----------- epilogue: hi + lo, ReLU, head weights, key scale ----------------
-    // two groups of four warps take alternate tiles, each warp 32 key rows x
-    // all heads
+  } else if ((warp == 2 || warp == 3) && live) {
+    // ------------- query operand: per head a power of two and hi / lo E4M3 -------------
+    // 64 threads, a half-warp per head, 8 dims per thread, 4 heads per pass
+    const int tid2 = threadIdx.x - 64;
+    const int hl = tid2 & 15, hsub = tid2 >> 4;
+    constexpr int kPass = H / 4;
+    TileWalk it;
+    it.start(pos, b0, j0, m, cap);
+    int left = count;
+    for (int u = 0; left > 0; ++u) {
+      const int64_t b = it.b;
+      const int here = min(left, it.nt - it.j);
+      const int slot = u & 1, ws = u % kWSlots;
+      // the B slot once the MMAs of sequence u-2 are done; the weight slot once
+      // the epilogue is past sequence u-16
+      if (u >= kBSlots && !mbar_wait(&bar->b_empty[slot], (uint32_t)(((u >> 1) - 1) & 1), err))
+        break;
+      if (u >= kWSlots &&
+          !mbar_wait(&bar->w_empty[ws], (uint32_t)(((u / kWSlots) - 1) & 1), err))
+        break;
+      uint8_t* dstB = sB + slot * C::B_BYTES;
+      float* dstW = sW + ws * H;
+      constexpr int kBatch = kPass < 16 ? kPass : 16;  // loads in flight per thread
+#pragma unroll 1
+      for (int p0 = 0; p0 < kPass; p0 += kBatch) {
+        uint4 raw[kBatch];
+        float wv[kBatch];
+#pragma unroll
+        for (int q = 0; q < kBatch; ++q) {
+          const int h = (p0 + q) * 4 + hsub;
+          raw[q] = *reinterpret_cast<const uint4*>(q_i + (b * H + h) * kCI + hl * 8);
+          wv[q] = hl == 0 ? w_i[b * H + h] : 0.f;
+        }
+#pragma unroll
+        for (int q = 0; q < kBatch; ++q) {
+          const int h = (p0 + q) * 4 + hsub;
+          const uint32_t wd[4] = {raw[q].x, raw[q].y, raw[q].z, raw[q].w};
+          float v[8];
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            v[2 * e] = __uint_as_float(wd[e] << 16);
+            v[2 * e + 1] = __uint_as_float(wd[e] & 0xffff0000u);
+          }
+          float amax = 0.f;
+#pragma unroll
+          for (int e = 0; e < 8; ++e) amax = fmaxf(amax, fabsf(v[e]));
+#pragma unroll
+          for (int off = 8; off > 0; off >>= 1)
+            amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, off));
+          float sc = 1.f;
+          if (amax > 0.f) {  // smallest power of two >= amax / 448
+            const uint32_t ub = __float_as_uint(amax / 448.f);
+            sc = (ub & 0x007fffffu) == 0 ? __uint_as_float(ub)
+                                         : __uint_as_float((ub & 0x7f800000u) + 0x00800000u);
+          }
+          uint32_t hi2[2] = {0u, 0u}, lo2[2] = {0u, 0u};
+#pragma unroll
+          for (int e = 0; e < 8; ++e) {
+            const float x = v[e] / sc;  // exact: sc is a power of two
+            const uint8_t hc = e4m3_code(x);
+            const uint8_t lc = e4m3_code(x - e4m3_value(hc));
+            hi2[e >> 2] |= (uint32_t)hc << (8 * (e & 3));
+            lo2[e >> 2] |= (uint32_t)lc << (8 * (e & 3));
+          }
+          const int d = hl * 8, ch = d >> 4;
+          const int rh = h, rl = H + h;
+          *reinterpret_cast<uint2*>(dstB + rh * 128 + ((ch ^ (rh & 7)) * 16) + (d & 15)) =
+              make_uint2(hi2[0], hi2[1]);
+          *reinterpret_cast<uint2*>(dstB + rl * 128 + ((ch ^ (rl & 7)) * 16) + (d & 15)) =
+              make_uint2(lo2[0], lo2[1]);
+          if (hl == 0) dstW[h] = wv[q] * sc;
+        }
+      }
+      fence_proxy_async();  // generic-proxy writes before the tensor core reads them
+      __syncwarp();
+      if (lane == 0) {
+        mbar_arrive(&bar->b_full[slot]);
+        mbar_arrive(&bar->w_full[ws]);
+      }
+      left -= here;
+      for (int r = 0; r < here; ++r) it.next(pos, batch, m, cap);
+    }
+  } else if (warp >= 4 && live) {
+    // ------- epilogue: ReLU, head weights, key scale (group g: tiles i % 2 == g) -------
     const int quad = warp & 3, grp = (warp - 4) >> 2;
     const int row = quad * 32 + lane;
     const uint32_t lane_addr = tmem + ((uint32_t)(quad * 32) << 16);
-    uint32_t kmax = 0u, kmin = 0xffffffffu;  // order keys of this thread's scores
-    // the key scales do not depend on the MMA: all of this thread's loads go
-    // out at once, so one DRAM latency is paid instead of one per tile
-    constexpr int kMine = kChunk / kKeys / 2;
-    float kscale[kMine];
-#pragma unroll
-    for (int i = 0; i < kMine; ++i) {
-      const int64_t s = c0 + (int64_t)(grp + 2 * i) * kKeys + row;
-      kscale[i] = s < V ? __ldcs(key_scale + b * cap + s) : 0.f;
-    }
-#pragma unroll 1
-    for (int i = 0; i < kMine; ++i) {
-      const int j = grp + 2 * i;
-      if (j >= ntiles) break;
-      const int p = j % C::DBUFS, v = j / C::DBUFS;
-      const int64_t s = c0 + (int64_t)j * kKeys + row;
-      const float ks = kscale[0];  // shift the queue (registers, not a local array)
-#pragma unroll
-      for (int q = 0; q + 1 < kMine; ++q) kscale[q] = kscale[q + 1];
-      if (!mbar_wait(&bar->d_full[p], (uint32_t)(v & 1), err)) break;
-      tc_fence_after();
-      float acc = 0.f;
-#pragma unroll
-      for (int c = 0; c < H / 32; ++c) {
-        uint32_t hi[32], lo[32];
-        tmem_ld32(lane_addr + p * C::N + c * 32, hi);
-        tmem_ld32(lane_addr + p * C::N + H + c * 32, lo);
-        tmem_ld_wait();
-#pragma unroll
-        for (int i = 0; i < 32; ++i)
-          acc = fmaf(sW[c * 32 + i],
-                     fmaxf(__uint_as_float(hi[i]) + __uint_as_float(lo[i]), 0.f), acc);
+    TileWalk it;
+    it.start(pos, b0, j0, m, cap);
+    int64_t V = 0;
+    // key scale of this group's next tile, loaded a tile ahead
+    auto scale_of = [&](const TileWalk& w) -> float {
+      const int64_t sidx = (int64_t)w.j * kKeys + row;
+      const int64_t Vw = min((pos[w.b] + 1) / m, cap);
+      return sidx < Vw ? __ldcs(key_scale + w.b * cap + sidx) : 0.f;
+    };
+    TileWalk ahead = it;
+    if (grp == 1 && count > 1) ahead.next(pos, batch, m, cap);
+    float ks_next = grp < count ? scale_of(ahead) : 0.f;
+    int u = -1;
+    for (int i = 0; i < count; ++i, it.next(pos, batch, m, cap)) {
+      if (i == 0 || it.j == 0) {
+        ++u;
+        V = min((pos[it.b] + 1) / m, cap);
       }
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&bar->d_empty[p]);
-      if (s < V) {
-        const float sc = acc * ks;
-        scores[b * cap + s] = sc;
-        const uint32_t ky = order_key(sc);
-        kmax = max(kmax, ky);
-        kmin = min(kmin, ky);
-      }
-    }
-    // the sequence's score range, for the selection kernel
+      const bool mine = (i & 1) == grp;
+      const bool seq_end = i + 1 == count || it.j + 1 == it.nt;
+      if (mine) {
+        const float ks = ks_next;
+        if (i + 2 < count) {
+          ahead.next(pos, batch, m, cap);
+          ahead.next(pos, batch, m, cap);
+          ks_next = scale_of(ahead);
+        }
+        const int p = i % DB;
+        // the head weights of this sequence are in place
+        if (!mbar_wait(&bar->w_full[u % kWSlots], (uint32_t)((u / kWSlots) & 1), err)) break;
+        const float* w = sW + (u % kWSlots) * H;
+        if (!mbar_wait(&bar->d_full[p], (uint32_t)((i / DB) & 1), err)) break;
+        tc_fence_after();
+        float acc[8];
 #pragma unroll
-    for (int off = 16; off > 0; off >>= 1) {
-      kmax = max(kmax, __shfl_xor_sync(0xffffffffu, kmax, off));
-      kmin = min(kmin, __shfl_xor_sync(0xffffffffu, kmin, off));
-    }
-    if (lane == 0) {
-      atomicMax(&range[b * 2 + 0], kmax);
-      atomicMin(&range[b * 2 + 1], kmin);
+        for (int e = 0; e < 8; ++e) acc[e] = 0.f;
+#pragma unroll
+        for (int c = 0; c < H / 32; ++c) {
+          uint32_t d[32];
+          tmem_ld32(lane_addr + p * H + c * 32, d);
+          tmem_ld_wait();
+#pragma unroll
+          for (int e = 0; e < 32; e += 4) {
+            const float4 w4 = *reinterpret_cast<const float4*>(w + c * 32 + e);
+            acc[(e >> 2) & 7] = fmaf(w4.x, fmaxf(__uint_as_float(d[e]), 0.f), acc[(e >> 2) & 7]);
+            acc[(e >> 2) & 7] = fmaf(w4.y, fmaxf(__uint_as_float(d[e + 1]), 0.f), acc[(e >> 2) & 7]);
+            acc[(e >> 2) & 7] = fmaf(w4.z, fmaxf(__uint_as_float(d[e + 2]), 0.f), acc[(e >> 2) & 7]);
+            acc[(e >> 2) & 7] = fmaf(w4.w, fmaxf(__uint_as_float(d[e + 3]), 0.f), acc[(e >> 2) & 7]);
+          }
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bar->d_empty[p]);
+        const float sum = ((acc[0] + acc[1]) + (acc[2] + acc[3])) + ((acc[4] + acc[5]) + (acc[6] + acc[7]));
+        const int64_t sidx = (int64_t)it.j * kKeys + row;
+        if (sidx < V) scores[it.b * cap + sidx] = sum * ks;
+      }
+      if (seq_end) {  // both groups release the sequence's weights once they pass its end
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bar->w_empty[u % kWSlots]);
+      }
     }
   }
   __syncwarp();
@@ -260,14 +403,14 @@ __global__ void __launch_bounds__(kThreads, 1) decode_index_tc_kernel(
   __syncthreads();
   if (warp == 1) {
     tc_fence_after();
-    tmem_dealloc(tmem, C::TMEM_COLS);
+    tmem_dealloc(tmem, 512);
   }
 }
 
 template <int H>
 cudaError_t launch_h(const csa_cache_desc& d, const CacheView& cv, const int64_t* pos,
-                     const void* q_i, const float* w_i, float* scores, unsigned int* range,
-                     unsigned int* err, cudaStream_t s) {
+                     const void* q_i, const float* w_i, float* scores, unsigned int* err,
+                     cudaStream_t s) {
   using C = DecIdxCfg<H>;
   CUtensorMap tk;
   if (!make_tmap_3d(&tk, cv.ikey_fp8, 1, kCI, (uint64_t)d.capacity, (uint64_t)d.batch, kCI,
@@ -276,10 +419,11 @@ cudaError_t launch_h(const csa_cache_desc& d, const CacheView& cv, const int64_t
   auto kern = decode_index_tc_kernel<H>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
   if (e != cudaSuccess) return e;
-  dim3 grid((unsigned)((d.capacity + kChunk - 1) / kChunk), (unsigned)d.batch);
-  kern<<<grid, kThreads, C::SMEM, s>>>(tk, cv.ikey_scale, (const __nv_bfloat16*)q_i, w_i, pos,
-                                       d.capacity, d.m, scores, range, err);
-  return cudaGetLastError();
+  const int64_t max_tiles = d.batch * ((d.capacity + kKeys - 1) / kKeys);
+  const unsigned grid = (unsigned)std::max<int64_t>(1, std::min<int64_t>(sm_count(), max_tiles));
+  return launch_pdl(kern, dim3(grid), dim3(kThreads), (size_t)C::SMEM, s, tk,
+                    (const float*)cv.ikey_scale, (const __nv_bfloat16*)q_i, w_i, pos,
+                    (int64_t)d.batch, (int64_t)d.capacity, d.m, scores, err);
 }
 
 }  // namespace
@@ -290,11 +434,10 @@ bool decode_index_tc_supported(const csa_cache_desc& d) {
 
 cudaError_t launch_decode_index_tc(const csa_cache_desc& d, const CacheView& cv,
                                    const int64_t* pos, const void* q_i, const float* w_i,
-                                   float* scores, unsigned int* range, unsigned int* err,
-                                   cudaStream_t s) {
+                                   float* scores, unsigned int* err, cudaStream_t s) {
   switch (d.nh_i) {
-    case 64: return launch_h<64>(d, cv, pos, q_i, w_i, scores, range, err, s);
-    case 128: return launch_h<128>(d, cv, pos, q_i, w_i, scores, range, err, s);
+    case 64: return launch_h<64>(d, cv, pos, q_i, w_i, scores, err, s);
+    case 128: return launch_h<128>(d, cv, pos, q_i, w_i, scores, err, s);
     default: return cudaErrorInvalidValue;
   }
 }

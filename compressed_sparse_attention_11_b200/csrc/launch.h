@@ -6,9 +6,34 @@
 #include <cuda_bf16.h>
 #include <stdint.h>
 
+#include <algorithm>
+#include <utility>
+
 #include "../../include/csa.h"
 
 namespace csa {
+
+// Launches `kern` with programmatic stream serialization: its CTAs may be
+// scheduled while the previous kernel on `s` drains; the kernel itself
+// waits (griddepcontrol.wait) before touching anything that kernel writes.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                       cudaStream_t s, Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...);
+}
+
+// Number of SMs of the current device (cached per device).
+int sm_count();
 
 // Records a one-line reason for `st` (read back by csa_last_error) and returns st.
 csa_status set_last_error(csa_status st, const char* fmt, ...);
@@ -31,15 +56,20 @@ cudaError_t launch_attn_tc(const void* q, const void* kv_comp, const int32_t* id
                            int64_t batch, int64_t n, int m, void* out, unsigned int* err,
                            cudaStream_t s);
 
-// tcgen05 decode indexer over FP8 keys (c_i = 128, nh_i in {16, 32, 64, 128}).
+// tcgen05 decode indexer over FP8 keys (c_i = 128, nh_i in {64, 128}), persistent.
 struct CacheView;
 bool decode_index_tc_supported(const csa_cache_desc& d);
-// scores [batch][capacity] fp32; range [batch][2] receives the largest and
-// smallest order key of each sequence's scores (0 / ~0 on entry).
+// scores [batch][capacity] fp32, written for s < V of each sequence.
 cudaError_t launch_decode_index_tc(const csa_cache_desc& d, const CacheView& cv,
                                    const int64_t* pos, const void* q_i, const float* w_i,
-                                   float* scores, unsigned int* range, unsigned int* err,
-                                   cudaStream_t s);
+                                   float* scores, unsigned int* err, cudaStream_t s);
+
+// Exact top-k over the indexer's scores, one thread-block cluster per
+// sequence with the scores staged in shared memory.  sel [batch][k]: the
+// chosen entry indices ascending, -1 padded when V <= k.
+bool decode_topk_supported(const csa_cache_desc& d);
+cudaError_t launch_decode_topk(const csa_cache_desc& d, const int64_t* pos, const float* scores,
+                               int32_t* sel, cudaStream_t s);
 
 // tcgen05 decode attention (64 heads x 512, FP8/bf16 cache): one 128-entry
 // tile per CTA (ntile = decode_attn_splits), merged by a combine kernel.

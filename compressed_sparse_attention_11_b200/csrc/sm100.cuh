@@ -78,6 +78,19 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, unsign
   return true;
 }
 
+// ---- programmatic dependent launch -------------------------------------------
+// A kernel launched with programmatic stream serialization may start while
+// the previous kernel in the stream is still running.  pdl_wait() blocks until
+// that kernel has completed and its writes are visible; every kernel here
+// reads and writes global memory only after it, and calls pdl_trigger()
+// (allowing the next kernel to be scheduled) only after it, so at most two
+// neighbouring kernels overlap and only in their set-up.  Without the launch
+// attribute both are no-ops.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 // ---- TMA ---------------------------------------------------------------------
 __device__ __forceinline__ void tma_prefetch_desc(const CUtensorMap* map) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");

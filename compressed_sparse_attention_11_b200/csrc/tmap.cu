@@ -1,7 +1,8 @@
-// Host-side TMA tensor-map encoding through the driver entry point (no
-// link-time dependency on libcuda).
+// Host-side helpers: TMA tensor-map encoding through the driver entry point
+// (no link-time dependency on libcuda) and the device's SM count.
 #include <mutex>
 
+#include "launch.h"
 #include "sm100.cuh"
 
 namespace csa {
@@ -40,6 +41,19 @@ bool make_tmap_3d(CUtensorMap* map, const void* base, int elem_bytes, uint64_t x
                         CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                         CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
+}
+
+int sm_count() {
+  constexpr int kMaxDev = 64;
+  static int counts[kMaxDev] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDev) dev = 0;
+  if (counts[dev] <= 0) {
+    int count = 0;
+    cudaDeviceGetAttribute(&count, cudaDevAttrMultiProcessorCount, dev);
+    counts[dev] = count > 0 ? count : 148;
+  }
+  return counts[dev];
 }
 
 }  // namespace csa

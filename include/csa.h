@@ -219,6 +219,10 @@ typedef struct {
   const float *iba, *ibb; /* [m][c_i] index-key compressor biases (CSA)      */
   const float* sink;      /* [nh] sink logits, or NULL                       */
   float scale;            /* logit scale                                     */
+  int32_t* sel_out;       /* CSA, optional: [batch][k] int32 device array that
+                           * receives each sequence's selected entry indices
+                           * (ascending, -1 padded when V <= k); NULL keeps
+                           * them in the workspace.  Ignored for HCA.        */
 } csa_decode_params;
 
 /* Offsets and total size of a cache for `desc`. Host-only, no launch. */

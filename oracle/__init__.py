@@ -338,10 +338,11 @@ def e4m3_encode(x) -> np.ndarray:
     return out
 
 
+_E4M3_ALL = np.array([e4m3_value(c) for c in range(256)])  # value of every byte
+
+
 def e4m3_decode(codes) -> np.ndarray:
-    codes = np.asarray(codes, dtype=np.uint8)
-    table = np.array([e4m3_value(c) for c in range(256)])
-    return table[codes]
+    return _E4M3_ALL[np.asarray(codes, dtype=np.uint8)]
 
 
 def bf16_round(x) -> np.ndarray:
@@ -378,6 +379,30 @@ def quantize_entry(x, rope_dims: int):
 def dequantize_entry(codes, scale, rope) -> np.ndarray:
     """x_hat = code value * scale (fp64) followed by the bf16 rope dims."""
     return np.concatenate([e4m3_decode(codes) * float(scale), f64(rope)])
+
+
+def quantize_entries(X, rope_dims: int, rows_per_pass: int = 4096):
+    """quantize_entry of every row of X [E, c], the rows taken a block at a time.
+
+    Returns (codes [E, c-rope] uint8, scales [E] float32, rope [E, rope] float64):
+    the same fp32 arithmetic per row as quantize_entry.
+    """
+    x32 = np.asarray(X, dtype=np.float32)
+    E, c = x32.shape
+    codes = np.zeros((E, c - rope_dims), dtype=np.uint8)
+    scales = np.ones(E, dtype=np.float32)
+    for r0 in range(0, E, rows_per_pass):
+        body = x32[r0:r0 + rows_per_pass, :c - rope_dims]
+        amax = np.abs(body).max(axis=1) if body.shape[1] else np.zeros(body.shape[0], np.float32)
+        sc = np.where(amax > 0, amax / np.float32(E4M3_MAX), np.float32(1.0)).astype(np.float32)
+        scales[r0:r0 + rows_per_pass] = sc
+        codes[r0:r0 + rows_per_pass] = e4m3_encode((body / sc[:, None]).astype(np.float32))
+    return codes, scales, bf16_round(x32[:, c - rope_dims:])
+
+
+def dequantize_entries(codes, scales, rope) -> np.ndarray:
+    """dequantize_entry of every row: [E, c] fp64."""
+    return np.concatenate([e4m3_decode(codes) * f64(scales)[:, None], f64(rope)], axis=1)
 
 
 # ---------------------------------------------------------------------------

@@ -9,7 +9,7 @@ import torch
 import compressed_sparse_attention_11_b200 as csa
 import csa_inputs as G
 import oracle as O
-from _util import check_close, host
+from _util import check_close, check_topk_row, host
 
 pytestmark = pytest.mark.gpu
 
@@ -54,10 +54,13 @@ def test_store_entries_bit_exact(dt):
             assert got["iscale"][b, 2 + e].item() == iscale
 
 
-def _setup(w, B, E, steps, seed):
-    """Cache with E stored entries and raw rows up to position t0-1 (t0 = m*E)."""
+def _setup(w, B, E, steps, seed, edit=None):
+    """Cache with E stored entries and raw rows up to position t0-1 (t0 = m*E).
+    ``edit(inp)`` may change the host inputs in place before anything uses them."""
     t0 = w.m * E
     inp = G.decode_inputs(w, entries=E, batch=B, t=t0, steps=steps, seed=seed)
+    if edit is not None:
+        edit(inp)
     first = int(inp["first_pos"])
     cap = E + steps // w.m + 2
     cache = csa.CsaCache(B, cap, w.c, w.rope_dims, w.m, w.window, w.nh, w.is_hca, c_i=w.c_i,
@@ -88,8 +91,8 @@ def _biases(inp, w):
     return {k: inp[k] for k in keys}
 
 
-def _run_and_compare(w, B, E, steps, seed, check_seqs=None):
-    inp, cache, t0, first, tail, names = _setup(w, B, E, steps, seed)
+def _run_and_compare(w, B, E, steps, seed, check_seqs=None, edit=None, sel_exact=False):
+    inp, cache, t0, first, tail, names = _setup(w, B, E, steps, seed, edit)
     biases = _biases(inp, w)
     dbias = {k: v.to(DEV) for k, v in biases.items()}
     sink = inp["sink"].to(DEV)
@@ -103,14 +106,25 @@ def _run_and_compare(w, B, E, steps, seed, check_seqs=None):
         q = inp["q"][s].to(DEV)
         qi = None if w.is_hca else inp["q_i"][s].to(DEV)
         wi = None if w.is_hca else inp["w_i"][s].to(DEV)
-        out = host(cache.decode_step(pos, rows, dbias, sink, w.scale, q, qi, wi))
+        sel = None if w.is_hca else torch.empty((B, w.k), dtype=torch.int32, device=DEV)
+        out = host(cache.decode_step(pos, rows, dbias, sink, w.scale, q, qi, wi, sel_out=sel))
         csa.csa_check()
         for b in check_seqs:
-            ref, _ = seqs[b].step(t, {nm: inp["rows_" + nm][b, r] for nm in names}, biases,
-                                  inp["q"][s, b], None if w.is_hca else inp["q_i"][s, b],
-                                  None if w.is_hca else inp["w_i"][s, b], inp["sink"], w.scale,
-                                  w.k)
+            ref, ref_sel = seqs[b].step(t, {nm: inp["rows_" + nm][b, r] for nm in names}, biases,
+                                        inp["q"][s, b], None if w.is_hca else inp["q_i"][s, b],
+                                        None if w.is_hca else inp["w_i"][s, b], inp["sink"],
+                                        w.scale, w.k)
             check_close(out[b], ref, torch.bfloat16, f"step t={t} b={b}")
+            if w.is_hca:
+                continue
+            if sel_exact:
+                assert np.array_equal(host(sel)[b].numpy(), np.asarray(ref_sel, dtype=np.int32)), \
+                    f"selection t={t} b={b}"
+            else:  # exact wherever the k-th gap exceeds the tolerance, else a valid top-k
+                V = min(O.visible(t, w.m), len(seqs[b].ikeys))
+                K = np.stack([O.dequantize_entry(*e) for e in seqs[b].ikeys[:V]])
+                scores = O.index_scores_row(inp["q_i"][s, b], inp["w_i"][s, b], K, V)
+                check_topk_row(host(sel)[b].numpy(), scores, w.k, f"selection t={t} b={b}")
     # emitted entries agree with the oracle's from-scratch compression
     got = {k: host(v) for k, v in cache.entries().items()}
     n_emit = (t0 + steps) // w.m - E
@@ -164,6 +178,45 @@ def test_decode_csa_many_sequences_one_split():
     w = G.Decode("csa_decode_many", 80, 0, 512, 64, 4, 64, 128, False, nh_i=64, c_i=128, k=64,
                  seed=105)
     _run_and_compare(w, B=80, E=40, steps=5, seed=12, check_seqs=[0, 37, 79])
+
+
+def _csa_dims(name, seed, k=512):
+    return G.Decode(name, 2, 0, 512, 64, 4, 64, 128, False, nh_i=64, c_i=128, k=k, seed=seed)
+
+
+def test_decode_csa_topk_cluster_of_four():
+    """~36000 visible entries: the top-k runs as a 4-CTA cluster per sequence."""
+    _run_and_compare(_csa_dims("csa_decode_cluster", 106), B=2, E=36000, steps=2, seed=13)
+
+
+def test_decode_csa_all_scores_tied():
+    """q_i = 0 makes every score 0: the selection is entries 0..k-1 (ties go to
+    the smaller index), across a 2-CTA cluster."""
+    def edit(inp):
+        inp["q_i"].zero_()
+    _run_and_compare(_csa_dims("csa_decode_ties", 107), B=2, E=20000, steps=2, seed=14, edit=edit,
+                     sel_exact=True)
+
+
+def test_decode_csa_topk_integer_scores_with_ties():
+    """Scores in {0, 1, 2, 3}, computed exactly on both sides: one index-key dim
+    holds the integer, one dim holds 448 (entry scale exactly 1), and one
+    query head reads the integer dim with weight 1.  The k-th largest score
+    sits inside a large tied group that spans the cluster's CTAs, so the
+    selection is fixed by the smaller-index rule alone."""
+    def edit(inp):
+        B, E, ci = inp["cache_ikey"].shape
+        gen = torch.Generator().manual_seed(15)
+        ik = torch.zeros(B, E, ci)
+        ik[:, :, 0] = torch.randint(0, 4, (B, E), generator=gen).float()
+        ik[:, :, ci - 1] = 448.0
+        inp["cache_ikey"].copy_(ik)
+        inp["q_i"].zero_()
+        inp["q_i"][:, :, 0, 0] = 1.0
+        inp["w_i"].fill_(0.5)
+        inp["w_i"][:, :, 0] = 1.0
+    _run_and_compare(_csa_dims("csa_decode_int", 108), B=2, E=20000, steps=2, seed=15, edit=edit,
+                     sel_exact=True)
 
 
 def test_write_rows_fills_ring_and_state():

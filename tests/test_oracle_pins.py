@@ -437,6 +437,21 @@ def test_quantize_entry_properties():
     assert zs == 1.0 and np.all(zc == 0)
 
 
+def test_quantize_entries_equals_row_by_row():
+    """The block form used at full workload sizes gives the per-entry results
+    bit for bit (blocks smaller than the row count, a zero row, a huge value)."""
+    r = np.random.default_rng(11)
+    X = r.standard_normal((37, 40)).astype(np.float32)
+    X[5] = 0.0
+    X[9, 3] = 1e5
+    codes, scales, rope = O.quantize_entries(X, 8, rows_per_pass=10)
+    deq = O.dequantize_entries(codes, scales, rope)
+    for e in range(X.shape[0]):
+        c1, s1, r1 = O.quantize_entry(X[e], 8)
+        assert np.array_equal(codes[e], c1) and scales[e] == s1 and np.array_equal(rope[e], r1)
+        assert np.array_equal(deq[e], O.dequantize_entry(c1, s1, r1))
+
+
 # ----------------------------------------------------------------- decode ---
 
 def test_decode_sequence_matches_prefill_pipeline():
