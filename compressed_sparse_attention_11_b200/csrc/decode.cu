@@ -295,14 +295,80 @@ __device__ void append_rows(const csa_cache_desc& d, const CacheView& cv, const 
   }
 }
 
+// The tensor-core indexer's query operand of one sequence (H heads of
+// dim 128): per head a power of two s_h >= max|q_h|/448 and the E4M3 pair
+// hi = E4M3(q/s_h), lo = E4M3(q/s_h - hi), written as the MMA's B operand
+// image (2H rows of 128 bytes with the 128-byte swizzle: hi rows 0..H-1, lo
+// rows H..2H-1), followed by the H weights w_h * s_h.  s_h (hi + lo) equals
+// the bf16 query except for elements below 2^-2 s_h in magnitude, whose
+// residual falls under E4M3's subnormal step (absolute error <= 2^-10 s_h).
+// A half-warp per head, eight dims per thread.
+__device__ void build_query_operand(const __nv_bfloat16* __restrict__ q,
+                                    const float* __restrict__ w, int H, uint8_t* rec) {
+  const int hw = threadIdx.x >> 4, hl = threadIdx.x & 15, nhw = blockDim.x >> 4;
+  float* wout = reinterpret_cast<float*>(rec + 2 * H * 128);
+  for (int h0 = 0; h0 < H; h0 += nhw) {  // the same trip count in every thread
+    const int h = h0 + hw;
+    const bool act = h < H;
+    const uint4 raw = act ? *reinterpret_cast<const uint4*>(q + (int64_t)h * 128 + hl * 8)
+                          : make_uint4(0, 0, 0, 0);
+    const uint32_t wd[4] = {raw.x, raw.y, raw.z, raw.w};
+    float v[8];
+    float amax = 0.f;
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      v[2 * e] = __uint_as_float(wd[e] << 16);
+      v[2 * e + 1] = __uint_as_float(wd[e] & 0xffff0000u);
+      amax = fmaxf(amax, fmaxf(fabsf(v[2 * e]), fabsf(v[2 * e + 1])));
+    }
+#pragma unroll
+    for (int off = 8; off > 0; off >>= 1)
+      amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, off));
+    float sc = 1.f;
+    if (amax > 0.f) {  // smallest power of two >= amax / 448
+      const uint32_t ub = __float_as_uint(amax / 448.f);
+      sc = (ub & 0x007fffffu) == 0 ? __uint_as_float(ub)
+                                   : __uint_as_float((ub & 0x7f800000u) + 0x00800000u);
+    }
+    const float inv = 1.f / sc;  // exact: sc is a normal power of two
+    uint32_t hi2[2] = {0u, 0u}, lo2[2] = {0u, 0u};
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const float2 x = make_float2(v[2 * e] * inv, v[2 * e + 1] * inv);  // exact scaling
+      const __nv_fp8x2_storage_t hc = __nv_cvt_float2_to_fp8x2(x, __NV_SATFINITE, __NV_E4M3);
+      const __half2_raw hr = __nv_cvt_fp8x2_to_halfraw2(hc, __NV_E4M3);
+      const float2 hv = __half22float2(*reinterpret_cast<const __half2*>(&hr));
+      const __nv_fp8x2_storage_t lc =
+          __nv_cvt_float2_to_fp8x2(make_float2(x.x - hv.x, x.y - hv.y), __NV_SATFINITE, __NV_E4M3);
+      hi2[e >> 1] |= (uint32_t)hc << (16 * (e & 1));
+      lo2[e >> 1] |= (uint32_t)lc << (16 * (e & 1));
+    }
+    if (act) {
+      const int dd = hl * 8, ch = dd >> 4;
+      const int rh = h, rl = H + h;
+      *reinterpret_cast<uint2*>(rec + rh * 128 + ((ch ^ (rh & 7)) * 16) + (dd & 15)) =
+          make_uint2(hi2[0], hi2[1]);
+      *reinterpret_cast<uint2*>(rec + rl * 128 + ((ch ^ (rl & 7)) * 16) + (dd & 15)) =
+          make_uint2(lo2[0], lo2[1]);
+      if (hl == 0) wout[h] = w[h] * sc;
+    }
+  }
+}
+
 __global__ void __launch_bounds__(1024) append_emit_kernel(csa_cache_desc d, CacheView cv,
                                                           const int64_t* __restrict__ pos,
-                                                          csa_rows rows, csa_decode_params p) {
+                                                          csa_rows rows, csa_decode_params p,
+                                                          const __nv_bfloat16* __restrict__ q_i,
+                                                          const float* __restrict__ w_i,
+                                                          uint8_t* __restrict__ qop) {
   extern __shared__ float sx[];  // [c + c_i] + 32
   const int64_t b = blockIdx.x;
   // the previous step's kernels read the window slot this token overwrites
   sm100::pdl_wait();
   sm100::pdl_trigger();
+  if (qop != nullptr)  // the indexer's query operand, for every sequence
+    build_query_operand(q_i + b * d.nh_i * 128, w_i + b * d.nh_i, d.nh_i,
+                        qop + b * decode_qop_bytes(d.nh_i));
   const int64_t t = pos[b];
   if (t < 0) return;  // no token for this sequence
   append_rows(d, cv, rows, b, t);
@@ -601,7 +667,7 @@ __global__ void __launch_bounds__(256) attn_combine_kernel(
 struct DecodeWs {
   int nchunks, nsplit;
   bool tc_index, tc_attn;
-  size_t cand_score, cand_idx, scores, sel, part_o, part_ms, total;
+  size_t cand_score, cand_idx, scores, qop, sel, part_o, part_ms, total;
 };
 
 static DecodeWs decode_ws_layout(const csa_cache_desc& d) {
@@ -617,6 +683,7 @@ static DecodeWs decode_ws_layout(const csa_cache_desc& d) {
   w.cand_score = off; off = align256(off + B * w.nchunks * d.k * 4);
   w.cand_idx = off;   off = align256(off + B * w.nchunks * d.k * 4);
   w.scores = off;     off = align256(off + (w.tc_index ? B * (size_t)d.capacity * 4 : 0));
+  w.qop = off;        off = align256(off + (w.tc_index ? B * decode_qop_bytes(d.nh_i) : 0));
   w.sel = off;        off = align256(off + B * (d.is_hca ? 0 : d.k) * 4);
   w.part_o = off;     off = align256(off + B * w.nsplit * d.nh * (size_t)d.c * 4);
   w.part_ms = off;    off = align256(off + B * w.nsplit * d.nh * 2 * 4);
@@ -642,14 +709,16 @@ cudaError_t launch_decode_step(const csa_cache_desc& d, const CacheView& cv, con
   const int dims = d.c + (d.is_hca ? 0 : d.c_i);
   const unsigned emit_threads = (unsigned)std::min(1024, std::max(256, (dims + 31) / 32 * 32));
   const size_t emit_smem = sizeof(float) * (dims + 32);
+  uint8_t* qop = w.tc_index ? wb + w.qop : nullptr;
   cudaError_t err = launch_pdl(append_emit_kernel, dim3((unsigned)d.batch), dim3(emit_threads),
-                               emit_smem, s, d, cv, pos, rows, p);
+                               emit_smem, s, d, cv, pos, rows, p,
+                               (const __nv_bfloat16*)q_i, w_i, qop);
   if (err != cudaSuccess) return err;
   if (!d.is_hca && w.tc_index) {
     float* scores = reinterpret_cast<float*>(wb + w.scores);
     unsigned int* flag = device_timeout_flag();
     if (flag == nullptr) return cudaErrorUnknown;
-    err = launch_decode_index_tc(d, cv, pos, q_i, w_i, scores, flag, s);
+    err = launch_decode_index_tc(d, cv, pos, qop, scores, flag, s);
     if (err != cudaSuccess) return err;
     if (decode_topk_supported(d)) {
       err = launch_decode_topk(d, pos, scores, sel, s);

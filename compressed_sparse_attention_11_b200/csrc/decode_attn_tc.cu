@@ -282,13 +282,10 @@ __global__ void __launch_bounds__(kThreads, 1) decode_attn_tc_kernel(
       mbar_wait(&bar->o_full, 0, err, false);  // every MMA done before TMEM is released
       if (!ok && issued == 0) mbar_wait(&bar->q_full, 0, err, false);  // the Q load has landed
     }
-  } else if (warp >= kSoftWarps) {
-    // ------------------------------ gather only ----------------------------------
-    for (int jt = 0; jt < ntile && live; ++jt)
-      if (!gather_tile(jt)) break;
   } else if (live) {
-    // ----------------------- gather, softmax and epilogue ---------------------------
-    const int quad = warp & 3, hh = warp >> 2;
+    // -------- gather (every warp here), softmax and epilogue (warps 0-7) ----------
+    const bool soft = warp < kSoftWarps;
+    const int quad = warp & 3, hh = (warp >> 2) & 1;
     const int row = quad * 32 + lane;  // entry row within a tile / dim within a chunk
     const uint32_t lane_base = tmem + ((uint32_t)(quad * 32) << 16);
     const uint32_t s_addr = lane_base + kColS + hh * 32;
@@ -301,6 +298,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_attn_tc_kernel(
     bool ok = true;
     for (int jt = 0; jt < ntile && ok; ++jt) {
       if (!(ok = gather_tile(jt))) break;
+      if (!soft) continue;
       if (!(ok = mbar_wait(&bar->s_full, (uint32_t)(jt & 1), err))) break;
       tc_fence_after();
       const bool valid = (tile0 + jt) * kTE + row < N;
@@ -376,6 +374,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_attn_tc_kernel(
       if (lane == 0) mbar_arrive(&bar->p_full);
     }
     // ---- epilogue: this range's O^T, max and sum (or, alone, the output) ----------
+    if (!soft) ok = false;
     if (ok) ok = mbar_wait(&bar->o_full, 0, err);
     if (ok) {
       tc_fence_after();

@@ -14,20 +14,17 @@
 // one per CTA (one CTA per SM); each CTA keeps a single TMA ring of 16 KB
 // tiles (128-byte swizzle) full across sequence boundaries, so the stream
 // never drains between sequences.  One lane issues M = 128 keys x N = 2H x
-// K = 128 kind::f8f6f4 MMAs straight from the ring.  The B operand holds each
-// query head twice: hi = E4M3(q/s_h) and lo = E4M3(q/s_h - hi), s_h a power
-// of two with max|q_h|/s_h <= 448, so s_h (hi + lo) reproduces the bf16 query
-// exactly except for elements below 2^-6 s_h in magnitude (absolute error
-// below 2^-10 s_h there); two warps build it for the next sequence of the
-// range while the current one streams (two operand slots, each freed by the
-// MMAs of its sequence's last tile; the head weights sit in a 16-deep ring
-// freed by the epilogue, which trails the MMAs by at most ten tiles, so no
-// phase of its barriers can alias).  Per K step two
-// N = H MMAs accumulate the hi and the lo halves into the same TMEM columns,
-// so the accumulator already holds q . code.  Two warpgroups of epilogue warps
-// take alternate tiles (eight accumulators in TMEM for H = 64) and apply
-// ReLU, the head weights (with s_h folded in) and the key scale; scores go to
-// a per-sequence fp32 array (L2-resident at these sizes) for the selection
+// K = 128 kind::f8f6f4 MMAs straight from the ring: the B operand holds each
+// query head twice, hi = E4M3(q/s_h) and lo = E4M3(q/s_h - hi) with s_h a
+// power of two, which together reproduce the bf16 query (the append step
+// builds this operand once per sequence; here one bulk copy per sequence
+// brings it in, two operand slots each freed by the MMAs of its sequence's
+// last tile, and the head weights w_h s_h into a 16-deep ring freed by the
+// epilogue, which trails the MMAs by at most ten tiles, so no phase of its
+// barriers can alias).  Two warpgroups of epilogue warps take alternate
+// tiles (four accumulators in TMEM for H = 64), add the hi and lo halves and
+// apply ReLU, the head weights and the key scale; scores go to a
+// per-sequence fp32 array (L2-resident at these sizes) for the selection
 // kernel.
 #include "common.cuh"
 #include "launch.h"
@@ -40,34 +37,39 @@ namespace {
 constexpr int kKeys = 128;               // keys per tile (MMA M)
 constexpr int kCI = 128;                 // index-key dim = bytes per FP8 key
 constexpr int kTileBytes = kKeys * kCI;  // 16 KB
-constexpr int kThreads = 384;  // warp 0 TMA, 1 MMA, 2-3 query split, 4-7 / 8-11 epilogue
+constexpr int kThreads = 384;  // warp 0 TMA, 1 MMA, 2 operand copies, 4-7 / 8-11 epilogue
 constexpr int kBSlots = 2;               // query operands (sequences) in flight
 constexpr int kWSlots = 16;              // head-weight vectors (sequences) in flight
 constexpr int kSmemLimit = 232448;
 
 template <int S>
 struct __align__(8) DecIdxBars {
-  uint64_t full[S], empty[S], d_full[8], d_empty[8], b_full[kBSlots], b_empty[kBSlots], drain;
+  uint64_t full[S], empty[S], d_full[2], d_empty[2], b_full[kBSlots], b_empty[kBSlots], drain;
   uint64_t w_full[kWSlots], w_empty[kWSlots];
   uint32_t tmem_base;
   int j0, count;  // the CTA's first tile (within sequence b0) and its number of tiles
   int64_t b0;
 };
 
+// Tiles travel in groups of TPP ("pairs"): one ring stage, one TMEM
+// accumulator set, and one commit each.  A tcgen05 commit or MMA costs the
+// issuing thread about as much as a 128-key MMA of the tensor core, so
+// committing once per two tiles is what keeps the MMA warp ahead of HBM.
 template <int H>
 struct DecIdxCfg {
   static constexpr int N = 2 * H;                  // hi and lo rows per head
   static constexpr int B_BYTES = N * 128;          // one query operand
+  static constexpr int TPP = 512 / N / 2;          // tiles per pair: 2 (H = 64), 1 (H = 128)
+  static constexpr int STAGE_BYTES = TPP * kTileBytes;
   static constexpr int STAGES =
-      (kSmemLimit - 1024 - kBSlots * B_BYTES - kWSlots * H * 4 - 768) / kTileBytes;
+      (kSmemLimit - 1024 - kBSlots * B_BYTES - kWSlots * H * 4 - 768) / STAGE_BYTES;
   static constexpr int OFF_RAW = 0;
-  static constexpr int OFF_B = OFF_RAW + STAGES * kTileBytes;
+  static constexpr int OFF_B = OFF_RAW + STAGES * STAGE_BYTES;
   static constexpr int OFF_W = OFF_B + kBSlots * B_BYTES;
   static constexpr int OFF_BAR = OFF_W + kWSlots * H * 4;
   static constexpr int SMEM = OFF_BAR + (int)sizeof(DecIdxBars<STAGES>) + 1024;
-  static constexpr int DBUFS = 512 / H;            // TMEM accumulators: 8 (H = 64), 4 (H = 128)
   static_assert(SMEM <= kSmemLimit, "shared memory budget");
-  static_assert(DBUFS >= 2 && DBUFS <= 8 && DBUFS % 2 == 0, "TMEM accumulators");
+  static_assert(TPP >= 1 && 2 * TPP * N <= 512, "two accumulator sets in TMEM");
 };
 
 __device__ __forceinline__ int tiles_of(const int64_t* pos, int64_t b, int m, int64_t cap) {
@@ -136,11 +138,10 @@ __device__ void locate_range(const int64_t* pos, int64_t batch, int m, int64_t c
 template <int H>
 __global__ void __launch_bounds__(kThreads, 1) decode_index_tc_kernel(
     const __grid_constant__ CUtensorMap tm_keys, const float* __restrict__ key_scale,
-    const __nv_bfloat16* __restrict__ q_i, const float* __restrict__ w_i,
-    const int64_t* __restrict__ pos, int64_t batch, int64_t cap, int m,
+    const uint8_t* __restrict__ qop, const int64_t* __restrict__ pos, int64_t batch, int64_t cap, int m,
     float* __restrict__ scores, unsigned int* __restrict__ err) {
   using C = DecIdxCfg<H>;
-  constexpr int S = C::STAGES, DB = C::DBUFS;
+  constexpr int S = C::STAGES;
   using namespace sm100;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = smem_raw + ((1024 - (smem_u32(smem_raw) & 1023)) & 1023);
@@ -156,16 +157,16 @@ __global__ void __launch_bounds__(kThreads, 1) decode_index_tc_kernel(
         mbar_init(&bar->full[s], 1);
         mbar_init(&bar->empty[s], 1);
       }
-      for (int p = 0; p < 8; ++p) {
-        mbar_init(&bar->d_full[p], 1);
-        mbar_init(&bar->d_empty[p], 4);
+      for (int q = 0; q < 2; ++q) {
+        mbar_init(&bar->d_full[q], 1);
+        mbar_init(&bar->d_empty[q], 4 * C::TPP);  // every epilogue warp with a tile in the pair
       }
       for (int u = 0; u < kBSlots; ++u) {
-        mbar_init(&bar->b_full[u], 2);
+        mbar_init(&bar->b_full[u], 1);
         mbar_init(&bar->b_empty[u], 1);  // the MMAs of the sequence's last tile
       }
       for (int u = 0; u < kWSlots; ++u) {
-        mbar_init(&bar->w_full[u], 2);
+        mbar_init(&bar->w_full[u], 1);
         mbar_init(&bar->w_empty[u], 8);  // every epilogue warp, once per sequence
       }
       mbar_init(&bar->drain, 1);
@@ -197,66 +198,75 @@ __global__ void __launch_bounds__(kThreads, 1) decode_index_tc_kernel(
   const int j0 = bar->j0;
   const bool live = count > 0 && flag_value(err) == 0;
 
+  constexpr int TPP = C::TPP;
+  const int npairs = (count + TPP - 1) / TPP;
   if (warp == 0 && live) {
     // ------------------------------- TMA producer --------------------------------
     TileWalk it;
     it.start(pos, b0, j0, m, cap);
-    int i = 0;
-    for (; i < count; ++i, it.next(pos, batch, m, cap)) {
-      const int s = i % S;
-      if (i >= S && !mbar_wait(&bar->empty[s], (uint32_t)(((i / S) - 1) & 1), err)) break;
-      if (lane == 0) {
-        mbar_arrive_expect_tx(&bar->full[s], kTileBytes);
-        tma_load_3d(sRaw + s * kTileBytes, &tm_keys, &bar->full[s], 0, it.j * kKeys, (int)it.b);
-      }
+    int k = 0;
+    for (; k < npairs; ++k) {
+      const int s = k % S;
+      if (k >= S && !mbar_wait(&bar->empty[s], (uint32_t)(((k / S) - 1) & 1), err)) break;
+      const int here = min(TPP, count - k * TPP);
+      if (lane == 0) mbar_arrive_expect_tx(&bar->full[s], here * kTileBytes);
+      for (int r = 0; r < here; ++r, it.next(pos, batch, m, cap))
+        if (lane == 0)
+          tma_load_3d(sRaw + s * C::STAGE_BYTES + r * kTileBytes, &tm_keys, &bar->full[s], 0,
+                      it.j * kKeys, (int)it.b);
       __syncwarp();
     }
-    // every issued tile has landed before the CTA exits
-    for (int r = (i > S ? i - S : 0); r < i; ++r)
+    // every issued stage has landed before the CTA exits
+    for (int r = (k > S ? k - S : 0); r < k; ++r)
       mbar_wait(&bar->full[r % S], (uint32_t)((r / S) & 1), err, false);
   } else if (warp == 1 && live) {
     // ------------------------------- MMA issuer ----------------------------------
-    constexpr uint32_t kIdesc = idesc_e4m3(kKeys, H);
+    constexpr uint32_t kIdesc = idesc_e4m3(kKeys, C::N);
     const uint32_t a0 = smem_u32(sRaw), bb0 = smem_u32(sB);
     TileWalk it;
     it.start(pos, b0, j0, m, cap);
     int u = -1;  // sequence counter within the range
-    for (int i = 0; i < count; ++i, it.next(pos, batch, m, cap)) {
-      const int s = i % S, p = i % DB;
-      if (i == 0 || it.j == 0) {
-        ++u;
-        if (!mbar_wait(&bar->b_full[u & 1], (uint32_t)((u >> 1) & 1), err)) break;
-      }
-      if (!mbar_wait(&bar->full[s], (uint32_t)((i / S) & 1), err)) break;
-      if (i >= DB && !mbar_wait(&bar->d_empty[p], (uint32_t)(((i / DB) - 1) & 1), err)) break;
+    bool ok = true;
+    for (int k = 0; k < npairs && ok; ++k) {
+      const int s = k % S, q = k & 1;
+      if (!(ok = mbar_wait(&bar->full[s], (uint32_t)((k / S) & 1), err))) break;
+      if (k >= 2 && !(ok = mbar_wait(&bar->d_empty[q], (uint32_t)(((k >> 1) - 1) & 1), err)))
+        break;
       tc_fence_after();
-      if (lane == 0) {
-        const uint32_t bslot = bb0 + (u & 1) * C::B_BYTES;
-#pragma unroll
-        for (int kk = 0; kk < kCI / 32; ++kk) {  // K = 32 bytes per instruction
-          const uint64_t a = desc_sw128(a0 + s * kTileBytes + kk * 32);
-          // hi rows 0..H-1, then lo rows H..2H-1 into the same columns
-          mma_f8(tmem + p * H, a, desc_sw128(bslot + kk * 32), kIdesc, kk > 0 ? 1u : 0u);
-          mma_f8(tmem + p * H, a, desc_sw128(bslot + H * 128 + kk * 32), kIdesc, 1u);
+      for (int r = 0; r < TPP && k * TPP + r < count; ++r, it.next(pos, batch, m, cap)) {
+        const int i = k * TPP + r;
+        if (i == 0 || it.j == 0) {
+          ++u;
+          if (!(ok = mbar_wait(&bar->b_full[u & 1], (uint32_t)((u >> 1) & 1), err))) break;
+          tc_fence_after();
         }
-        mma_commit(&bar->d_full[p]);
+        if (lane == 0) {
+          const uint32_t bslot = bb0 + (u & 1) * C::B_BYTES;
+          const uint32_t at = a0 + s * C::STAGE_BYTES + r * kTileBytes;
+#pragma unroll
+          for (int kk = 0; kk < kCI / 32; ++kk)  // K = 32 bytes per instruction
+            mma_f8(tmem + (q * TPP + r) * C::N, desc_sw128(at + kk * 32),
+                   desc_sw128(bslot + kk * 32), kIdesc, kk > 0 ? 1u : 0u);
+          if (i + 1 == count || it.j + 1 == it.nt) mma_commit(&bar->b_empty[u & 1]);
+        }
+        __syncwarp();
+      }
+      if (!ok) break;
+      if (lane == 0) {
+        mma_commit(&bar->d_full[q]);
         mma_commit(&bar->empty[s]);
-        if (i + 1 == count || it.j + 1 == it.nt) mma_commit(&bar->b_empty[u & 1]);
       }
       __syncwarp();
     }
     if (lane == 0) mma_commit(&bar->drain);
     __syncwarp();
     mbar_wait(&bar->drain, 0, err, false);
-  } else if ((warp == 2 || warp == 3) && live) {
-    // ------------- query operand: per head a power of two and hi / lo E4M3 -------------
-    // 64 threads, a half-warp per head, 8 dims per thread, 4 heads per pass
-    const int tid2 = threadIdx.x - 64;
-    const int hl = tid2 & 15, hsub = tid2 >> 4;
-    constexpr int kPass = H / 4;
+  } else if (warp == 2 && live) {
+    // ----------- query operands: one bulk copy each, per sequence of the range -----------
     TileWalk it;
     it.start(pos, b0, j0, m, cap);
     int left = count;
+    constexpr uint32_t kRec = (uint32_t)(C::B_BYTES + H * 4);
     for (int u = 0; left > 0; ++u) {
       const int64_t b = it.b;
       const int here = min(left, it.nt - it.j);
@@ -268,73 +278,24 @@ __global__ void __launch_bounds__(kThreads, 1) decode_index_tc_kernel(
       if (u >= kWSlots &&
           !mbar_wait(&bar->w_empty[ws], (uint32_t)(((u / kWSlots) - 1) & 1), err))
         break;
-      uint8_t* dstB = sB + slot * C::B_BYTES;
-      float* dstW = sW + ws * H;
-      constexpr int kBatch = kPass < 16 ? kPass : 16;  // loads in flight per thread
-#pragma unroll 1
-      for (int p0 = 0; p0 < kPass; p0 += kBatch) {
-        uint4 raw[kBatch];
-        float wv[kBatch];
-#pragma unroll
-        for (int q = 0; q < kBatch; ++q) {
-          const int h = (p0 + q) * 4 + hsub;
-          raw[q] = *reinterpret_cast<const uint4*>(q_i + (b * H + h) * kCI + hl * 8);
-          wv[q] = hl == 0 ? w_i[b * H + h] : 0.f;
-        }
-#pragma unroll
-        for (int q = 0; q < kBatch; ++q) {
-          const int h = (p0 + q) * 4 + hsub;
-          const uint32_t wd[4] = {raw[q].x, raw[q].y, raw[q].z, raw[q].w};
-          float v[8];
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            v[2 * e] = __uint_as_float(wd[e] << 16);
-            v[2 * e + 1] = __uint_as_float(wd[e] & 0xffff0000u);
-          }
-          float amax = 0.f;
-#pragma unroll
-          for (int e = 0; e < 8; ++e) amax = fmaxf(amax, fabsf(v[e]));
-#pragma unroll
-          for (int off = 8; off > 0; off >>= 1)
-            amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, off));
-          float sc = 1.f;
-          if (amax > 0.f) {  // smallest power of two >= amax / 448
-            const uint32_t ub = __float_as_uint(amax / 448.f);
-            sc = (ub & 0x007fffffu) == 0 ? __uint_as_float(ub)
-                                         : __uint_as_float((ub & 0x7f800000u) + 0x00800000u);
-          }
-          uint32_t hi2[2] = {0u, 0u}, lo2[2] = {0u, 0u};
-#pragma unroll
-          for (int e = 0; e < 8; ++e) {
-            const float x = v[e] / sc;  // exact: sc is a power of two
-            const uint8_t hc = e4m3_code(x);
-            const uint8_t lc = e4m3_code(x - e4m3_value(hc));
-            hi2[e >> 2] |= (uint32_t)hc << (8 * (e & 3));
-            lo2[e >> 2] |= (uint32_t)lc << (8 * (e & 3));
-          }
-          const int d = hl * 8, ch = d >> 4;
-          const int rh = h, rl = H + h;
-          *reinterpret_cast<uint2*>(dstB + rh * 128 + ((ch ^ (rh & 7)) * 16) + (d & 15)) =
-              make_uint2(hi2[0], hi2[1]);
-          *reinterpret_cast<uint2*>(dstB + rl * 128 + ((ch ^ (rl & 7)) * 16) + (d & 15)) =
-              make_uint2(lo2[0], lo2[1]);
-          if (hl == 0) dstW[h] = wv[q] * sc;
-        }
-      }
-      fence_proxy_async();  // generic-proxy writes before the tensor core reads them
-      __syncwarp();
       if (lane == 0) {
-        mbar_arrive(&bar->b_full[slot]);
-        mbar_arrive(&bar->w_full[ws]);
+        const uint8_t* rec = qop + b * kRec;
+        mbar_arrive_expect_tx(&bar->b_full[slot], C::B_BYTES);
+        bulk_load(sB + slot * C::B_BYTES, rec, C::B_BYTES, &bar->b_full[slot]);
+        mbar_arrive_expect_tx(&bar->w_full[ws], H * 4);
+        bulk_load(sW + ws * H, rec + C::B_BYTES, H * 4, &bar->w_full[ws]);
       }
+      __syncwarp();
       left -= here;
       for (int r = 0; r < here; ++r) it.next(pos, batch, m, cap);
     }
   } else if (warp >= 4 && live) {
-    // ------- epilogue: ReLU, head weights, key scale (group g: tiles i % 2 == g) -------
+    // --- epilogue: hi + lo, ReLU, head weights, key scale (group g: tile g of each pair,
+    //     or every other pair when a pair is one tile) ---
     const int quad = warp & 3, grp = (warp - 4) >> 2;
     const int row = quad * 32 + lane;
     const uint32_t lane_addr = tmem + ((uint32_t)(quad * 32) << 16);
+    auto mine_of = [&](int i) { return TPP == 2 ? (i & 1) == grp : ((i / TPP) & 1) == grp; };
     TileWalk it;
     it.start(pos, b0, j0, m, cap);
     int64_t V = 0;
@@ -345,49 +306,55 @@ __global__ void __launch_bounds__(kThreads, 1) decode_index_tc_kernel(
       return sidx < Vw ? __ldcs(key_scale + w.b * cap + sidx) : 0.f;
     };
     TileWalk ahead = it;
-    if (grp == 1 && count > 1) ahead.next(pos, batch, m, cap);
-    float ks_next = grp < count ? scale_of(ahead) : 0.f;
+    int first = 0;  // this group's first tile
+    while (first < count && !mine_of(first)) {
+      ahead.next(pos, batch, m, cap);
+      ++first;
+    }
+    float ks_next = first < count ? scale_of(ahead) : 0.f;
     int u = -1;
     for (int i = 0; i < count; ++i, it.next(pos, batch, m, cap)) {
       if (i == 0 || it.j == 0) {
         ++u;
         V = min((pos[it.b] + 1) / m, cap);
       }
-      const bool mine = (i & 1) == grp;
       const bool seq_end = i + 1 == count || it.j + 1 == it.nt;
-      if (mine) {
+      if (mine_of(i)) {
         const float ks = ks_next;
-        if (i + 2 < count) {
+        if (i + 2 < count) {  // this group's next tile is i + 2
           ahead.next(pos, batch, m, cap);
           ahead.next(pos, batch, m, cap);
           ks_next = scale_of(ahead);
         }
-        const int p = i % DB;
+        const int k = i / TPP, q = k & 1;
+        const uint32_t acc_col = (uint32_t)((q * TPP + i % TPP) * C::N);
         // the head weights of this sequence are in place
         if (!mbar_wait(&bar->w_full[u % kWSlots], (uint32_t)((u / kWSlots) & 1), err)) break;
         const float* w = sW + (u % kWSlots) * H;
-        if (!mbar_wait(&bar->d_full[p], (uint32_t)((i / DB) & 1), err)) break;
+        if (!mbar_wait(&bar->d_full[q], (uint32_t)((k >> 1) & 1), err)) break;
         tc_fence_after();
         float acc[8];
 #pragma unroll
         for (int e = 0; e < 8; ++e) acc[e] = 0.f;
 #pragma unroll
         for (int c = 0; c < H / 32; ++c) {
-          uint32_t d[32];
-          tmem_ld32(lane_addr + p * H + c * 32, d);
+          uint32_t dh[32], dl[32];
+          tmem_ld32(lane_addr + acc_col + c * 32, dh);
+          tmem_ld32(lane_addr + acc_col + H + c * 32, dl);
           tmem_ld_wait();
 #pragma unroll
           for (int e = 0; e < 32; e += 4) {
             const float4 w4 = *reinterpret_cast<const float4*>(w + c * 32 + e);
-            acc[(e >> 2) & 7] = fmaf(w4.x, fmaxf(__uint_as_float(d[e]), 0.f), acc[(e >> 2) & 7]);
-            acc[(e >> 2) & 7] = fmaf(w4.y, fmaxf(__uint_as_float(d[e + 1]), 0.f), acc[(e >> 2) & 7]);
-            acc[(e >> 2) & 7] = fmaf(w4.z, fmaxf(__uint_as_float(d[e + 2]), 0.f), acc[(e >> 2) & 7]);
-            acc[(e >> 2) & 7] = fmaf(w4.w, fmaxf(__uint_as_float(d[e + 3]), 0.f), acc[(e >> 2) & 7]);
+            float* a = &acc[(e >> 2) & 7];
+            *a = fmaf(w4.x, fmaxf(__uint_as_float(dh[e]) + __uint_as_float(dl[e]), 0.f), *a);
+            *a = fmaf(w4.y, fmaxf(__uint_as_float(dh[e + 1]) + __uint_as_float(dl[e + 1]), 0.f), *a);
+            *a = fmaf(w4.z, fmaxf(__uint_as_float(dh[e + 2]) + __uint_as_float(dl[e + 2]), 0.f), *a);
+            *a = fmaf(w4.w, fmaxf(__uint_as_float(dh[e + 3]) + __uint_as_float(dl[e + 3]), 0.f), *a);
           }
         }
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(&bar->d_empty[p]);
+        if (lane == 0) mbar_arrive(&bar->d_empty[q]);
         const float sum = ((acc[0] + acc[1]) + (acc[2] + acc[3])) + ((acc[4] + acc[5]) + (acc[6] + acc[7]));
         const int64_t sidx = (int64_t)it.j * kKeys + row;
         if (sidx < V) scores[it.b * cap + sidx] = sum * ks;
@@ -409,8 +376,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_index_tc_kernel(
 
 template <int H>
 cudaError_t launch_h(const csa_cache_desc& d, const CacheView& cv, const int64_t* pos,
-                     const void* q_i, const float* w_i, float* scores, unsigned int* err,
-                     cudaStream_t s) {
+                     const uint8_t* qop, float* scores, unsigned int* err, cudaStream_t s) {
   using C = DecIdxCfg<H>;
   CUtensorMap tk;
   if (!make_tmap_3d(&tk, cv.ikey_fp8, 1, kCI, (uint64_t)d.capacity, (uint64_t)d.batch, kCI,
@@ -422,7 +388,7 @@ cudaError_t launch_h(const csa_cache_desc& d, const CacheView& cv, const int64_t
   const int64_t max_tiles = d.batch * ((d.capacity + kKeys - 1) / kKeys);
   const unsigned grid = (unsigned)std::max<int64_t>(1, std::min<int64_t>(sm_count(), max_tiles));
   return launch_pdl(kern, dim3(grid), dim3(kThreads), (size_t)C::SMEM, s, tk,
-                    (const float*)cv.ikey_scale, (const __nv_bfloat16*)q_i, w_i, pos,
+                    (const float*)cv.ikey_scale, qop, pos,
                     (int64_t)d.batch, (int64_t)d.capacity, d.m, scores, err);
 }
 
@@ -433,11 +399,11 @@ bool decode_index_tc_supported(const csa_cache_desc& d) {
 }
 
 cudaError_t launch_decode_index_tc(const csa_cache_desc& d, const CacheView& cv,
-                                   const int64_t* pos, const void* q_i, const float* w_i,
-                                   float* scores, unsigned int* err, cudaStream_t s) {
+                                   const int64_t* pos, const uint8_t* qop, float* scores,
+                                   unsigned int* err, cudaStream_t s) {
   switch (d.nh_i) {
-    case 64: return launch_h<64>(d, cv, pos, q_i, w_i, scores, err, s);
-    case 128: return launch_h<128>(d, cv, pos, q_i, w_i, scores, err, s);
+    case 64: return launch_h<64>(d, cv, pos, qop, scores, err, s);
+    case 128: return launch_h<128>(d, cv, pos, qop, scores, err, s);
     default: return cudaErrorInvalidValue;
   }
 }

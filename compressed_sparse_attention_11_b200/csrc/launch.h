@@ -59,10 +59,14 @@ cudaError_t launch_attn_tc(const void* q, const void* kv_comp, const int32_t* id
 // tcgen05 decode indexer over FP8 keys (c_i = 128, nh_i in {64, 128}), persistent.
 struct CacheView;
 bool decode_index_tc_supported(const csa_cache_desc& d);
-// scores [batch][capacity] fp32, written for s < V of each sequence.
+// Bytes of one sequence's indexer query operand: the swizzled hi / lo E4M3
+// image (2 H rows of 128 bytes) followed by H fp32 weights.
+__host__ __device__ inline size_t decode_qop_bytes(int nh_i) { return (size_t)nh_i * (2 * 128 + 4); }
+// qop: [batch] query operands (written by the append step); scores
+// [batch][capacity] fp32, written for s < V of each sequence.
 cudaError_t launch_decode_index_tc(const csa_cache_desc& d, const CacheView& cv,
-                                   const int64_t* pos, const void* q_i, const float* w_i,
-                                   float* scores, unsigned int* err, cudaStream_t s);
+                                   const int64_t* pos, const uint8_t* qop, float* scores,
+                                   unsigned int* err, cudaStream_t s);
 
 // Exact top-k over the indexer's scores, one thread-block cluster per
 // sequence with the scores staged in shared memory.  sel [batch][k]: the
