@@ -43,7 +43,11 @@ UNIT = "tokens/s"
 # call's kernels, one capture of the full workload; the summary is under
 # profiles/).  A figure is reported only while the kernel sources it was
 # measured on are unchanged (sha256 prefix per file), else null.
-MEASURED_TRAFFIC = {}
+MEASURED_TRAFFIC = {
+    # index_scores_tc_kernel 1127.5 MB read + 2136.4 MB written, topk_rows_staged_kernel
+    # 2150.5 MB read + 76.6 MB written (n = 65536; profiles/dram_bytes_prefill_calls.md)
+    "index_topk": {"bytes": 5491000000, "sources": {'compressed_sparse_attention_11_b200/csrc/indexer_tc.cu': '7f5543f1ca4e8e9e', 'compressed_sparse_attention_11_b200/csrc/topk.cu': 'b5c2b3e3bbbddc89', 'compressed_sparse_attention_11_b200/csrc/sm100.cuh': 'dc33b8fd81a2190a', 'compressed_sparse_attention_11_b200/csrc/common.cuh': '2c8e048cf6f6eadb'}},
+}
 
 
 # ----------------------------------------------------------------- helpers ---
@@ -423,6 +427,40 @@ def run_reference(args):
 
 # -------------------------------------------------------------------- main ---
 
+def run_profile_case(args):
+    """A few steps of one workload, optionally resized, for ncu captures."""
+    import dataclasses
+    import compressed_sparse_attention_11_b200 as csa
+    dev = torch.device("cuda", 0)
+    if args.profile in ("prefill", "hca"):
+        base = G.CSA_PREFILL if args.profile == "prefill" else G.HCA_PREFILL
+        w = dataclasses.replace(base, n=args.n) if args.n else base
+        if args.profile == "prefill":
+            L = CsaPrefill(w, dev)
+            for _ in range(args.steps):
+                L.step()
+        else:
+            d = {k: v.to(dev) for k, v in G.prefill_inputs(w).items()}
+            for _ in range(args.steps):
+                kv = csa.csa_compress(d["ca"], None, d["za"], None, d["ba"], None, w.m)
+                csa.hca_attn(d["q"], kv, d["kv_win"], w.window, d["sink"], w.scale, w.m)
+    else:
+        layers = [G.CSA_DECODE] if args.profile == "decode_csa" else \
+            [G.MIXED_DECODE_CSA, G.MIXED_DECODE_HCA]
+        if args.batch:
+            layers = [dataclasses.replace(x, batch=args.batch) for x in layers]
+        built = [_decode_layer(x, dev, 4) for x in layers]
+        for it in range(args.steps):
+            for x, (cache, ps, biases, sink, out) in zip(layers, built):
+                st = ps[it % 4]
+                cache.decode_step(st["pos"], st["rows"], biases, sink, x.scale, st["q"],
+                                  st["q_i"], st["w_i"], out=out)
+    torch.cuda.synchronize()
+    csa.csa_check()
+    print(json.dumps({"profile": args.profile, "steps": args.steps, "n": args.n,
+                      "batch": args.batch, "ok": True}), flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -431,9 +469,16 @@ def main():
     ap.add_argument("--impl", default="ours", choices=("ours", "reference"))
     ap.add_argument("--skip-extras", action="store_true", help="headline workload only")
     ap.add_argument("--skip-cpu", action="store_true", help="no oracle timing")
+    ap.add_argument("--profile", choices=("prefill", "hca", "decode_csa", "decode_mixed"),
+                    help="run --steps steps of one workload (for a profiler) and exit")
+    ap.add_argument("--n", type=int, default=None, help="--profile prefill/hca: tokens")
+    ap.add_argument("--batch", type=int, default=None, help="--profile decode_*: sequences")
     args = ap.parse_args()
     if args.impl == "reference":
         run_reference(args)
+        return
+    if args.profile:
+        run_profile_case(args)
         return
     rank, world, local = dist_setup()
     dev = torch.device("cuda", local)

@@ -38,8 +38,228 @@ __global__ void __launch_bounds__(kSelThreads) topk_rows_kernel(
   }
 }
 
+// ---------------------------------------------------------------------------
+// One CTA per row, the row staged in shared memory as order keys (unsigned
+// integers with the float order).  One radix pass histograms the keys into
+// 2048 bins spanning [min, max] of the row; the bin T where the count from
+// the top reaches k decides: keys above T are chosen, and the keys of bin T
+// (few, when the bins are fine enough) are ranked among themselves by (key
+// descending, index ascending) to give the exact cut (key, index) of the
+// k-th choice.  A crowded bin T narrows the window to that bin with 2048x
+// finer bins and repeats.  The chosen indices are written in ascending order
+// by warps over contiguous segments.  About eight block barriers per row.
+// ---------------------------------------------------------------------------
+constexpr int kRowThreads = 512;
+constexpr int kRowWarps = kRowThreads / 32;
+constexpr int kRowBins = 2048;
+constexpr int kRowBinBits = 11;
+constexpr int kRowBinsPerThread = kRowBins / kRowThreads;  // 4
+constexpr int kRowCand = 256;                              // bin-T keys ranked directly (3 CTAs per SM at 16K keys)
+constexpr int64_t kRowMaxKeys = 40960;                     // keys staged per row
+
+struct __align__(16) RowTopkShared {
+  uint32_t hist[kRowBins];
+  uint32_t cand_key[kRowCand];
+  int32_t cand_pos[kRowCand];
+  uint32_t wred[2][kRowWarps];
+  uint32_t wcnt[kRowWarps];
+  uint32_t T, G, C, cand_n, cut_key;
+  int32_t cut_pos;
+};
+
+__device__ __forceinline__ uint32_t bit_length(uint32_t x) { return x == 0 ? 0u : 32u - __clz(x); }
+
+__global__ void __launch_bounds__(kRowThreads) topk_rows_staged_kernel(
+    const float* __restrict__ scores, int64_t ld, int64_t n, int m, int64_t E, int k,
+    int32_t* __restrict__ idx) {
+  extern __shared__ __align__(16) unsigned char smem_raw[];
+  RowTopkShared& sh = *reinterpret_cast<RowTopkShared*>(smem_raw);
+  uint32_t* key = reinterpret_cast<uint32_t*>(smem_raw + sizeof(RowTopkShared));
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int64_t t = blockIdx.x, b = blockIdx.y;
+  const int V = (int)min((t + 1) / m, E);
+  int32_t* out = idx + (b * n + t) * k;
+  if (V <= k) {
+    for (int j = tid; j < k; j += kRowThreads) out[j] = j < V ? j : -1;
+    return;
+  }
+  // 1. the row as order keys, with its key range
+  const float* row = scores + (b * n + t) * ld;
+  uint32_t mn = 0xffffffffu, mx = 0u;
+  {
+    constexpr int kBatch = 8;
+    for (int i0 = tid; i0 < V; i0 += kRowThreads * kBatch) {
+      float v[kBatch];
+#pragma unroll
+      for (int u = 0; u < kBatch; ++u) {
+        const int i = i0 + u * kRowThreads;
+        v[u] = i < V ? __ldcs(row + i) : 0.f;
+      }
+#pragma unroll
+      for (int u = 0; u < kBatch; ++u) {
+        const int i = i0 + u * kRowThreads;
+        if (i < V) {
+          const uint32_t ky = order_key(v[u]);
+          key[i] = ky;
+          mn = min(mn, ky);
+          mx = max(mx, ky);
+        }
+      }
+    }
+  }
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) {
+    mn = min(mn, __shfl_xor_sync(0xffffffffu, mn, off));
+    mx = max(mx, __shfl_xor_sync(0xffffffffu, mx, off));
+  }
+  if (lane == 0) {
+    sh.wred[0][warp] = mn;
+    sh.wred[1][warp] = mx;
+  }
+  if (tid == 0) sh.cand_n = 0u;
+  __syncthreads();
+  uint32_t kmin = 0xffffffffu, kmax = 0u;
+  for (int w = 0; w < kRowWarps; ++w) {
+    kmin = min(kmin, sh.wred[0][w]);
+    kmax = max(kmax, sh.wred[1][w]);
+  }
+  // 2. radix refinement of the window [base, base + 2048 << shift)
+  uint32_t base = kmin, need = (uint32_t)k;
+  int shift = (int)bit_length(kmax - kmin) - kRowBinBits;
+  shift = shift < 0 ? 0 : shift;
+  uint32_t klo, khi, need_w = 0u, cut_key = 0u;
+  int32_t cut_pos = 0;
+  bool exact = false;
+  for (;;) {
+    for (int i = tid; i < kRowBins; i += kRowThreads) sh.hist[i] = 0u;
+    __syncthreads();
+    for (int i = tid; i < V; i += kRowThreads) {
+      const uint32_t ky = key[i];
+      if (ky >= base) {
+        const uint32_t bin = (ky - base) >> shift;
+        if (bin < (uint32_t)kRowBins) atomicAdd(&sh.hist[bin], 1u);
+      }
+    }
+    __syncthreads();
+    {  // the bin where the count from the top reaches `need` (thread tid owns
+       // bins 2047 - 4 tid .. 2044 - 4 tid, descending)
+      uint32_t mine[kRowBinsPerThread], loc = 0;
+#pragma unroll
+      for (int j = 0; j < kRowBinsPerThread; ++j) {
+        mine[j] = sh.hist[kRowBins - 1 - (tid * kRowBinsPerThread + j)];
+        loc += mine[j];
+      }
+      uint32_t inc = loc;
+#pragma unroll
+      for (int off = 1; off < 32; off <<= 1) {
+        const uint32_t x = __shfl_up_sync(0xffffffffu, inc, off);
+        if (lane >= off) inc += x;
+      }
+      if (lane == 31) sh.wred[0][warp] = inc;
+      __syncthreads();
+      uint32_t acc = inc - loc;
+      for (int w = 0; w < warp; ++w) acc += sh.wred[0][w];
+#pragma unroll
+      for (int j = 0; j < kRowBinsPerThread; ++j) {
+        if (acc < need && acc + mine[j] >= need) {
+          sh.T = (uint32_t)(kRowBins - 1 - (tid * kRowBinsPerThread + j));
+          sh.G = acc;
+          sh.C = mine[j];
+        }
+        acc += mine[j];
+      }
+      __syncthreads();
+    }
+    const uint32_t T = sh.T, G = sh.G, C = sh.C;
+    klo = base + (T << shift);
+    khi = klo + ((1u << shift) - 1u);
+    need -= G;
+    if (shift == 0 || C == need) {
+      need_w = need;
+      break;
+    }
+    if (C <= (uint32_t)kRowCand) {  // rank the bin-T keys among themselves
+      for (int i = tid; i < V; i += kRowThreads) {
+        const uint32_t ky = key[i];
+        if (ky >= klo && ky <= khi) {
+          const uint32_t slot = atomicAdd(&sh.cand_n, 1u);
+          sh.cand_key[slot] = ky;
+          sh.cand_pos[slot] = i;
+        }
+      }
+      __syncthreads();
+      for (int e = tid; e < (int)C; e += kRowThreads) {
+        const uint32_t ke = sh.cand_key[e];
+        const int32_t pe = sh.cand_pos[e];
+        uint32_t rank = 0;
+        for (int f = 0; f < (int)C; ++f) {
+          const uint32_t kf = sh.cand_key[f];
+          rank += (kf > ke || (kf == ke && sh.cand_pos[f] < pe)) ? 1u : 0u;
+        }
+        if (rank == need - 1) {
+          sh.cut_key = ke;
+          sh.cut_pos = pe;
+        }
+      }
+      __syncthreads();
+      exact = true;
+      cut_key = sh.cut_key;
+      cut_pos = sh.cut_pos;
+      break;
+    }
+    base = klo;
+    shift = shift > kRowBinBits ? shift - kRowBinBits : 0;
+    __syncthreads();  // T / G / C are rewritten by the next pass
+  }
+  // 3. chosen: above the window, or in it and among the first need_w by index
+  auto strict_of = [&](uint32_t ky, int i) {
+    return exact ? (ky > cut_key || (ky == cut_key && i <= cut_pos)) : ky > khi;
+  };
+  auto window_of = [&](uint32_t ky) { return !exact && ky >= klo && ky <= khi; };
+  const int seg = ((V + kRowWarps - 1) / kRowWarps + 31) & ~31;
+  const int s0 = min(V, warp * seg), s1 = min(V, s0 + seg);
+  uint32_t strict = 0, win = 0;
+  for (int i0 = s0; i0 < s1; i0 += 32) {
+    const int i = i0 + lane;
+    const uint32_t ky = i < s1 ? key[i] : 0u;
+    strict += __popc(__ballot_sync(0xffffffffu, i < s1 && strict_of(ky, i)));
+    win += __popc(__ballot_sync(0xffffffffu, i < s1 && window_of(ky)));
+  }
+  if (lane == 0) sh.wcnt[warp] = (strict << 16) | win;  // both < 2^16
+  __syncthreads();
+  uint32_t win_before = 0, out_before = 0;
+  for (int w = 0; w < warp; ++w) {
+    const uint32_t st = sh.wcnt[w] >> 16, wi = sh.wcnt[w] & 0xffffu;
+    const uint32_t take = need_w > win_before ? min(wi, need_w - win_before) : 0u;
+    out_before += st + take;
+    win_before += wi;
+  }
+  const uint32_t lt = (1u << lane) - 1u;
+  for (int i0 = s0; i0 < s1; i0 += 32) {
+    const int i = i0 + lane;
+    const uint32_t ky = i < s1 ? key[i] : 0u;
+    const bool is_w = i < s1 && window_of(ky);
+    const uint32_t wm = __ballot_sync(0xffffffffu, is_w);
+    const bool pick = (i < s1 && strict_of(ky, i)) || (is_w && win_before + __popc(wm & lt) < need_w);
+    const uint32_t pm = __ballot_sync(0xffffffffu, pick);
+    const uint32_t o = out_before + __popc(pm & lt);
+    if (pick && o < (uint32_t)k) out[o] = i;
+    out_before += __popc(pm);
+    win_before += __popc(wm);
+  }
+}
+
 cudaError_t launch_topk_rows(const float* scores, int64_t ld, int64_t batch, int64_t n, int m,
                              int64_t E, int k, int32_t* idx, cudaStream_t s) {
+  if (E <= kRowMaxKeys) {
+    const size_t smem = sizeof(RowTopkShared) + (size_t)E * sizeof(uint32_t);
+    cudaError_t e = cudaFuncSetAttribute(topk_rows_staged_kernel,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    topk_rows_staged_kernel<<<dim3((unsigned)n, (unsigned)batch), kRowThreads, smem, s>>>(
+        scores, ld, n, m, E, k, idx);
+    return cudaGetLastError();
+  }
   const int64_t smem_keys = E <= kSelSmemKeys ? E : 0;
   const size_t smem = sizeof(SelectShared<kSelThreads>) + (size_t)kSelCap * 4 +
                       (size_t)kSelSample * 4 + (size_t)smem_keys * sizeof(uint32_t);
