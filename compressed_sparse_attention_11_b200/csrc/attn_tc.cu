@@ -10,25 +10,28 @@
 // context"; B9 of the "Core formulas chapter"; one softmax shared by the
 // window, the compressed entries and the sink).
 //
-// Every query reads its own gathered entries, so the 64 heads of ONE query
-// are the whole reuse available; the contractions therefore run "swapped":
-//   S^T[e, h] = K[e, :] . Q[h, :]           M = 128 entries, N = 64 heads
-//   O^T[d, h] += sum_e V[e, d] P^T[e, h]     M = 128 dims (x4), N = 64 heads
-// The gathered 128 x 512 entry tile is stored once (eight 64-dim slabs,
-// 128-byte swizzle) and read as the K-major A operand of Q.K and as the
-// MN-major A operand (V^T) of P.V.  S^T lands one entry per TMEM lane, so the
-// per-head softmax statistics need cross-lane reductions (a 31-shuffle
-// transpose-reduce per warp, then 4 warps through shared memory); the
-// running max is only moved -- and O^T rescaled in TMEM -- when a tile's max
-// exceeds it by more than 2^8.
+// Heads on TMEM lanes, 64 rows (M = 64): a tcgen05 MMA costs about the same
+// tensor-pipe time whatever its N, so the 64 heads of one query take the M
+// side and the N side is as wide as the operands allow:
+//   S[h, e]  = Q[h, :] . K[e, :]           M = 64 heads, N = 128 entries
+//   O[h, d] += sum_e P[h, e] V[e, d]        M = 64 heads, N = 256 dims (x2)
+// -- 48 MMAs per 128-entry tile.  An M = 64 accumulator fills 16 lanes of
+// each TMEM lane quarter: O (512 columns) takes the low 16 lanes of every
+// quarter and S (two 128-column buffers) the high 16, so one warp per quarter
+// holds both the scores and the output of its 16 heads, two threads per head
+// (one per 32-column half of each 64-column load).  The softmax is per
+// thread with one partner shuffle; the running max moves (and the head's O
+// row is rescaled in TMEM) only when a tile's max exceeds it by 2^8.
 //
+// The gathered 128 x 512 entry tile is stored once (eight 64-dim slabs,
+// 128-byte swizzle): the K-major B operand of Q.K and the MN-major B operand
+// (V) of P.V; each half of P.V frees four slabs for the next tile's gather.
 // Persistent CTAs (one per SM) walk the queries.  Every wait is bounded
 // (including the warp-group exchanges, which use mbarriers rather than
 // named barriers), so a fault upstream ends the kernel with the timeout flag
-// set instead of a hang.  Warp roles: warps 0-7
-// softmax + epilogue (warp w: TMEM lanes 32*(w%4), heads 32*(w/4)), warps
-// 8-10 gather (cp.async, zero-filled past the end of E_t; they also compact
-// the query's valid selected indices), warp 11 issues the MMAs.
+// set instead of a hang.  Warp roles: warps 0-3 softmax + epilogue, warps 4-10
+// gather (cp.async, zero-filled past the end of E_t; they also compact the
+// query's valid selected indices), warp 11 issues the MMAs.
 #include "common.cuh"
 #include "launch.h"
 #include "sm100.cuh"
@@ -40,23 +43,25 @@ namespace csa {
 
 namespace {
 
-constexpr int kNH = 64;                  // query heads (MMA N)
+constexpr int kNH = 64;                  // query heads (MMA M)
 constexpr int kC = 512;                  // entry dim
-constexpr int kTE = 128;                 // entries per tile
+constexpr int kTE = 128;                 // entries per tile (QK N)
 constexpr int kSlabs = kC / 64;          // 64-dim slabs
 constexpr int kSlabBytes = kTE * 128;    // 16 KB
 constexpr int kQSlabBytes = kNH * 128;   // 8 KB
-constexpr int kSoftWarps = 8, kProdWarps = 3;
+constexpr int kPSlabBytes = kNH * 128;   // 8 KB: 64 heads x 64 entries
+constexpr int kSoftWarps = 4, kProdWarps = 7;
 constexpr int kProdThreads = kProdWarps * 32;
 constexpr int kMmaWarp = kSoftWarps + kProdWarps;
-constexpr int kThreads = (kMmaWarp + 1) * 32;  // 384: 3 warps per SM sub-partition
-constexpr int kRowsPerPass = kProdThreads / 8;  // 12 rows x 8 16-byte chunks per pass
-constexpr int kPasses = (kTE + kRowsPerPass - 1) / kRowsPerPass;  // 11
+constexpr int kThreads = (kMmaWarp + 1) * 32;  // 384
+constexpr int kRowsPerPass = kProdThreads / 8;  // 28 rows x 8 16-byte chunks per pass
+constexpr int kPasses = (kTE + kRowsPerPass - 1) / kRowsPerPass;  // 5
 constexpr int kMaxSel = 2048;                  // selected entries per query
 constexpr float kRescaleLog2 = 8.f;            // move the running max only past 2^8
 
-constexpr uint32_t kColS = 0;    // S^T, double-buffered: 2 x 64 columns
-constexpr uint32_t kColO = 128;  // O^T: 4 chunks x 64 columns
+constexpr uint32_t kLaneS = 16u << 16;  // S: the high 16 lanes of each quarter
+constexpr uint32_t kColS = 0;           // S buffers at columns 0 and 128
+constexpr uint32_t kColO = 0;           // O: the low 16 lanes, columns 0-511
 
 struct __align__(16) AttnMeta {
   int ntiles, nrows;
@@ -64,18 +69,19 @@ struct __align__(16) AttnMeta {
 };
 
 struct __align__(8) AttnBars {
-  uint64_t slab_full[kSlabs], slab_empty[kSlabs];
-  uint64_t s_full[2], s_empty[2], p_full, p_empty, q_full, q_empty, o_empty, meta_full[2], drain;
-  uint64_t grp_soft[2], grp_prod;  // bounded group barriers (one arrive per warp)
+  uint64_t slab_full[kSlabs];
+  // half hf of P.V (slabs 4 hf .. 4 hf + 3) done; slab_free[1] also frees P
+  uint64_t slab_free[2];
+  uint64_t s_full[2], s_empty[2], p_full, q_full, q_empty, o_empty, meta_full[2], drain;
+  uint64_t grp_prod;  // bounded group barrier of the producer warps (one arrive per warp)
   uint32_t tmem_base;
 };
 
 constexpr int OFF_Q = 0;
 constexpr int OFF_KV = OFF_Q + kSlabs * kQSlabBytes;        // 65536
 constexpr int OFF_P = OFF_KV + kSlabs * kSlabBytes;         // 196608
-constexpr int OFF_LIST = OFF_P + kTE * 128;                 // 212992
-constexpr int OFF_RED = OFF_LIST + kMaxSel * 4;             // [3][2 hh][4 quad][32] floats
-constexpr int OFF_META = OFF_RED + 3 * 2 * 4 * 32 * 4;
+constexpr int OFF_LIST = OFF_P + 2 * kPSlabBytes;           // 212992
+constexpr int OFF_META = OFF_LIST + kMaxSel * 4;
 constexpr int OFF_SCAN = OFF_META + 2 * (int)sizeof(AttnMeta);
 constexpr int OFF_BAR = OFF_SCAN + 64;
 constexpr int SMEM = OFF_BAR + (int)sizeof(AttnBars) + 1024;
@@ -93,7 +99,6 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(
   uint8_t* sKV = smem + OFF_KV;
   uint8_t* sP = smem + OFF_P;
   int32_t* list = reinterpret_cast<int32_t*>(smem + OFF_LIST);
-  float* red = reinterpret_cast<float*>(smem + OFF_RED);
   AttnMeta* meta = reinterpret_cast<AttnMeta*>(smem + OFF_META);
   int* pscan = reinterpret_cast<int*>(smem + OFF_SCAN);
   AttnBars* bar = reinterpret_cast<AttnBars*>(smem + OFF_BAR);
@@ -103,23 +108,19 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(
   if (flag_value(err) != 0) return;
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < kSlabs; ++s) {
-      mbar_init(&bar->slab_full[s], kProdThreads);
-      mbar_init(&bar->slab_empty[s], 1);
-    }
+    for (int s = 0; s < kSlabs; ++s) mbar_init(&bar->slab_full[s], kProdThreads);
+    mbar_init(&bar->slab_free[0], 1);
+    mbar_init(&bar->slab_free[1], 1);
     for (int i = 0; i < 2; ++i) {
       mbar_init(&bar->s_full[i], 1);
       mbar_init(&bar->s_empty[i], kSoftWarps);
       mbar_init(&bar->meta_full[i], 1);
     }
     mbar_init(&bar->p_full, kSoftWarps);
-    mbar_init(&bar->p_empty, 1);
     mbar_init(&bar->q_full, 1);
     mbar_init(&bar->q_empty, 1);
     mbar_init(&bar->o_empty, kSoftWarps);
     mbar_init(&bar->drain, 1);
-    mbar_init(&bar->grp_soft[0], 4);
-    mbar_init(&bar->grp_soft[1], 4);
     mbar_init(&bar->grp_prod, kProdWarps);
     fence_mbar_init();
   }
@@ -133,7 +134,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(
   const uint32_t tmem = bar->tmem_base;
 
   if (warp >= kSoftWarps && warp < kMmaWarp) {
-    // ======================= gather producer (128 threads) =====================
+    // ======================= gather producer (224 threads) =====================
     const int ptid = threadIdx.x - kSoftWarps * 32;
     const int pw = ptid >> 5;
     const int chunk = ptid & 7;
@@ -141,6 +142,9 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(
     uint32_t gphase = 0;
     int64_t q_issued = -1;  // last query whose Q load was issued
     bool ok = true;
+    // queries are read once; the entries and window rows are re-read by many
+    // queries and should stay in L2
+    const uint64_t pol_q = l2_policy_evict_first(), pol_kv = l2_policy_evict_last();
     for (int64_t kq = 0; ok; ++kq) {
       const int64_t qi = blockIdx.x + kq * gridDim.x;
       if (qi >= total) break;
@@ -198,7 +202,8 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(
         if (ok) {
           mbar_arrive_expect_tx(&bar->q_full, kSlabs * kQSlabBytes);
           for (int s = 0; s < kSlabs; ++s)
-            tma_load_3d(sQ + s * kQSlabBytes, &tm_q, &bar->q_full, s * 64, (int)(t * kNH), (int)b);
+            tma_load_3d_hint(sQ + s * kQSlabBytes, &tm_q, &bar->q_full, s * 64, (int)(t * kNH),
+                             (int)b, pol_q);
           q_issued = kq;
         }
       }
@@ -218,7 +223,8 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(
           src[rr] = p;
         }
         for (int s = 0; s < kSlabs; ++s) {
-          if (g >= 1 && !mbar_wait(&bar->slab_empty[s], (uint32_t)((g - 1) & 1), err)) {
+          if (g >= 1 && (s & 3) == 0 &&
+              !mbar_wait(&bar->slab_free[s >> 2], (uint32_t)((g - 1) & 1), err)) {
             ok = false;
             break;
           }
@@ -228,8 +234,8 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(
             const int row = (ptid >> 3) + kRowsPerPass * rr;
             if (row >= kTE) continue;
             const __nv_bfloat16* p = src[rr] != nullptr ? src[rr] + s * 64 + chunk * 8 : kv_win;
-            cp_async_16(dst + row * 128 + ((chunk ^ (row & 7)) * 16), p,
-                        src[rr] != nullptr ? 16u : 0u);
+            cp_async_16_hint(dst + row * 128 + ((chunk ^ (row & 7)) * 16), p,
+                             src[rr] != nullptr ? 16u : 0u, pol_kv);
           }
           cp_async_arrive_noinc(&bar->slab_full[s]);
         }
@@ -240,8 +246,8 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(
       mbar_wait(&bar->q_full, (uint32_t)(q_issued & 1), err, false);
   } else if (warp == kMmaWarp) {
     // ======================= MMA issuer (one lane) =============================
-    constexpr uint32_t kIdQK = idesc_bf16(kTE, kNH, 0, 0);
-    constexpr uint32_t kIdPV = idesc_bf16(128, kNH, 1, 1);
+    constexpr uint32_t kIdQK = idesc_bf16(kNH, kTE, 0, 0);   // Q K-major, K K-major
+    constexpr uint32_t kIdPV = idesc_bf16(kNH, 256, 0, 1);   // P K-major, V MN-major
     const uint32_t kv0 = smem_u32(sKV), q0 = smem_u32(sQ), p0 = smem_u32(sP);
     int g = 0;
     bool ok = true;
@@ -253,6 +259,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(
       if (!mbar_wait(&bar->q_full, (uint32_t)(kq & 1), err)) break;
       for (int tt = 0; tt < T; ++tt, ++g) {
         const int sb = g & 1;
+        // S buffer sb is free once the softmax has read it (tile g - 2)
         if (g >= 2 && !mbar_wait(&bar->s_empty[sb], (uint32_t)(((g >> 1) - 1) & 1), err)) {
           ok = false;
           break;
@@ -265,8 +272,9 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(
           if (lane == 0) {
 #pragma unroll
             for (int kk = 0; kk < 4; ++kk)
-              mma_bf16(tmem + kColS + sb * kNH, desc_sw128(kv0 + s * kSlabBytes + kk * 32),
-                       desc_sw128(q0 + s * kQSlabBytes + kk * 32), kIdQK,
+              mma_bf16(tmem + kLaneS + kColS + sb * kTE,
+                       desc_sw128(q0 + s * kQSlabBytes + kk * 32),
+                       desc_sw128(kv0 + s * kSlabBytes + kk * 32), kIdQK,
                        (s | kk) != 0 ? 1u : 0u);
           }
           __syncwarp();
@@ -284,17 +292,15 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(
         }
         tc_fence_after();
         if (lane == 0) {
-          for (int c = 0; c < 4; ++c) {
+          for (int hf = 0; hf < 2; ++hf) {  // dims 256 hf .. 256 hf + 255 = slabs 4 hf .. 4 hf + 3
 #pragma unroll
             for (int kk = 0; kk < kTE / 16; ++kk)
-              mma_bf16(tmem + kColO + c * kNH,
-                       desc_sw128_mn(kv0 + 2 * c * kSlabBytes + kk * 2048, kSlabBytes, 1024),
-                       desc_sw128_mn(p0 + kk * 2048, 1024, 1024), kIdPV,
-                       (tt == 0 && kk == 0) ? 0u : 1u);
-            mma_commit(&bar->slab_empty[2 * c]);
-            mma_commit(&bar->slab_empty[2 * c + 1]);
+              mma_bf16(tmem + kColO + hf * 256,
+                       desc_sw128(p0 + (kk >> 2) * kPSlabBytes + (kk & 3) * 32),
+                       desc_sw128_mn(kv0 + 4 * hf * kSlabBytes + kk * 2048, kSlabBytes, 1024),
+                       kIdPV, (tt == 0 && kk == 0) ? 0u : 1u);
+            mma_commit(&bar->slab_free[hf]);
           }
-          mma_commit(&bar->p_empty);
         }
         __syncwarp();
       }
@@ -303,132 +309,121 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(
     __syncwarp();
     mbar_wait(&bar->drain, 0, err, false);
   } else {
-    // ======================= softmax + epilogue (8 warps) ======================
-    const int quad = warp & 3, hh = warp >> 2;
-    const uint32_t lane_base = tmem + ((uint32_t)(quad * 32) << 16);
+    // ======================= softmax + epilogue (4 warps) ======================
+    // warp q: TMEM lane quarter q = heads 16 q .. 16 q + 15; thread (hl, ch):
+    // head 16 q + hl, columns 32 ch .. 32 ch + 31 of every 64-column load
+    const int hl = lane & 15, ch = lane >> 4;
+    const int hd = warp * 16 + hl;
+    const uint32_t o_lane = tmem + ((uint32_t)(warp * 32) << 16) + kColO;
+    const uint32_t s_lane = tmem + ((uint32_t)(warp * 32) << 16) + kLaneS + kColS;
     const float qscale = scale * kLog2e;
-    const int row = quad * 32 + lane;  // entry row within a tile / dim within a chunk
-    uint32_t gphase = 0;
     int g = 0;
     for (int64_t kq = 0;; ++kq) {
       const int64_t qi = blockIdx.x + kq * gridDim.x;
       if (qi >= total) break;
       if (!mbar_wait(&bar->meta_full[kq & 1], (uint32_t)((kq >> 1) & 1), err)) break;
       const AttnMeta mt = meta[kq & 1];
-      float m_run = kNegInf;  // lane i: running max (log2 units) of head hh*32+i
-      float psum[32];
-#pragma unroll
-      for (int i = 0; i < 32; ++i) psum[i] = 0.f;
+      float m_run = kNegInf;  // running max (log2 units) of head hd
+      float l_run = 0.f;      // this thread's share of the head's sum
       bool ok = true;
       for (int tt = 0; tt < mt.ntiles; ++tt, ++g) {
         const int sb = g & 1;
         if (!mbar_wait(&bar->s_full[sb], (uint32_t)((g >> 1) & 1), err)) { ok = false; break; }
         tc_fence_after();
-        const uint32_t s_addr = lane_base + kColS + sb * kNH + hh * 32;
-        const bool valid = tt * kTE + row < mt.nrows;
-        float v[32];
+        float lg[64];  // logits of columns 64 c + 32 ch + i, c = 0, 1
         {
           uint32_t r[32];
-          tmem_ld32(s_addr, r);
-          tmem_ld_wait();
+          const int nv = mt.nrows - tt * kTE;  // valid columns of this tile
 #pragma unroll
-          for (int i = 0; i < 32; ++i) v[i] = valid ? __uint_as_float(r[i]) * qscale : kNegInf;
-        }
-        float* rmax = red + ((sb * 2 + hh) * 4) * 32;
-        rmax[quad * 32 + lane] = transpose_reduce<true>(v);
-        if (!group_sync(&bar->grp_soft[hh], gphase, err)) { ok = false; break; }
-        const float mtile = fmaxf(fmaxf(rmax[lane], rmax[32 + lane]),
-                                  fmaxf(rmax[64 + lane], rmax[96 + lane]));
-        float m_new, f_lane = 1.f;
-        bool resc = false;
-        if (tt == 0) {
-          m_new = mtile;
-        } else {
-          resc = mtile > m_run + kRescaleLog2;
-          m_new = resc ? mtile : m_run;
-          f_lane = resc ? ex2(m_run - m_new) : 1.f;
-        }
-        m_run = m_new;
-        // the P^T buffer (and, for a rescale, O^T) is free once the previous P.V is done
-        if (g >= 1 && !mbar_wait(&bar->p_empty, (uint32_t)((g - 1) & 1), err)) { ok = false; break; }
-        tc_fence_after();
-        if (__any_sync(0xffffffffu, resc)) {
-          float f[32];
-#pragma unroll
-          for (int i = 0; i < 32; ++i) {
-            f[i] = __shfl_sync(0xffffffffu, f_lane, i);
-            psum[i] *= f[i];
-          }
-          for (int c = 0; c < 4; ++c) {
-            uint32_t o[32];
-            tmem_ld32(lane_base + kColO + c * kNH + hh * 32, o);
+          for (int c = 0; c < 2; ++c) {
+            tmem_ld16x64(s_lane + sb * kTE + c * 64, r);
             tmem_ld_wait();
 #pragma unroll
-            for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * f[i]);
-            tmem_st32(lane_base + kColO + c * kNH + hh * 32, o);
+            for (int i = 0; i < 32; ++i)
+              lg[c * 32 + i] = 64 * c + 32 * ch + i < nv ? __uint_as_float(r[i]) * qscale : kNegInf;
           }
-          tmem_st_wait();
         }
-        // the logits again (cheaper than holding them across the reductions)
-        uint32_t r[32];
-        tmem_ld32(s_addr, r);
-        tmem_ld_wait();
+        // the S buffer is free for the Q.K of tile g + 2
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(&bar->s_empty[sb]);
-        uint32_t pk[16];
+        float mx = kNegInf;
 #pragma unroll
-        for (int i = 0; i < 32; i += 2) {
-          float ma = __shfl_sync(0xffffffffu, m_run, i);
-          float mb = __shfl_sync(0xffffffffu, m_run, i + 1);
-          ma = ma == kNegInf ? 0.f : ma;
-          mb = mb == kNegInf ? 0.f : mb;
-          const float la = valid ? __uint_as_float(r[i]) * qscale : kNegInf;
-          const float lb = valid ? __uint_as_float(r[i + 1]) * qscale : kNegInf;
-          const float pa = ex2(la - ma), pb = ex2(lb - mb);
-          psum[i] += pa;
-          psum[i + 1] += pb;
-          pk[i >> 1] = pack_bf16x2(pa, pb);
+        for (int i = 0; i < 64; ++i) mx = fmaxf(mx, lg[i]);
+        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));  // the head's other half
+        float f = 1.f;
+        bool resc = false;
+        if (tt == 0) {
+          m_run = mx;
+        } else if (mx > m_run + kRescaleLog2) {
+          resc = true;
+          f = ex2(m_run - mx);
+          m_run = mx;
         }
-        uint8_t* prow = sP + row * 128;
+        // P (and, for a rescale, O) is free once the previous P.V is done
+        if (g >= 1 && !mbar_wait(&bar->slab_free[1], (uint32_t)((g - 1) & 1), err)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        if (__any_sync(0xffffffffu, resc)) {
+          l_run *= f;
+          for (int c = 0; c < kC / 64; ++c) {
+            uint32_t o[32];
+            tmem_ld16x64(o_lane + c * 64, o);
+            tmem_ld_wait();
 #pragma unroll
-        for (int j = 0; j < 4; ++j)
-          *reinterpret_cast<uint4*>(prow + (((hh * 4 + j) ^ (row & 7)) * 16)) =
-              make_uint4(pk[4 * j], pk[4 * j + 1], pk[4 * j + 2], pk[4 * j + 3]);
+            for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * f);
+            tmem_st16x64(o_lane + c * 64, o);
+          }
+          tmem_st_wait();
+        }
+        const float mref = m_run == kNegInf ? 0.f : m_run;
+#pragma unroll
+        for (int c = 0; c < 2; ++c) {
+          uint32_t pk[16];
+#pragma unroll
+          for (int i = 0; i < 32; i += 2) {
+            const float pa = ex2(lg[c * 32 + i] - mref), pb = ex2(lg[c * 32 + i + 1] - mref);
+            l_run += pa + pb;
+            pk[i >> 1] = pack_bf16x2(pa, pb);
+          }
+          uint8_t* prow = sP + c * kPSlabBytes + hd * 128;
+#pragma unroll
+          for (int j = 0; j < 4; ++j)
+            *reinterpret_cast<uint4*>(prow + (((4 * ch + j) ^ (hd & 7)) * 16)) =
+                make_uint4(pk[4 * j], pk[4 * j + 1], pk[4 * j + 2], pk[4 * j + 3]);
+        }
         fence_proxy_async();
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(&bar->p_full);
       }
       if (!ok) break;
-      // ---- epilogue: o = O^T / (sum_j p_j + 2^(sink - m)) ----------------------
-      if (!mbar_wait(&bar->p_empty, (uint32_t)((g - 1) & 1), err)) break;
+      // ---- epilogue: o = O / (sum_j p_j + 2^(sink - m)) -------------------------
+      if (!mbar_wait(&bar->slab_free[1], (uint32_t)((g - 1) & 1), err)) break;
       tc_fence_after();
-      float* rsum = red + (2 * 2 * 4 + hh * 4) * 32;
-      rsum[quad * 32 + lane] = transpose_reduce<false>(psum);
-      if (!group_sync(&bar->grp_soft[hh], gphase, err)) break;
-      const int h_lane = hh * 32 + lane;
-      const float tot = rsum[lane] + rsum[32 + lane] + rsum[64 + lane] + rsum[96 + lane];
+      const float l = l_run + __shfl_xor_sync(0xffffffffu, l_run, 16);
       const float mref = m_run == kNegInf ? 0.f : m_run;
-      const float z = sink != nullptr ? sink[h_lane] * kLog2e : kNegInf;
-      const float den = tot + (z == kNegInf ? 0.f : ex2(z - mref));
-      const float inv = 1.f / den;
-      __nv_bfloat16* ob = out + ((mt.b * n + mt.t) * kNH) * kC;
-      for (int c = 0; c < 4; ++c) {
+      const float z = sink != nullptr ? sink[hd] * kLog2e : kNegInf;
+      const float inv = 1.f / (l + (z == kNegInf ? 0.f : ex2(z - mref)));
+      __nv_bfloat16* ob = out + ((mt.b * n + mt.t) * kNH + hd) * kC + 32 * ch;
+      for (int c = 0; c < kC / 64; ++c) {
         uint32_t o[32];
-        tmem_ld32(lane_base + kColO + c * kNH + hh * 32, o);
+        tmem_ld16x64(o_lane + c * 64, o);
         tmem_ld_wait();
-        const int d = c * 128 + row;
+        uint32_t pk[16];
 #pragma unroll
-        for (int i = 0; i < 32; ++i) {
-          const float iv = __shfl_sync(0xffffffffu, inv, i);
-          ob[(int64_t)(hh * 32 + i) * kC + d] = __float2bfloat16_rn(__uint_as_float(o[i]) * iv);
-        }
+        for (int i = 0; i < 32; i += 2)
+          pk[i >> 1] = pack_bf16x2(__uint_as_float(o[i]) * inv, __uint_as_float(o[i + 1]) * inv);
+#pragma unroll
+        for (int j = 0; j < 4; ++j)
+          __stcs(reinterpret_cast<uint4*>(ob + c * 64 + 8 * j),  // streamed: not re-read
+                 make_uint4(pk[4 * j], pk[4 * j + 1], pk[4 * j + 2], pk[4 * j + 3]));
       }
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&bar->o_empty);
-      if (!group_sync(&bar->grp_soft[hh], gphase, err)) break;  // rsum is reused next query
     }
   }
   __syncwarp();
