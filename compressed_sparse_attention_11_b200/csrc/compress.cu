@@ -6,100 +6,294 @@
 // (CSA: m own-block rows of Za/Ca and m previous-block rows of Zb/Cb; the
 // first entry has no previous block), applied as Hadamard weights to C.
 //
-// HBM-streaming kernel: every input row is read exactly once, 16 bytes per
-// thread per row (8 dims), and the softmax is kept online in registers
-// (running max, running sum, running weighted sum per dim).  The 2m (or m)
-// rows of one entry are split over R adjacent lanes (R = 1 for CSA's 8 rows,
-// larger for HCA's 128) and merged with warp shuffles.
+// HBM-streaming kernels: every input row is read exactly once, 16 bytes per
+// thread per row (8 dims), lanes along the dims so that each load
+// instruction of a warp reads 512 contiguous bytes of one row.  Entries of
+// at most eight rows (CSA m <= 4) take one thread per (entry, 8-dim chunk)
+// with the softmax kept online in registers over its rows.  Larger row sets
+// are split over R warps of one block; a thread's rows are read in rounds of
+// four with all loads of a round issued before its arithmetic (a two-pass
+// softmax over registers), and the R partial states are merged through
+// shared memory.  A row whose logit equals the running maximum gets weight 1
+// exactly, so a single +inf logit selects its row.
 #include "common.cuh"
 #include "launch.h"
 
 namespace csa {
 
+namespace {
+
+// Eight elements of one row, raw, and the rows per thread per round.
 template <typename T>
-__global__ void __launch_bounds__(256) compress_kernel(
+struct Raw8;
+template <>
+struct Raw8<__nv_bfloat16> {
+  static constexpr int kSlots = 4;
+  uint4 u;
+  __device__ __forceinline__ void load(const __nv_bfloat16* p) {
+    u = __ldcs(reinterpret_cast<const uint4*>(p));
+  }
+  __device__ __forceinline__ float get(int q) const {
+    const uint32_t w = q < 2 ? u.x : q < 4 ? u.y : q < 6 ? u.z : u.w;
+    return __uint_as_float((q & 1) ? (w & 0xffff0000u) : (w << 16));
+  }
+};
+template <>
+struct Raw8<float> {
+  static constexpr int kSlots = 4;
+  float4 a, b;
+  __device__ __forceinline__ void load(const float* p) {
+    a = __ldcs(reinterpret_cast<const float4*>(p));
+    b = __ldcs(reinterpret_cast<const float4*>(p) + 1);
+  }
+  __device__ __forceinline__ float get(int q) const {
+    switch (q) {
+      case 0: return a.x;
+      case 1: return a.y;
+      case 2: return a.z;
+      case 3: return a.w;
+      case 4: return b.x;
+      case 5: return b.y;
+      case 6: return b.z;
+      default: return b.w;
+    }
+  }
+};
+
+// Softmax state of one dim over a set of rows: max logit M, sum of
+// exp(l - M) S, weighted sum A.  A row whose logit equals the max gets weight
+// 1 exactly, so a single +inf logit selects its row.
+struct Osm {
+  float M, S, A;
+};
+
+__device__ __forceinline__ Osm osm_combine(Osm x, Osm y) {
+  const float mn = fmaxf(x.M, y.M);
+  if (mn == kNegInf) return x;
+  const float fx = x.M >= mn ? 1.f : ex2((x.M - mn) * kLog2e);
+  const float fy = y.M >= mn ? 1.f : ex2((y.M - mn) * kLog2e);
+  return Osm{mn, x.S * fx + y.S * fy, x.A * fx + y.A * fy};
+}
+
+// Row j (0 <= j < rows) of entry i: own block rows first, then (CSA) the
+// previous block's rows.  Returns false for the previous block of entry 0.
+template <typename T>
+__device__ __forceinline__ bool row_ptrs(const T* ca, const T* cb, const T* za, const T* zb,
+                                         const float* ba, const float* bb, int64_t seq,
+                                         int64_t i, int j, int m, int c, int d0, const T*& cp,
+                                         const T*& zp, const float*& bp) {
+  if (j < m) {
+    const int64_t row = seq + i * m + j;
+    cp = ca + row * c + d0;
+    zp = za + row * c + d0;
+    bp = ba + (int64_t)j * c + d0;
+    return true;
+  }
+  if (i == 0) return false;
+  const int64_t row = seq + (i - 1) * m + (j - m);
+  cp = cb + row * c + d0;
+  zp = zb + row * c + d0;
+  bp = bb + (int64_t)(j - m) * c + d0;
+  return true;
+}
+
+// One round: rows j = r0 + stride * t, t < kSlots, of one entry and one
+// 8-dim chunk; all loads first, then the two-pass softmax into st[8].
+template <typename T>
+__device__ __forceinline__ void round_rows(const T* ca, const T* cb, const T* za, const T* zb,
+                                           const float* ba, const float* bb, int64_t seq,
+                                           int64_t i, int m, int rows, int c, int d0, int r0,
+                                           int stride, Osm st[8]) {
+  constexpr int kSlots = Raw8<T>::kSlots;
+  Raw8<T> cr[kSlots], zr[kSlots];
+  const float* bp[kSlots];
+  bool act[kSlots];
+#pragma unroll
+  for (int t = 0; t < kSlots; ++t) {
+    const int j = r0 + stride * t;
+    const T* cp = nullptr;
+    const T* zp = nullptr;
+    bp[t] = nullptr;
+    act[t] = j < rows && row_ptrs(ca, cb, za, zb, ba, bb, seq, i, j, m, c, d0, cp, zp, bp[t]);
+    if (act[t]) {
+      cr[t].load(cp);
+      zr[t].load(zp);
+    }
+  }
+  float bv[kSlots][8];
+#pragma unroll
+  for (int t = 0; t < kSlots; ++t) {
+    if (act[t]) {
+      load8(bp[t], bv[t]);
+    } else {
+#pragma unroll
+      for (int q = 0; q < 8; ++q) bv[t][q] = kNegInf;
+    }
+  }
+#pragma unroll
+  for (int q = 0; q < 8; ++q) {
+    float mx = kNegInf;
+#pragma unroll
+    for (int t = 0; t < kSlots; ++t)
+      if (act[t]) mx = fmaxf(mx, zr[t].get(q) + bv[t][q]);
+    float s = 0.f, a = 0.f;
+    if (mx != kNegInf) {
+#pragma unroll
+      for (int t = 0; t < kSlots; ++t) {
+        if (!act[t]) continue;
+        const float l = zr[t].get(q) + bv[t][q];
+        const float w = l >= mx ? 1.f : ex2((l - mx) * kLog2e);
+        s += w;
+        a = fmaf(w, cr[t].get(q), a);
+      }
+    }
+    st[q] = Osm{mx, s, a};
+  }
+}
+
+// Entries with at most eight rows: one thread per (entry, 8-dim chunk).
+template <typename T>
+__global__ void __launch_bounds__(256) compress_rows_kernel(
     const T* __restrict__ ca, const T* __restrict__ cb, const T* __restrict__ za,
     const T* __restrict__ zb, const float* __restrict__ ba, const float* __restrict__ bb,
-    int64_t n, int c, int m, int overlap, int64_t E, int r_log2, int64_t items,
-    T* __restrict__ out) {
+    int64_t n, int c, int m, int rows, int64_t E, int64_t items, T* __restrict__ out) {
   const int64_t g = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
-  const bool valid = g < items;
-  const int R = 1 << r_log2;
-  const int r = (int)(g & (R - 1));
-  int64_t rest = g >> r_log2;
+  if (g >= items) return;
   const int chunks = c >> 3;
-  const int chunk = (int)(rest % chunks);
-  rest /= chunks;
-  const int64_t i = rest % E;
-  const int64_t b = rest / E;
-  const int d0 = chunk * 8;
-
+  const int d0 = (int)(g % chunks) * 8;
+  const int64_t rest = g / chunks;
+  const int64_t i = rest % E, b = rest / E;
   float M[8], S[8], A[8];
 #pragma unroll
-  for (int q = 0; q < 8; ++q) { M[q] = kNegInf; S[q] = 0.f; A[q] = 0.f; }
-
-  if (valid) {
-    const int rows = overlap ? 2 * m : m;
-    const int64_t seq = b * n;
-    for (int j = r; j < rows; j += R) {
-      const T* cp;
-      const T* zp;
-      const float* bp;
-      if (j < m) {
-        const int64_t row = seq + i * m + j;
-        cp = ca + row * c + d0;
-        zp = za + row * c + d0;
-        bp = ba + (int64_t)j * c + d0;
-      } else {
-        if (i == 0) continue;  // previous block of entry 0: logits -inf, rows 0
-        const int64_t row = seq + (i - 1) * m + (j - m);
-        cp = cb + row * c + d0;
-        zp = zb + row * c + d0;
-        bp = bb + (int64_t)(j - m) * c + d0;
-      }
-      float cv[8], zv[8], bv[8];
-      load8(cp, cv);
-      load8(zp, zv);
-      load8(bp, bv);
-#pragma unroll
-      for (int q = 0; q < 8; ++q) osm_update(M[q], S[q], A[q], zv[q] + bv[q], cv[q]);
-    }
+  for (int q = 0; q < 8; ++q) {
+    M[q] = kNegInf;
+    S[q] = 0.f;
+    A[q] = 0.f;
   }
-  // merge the R partial states of this entry's rows
-  for (int off = 1; off < R; off <<= 1) {
+  for (int j = 0; j < rows; ++j) {
+    const T* cp;
+    const T* zp;
+    const float* bp;
+    if (!row_ptrs(ca, cb, za, zb, ba, bb, b * n, i, j, m, c, d0, cp, zp, bp)) continue;
+    float cv[8], zv[8], bv[8];
+    load8(cp, cv);
+    load8(zp, zv);
+    load8(bp, bv);
 #pragma unroll
     for (int q = 0; q < 8; ++q) {
-      const float m2 = __shfl_xor_sync(0xffffffffu, M[q], off);
-      const float s2 = __shfl_xor_sync(0xffffffffu, S[q], off);
-      const float a2 = __shfl_xor_sync(0xffffffffu, A[q], off);
-      osm_merge(M[q], S[q], A[q], m2, s2, a2);
+      const float l = zv[q] + bv[q];
+      if (l >= M[q]) {  // new maximum (or equal to it): weight 1 for this row
+        const float f = M[q] == l ? 1.f : ex2((M[q] - l) * kLog2e);
+        S[q] = S[q] * f + 1.f;
+        A[q] = A[q] * f + cv[q];
+        M[q] = l;
+      } else {
+        const float w = ex2((l - M[q]) * kLog2e);
+        S[q] += w;
+        A[q] = fmaf(w, cv[q], A[q]);
+      }
     }
   }
-  if (valid && r == 0) {
+  float o[8];
+#pragma unroll
+  for (int q = 0; q < 8; ++q) o[q] = A[q] / S[q];
+  store8(out + (b * E + i) * c + d0, o);
+}
+
+// Entries with more rows: block (32 chunks) x (R row groups); thread (lane, r)
+// reads rows r, r + R, r + 2R, ... of its chunk in rounds of four; the R
+// states are merged in shared memory.
+template <typename T>
+__global__ void __launch_bounds__(256) compress_split_kernel(
+    const T* __restrict__ ca, const T* __restrict__ cb, const T* __restrict__ za,
+    const T* __restrict__ zb, const float* __restrict__ ba, const float* __restrict__ bb,
+    int64_t n, int c, int m, int rows, int64_t E, int chunk_blocks, T* __restrict__ out) {
+  extern __shared__ float sh[];  // [3][R][8][32]
+  const int lane = threadIdx.x, r = threadIdx.y, R = blockDim.y;
+  const int cblk = (int)(blockIdx.x % chunk_blocks);
+  const int64_t ent = blockIdx.x / chunk_blocks;
+  const int64_t i = ent % E, b = ent / E;
+  const int chunks = c >> 3;
+  const int chunk = cblk * 32 + lane;
+  const bool valid = chunk < chunks;
+  const int d0 = valid ? chunk * 8 : 0;
+
+  Osm st[8];
+#pragma unroll
+  for (int q = 0; q < 8; ++q) st[q] = Osm{kNegInf, 0.f, 0.f};
+  if (valid) {
+    for (int r0 = r; r0 < rows; r0 += R * Raw8<T>::kSlots) {
+      Osm part[8];
+      round_rows(ca, cb, za, zb, ba, bb, b * n, i, m, rows, c, d0, r0, R, part);
+#pragma unroll
+      for (int q = 0; q < 8; ++q) st[q] = osm_combine(st[q], part[q]);
+    }
+  }
+  const int plane = R * 8 * 32;
+#pragma unroll
+  for (int q = 0; q < 8; ++q) {
+    const int at = (r * 8 + q) * 32 + lane;
+    sh[at] = st[q].M;
+    sh[plane + at] = st[q].S;
+    sh[2 * plane + at] = st[q].A;
+  }
+  __syncthreads();
+  // thread (lane, r) merges dims r, r + R, ... of its chunk over the R groups
+  float* res = sh;  // reused after the merge: [8][32]
+  float v[8];  // v[u]: dim r + u R
+  int nq = 0;
+  for (int q = r; q < 8; q += R, ++nq) {
+    Osm acc{kNegInf, 0.f, 0.f};
+    for (int u = 0; u < R; ++u) {
+      const int at = (u * 8 + q) * 32 + lane;
+      acc = osm_combine(acc, Osm{sh[at], sh[plane + at], sh[2 * plane + at]});
+    }
+    v[nq] = acc.A / acc.S;
+  }
+  __syncthreads();
+  for (int u = 0; u < nq; ++u) res[(r + u * R) * 32 + lane] = v[u];
+  __syncthreads();
+  if (r == 0 && valid) {
     float o[8];
 #pragma unroll
-    for (int q = 0; q < 8; ++q) o[q] = A[q] / S[q];
+    for (int q = 0; q < 8; ++q) o[q] = res[q * 32 + lane];
     store8(out + (b * E + i) * c + d0, o);
   }
 }
 
 template <typename T>
-static cudaError_t launch_compress_t(const void* ca, const void* cb, const void* za,
-                                     const void* zb, const float* ba, const float* bb,
-                                     int64_t batch, int64_t n, int c, int m, int overlap,
-                                     void* out, cudaStream_t s) {
+cudaError_t launch_compress_t(const void* ca, const void* cb, const void* za, const void* zb,
+                              const float* ba, const float* bb, int64_t batch, int64_t n, int c,
+                              int m, int overlap, void* out, cudaStream_t s) {
   const int64_t E = n / m;
   const int rows = overlap ? 2 * m : m;
-  // lanes per entry-chunk: about 8 rows per lane, at most 32
-  int r_log2 = 0;
-  while ((1 << r_log2) < 32 && (rows >> r_log2) > 8) ++r_log2;
-  const int64_t items = batch * E * (c / 8) << r_log2;
-  const int64_t blocks = (items + 255) / 256;
-  compress_kernel<T><<<(unsigned)blocks, 256, 0, s>>>(
-      (const T*)ca, (const T*)cb, (const T*)za, (const T*)zb, ba, bb, n, c, m, overlap, E,
-      r_log2, items, (T*)out);
+  if (batch * E == 0) return cudaSuccess;
+  if (rows <= 8) {
+    const int64_t items = batch * E * (c / 8);
+    compress_rows_kernel<T><<<(unsigned)((items + 255) / 256), 256, 0, s>>>(
+        (const T*)ca, (const T*)cb, (const T*)za, (const T*)zb, ba, bb, n, c, m, rows, E, items,
+        (T*)out);
+    return cudaGetLastError();
+  }
+  // R = groups of rows: one round per thread where possible, at most 8 groups
+  constexpr int kSlots = Raw8<T>::kSlots;
+  int R = 1;
+  while (R < 8 && R * kSlots < rows) R <<= 1;
+  const int chunk_blocks = (c / 8 + 31) / 32;
+  const size_t smem = (size_t)3 * R * 8 * 32 * sizeof(float);
+  auto kern = compress_split_kernel<T>;
+  if (smem > 48 * 1024) {
+    const cudaError_t e =
+        cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+  }
+  kern<<<(unsigned)(batch * E * chunk_blocks), dim3(32, R), smem, s>>>(
+      (const T*)ca, (const T*)cb, (const T*)za, (const T*)zb, ba, bb, n, c, m, rows, E,
+      chunk_blocks, (T*)out);
   return cudaGetLastError();
 }
+
+}  // namespace
 
 cudaError_t launch_compress(const void* ca, const void* cb, const void* za, const void* zb,
                             const float* ba, const float* bb, int64_t batch, int64_t n, int c,

@@ -345,7 +345,7 @@ __device__ void build_query_operand(const __nv_bfloat16* __restrict__ q,
     }
     if (act) {
       const int dd = hl * 8, ch = dd >> 4;
-      const int rh = h, rl = H + h;
+      const int rh = decode_qop_row(h, 0, H), rl = decode_qop_row(h, 1, H);
       *reinterpret_cast<uint2*>(rec + rh * 128 + ((ch ^ (rh & 7)) * 16) + (dd & 15)) =
           make_uint2(hi2[0], hi2[1]);
       *reinterpret_cast<uint2*>(rec + rl * 128 + ((ch ^ (rl & 7)) * 16) + (dd & 15)) =

@@ -72,39 +72,42 @@ struct DecIdxCfg {
   static_assert(TPP >= 1 && 2 * TPP * N <= 512, "two accumulator sets in TMEM");
 };
 
-__device__ __forceinline__ int tiles_of(const int64_t* pos, int64_t b, int m, int64_t cap) {
+// Tiles of tk keys of sequence b.
+__device__ __forceinline__ int tiles_of(const int64_t* pos, int64_t b, int m, int64_t cap,
+                                        int tk) {
   const int64_t t = pos[b];
   const int64_t V = t < 0 ? 0 : min((t + 1) / m, cap);
-  return (int)((V + kKeys - 1) / kKeys);
+  return (int)((V + tk - 1) / tk);
 }
 
 // Walks the CTA's tiles in order: sequence b, tile j of nt.
 struct TileWalk {
   int64_t b;
-  int j, nt;
-  __device__ void start(const int64_t* pos, int64_t b0, int j0, int m, int64_t cap) {
+  int j, nt, tk;
+  __device__ void start(const int64_t* pos, int64_t b0, int j0, int m, int64_t cap, int tk_) {
+    tk = tk_;
     b = b0;
     j = j0;
-    nt = tiles_of(pos, b0, m, cap);
+    nt = tiles_of(pos, b0, m, cap, tk);
   }
   __device__ void next(const int64_t* pos, int64_t batch, int m, int64_t cap) {
     if (++j < nt) return;
     j = 0;
     do {
       ++b;
-      nt = b < batch ? tiles_of(pos, b, m, cap) : 1;
+      nt = b < batch ? tiles_of(pos, b, m, cap, tk) : 1;
     } while (nt == 0);
   }
 };
 
 // Warp 0: this CTA's contiguous share [g0, g1) of the flattened tile list
 // and the sequence / tile where it starts.
-__device__ void locate_range(const int64_t* pos, int64_t batch, int m, int64_t cap,
+__device__ void locate_range(const int64_t* pos, int64_t batch, int m, int64_t cap, int tk,
                              int64_t& b0, int& j0, int& count) {
   const int lane = threadIdx.x & 31;
   int64_t total = 0;
   for (int64_t base = 0; base < batch; base += 32) {
-    int64_t nt = base + lane < batch ? tiles_of(pos, base + lane, m, cap) : 0;
+    int64_t nt = base + lane < batch ? tiles_of(pos, base + lane, m, cap, tk) : 0;
 #pragma unroll
     for (int off = 16; off > 0; off >>= 1) nt += __shfl_xor_sync(0xffffffffu, nt, off);
     total += nt;
@@ -116,7 +119,7 @@ __device__ void locate_range(const int64_t* pos, int64_t batch, int m, int64_t c
   if (count == 0) return;
   int64_t run = 0;
   for (int64_t base = 0; base < batch; base += 32) {
-    const int64_t nt = base + lane < batch ? tiles_of(pos, base + lane, m, cap) : 0;
+    const int64_t nt = base + lane < batch ? tiles_of(pos, base + lane, m, cap, tk) : 0;
     int64_t inc = nt;
 #pragma unroll
     for (int off = 1; off < 32; off <<= 1) {
@@ -175,7 +178,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_index_tc_kernel(
     }
     int64_t b0;
     int j0, count;
-    locate_range(pos, batch, m, cap, b0, j0, count);
+    locate_range(pos, batch, m, cap, kKeys, b0, j0, count);
     if (lane == 0) {
       bar->b0 = b0;
       bar->j0 = j0;
@@ -203,7 +206,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_index_tc_kernel(
   if (warp == 0 && live) {
     // ------------------------------- TMA producer --------------------------------
     TileWalk it;
-    it.start(pos, b0, j0, m, cap);
+    it.start(pos, b0, j0, m, cap, kKeys);
     int k = 0;
     for (; k < npairs; ++k) {
       const int s = k % S;
@@ -224,7 +227,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_index_tc_kernel(
     constexpr uint32_t kIdesc = idesc_e4m3(kKeys, C::N);
     const uint32_t a0 = smem_u32(sRaw), bb0 = smem_u32(sB);
     TileWalk it;
-    it.start(pos, b0, j0, m, cap);
+    it.start(pos, b0, j0, m, cap, kKeys);
     int u = -1;  // sequence counter within the range
     bool ok = true;
     for (int k = 0; k < npairs && ok; ++k) {
@@ -264,7 +267,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_index_tc_kernel(
   } else if (warp == 2 && live) {
     // ----------- query operands: one bulk copy each, per sequence of the range -----------
     TileWalk it;
-    it.start(pos, b0, j0, m, cap);
+    it.start(pos, b0, j0, m, cap, kKeys);
     int left = count;
     constexpr uint32_t kRec = (uint32_t)(C::B_BYTES + H * 4);
     for (int u = 0; left > 0; ++u) {
@@ -297,7 +300,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_index_tc_kernel(
     const uint32_t lane_addr = tmem + ((uint32_t)(quad * 32) << 16);
     auto mine_of = [&](int i) { return TPP == 2 ? (i & 1) == grp : ((i / TPP) & 1) == grp; };
     TileWalk it;
-    it.start(pos, b0, j0, m, cap);
+    it.start(pos, b0, j0, m, cap, kKeys);
     int64_t V = 0;
     // key scale of this group's next tile, loaded a tile ahead
     auto scale_of = [&](const TileWalk& w) -> float {
@@ -374,6 +377,298 @@ __global__ void __launch_bounds__(kThreads, 1) decode_index_tc_kernel(
   }
 }
 
+// ---------------------------------------------------------------------------
+// 64 heads: the query operand on the M side.  Its 128 rows (64 heads x hi,
+// lo) come in blocks of 16: rows 0-7 the hi halves and rows 8-15 the lo
+// halves of 8 heads, so that one 16-lane x 256-bit TMEM load gives a thread
+// the hi and the lo accumulator of the same head and keys.  One M = 128 x
+// N = 256 keys x K = 128 tile is four MMAs, half the instructions per key of
+// the keys-on-M form.  The epilogue (four warps per tile, two groups taking
+// alternate tiles) adds hi and lo, applies ReLU and the head weights of the
+// thread's two heads, sums over the 8 lanes that hold the same keys by a
+// shuffle reduce-scatter and over the four warps in shared memory, then
+// scales by the key scale.
+// ---------------------------------------------------------------------------
+constexpr int kSwH = 64;
+constexpr int kSwKeys = 256;                        // keys per tile (MMA N)
+constexpr int kSwTileBytes = kSwKeys * kCI;         // 32 KB, one ring stage
+constexpr int kSwABytes = 2 * kSwH * 128;           // query operand, 16 KB
+constexpr int kSwRedBytes = 2 * 2 * 4 * kSwKeys * 4;  // [group][buffer][warp][key] fp32
+constexpr int kSwStages =
+    (kSmemLimit - 2048 - kBSlots * kSwABytes - kWSlots * kSwH * 4 - kSwRedBytes) / kSwTileBytes;
+constexpr int kSwOffA = kSwStages * kSwTileBytes;
+constexpr int kSwOffW = kSwOffA + kBSlots * kSwABytes;
+constexpr int kSwOffRed = kSwOffW + kWSlots * kSwH * 4;
+constexpr int kSwOffBar = kSwOffRed + kSwRedBytes;
+constexpr int kSwSmem = kSwOffBar + (int)sizeof(DecIdxBars<kSwStages>) + 1024;
+static_assert(kSwStages >= 4 && kSwSmem <= kSmemLimit, "shared memory budget");
+static_assert(kSwABytes + kSwH * 4 == 64 * (2 * 128 + 4), "query operand record");
+
+// Sum of v over the 8 lanes that share lane % 4, reduce-scattered: on
+// return v[0] holds entry (lane / 4) % 8 of the 8 summed.
+__device__ __forceinline__ void reduce_scatter8(float (&v)[8], int lane) {
+#pragma unroll
+  for (int w = 4, sh = 16; w >= 1; w >>= 1, sh >>= 1) {
+    const bool up = (lane & sh) != 0;
+#pragma unroll
+    for (int i = 0; i < w; ++i) {
+      const float send = up ? v[i] : v[i + w];
+      const float keep = up ? v[i + w] : v[i];
+      v[i] = keep + __shfl_xor_sync(0xffffffffu, send, sh);
+    }
+  }
+}
+
+__global__ void __launch_bounds__(kThreads, 1) decode_index_sw_kernel(
+    const __grid_constant__ CUtensorMap tm_keys, const float* __restrict__ key_scale,
+    const uint8_t* __restrict__ qop, const int64_t* __restrict__ pos, int64_t batch, int64_t cap,
+    int m, float* __restrict__ scores, unsigned int* __restrict__ err) {
+  constexpr int S = kSwStages;
+  using namespace sm100;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = smem_raw + ((1024 - (smem_u32(smem_raw) & 1023)) & 1023);
+  uint8_t* sRaw = smem;
+  uint8_t* sA = smem + kSwOffA;
+  float* sW = reinterpret_cast<float*>(smem + kSwOffW);
+  float* sRed = reinterpret_cast<float*>(smem + kSwOffRed);
+  DecIdxBars<S>* bar = reinterpret_cast<DecIdxBars<S>*>(smem + kSwOffBar);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      for (int s = 0; s < S; ++s) {
+        mbar_init(&bar->full[s], 1);
+        mbar_init(&bar->empty[s], 1);
+      }
+      for (int q = 0; q < 2; ++q) {
+        mbar_init(&bar->d_full[q], 1);
+        mbar_init(&bar->d_empty[q], 4);  // the four warps of the tile's group
+      }
+      for (int u = 0; u < kBSlots; ++u) {
+        mbar_init(&bar->b_full[u], 1);
+        mbar_init(&bar->b_empty[u], 1);  // the MMAs of the sequence's last tile
+      }
+      for (int u = 0; u < kWSlots; ++u) {
+        mbar_init(&bar->w_full[u], 1);
+        mbar_init(&bar->w_empty[u], 8);  // every epilogue warp, once per sequence
+      }
+      mbar_init(&bar->drain, 1);
+      fence_mbar_init();
+      tma_prefetch_desc(&tm_keys);
+    }
+    int64_t b0;
+    int j0, count;
+    locate_range(pos, batch, m, cap, kSwKeys, b0, j0, count);
+    if (lane == 0) {
+      bar->b0 = b0;
+      bar->j0 = j0;
+      bar->count = count;
+    }
+  } else if (warp == 1) {
+    tmem_alloc(&bar->tmem_base, 512);
+    tmem_relinquish();
+  }
+  // everything above is set-up; the cache (the emitted key) is written by the
+  // previous kernel
+  pdl_wait();
+  pdl_trigger();
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = bar->tmem_base;
+  const int count = bar->count;
+  const int64_t b0 = bar->b0;
+  const int j0 = bar->j0;
+  const bool live = count > 0 && flag_value(err) == 0;
+
+  if (warp == 0 && live) {
+    // ------------------------------- TMA producer --------------------------------
+    TileWalk it;
+    it.start(pos, b0, j0, m, cap, kSwKeys);
+    int i = 0;
+    for (; i < count; ++i, it.next(pos, batch, m, cap)) {
+      const int s = i % S;
+      if (i >= S && !mbar_wait(&bar->empty[s], (uint32_t)(((i / S) - 1) & 1), err)) break;
+      if (lane == 0) {
+        mbar_arrive_expect_tx(&bar->full[s], kSwTileBytes);
+        tma_load_3d(sRaw + s * kSwTileBytes, &tm_keys, &bar->full[s], 0, it.j * kSwKeys,
+                    (int)it.b);
+      }
+      __syncwarp();
+    }
+    // every issued stage has landed before the CTA exits
+    for (int r = (i > S ? i - S : 0); r < i; ++r)
+      mbar_wait(&bar->full[r % S], (uint32_t)((r / S) & 1), err, false);
+  } else if (warp == 1 && live) {
+    // ------------------------------- MMA issuer ----------------------------------
+    constexpr uint32_t kIdesc = idesc_e4m3(2 * kSwH, kSwKeys);
+    const uint32_t raw0 = smem_u32(sRaw), a0 = smem_u32(sA);
+    TileWalk it;
+    it.start(pos, b0, j0, m, cap, kSwKeys);
+    int u = -1;  // sequence counter within the range
+    for (int i = 0; i < count; ++i, it.next(pos, batch, m, cap)) {
+      const int s = i % S, q = i & 1;
+      if (!mbar_wait(&bar->full[s], (uint32_t)((i / S) & 1), err)) break;
+      if (i >= 2 && !mbar_wait(&bar->d_empty[q], (uint32_t)(((i >> 1) - 1) & 1), err)) break;
+      if (i == 0 || it.j == 0) {
+        ++u;
+        if (!mbar_wait(&bar->b_full[u & 1], (uint32_t)((u >> 1) & 1), err)) break;
+      }
+      tc_fence_after();
+      if (lane == 0) {
+        const uint32_t aslot = a0 + (u & 1) * kSwABytes;
+        const uint32_t bt = raw0 + s * kSwTileBytes;
+#pragma unroll
+        for (int kk = 0; kk < kCI / 32; ++kk)  // K = 32 bytes per instruction
+          mma_f8(tmem + q * kSwKeys, desc_sw128(aslot + kk * 32), desc_sw128(bt + kk * 32),
+                 kIdesc, kk > 0 ? 1u : 0u);
+        if (i + 1 == count || it.j + 1 == it.nt) mma_commit(&bar->b_empty[u & 1]);
+        mma_commit(&bar->d_full[q]);
+        mma_commit(&bar->empty[s]);
+      }
+      __syncwarp();
+    }
+    if (lane == 0) mma_commit(&bar->drain);
+    __syncwarp();
+    mbar_wait(&bar->drain, 0, err, false);
+  } else if (warp == 2 && live) {
+    // ----------- query operands: one bulk copy each, per sequence of the range -----------
+    TileWalk it;
+    it.start(pos, b0, j0, m, cap, kSwKeys);
+    int left = count;
+    constexpr uint32_t kRec = (uint32_t)(kSwABytes + kSwH * 4);
+    for (int u = 0; left > 0; ++u) {
+      const int64_t b = it.b;
+      const int here = min(left, it.nt - it.j);
+      const int slot = u & 1, ws = u % kWSlots;
+      if (u >= kBSlots && !mbar_wait(&bar->b_empty[slot], (uint32_t)(((u >> 1) - 1) & 1), err))
+        break;
+      if (u >= kWSlots &&
+          !mbar_wait(&bar->w_empty[ws], (uint32_t)(((u / kWSlots) - 1) & 1), err))
+        break;
+      if (lane == 0) {
+        const uint8_t* rec = qop + b * kRec;
+        mbar_arrive_expect_tx(&bar->b_full[slot], kSwABytes);
+        bulk_load(sA + slot * kSwABytes, rec, kSwABytes, &bar->b_full[slot]);
+        mbar_arrive_expect_tx(&bar->w_full[ws], kSwH * 4);
+        bulk_load(sW + ws * kSwH, rec + kSwABytes, kSwH * 4, &bar->w_full[ws]);
+      }
+      __syncwarp();
+      left -= here;
+      for (int r = 0; r < here; ++r) it.next(pos, batch, m, cap);
+    }
+  } else if (warp >= 4 && live) {
+    // ---- epilogue: group grp takes the tiles i with i % 2 == grp (accumulator grp) ----
+    const int wq = warp & 3, grp = (warp - 4) >> 2;
+    // this thread's heads: 16 wq + lane / 4 (TMEM lanes 32 wq + lane / 4 and
+    // + 8) and 16 wq + 8 + lane / 4 (lanes 32 wq + 16 + lane / 4 and + 8)
+    const int head_a = wq * 16 + (lane >> 2), head_b = head_a + 8;
+    const uint32_t acc_a = tmem + ((uint32_t)(wq * 32) << 16) + (uint32_t)(grp * kSwKeys);
+    const uint32_t acc_b = acc_a + (16u << 16);
+    // key of each 32-key chunk that this lane holds after the reduce-scatter
+    const int vk = (lane >> 2) & 7;
+    const int key_in_chunk = 8 * (vk >> 1) + 2 * (lane & 3) + (vk & 1);
+    float* red_g = sRed + grp * (2 * 4 * kSwKeys);
+    const int p = wq * 32 + lane;  // this thread's key pair in the final sum
+    TileWalk it;
+    it.start(pos, b0, j0, m, cap, kSwKeys);
+    int64_t V = 0;
+    int u = -1, mine = 0;
+    for (int i = 0; i < count; ++i, it.next(pos, batch, m, cap)) {
+      if (i == 0 || it.j == 0) {
+        ++u;
+        V = min((pos[it.b] + 1) / m, cap);
+      }
+      const bool seq_end = i + 1 == count || it.j + 1 == it.nt;
+      if ((i & 1) == grp) {
+        // key scales of this thread's two keys, ahead of the accumulator
+        const int64_t s0 = (int64_t)it.j * kSwKeys + 2 * p;
+        const float* ksp = key_scale + it.b * cap + s0;
+        const float ks0 = s0 < V ? __ldcs(ksp) : 0.f;
+        const float ks1 = s0 + 1 < V ? __ldcs(ksp + 1) : 0.f;
+        const bool ok =
+            mbar_wait(&bar->w_full[u % kWSlots], (uint32_t)((u / kWSlots) & 1), err) &&
+            mbar_wait(&bar->d_full[grp], (uint32_t)(mine & 1), err);
+        float* red = red_g + (mine & 1) * (4 * kSwKeys) + wq * kSwKeys;
+        if (ok) {
+          const float* wr = sW + (u % kWSlots) * kSwH;
+          const float wa = wr[head_a], wb = wr[head_b];  // w_h s_h
+          tc_fence_after();
+#pragma unroll 1
+          for (int c = 0; c < 4; ++c) {  // 64 keys per pass
+            uint32_t ra[32], rb[32];
+            tmem_ld16x256_x8(acc_a + c * 64, ra);
+            tmem_ld16x256_x8(acc_b + c * 64, rb);
+            tmem_ld_wait();
+            if (c == 3) {  // the accumulator is free for the tile after next
+              tc_fence_before();
+              __syncwarp();
+              if (lane == 0) mbar_arrive(&bar->d_empty[grp]);
+            }
+#pragma unroll
+            for (int half = 0; half < 2; ++half) {  // 32-key chunk 2 c + half
+              float v[8];
+#pragma unroll
+              for (int k = 0; k < 4; ++k) {
+#pragma unroll
+                for (int e = 0; e < 2; ++e) {
+                  const int r = 4 * (4 * half + k);
+                  const float ha = __uint_as_float(ra[r + e]) + __uint_as_float(ra[r + 2 + e]);
+                  const float hb = __uint_as_float(rb[r + e]) + __uint_as_float(rb[r + 2 + e]);
+                  v[2 * k + e] = fmaf(wa, fmaxf(ha, 0.f), wb * fmaxf(hb, 0.f));
+                }
+              }
+              reduce_scatter8(v, lane);
+              red[(2 * c + half) * 32 + key_in_chunk] = v[0];
+            }
+          }
+        }
+        // a failed wait set the error flag; the group leaves together
+        if (named_bar_or(1 + grp, 128, !ok)) break;
+        const float* rs = red_g + (mine & 1) * (4 * kSwKeys) + 2 * p;
+        float2 sum = *reinterpret_cast<const float2*>(rs);
+#pragma unroll
+        for (int w = 1; w < 4; ++w) {
+          const float2 x = *reinterpret_cast<const float2*>(rs + w * kSwKeys);
+          sum.x += x.x;
+          sum.y += x.y;
+        }
+        float* out = scores + it.b * cap + s0;
+        if (s0 < V) __stcg(out, sum.x * ks0);
+        if (s0 + 1 < V) __stcg(out + 1, sum.y * ks1);
+        ++mine;
+      }
+      if (seq_end) {  // both groups release the sequence's weights once they pass its end
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bar->w_empty[u % kWSlots]);
+      }
+    }
+  }
+  __syncwarp();
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+cudaError_t launch_sw(const csa_cache_desc& d, const CacheView& cv, const int64_t* pos,
+                      const uint8_t* qop, float* scores, unsigned int* err, cudaStream_t s) {
+  CUtensorMap tk;
+  if (!make_tmap_3d(&tk, cv.ikey_fp8, 1, kCI, (uint64_t)d.capacity, (uint64_t)d.batch, kCI,
+                    (uint64_t)d.capacity * kCI, kCI, kSwKeys))
+    return cudaErrorInvalidValue;
+  cudaError_t e = cudaFuncSetAttribute(decode_index_sw_kernel,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize, kSwSmem);
+  if (e != cudaSuccess) return e;
+  const int64_t max_tiles = d.batch * ((d.capacity + kSwKeys - 1) / kSwKeys);
+  const unsigned grid = (unsigned)std::max<int64_t>(1, std::min<int64_t>(sm_count(), max_tiles));
+  return launch_pdl(decode_index_sw_kernel, dim3(grid), dim3(kThreads), (size_t)kSwSmem, s, tk,
+                    (const float*)cv.ikey_scale, qop, pos, (int64_t)d.batch, (int64_t)d.capacity,
+                    d.m, scores, err);
+}
+
 template <int H>
 cudaError_t launch_h(const csa_cache_desc& d, const CacheView& cv, const int64_t* pos,
                      const uint8_t* qop, float* scores, unsigned int* err, cudaStream_t s) {
@@ -402,7 +697,7 @@ cudaError_t launch_decode_index_tc(const csa_cache_desc& d, const CacheView& cv,
                                    const int64_t* pos, const uint8_t* qop, float* scores,
                                    unsigned int* err, cudaStream_t s) {
   switch (d.nh_i) {
-    case 64: return launch_h<64>(d, cv, pos, qop, scores, err, s);
+    case 64: return launch_sw(d, cv, pos, qop, scores, err, s);
     case 128: return launch_h<128>(d, cv, pos, qop, scores, err, s);
     default: return cudaErrorInvalidValue;
   }

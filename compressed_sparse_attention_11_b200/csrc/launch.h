@@ -62,6 +62,15 @@ bool decode_index_tc_supported(const csa_cache_desc& d);
 // Bytes of one sequence's indexer query operand: the swizzled hi / lo E4M3
 // image (2 H rows of 128 bytes) followed by H fp32 weights.
 __host__ __device__ inline size_t decode_qop_bytes(int nh_i) { return (size_t)nh_i * (2 * 128 + 4); }
+// Row of head h's hi (part 0) or lo (part 1) FP8 half in the query operand.
+// With 64 heads the operand is the M side of the indexer MMA and its rows
+// are ordered for the 16-lane TMEM loads of the epilogue: in each block of 16
+// rows, rows 0-7 hold the hi halves and rows 8-15 the lo halves of 8 heads
+// (row 16 (h / 8) + 8 part + h % 8).  Otherwise the H hi rows come first,
+// then the H lo rows.
+__host__ __device__ inline int decode_qop_row(int h, int part, int H) {
+  return H == 64 ? ((h >> 3) << 4) + (part << 3) + (h & 7) : part * H + h;
+}
 // qop: [batch] query operands (written by the append step); scores
 // [batch][capacity] fp32, written for s < V of each sequence.
 cudaError_t launch_decode_index_tc(const csa_cache_desc& d, const CacheView& cv,

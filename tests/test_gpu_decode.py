@@ -166,6 +166,14 @@ def test_decode_csa_realistic_dims_two_chunks():
     _run_and_compare(w, B=2, E=2500, steps=4, seed=10)
 
 
+def test_decode_csa_128_index_heads():
+    """128 indexer heads: the query operand fills N = 256 of the keys-on-M
+    indexer form (64 heads use the heads-on-M form)."""
+    w = G.Decode("csa_decode_h128", 3, 0, 512, 64, 4, 64, 128, False, nh_i=128, c_i=128, k=256,
+                 seed=109)
+    _run_and_compare(w, B=3, E=1300, steps=3, seed=16)
+
+
 def test_decode_hca_realistic_dims_split_k():
     """64 heads x 512, FP8/bf16 cache, dense over ~300 entries: the tensor-core
     attention splits the entry set over several CTAs and a combine kernel."""

@@ -34,6 +34,9 @@ def _streams(B, n, c, m, dt, seed, overlap=True):
     (1, 4100, 512, 4, torch.bfloat16),
     (3, 64, 8, 4, torch.float32),         # narrowest dim
     (1, 7, 16, 4, torch.bfloat16),        # one entry + tail
+    (1, 1030, 136, 8, torch.bfloat16),    # 16 rows per entry: rows split over thread groups
+    (2, 2048 + 64, 512, 64, torch.bfloat16),  # 128 rows: two rounds per thread
+    (1, 512, 40, 16, torch.float32),      # fp32, 32 rows, 5 chunks
 ])
 def test_csa_compress_parity(B, n, c, m, dt):
     s = _streams(B, n, c, m, dt, seed=11)
@@ -51,6 +54,8 @@ def test_csa_compress_parity(B, n, c, m, dt):
     (1, 640, 64, 128, torch.float32),
     (1, 300, 32, 1, torch.float32),       # m = 1: identity
     (1, 96, 16, 32, torch.bfloat16),
+    (1, 2048 + 5, 264, 512, torch.bfloat16),  # 512 rows: eight rounds per thread, 33 chunks
+    (2, 40, 24, 5, torch.bfloat16),       # odd m within one round
 ])
 def test_hca_compress_parity(B, n, c, m, dt):
     s = _streams(B, n, c, m, dt, seed=12, overlap=False)
@@ -62,6 +67,25 @@ def test_hca_compress_parity(B, n, c, m, dt):
         check_close(out[b], ref, dt, f"hca compress b={b}")
     if m == 1:
         assert torch.equal(host(out), s["ca"])
+
+
+@pytest.mark.parametrize("overlap,m,c", [(True, 4, 512), (False, 128, 512), (True, 64, 136)])
+def test_compress_single_infinite_logit_copies_its_row(overlap, m, c):
+    """One logit at +inf (every dim of one own-block row per entry) takes all
+    the weight: the entry is that row of C, bit for bit."""
+    n = 64 * m
+    s = _streams(1, n, c, m, torch.bfloat16, seed=14, overlap=overlap)
+    E = n // m
+    pick = np.random.default_rng(14).integers(0, m, E)
+    rows = np.arange(E) * m + pick
+    s["za"][0, rows] = float("inf")
+    d = {k: v.to(DEV) for k, v in s.items()}
+    if overlap:
+        out = csa.csa_compress(d["ca"], d["cb"], d["za"], d["zb"], d["ba"], d["bb"], m)
+    else:
+        out = csa.csa_compress(d["ca"], None, d["za"], None, d["ba"], None, m)
+    torch.cuda.synchronize()
+    assert torch.equal(host(out)[0], s["ca"][0, rows])
 
 
 def test_compress_empty_and_short():
