@@ -366,9 +366,11 @@ __global__ void __launch_bounds__(1024) append_emit_kernel(csa_cache_desc d, Cac
   // the previous step's kernels read the window slot this token overwrites
   sm100::pdl_wait();
   sm100::pdl_trigger();
-  if (qop != nullptr)  // the indexer's query operand, for every sequence
+  if (blockIdx.y == 1) {  // the indexer's query operand, for every sequence
     build_query_operand(q_i + b * d.nh_i * 128, w_i + b * d.nh_i, d.nh_i,
                         qop + b * decode_qop_bytes(d.nh_i));
+    return;
+  }
   const int64_t t = pos[b];
   if (t < 0) return;  // no token for this sequence
   append_rows(d, cv, rows, b, t);
@@ -705,13 +707,17 @@ cudaError_t launch_decode_step(const csa_cache_desc& d, const CacheView& cv, con
   float* part_o = reinterpret_cast<float*>(wb + w.part_o);
   float* part_ms = reinterpret_cast<float*>(wb + w.part_ms);
 
-  // one thread per emitted dim (c + c_i of them), 256 to 1024 threads
+  // one thread per emitted dim (c + c_i of them), 256 to 1024 threads; with
+  // the indexer's query operand, a second block per sequence builds it (one
+  // half-warp per head)
   const int dims = d.c + (d.is_hca ? 0 : d.c_i);
-  const unsigned emit_threads = (unsigned)std::min(1024, std::max(256, (dims + 31) / 32 * 32));
-  const size_t emit_smem = sizeof(float) * (dims + 32);
   uint8_t* qop = w.tc_index ? wb + w.qop : nullptr;
-  cudaError_t err = launch_pdl(append_emit_kernel, dim3((unsigned)d.batch), dim3(emit_threads),
-                               emit_smem, s, d, cv, pos, rows, p,
+  const int want = std::max(dims, qop != nullptr ? d.nh_i * 16 : 0);
+  const unsigned emit_threads = (unsigned)std::min(1024, std::max(256, (want + 31) / 32 * 32));
+  const size_t emit_smem = sizeof(float) * (dims + 32);
+  cudaError_t err = launch_pdl(append_emit_kernel,
+                               dim3((unsigned)d.batch, qop != nullptr ? 2u : 1u),
+                               dim3(emit_threads), emit_smem, s, d, cv, pos, rows, p,
                                (const __nv_bfloat16*)q_i, w_i, qop);
   if (err != cudaSuccess) return err;
   if (!d.is_hca && w.tc_index) {

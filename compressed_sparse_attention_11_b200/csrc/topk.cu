@@ -55,7 +55,10 @@ constexpr int kRowBins = 2048;
 constexpr int kRowBinBits = 11;
 constexpr int kRowBinsPerThread = kRowBins / kRowThreads;  // 4
 constexpr int kRowCand = 256;                              // bin-T keys ranked directly (3 CTAs per SM at 16K keys)
-constexpr int64_t kRowMaxKeys = 40960;                     // keys staged per row
+constexpr int64_t kRowMaxKeys = 32768;                     // keys staged per row
+// 32-key groups of one warp's compaction segment (two masks each in the histogram)
+constexpr int kRowMaxGroups = (int)((kRowMaxKeys / kRowWarps + 31) / 32);
+static_assert(2 * kRowMaxGroups * kRowWarps <= kRowBins, "masks fit in the histogram");
 
 struct __align__(16) RowTopkShared {
   uint32_t hist[kRowBins];
@@ -118,11 +121,16 @@ __global__ void __launch_bounds__(kRowThreads) topk_rows_staged_kernel(
   }
   if (tid == 0) sh.cand_n = 0u;
   __syncthreads();
-  uint32_t kmin = 0xffffffffu, kmax = 0u;
-  for (int w = 0; w < kRowWarps; ++w) {
-    kmin = min(kmin, sh.wred[0][w]);
-    kmax = max(kmax, sh.wred[1][w]);
+  // the 16 warps' extremes, reduced by shuffles in every warp
+  uint32_t kmin = lane < kRowWarps ? sh.wred[0][lane] : 0xffffffffu;
+  uint32_t kmax = lane < kRowWarps ? sh.wred[1][lane] : 0u;
+#pragma unroll
+  for (int off = 8; off > 0; off >>= 1) {
+    kmin = min(kmin, __shfl_xor_sync(0xffffffffu, kmin, off));
+    kmax = max(kmax, __shfl_xor_sync(0xffffffffu, kmax, off));
   }
+  kmin = __shfl_sync(0xffffffffu, kmin, 0);
+  kmax = __shfl_sync(0xffffffffu, kmax, 0);
   // 2. radix refinement of the window [base, base + 2048 << shift)
   uint32_t base = kmin, need = (uint32_t)k;
   int shift = (int)bit_length(kmax - kmin) - kRowBinBits;
@@ -158,7 +166,16 @@ __global__ void __launch_bounds__(kRowThreads) topk_rows_staged_kernel(
       if (lane == 31) sh.wred[0][warp] = inc;
       __syncthreads();
       uint32_t acc = inc - loc;
-      for (int w = 0; w < warp; ++w) acc += sh.wred[0][w];
+      {  // plus the totals of the warps before this one (a 16-lane scan)
+        uint32_t wt = lane < kRowWarps ? sh.wred[0][lane] : 0u;
+#pragma unroll
+        for (int off = 1; off < kRowWarps; off <<= 1) {
+          const uint32_t x = __shfl_up_sync(0xffffffffu, wt, off);
+          if (lane >= off) wt += x;
+        }
+        const uint32_t before = __shfl_sync(0xffffffffu, wt, warp > 0 ? warp - 1 : 0);
+        acc += warp > 0 ? before : 0u;
+      }
 #pragma unroll
       for (int j = 0; j < kRowBinsPerThread; ++j) {
         if (acc < need && acc + mine[j] >= need) {
@@ -218,30 +235,53 @@ __global__ void __launch_bounds__(kRowThreads) topk_rows_staged_kernel(
   auto window_of = [&](uint32_t ky) { return !exact && ky >= klo && ky <= khi; };
   const int seg = ((V + kRowWarps - 1) / kRowWarps + 31) & ~31;
   const int s0 = min(V, warp * seg), s1 = min(V, s0 + seg);
+  // per 32-key group of the warp's segment: the masks of chosen and window
+  // keys, kept in the (now unused) histogram for the writing pass
+  uint32_t* gmask = sh.hist + warp * (2 * kRowMaxGroups);
   uint32_t strict = 0, win = 0;
-  for (int i0 = s0; i0 < s1; i0 += 32) {
+  for (int i0 = s0, gi = 0; i0 < s1; i0 += 32, ++gi) {
     const int i = i0 + lane;
     const uint32_t ky = i < s1 ? key[i] : 0u;
-    strict += __popc(__ballot_sync(0xffffffffu, i < s1 && strict_of(ky, i)));
-    win += __popc(__ballot_sync(0xffffffffu, i < s1 && window_of(ky)));
+    const uint32_t sm = __ballot_sync(0xffffffffu, i < s1 && strict_of(ky, i));
+    const uint32_t wm = __ballot_sync(0xffffffffu, i < s1 && window_of(ky));
+    if (lane == 0) {
+      gmask[2 * gi] = sm;
+      gmask[2 * gi + 1] = wm;
+    }
+    strict += __popc(sm);
+    win += __popc(wm);
   }
   if (lane == 0) sh.wcnt[warp] = (strict << 16) | win;  // both < 2^16
   __syncthreads();
-  uint32_t win_before = 0, out_before = 0;
-  for (int w = 0; w < warp; ++w) {
-    const uint32_t st = sh.wcnt[w] >> 16, wi = sh.wcnt[w] & 0xffffu;
-    const uint32_t take = need_w > win_before ? min(wi, need_w - win_before) : 0u;
-    out_before += st + take;
-    win_before += wi;
+  uint32_t win_before, out_before;
+  {  // lane w < 16: warp w's chosen count; exclusive 16-lane scans
+    const uint32_t cw = lane < kRowWarps ? sh.wcnt[lane] : 0u;
+    const uint32_t st = cw >> 16, wi = cw & 0xffffu;
+    uint32_t wscan = wi;
+#pragma unroll
+    for (int off = 1; off < kRowWarps; off <<= 1) {
+      const uint32_t x = __shfl_up_sync(0xffffffffu, wscan, off);
+      if (lane >= off) wscan += x;
+    }
+    const uint32_t wpre = wscan - wi;  // window keys in the warps before
+    const uint32_t take = need_w > wpre ? min(wi, need_w - wpre) : 0u;
+    const uint32_t v = lane < kRowWarps ? st + take : 0u;
+    uint32_t oscan = v;
+#pragma unroll
+    for (int off = 1; off < kRowWarps; off <<= 1) {
+      const uint32_t x = __shfl_up_sync(0xffffffffu, oscan, off);
+      if (lane >= off) oscan += x;
+    }
+    win_before = __shfl_sync(0xffffffffu, wpre, warp);
+    out_before = __shfl_sync(0xffffffffu, oscan - v, warp);
   }
   const uint32_t lt = (1u << lane) - 1u;
-  for (int i0 = s0; i0 < s1; i0 += 32) {
+  for (int i0 = s0, gi = 0; i0 < s1; i0 += 32, ++gi) {
     const int i = i0 + lane;
-    const uint32_t ky = i < s1 ? key[i] : 0u;
-    const bool is_w = i < s1 && window_of(ky);
-    const uint32_t wm = __ballot_sync(0xffffffffu, is_w);
-    const bool pick = (i < s1 && strict_of(ky, i)) || (is_w && win_before + __popc(wm & lt) < need_w);
-    const uint32_t pm = __ballot_sync(0xffffffffu, pick);
+    const uint32_t sm = gmask[2 * gi], wm = gmask[2 * gi + 1];
+    const bool is_w = (wm >> lane) & 1u;
+    const bool pick = ((sm >> lane) & 1u) || (is_w && win_before + __popc(wm & lt) < need_w);
+    const uint32_t pm = wm == 0u ? sm : __ballot_sync(0xffffffffu, pick);
     const uint32_t o = out_before + __popc(pm & lt);
     if (pick && o < (uint32_t)k) out[o] = i;
     out_before += __popc(pm);
