@@ -10,28 +10,33 @@
 // context"; B9 of the "Core formulas chapter"; one softmax shared by the
 // window, the compressed entries and the sink).
 //
-// Heads on TMEM lanes, 64 rows (M = 64): a tcgen05 MMA costs about the same
-// tensor-pipe time whatever its N, so the 64 heads of one query take the M
-// side and the N side is as wide as the operands allow:
+// Heads on TMEM lanes, 64 rows (M = 64): the 64 heads of one query take the
+// M side of both products and the N side is as wide as the operands allow:
 //   S[h, e]  = Q[h, :] . K[e, :]           M = 64 heads, N = 128 entries
 //   O[h, d] += sum_e P[h, e] V[e, d]        M = 64 heads, N = 256 dims (x2)
-// -- 48 MMAs per 128-entry tile.  An M = 64 accumulator fills 16 lanes of
-// each TMEM lane quarter: O (512 columns) takes the low 16 lanes of every
-// quarter and S (two 128-column buffers) the high 16, so one warp per quarter
-// holds both the scores and the output of its 16 heads, two threads per head
-// (one per 32-column half of each 64-column load).  The softmax is per
-// thread with one partner shuffle; the running max moves (and the head's O
-// row is rescaled in TMEM) only when a tile's max exceeds it by 2^8.
+// -- 48 MMAs per 128-entry tile.  An M = 64 operand or accumulator fills 16
+// lanes of each TMEM lane quarter.  The low 16 lanes hold the query itself
+// (the A operand of Q.K, read from tensor memory: 512 bf16 = 256 columns)
+// and the two 128-column S buffers; the high 16 lanes hold O (512 columns).
+// One warp per quarter owns the scores and the output of its 16 heads, two
+// threads per head; the softmax is per thread with one partner shuffle; the
+// running max moves (and the head's O row is rescaled in TMEM) only when a
+// tile's max exceeds it by 2^8.
 //
-// The gathered 128 x 512 entry tile is stored once (eight 64-dim slabs,
-// 128-byte swizzle): the K-major B operand of Q.K and the MN-major B operand
-// (V) of P.V; each half of P.V frees four slabs for the next tile's gather.
-// Persistent CTAs (one per SM) walk the queries.  Every wait is bounded
-// (including the warp-group exchanges, which use mbarriers rather than
-// named barriers), so a fault upstream ends the kernel with the timeout flag
-// set instead of a hang.  Warp roles: warps 0-3 softmax + epilogue, warps 4-10
-// gather (cp.async, zero-filled past the end of E_t; they also compact the
-// query's valid selected indices), warp 11 issues the MMAs.
+// With the query out of shared memory, the entry tiles (128 entries x 512
+// dims, stored once as eight 64-dim 128-byte-swizzled slabs: the K-major B
+// operand of Q.K and the MN-major B operand (V) of P.V) live in a ring of
+// three 64 KB groups of four slabs; tile g takes groups 2g and 2g + 1 (mod 3).
+// The MMA warp issues Q.K(g) over its first group, then P.V(g - 1) (whose
+// first half frees the group that Q.K(g) needs next), then Q.K(g) over its
+// second group: the gather and the first half of Q.K of the next tile run
+// while the softmax of this one does.  Persistent CTAs (one per SM) walk the
+// queries.  Every wait is bounded (including the warp-group exchanges,
+// which use mbarriers rather than named barriers), so a fault upstream ends
+// the kernel with the timeout flag set instead of a hang.  Warp roles: warps
+// 0-3 softmax + epilogue; warps 4-10 gather (cp.async, zero-filled past the
+// end of E_t; they also compact the query's valid selected indices), and
+// warps 4-7 write each query into tensor memory; warp 11 issues the MMAs.
 #include "common.cuh"
 #include "launch.h"
 #include "sm100.cuh"
@@ -48,7 +53,9 @@ constexpr int kC = 512;                  // entry dim
 constexpr int kTE = 128;                 // entries per tile (QK N)
 constexpr int kSlabs = kC / 64;          // 64-dim slabs
 constexpr int kSlabBytes = kTE * 128;    // 16 KB
-constexpr int kQSlabBytes = kNH * 128;   // 8 KB
+constexpr int kGroupBytes = 4 * kSlabBytes;  // 64 KB: half a tile
+constexpr int kGroups = 3;               // the ring
+static_assert(kSlabs == 8, "a tile is two groups of four slabs");
 constexpr int kPSlabBytes = kNH * 128;   // 8 KB: 64 heads x 64 entries
 constexpr int kSoftWarps = 4, kProdWarps = 7;
 constexpr int kProdThreads = kProdWarps * 32;
@@ -57,11 +64,12 @@ constexpr int kThreads = (kMmaWarp + 1) * 32;  // 384
 constexpr int kRowsPerPass = kProdThreads / 8;  // 28 rows x 8 16-byte chunks per pass
 constexpr int kPasses = (kTE + kRowsPerPass - 1) / kRowsPerPass;  // 5
 constexpr int kMaxSel = 2048;                  // selected entries per query
+constexpr int kMeta = 4;                       // queries in flight between the roles
 constexpr float kRescaleLog2 = 8.f;            // move the running max only past 2^8
 
-constexpr uint32_t kLaneS = 16u << 16;  // S: the high 16 lanes of each quarter
-constexpr uint32_t kColS = 0;           // S buffers at columns 0 and 128
-constexpr uint32_t kColO = 0;           // O: the low 16 lanes, columns 0-511
+constexpr uint32_t kColQ = 256;         // Q: the low 16 lanes, columns 256-511
+constexpr uint32_t kColS = 0;           // S buffers: the low 16 lanes, columns 0 and 128
+constexpr uint32_t kLaneO = 16u << 16;  // O: the high 16 lanes, columns 0-511
 
 struct __align__(16) AttnMeta {
   int ntiles, nrows;
@@ -69,33 +77,31 @@ struct __align__(16) AttnMeta {
 };
 
 struct __align__(8) AttnBars {
-  uint64_t slab_full[kSlabs];
-  // half hf of P.V (slabs 4 hf .. 4 hf + 3) done; slab_free[1] also frees P
-  uint64_t slab_free[2];
-  uint64_t s_full[2], s_empty[2], p_full, q_full, q_empty, o_empty, meta_full[2], drain;
+  uint64_t grp_full[kGroups];  // a group's four slabs are stored
+  uint64_t grp_free[kGroups];  // the P.V half that reads a group is done
+  uint64_t s_full[2], s_empty[2], p_full, p_free, q_full, q_empty, o_empty, meta_full[kMeta];
+  uint64_t drain;
   uint64_t grp_prod;  // bounded group barrier of the producer warps (one arrive per warp)
   uint32_t tmem_base;
 };
 
-constexpr int OFF_Q = 0;
-constexpr int OFF_KV = OFF_Q + kSlabs * kQSlabBytes;        // 65536
-constexpr int OFF_P = OFF_KV + kSlabs * kSlabBytes;         // 196608
+constexpr int OFF_KV = 0;
+constexpr int OFF_P = OFF_KV + kGroups * kGroupBytes;      // 196608
 constexpr int OFF_LIST = OFF_P + 2 * kPSlabBytes;           // 212992
 constexpr int OFF_META = OFF_LIST + kMaxSel * 4;
-constexpr int OFF_SCAN = OFF_META + 2 * (int)sizeof(AttnMeta);
+constexpr int OFF_SCAN = OFF_META + kMeta * (int)sizeof(AttnMeta);
 constexpr int OFF_BAR = OFF_SCAN + 64;
 constexpr int SMEM = OFF_BAR + (int)sizeof(AttnBars) + 1024;
 static_assert(SMEM <= 232448, "shared memory budget");
 
 __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(
-    const __grid_constant__ CUtensorMap tm_q, const __nv_bfloat16* __restrict__ kv_comp,
+    const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ kv_comp,
     const int32_t* __restrict__ idx, int k, const __nv_bfloat16* __restrict__ kv_win,
     int window, const float* __restrict__ sink, float scale, int64_t n, int m, int64_t E,
     int64_t total, __nv_bfloat16* __restrict__ out, unsigned int* __restrict__ err) {
   using namespace sm100;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = smem_raw + ((1024 - (smem_u32(smem_raw) & 1023)) & 1023);
-  uint8_t* sQ = smem + OFF_Q;
   uint8_t* sKV = smem + OFF_KV;
   uint8_t* sP = smem + OFF_P;
   int32_t* list = reinterpret_cast<int32_t*>(smem + OFF_LIST);
@@ -108,16 +114,18 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(
   if (flag_value(err) != 0) return;
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < kSlabs; ++s) mbar_init(&bar->slab_full[s], kProdThreads);
-    mbar_init(&bar->slab_free[0], 1);
-    mbar_init(&bar->slab_free[1], 1);
-    for (int i = 0; i < 2; ++i) {
-      mbar_init(&bar->s_full[i], 1);
-      mbar_init(&bar->s_empty[i], kSoftWarps);
-      mbar_init(&bar->meta_full[i], 1);
+    for (int u = 0; u < kGroups; ++u) {
+      mbar_init(&bar->grp_full[u], kProdThreads);
+      mbar_init(&bar->grp_free[u], 1);
     }
+    for (int u = 0; u < 2; ++u) {
+      mbar_init(&bar->s_full[u], 1);
+      mbar_init(&bar->s_empty[u], kSoftWarps);
+    }
+    for (int u = 0; u < kMeta; ++u) mbar_init(&bar->meta_full[u], 1);
     mbar_init(&bar->p_full, kSoftWarps);
-    mbar_init(&bar->q_full, 1);
+    mbar_init(&bar->p_free, 1);
+    mbar_init(&bar->q_full, 4);  // the four warps that write the query
     mbar_init(&bar->q_empty, 1);
     mbar_init(&bar->o_empty, kSoftWarps);
     mbar_init(&bar->drain, 1);
@@ -140,11 +148,9 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(
     const int chunk = ptid & 7;
     int g = 0;
     uint32_t gphase = 0;
-    int64_t q_issued = -1;  // last query whose Q load was issued
     bool ok = true;
-    // queries are read once; the entries and window rows are re-read by many
-    // queries and should stay in L2
-    const uint64_t pol_q = l2_policy_evict_first(), pol_kv = l2_policy_evict_last();
+    // the entries and window rows are re-read by many queries: keep them in L2
+    const uint64_t pol_kv = l2_policy_evict_last();
     for (int64_t kq = 0; ok; ++kq) {
       const int64_t qi = blockIdx.x + kq * gridDim.x;
       if (qi >= total) break;
@@ -191,21 +197,44 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(
       const int N = nsel + nwin;
       const int T = (N + kTE - 1) / kTE;
       if (ptid == 0) {
-        AttnMeta& mt = meta[kq & 1];
+        AttnMeta& mt = meta[kq % kMeta];
         mt.ntiles = T;
         mt.nrows = N;
         mt.t = t;
         mt.b = b;
-        mbar_arrive(&bar->meta_full[kq & 1]);
-        // the query's 64 heads, once the previous query's Q.K has finished
-        if (kq >= 1 && !mbar_wait(&bar->q_empty, (uint32_t)((kq - 1) & 1), err)) ok = false;
-        if (ok) {
-          mbar_arrive_expect_tx(&bar->q_full, kSlabs * kQSlabBytes);
-          for (int s = 0; s < kSlabs; ++s)
-            tma_load_3d_hint(sQ + s * kQSlabBytes, &tm_q, &bar->q_full, s * 64, (int)(t * kNH),
-                             (int)b, pol_q);
-          q_issued = kq;
+        mbar_arrive(&bar->meta_full[kq % kMeta]);
+      }
+      if (pw < 4) {
+        // ---- the query into tensor memory: warp pw writes heads 16 pw .. 16 pw + 15
+        // (lanes 32 pw + r), thread (r, half) the 64 dims 128 c + 64 half .. of
+        // round c; each 32-bit column holds two consecutive dims ----
+        const int hd = pw * 16 + (lane & 15), half = lane >> 4;
+        const uint4* src =
+            reinterpret_cast<const uint4*>(q + ((b * n + t) * kNH + hd) * kC + 64 * half);
+        const uint32_t qaddr = tmem + ((uint32_t)(pw * 32) << 16) + kColQ;
+        for (int c = 0; c < kC / 128 && ok; ++c) {
+          uint32_t r[32];
+#pragma unroll
+          for (int j = 0; j < 8; ++j) {
+            const uint4 v = __ldcs(src + c * 16 + j);  // read once
+            r[4 * j] = v.x;
+            r[4 * j + 1] = v.y;
+            r[4 * j + 2] = v.z;
+            r[4 * j + 3] = v.w;
+          }
+          // the previous query's Q.K has finished reading the old query
+          if (c == 0 && kq >= 1 && !mbar_wait(&bar->q_empty, (uint32_t)((kq - 1) & 1), err)) {
+            ok = false;
+            break;
+          }
+          if (c == 0) tc_fence_after();
+          tmem_st16x64(qaddr + c * 64, r);
         }
+        if (!ok) break;
+        tmem_st_wait();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bar->q_full);
       }
       for (int tt = 0; tt < T && ok; ++tt, ++g) {
         // this thread's rows of the tile: global row pointers (nullptr = zero fill)
@@ -222,41 +251,96 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(
           }
           src[rr] = p;
         }
-        for (int s = 0; s < kSlabs; ++s) {
-          if (g >= 1 && (s & 3) == 0 &&
-              !mbar_wait(&bar->slab_free[s >> 2], (uint32_t)((g - 1) & 1), err)) {
+        for (int h = 0; h < 2 && ok; ++h) {
+          // half h of tile g: group u = 2 g + h of the ring, free once the P.V
+          // half that read it three groups ago is done
+          const int u = 2 * g + h, gp = u % kGroups;
+          if (u >= kGroups &&
+              !mbar_wait(&bar->grp_free[gp], (uint32_t)(((u / kGroups) - 1) & 1), err)) {
             ok = false;
             break;
           }
-          uint8_t* dst = sKV + s * kSlabBytes;
+          uint8_t* dst0 = sKV + gp * kGroupBytes;
+          for (int j = 0; j < 4; ++j) {
+            const int s = 4 * h + j;
+            uint8_t* dst = dst0 + j * kSlabBytes;
 #pragma unroll
-          for (int rr = 0; rr < kPasses; ++rr) {
-            const int row = (ptid >> 3) + kRowsPerPass * rr;
-            if (row >= kTE) continue;
-            const __nv_bfloat16* p = src[rr] != nullptr ? src[rr] + s * 64 + chunk * 8 : kv_win;
-            cp_async_16_hint(dst + row * 128 + ((chunk ^ (row & 7)) * 16), p,
-                             src[rr] != nullptr ? 16u : 0u, pol_kv);
+            for (int rr = 0; rr < kPasses; ++rr) {
+              const int row = (ptid >> 3) + kRowsPerPass * rr;
+              if (row >= kTE) continue;
+              const __nv_bfloat16* p = src[rr] != nullptr ? src[rr] + s * 64 + chunk * 8 : kv_win;
+              cp_async_16_hint(dst + row * 128 + ((chunk ^ (row & 7)) * 16), p,
+                               src[rr] != nullptr ? 16u : 0u, pol_kv);
+            }
           }
-          cp_async_arrive_noinc(&bar->slab_full[s]);
+          cp_async_arrive_noinc(&bar->grp_full[gp]);
         }
       }
     }
     asm volatile("cp.async.wait_all;" ::: "memory");
-    if (ptid == 0 && q_issued >= 0)  // the last Q load has landed before exit
-      mbar_wait(&bar->q_full, (uint32_t)(q_issued & 1), err, false);
   } else if (warp == kMmaWarp) {
     // ======================= MMA issuer (one lane) =============================
     constexpr uint32_t kIdQK = idesc_bf16(kNH, kTE, 0, 0);   // Q K-major, K K-major
     constexpr uint32_t kIdPV = idesc_bf16(kNH, 256, 0, 1);   // P K-major, V MN-major
-    const uint32_t kv0 = smem_u32(sKV), q0 = smem_u32(sQ), p0 = smem_u32(sP);
+    const uint32_t kv0 = smem_u32(sKV), p0 = smem_u32(sP);
     int g = 0;
     bool ok = true;
+    // the tile whose P.V is still to be issued: index, first of its query, query
+    int pend = -1;
+    bool pend_first = false;
+    int64_t pend_kq = 0;
+    auto issue_pv = [&]() -> bool {
+      if (!mbar_wait(&bar->p_full, (uint32_t)(pend & 1), err)) return false;
+      // the first P.V of a query overwrites O: the previous epilogue has read it
+      if (pend_first && pend_kq >= 1 &&
+          !mbar_wait(&bar->o_empty, (uint32_t)((pend_kq - 1) & 1), err))
+        return false;
+      tc_fence_after();
+      if (lane == 0) {
+        for (int hf = 0; hf < 2; ++hf) {  // dims 256 hf .. 256 hf + 255: group 2 pend + hf
+          const int gp = (2 * pend + hf) % kGroups;
+#pragma unroll
+          for (int kk = 0; kk < kTE / 16; ++kk)
+            mma_bf16(tmem + kLaneO + hf * 256,
+                     desc_sw128(p0 + (kk >> 2) * kPSlabBytes + (kk & 3) * 32),
+                     desc_sw128_mn(kv0 + gp * kGroupBytes + kk * 2048, kSlabBytes, 1024),
+                     kIdPV, (pend_first && kk == 0) ? 0u : 1u);
+          mma_commit(&bar->grp_free[gp]);
+        }
+        mma_commit(&bar->p_free);
+      }
+      __syncwarp();
+      pend = -1;
+      return true;
+    };
+    // Q.K over group u (slabs 4 h .. 4 h + 3 of tile g, h = u - 2 g)
+    auto issue_qk_half = [&](int h, int sb) -> bool {
+      const int u = 2 * g + h, gp = u % kGroups;
+      if (!mbar_wait(&bar->grp_full[gp], (uint32_t)((u / kGroups) & 1), err)) return false;
+      fence_proxy_async();
+      tc_fence_after();
+      if (lane == 0) {
+        for (int j = 0; j < 4; ++j) {
+          const int s = 4 * h + j;
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk)  // 16 dims = 8 columns of the query per step
+            mma_bf16_ts(tmem + kColS + sb * kTE, tmem + kColQ + s * 32 + kk * 8,
+                        desc_sw128(kv0 + gp * kGroupBytes + j * kSlabBytes + kk * 32), kIdQK,
+                        (s | kk) != 0 ? 1u : 0u);
+        }
+      }
+      __syncwarp();
+      return true;
+    };
     for (int64_t kq = 0; ok; ++kq) {
       const int64_t qi = blockIdx.x + kq * gridDim.x;
       if (qi >= total) break;
-      if (!mbar_wait(&bar->meta_full[kq & 1], (uint32_t)((kq >> 1) & 1), err)) break;
-      const int T = meta[kq & 1].ntiles;
+      if (!mbar_wait(&bar->meta_full[kq % kMeta], (uint32_t)((kq / kMeta) & 1), err)) break;
+      const int T = meta[kq % kMeta].ntiles;
+      // the previous query's last P.V first: its epilogue need not wait for this query
+      if (pend >= 0 && !issue_pv()) break;
       if (!mbar_wait(&bar->q_full, (uint32_t)(kq & 1), err)) break;
+      tc_fence_after();
       for (int tt = 0; tt < T; ++tt, ++g) {
         const int sb = g & 1;
         // S buffer sb is free once the softmax has read it (tile g - 2)
@@ -264,47 +348,22 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(
           ok = false;
           break;
         }
-        tc_fence_after();
-        for (int s = 0; s < kSlabs && ok; ++s) {
-          if (!mbar_wait(&bar->slab_full[s], (uint32_t)(g & 1), err)) { ok = false; break; }
-          fence_proxy_async();
-          tc_fence_after();
-          if (lane == 0) {
-#pragma unroll
-            for (int kk = 0; kk < 4; ++kk)
-              mma_bf16(tmem + kLaneS + kColS + sb * kTE,
-                       desc_sw128(q0 + s * kQSlabBytes + kk * 32),
-                       desc_sw128(kv0 + s * kSlabBytes + kk * 32), kIdQK,
-                       (s | kk) != 0 ? 1u : 0u);
-          }
-          __syncwarp();
-        }
-        if (!ok) break;
+        if (!(ok = issue_qk_half(0, sb))) break;
+        // P.V of the previous tile: its first half frees the group of this
+        // tile's second half
+        if (pend >= 0 && !(ok = issue_pv())) break;
+        if (!(ok = issue_qk_half(1, sb))) break;
         if (lane == 0) {
           mma_commit(&bar->s_full[sb]);
           if (tt == T - 1) mma_commit(&bar->q_empty);
         }
         __syncwarp();
-        if (!mbar_wait(&bar->p_full, (uint32_t)(g & 1), err)) { ok = false; break; }
-        if (tt == 0 && kq >= 1 && !mbar_wait(&bar->o_empty, (uint32_t)((kq - 1) & 1), err)) {
-          ok = false;
-          break;
-        }
-        tc_fence_after();
-        if (lane == 0) {
-          for (int hf = 0; hf < 2; ++hf) {  // dims 256 hf .. 256 hf + 255 = slabs 4 hf .. 4 hf + 3
-#pragma unroll
-            for (int kk = 0; kk < kTE / 16; ++kk)
-              mma_bf16(tmem + kColO + hf * 256,
-                       desc_sw128(p0 + (kk >> 2) * kPSlabBytes + (kk & 3) * 32),
-                       desc_sw128_mn(kv0 + 4 * hf * kSlabBytes + kk * 2048, kSlabBytes, 1024),
-                       kIdPV, (tt == 0 && kk == 0) ? 0u : 1u);
-            mma_commit(&bar->slab_free[hf]);
-          }
-        }
-        __syncwarp();
+        pend = g;
+        pend_first = tt == 0;
+        pend_kq = kq;
       }
     }
+    if (ok && pend >= 0) issue_pv();
     if (lane == 0) mma_commit(&bar->drain);
     __syncwarp();
     mbar_wait(&bar->drain, 0, err, false);
@@ -314,15 +373,15 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(
     // head 16 q + hl, columns 32 ch .. 32 ch + 31 of every 64-column load
     const int hl = lane & 15, ch = lane >> 4;
     const int hd = warp * 16 + hl;
-    const uint32_t o_lane = tmem + ((uint32_t)(warp * 32) << 16) + kColO;
-    const uint32_t s_lane = tmem + ((uint32_t)(warp * 32) << 16) + kLaneS + kColS;
+    const uint32_t o_lane = tmem + ((uint32_t)(warp * 32) << 16) + kLaneO;
+    const uint32_t s_lane = tmem + ((uint32_t)(warp * 32) << 16) + kColS;
     const float qscale = scale * kLog2e;
     int g = 0;
     for (int64_t kq = 0;; ++kq) {
       const int64_t qi = blockIdx.x + kq * gridDim.x;
       if (qi >= total) break;
-      if (!mbar_wait(&bar->meta_full[kq & 1], (uint32_t)((kq >> 1) & 1), err)) break;
-      const AttnMeta mt = meta[kq & 1];
+      if (!mbar_wait(&bar->meta_full[kq % kMeta], (uint32_t)((kq / kMeta) & 1), err)) break;
+      const AttnMeta mt = meta[kq % kMeta];
       float m_run = kNegInf;  // running max (log2 units) of head hd
       float l_run = 0.f;      // this thread's share of the head's sum
       bool ok = true;
@@ -361,7 +420,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(
           m_run = mx;
         }
         // P (and, for a rescale, O) is free once the previous P.V is done
-        if (g >= 1 && !mbar_wait(&bar->slab_free[1], (uint32_t)((g - 1) & 1), err)) {
+        if (g >= 1 && !mbar_wait(&bar->p_free, (uint32_t)((g - 1) & 1), err)) {
           ok = false;
           break;
         }
@@ -401,7 +460,8 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(
       }
       if (!ok) break;
       // ---- epilogue: o = O / (sum_j p_j + 2^(sink - m)) -------------------------
-      if (!mbar_wait(&bar->slab_free[1], (uint32_t)((g - 1) & 1), err)) break;
+      // O is complete once the P.V of the query's last tile (g - 1) is done
+      if (!mbar_wait(&bar->p_free, (uint32_t)((g - 1) & 1), err)) break;
       tc_fence_after();
       const float l = l_run + __shfl_xor_sync(0xffffffffu, l_run, 16);
       const float mref = m_run == kNegInf ? 0.f : m_run;
@@ -448,18 +508,15 @@ cudaError_t launch_attn_tc(const void* q, const void* kv_comp, const int32_t* id
                            const void* kv_win, int window, const float* sink, float scale,
                            int64_t batch, int64_t n, int m, void* out, unsigned int* err,
                            cudaStream_t s) {
-  CUtensorMap tq;
-  if (!make_tmap_bf16_3d(&tq, q, kC, (uint64_t)n * kNH, batch, kC * 2ull,
-                         (uint64_t)n * kNH * kC * 2, 64, kNH))
-    return cudaErrorInvalidValue;
   cudaError_t e = cudaFuncSetAttribute(attn_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        SMEM);
   if (e != cudaSuccess) return e;
   const int64_t total = batch * n;
   const int64_t grid = std::min<int64_t>(total, sm_count());
   attn_tc_kernel<<<(unsigned)grid, kThreads, SMEM, s>>>(
-      tq, (const __nv_bfloat16*)kv_comp, idx, k, (const __nv_bfloat16*)kv_win, window, sink,
-      scale, n, m, n / m, total, (__nv_bfloat16*)out, err);
+      (const __nv_bfloat16*)q, (const __nv_bfloat16*)kv_comp, idx, k,
+      (const __nv_bfloat16*)kv_win, window, sink, scale, n, m, n / m, total,
+      (__nv_bfloat16*)out, err);
   return cudaGetLastError();
 }
 
