@@ -146,10 +146,12 @@ def dist_setup():
 
 
 def max_over_ranks(x: float, world: int) -> float:
+    """The largest of the ranks' values (every rank gets it)."""
     if world == 1:
         return x
     import torch.distributed as dist
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
 
@@ -158,7 +160,14 @@ def barrier(world):
     if world > 1:
         import torch.distributed as dist
         dist.barrier()
-    torch.cuda.synchronize()
+    if torch.cuda.is_available():
+        torch.cuda.synchronize()
+
+
+def job_throughput(units_per_rank: float, world: int, ms_max: float) -> float:
+    """Whole-job units per second: every rank's units over the slowest rank's
+    time (replicas: each rank runs the same workload)."""
+    return units_per_rank * world / (ms_max * 1e-3)
 
 
 # ------------------------------------------------------- CSA prefill layer ---
@@ -497,7 +506,7 @@ def main():
     clocks = clk.stop()
     total = max_over_ranks(total, world)
     ms = total / args.steps
-    value = w.n * w.batch * world / (ms * 1e-3)
+    value = job_throughput(w.n * w.batch, world, ms)
     work = L.work()
     calls = {name: round(t, 4) for name, t in zip(L.calls, per_call)}
     roof = {name: roofline(*work[name], per_call[i], peaks) for i, name in enumerate(L.calls)}
