@@ -26,7 +26,8 @@ CSA_OK, CSA_ERR_INVALID_ARG, CSA_ERR_UNSUPPORTED, CSA_ERR_WORKSPACE, CSA_ERR_CUD
 CSA_F32, CSA_BF16 = 0, 1
 
 EXPORTED = (
-    "csa_status_string", "csa_last_error", "csa_abi_version", "csa_check", "csa_compress",
+    "csa_status_string", "csa_last_error", "csa_abi_version", "csa_check", "csa_selftest_wait",
+    "csa_compress",
     "csa_index_topk_workspace", "csa_index_topk", "csa_index_topk_noalloc", "csa_sparse_attn",
     "hca_attn",
     "csa_cache_layout", "csa_cache_store_entries", "csa_cache_write_rows",
@@ -83,6 +84,7 @@ def lib() -> ctypes.CDLL:
         "csa_last_error": (ctypes.c_char_p, []),
         "csa_abi_version": (i32, []),
         "csa_check": (i32, [vp]),
+        "csa_selftest_wait": (i32, [ctypes.c_uint32, i32, vp]),
         "csa_compress": (i32, [vp, vp, vp, vp, vp, vp, i64, i64, i32, i32, i32, i32, vp, vp]),
         "csa_index_topk_workspace": (sz, [i64, i64, i32, i32, i32, i32]),
         "csa_index_topk": (i32, [vp, vp, vp, i64, i64, i32, i32, i32, i32, i32, vp, vp, sz, vp]),
@@ -119,6 +121,16 @@ def _check(status: int):
 def csa_check(device=None):
     """Synchronises the current stream and raises if a kernel gave up a bounded wait."""
     _check(lib().csa_check(torch.cuda.current_stream(device).cuda_stream))
+
+
+def selftest_wait(limit_us: int, arrive: bool, device=None) -> int:
+    """Runs the library's bounded-wait self-test on the current stream and
+    returns the status csa_check reports afterwards (CSA_OK when the barrier
+    was completed, CSA_ERR_TIMEOUT when the wait gave up)."""
+    L = lib()
+    stream = torch.cuda.current_stream(device).cuda_stream
+    _check(L.csa_selftest_wait(int(limit_us), 1 if arrive else 0, stream))
+    return int(L.csa_check(stream))
 
 
 def _dt(t: torch.Tensor) -> int:

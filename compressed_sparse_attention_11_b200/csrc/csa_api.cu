@@ -156,6 +156,15 @@ csa_status csa_check(void* stream) {
   return ok();
 }
 
+csa_status csa_selftest_wait(uint32_t limit_us, int arrive, void* stream) {
+  if (limit_us < 1 || limit_us > 2000000u)
+    return fail(CSA_ERR_INVALID_ARG, "csa_selftest_wait: limit_us out of range");
+  unsigned int* flag = device_timeout_flag();
+  if (flag == nullptr) return fail(CSA_ERR_CUDA, "csa_selftest_wait: no device flag");
+  return cuda_status(launch_selftest_wait(limit_us, arrive != 0, flag, (cudaStream_t)stream),
+                     "csa_selftest_wait");
+}
+
 csa_status csa_compress(const void* ca, const void* cb, const void* za, const void* zb,
                         const float* ba, const float* bb, int64_t batch, int64_t n, int c,
                         int m, int overlap, csa_dtype dt, void* out, void* stream) {

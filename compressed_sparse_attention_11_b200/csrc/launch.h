@@ -51,6 +51,10 @@ cudaError_t launch_index_scores_tc(const void* q_i, const float* w_i, const void
 // tcgen05 attention (bf16, 64 heads of dim 512, up to 2048 selected entries).
 bool attn_tc_supported(int nh, int c, int k, csa_dtype dt, const void* q, const void* kv_comp,
                        const void* kv_win);
+// One warp waits on a barrier that is completed first (arrive) or never; the
+// wait gives up after limit_us and sets *err.
+cudaError_t launch_selftest_wait(uint32_t limit_us, bool arrive, unsigned int* err,
+                                 cudaStream_t s);
 cudaError_t launch_attn_tc(const void* q, const void* kv_comp, const int32_t* idx, int k,
                            const void* kv_win, int window, const float* sink, float scale,
                            int64_t batch, int64_t n, int m, void* out, unsigned int* err,

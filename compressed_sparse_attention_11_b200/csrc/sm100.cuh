@@ -78,6 +78,20 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, unsign
   return true;
 }
 
+// mbar_wait with an explicit limit (ns) and no early exit on the flag.
+__device__ __forceinline__ bool mbar_wait_limit(uint64_t* bar, uint32_t parity,
+                                                unsigned int* flag, uint64_t limit_ns) {
+  const uint64_t t0 = globaltimer();
+  uint32_t spins = 0;
+  while (!mbar_try_wait(bar, parity)) {
+    if ((++spins & 255u) == 0 && globaltimer() - t0 > limit_ns) {
+      atomicOr(flag, 1u);
+      return false;
+    }
+  }
+  return true;
+}
+
 // ---- programmatic dependent launch -------------------------------------------
 // A kernel launched with programmatic stream serialization may start while
 // the previous kernel in the stream is still running.  pdl_wait() blocks until

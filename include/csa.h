@@ -67,6 +67,15 @@ int csa_abi_version(void);
  * (the outputs of that launch are invalid), and clears that record.  The one
  * entry point that synchronises. */
 csa_status csa_check(void* stream);
+/* Exercises the bounded-wait path on the device (no counterpart on the
+ * pages; a library self-test).  One warp waits on a shared-memory barrier;
+ * if `arrive` is non-zero the barrier is completed first and the wait
+ * succeeds, otherwise nothing completes it and the wait gives up after
+ * `limit_us` microseconds (1 .. 2,000,000), recording the timeout exactly as
+ * a kernel of the layer would: the next csa_check on that device returns
+ * CSA_ERR_TIMEOUT.  No fault, trap or hang is involved; the context stays
+ * usable.  Returns CSA_ERR_INVALID_ARG for a limit out of range. */
+csa_status csa_selftest_wait(uint32_t limit_us, int arrive, void* stream);
 
 /* ------------------------------------------------------------------------
  * csa_compress -- token-level KV compressor ([Formulas B9] CSA and HCA

@@ -180,3 +180,9 @@ def test_decode_step_validation():
         csa.CSA_OK
     assert L.csa_cache_write_rows(ctypes.byref(d), FAKE, -1, 4, ctypes.byref(rows), None) == \
         csa.CSA_ERR_INVALID_ARG
+
+
+def test_selftest_wait_rejects_limits_out_of_range():
+    L = csa.lib()
+    assert L.csa_selftest_wait(0, 1, None) == csa.CSA_ERR_INVALID_ARG
+    assert L.csa_selftest_wait(2000001, 0, None) == csa.CSA_ERR_INVALID_ARG
