@@ -44,9 +44,19 @@ UNIT = "tokens/s"
 # profiles/).  A figure is reported only while the kernel sources it was
 # measured on are unchanged (sha256 prefix per file), else null.
 MEASURED_TRAFFIC = {
-    # index_scores_tc_kernel 1127.5 MB read + 2136.4 MB written, topk_rows_staged_kernel
-    # 2150.5 MB read + 76.6 MB written (n = 65536; profiles/dram_bytes_prefill_calls.md)
-    "index_topk": {"bytes": 5491000000, "sources": {'compressed_sparse_attention_11_b200/csrc/indexer_tc.cu': '7f5543f1ca4e8e9e', 'compressed_sparse_attention_11_b200/csrc/topk.cu': 'b5c2b3e3bbbddc89', 'compressed_sparse_attention_11_b200/csrc/sm100.cuh': 'dc33b8fd81a2190a', 'compressed_sparse_attention_11_b200/csrc/common.cuh': '2c8e048cf6f6eadb'}},
+    # index_scores_tc_kernel 1146.5 MB read + 2136.4 MB written, topk_rows_staged_kernel
+    # 2150.0 MB read + 77.0 MB written (n = 65536; profiles/dram_bytes_prefill_calls.md)
+    "index_topk": {"bytes": 5510017024, "sources": {
+        'compressed_sparse_attention_11_b200/csrc/indexer_tc.cu': '7f5543f1ca4e8e9e',
+        'compressed_sparse_attention_11_b200/csrc/topk.cu': 'b124a41d87752842',
+        'compressed_sparse_attention_11_b200/csrc/sm100.cuh': '1f37f1c1af8b9d58',
+        'compressed_sparse_attention_11_b200/csrc/common.cuh': '2c8e048cf6f6eadb'}},
+    # attn_tc_kernel 4530.0 MB read + 4238.6 MB written (n = 65536)
+    "sparse_attn": {"bytes": 8768529408, "sources": {
+        'compressed_sparse_attention_11_b200/csrc/attn_tc.cu': 'e6284f671315d58b',
+        'compressed_sparse_attention_11_b200/csrc/sm100.cuh': '1f37f1c1af8b9d58',
+        'compressed_sparse_attention_11_b200/csrc/common.cuh': '2c8e048cf6f6eadb',
+        'compressed_sparse_attention_11_b200/csrc/tc_attn_util.cuh': 'fbd5bcb87c834e55'}},
 }
 
 
