@@ -45,7 +45,7 @@ UNIT = "tokens/s"
 # measured on are unchanged (sha256 prefix per file), else null.
 MEASURED_TRAFFIC = {
     # index_scores_tc_kernel 1146.5 MB read + 2136.4 MB written, topk_rows_staged_kernel
-    # 2150.0 MB read + 77.0 MB written (n = 65536; profiles/dram_bytes_prefill_calls.md)
+    # 2150.0 MB read + 77.0 MB written (n = 65536; ncu dram__bytes_read/write.sum)
     "index_topk": {"bytes": 5510017024, "sources": {
         'compressed_sparse_attention_11_b200/csrc/indexer_tc.cu': '7f5543f1ca4e8e9e',
         'compressed_sparse_attention_11_b200/csrc/topk.cu': 'b124a41d87752842',
