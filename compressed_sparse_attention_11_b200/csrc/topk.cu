@@ -89,7 +89,27 @@ __global__ void __launch_bounds__(kRowThreads) topk_rows_staged_kernel(
   // 1. the row as order keys, with its key range
   const float* row = scores + (b * n + t) * ld;
   uint32_t mn = 0xffffffffu, mx = 0u;
-  {
+  if ((ld & 3) == 0 && (reinterpret_cast<uintptr_t>(scores) & 15) == 0) {
+    // 16-byte rows: the whole row lands in shared memory in one round trip
+    // (cp.async, zero past V), then becomes order keys in place
+    const int nch = (V + 3) >> 2;
+    for (int c = tid; c < nch; c += kRowThreads) {
+      const int rem = V - 4 * c;
+      const uint32_t bytes = rem >= 4 ? 16u : (uint32_t)rem * 4u;
+      asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(
+                       (uint32_t)__cvta_generic_to_shared(key + 4 * c)),
+                   "l"(row + 4 * c), "r"(bytes)
+                   : "memory");
+    }
+    asm volatile("cp.async.commit_group;\n\tcp.async.wait_all;" ::: "memory");
+    __syncthreads();
+    for (int i = tid; i < V; i += kRowThreads) {
+      const uint32_t ky = order_key(__uint_as_float(key[i]));
+      key[i] = ky;
+      mn = min(mn, ky);
+      mx = max(mx, ky);
+    }
+  } else {
     constexpr int kBatch = 8;
     for (int i0 = tid; i0 < V; i0 += kRowThreads * kBatch) {
       float v[kBatch];
@@ -131,6 +151,9 @@ __global__ void __launch_bounds__(kRowThreads) topk_rows_staged_kernel(
   }
   kmin = __shfl_sync(0xffffffffu, kmin, 0);
   kmax = __shfl_sync(0xffffffffu, kmax, 0);
+  // warp w's contiguous segment of the row (the candidate and writing passes)
+  const int seg = ((V + kRowWarps - 1) / kRowWarps + 31) & ~31;
+  const int s0 = min(V, warp * seg), s1 = min(V, s0 + seg);
   // 2. radix refinement of the window [base, base + 2048 << shift)
   uint32_t base = kmin, need = (uint32_t)k;
   int shift = (int)bit_length(kmax - kmin) - kRowBinBits;
@@ -196,14 +219,30 @@ __global__ void __launch_bounds__(kRowThreads) topk_rows_staged_kernel(
       break;
     }
     if (C <= (uint32_t)kRowCand) {  // rank the bin-T keys among themselves
-      for (int i = tid; i < V; i += kRowThreads) {
-        const uint32_t ky = key[i];
-        if (ky >= klo && ky <= khi) {
+      // One pass over the warps' segments gathers the bin-T keys and keeps,
+      // per 32-key group, the masks of keys above bin T (chosen outright) and
+      // in it (chosen by rank) and each warp's count of the former; the
+      // writing pass below needs no counting pass of its own.
+      uint32_t* gm = sh.hist + warp * (2 * kRowMaxGroups);  // the histogram is no longer read
+      uint32_t above = 0;
+      for (int i0 = s0, gi = 0; i0 < s1; i0 += 32, ++gi) {
+        const int i = i0 + lane;
+        const uint32_t ky = i < s1 ? key[i] : 0u;
+        const bool in_t = i < s1 && ky >= klo && ky <= khi;
+        const uint32_t am = __ballot_sync(0xffffffffu, i < s1 && ky > khi);
+        const uint32_t tm = __ballot_sync(0xffffffffu, in_t);
+        if (lane == 0) {
+          gm[2 * gi] = am;
+          gm[2 * gi + 1] = tm;
+        }
+        above += __popc(am);
+        if (in_t) {
           const uint32_t slot = atomicAdd(&sh.cand_n, 1u);
           sh.cand_key[slot] = ky;
           sh.cand_pos[slot] = i;
         }
       }
+      if (lane == 0) sh.wcnt[warp] = above << 16;
       __syncthreads();
       for (int e = tid; e < (int)C; e += kRowThreads) {
         const uint32_t ke = sh.cand_key[e];
@@ -213,6 +252,7 @@ __global__ void __launch_bounds__(kRowThreads) topk_rows_staged_kernel(
           const uint32_t kf = sh.cand_key[f];
           rank += (kf > ke || (kf == ke && sh.cand_pos[f] < pe)) ? 1u : 0u;
         }
+        if (rank < need) atomicAdd(&sh.wcnt[pe / seg], 1u << 16);  // chosen by rank
         if (rank == need - 1) {
           sh.cut_key = ke;
           sh.cut_pos = pe;
@@ -233,13 +273,12 @@ __global__ void __launch_bounds__(kRowThreads) topk_rows_staged_kernel(
     return exact ? (ky > cut_key || (ky == cut_key && i <= cut_pos)) : ky > khi;
   };
   auto window_of = [&](uint32_t ky) { return !exact && ky >= klo && ky <= khi; };
-  const int seg = ((V + kRowWarps - 1) / kRowWarps + 31) & ~31;
-  const int s0 = min(V, warp * seg), s1 = min(V, s0 + seg);
   // per 32-key group of the warp's segment: the masks of chosen and window
-  // keys, kept in the (now unused) histogram for the writing pass
+  // keys, kept in the (now unused) histogram for the writing pass (the exact
+  // case recorded them, and the counts, while gathering the bin-T keys)
   uint32_t* gmask = sh.hist + warp * (2 * kRowMaxGroups);
   uint32_t strict = 0, win = 0;
-  for (int i0 = s0, gi = 0; i0 < s1; i0 += 32, ++gi) {
+  for (int i0 = s0, gi = 0; i0 < s1 && !exact; i0 += 32, ++gi) {
     const int i = i0 + lane;
     const uint32_t ky = i < s1 ? key[i] : 0u;
     const uint32_t sm = __ballot_sync(0xffffffffu, i < s1 && strict_of(ky, i));
@@ -251,8 +290,10 @@ __global__ void __launch_bounds__(kRowThreads) topk_rows_staged_kernel(
     strict += __popc(sm);
     win += __popc(wm);
   }
-  if (lane == 0) sh.wcnt[warp] = (strict << 16) | win;  // both < 2^16
-  __syncthreads();
+  if (!exact) {
+    if (lane == 0) sh.wcnt[warp] = (strict << 16) | win;  // both < 2^16
+    __syncthreads();
+  }
   uint32_t win_before, out_before;
   {  // lane w < 16: warp w's chosen count; exclusive 16-lane scans
     const uint32_t cw = lane < kRowWarps ? sh.wcnt[lane] : 0u;
@@ -280,7 +321,11 @@ __global__ void __launch_bounds__(kRowThreads) topk_rows_staged_kernel(
     const int i = i0 + lane;
     const uint32_t sm = gmask[2 * gi], wm = gmask[2 * gi + 1];
     const bool is_w = (wm >> lane) & 1u;
-    const bool pick = ((sm >> lane) & 1u) || (is_w && win_before + __popc(wm & lt) < need_w);
+    // exact: wm marks bin-T keys, chosen by the cut; else window keys, chosen
+    // in index order up to need_w
+    const bool pick = ((sm >> lane) & 1u) ||
+                      (is_w && (exact ? strict_of(key[i], i)
+                                      : win_before + __popc(wm & lt) < need_w));
     const uint32_t pm = wm == 0u ? sm : __ballot_sync(0xffffffffu, pick);
     const uint32_t o = out_before + __popc(pm & lt);
     if (pick && o < (uint32_t)k) out[o] = i;
