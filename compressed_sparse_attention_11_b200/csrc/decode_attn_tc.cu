@@ -434,54 +434,46 @@ __global__ void __launch_bounds__(128) decode_combine_kernel(
   const int h = blockIdx.x;
   const float z = sink != nullptr ? sink[h] * kLog2e : kNegInf;
   const int d0 = threadIdx.x * 4;
-  // every range's max, sum and slice of O in flight at once
-  float mi[kMaxCombine], li[kMaxCombine];
-  float4 oi[kMaxCombine];
-#pragma unroll
-  for (int i = 0; i < kMaxCombine; ++i) {
-    mi[i] = kNegInf;
-    li[i] = 0.f;
-    oi[i] = make_float4(0.f, 0.f, 0.f, 0.f);
-    if (i < nsplit) {
-      const int64_t base = (b * nsplit + i) * kNH + h;
-      mi[i] = part_ms[base * 2];
-      li[i] = part_ms[base * 2 + 1];
-      oi[i] = __ldcs(reinterpret_cast<const float4*>(part_o + base * kC + d0));
-    }
-  }
+  // ranges in chunks of kMaxCombine, each chunk's max, sum and slice of O
+  // in flight at once; the running max moves between chunks
   float M = z;
-#pragma unroll
-  for (int i = 0; i < kMaxCombine; ++i) M = fmaxf(M, mi[i]);
-  float den = z == kNegInf ? 0.f : ex2(z - M);
+  float den = z == kNegInf ? 0.f : 1.f;
   float acc[4] = {0.f, 0.f, 0.f, 0.f};
+  for (int c0 = 0; c0 < nsplit; c0 += kMaxCombine) {
+    float mi[kMaxCombine], li[kMaxCombine];
+    float4 oi[kMaxCombine];
 #pragma unroll
-  for (int i = 0; i < kMaxCombine; ++i) {
-    if (mi[i] == kNegInf) continue;
-    const float wgt = ex2(mi[i] - M);
-    den = fmaf(wgt, li[i], den);
-    acc[0] = fmaf(wgt, oi[i].x, acc[0]);
-    acc[1] = fmaf(wgt, oi[i].y, acc[1]);
-    acc[2] = fmaf(wgt, oi[i].z, acc[2]);
-    acc[3] = fmaf(wgt, oi[i].w, acc[3]);
-  }
-  // more ranges than the unrolled set (long dense HCA layers)
-  for (int i = kMaxCombine; i < nsplit; ++i) {
-    const int64_t base = (b * nsplit + i) * kNH + h;
-    const float mx = part_ms[base * 2];
-    if (mx == kNegInf) continue;
-    float f_old = 1.f, wgt = 1.f;
-    if (mx > M) {
-      f_old = ex2(M - mx);
-      M = mx;
-    } else {
-      wgt = ex2(mx - M);
+    for (int i = 0; i < kMaxCombine; ++i) {
+      mi[i] = kNegInf;
+      li[i] = 0.f;
+      oi[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+      if (c0 + i < nsplit) {
+        const int64_t base = (b * nsplit + c0 + i) * kNH + h;
+        mi[i] = part_ms[base * 2];
+        li[i] = part_ms[base * 2 + 1];
+        oi[i] = __ldcs(reinterpret_cast<const float4*>(part_o + base * kC + d0));
+      }
     }
-    const float4 o = __ldcs(reinterpret_cast<const float4*>(part_o + base * kC + d0));
-    den = den * f_old + wgt * part_ms[base * 2 + 1];
-    acc[0] = acc[0] * f_old + wgt * o.x;
-    acc[1] = acc[1] * f_old + wgt * o.y;
-    acc[2] = acc[2] * f_old + wgt * o.z;
-    acc[3] = acc[3] * f_old + wgt * o.w;
+    float mc = kNegInf;
+#pragma unroll
+    for (int i = 0; i < kMaxCombine; ++i) mc = fmaxf(mc, mi[i]);
+    if (mc > M) {  // rescale what is summed so far to the new max
+      const float f = M == kNegInf ? 0.f : ex2(M - mc);
+      den *= f;
+#pragma unroll
+      for (int j = 0; j < 4; ++j) acc[j] *= f;
+      M = mc;
+    }
+#pragma unroll
+    for (int i = 0; i < kMaxCombine; ++i) {
+      if (mi[i] == kNegInf) continue;
+      const float wgt = ex2(mi[i] - M);
+      den = fmaf(wgt, li[i], den);
+      acc[0] = fmaf(wgt, oi[i].x, acc[0]);
+      acc[1] = fmaf(wgt, oi[i].y, acc[1]);
+      acc[2] = fmaf(wgt, oi[i].z, acc[2]);
+      acc[3] = fmaf(wgt, oi[i].w, acc[3]);
+    }
   }
   const float inv = 1.f / den;
   __nv_bfloat16* o = out + (b * kNH + h) * kC + d0;

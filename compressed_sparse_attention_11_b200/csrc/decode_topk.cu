@@ -3,7 +3,7 @@
 // of "DeepSeek-V4: million-token context"; ties to the smaller index, the
 // chosen indices listed ascending; all V entries when V <= k).
 //
-// One thread-block cluster per sequence (up to 8 CTAs); CTA r of the cluster
+// One thread-block cluster per sequence (up to 16 CTAs); CTA r of the cluster
 // copies the contiguous slice r of the sequence's scores (L2-resident after
 // the indexer) into shared memory as order keys -- unsigned integers whose
 // order is the float order -- so every later pass reads shared memory only.
@@ -39,7 +39,7 @@ constexpr int kBins = 4096;
 constexpr int kBinBits = 12;
 constexpr int kBinsPerThread = kBins / kThreads;  // 8
 constexpr int kMaxSlice = 45056;                  // keys per CTA (176 KB)
-constexpr int kMaxCluster = 8;
+constexpr int kMaxCluster = 16;                   // above 8: a non-portable cluster size
 constexpr int kSliceTarget = 16384;               // keys per CTA the cluster size aims for
 constexpr int kSmallWin = 512;                    // bin-T keys ranked directly
 
@@ -326,24 +326,43 @@ cudaError_t launch_decode_topk(const csa_cache_desc& d, const int64_t* pos, cons
   int cs, slice;
   topk_shape(d.capacity, cs, slice);
   if (slice > kMaxSlice) return cudaErrorInvalidValue;
-  const size_t smem = sizeof(TopkShared) + (size_t)slice * 4;
-  cudaError_t e = cudaFuncSetAttribute(decode_topk_kernel,
-                                       cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-  if (e != cudaSuccess) return e;
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3((unsigned)cs, (unsigned)d.batch);
-  cfg.blockDim = dim3(kThreads);
-  cfg.dynamicSmemBytes = smem;
-  cfg.stream = s;
   cudaLaunchAttribute attr[2];
-  attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = (unsigned)cs;
-  attr[0].val.clusterDim.y = 1;
-  attr[0].val.clusterDim.z = 1;
-  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  attr[1].val.programmaticStreamSerializationAllowed = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 2;
+  auto configure = [&]() -> cudaError_t {
+    const size_t smem = sizeof(TopkShared) + (size_t)slice * 4;
+    cudaError_t e = cudaFuncSetAttribute(decode_topk_kernel,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    cfg.gridDim = dim3((unsigned)cs, (unsigned)d.batch);
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = (unsigned)cs;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[1].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 2;
+    return cudaSuccess;
+  };
+  cudaError_t e = configure();
+  if (e != cudaSuccess) return e;
+  if (cs > 8) {  // a non-portable cluster: use it only where the device can place one
+    int clusters = 0;
+    if (cudaFuncSetAttribute(decode_topk_kernel,
+                             cudaFuncAttributeNonPortableClusterSizeAllowed, 1) != cudaSuccess ||
+        cudaOccupancyMaxActiveClusters(&clusters, decode_topk_kernel, &cfg) != cudaSuccess ||
+        clusters < 1) {
+      cudaGetLastError();  // clear a refusal; fall back to eight CTAs
+      cs = 8;
+      const int64_t sl = (d.capacity + cs - 1) / cs;
+      slice = (int)((sl + 31) & ~(int64_t)31);
+      if (slice > kMaxSlice) return cudaErrorInvalidValue;
+      if ((e = configure()) != cudaSuccess) return e;
+    }
+  }
   return cudaLaunchKernelEx(&cfg, decode_topk_kernel, pos, (int64_t)d.capacity, d.m, d.k,
                             scores, sel, slice);
 }
