@@ -44,15 +44,15 @@ UNIT = "tokens/s"
 # profiles/).  A figure is reported only while the kernel sources it was
 # measured on are unchanged (sha256 prefix per file), else null.
 MEASURED_TRAFFIC = {
-    # index_scores_tc_kernel 1146.5 MB read + 2136.4 MB written, topk_rows_staged_kernel
-    # 2150.0 MB read + 77.0 MB written (n = 65536; ncu dram__bytes_read/write.sum)
-    "index_topk": {"bytes": 5510017024, "sources": {
+    # index_scores_tc_kernel 1133.3 MB read + 2136.3 MB written, topk_rows_staged_kernel
+    # 2149.4 MB read + 131.0 MB written (n = 65536; ncu dram__bytes_read/write.sum)
+    "index_topk": {"bytes": 5550000640, "sources": {
         'compressed_sparse_attention_11_b200/csrc/indexer_tc.cu': '7f5543f1ca4e8e9e',
-        'compressed_sparse_attention_11_b200/csrc/topk.cu': 'b124a41d87752842',
+        'compressed_sparse_attention_11_b200/csrc/topk.cu': '44874bde73cf3699',
         'compressed_sparse_attention_11_b200/csrc/sm100.cuh': '1f37f1c1af8b9d58',
         'compressed_sparse_attention_11_b200/csrc/common.cuh': '2c8e048cf6f6eadb'}},
-    # attn_tc_kernel 4530.0 MB read + 4238.6 MB written (n = 65536)
-    "sparse_attn": {"bytes": 8768529408, "sources": {
+    # attn_tc_kernel 4532.9 MB read + 4240.2 MB written (n = 65536)
+    "sparse_attn": {"bytes": 8773083392, "sources": {
         'compressed_sparse_attention_11_b200/csrc/attn_tc.cu': 'e6284f671315d58b',
         'compressed_sparse_attention_11_b200/csrc/sm100.cuh': '1f37f1c1af8b9d58',
         'compressed_sparse_attention_11_b200/csrc/common.cuh': '2c8e048cf6f6eadb',
