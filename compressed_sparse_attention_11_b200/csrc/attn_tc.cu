@@ -36,7 +36,8 @@
 // the kernel with the timeout flag set instead of a hang.  Warp roles: warps
 // 0-3 softmax + epilogue; warps 4-10 gather (cp.async, zero-filled past the
 // end of E_t; they also compact the query's valid selected indices), and
-// warps 4-7 write each query into tensor memory; warp 11 issues the MMAs.
+// warps 4-7 write each query into tensor memory once its first half-tile is
+// under way; warp 11 issues the MMAs.
 #include "common.cuh"
 #include "launch.h"
 #include "sm100.cuh"
@@ -79,7 +80,11 @@ struct __align__(16) AttnMeta {
 struct __align__(8) AttnBars {
   uint64_t grp_full[kGroups];  // a group's four slabs are stored
   uint64_t grp_free[kGroups];  // the P.V half that reads a group is done
-  uint64_t s_full[2], s_empty[2], p_full, p_free, q_full, q_empty, o_empty, meta_full[kMeta];
+  uint64_t s_full[2], s_empty[2], p_full, p_free, o_empty, meta_full[kMeta];
+  // the query's dims 0-255 (lo) and 256-511 (hi) in tensor memory: written /
+  // no longer read by the Q.K halves
+  uint64_t q_full_lo, q_full_hi, q_empty_lo, q_empty_hi;
+  uint64_t idx_full;  // the next query's selection row is in shared memory
   uint64_t drain;
   uint64_t grp_prod;  // bounded group barrier of the producer warps (one arrive per warp)
   uint32_t tmem_base;
@@ -88,11 +93,25 @@ struct __align__(8) AttnBars {
 constexpr int OFF_KV = 0;
 constexpr int OFF_P = OFF_KV + kGroups * kGroupBytes;      // 196608
 constexpr int OFF_LIST = OFF_P + 2 * kPSlabBytes;           // 212992
-constexpr int OFF_META = OFF_LIST + kMaxSel * 4;
+constexpr int OFF_IDXN = OFF_LIST + kMaxSel * 4;             // the next query's row
+constexpr int OFF_META = OFF_IDXN + kMaxSel * 4;
 constexpr int OFF_SCAN = OFF_META + kMeta * (int)sizeof(AttnMeta);
 constexpr int OFF_BAR = OFF_SCAN + 64;
 constexpr int SMEM = OFF_BAR + (int)sizeof(AttnBars) + 1024;
 static_assert(SMEM <= 232448, "shared memory budget");
+
+// One 128-dim round of a query row for tensor memory: the 64 dims of this
+// thread's half, two per 32-bit column.
+__device__ __forceinline__ void load_q_round(const uint4* src, uint32_t (&r)[32]) {
+#pragma unroll
+  for (int j = 0; j < 8; ++j) {
+    const uint4 v = __ldcs(src + j);
+    r[4 * j] = v.x;
+    r[4 * j + 1] = v.y;
+    r[4 * j + 2] = v.z;
+    r[4 * j + 3] = v.w;
+  }
+}
 
 __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(
     const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ kv_comp,
@@ -105,6 +124,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(
   uint8_t* sKV = smem + OFF_KV;
   uint8_t* sP = smem + OFF_P;
   int32_t* list = reinterpret_cast<int32_t*>(smem + OFF_LIST);
+  int32_t* idxn = reinterpret_cast<int32_t*>(smem + OFF_IDXN);
   AttnMeta* meta = reinterpret_cast<AttnMeta*>(smem + OFF_META);
   int* pscan = reinterpret_cast<int*>(smem + OFF_SCAN);
   AttnBars* bar = reinterpret_cast<AttnBars*>(smem + OFF_BAR);
@@ -125,8 +145,11 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(
     for (int u = 0; u < kMeta; ++u) mbar_init(&bar->meta_full[u], 1);
     mbar_init(&bar->p_full, kSoftWarps);
     mbar_init(&bar->p_free, 1);
-    mbar_init(&bar->q_full, 4);  // the four warps that write the query
-    mbar_init(&bar->q_empty, 1);
+    mbar_init(&bar->q_full_lo, 4);  // the four warps that write the query
+    mbar_init(&bar->q_full_hi, 4);
+    mbar_init(&bar->q_empty_lo, 1);
+    mbar_init(&bar->q_empty_hi, 1);
+    mbar_init(&bar->idx_full, 1);
     mbar_init(&bar->o_empty, kSoftWarps);
     mbar_init(&bar->drain, 1);
     mbar_init(&bar->grp_prod, kProdWarps);
@@ -151,6 +174,18 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(
     bool ok = true;
     // the entries and window rows are re-read by many queries: keep them in L2
     const uint64_t pol_kv = l2_policy_evict_last();
+    // the selection rows move into shared memory one query ahead (one bulk
+    // copy) when they are whole 16-byte units; otherwise they are read in place
+    const bool stage = idx != nullptr && k > 0 && (k & 3) == 0 &&
+                       (reinterpret_cast<uintptr_t>(idx) & 15) == 0;
+    int idx_issued = 0;  // bulk copies issued (thread 0) / consumed
+    auto stage_row = [&](int64_t qn) {
+      fence_proxy_async();
+      mbar_arrive_expect_tx(&bar->idx_full, (uint32_t)k * 4u);
+      bulk_load(idxn, idx + qn * k, (uint32_t)k * 4u, &bar->idx_full);
+      ++idx_issued;
+    };
+    if (stage && ptid == 0) stage_row(blockIdx.x);
     for (int64_t kq = 0; ok; ++kq) {
       const int64_t qi = blockIdx.x + kq * gridDim.x;
       if (qi >= total) break;
@@ -158,6 +193,20 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(
       const int64_t V = min((t + 1) / m, E);
       const int64_t w0 = max((int64_t)0, t - window + 1);
       const int nwin = (int)(t - w0 + 1);
+      // the next query of this CTA (64 KB, contiguous) starts moving into L2
+      if (ptid == 0 && qi + gridDim.x < total)
+        bulk_prefetch_l2(q + (qi + gridDim.x) * (kNH * kC), kNH * kC * 2);
+      // warps 0-3: the first two of the four 128-dim rounds of this query
+      // (thread (r, half): head 16 pw + r, the 64 dims 128 c + 64 half ..) start
+      // loading now, under the list compaction and the first half-tile's
+      // gather (read once: evict first)
+      const uint4* qsrc = reinterpret_cast<const uint4*>(
+          q + ((b * n + t) * kNH + pw * 16 + (lane & 15)) * kC + 64 * (lane >> 4));
+      uint32_t ra[32], rb[32];
+      if (pw < 4) {
+        load_q_round(qsrc, ra);
+        load_q_round(qsrc + 16, rb);
+      }
       // the previous query's list is no longer read
       if (!group_sync(&bar->grp_prod, gphase, err)) break;
       int nsel;
@@ -166,6 +215,10 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(
         const int per = (k + kProdThreads - 1) / kProdThreads;
         const int lo = min(k, ptid * per), hi = min(k, lo + per);
         const int32_t* row = idx + (b * n + t) * k;
+        if (stage) {
+          if (!mbar_wait(&bar->idx_full, (uint32_t)(kq & 1), err)) break;
+          row = idxn;
+        }
         int cnt = 0;
         for (int j = lo; j < hi; ++j) {
           const int s = row[j];
@@ -191,6 +244,8 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(
           if (s >= 0 && s < V) list[pos++] = s;
         }
         if (!group_sync(&bar->grp_prod, gphase, err)) break;
+        // every thread is done with the staged row: the next query's comes in
+        if (stage && ptid == 0 && qi + gridDim.x < total) stage_row(qi + gridDim.x);
       } else {
         nsel = (int)V;
       }
@@ -204,54 +259,51 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(
         mt.b = b;
         mbar_arrive(&bar->meta_full[kq % kMeta]);
       }
-      if (pw < 4) {
-        // ---- the query into tensor memory: warp pw writes heads 16 pw .. 16 pw + 15
-        // (lanes 32 pw + r), thread (r, half) the 64 dims 128 c + 64 half .. of
-        // round c; each 32-bit column holds two consecutive dims ----
-        const int hd = pw * 16 + (lane & 15), half = lane >> 4;
-        const uint4* src =
-            reinterpret_cast<const uint4*>(q + ((b * n + t) * kNH + hd) * kC + 64 * half);
-        const uint32_t qaddr = tmem + ((uint32_t)(pw * 32) << 16) + kColQ;
-        for (int c = 0; c < kC / 128 && ok; ++c) {
-          uint32_t r[32];
-#pragma unroll
-          for (int j = 0; j < 8; ++j) {
-            const uint4 v = __ldcs(src + c * 16 + j);  // read once
-            r[4 * j] = v.x;
-            r[4 * j + 1] = v.y;
-            r[4 * j + 2] = v.z;
-            r[4 * j + 3] = v.w;
-          }
-          // the previous query's Q.K has finished reading the old query
-          if (c == 0 && kq >= 1 && !mbar_wait(&bar->q_empty, (uint32_t)((kq - 1) & 1), err)) {
-            ok = false;
-            break;
-          }
-          if (c == 0) tc_fence_after();
-          tmem_st16x64(qaddr + c * 64, r);
-        }
-        if (!ok) break;
+      // ---- the query into tensor memory, warps pw < 4 (lanes 32 pw + r; each
+      // 32-bit column two consecutive dims): dims 0-255 once the first
+      // half-tile's gather is under way and the old query's first Q.K half is
+      // done (rounds 2-3 then load), dims 256-511 after the second half-tile ----
+      const uint32_t qaddr = tmem + ((uint32_t)(pw * 32) << 16) + kColQ;
+      auto write_q_lo = [&]() -> bool {
+        if (kq >= 1 && !mbar_wait(&bar->q_empty_lo, (uint32_t)((kq - 1) & 1), err)) return false;
+        tc_fence_after();
+        tmem_st16x64(qaddr, ra);
+        tmem_st16x64(qaddr + 64, rb);
+        load_q_round(qsrc + 32, ra);
+        load_q_round(qsrc + 48, rb);
         tmem_st_wait();
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(&bar->q_full);
-      }
+        if (lane == 0) mbar_arrive(&bar->q_full_lo);
+        return true;
+      };
+      auto write_q_hi = [&]() -> bool {
+        if (kq >= 1 && !mbar_wait(&bar->q_empty_hi, (uint32_t)((kq - 1) & 1), err)) return false;
+        tc_fence_after();
+        tmem_st16x64(qaddr + 128, ra);
+        tmem_st16x64(qaddr + 192, rb);
+        tmem_st_wait();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bar->q_full_hi);
+        return true;
+      };
       for (int tt = 0; tt < T && ok; ++tt, ++g) {
-        // this thread's rows of the tile: global row pointers (nullptr = zero fill)
-        const __nv_bfloat16* src[kPasses];
-#pragma unroll
-        for (int rr = 0; rr < kPasses; ++rr) {
-          const int slot = tt * kTE + (ptid >> 3) + kRowsPerPass * rr;
-          const __nv_bfloat16* p = nullptr;
-          if (slot < nsel) {
-            const int64_t e = idx != nullptr ? (int64_t)list[slot] : (int64_t)slot;
-            p = kv_comp + (b * E + e) * kC;
-          } else if (slot < N) {
-            p = kv_win + (b * n + w0 + (slot - nsel)) * kC;
-          }
-          src[rr] = p;
-        }
         for (int h = 0; h < 2 && ok; ++h) {
+          // this thread's rows of the tile: global row pointers (nullptr = zero fill)
+          const __nv_bfloat16* src[kPasses];
+#pragma unroll
+          for (int rr = 0; rr < kPasses; ++rr) {
+            const int slot = tt * kTE + (ptid >> 3) + kRowsPerPass * rr;
+            const __nv_bfloat16* p = nullptr;
+            if (slot < nsel) {
+              const int64_t e = idx != nullptr ? (int64_t)list[slot] : (int64_t)slot;
+              p = kv_comp + (b * E + e) * kC;
+            } else if (slot < N) {
+              p = kv_win + (b * n + w0 + (slot - nsel)) * kC;
+            }
+            src[rr] = p;
+          }
           // half h of tile g: group u = 2 g + h of the ring, free once the P.V
           // half that read it three groups ago is done
           const int u = 2 * g + h, gp = u % kGroups;
@@ -274,10 +326,17 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(
             }
           }
           cp_async_arrive_noinc(&bar->grp_full[gp]);
+          if (tt == 0 && pw < 4 && !(h == 0 ? write_q_lo() : write_q_hi())) {
+            ok = false;
+            break;
+          }
         }
       }
     }
     asm volatile("cp.async.wait_all;" ::: "memory");
+    // a staged row that an early exit left unread has landed before the exit
+    if (ptid == 0 && idx_issued > 0)
+      mbar_wait(&bar->idx_full, (uint32_t)((idx_issued - 1) & 1), err, false);
   } else if (warp == kMmaWarp) {
     // ======================= MMA issuer (one lane) =============================
     constexpr uint32_t kIdQK = idesc_bf16(kNH, kTE, 0, 0);   // Q K-major, K K-major
@@ -335,11 +394,12 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(
     for (int64_t kq = 0; ok; ++kq) {
       const int64_t qi = blockIdx.x + kq * gridDim.x;
       if (qi >= total) break;
+      // the previous query's last P.V first: neither its epilogue nor the ring
+      // waits for this query's list
+      if (pend >= 0 && !issue_pv()) break;
       if (!mbar_wait(&bar->meta_full[kq % kMeta], (uint32_t)((kq / kMeta) & 1), err)) break;
       const int T = meta[kq % kMeta].ntiles;
-      // the previous query's last P.V first: its epilogue need not wait for this query
-      if (pend >= 0 && !issue_pv()) break;
-      if (!mbar_wait(&bar->q_full, (uint32_t)(kq & 1), err)) break;
+      if (!mbar_wait(&bar->q_full_lo, (uint32_t)(kq & 1), err)) break;
       tc_fence_after();
       for (int tt = 0; tt < T; ++tt, ++g) {
         const int sb = g & 1;
@@ -349,13 +409,18 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(
           break;
         }
         if (!(ok = issue_qk_half(0, sb))) break;
+        if (tt == T - 1 && lane == 0) mma_commit(&bar->q_empty_lo);
         // P.V of the previous tile: its first half frees the group of this
         // tile's second half
         if (pend >= 0 && !(ok = issue_pv())) break;
+        if (tt == 0) {
+          if (!(ok = mbar_wait(&bar->q_full_hi, (uint32_t)(kq & 1), err))) break;
+          tc_fence_after();
+        }
         if (!(ok = issue_qk_half(1, sb))) break;
         if (lane == 0) {
           mma_commit(&bar->s_full[sb]);
-          if (tt == T - 1) mma_commit(&bar->q_empty);
+          if (tt == T - 1) mma_commit(&bar->q_empty_hi);
         }
         __syncwarp();
         pend = g;
@@ -376,6 +441,8 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(
     const uint32_t o_lane = tmem + ((uint32_t)(warp * 32) << 16) + kLaneO;
     const uint32_t s_lane = tmem + ((uint32_t)(warp * 32) << 16) + kColS;
     const float qscale = scale * kLog2e;
+    // the sink of head hd (log2 units), the same for every query
+    const float z = sink != nullptr ? sink[hd] * kLog2e : kNegInf;
     int g = 0;
     for (int64_t kq = 0;; ++kq) {
       const int64_t qi = blockIdx.x + kq * gridDim.x;
@@ -465,21 +532,42 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(
       tc_fence_after();
       const float l = l_run + __shfl_xor_sync(0xffffffffu, l_run, 16);
       const float mref = m_run == kNegInf ? 0.f : m_run;
-      const float z = sink != nullptr ? sink[hd] * kLog2e : kNegInf;
       const float inv = 1.f / (l + (z == kNegInf ? 0.f : ex2(z - mref)));
-      __nv_bfloat16* ob = out + ((mt.b * n + mt.t) * kNH + hd) * kC + 32 * ch;
+      // 128 dims a pass: the warp's 16 head rows (256 bytes each) go through
+      // its own 4 KB of the P buffer (free until the warp writes the next P),
+      // 16-byte chunks XOR-swizzled by row, so that every global store writes
+      // two whole 256-byte row pieces; the next 64-column TMEM load overlaps
+      uint8_t* ebuf = sP + (hl >> 3) * kPSlabBytes + warp * 2048 + (hl & 7) * 256;
+      __nv_bfloat16* ow = out + ((mt.b * n + mt.t) * kNH + warp * 16) * kC;
+      uint32_t o[2][32];
+      tmem_ld16x64(o_lane, o[0]);
+      tmem_ld_wait();
+#pragma unroll
       for (int c = 0; c < kC / 64; ++c) {
-        uint32_t o[32];
-        tmem_ld16x64(o_lane + c * 64, o);
-        tmem_ld_wait();
+        if (c + 1 < kC / 64) tmem_ld16x64(o_lane + (c + 1) * 64, o[(c + 1) & 1]);
         uint32_t pk[16];
 #pragma unroll
         for (int i = 0; i < 32; i += 2)
-          pk[i >> 1] = pack_bf16x2(__uint_as_float(o[i]) * inv, __uint_as_float(o[i + 1]) * inv);
+          pk[i >> 1] = pack_bf16x2(__uint_as_float(o[c & 1][i]) * inv,
+                                   __uint_as_float(o[c & 1][i + 1]) * inv);
+        // dims 64 c + 32 ch + 8 j ..: chunk 8 (c & 1) + 4 ch + j of the row piece
 #pragma unroll
         for (int j = 0; j < 4; ++j)
-          __stcs(reinterpret_cast<uint4*>(ob + c * 64 + 8 * j),  // streamed: not re-read
-                 make_uint4(pk[4 * j], pk[4 * j + 1], pk[4 * j + 2], pk[4 * j + 3]));
+          *reinterpret_cast<uint4*>(ebuf + (((8 * (c & 1) + 4 * ch + j) ^ (hl & 7)) * 16)) =
+              make_uint4(pk[4 * j], pk[4 * j + 1], pk[4 * j + 2], pk[4 * j + 3]);
+        if (c & 1) {
+          __syncwarp();
+          // row r = 2 i + lane / 16, chunk lane % 16 of dims 128 (c / 2) ..
+#pragma unroll
+          for (int i = 0; i < 8; ++i) {
+            const int r = 2 * i + (lane >> 4), x = lane & 15;
+            const uint4 v = *reinterpret_cast<const uint4*>(
+                sP + (r >> 3) * kPSlabBytes + warp * 2048 + (r & 7) * 256 + ((x ^ (r & 7)) * 16));
+            __stcs(reinterpret_cast<uint4*>(ow + r * kC + 128 * (c >> 1) + 8 * x), v);
+          }
+          __syncwarp();
+        }
+        tmem_ld_wait();
       }
       tc_fence_before();
       __syncwarp();

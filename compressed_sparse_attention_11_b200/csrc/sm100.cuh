@@ -106,6 +106,11 @@ __device__ __forceinline__ void pdl_trigger() {
 }
 
 // ---- TMA ---------------------------------------------------------------------
+// Starts moving `bytes` (a multiple of 16, from a 16-byte aligned address) of
+// global memory into L2 without waiting for it.
+__device__ __forceinline__ void bulk_prefetch_l2(const void* p, uint32_t bytes) {
+  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(p), "r"(bytes) : "memory");
+}
 __device__ __forceinline__ void tma_prefetch_desc(const CUtensorMap* map) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
 }
