@@ -536,38 +536,34 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(
       // 128 dims a pass: the warp's 16 head rows (256 bytes each) go through
       // its own 4 KB of the P buffer (free until the warp writes the next P),
       // 16-byte chunks XOR-swizzled by row, so that every global store writes
-      // two whole 256-byte row pieces; the next 64-column TMEM load overlaps
+      // two whole 256-byte row pieces; thread (hl, ch) loads dims
+      // 128 pp + 64 ch .. + 63 of head hl
       uint8_t* ebuf = sP + (hl >> 3) * kPSlabBytes + warp * 2048 + (hl & 7) * 256;
       __nv_bfloat16* ow = out + ((mt.b * n + mt.t) * kNH + warp * 16) * kC;
-      uint32_t o[2][32];
-      tmem_ld16x64(o_lane, o[0]);
-      tmem_ld_wait();
-#pragma unroll
-      for (int c = 0; c < kC / 64; ++c) {
-        if (c + 1 < kC / 64) tmem_ld16x64(o_lane + (c + 1) * 64, o[(c + 1) & 1]);
-        uint32_t pk[16];
-#pragma unroll
-        for (int i = 0; i < 32; i += 2)
-          pk[i >> 1] = pack_bf16x2(__uint_as_float(o[c & 1][i]) * inv,
-                                   __uint_as_float(o[c & 1][i + 1]) * inv);
-        // dims 64 c + 32 ch + 8 j ..: chunk 8 (c & 1) + 4 ch + j of the row piece
-#pragma unroll
-        for (int j = 0; j < 4; ++j)
-          *reinterpret_cast<uint4*>(ebuf + (((8 * (c & 1) + 4 * ch + j) ^ (hl & 7)) * 16)) =
-              make_uint4(pk[4 * j], pk[4 * j + 1], pk[4 * j + 2], pk[4 * j + 3]);
-        if (c & 1) {
-          __syncwarp();
-          // row r = 2 i + lane / 16, chunk lane % 16 of dims 128 (c / 2) ..
-#pragma unroll
-          for (int i = 0; i < 8; ++i) {
-            const int r = 2 * i + (lane >> 4), x = lane & 15;
-            const uint4 v = *reinterpret_cast<const uint4*>(
-                sP + (r >> 3) * kPSlabBytes + warp * 2048 + (r & 7) * 256 + ((x ^ (r & 7)) * 16));
-            __stcs(reinterpret_cast<uint4*>(ow + r * kC + 128 * (c >> 1) + 8 * x), v);
-          }
-          __syncwarp();
-        }
+#pragma unroll 1
+      for (int pp = 0; pp < kC / 128; ++pp) {
+        uint32_t o[64];
+        tmem_ld16x128(o_lane + pp * 128, o);
         tmem_ld_wait();
+#pragma unroll
+        for (int jj = 0; jj < 8; ++jj) {
+          uint32_t pk[4];
+#pragma unroll
+          for (int i = 0; i < 4; ++i)
+            pk[i] = pack_bf16x2(__uint_as_float(o[8 * jj + 2 * i]) * inv,
+                                __uint_as_float(o[8 * jj + 2 * i + 1]) * inv);
+          *reinterpret_cast<uint4*>(ebuf + (((8 * ch + jj) ^ (hl & 7)) * 16)) =
+              make_uint4(pk[0], pk[1], pk[2], pk[3]);
+        }
+        __syncwarp();
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          const int r = 2 * i + (lane >> 4), x = lane & 15;
+          const uint4 v = *reinterpret_cast<const uint4*>(
+              sP + (r >> 3) * kPSlabBytes + warp * 2048 + (r & 7) * 256 + ((x ^ (r & 7)) * 16));
+          __stcs(reinterpret_cast<uint4*>(ow + r * kC + 128 * pp + 8 * x), v);
+        }
+        __syncwarp();
       }
       tc_fence_before();
       __syncwarp();
