@@ -31,13 +31,23 @@
 // first half frees the group that Q.K(g) needs next), then Q.K(g) over its
 // second group: the gather and the first half of Q.K of the next tile run
 // while the softmax of this one does.  Persistent CTAs (one per SM) walk the
-// queries.  Every wait is bounded (including the warp-group exchanges,
-// which use mbarriers rather than named barriers), so a fault upstream ends
-// the kernel with the timeout flag set instead of a hang.  Warp roles: warps
-// 0-3 softmax + epilogue; warps 4-10 gather (cp.async, zero-filled past the
-// end of E_t; they also compact the query's valid selected indices), and
-// warps 4-7 write each query into tensor memory once its first half-tile is
-// under way; warp 11 issues the MMAs.
+// queries.
+//
+// Query boundaries are kept off the tensor pipe's path: the next query's
+// selection row is bulk-copied into shared memory while this one runs; the
+// query reaches tensor memory in two halves (dims 0-255, then 256-511), each
+// written as soon as the previous query's Q.K half that read it is done, from
+// registers loaded at the top of the query; the last P.V of a query is issued
+// before anything of the next query is awaited; and the epilogue passes each
+// warp's rows through the idle P buffer so that its global stores are whole
+// 256-byte row pieces.
+//
+// Every wait is bounded (including the warp-group exchanges, which use
+// mbarriers rather than named barriers), so a fault upstream ends the kernel
+// with the timeout flag set instead of a hang.  Warp roles: warps 0-3
+// softmax + epilogue; warps 4-10 gather (cp.async, zero-filled past the end
+// of E_t; they also compact the query's valid selected indices), and warps
+// 4-7 write each query into tensor memory; warp 11 issues the MMAs.
 #include "common.cuh"
 #include "launch.h"
 #include "sm100.cuh"
