@@ -124,27 +124,12 @@ __device__ __forceinline__ void tma_load_3d(void* dst, const CUtensorMap* map, u
       : "memory");
 }
 
-// L2 eviction policies (createpolicy): data read once (streamed queries) is
-// marked evict-first, data re-read by many CTAs (gathered entries) evict-last.
-__device__ __forceinline__ uint64_t l2_policy_evict_first() {
-  uint64_t p;
-  asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(p));
-  return p;
-}
+// L2 eviction policy (createpolicy) for data re-read by many CTAs (gathered
+// entries): evict-last.
 __device__ __forceinline__ uint64_t l2_policy_evict_last() {
   uint64_t p;
   asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(p));
   return p;
-}
-// tma_load_3d with an L2 cache policy.
-__device__ __forceinline__ void tma_load_3d_hint(void* dst, const CUtensorMap* map, uint64_t* bar,
-                                                 int x, int y, int z, uint64_t policy) {
-  asm volatile(
-      "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint"
-      " [%0], [%1, {%2, %3, %4}], [%5], %6;" ::"r"(smem_u32(dst)),
-      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(z), "r"(smem_u32(bar)),
-      "l"(policy)
-      : "memory");
 }
 
 // 1-D bulk copy global -> shared (no tensor map); completes `bytes` on `bar`.
@@ -181,13 +166,8 @@ __device__ __forceinline__ void tc_fence_after() {
 }
 
 // ---- cp.async (16-byte, L2-only) with zero fill --------------------------------
-// Copies `bytes` (0 or 16) from global to shared; the rest of the 16 bytes is zero.
-__device__ __forceinline__ void cp_async_16(void* dst, const void* src, uint32_t bytes) {
-  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(smem_u32(dst)), "l"(src),
-               "r"(bytes)
-               : "memory");
-}
-// cp_async_16 with an L2 cache policy.
+// Copies `bytes` (0 or 16) from global to shared under an L2 cache policy; the
+// rest of the 16 bytes is zero.
 __device__ __forceinline__ void cp_async_16_hint(void* dst, const void* src, uint32_t bytes,
                                                  uint64_t policy) {
   asm volatile("cp.async.cg.shared.global.L2::cache_hint [%0], [%1], 16, %2, %3;" ::"r"(
@@ -206,12 +186,8 @@ __device__ __forceinline__ void cp_async_arrive_noinc(uint64_t* bar) {
 __device__ __forceinline__ void fence_proxy_async() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
-// Named barrier over `count` threads (ids 1..15; 0 is __syncthreads).
-__device__ __forceinline__ void named_bar(int id, int count) {
-  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
-}
-// Named barrier that also returns whether any participating thread passed
-// pred = true.
+// Named barrier over `count` threads (ids 1..15; 0 is __syncthreads) that
+// also returns whether any participating thread passed pred = true.
 __device__ __forceinline__ bool named_bar_or(int id, int count, bool pred) {
   uint32_t r;
   asm volatile(
