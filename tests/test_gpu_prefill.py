@@ -239,8 +239,29 @@ def test_sparse_attn_tensor_core_messy_selection(B, n, k, W, sink_none):
         check_close(g[b, rr], ref, torch.bfloat16, f"sparse attn b={b}")
 
 
+@pytest.mark.parametrize("B,n,k,W", [
+    (1, 3, 4, 128),      # fewer queries than SMs, no compressed entry visible yet
+    (2, 300, 130, 64),   # selection rows not whole 16-byte units: read in place
+    (1, 150, 1, 5),      # a single selection, a short window
+])
+def test_sparse_attn_tensor_core_edge_shapes(B, n, k, W):
+    nh, c, m = 64, 512, 4
+    q, kv, win, sink = _attn_inputs(B, n, nh, c, m, torch.bfloat16, seed=47)
+    idx = _random_selection(B, n, m, k, seed=8)
+    out = csa.csa_sparse_attn(q.to(DEV), kv.to(DEV), torch.tensor(idx).to(DEV), win.to(DEV), W,
+                              sink.to(DEV), 1 / math.sqrt(c), m)
+    csa.csa_check()
+    g = host(out)
+    rr = sorted(set(list(range(0, min(n, 12))) + list(range(max(0, n - 12), n)) +
+                    list(range(5, n, 29))))
+    for b in range(B):
+        ref = O.sparse_attn(q[b], kv[b], idx[b], win[b], W, sink, 1 / math.sqrt(c), m, rows=rr)
+        check_close(g[b, rr], ref, torch.bfloat16, f"sparse attn b={b}")
+
+
 @pytest.mark.parametrize("B,n,nh,c,m,W,dt,rows", [
     (1, 2048, 64, 512, 128, 128, torch.bfloat16, "sample"),
+    (1, 5, 64, 512, 128, 128, torch.bfloat16, None),        # window only, 5 queries
     (2, 1100, 64, 512, 16, 64, torch.bfloat16, "sample"),   # more entries than a tile
     (2, 700, 16, 128, 32, 50, torch.float32, None),
     (1, 64, 4, 32, 128, 128, torch.float32, None),    # no entry complete: window only
