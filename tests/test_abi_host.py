@@ -9,6 +9,7 @@ import os
 import re
 
 import pytest
+import torch
 
 import compressed_sparse_attention_11_b200 as csa
 
@@ -186,3 +187,18 @@ def test_selftest_wait_rejects_limits_out_of_range():
     L = csa.lib()
     assert L.csa_selftest_wait(0, 1, None) == csa.CSA_ERR_INVALID_ARG
     assert L.csa_selftest_wait(2000001, 0, None) == csa.CSA_ERR_INVALID_ARG
+
+
+def test_binding_rejects_host_tensors_and_bad_layouts():
+    """The Python binding only marshals: it refuses what the C ABI cannot take
+    (host memory, other dtypes, non-contiguous views) before any call."""
+    x = torch.zeros(1, 8, 16)
+    with pytest.raises(ValueError, match="CUDA device"):
+        csa.csa_compress(x, None, x, None, torch.zeros(4, 16), None, 4)
+    with pytest.raises(ValueError, match="dtype"):
+        csa._dt(torch.zeros(2, dtype=torch.int32))
+    assert csa._dt(torch.zeros(2)) == csa.CSA_F32
+    assert csa._dt(torch.zeros(2, dtype=torch.bfloat16)) == csa.CSA_BF16
+    assert csa._ptr(None) is None
+    with pytest.raises(ValueError, match="CUDA device"):
+        csa._ptr(torch.zeros(4, 4).t())
