@@ -64,7 +64,7 @@ def test_workload_figures():
 
 
 def test_roofline_arithmetic():
-    peaks = {"hbm_gbs": 5000.0, "bf16_sustained": 1000.0, "source": "measured"}
+    peaks = {"hbm_gbs": 5000.0, "bf16": 1000.0, "bf16_sustained": 800.0, "source": "measured"}
     r = bench.roofline("flops", 2e12, 4.0, peaks)      # 2 TFLOP in 4 ms
     assert r["bound"] == "tensor" and r["achieved"] == pytest.approx(500.0)
     assert r["frac"] == pytest.approx(0.5)
