@@ -63,9 +63,11 @@ const char* csa_last_error(void);
 /* ABI version, bumped on any signature or layout change. */
 int csa_abi_version(void);
 /* Synchronises `stream`, then returns CSA_ERR_TIMEOUT if any kernel of this
- * library on the current device gave up a bounded wait since the last check
- * (the outputs of that launch are invalid), and clears that record.  The one
- * entry point that synchronises. */
+ * library on the current device gave up a bounded wait since the last check,
+ * and clears that record.  While the record is set, every later kernel of the
+ * library on that device skips or cuts short its work, so the outputs of ALL
+ * launches on the device since the last check are invalid, not only those of
+ * the launch that gave up.  The one entry point that synchronises. */
 csa_status csa_check(void* stream);
 /* Exercises the bounded-wait path on the device (no counterpart on the
  * pages; a library self-test).  One warp waits on a shared-memory barrier;
@@ -128,12 +130,18 @@ csa_status csa_index_topk(const void* q_i, const float* w_i, const void* k_i, in
  *
  * Same arguments, results and errors as csa_index_topk, without `ws`: the
  * score scratch is a fixed array inside the library (8 MiB per device, held
- * by every GPU that loads the library until the process exits).  Calls that
- * need more than 2^21 fp32 scores (batch * n * floor(n/m)) return
- * CSA_ERR_UNSUPPORTED.  All calls share that array, so calls whose work
- * overlaps on the GPU race on it.  The first call on a device looks up the
- * array's address (cudaGetSymbolAddress with that device current); make it
- * before any stream capture.  Never allocates.
+ * by every GPU that loads the library until the process exits).  Arguments
+ * are checked first (CSA_ERR_INVALID_ARG as for csa_index_topk); a valid
+ * call that needs more than 2^21 fp32 scores (batch * n * floor(n/m),
+ * computed without overflow) returns CSA_ERR_UNSUPPORTED and launches
+ * nothing.  All calls share that array, so calls whose work overlaps on the
+ * GPU race on it.  The first call on a device looks up the array's address
+ * (cudaGetSymbolAddress with that device current); with the CUDA runtime's
+ * lazy module loading that lookup may load the library's device code and
+ * the array itself (a device allocation made by the runtime, which may
+ * synchronise), so make the first call before any stream capture.  Calls
+ * after cudaDeviceReset of that device are unsupported (the cached address
+ * is stale).  The entry point itself calls no allocator.
  * ------------------------------------------------------------------------ */
 csa_status csa_index_topk_noalloc(const void* q_i, const float* w_i, const void* k_i,
                                   int64_t batch, int64_t n, int nh_i, int c_i, int m, int k,

@@ -202,3 +202,33 @@ def test_binding_rejects_host_tensors_and_bad_layouts():
     assert csa._ptr(None) is None
     with pytest.raises(ValueError, match="CUDA device"):
         csa._ptr(torch.zeros(4, 4).t())
+
+
+def _noalloc(**kw):
+    a = dict(q=FAKE, w=FAKE, k_i=FAKE, batch=1, n=64, nh=4, ci=64, m=4, k=8, dt=1, idx=FAKE)
+    a.update(kw)
+    return csa.lib().csa_index_topk_noalloc(a["q"], a["w"], a["k_i"], a["batch"], a["n"],
+                                            a["nh"], a["ci"], a["m"], a["k"], a["dt"], a["idx"],
+                                            None)
+
+
+@pytest.mark.parametrize("kw,why", [
+    (dict(k=0, n=1 << 40), "k must"),          # a bad argument wins over the size check
+    (dict(ci=12, n=1 << 40), "multiple of 8"),
+    (dict(dt=5, n=1 << 40), "dt must"),
+    (dict(m=0), "m must"),
+    (dict(n=-1), "must be >= 0"),
+])
+def test_noalloc_checks_arguments_before_its_size(kw, why):
+    assert _noalloc(**kw) == csa.CSA_ERR_INVALID_ARG
+    assert why in csa.lib().csa_last_error().decode()
+
+
+@pytest.mark.parametrize("batch,n,m", [
+    (1, 1 << 40, 1),          # batch * n * n/m overflows 64 bits
+    (1 << 30, 1 << 20, 4),
+    (1, 2050, 2),             # 2050 * 1025 > 2^21
+])
+def test_noalloc_refuses_sizes_beyond_its_scratch_without_overflow(batch, n, m):
+    assert _noalloc(batch=batch, n=n, m=m) == csa.CSA_ERR_UNSUPPORTED
+    assert "built-in scratch" in csa.lib().csa_last_error().decode()
