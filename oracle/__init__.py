@@ -287,6 +287,112 @@ def reads_per_query(t: int, m: int, k: Optional[int], window: int) -> int:
 
 
 # ---------------------------------------------------------------------------
+# Query / KV-entry RMSNorm and partial RoPE ([Walk-through] §4.5 "other
+# details" and §7.1 Partial RoPE, §7.4 Query/KV Entry Normalization).
+#
+# The pages state: every query head and every KV entry is RMSNorm-ed before
+# core attention; RoPE is applied to the last 64 dims of queries and KV
+# entries; because each entry is both key and value, the attention output's
+# last 64 dims are rotated by position -t so the output carries relative
+# position only.  Readings where they are silent (listed in the design notes):
+#   * RMSNorm(x) = x / sqrt(mean(x^2) + eps) * gamma over the head dim, one
+#     learnable gamma for queries and one for KV entries, eps = 1e-6;
+#   * the norm applies to every entry core attention reads (compressed and
+#     window rows alike), before the rotation;
+#   * RoPE pairs the trailing dims as (2j, 2j+1), j = 0 .. rope_dims/2 - 1,
+#     and turns pair j by angle pos * base^(-2j/rope_dims), base = 10000;
+#   * a window row sits at its token position u; a compressed entry s at the
+#     position of its block's first token, m * s.
+# ---------------------------------------------------------------------------
+
+ROPE_BASE = 10000.0
+NORM_EPS = 1e-6
+
+
+def rms_norm(x, gamma, eps: float = NORM_EPS) -> np.ndarray:
+    """x / sqrt(mean(x^2) + eps) * gamma over the last axis (fp64)."""
+    x = f64(x)
+    ms = (x * x).mean(axis=-1, keepdims=True)
+    return x / np.sqrt(ms + eps) * f64(gamma)
+
+
+def rope_theta(rope_dims: int, base: float = ROPE_BASE) -> np.ndarray:
+    """Angle per unit position of each rotated pair: base^(-2j/rope_dims)."""
+    j = np.arange(rope_dims // 2, dtype=np.float64)
+    return base ** (-2.0 * j / rope_dims)
+
+
+def rope_rotate(x, pos, rope_dims: int, base: float = ROPE_BASE) -> np.ndarray:
+    """Rotates the last `rope_dims` dims of x in pairs (2j, 2j+1) by pos * theta_j.
+
+    x [..., c]; pos a scalar or an array broadcast against x's leading axes.
+    The leading c - rope_dims dims are returned unchanged.
+    """
+    x = f64(x).copy()
+    if rope_dims == 0:
+        return x
+    c = x.shape[-1]
+    ang = np.asarray(pos, dtype=np.float64)[..., None] * rope_theta(rope_dims, base)
+    cs, sn = np.cos(ang), np.sin(ang)
+    a = x[..., c - rope_dims::2].copy()
+    b = x[..., c - rope_dims + 1::2].copy()
+    x[..., c - rope_dims::2] = a * cs - b * sn
+    x[..., c - rope_dims + 1::2] = a * sn + b * cs
+    return x
+
+
+def entry_position(s, m: int):
+    """Position a compressed entry is rotated with: its block's first token."""
+    return m * np.asarray(s)
+
+
+def attend_norm_rope(q_t, t: int, entries, entry_pos, sink, scale: float, q_gamma, kv_gamma,
+                     rope_dims: int, eps: float = NORM_EPS,
+                     base: float = ROPE_BASE) -> np.ndarray:
+    """Core attention of one query with the norm and partial RoPE around it.
+
+    q_t [nh, c] raw query heads at position t; entries [N, c] raw entries at
+    positions entry_pos [N].  q' = RoPE_t(RMSNorm(q)), e' = RoPE_p(RMSNorm(e)),
+    o = attend(q', e', sink), returned as RoPE_{-t}(o).
+    """
+    q = rope_rotate(rms_norm(q_t, q_gamma, eps), t, rope_dims, base)
+    E = rope_rotate(rms_norm(entries, kv_gamma, eps), np.asarray(entry_pos), rope_dims, base)
+    return rope_rotate(attend(q, E, sink, scale), -t, rope_dims, base)
+
+
+def sparse_attn_norm_rope(q, kv_comp, idx, kv_win, window: int, sink, scale: float, m: int,
+                          q_gamma, kv_gamma, rope_dims: int, rows: Optional[Sequence[int]] = None,
+                          eps: float = NORM_EPS) -> np.ndarray:
+    """CSA core attention with the norm and RoPE, on raw (un-normed) entries
+    kv_comp [E, c] and window rows kv_win [n, c]: [len(rows), nh, c]."""
+    kv_comp, kv_win = f64(kv_comp), f64(kv_win)
+    n = q.shape[0]
+    rows = range(n) if rows is None else rows
+    out = []
+    for t in rows:
+        V = min(visible(t, m), kv_comp.shape[0])
+        sel = [int(s) for s in np.asarray(idx[t]) if 0 <= int(s) < V]
+        win = list(window_rows(t, window))
+        ents = np.concatenate([kv_comp[sel], kv_win[win]], axis=0)
+        pos = np.concatenate([entry_position(np.asarray(sel, dtype=np.int64), m),
+                              np.asarray(win, dtype=np.int64)])
+        out.append(attend_norm_rope(q[t], t, ents, pos, sink, scale, q_gamma, kv_gamma,
+                                    rope_dims, eps))
+    return np.stack(out)
+
+
+def hca_attn_norm_rope(q, kv_comp, kv_win, window: int, sink, scale: float, m: int, q_gamma,
+                       kv_gamma, rope_dims: int, rows: Optional[Sequence[int]] = None,
+                       eps: float = NORM_EPS) -> np.ndarray:
+    """HCA core attention (every visible entry) with the norm and RoPE."""
+    E = f64(kv_comp).shape[0]
+    n = q.shape[0]
+    idx = [np.arange(min(visible(t, m), E)) for t in range(n)]
+    return sparse_attn_norm_rope(q, kv_comp, idx, kv_win, window, sink, scale, m, q_gamma,
+                                 kv_gamma, rope_dims, rows, eps)
+
+
+# ---------------------------------------------------------------------------
 # FP8 E4M3 and bf16 storage ([Analysis] §7.3 "KV mixed-precision storage":
 # RoPE dims in BF16, the other dims in FP8)
 # ---------------------------------------------------------------------------

@@ -490,3 +490,113 @@ def test_decode_sequence_matches_prefill_pipeline():
     for i, (codes, scale, _) in enumerate(seq.ikeys):
         ref_codes, ref_scale, _ = O.quantize_entry(np.float32(ik_all[i]), 0)
         assert np.array_equal(codes, ref_codes) and scale == ref_scale
+
+
+# ------------------------------------------- RMSNorm and partial RoPE ---------
+# Pins of the norm / rotation applied around core attention ([Walk-through]
+# §4.5, §7.1, §7.4): closed forms of RMSNorm, the rotation written a second
+# way (complex multiplication), group properties of the rotation, and the
+# property the pages give as the reason for the output rotation: with the
+# output turned back by -t, the layer depends on relative positions only.
+
+def test_rms_norm_closed_forms():
+    x = rng.standard_normal((5, 512)) * 3.0
+    y = O.rms_norm(x, np.ones(512), eps=0.0)
+    assert np.allclose((y * y).mean(axis=1), 1.0, atol=1e-12)      # unit RMS
+    ms = (x * x).mean(axis=1)
+    y = O.rms_norm(x, np.ones(512), eps=0.5)
+    assert np.allclose((y * y).mean(axis=1), ms / (ms + 0.5), rtol=1e-12)
+    g = rng.uniform(0.5, 2.0, 512)
+    assert np.allclose(O.rms_norm(x, g, 0.0), O.rms_norm(x, np.ones(512), 0.0) * g)
+    assert np.allclose(O.rms_norm(7.0 * x, g, 0.0), O.rms_norm(x, g, 0.0))  # scale-free
+    assert np.all(O.rms_norm(np.zeros((2, 8)), np.ones(8)) == 0.0)
+
+
+def test_rope_matches_complex_multiplication():
+    c, R, base = 512, 64, 10000.0
+    x = rng.standard_normal((3, c))
+    pos = np.array([0, 7, 131071])
+    got = O.rope_rotate(x, pos, R, base)
+    assert np.array_equal(got[:, :c - R], x[:, :c - R])        # only the last 64 dims
+    z = x[:, c - R::2] + 1j * x[:, c - R + 1::2]
+    theta = np.array([base ** (-(2.0 * j) / R) for j in range(R // 2)])
+    zr = z * np.exp(1j * pos[:, None] * theta[None, :])
+    assert np.allclose(got[:, c - R::2], zr.real, atol=1e-12)
+    assert np.allclose(got[:, c - R + 1::2], zr.imag, atol=1e-12)
+    assert np.array_equal(O.rope_rotate(x, 0, R), x)              # angle 0: identity
+    assert O.rope_theta(R)[0] == 1.0                                # the first pair: 1 rad / pos
+
+
+def test_rope_group_properties():
+    R = 64
+    x = rng.standard_normal((4, 128))
+    a, b = 1234, -987
+    assert np.allclose(O.rope_rotate(O.rope_rotate(x, a, R), b, R), O.rope_rotate(x, a + b, R),
+                       atol=1e-12)
+    assert np.allclose(O.rope_rotate(O.rope_rotate(x, a, R), -a, R), x, atol=1e-12)
+    pairs = lambda v: v[:, -R::2] ** 2 + v[:, -R + 1::2] ** 2        # noqa: E731
+    assert np.allclose(pairs(O.rope_rotate(x, a, R)), pairs(x), atol=1e-12)
+    # relative: <rot(q, a), rot(k, b)> = <rot(q, a - b), k>
+    q, k = rng.standard_normal(128), rng.standard_normal(128)
+    lhs = O.rope_rotate(q, a, R) @ O.rope_rotate(k, b, R)
+    assert np.isclose(lhs, O.rope_rotate(q, a - b, R) @ k, atol=1e-10)
+
+
+def test_norm_rope_attention_depends_on_relative_positions_only():
+    nh, c, N, R = 4, 128, 9, 64
+    q = rng.standard_normal((nh, c))
+    ents = rng.standard_normal((N, c))
+    pos = np.array([0, 4, 8, 20, 21, 22, 23, 24, 25])
+    t = 25
+    gq, gk = rng.uniform(0.5, 1.5, c), rng.uniform(0.5, 1.5, c)
+    sink = rng.standard_normal(nh)
+    o1 = O.attend_norm_rope(q, t, ents, pos, sink, c ** -0.5, gq, gk, R)
+    o2 = O.attend_norm_rope(q, t + 100003, ents, pos + 100003, sink, c ** -0.5, gq, gk, R)
+    assert np.allclose(o1, o2, atol=1e-10)
+    # without the output rotation the result would move with the shift
+    raw = lambda tt, pp: O.rope_rotate(                                # noqa: E731
+        O.attend_norm_rope(q, tt, ents, pp, sink, c ** -0.5, gq, gk, R), tt, R)
+    assert not np.allclose(raw(t, pos), raw(t + 100003, pos + 100003), atol=1e-3)
+
+
+def test_norm_rope_attention_reduces_to_plain_attention():
+    nh, c, N = 3, 64, 6
+    q = rng.standard_normal((nh, c)) * 5
+    ents = rng.standard_normal((N, c)) * 0.2
+    pos = np.arange(N)
+    ones = np.ones(c)
+    # no rotation: plain attention of the normalised vectors, an explicit
+    # softmax written out here
+    got = O.attend_norm_rope(q, 5, ents, pos, None, 0.125, ones, ones, 0, eps=0.0)
+    qn = q / np.sqrt((q * q).mean(axis=1, keepdims=True))
+    en = ents / np.sqrt((ents * ents).mean(axis=1, keepdims=True))
+    p = scipy.special.softmax(0.125 * qn @ en.T, axis=1)
+    assert np.allclose(got, p @ en, atol=1e-12)
+    # the norm bounds every logit: |l| <= scale * c * max|gq| * max|gk| (Cauchy-Schwarz)
+    gq, gk = rng.uniform(0.5, 2.0, c), rng.uniform(0.5, 2.0, c)
+    qq = O.rms_norm(q, gq)
+    ee = O.rms_norm(ents, gk)
+    assert np.abs(qq @ ee.T).max() <= c * gq.max() * gk.max()
+
+
+def test_norm_rope_sparse_attn_entry_positions():
+    # the per-row set and positions: entry s at m*s, window row u at u,
+    # checked against attend_norm_rope on a set assembled by hand
+    n, m, c, nh, W, R = 40, 4, 128, 2, 8, 64
+    q = rng.standard_normal((n, nh, c))
+    kv = rng.standard_normal((n // m, c))
+    win = rng.standard_normal((n, c))
+    g = np.ones(c)
+    t = 37
+    idx = np.full((n, 3), -1)
+    idx[t] = [2, 8, 5]                  # V(37) = 9: entries 0..8 are visible
+    got = O.sparse_attn_norm_rope(q, kv, idx, win, W, None, 0.1, m, g, g, R, rows=[t])[0]
+    ents = np.concatenate([kv[[2, 8, 5]], win[t - W + 1:t + 1]])
+    pos = np.concatenate([[8, 32, 20], np.arange(t - W + 1, t + 1)])
+    assert np.allclose(got, O.attend_norm_rope(q[t], t, ents, pos, None, 0.1, g, g, R),
+                       atol=1e-12)
+    dense = O.hca_attn_norm_rope(q, kv, win, W, None, 0.1, m, g, g, R, rows=[t])[0]
+    ents = np.concatenate([kv[:9], win[t - W + 1:t + 1]])
+    pos = np.concatenate([4 * np.arange(9), np.arange(t - W + 1, t + 1)])
+    assert np.allclose(dense, O.attend_norm_rope(q[t], t, ents, pos, None, 0.1, g, g, R),
+                       atol=1e-12)
