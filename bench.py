@@ -671,6 +671,7 @@ def main():
     del pinned, out_host, sets
 
     launches_per_step = L.launches_per_step
+    layer_calls = L.calls
     workloads = {}
     if not args.skip_extras:
         del L
@@ -701,7 +702,7 @@ def main():
             "roofline": dominant,
             "roofline_per_call": roof,
             "gpu_launches": launches_per_step * args.steps,
-            "kernels_per_call": {c: list(CALL_KERNELS[c]) for c in L.calls},
+            "kernels_per_call": {c: list(CALL_KERNELS[c]) for c in layer_calls},
             "e2e": {"value": round(w.n * w.batch * world / (e2e_ms * 1e-3), 1), "unit": UNIT,
                     "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                     "ms_per_step": round(e2e_ms, 3), "steps": n_e2e,
