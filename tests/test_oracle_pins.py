@@ -600,3 +600,45 @@ def test_norm_rope_sparse_attn_entry_positions():
     pos = np.concatenate([4 * np.arange(9), np.arange(t - W + 1, t + 1)])
     assert np.allclose(dense, O.attend_norm_rope(q[t], t, ents, pos, None, 0.1, g, g, R),
                        atol=1e-12)
+
+
+# --------------------------------------------- low-precision indexer ---------
+
+def test_fp8_index_scores_exact_when_inputs_are_e4m3_values():
+    # vectors whose largest magnitude is 448 get scale 1, and small integers
+    # are E4M3 values: the FP8 form is then exact and equals the plain scores
+    r = np.random.default_rng(7)
+    H, ci, E = 4, 64, 50
+    q = r.integers(-8, 9, (H, ci)).astype(np.float64)
+    q[:, 0] = 448.0
+    K = r.integers(-6, 7, (E, ci)).astype(np.float64)
+    K[:, 1] = -448.0
+    w = r.uniform(0, 1, H)
+    assert np.array_equal(O.index_scores_row_fp8(q, w, K, 40), O.index_scores_row(q, w, K, 40))
+
+
+def test_fp8_index_scores_close_to_plain_on_random_inputs():
+    # E4M3 keeps 3 mantissa bits: each product is off by at most ~2^-3 of its
+    # size, so scores agree to a few percent and most of the top-k survives
+    r = np.random.default_rng(8)
+    H, ci, E, k = 8, 128, 2000, 64
+    q, K, w = r.standard_normal((H, ci)), r.standard_normal((E, ci)), r.uniform(0, 1, H)
+    a = O.index_scores_row(q, w, K, E)
+    b = O.index_scores_row_fp8(q, w, K, E)
+    assert np.abs(a - b).max() <= 0.1 * np.abs(a).max()
+    assert O.selection_recall(O.topk_row(b, k), O.topk_row(a, k)) > 0.8
+
+
+def test_bf16_score_selection_and_recall():
+    # integer scores below 256 are bf16 values: the bf16 selection is exact
+    r = np.random.default_rng(9)
+    sc = r.integers(0, 256, 1000).astype(np.float64)
+    assert np.array_equal(O.topk_row_bf16_scores(sc, 50), O.topk_row(sc, 50))
+    # bf16 spacing is 2 in [256, 512): 257 rounds (to even) to 256 and ties
+    # with it, and the tie goes to the smaller index
+    sc = np.array([256.0, 257.0])
+    assert list(O.topk_row_bf16_scores(sc, 1)) == [0]
+    assert list(O.topk_row(sc, 1)) == [1]
+    assert list(O.bf16_round(np.array([257.0, 259.0]))) == [256.0, 260.0]
+    assert O.selection_recall([1, 2, 3, -1], [2, 3, 4, 5]) == 0.5
+    assert O.selection_recall([-1], [-1]) == 1.0
