@@ -512,6 +512,25 @@ def dequantize_entries(codes, scales, rope) -> np.ndarray:
 
 
 # ---------------------------------------------------------------------------
+# Grouped output projection ([Walk-through] §4.4: the n_h heads are split
+# into G groups; each group's concatenated outputs (n_h/G * c values) are
+# projected to an intermediate dim d_G, and the G intermediate outputs,
+# concatenated, are projected to the model dim d; [Formulas B9] gives
+# V4-Flash n_h = 64, g = 8, d = 4096 and d_g = 1024).  Weights are stored
+# [out, in]: W1 [G, d_G, (n_h/G) c], W2 [d, G d_G].
+# ---------------------------------------------------------------------------
+
+def grouped_output_projection(o, W1, W2) -> np.ndarray:
+    """o [n, n_h, c] -> y [n, d]:  z_g = o_g W1[g]^T,  y = [z_1 .. z_G] W2^T."""
+    o, W1, W2 = f64(o), f64(W1), f64(W2)
+    n, nh, c = o.shape
+    G = W1.shape[0]
+    hpg = nh // G
+    z = [o[:, g * hpg:(g + 1) * hpg, :].reshape(n, hpg * c) @ W1[g].T for g in range(G)]
+    return np.concatenate(z, axis=1) @ W2.T
+
+
+# ---------------------------------------------------------------------------
 # Low-precision lightning indexer ([Analysis] "Lightning Indexer": small head
 # count + FP8 keep the indexer cheap, the ReLU suits FP8; [Analysis] "FP4
 # Quantization-Aware Training": index scores stored in BF16 instead of FP32,

@@ -642,3 +642,36 @@ def test_bf16_score_selection_and_recall():
     assert list(O.bf16_round(np.array([257.0, 259.0]))) == [256.0, 260.0]
     assert O.selection_recall([1, 2, 3, -1], [2, 3, 4, 5]) == 0.5
     assert O.selection_recall([-1], [-1]) == 1.0
+
+
+# --------------------------------------------- grouped output projection ------
+
+def test_grouped_projection_equals_block_diagonal_dense():
+    # the grouped first stage is one dense product with a block-diagonal weight
+    r = np.random.default_rng(11)
+    n, nh, c, G, dg, d = 5, 8, 6, 4, 3, 7
+    o = r.standard_normal((n, nh, c))
+    W1 = r.standard_normal((G, dg, nh // G * c))
+    W2 = r.standard_normal((d, G * dg))
+    blk = np.zeros((G * dg, nh * c))
+    for g in range(G):
+        blk[g * dg:(g + 1) * dg, g * (nh // G) * c:(g + 1) * (nh // G) * c] = W1[g]
+    ref = (o.reshape(n, nh * c) @ blk.T) @ W2.T
+    assert np.allclose(O.grouped_output_projection(o, W1, W2), ref, atol=1e-12)
+
+
+def test_grouped_projection_special_cases():
+    r = np.random.default_rng(12)
+    n, nh, c = 4, 4, 3
+    o = r.standard_normal((n, nh, c))
+    # one group with identity weights returns the flattened heads
+    eye = np.eye(nh * c)[None]
+    assert np.allclose(O.grouped_output_projection(o, eye, np.eye(nh * c)), o.reshape(n, -1))
+    # a head outside group g never reaches z_g: zeroing group 1's heads leaves
+    # only group 0 in y when W2 reads group 0 alone
+    W1 = r.standard_normal((2, 5, 2 * c))
+    W2 = np.concatenate([r.standard_normal((3, 5)), np.zeros((3, 5))], axis=1)
+    o2 = o.copy()
+    o2[:, 2:, :] = r.standard_normal((n, 2, c))
+    assert np.allclose(O.grouped_output_projection(o, W1, W2),
+                       O.grouped_output_projection(o2, W1, W2), atol=1e-12)
