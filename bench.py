@@ -297,7 +297,100 @@ def roofline(kind, amount, ms, peaks):
             "peak_source": peaks["source"] + " bf16_tflops (burst)"}
 
 
-# ------------------------------------------------------------ other layers ---
+def time_region(fn, K, W):
+    """Mean ms of fn() over K runs after W warm-up runs (CUDA events)."""
+    for _ in range(W):
+        fn()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    e0.record()
+    for _ in range(K):
+        fn()
+    e1.record()
+    torch.cuda.synchronize()
+    return e0.elapsed_time(e1) / K
+
+
+def bench_prefill_extras(L, dev, K, W, peaks):
+    """The 'next' rows on the headline workload's tensors: the layer with the
+    query / entry RMSNorm and partial RoPE, the low-precision indexer forms
+    (with their recall against the exact selection on sampled rows), and
+    the grouped output projection (V4-Flash: 8 groups, d_g 1024, d 4096)."""
+    import numpy as np
+    csa, d, w = L.csa, L.d, L.w
+    out = {}
+    # 1. norm + partial RoPE: entries normed as compressed, window rows by the
+    #    row kernel, the query in the attention prologue, the output turned back
+    g = torch.Generator(device="cpu").manual_seed(7)
+    gq = (1.0 + 0.25 * torch.randn(w.c, generator=g)).to(dev)
+    gk = (1.0 + 0.25 * torch.randn(w.c, generator=g)).to(dev)
+    win_n = torch.empty_like(d["kv_win"])
+
+    def nr_step():
+        csa.csa_compress_norm_rope(d["ca"], d["cb"], d["za"], d["zb"], d["ba"], d["bb"], w.m, gk,
+                                   out=L.kv)
+        csa.csa_compress(d["ica"], d["icb"], d["iza"], d["izb"], d["iba"], d["ibb"], w.m,
+                         out=L.ki)
+        csa.csa_index_topk(d["q_i"], d["w_i"], L.ki, w.m, w.k, ws=L.ws, out=L.idx)
+        csa.csa_norm_rope_rows(d["kv_win"], gk, out=win_n)
+        csa.csa_sparse_attn_norm_rope(d["q"], L.kv, L.idx, win_n, w.window, d["sink"], w.scale,
+                                      w.m, gq, out=L.out)
+
+    ms_nr = time_region(nr_step, K, W)
+    ms_plain = time_region(L.step, K, W)
+    ms_rows = time_region(lambda: csa.csa_norm_rope_rows(d["kv_win"], gk, out=win_n), K, W)
+    rows_bytes = 2 * d["kv_win"].numel() * 2
+    out["norm_rope_layer"] = {
+        "metric": "query-tokens/s", "value": round(w.n / (ms_nr * 1e-3), 1),
+        "ms_per_step": round(ms_nr, 4), "plain_ms_per_step": round(ms_plain, 4),
+        "cost_ms": round(ms_nr - ms_plain, 4),
+        "window_rows_kernel": roofline("bytes", rows_bytes, ms_rows, peaks)}
+    # 2. low-precision indexer forms, recall against the exact selection
+    csa.csa_index_topk(d["q_i"], d["w_i"], L.ki, w.m, w.k, ws=L.ws, out=L.idx)
+    ref = L.idx.clone()
+    rows = list(range(w.n - 1, w.k * w.m, -(w.n // 512)))
+    ref_h = ref[0, rows].cpu().numpy()
+    flops = 2 * w.nh_i * w.c_i * sum_visible(w.n, w.m)
+    lw = {}
+    for name, fp8, bf16s in (("fp8_qk+bf16_scores", True, True), ("fp8_qk", True, False),
+                             ("bf16_scores", False, True)):
+        nb = csa.lib().csa_index_topk_lowp_workspace(1, w.n, w.nh_i, w.c_i, w.m, w.k,
+                                                     (1 if fp8 else 0) | (2 if bf16s else 0))
+        ws = torch.empty(nb, dtype=torch.uint8, device=dev)
+        idx = torch.empty_like(L.idx)
+        fn = lambda: csa.csa_index_topk_lowp(d["q_i"], d["w_i"], L.ki, w.m, w.k,  # noqa: E731
+                                             fp8_qk=fp8, bf16_scores=bf16s, ws=ws, out=idx)
+        ms = time_region(fn, K, W)
+        got = idx[0, rows].cpu().numpy()
+        rec = float(np.mean([len(np.intersect1d(a[a >= 0], b[b >= 0])) / max(1, (b >= 0).sum())
+                             for a, b in zip(got, ref_h)]))
+        lw[name] = {"ms": round(ms, 4), "recall_vs_exact": round(rec, 5),
+                    "rows_for_recall": len(rows),
+                    "roofline": roofline("flops", flops, ms, peaks)}
+        del ws, idx
+    lw["exact_ms"] = round(time_region(
+        lambda: csa.csa_index_topk(d["q_i"], d["w_i"], L.ki, w.m, w.k, ws=L.ws, out=L.idx), K, W), 4)
+    lw["note"] = ("fp8 tensor-core peak taken as 2x the measured bf16 burst figure (the recipe's "
+                  "nominal ratio); the roofline lines above are against bf16")
+    out["index_topk_lowp"] = lw
+    # 3. grouped output projection on the attention output
+    G_, dg, dm = 8, 1024, 4096
+    kin = w.nh // G_ * w.c
+    w1 = (torch.randn(G_, dg, kin, generator=g) * kin ** -0.5).to(torch.bfloat16).to(dev)
+    w2 = (torch.randn(dm, G_ * dg, generator=g) * (G_ * dg) ** -0.5).to(torch.bfloat16).to(dev)
+    zws = torch.empty(w.n * G_ * dg * 2, dtype=torch.uint8, device=dev)
+    y = torch.empty((1, w.n, dm), dtype=torch.bfloat16, device=dev)
+    ms_p = time_region(lambda: csa.csa_grouped_out_proj(L.out, w1, w2, ws=zws, out=y), K, W)
+    pflops = 2 * w.n * (G_ * dg * kin + dm * G_ * dg)
+    out["grouped_out_proj"] = {"shape": f"rows {w.n}, heads {w.nh} x {w.c}, {G_} groups, "
+                                        f"d_g {dg}, d {dm}",
+                               "ms": round(ms_p, 4), "roofline": roofline("flops", pflops, ms_p,
+                                                                          peaks)}
+    del w1, w2, zws, y, win_n
+    return out
+
+
+# ------------------------------------------------------------ other layers ---# ------------------------------------------------------------ other layers ---
 
 def bench_hca_prefill(dev, K, W, peaks):
     import compressed_sparse_attention_11_b200 as csa
@@ -673,6 +766,9 @@ def main():
     launches_per_step = L.launches_per_step
     layer_calls = L.calls
     workloads = {}
+    if not args.skip_extras:
+        workloads["csa_prefill_next_rows"] = bench_prefill_extras(L, dev, max(2, args.steps // 4),
+                                                                  2, peaks)
     if not args.skip_extras:
         del L
         torch.cuda.empty_cache()

@@ -32,7 +32,11 @@ EXPORTED = (
     "hca_attn",
     "csa_cache_layout", "csa_cache_store_entries", "csa_cache_write_rows",
     "csa_decode_workspace", "csa_decode_step",
+    "csa_norm_rope_rows", "csa_compress_norm_rope", "csa_sparse_attn_norm_rope",
+    "hca_attn_norm_rope", "csa_index_topk_lowp_workspace", "csa_index_topk_lowp",
+    "csa_grouped_out_proj_workspace", "csa_grouped_out_proj",
 )
+CSA_INDEX_FP8_QK, CSA_INDEX_BF16_SCORES = 1, 2
 
 
 class CsaError(RuntimeError):
@@ -62,7 +66,12 @@ class Rows(ctypes.Structure):
 class DecodeParams(ctypes.Structure):
     _fields_ = [("ba", ctypes.c_void_p), ("bb", ctypes.c_void_p), ("iba", ctypes.c_void_p),
                 ("ibb", ctypes.c_void_p), ("sink", ctypes.c_void_p), ("scale", ctypes.c_float),
-                ("sel_out", ctypes.c_void_p)]
+                ("sel_out", ctypes.c_void_p), ("scores_out", ctypes.c_void_p)]
+
+
+class NormRope(ctypes.Structure):
+    _fields_ = [("gamma", ctypes.c_void_p), ("eps", ctypes.c_float),
+                ("rope_dims", ctypes.c_int32), ("rope_base", ctypes.c_float)]
 
 
 _lib = None
@@ -100,6 +109,19 @@ def lib() -> ctypes.CDLL:
         "csa_decode_workspace": (sz, [ctypes.POINTER(CacheDesc)]),
         "csa_decode_step": (i32, [ctypes.POINTER(CacheDesc), vp, vp, ctypes.POINTER(Rows),
                                   ctypes.POINTER(DecodeParams), vp, vp, vp, vp, vp, sz, vp]),
+        "csa_norm_rope_rows": (i32, [vp, i64, i64, i32, i32, i64, ctypes.POINTER(NormRope), i32,
+                                     vp, vp]),
+        "csa_compress_norm_rope": (i32, [vp, vp, vp, vp, vp, vp, i64, i64, i32, i32, i32, i32,
+                                         ctypes.POINTER(NormRope), vp, vp]),
+        "csa_sparse_attn_norm_rope": (i32, [vp, vp, vp, i32, vp, i32, vp, f32, i64, i64, i32, i32,
+                                            i32, i32, ctypes.POINTER(NormRope), vp, vp]),
+        "hca_attn_norm_rope": (i32, [vp, vp, vp, i32, vp, f32, i64, i64, i32, i32, i32, i32,
+                                     ctypes.POINTER(NormRope), vp, vp]),
+        "csa_grouped_out_proj_workspace": (sz, [i64, i32, i32]),
+        "csa_grouped_out_proj": (i32, [vp, i64, i32, i32, i32, i32, i32, vp, vp, vp, sz, vp, vp]),
+        "csa_index_topk_lowp_workspace": (sz, [i64, i64, i32, i32, i32, i32, i32]),
+        "csa_index_topk_lowp": (i32, [vp, vp, vp, i64, i64, i32, i32, i32, i32, i32, i32, vp, vp,
+                                      sz, vp]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(L, name)
@@ -204,6 +226,24 @@ def csa_index_topk_noalloc(q_i, w_i, k_i, m: int, k: int, out: Optional[torch.Te
     return out
 
 
+def csa_index_topk_lowp(q_i, w_i, k_i, m: int, k: int, fp8_qk: bool = True,
+                        bf16_scores: bool = True, ws: Optional[torch.Tensor] = None,
+                        out: Optional[torch.Tensor] = None):
+    """The indexer + top-k with FP8 query/key scoring and / or bf16-stored
+    scores: indices [B, n, k] int32 (ascending, -1 padded)."""
+    B, n, H, ci = q_i.shape
+    flags = (CSA_INDEX_FP8_QK if fp8_qk else 0) | (CSA_INDEX_BF16_SCORES if bf16_scores else 0)
+    need = int(lib().csa_index_topk_lowp_workspace(B, n, H, ci, m, k, flags))
+    if ws is None:
+        ws = torch.empty(max(need, 16), dtype=torch.uint8, device=q_i.device)
+    if out is None:
+        out = torch.empty((B, n, k), dtype=torch.int32, device=q_i.device)
+    _check(lib().csa_index_topk_lowp(_ptr(q_i), _ptr(w_i), _ptr(k_i), B, n, H, ci, m, k, _dt(q_i),
+                                     flags, _ptr(out), _ptr(ws), ws.numel() * ws.element_size(),
+                                     _stream(q_i)))
+    return out
+
+
 def csa_sparse_attn(q, kv_comp, idx, kv_win, window: int, sink, scale: float, m: int,
                     out: Optional[torch.Tensor] = None):
     B, n, nh, c = q.shape
@@ -222,6 +262,101 @@ def hca_attn(q, kv_comp, kv_win, window: int, sink, scale: float, m_heavy: int,
         out = torch.empty_like(q)
     _check(lib().hca_attn(_ptr(q), _ptr(kv_comp), _ptr(kv_win), window, _ptr(sink), float(scale),
                           B, n, nh, c, m_heavy, _dt(q), _ptr(out), _stream(q)))
+    return out
+
+
+# ------------------------------------------------- RMSNorm and partial RoPE ---
+
+ROPE_BASE = 10000.0
+NORM_EPS = 1e-6
+
+
+def _norm_rope(gamma, eps: float, rope_dims: int, rope_base: float) -> NormRope:
+    if gamma is None or gamma.dtype != torch.float32:
+        raise ValueError("gamma must be a float32 tensor")
+    return NormRope(_ptr(gamma), float(eps), int(rope_dims), float(rope_base))
+
+
+def csa_norm_rope_rows(x, gamma, pos_mul: int = 1, eps: float = NORM_EPS, rope_dims: int = 64,
+                       rope_base: float = ROPE_BASE, out: Optional[torch.Tensor] = None):
+    """RMSNorm + rotation of the trailing dims of every row of x [B, n, c] or
+    [B, n, heads, c]; row t turns for position t * pos_mul (out may be x)."""
+    B, n = x.shape[0], x.shape[1]
+    heads = x.shape[2] if x.dim() == 4 else 1
+    c = x.shape[-1]
+    if out is None:
+        out = torch.empty_like(x)
+    nr = _norm_rope(gamma, eps, rope_dims, rope_base)
+    _check(lib().csa_norm_rope_rows(_ptr(x), B, n, heads, c, int(pos_mul), ctypes.byref(nr),
+                                    _dt(x), _ptr(out), _stream(x)))
+    return out
+
+
+def csa_compress_norm_rope(ca, cb, za, zb, ba, bb, m: int, gamma, eps: float = NORM_EPS,
+                           rope_dims: int = 64, rope_base: float = ROPE_BASE,
+                           out: Optional[torch.Tensor] = None):
+    """csa_compress with each entry i RMSNorm-ed and rotated for position m * i."""
+    overlap = 1 if cb is not None else 0
+    B, n, c = ca.shape
+    if out is None:
+        out = torch.empty((B, n // m, c), dtype=ca.dtype, device=ca.device)
+    nr = _norm_rope(gamma, eps, rope_dims, rope_base)
+    _check(lib().csa_compress_norm_rope(_ptr(ca), _ptr(cb), _ptr(za), _ptr(zb), _ptr(ba),
+                                        _ptr(bb), B, n, c, m, overlap, _dt(ca), ctypes.byref(nr),
+                                        _ptr(out), _stream(ca)))
+    return out
+
+
+def csa_sparse_attn_norm_rope(q, kv_comp, idx, kv_win, window: int, sink, scale: float, m: int,
+                              q_gamma, eps: float = NORM_EPS, rope_dims: int = 64,
+                              rope_base: float = ROPE_BASE, out: Optional[torch.Tensor] = None):
+    """csa_sparse_attn with the query norm + rotation and the output rotation
+    by -t; kv_comp and kv_win must already be normed and rotated."""
+    B, n, nh, c = q.shape
+    if out is None:
+        out = torch.empty_like(q)
+    nr = _norm_rope(q_gamma, eps, rope_dims, rope_base)
+    _check(lib().csa_sparse_attn_norm_rope(_ptr(q), _ptr(kv_comp), _ptr(idx), idx.shape[-1],
+                                           _ptr(kv_win), window, _ptr(sink), float(scale), B, n,
+                                           nh, c, m, _dt(q), ctypes.byref(nr), _ptr(out),
+                                           _stream(q)))
+    return out
+
+
+def hca_attn_norm_rope(q, kv_comp, kv_win, window: int, sink, scale: float, m_heavy: int,
+                       q_gamma, eps: float = NORM_EPS, rope_dims: int = 64,
+                       rope_base: float = ROPE_BASE, out: Optional[torch.Tensor] = None):
+    """hca_attn with the query norm + rotation and the output rotation by -t."""
+    B, n, nh, c = q.shape
+    if out is None:
+        out = torch.empty_like(q)
+    nr = _norm_rope(q_gamma, eps, rope_dims, rope_base)
+    _check(lib().hca_attn_norm_rope(_ptr(q), _ptr(kv_comp), _ptr(kv_win), window, _ptr(sink),
+                                    float(scale), B, n, nh, c, m_heavy, _dt(q), ctypes.byref(nr),
+                                    _ptr(out), _stream(q)))
+    return out
+
+
+# ------------------------------------------------------ output projection ---
+
+def csa_grouped_out_proj(o, w1, w2, ws: Optional[torch.Tensor] = None,
+                         out: Optional[torch.Tensor] = None):
+    """Grouped output projection: o [rows, nh, c] (or [B, n, nh, c]) with
+    w1 [G, d_g, nh/G * c] and w2 [d, G * d_g] -> y [rows, d] (bf16)."""
+    nh, c = o.shape[-2], o.shape[-1]
+    rows = o.numel() // (nh * c)
+    G, dg = w1.shape[0], w1.shape[1]
+    d = w2.shape[0]
+    need = int(lib().csa_grouped_out_proj_workspace(rows, G, dg))
+    if ws is None:
+        ws = torch.empty(max(need, 16), dtype=torch.uint8, device=o.device)
+    if out is None:
+        out = torch.empty(o.shape[:-2] + (d,), dtype=o.dtype, device=o.device)
+    if o.dtype != torch.bfloat16 or w1.dtype != torch.bfloat16 or w2.dtype != torch.bfloat16:
+        raise ValueError("the grouped output projection takes bfloat16 tensors")
+    _check(lib().csa_grouped_out_proj(_ptr(o), rows, nh, c, G, dg, d, _ptr(w1), _ptr(w2),
+                                      _ptr(ws), ws.numel() * ws.element_size(), _ptr(out),
+                                      _stream(o)))
     return out
 
 
@@ -282,20 +417,27 @@ class CsaCache:
 
     def decode_step(self, pos, rows: dict, biases: dict, sink, scale: float, q, q_i=None,
                     w_i=None, out: Optional[torch.Tensor] = None,
-                    sel_out: Optional[torch.Tensor] = None):
+                    sel_out: Optional[torch.Tensor] = None,
+                    scores_out: Optional[torch.Tensor] = None):
         """One token per sequence at positions ``pos`` (int64 [B] on device).
 
         ``rows``: per-stream [B, dim] bf16 tensors; ``biases``: ba, bb, iba, ibb
         fp32; returns out [B, nh, c] bf16.  ``sel_out`` (CSA, optional, int32
-        [B, k] on device) receives the selected entry indices."""
+        [B, k] on device) receives the selected entry indices; ``scores_out``
+        (CSA, optional, fp32 [B, capacity] on device) the indexer scores."""
         if out is None:
             out = torch.empty_like(q)
         r = self._rows({k: v for k, v in rows.items()})
         if sel_out is not None and (sel_out.dtype != torch.int32 or not sel_out.is_contiguous()
                                     or sel_out.numel() != self.desc.batch * self.desc.k):
             raise ValueError("sel_out must be a contiguous int32 [batch, k] tensor")
+        if scores_out is not None and (
+                scores_out.dtype != torch.float32 or not scores_out.is_contiguous()
+                or scores_out.numel() != self.desc.batch * self.desc.capacity):
+            raise ValueError("scores_out must be a contiguous float32 [batch, capacity] tensor")
         p = DecodeParams(_ptr(biases.get("ba")), _ptr(biases.get("bb")), _ptr(biases.get("iba")),
-                         _ptr(biases.get("ibb")), _ptr(sink), float(scale), _ptr(sel_out))
+                         _ptr(biases.get("ibb")), _ptr(sink), float(scale), _ptr(sel_out),
+                         _ptr(scores_out))
         if pos.dtype != torch.int64:
             raise ValueError("pos must be int64")
         _check(lib().csa_decode_step(ctypes.byref(self.desc), _ptr(self.buffer), _ptr(pos),

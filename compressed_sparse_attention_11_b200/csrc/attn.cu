@@ -16,6 +16,7 @@
 // head) in the log2 domain (q is pre-scaled by scale*log2(e)).
 #include "common.cuh"
 #include "launch.h"
+#include "rope.cuh"
 
 namespace csa {
 
@@ -27,7 +28,8 @@ template <typename T>
 __global__ void __launch_bounds__(kAttnThreads) attn_kernel(
     const T* __restrict__ q, const T* __restrict__ kv_comp, const int32_t* __restrict__ idx,
     int k, const T* __restrict__ kv_win, int window, const float* __restrict__ sink,
-    float scale, int64_t n, int nh, int c, int m, int64_t E, T* __restrict__ out) {
+    float scale, int64_t n, int nh, int c, int m, int64_t E, QNormRope qn,
+    T* __restrict__ out) {
   extern __shared__ float smem[];
   const int ld = c + 1;
   float* Es = smem;                              // [kAttnTE][c+1]
@@ -46,9 +48,31 @@ __global__ void __launch_bounds__(kAttnThreads) attn_kernel(
   const float qscale = scale * kLog2e;
   for (int e = tid; e < kAttnHG * c; e += kAttnThreads) {
     const int h = e / c, d = e % c;
-    Qs[e] = (h0 + h < nh) ? to_f32(q[((b * n + t) * nh + h0 + h) * c + d]) * qscale : 0.f;
+    const float x = (h0 + h < nh) ? to_f32(q[((b * n + t) * nh + h0 + h) * c + d]) : 0.f;
+    Qs[e] = qn.gamma != nullptr ? x : x * qscale;
   }
   const int my_h = h0 + warp;
+  if (qn.gamma != nullptr) {
+    // the query head's RMSNorm and rotation for position t (warp = head)
+    __syncthreads();
+    float* qh = Qs + warp * c;
+    float ss = 0.f;
+    for (int d = lane; d < c; d += 32) ss = fmaf(qh[d], qh[d], ss);
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, off);
+    const float inv = 1.f / sqrtf(ss / (float)c + qn.eps);
+    __syncwarp();
+    for (int d = lane; d < c; d += 32) qh[d] = qh[d] * inv * __ldg(qn.gamma + d);
+    __syncwarp();
+    for (int j = lane; j < qn.rope_dims / 2; j += 32) {
+      float cs, sn;
+      rope_cos_sin(t, j, qn.rope_dims, qn.base, cs, sn);
+      const int d = c - qn.rope_dims + 2 * j;
+      rope_turn(qh[d], qh[d + 1], cs, sn);
+    }
+    __syncwarp();
+    for (int d = lane; d < c; d += 32) qh[d] *= qscale;
+  }
   const int nd = c / 32;  // dims per thread (c % 32 == 0 here; see launcher)
   float acc[16];
 #pragma unroll
@@ -126,6 +150,20 @@ __global__ void __launch_bounds__(kAttnThreads) attn_kernel(
     const float den = run_sum + (z == kNegInf ? 0.f : ex2(z - run_max));
     const float inv = 1.f / den;
     T* o = out + ((b * n + t) * nh + my_h) * c;
+    if (qn.gamma != nullptr && qn.rope_dims > 0) {
+      // the output's trailing dims turned back by position -t: dims lane + 32 j
+      // pair with their neighbour lane (lane ^ 1)
+#pragma unroll
+      for (int j = 0; j < 16; ++j) {
+        const int d = lane + 32 * j;
+        const float other = __shfl_xor_sync(0xffffffffu, acc[j], 1);
+        if (j < nd && d >= c - qn.rope_dims) {
+          float cs, sn;
+          rope_cos_sin(-t, (d - (c - qn.rope_dims)) >> 1, qn.rope_dims, qn.base, cs, sn);
+          acc[j] = (lane & 1) == 0 ? acc[j] * cs - other * sn : other * sn + acc[j] * cs;
+        }
+      }
+    }
 #pragma unroll
     for (int j = 0; j < 16; ++j)
       if (j < nd) from_f32(o[lane + 32 * j], acc[j] * inv);
@@ -135,12 +173,16 @@ __global__ void __launch_bounds__(kAttnThreads) attn_kernel(
 cudaError_t launch_attn(const void* q, const void* kv_comp, const int32_t* idx, int k,
                         const void* kv_win, int window, const float* sink, float scale,
                         int64_t batch, int64_t n, int nh, int c, int m, csa_dtype dt,
-                        void* out, cudaStream_t s) {
+                        const csa_norm_rope* q_nr, void* out, cudaStream_t s) {
   const int64_t E = n / m;
-  if (attn_tc_supported(nh, c, idx ? k : 0, dt, q, kv_comp ? kv_comp : q, kv_win)) {
+  const QNormRope qn = q_nr != nullptr
+                           ? QNormRope{q_nr->gamma, q_nr->eps, q_nr->rope_dims, q_nr->rope_base}
+                           : QNormRope{nullptr, 0.f, 0, 0.f};
+  if (attn_tc_supported(nh, c, idx ? k : 0, dt, q, kv_comp ? kv_comp : q, kv_win,
+                        qn.gamma != nullptr ? qn.rope_dims : 0)) {
     unsigned int* err = device_timeout_flag();
     if (err == nullptr) return cudaErrorUnknown;
-    return launch_attn_tc(q, kv_comp, idx, k, kv_win, window, sink, scale, batch, n, m, out,
+    return launch_attn_tc(q, kv_comp, idx, k, kv_win, window, sink, scale, batch, n, m, qn, out,
                           err, s);
   }
   const size_t smem = sizeof(float) * ((size_t)kAttnTE * (c + 1) + (size_t)kAttnHG * c +
@@ -151,13 +193,13 @@ cudaError_t launch_attn(const void* q, const void* kv_comp, const int32_t* idx, 
     cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     kern<<<grid, kAttnThreads, smem, s>>>((const float*)q, (const float*)kv_comp, idx, k,
                                           (const float*)kv_win, window, sink, scale, n, nh, c,
-                                          m, E, (float*)out);
+                                          m, E, qn, (float*)out);
   } else {
     auto kern = attn_kernel<__nv_bfloat16>;
     cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     kern<<<grid, kAttnThreads, smem, s>>>(
         (const __nv_bfloat16*)q, (const __nv_bfloat16*)kv_comp, idx, k,
-        (const __nv_bfloat16*)kv_win, window, sink, scale, n, nh, c, m, E,
+        (const __nv_bfloat16*)kv_win, window, sink, scale, n, nh, c, m, E, qn,
         (__nv_bfloat16*)out);
   }
   return cudaGetLastError();

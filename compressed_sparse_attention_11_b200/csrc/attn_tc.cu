@@ -50,6 +50,7 @@
 // 4-7 write each query into tensor memory; warp 11 issues the MMAs.
 #include "common.cuh"
 #include "launch.h"
+#include "rope.cuh"
 #include "sm100.cuh"
 #include "tc_attn_util.cuh"
 
@@ -97,6 +98,7 @@ struct __align__(8) AttnBars {
   uint64_t idx_full;  // the next query's selection row is in shared memory
   uint64_t drain;
   uint64_t grp_prod;  // bounded group barrier of the producer warps (one arrive per warp)
+  uint64_t qinv_full[kMeta];  // (query norm) the query's per-head 1/RMS is in qinv
   uint32_t tmem_base;
 };
 
@@ -106,7 +108,8 @@ constexpr int OFF_LIST = OFF_P + 2 * kPSlabBytes;           // 212992
 constexpr int OFF_IDXN = OFF_LIST + kMaxSel * 4;             // the next query's row
 constexpr int OFF_META = OFF_IDXN + kMaxSel * 4;
 constexpr int OFF_SCAN = OFF_META + kMeta * (int)sizeof(AttnMeta);
-constexpr int OFF_BAR = OFF_SCAN + 64;
+constexpr int OFF_QINV = OFF_SCAN + 64;                       // [kMeta][64] fp32
+constexpr int OFF_BAR = OFF_QINV + kMeta * kNH * 4;
 constexpr int SMEM = OFF_BAR + (int)sizeof(AttnBars) + 1024;
 static_assert(SMEM <= 232448, "shared memory budget");
 
@@ -123,11 +126,46 @@ __device__ __forceinline__ void load_q_round(const uint4* src, uint32_t (&r)[32]
   }
 }
 
+// Query norm: a 64-dim round r (dims d0 .. d0 + 63, two per word) multiplied
+// by gamma, its raw squares added to ss.  The 1/RMS factor itself is applied
+// to the logits (it is one scalar per head).
+__device__ __forceinline__ void q_round_gamma(uint32_t (&r)[32], int d0,
+                                              const float* __restrict__ gamma, float& ss) {
+#pragma unroll
+  for (int w = 0; w < 32; w += 2) {
+    const float4 g = __ldg(reinterpret_cast<const float4*>(gamma + d0 + 2 * w));
+    const float x0 = __uint_as_float(r[w] << 16), x1 = __uint_as_float(r[w] & 0xffff0000u);
+    const float x2 = __uint_as_float(r[w + 1] << 16), x3 = __uint_as_float(r[w + 1] & 0xffff0000u);
+    ss = fmaf(x0, x0, fmaf(x1, x1, fmaf(x2, x2, fmaf(x3, x3, ss))));
+    r[w] = pack_bf16x2(x0 * g.x, x1 * g.y);
+    r[w + 1] = pack_bf16x2(x2 * g.z, x3 * g.w);
+  }
+}
+
+// The last round's pairs that lie in the trailing rope_dims dims (word p =
+// pair p of dims 448 .. 511), turned by the angles of pairs p - (64 - R) / 2
+// whose cosine and sine lane j of the warp holds for pair j.  Every lane of
+// the warp calls it (the shuffles); only `mine` lanes change their words.
+__device__ __forceinline__ void q_round_rope(uint32_t (&r)[32], bool mine, int rope_dims,
+                                             float cs_lane, float sn_lane) {
+  const int p0 = 32 - rope_dims / 2;
+#pragma unroll
+  for (int p = 0; p < 32; ++p) {
+    const float cs = __shfl_sync(0xffffffffu, cs_lane, p >= p0 ? p - p0 : 0);
+    const float sn = __shfl_sync(0xffffffffu, sn_lane, p >= p0 ? p - p0 : 0);
+    if (mine && p >= p0) {
+      float x = __uint_as_float(r[p] << 16), y = __uint_as_float(r[p] & 0xffff0000u);
+      rope_turn(x, y, cs, sn);
+      r[p] = pack_bf16x2(x, y);
+    }
+  }
+}
+
 __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(
     const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ kv_comp,
     const int32_t* __restrict__ idx, int k, const __nv_bfloat16* __restrict__ kv_win,
     int window, const float* __restrict__ sink, float scale, int64_t n, int m, int64_t E,
-    int64_t total, __nv_bfloat16* __restrict__ out, unsigned int* __restrict__ err) {
+    int64_t total, QNormRope qn, __nv_bfloat16* __restrict__ out, unsigned int* __restrict__ err) {
   using namespace sm100;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = smem_raw + ((1024 - (smem_u32(smem_raw) & 1023)) & 1023);
@@ -137,7 +175,9 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(
   int32_t* idxn = reinterpret_cast<int32_t*>(smem + OFF_IDXN);
   AttnMeta* meta = reinterpret_cast<AttnMeta*>(smem + OFF_META);
   int* pscan = reinterpret_cast<int*>(smem + OFF_SCAN);
+  float* qinv = reinterpret_cast<float*>(smem + OFF_QINV);
   AttnBars* bar = reinterpret_cast<AttnBars*>(smem + OFF_BAR);
+  const bool qnorm = qn.gamma != nullptr;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if ((int64_t)blockIdx.x >= total) return;
@@ -152,7 +192,10 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(
       mbar_init(&bar->s_full[u], 1);
       mbar_init(&bar->s_empty[u], kSoftWarps);
     }
-    for (int u = 0; u < kMeta; ++u) mbar_init(&bar->meta_full[u], 1);
+    for (int u = 0; u < kMeta; ++u) {
+      mbar_init(&bar->meta_full[u], 1);
+      mbar_init(&bar->qinv_full[u], 4);  // the four warps that write the query
+    }
     mbar_init(&bar->p_full, kSoftWarps);
     mbar_init(&bar->p_free, 1);
     mbar_init(&bar->q_full_lo, 4);  // the four warps that write the query
@@ -274,7 +317,15 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(
       // half-tile's gather is under way and the old query's first Q.K half is
       // done (rounds 2-3 then load), dims 256-511 after the second half-tile ----
       const uint32_t qaddr = tmem + ((uint32_t)(pw * 32) << 16) + kColQ;
+      // (query norm) this thread's dims of rounds 0-1 start at 64 half, of
+      // rounds 2-3 at 256 + 64 half; raw squares summed over all four rounds
+      const int qhalf = lane >> 4;
+      float qss = 0.f;
       auto write_q_lo = [&]() -> bool {
+        if (qnorm) {
+          q_round_gamma(ra, 64 * qhalf, qn.gamma, qss);
+          q_round_gamma(rb, 128 + 64 * qhalf, qn.gamma, qss);
+        }
         if (kq >= 1 && !mbar_wait(&bar->q_empty_lo, (uint32_t)((kq - 1) & 1), err)) return false;
         tc_fence_after();
         tmem_st16x64(qaddr, ra);
@@ -288,6 +339,19 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(
         return true;
       };
       auto write_q_hi = [&]() -> bool {
+        if (qnorm) {
+          q_round_gamma(ra, 256 + 64 * qhalf, qn.gamma, qss);
+          q_round_gamma(rb, 384 + 64 * qhalf, qn.gamma, qss);
+          if (qn.rope_dims > 0) {  // dims 448 .. 511 sit in round 3 of the upper half
+            float cs = 1.f, sn = 0.f;
+            if (lane < qn.rope_dims / 2) rope_cos_sin(t, lane, qn.rope_dims, qn.base, cs, sn);
+            q_round_rope(rb, qhalf == 1, qn.rope_dims, cs, sn);
+          }
+          const float tot = qss + __shfl_xor_sync(0xffffffffu, qss, 16);
+          if (lane < 16) qinv[(kq % kMeta) * kNH + pw * 16 + lane] = 1.f / sqrtf(tot / kC + qn.eps);
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&bar->qinv_full[kq % kMeta]);
+        }
         if (kq >= 1 && !mbar_wait(&bar->q_empty_hi, (uint32_t)((kq - 1) & 1), err)) return false;
         tc_fence_after();
         tmem_st16x64(qaddr + 128, ra);
@@ -459,6 +523,12 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(
       if (qi >= total) break;
       if (!mbar_wait(&bar->meta_full[kq % kMeta], (uint32_t)((kq / kMeta) & 1), err)) break;
       const AttnMeta mt = meta[kq % kMeta];
+      // (query norm) this head's 1/RMS scales its logits
+      float qscale_h = qscale;
+      if (qnorm) {
+        if (!mbar_wait(&bar->qinv_full[kq % kMeta], (uint32_t)((kq / kMeta) & 1), err)) break;
+        qscale_h = qscale * qinv[(kq % kMeta) * kNH + hd];
+      }
       float m_run = kNegInf;  // running max (log2 units) of head hd
       float l_run = 0.f;      // this thread's share of the head's sum
       bool ok = true;
@@ -476,7 +546,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(
             tmem_ld_wait();
 #pragma unroll
             for (int i = 0; i < 32; ++i)
-              lg[c * 32 + i] = 64 * c + 32 * ch + i < nv ? __uint_as_float(r[i]) * qscale : kNegInf;
+              lg[c * 32 + i] = 64 * c + 32 * ch + i < nv ? __uint_as_float(r[i]) * qscale_h : kNegInf;
           }
         }
         // the S buffer is free for the Q.K of tile g + 2
@@ -550,11 +620,30 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(
       // 128 pp + 64 ch .. + 63 of head hl
       uint8_t* ebuf = sP + (hl >> 3) * kPSlabBytes + warp * 2048 + (hl & 7) * 256;
       __nv_bfloat16* ow = out + ((mt.b * n + mt.t) * kNH + warp * 16) * kC;
+      // (query norm) the output's trailing dims turn back by position -t: lane j
+      // holds the angle of pair j
+      float ocs = 1.f, osn = 0.f;
+      if (qnorm && qn.rope_dims > 0 && lane < qn.rope_dims / 2)
+        rope_cos_sin(-mt.t, lane, qn.rope_dims, qn.base, ocs, osn);
 #pragma unroll 1
       for (int pp = 0; pp < kC / 128; ++pp) {
         uint32_t o[64];
         tmem_ld16x128(o_lane + pp * 128, o);
         tmem_ld_wait();
+        if (qnorm && qn.rope_dims > 0 && pp == kC / 128 - 1) {  // dims 448 .. 511: ch == 1
+          const int p0 = 32 - qn.rope_dims / 2;
+#pragma unroll
+          for (int p = 0; p < 32; ++p) {
+            const float cs = __shfl_sync(0xffffffffu, ocs, p >= p0 ? p - p0 : 0);
+            const float sn = __shfl_sync(0xffffffffu, osn, p >= p0 ? p - p0 : 0);
+            if (ch == 1 && p >= p0) {
+              float x = __uint_as_float(o[2 * p]), y = __uint_as_float(o[2 * p + 1]);
+              rope_turn(x, y, cs, sn);
+              o[2 * p] = __float_as_uint(x);
+              o[2 * p + 1] = __float_as_uint(y);
+            }
+          }
+        }
 #pragma unroll
         for (int jj = 0; jj < 8; ++jj) {
           uint32_t pk[4];
@@ -592,16 +681,16 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(
 }  // namespace
 
 bool attn_tc_supported(int nh, int c, int k, csa_dtype dt, const void* q, const void* kv_comp,
-                       const void* kv_win) {
-  if (dt != CSA_BF16 || nh != kNH || c != kC || k > kMaxSel) return false;
+                       const void* kv_win, int rope_dims) {
+  if (dt != CSA_BF16 || nh != kNH || c != kC || k > kMaxSel || rope_dims > 64) return false;
   return ((reinterpret_cast<uintptr_t>(q) | reinterpret_cast<uintptr_t>(kv_comp) |
            reinterpret_cast<uintptr_t>(kv_win)) & 15) == 0;
 }
 
 cudaError_t launch_attn_tc(const void* q, const void* kv_comp, const int32_t* idx, int k,
                            const void* kv_win, int window, const float* sink, float scale,
-                           int64_t batch, int64_t n, int m, void* out, unsigned int* err,
-                           cudaStream_t s) {
+                           int64_t batch, int64_t n, int m, const QNormRope& qn, void* out,
+                           unsigned int* err, cudaStream_t s) {
   cudaError_t e = cudaFuncSetAttribute(attn_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        SMEM);
   if (e != cudaSuccess) return e;
@@ -609,7 +698,7 @@ cudaError_t launch_attn_tc(const void* q, const void* kv_comp, const int32_t* id
   const int64_t grid = std::min<int64_t>(total, sm_count());
   attn_tc_kernel<<<(unsigned)grid, kThreads, SMEM, s>>>(
       (const __nv_bfloat16*)q, (const __nv_bfloat16*)kv_comp, idx, k,
-      (const __nv_bfloat16*)kv_win, window, sink, scale, n, m, n / m, total,
+      (const __nv_bfloat16*)kv_win, window, sink, scale, n, m, n / m, total, qn,
       (__nv_bfloat16*)out, err);
   return cudaGetLastError();
 }

@@ -18,6 +18,7 @@
 // exactly, so a single +inf logit selects its row.
 #include "common.cuh"
 #include "launch.h"
+#include "rope.cuh"
 
 namespace csa {
 
@@ -151,14 +152,29 @@ __device__ __forceinline__ void round_rows(const T* ca, const T* cb, const T* za
   }
 }
 
-// Entries with at most eight rows: one thread per (entry, 8-dim chunk).
-template <typename T>
+// RMSNorm + partial RoPE of the compressed entries (sections 4.5 / 7.4 of
+// "DeepSeek-V4: million-token context"), applied as they are written; entry
+// i is rotated for position m * i.  NULL gamma: plain compression.
+struct EntryNormRope {
+  const float* gamma;
+  float eps;
+  int rope_dims;
+  float base;
+};
+
+// Entries with at most eight rows: one thread per (entry, 8-dim chunk).  With
+// the norm, an entry's c / 8 threads (a power of two dividing the block) sum
+// their squares by shuffles, and across warps through shared memory.
+template <typename T, bool kNorm>
 __global__ void __launch_bounds__(256) compress_rows_kernel(
     const T* __restrict__ ca, const T* __restrict__ cb, const T* __restrict__ za,
     const T* __restrict__ zb, const float* __restrict__ ba, const float* __restrict__ bb,
-    int64_t n, int c, int m, int rows, int64_t E, int64_t items, T* __restrict__ out) {
-  const int64_t g = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
-  if (g >= items) return;
+    int64_t n, int c, int m, int rows, int64_t E, int64_t items, EntryNormRope nr,
+    T* __restrict__ out) {
+  const int64_t g0 = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (!kNorm && g0 >= items) return;
+  const bool act = g0 < items;  // (with the norm every thread reaches the block barrier)
+  const int64_t g = act ? g0 : items - 1;
   const int chunks = c >> 3;
   const int d0 = (int)(g % chunks) * 8;
   const int64_t rest = g / chunks;
@@ -197,24 +213,45 @@ __global__ void __launch_bounds__(256) compress_rows_kernel(
   float o[8];
 #pragma unroll
   for (int q = 0; q < 8; ++q) o[q] = A[q] / S[q];
-  store8(out + (b * E + i) * c + d0, o);
+  if constexpr (kNorm) {
+    __shared__ float wsum[8];
+    float ss = 0.f;
+#pragma unroll
+    for (int q = 0; q < 8; ++q) ss = fmaf(o[q], o[q], ss);
+    const int seg = chunks < 32 ? chunks : 32;
+    for (int off = seg >> 1; off > 0; off >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, off);
+    if (chunks > 32) {  // the entry spans chunks / 32 warps of the block
+      const int warp = threadIdx.x >> 5;
+      if ((threadIdx.x & 31) == 0) wsum[warp] = ss;
+      __syncthreads();
+      const int w0 = warp & ~(chunks / 32 - 1);
+      ss = 0.f;
+      for (int w = 0; w < chunks / 32; ++w) ss += wsum[w0 + w];
+    }
+    const float inv = 1.f / sqrtf(ss / (float)c + nr.eps);
+    norm_rope8(o, d0, c, inv, nr.gamma, (int64_t)m * i, nr.rope_dims, nr.base);
+  }
+  if (act) store8(out + (b * E + i) * c + d0, o);
 }
 
-// Entries with more rows: block (32 chunks) x (R row groups); thread (lane, r)
+// Entries with more rows: block (CX chunks) x (R row groups); thread (x, r)
 // reads rows r, r + R, r + 2R, ... of its chunk in rounds of four; the R
-// states are merged in shared memory.
-template <typename T>
+// states are merged in shared memory.  CX = blockDim.x is 32, or the whole
+// entry's c / 8 chunks (at most 64) when the entry is normed (kNorm): the
+// block then holds the entry and sums its squares itself.
+template <typename T, bool kNorm>
 __global__ void __launch_bounds__(256) compress_split_kernel(
     const T* __restrict__ ca, const T* __restrict__ cb, const T* __restrict__ za,
     const T* __restrict__ zb, const float* __restrict__ ba, const float* __restrict__ bb,
-    int64_t n, int c, int m, int rows, int64_t E, int chunk_blocks, T* __restrict__ out) {
-  extern __shared__ float sh[];  // [3][R][8][32]
-  const int lane = threadIdx.x, r = threadIdx.y, R = blockDim.y;
+    int64_t n, int c, int m, int rows, int64_t E, int chunk_blocks, EntryNormRope nr,
+    T* __restrict__ out) {
+  extern __shared__ float sh[];  // [3][R][8][CX]
+  const int x = threadIdx.x, r = threadIdx.y, R = blockDim.y, CX = blockDim.x;
   const int cblk = (int)(blockIdx.x % chunk_blocks);
   const int64_t ent = blockIdx.x / chunk_blocks;
   const int64_t i = ent % E, b = ent / E;
   const int chunks = c >> 3;
-  const int chunk = cblk * 32 + lane;
+  const int chunk = cblk * CX + x;
   const bool valid = chunk < chunks;
   const int d0 = valid ? chunk * 8 : 0;
 
@@ -229,78 +266,134 @@ __global__ void __launch_bounds__(256) compress_split_kernel(
       for (int q = 0; q < 8; ++q) st[q] = osm_combine(st[q], part[q]);
     }
   }
-  const int plane = R * 8 * 32;
+  const int plane = R * 8 * CX;
 #pragma unroll
   for (int q = 0; q < 8; ++q) {
-    const int at = (r * 8 + q) * 32 + lane;
+    const int at = (r * 8 + q) * CX + x;
     sh[at] = st[q].M;
     sh[plane + at] = st[q].S;
     sh[2 * plane + at] = st[q].A;
   }
   __syncthreads();
-  // thread (lane, r) merges dims r, r + R, ... of its chunk over the R groups
-  float* res = sh;  // reused after the merge: [8][32]
+  // thread (x, r) merges dims r, r + R, ... of its chunk over the R groups
+  float* res = sh;  // reused after the merge: [8][CX]
   float v[8];  // v[u]: dim r + u R
   int nq = 0;
   for (int q = r; q < 8; q += R, ++nq) {
     Osm acc{kNegInf, 0.f, 0.f};
     for (int u = 0; u < R; ++u) {
-      const int at = (u * 8 + q) * 32 + lane;
+      const int at = (u * 8 + q) * CX + x;
       acc = osm_combine(acc, Osm{sh[at], sh[plane + at], sh[2 * plane + at]});
     }
     v[nq] = acc.A / acc.S;
   }
   __syncthreads();
-  for (int u = 0; u < nq; ++u) res[(r + u * R) * 32 + lane] = v[u];
+  for (int u = 0; u < nq; ++u) res[(r + u * R) * CX + x] = v[u];
   __syncthreads();
-  if (r == 0 && valid) {
+  if (r == 0) {
     float o[8];
 #pragma unroll
-    for (int q = 0; q < 8; ++q) o[q] = res[q * 32 + lane];
-    store8(out + (b * E + i) * c + d0, o);
+    for (int q = 0; q < 8; ++q) o[q] = res[q * CX + x];
+    if constexpr (kNorm) {
+      // the block holds the whole entry: sum of squares over its CX chunks
+      float ss = 0.f;
+      if (valid)
+#pragma unroll
+        for (int q = 0; q < 8; ++q) ss = fmaf(o[q], o[q], ss);
+#pragma unroll
+      for (int off = 16; off > 0; off >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, off);
+      float* wsum = sh + 8 * CX;  // past res
+      if ((x & 31) == 0) wsum[x >> 5] = ss;
+      asm volatile("bar.sync 1, %0;" ::"r"(CX) : "memory");  // the r == 0 threads only
+      ss = 0.f;
+      for (int w = 0; w < (CX + 31) / 32; ++w) ss += wsum[w];
+      const float inv = 1.f / sqrtf(ss / (float)c + nr.eps);
+      if (valid) norm_rope8(o, d0, c, inv, nr.gamma, (int64_t)m * i, nr.rope_dims, nr.base);
+    }
+    if (valid) store8(out + (b * E + i) * c + d0, o);
   }
 }
 
 template <typename T>
 cudaError_t launch_compress_t(const void* ca, const void* cb, const void* za, const void* zb,
                               const float* ba, const float* bb, int64_t batch, int64_t n, int c,
-                              int m, int overlap, void* out, cudaStream_t s) {
+                              int m, int overlap, const csa_norm_rope* nr, void* out,
+                              cudaStream_t s) {
   const int64_t E = n / m;
   const int rows = overlap ? 2 * m : m;
   if (batch * E == 0) return cudaSuccess;
+  const int chunks = c / 8;
+  const bool fused = nr != nullptr && chunks <= 256 && 256 % chunks == 0;
   if (rows <= 8) {
-    const int64_t items = batch * E * (c / 8);
-    compress_rows_kernel<T><<<(unsigned)((items + 255) / 256), 256, 0, s>>>(
+    const int64_t items = batch * E * chunks;
+    const unsigned grid = (unsigned)((items + 255) / 256);
+    if (fused) {
+      const EntryNormRope enr{nr->gamma, nr->eps, nr->rope_dims, nr->rope_base};
+      compress_rows_kernel<T, true><<<grid, 256, 0, s>>>(
+          (const T*)ca, (const T*)cb, (const T*)za, (const T*)zb, ba, bb, n, c, m, rows, E,
+          items, enr, (T*)out);
+      return cudaGetLastError();
+    }
+    compress_rows_kernel<T, false><<<grid, 256, 0, s>>>(
         (const T*)ca, (const T*)cb, (const T*)za, (const T*)zb, ba, bb, n, c, m, rows, E, items,
-        (T*)out);
+        EntryNormRope{nullptr, 0.f, 0, 0.f}, (T*)out);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess || nr == nullptr) return e;
+    // the entry's chunks do not tile a block: norm and rotation as a second
+    // pass over the (small) compressed output, in place
+    return launch_norm_rope_rows(out, batch, E, 1, c, m, nr,
+                                 sizeof(T) == 2 ? CSA_BF16 : CSA_F32, out, s);
+  }
+  // R = groups of rows: one round per thread where possible; with the norm
+  // the block takes the whole entry (c / 8 <= 64 chunks, a multiple of 32)
+  constexpr int kSlots = Raw8<T>::kSlots;
+  const bool split_fused = nr != nullptr && chunks <= 64 && chunks % 32 == 0;
+  const int CX = split_fused ? chunks : 32;
+  const int max_r = 256 / CX;
+  int R = 1;
+  while (R < max_r && R * kSlots < rows) R <<= 1;
+  const int chunk_blocks = (chunks + CX - 1) / CX;
+  const size_t smem = (size_t)3 * R * 8 * CX * sizeof(float) + 64;
+  const unsigned grid = (unsigned)(batch * E * chunk_blocks);
+  cudaError_t e;
+  if (split_fused) {
+    auto kern = compress_split_kernel<T, true>;
+    if (smem > 48 * 1024 &&
+        (e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem)) !=
+            cudaSuccess)
+      return e;
+    kern<<<grid, dim3(CX, R), smem, s>>>((const T*)ca, (const T*)cb, (const T*)za,
+                                         (const T*)zb, ba, bb, n, c, m, rows, E, chunk_blocks,
+                                         EntryNormRope{nr->gamma, nr->eps, nr->rope_dims,
+                                                       nr->rope_base},
+                                         (T*)out);
     return cudaGetLastError();
   }
-  // R = groups of rows: one round per thread where possible, at most 8 groups
-  constexpr int kSlots = Raw8<T>::kSlots;
-  int R = 1;
-  while (R < 8 && R * kSlots < rows) R <<= 1;
-  const int chunk_blocks = (c / 8 + 31) / 32;
-  const size_t smem = (size_t)3 * R * 8 * 32 * sizeof(float);
-  auto kern = compress_split_kernel<T>;
-  if (smem > 48 * 1024) {
-    const cudaError_t e =
-        cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (e != cudaSuccess) return e;
-  }
-  kern<<<(unsigned)(batch * E * chunk_blocks), dim3(32, R), smem, s>>>(
-      (const T*)ca, (const T*)cb, (const T*)za, (const T*)zb, ba, bb, n, c, m, rows, E,
-      chunk_blocks, (T*)out);
-  return cudaGetLastError();
+  auto kern = compress_split_kernel<T, false>;
+  if (smem > 48 * 1024 &&
+      (e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem)) !=
+          cudaSuccess)
+    return e;
+  kern<<<grid, dim3(CX, R), smem, s>>>((const T*)ca, (const T*)cb, (const T*)za, (const T*)zb,
+                                       ba, bb, n, c, m, rows, E, chunk_blocks,
+                                       EntryNormRope{nullptr, 0.f, 0, 0.f}, (T*)out);
+  e = cudaGetLastError();
+  if (e != cudaSuccess || nr == nullptr) return e;
+  // an entry of this kernel spans several blocks: the norm and rotation run as
+  // a second pass over the (n/m rows of) compressed output, in place
+  return launch_norm_rope_rows(out, batch, E, 1, c, m, nr, sizeof(T) == 2 ? CSA_BF16 : CSA_F32,
+                               out, s);
 }
 
 }  // namespace
 
 cudaError_t launch_compress(const void* ca, const void* cb, const void* za, const void* zb,
                             const float* ba, const float* bb, int64_t batch, int64_t n, int c,
-                            int m, int overlap, csa_dtype dt, void* out, cudaStream_t s) {
+                            int m, int overlap, csa_dtype dt, const csa_norm_rope* nr, void* out,
+                            cudaStream_t s) {
   if (dt == CSA_F32)
-    return launch_compress_t<float>(ca, cb, za, zb, ba, bb, batch, n, c, m, overlap, out, s);
-  return launch_compress_t<__nv_bfloat16>(ca, cb, za, zb, ba, bb, batch, n, c, m, overlap,
+    return launch_compress_t<float>(ca, cb, za, zb, ba, bb, batch, n, c, m, overlap, nr, out, s);
+  return launch_compress_t<__nv_bfloat16>(ca, cb, za, zb, ba, bb, batch, n, c, m, overlap, nr,
                                           out, s);
 }
 

@@ -92,6 +92,16 @@ csa_status check_desc(const csa_cache_desc* d) {
   return ok();
 }
 
+csa_status check_norm_rope(const csa_norm_rope* nr, int c) {
+  REQUIRE(nr != nullptr, "nr is NULL");
+  REQUIRE_PTR(nr->gamma);
+  REQUIRE(nr->eps >= 0.f && nr->eps < 3.4e38f, "eps must be finite and >= 0");
+  REQUIRE(nr->rope_dims >= 0 && nr->rope_dims <= c && nr->rope_dims % 8 == 0,
+          "rope_dims must be a multiple of 8 in [0, c]");
+  REQUIRE(nr->rope_base > 1.f && nr->rope_base < 3.4e38f, "rope_base must be finite and > 1");
+  return ok();
+}
+
 }  // namespace
 
 namespace {
@@ -138,7 +148,7 @@ const char* csa_status_string(int status) {
 
 const char* csa_last_error(void) { return g_err; }
 
-int csa_abi_version(void) { return 1; }
+int csa_abi_version(void) { return 2; }
 
 csa_status csa_check(void* stream) {
   cudaError_t e = cudaStreamSynchronize((cudaStream_t)stream);
@@ -186,7 +196,7 @@ csa_status csa_compress(const void* ca, const void* cb, const void* za, const vo
     REQUIRE_PTR(zb);
     REQUIRE_PTR(bb);
   }
-  return cuda_status(launch_compress(ca, cb, za, zb, ba, bb, batch, n, c, m, overlap, dt, out,
+  return cuda_status(launch_compress(ca, cb, za, zb, ba, bb, batch, n, c, m, overlap, dt, nullptr, out,
                                      (cudaStream_t)stream),
                      "csa_compress");
 }
@@ -233,6 +243,98 @@ csa_status csa_index_topk(const void* q_i, const float* w_i, const void* k_i, in
                      "csa_index_topk (top-k)");
 }
 
+namespace {
+// Workspace regions of the low-precision indexer (byte offsets, 256-aligned).
+struct LowpWs {
+  size_t scores, q8, qs, k8, ks, total;
+};
+LowpWs lowp_ws(int64_t batch, int64_t n, int nh_i, int c_i, int m, int flags) {
+  LowpWs w{};
+  const int64_t E = n / m;
+  auto al = [](size_t x) { return (x + 255) & ~(size_t)255; };
+  size_t off = 0;
+  w.scores = off;
+  off = al(off + (size_t)batch * n * E * ((flags & CSA_INDEX_BF16_SCORES) ? 2 : 4));
+  if (flags & CSA_INDEX_FP8_QK) {
+    w.q8 = off; off = al(off + (size_t)batch * n * nh_i * c_i);
+    w.qs = off; off = al(off + (size_t)batch * n * nh_i * 4);
+    w.k8 = off; off = al(off + (size_t)batch * E * c_i);
+    w.ks = off; off = al(off + (size_t)batch * E * 4);
+  }
+  w.total = off;
+  return w;
+}
+}  // namespace
+
+size_t csa_index_topk_lowp_workspace(int64_t batch, int64_t n, int nh_i, int c_i, int m, int k,
+                                     int flags) {
+  (void)k;
+  if (batch <= 0 || n <= 0 || m <= 0 || nh_i <= 0 || c_i <= 0 || flags < 1 || flags > 3) return 0;
+  return lowp_ws(batch, n, nh_i, c_i, m, flags).total;
+}
+
+csa_status csa_index_topk_lowp(const void* q_i, const float* w_i, const void* k_i, int64_t batch,
+                               int64_t n, int nh_i, int c_i, int m, int k, csa_dtype dt,
+                               int flags, int32_t* idx, void* ws, size_t ws_bytes, void* stream) {
+  REQUIRE(valid_dt(dt), "dt must be CSA_F32 or CSA_BF16");
+  REQUIRE(batch >= 0 && n >= 0, "batch and n must be >= 0");
+  REQUIRE(nh_i >= 1, "nh_i must be >= 1");
+  REQUIRE(c_i >= 8 && c_i % 8 == 0, "c_i must be a positive multiple of 8");
+  REQUIRE(m >= 1, "m must be >= 1");
+  REQUIRE(k >= 1, "k must be >= 1");
+  REQUIRE(flags >= 1 && flags <= 3, "flags must combine CSA_INDEX_FP8_QK and CSA_INDEX_BF16_SCORES");
+  const bool fp8 = (flags & CSA_INDEX_FP8_QK) != 0, bf16s = (flags & CSA_INDEX_BF16_SCORES) != 0;
+  if (dt != CSA_BF16) return fail(CSA_ERR_UNSUPPORTED, "the low-precision indexer takes bf16 inputs");
+  if (fp8 && !index_fp8_supported(nh_i, c_i))
+    return fail(CSA_ERR_UNSUPPORTED, "the FP8 indexer needs c_i = 128 and nh_i in {16, 32, 64, 128}");
+  const int64_t E = n / m;
+  if (bf16s && E > 32768)
+    return fail(CSA_ERR_UNSUPPORTED, "bf16 scores need n/m <= 32768");
+  if (batch == 0 || n == 0) return ok();
+  REQUIRE_PTR(idx);
+  if (bf16s && !fp8 && !index_scores_tc_supported(nh_i, c_i, dt, q_i, k_i))
+    return fail(CSA_ERR_UNSUPPORTED, "bf16 scores need the tensor-core indexer shape");
+  if (E > 0) {
+    REQUIRE_PTR(q_i);
+    REQUIRE_PTR(w_i);
+    REQUIRE_PTR(k_i);
+    const size_t need = csa_index_topk_lowp_workspace(batch, n, nh_i, c_i, m, k, flags);
+    if (ws_bytes < need || ws == nullptr)
+      return fail(CSA_ERR_WORKSPACE, "workspace %zu bytes < required %zu", ws_bytes, need);
+    REQUIRE_PTR(ws);
+  }
+  cudaStream_t s = (cudaStream_t)stream;
+  const LowpWs L = lowp_ws(batch, n, nh_i, c_i, m, flags);
+  uint8_t* wb = static_cast<uint8_t*>(ws);
+  if (E > 0) {
+    unsigned int* flag = device_timeout_flag();
+    if (flag == nullptr) return fail(CSA_ERR_CUDA, "csa_index_topk_lowp: no device flag");
+    cudaError_t e;
+    if (fp8) {
+      uint8_t* q8 = wb + L.q8;
+      float* qs = reinterpret_cast<float*>(wb + L.qs);
+      uint8_t* k8 = wb + L.k8;
+      float* ks = reinterpret_cast<float*>(wb + L.ks);
+      if ((e = launch_quantize_rows_fp8(q_i, batch * n * nh_i, q8, qs, s)) != cudaSuccess ||
+          (e = launch_quantize_rows_fp8(k_i, batch * E, k8, ks, s)) != cudaSuccess)
+        return cuda_status(e, "csa_index_topk_lowp (quantize)");
+      e = launch_index_scores_fp8(q8, qs, k8, ks, w_i, batch, n, nh_i, m, wb + L.scores, bf16s, E,
+                                  flag, s);
+    } else {
+      e = launch_index_scores_tc(q_i, w_i, k_i, batch, n, nh_i, c_i, m, wb + L.scores, true, E,
+                                 flag, s);
+    }
+    if (e != cudaSuccess) return cuda_status(e, "csa_index_topk_lowp (scores)");
+  }
+  if (bf16s)
+    return cuda_status(launch_topk_rows_bf16(reinterpret_cast<const __nv_bfloat16*>(wb + L.scores),
+                                             E, batch, n, m, E, k, idx, s),
+                       "csa_index_topk_lowp (top-k)");
+  return cuda_status(launch_topk_rows(reinterpret_cast<const float*>(wb + L.scores), E, batch, n,
+                                      m, E, k, idx, s),
+                     "csa_index_topk_lowp (top-k)");
+}
+
 csa_status csa_sparse_attn(const void* q, const void* kv_comp, const int32_t* idx, int k,
                            const void* kv_win, int window, const float* sink, float scale,
                            int64_t batch, int64_t n, int nh, int c, int m, csa_dtype dt,
@@ -243,7 +345,7 @@ csa_status csa_sparse_attn(const void* q, const void* kv_comp, const int32_t* id
   if (st != CSA_OK || batch == 0 || n == 0) return st;
   REQUIRE_PTR(idx);
   return cuda_status(launch_attn(q, kv_comp, idx, k, kv_win, window, sink, scale, batch, n, nh,
-                                 c, m, dt, out, (cudaStream_t)stream),
+                                 c, m, dt, nullptr, out, (cudaStream_t)stream),
                      "csa_sparse_attn");
 }
 
@@ -254,8 +356,118 @@ csa_status hca_attn(const void* q, const void* kv_comp, const void* kv_win, int 
                                     dt, out, sink);
   if (st != CSA_OK || batch == 0 || n == 0) return st;
   return cuda_status(launch_attn(q, kv_comp, nullptr, 0, kv_win, window, sink, scale, batch, n,
-                                 nh, c, m_heavy, dt, out, (cudaStream_t)stream),
+                                 nh, c, m_heavy, dt, nullptr, out, (cudaStream_t)stream),
                      "hca_attn");
+}
+
+csa_status csa_norm_rope_rows(const void* x, int64_t batch, int64_t n, int heads, int c,
+                              int64_t pos_mul, const csa_norm_rope* nr, csa_dtype dt, void* out,
+                              void* stream) {
+  REQUIRE(valid_dt(dt), "dt must be CSA_F32 or CSA_BF16");
+  REQUIRE(batch >= 0 && n >= 0, "batch and n must be >= 0");
+  REQUIRE(heads >= 1, "heads must be >= 1");
+  REQUIRE(c >= 8 && c % 8 == 0, "c must be a positive multiple of 8");
+  REQUIRE(pos_mul >= 0, "pos_mul must be >= 0");
+  csa_status st = check_norm_rope(nr, c);
+  if (st != CSA_OK) return st;
+  if (c > 1024) return fail(CSA_ERR_UNSUPPORTED, "csa_norm_rope_rows needs c <= 1024");
+  if (batch == 0 || n == 0) return ok();
+  REQUIRE_PTR(x);
+  REQUIRE_PTR(out);
+  return cuda_status(launch_norm_rope_rows(x, batch, n, heads, c, pos_mul, nr, dt, out,
+                                           (cudaStream_t)stream),
+                     "csa_norm_rope_rows");
+}
+
+csa_status csa_compress_norm_rope(const void* ca, const void* cb, const void* za,
+                                  const void* zb, const float* ba, const float* bb,
+                                  int64_t batch, int64_t n, int c, int m, int overlap,
+                                  csa_dtype dt, const csa_norm_rope* nr, void* out,
+                                  void* stream) {
+  REQUIRE(valid_dt(dt), "dt must be CSA_F32 or CSA_BF16");
+  REQUIRE(batch >= 0 && n >= 0, "batch and n must be >= 0");
+  REQUIRE(c >= 8 && c % 8 == 0, "c must be a positive multiple of 8");
+  REQUIRE(m >= 1, "m must be >= 1");
+  REQUIRE(overlap == 0 || overlap == 1, "overlap must be 0 or 1");
+  if (!overlap)
+    REQUIRE(cb == nullptr && zb == nullptr && bb == nullptr,
+            "cb, zb and bb must be NULL when overlap == 0");
+  csa_status st = check_norm_rope(nr, c);
+  if (st != CSA_OK) return st;
+  if (c > 1024) return fail(CSA_ERR_UNSUPPORTED, "the entry norm needs c <= 1024");
+  if (batch == 0 || n / m == 0) return ok();
+  REQUIRE_PTR(ca);
+  REQUIRE_PTR(za);
+  REQUIRE_PTR(ba);
+  REQUIRE_PTR(out);
+  if (overlap) {
+    REQUIRE_PTR(cb);
+    REQUIRE_PTR(zb);
+    REQUIRE_PTR(bb);
+  }
+  return cuda_status(launch_compress(ca, cb, za, zb, ba, bb, batch, n, c, m, overlap, dt, nr,
+                                     out, (cudaStream_t)stream),
+                     "csa_compress_norm_rope");
+}
+
+csa_status csa_sparse_attn_norm_rope(const void* q, const void* kv_comp, const int32_t* idx,
+                                     int k, const void* kv_win, int window, const float* sink,
+                                     float scale, int64_t batch, int64_t n, int nh, int c, int m,
+                                     csa_dtype dt, const csa_norm_rope* nr, void* out,
+                                     void* stream) {
+  REQUIRE(k >= 1, "k must be >= 1");
+  csa_status st = check_attn_common(q, kv_comp, kv_win, window, scale, batch, n, nh, c, m, dt,
+                                    out, sink);
+  if (st != CSA_OK) return st;
+  if ((st = check_norm_rope(nr, c)) != CSA_OK) return st;
+  if (batch == 0 || n == 0) return ok();
+  REQUIRE_PTR(idx);
+  return cuda_status(launch_attn(q, kv_comp, idx, k, kv_win, window, sink, scale, batch, n, nh,
+                                 c, m, dt, nr, out, (cudaStream_t)stream),
+                     "csa_sparse_attn_norm_rope");
+}
+
+csa_status hca_attn_norm_rope(const void* q, const void* kv_comp, const void* kv_win, int window,
+                              const float* sink, float scale, int64_t batch, int64_t n, int nh,
+                              int c, int m_heavy, csa_dtype dt, const csa_norm_rope* nr,
+                              void* out, void* stream) {
+  csa_status st = check_attn_common(q, kv_comp, kv_win, window, scale, batch, n, nh, c, m_heavy,
+                                    dt, out, sink);
+  if (st != CSA_OK) return st;
+  if ((st = check_norm_rope(nr, c)) != CSA_OK) return st;
+  if (batch == 0 || n == 0) return ok();
+  return cuda_status(launch_attn(q, kv_comp, nullptr, 0, kv_win, window, sink, scale, batch, n,
+                                 nh, c, m_heavy, dt, nr, out, (cudaStream_t)stream),
+                     "hca_attn_norm_rope");
+}
+
+size_t csa_grouped_out_proj_workspace(int64_t rows, int groups, int d_g) {
+  if (rows <= 0 || groups <= 0 || d_g <= 0) return 0;
+  return (size_t)rows * groups * d_g * 2;
+}
+
+csa_status csa_grouped_out_proj(const void* o, int64_t rows, int nh, int c, int groups, int d_g,
+                                int d, const void* w1, const void* w2, void* ws,
+                                size_t ws_bytes, void* y, void* stream) {
+  REQUIRE(rows >= 0, "rows must be >= 0");
+  REQUIRE(nh >= 1 && c >= 1 && groups >= 1 && d_g >= 1 && d >= 1,
+          "nh, c, groups, d_g and d must be >= 1");
+  REQUIRE(nh % groups == 0, "nh must be a multiple of groups");
+  if ((int64_t)(nh / groups) * c % 64 != 0 || d_g % 256 != 0 || d % 256 != 0)
+    return fail(CSA_ERR_UNSUPPORTED,
+                "grouped projection needs (nh/groups)*c %% 64 == 0, d_g %% 256 == 0, d %% 256 == 0");
+  if (rows == 0) return ok();
+  REQUIRE_PTR(o);
+  REQUIRE_PTR(w1);
+  REQUIRE_PTR(w2);
+  REQUIRE_PTR(y);
+  const size_t need = csa_grouped_out_proj_workspace(rows, groups, d_g);
+  if (ws == nullptr || ws_bytes < need)
+    return fail(CSA_ERR_WORKSPACE, "workspace %zu bytes < required %zu", ws_bytes, need);
+  REQUIRE_PTR(ws);
+  return cuda_status(launch_grouped_out_proj(o, rows, nh, c, groups, d_g, d, w1, w2, ws, y,
+                                             (cudaStream_t)stream),
+                     "csa_grouped_out_proj");
 }
 
 csa_status csa_cache_layout(const csa_cache_desc* desc, csa_cache_layout_t* layout) {
@@ -339,6 +551,11 @@ csa_status csa_decode_step(const csa_cache_desc* desc, void* cache, const int64_
     REQUIRE_PTR(q_i);
     REQUIRE_PTR(w_i);
   }
+  REQUIRE_OPT_PTR(params->sel_out);
+  REQUIRE_OPT_PTR(params->scores_out);
+  if (!desc->is_hca && params->scores_out != nullptr && !decode_index_tc_supported(*desc))
+    return fail(CSA_ERR_UNSUPPORTED,
+                "scores_out needs the tensor-core indexer shape (c_i = 128, nh_i 64 or 128)");
   const size_t need = decode_workspace(*desc);
   if (ws == nullptr || ws_bytes < need)
     return fail(CSA_ERR_WORKSPACE, "workspace %zu bytes < required %zu", ws_bytes, need);

@@ -360,7 +360,9 @@ __global__ void __launch_bounds__(1024) append_emit_kernel(csa_cache_desc d, Cac
                                                           csa_rows rows, csa_decode_params p,
                                                           const __nv_bfloat16* __restrict__ q_i,
                                                           const float* __restrict__ w_i,
-                                                          uint8_t* __restrict__ qop) {
+                                                          uint8_t* __restrict__ qop,
+                                                          uint32_t* __restrict__ ghist,
+                                                          uint32_t* __restrict__ sel_done) {
   extern __shared__ float sx[];  // [c + c_i] + 32
   const int64_t b = blockIdx.x;
   // the previous step's kernels read the window slot this token overwrites
@@ -369,6 +371,13 @@ __global__ void __launch_bounds__(1024) append_emit_kernel(csa_cache_desc d, Cac
   if (blockIdx.y == 1) {  // the indexer's query operand, for every sequence
     build_query_operand(q_i + b * d.nh_i * 128, w_i + b * d.nh_i, d.nh_i,
                         qop + b * decode_qop_bytes(d.nh_i));
+    // the score histogram the indexer adds to, and the selection's count of
+    // finished slices, start at zero
+    if (ghist != nullptr) {
+      uint4* gh = reinterpret_cast<uint4*>(ghist + b * kDecHistBins);
+      for (int e = threadIdx.x; e < kDecHistBins / 4; e += blockDim.x) gh[e] = make_uint4(0, 0, 0, 0);
+      if (threadIdx.x == 0) sel_done[b] = 0u;
+    }
     return;
   }
   const int64_t t = pos[b];
@@ -668,8 +677,8 @@ __global__ void __launch_bounds__(256) attn_combine_kernel(
 // ---------------------------------------------------------------------------
 struct DecodeWs {
   int nchunks, nsplit;
-  bool tc_index, tc_attn;
-  size_t cand_score, cand_idx, scores, qop, sel, part_o, part_ms, total;
+  bool tc_index, tc_attn, hist_select;
+  size_t cand_score, cand_idx, scores, qop, sel, part_o, part_ms, select, total;
 };
 
 static DecodeWs decode_ws_layout(const csa_cache_desc& d) {
@@ -689,6 +698,10 @@ static DecodeWs decode_ws_layout(const csa_cache_desc& d) {
   w.sel = off;        off = align256(off + B * (d.is_hca ? 0 : d.k) * 4);
   w.part_o = off;     off = align256(off + B * w.nsplit * d.nh * (size_t)d.c * 4);
   w.part_ms = off;    off = align256(off + B * w.nsplit * d.nh * 2 * 4);
+  w.hist_select = w.tc_index && decode_select_supported(d);
+  size_t sel_bytes = 0;
+  if (w.hist_select) decode_select_ws(d, nullptr, &sel_bytes);
+  w.select = off;     off = align256(off + sel_bytes);
   w.total = off;
   return w;
 }
@@ -715,19 +728,24 @@ cudaError_t launch_decode_step(const csa_cache_desc& d, const CacheView& cv, con
   const int want = std::max(dims, qop != nullptr ? d.nh_i * 16 : 0);
   const unsigned emit_threads = (unsigned)std::min(1024, std::max(256, (want + 31) / 32 * 32));
   const size_t emit_smem = sizeof(float) * (dims + 32);
+  size_t sel_bytes = 0;
+  const DecodeSelectWs sws =
+      decode_select_ws(d, w.hist_select ? wb + w.select : nullptr, &sel_bytes);
   cudaError_t err = launch_pdl(append_emit_kernel,
                                dim3((unsigned)d.batch, qop != nullptr ? 2u : 1u),
                                dim3(emit_threads), emit_smem, s, d, cv, pos, rows, p,
-                               (const __nv_bfloat16*)q_i, w_i, qop);
+                               (const __nv_bfloat16*)q_i, w_i, qop, sws.ghist, sws.done);
   if (err != cudaSuccess) return err;
   if (!d.is_hca && w.tc_index) {
-    float* scores = reinterpret_cast<float*>(wb + w.scores);
+    float* scores = p.scores_out != nullptr ? p.scores_out : reinterpret_cast<float*>(wb + w.scores);
     unsigned int* flag = device_timeout_flag();
     if (flag == nullptr) return cudaErrorUnknown;
-    err = launch_decode_index_tc(d, cv, pos, qop, scores, flag, s);
+    // (sws.ghist is NULL when the selection below does not use it: the
+    // indexer then keeps no histogram)
+    err = launch_decode_index_tc(d, cv, pos, qop, scores, sws.ghist, flag, s);
     if (err != cudaSuccess) return err;
-    if (decode_topk_supported(d)) {
-      err = launch_decode_topk(d, pos, scores, sel, s);
+    if (w.hist_select) {
+      err = launch_decode_select(d, pos, scores, sws, sel, s);
     } else {
       decode_select_kernel<<<(unsigned)d.batch, kDecSelThreads, 0, s>>>(d, pos, scores, sel);
       err = cudaGetLastError();

@@ -41,6 +41,14 @@ constexpr int kThreads = 384;  // warp 0 TMA, 1 MMA, 2 operand copies, 4-7 / 8-1
 constexpr int kBSlots = 2;               // query operands (sequences) in flight
 constexpr int kWSlots = 16;              // head-weight vectors (sequences) in flight
 constexpr int kSmemLimit = 232448;
+// Per-sequence histogram of the scores' order keys (their top 12 bits): the
+// selection step reads it to find the bin holding the k-th largest score
+// without another pass over the scores.  Two slots, since the two epilogue
+// groups can be on neighbouring sequences at a boundary.
+constexpr int kHistBins = 4096;
+constexpr int kHistShift = 20;
+constexpr int kHistBytes = 2 * kHistBins * 4;
+constexpr int kEpiThreads = 256;  // warps 4-11
 
 template <int S>
 struct __align__(8) DecIdxBars {
@@ -49,6 +57,7 @@ struct __align__(8) DecIdxBars {
   uint32_t tmem_base;
   int j0, count;  // the CTA's first tile (within sequence b0) and its number of tiles
   int64_t b0;
+  unsigned int abort;  // the timeout flag as read once for the whole CTA
 };
 
 // Tiles travel in groups of TPP ("pairs"): one ring stage, one TMEM
@@ -62,15 +71,36 @@ struct DecIdxCfg {
   static constexpr int TPP = 512 / N / 2;          // tiles per pair: 2 (H = 64), 1 (H = 128)
   static constexpr int STAGE_BYTES = TPP * kTileBytes;
   static constexpr int STAGES =
-      (kSmemLimit - 1024 - kBSlots * B_BYTES - kWSlots * H * 4 - 768) / STAGE_BYTES;
+      (kSmemLimit - 1024 - kBSlots * B_BYTES - kWSlots * H * 4 - kHistBytes - 768) / STAGE_BYTES;
   static constexpr int OFF_RAW = 0;
   static constexpr int OFF_B = OFF_RAW + STAGES * STAGE_BYTES;
   static constexpr int OFF_W = OFF_B + kBSlots * B_BYTES;
-  static constexpr int OFF_BAR = OFF_W + kWSlots * H * 4;
+  static constexpr int OFF_HIST = OFF_W + kWSlots * H * 4;
+  static constexpr int OFF_BAR = OFF_HIST + kHistBytes;
   static constexpr int SMEM = OFF_BAR + (int)sizeof(DecIdxBars<STAGES>) + 1024;
   static_assert(SMEM <= kSmemLimit, "shared memory budget");
   static_assert(TPP >= 1 && 2 * TPP * N <= 512, "two accumulator sets in TMEM");
 };
+
+// Adds histogram slot `slot` of this CTA into sequence b's global histogram
+// and clears it.  Called by the 256 epilogue threads once every score of the
+// sequence in this CTA's range has been counted (after a barrier over them).
+__device__ __forceinline__ void flush_hist(uint32_t* hist, int slot, uint32_t* ghist, int64_t b,
+                                           int etid) {
+  uint32_t* hs = hist + slot * kHistBins;
+  uint32_t* gh = ghist + b * kHistBins;
+  for (int j = etid; j < kHistBins; j += kEpiThreads) {
+    const uint32_t c = hs[j];
+    if (c != 0u) {
+      atomicAdd(gh + j, c);
+      hs[j] = 0u;
+    }
+  }
+}
+
+__device__ __forceinline__ void hist_add(uint32_t* hist, int slot, float score) {
+  atomicAdd(hist + slot * kHistBins + (order_key(score) >> kHistShift), 1u);
+}
 
 // Tiles of tk keys of sequence b.
 __device__ __forceinline__ int tiles_of(const int64_t* pos, int64_t b, int m, int64_t cap,
@@ -142,7 +172,7 @@ template <int H>
 __global__ void __launch_bounds__(kThreads, 1) decode_index_tc_kernel(
     const __grid_constant__ CUtensorMap tm_keys, const float* __restrict__ key_scale,
     const uint8_t* __restrict__ qop, const int64_t* __restrict__ pos, int64_t batch, int64_t cap, int m,
-    float* __restrict__ scores, unsigned int* __restrict__ err) {
+    float* __restrict__ scores, uint32_t* __restrict__ ghist, unsigned int* __restrict__ err) {
   using C = DecIdxCfg<H>;
   constexpr int S = C::STAGES;
   using namespace sm100;
@@ -151,8 +181,10 @@ __global__ void __launch_bounds__(kThreads, 1) decode_index_tc_kernel(
   uint8_t* sRaw = smem + C::OFF_RAW;
   uint8_t* sB = smem + C::OFF_B;
   float* sW = reinterpret_cast<float*>(smem + C::OFF_W);
+  uint32_t* sHist = reinterpret_cast<uint32_t*>(smem + C::OFF_HIST);
   DecIdxBars<S>* bar = reinterpret_cast<DecIdxBars<S>*>(smem + C::OFF_BAR);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  for (int j = threadIdx.x; j < 2 * kHistBins; j += kThreads) sHist[j] = 0u;
 
   if (warp == 0) {
     if (lane == 0) {
@@ -192,6 +224,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_index_tc_kernel(
   // previous kernel
   pdl_wait();
   pdl_trigger();
+  if (threadIdx.x == 0) bar->abort = flag_value(err);
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -199,7 +232,8 @@ __global__ void __launch_bounds__(kThreads, 1) decode_index_tc_kernel(
   const int count = bar->count;
   const int64_t b0 = bar->b0;
   const int j0 = bar->j0;
-  const bool live = count > 0 && flag_value(err) == 0;
+  // the same decision in every thread: the barriers of the epilogue need all
+  const bool live = count > 0 && bar->abort == 0;
 
   constexpr int TPP = C::TPP;
   const int npairs = (count + TPP - 1) / TPP;
@@ -315,7 +349,11 @@ __global__ void __launch_bounds__(kThreads, 1) decode_index_tc_kernel(
       ++first;
     }
     float ks_next = first < count ? scale_of(ahead) : 0.f;
+    const int etid = threadIdx.x - 4 * 32;
     int u = -1;
+    // false once a wait of this warp gave up (the flag is set): from then on
+    // nothing is awaited or written, but every barrier below is still reached
+    bool alive = true;
     for (int i = 0; i < count; ++i, it.next(pos, batch, m, cap)) {
       if (i == 0 || it.j == 0) {
         ++u;
@@ -331,40 +369,53 @@ __global__ void __launch_bounds__(kThreads, 1) decode_index_tc_kernel(
         }
         const int k = i / TPP, q = k & 1;
         const uint32_t acc_col = (uint32_t)((q * TPP + i % TPP) * C::N);
-        // the head weights of this sequence are in place
-        if (!mbar_wait(&bar->w_full[u % kWSlots], (uint32_t)((u / kWSlots) & 1), err)) break;
-        const float* w = sW + (u % kWSlots) * H;
-        if (!mbar_wait(&bar->d_full[q], (uint32_t)((k >> 1) & 1), err)) break;
-        tc_fence_after();
-        float acc[8];
+        // the head weights of this sequence are in place, then the accumulator
+        bool ok = alive &&
+                  mbar_wait(&bar->w_full[u % kWSlots], (uint32_t)((u / kWSlots) & 1), err) &&
+                  mbar_wait(&bar->d_full[q], (uint32_t)((k >> 1) & 1), err);
+        ok = __all_sync(0xffffffffu, ok);
+        if (ok) {
+          const float* w = sW + (u % kWSlots) * H;
+          tc_fence_after();
+          float acc[8];
 #pragma unroll
-        for (int e = 0; e < 8; ++e) acc[e] = 0.f;
+          for (int e = 0; e < 8; ++e) acc[e] = 0.f;
 #pragma unroll
-        for (int c = 0; c < H / 32; ++c) {
-          uint32_t dh[32], dl[32];
-          tmem_ld32(lane_addr + acc_col + c * 32, dh);
-          tmem_ld32(lane_addr + acc_col + H + c * 32, dl);
-          tmem_ld_wait();
+          for (int c = 0; c < H / 32; ++c) {
+            uint32_t dh[32], dl[32];
+            tmem_ld32(lane_addr + acc_col + c * 32, dh);
+            tmem_ld32(lane_addr + acc_col + H + c * 32, dl);
+            tmem_ld_wait();
 #pragma unroll
-          for (int e = 0; e < 32; e += 4) {
-            const float4 w4 = *reinterpret_cast<const float4*>(w + c * 32 + e);
-            float* a = &acc[(e >> 2) & 7];
-            *a = fmaf(w4.x, fmaxf(__uint_as_float(dh[e]) + __uint_as_float(dl[e]), 0.f), *a);
-            *a = fmaf(w4.y, fmaxf(__uint_as_float(dh[e + 1]) + __uint_as_float(dl[e + 1]), 0.f), *a);
-            *a = fmaf(w4.z, fmaxf(__uint_as_float(dh[e + 2]) + __uint_as_float(dl[e + 2]), 0.f), *a);
-            *a = fmaf(w4.w, fmaxf(__uint_as_float(dh[e + 3]) + __uint_as_float(dl[e + 3]), 0.f), *a);
+            for (int e = 0; e < 32; e += 4) {
+              const float4 w4 = *reinterpret_cast<const float4*>(w + c * 32 + e);
+              float* a = &acc[(e >> 2) & 7];
+              *a = fmaf(w4.x, fmaxf(__uint_as_float(dh[e]) + __uint_as_float(dl[e]), 0.f), *a);
+              *a = fmaf(w4.y, fmaxf(__uint_as_float(dh[e + 1]) + __uint_as_float(dl[e + 1]), 0.f), *a);
+              *a = fmaf(w4.z, fmaxf(__uint_as_float(dh[e + 2]) + __uint_as_float(dl[e + 2]), 0.f), *a);
+              *a = fmaf(w4.w, fmaxf(__uint_as_float(dh[e + 3]) + __uint_as_float(dl[e + 3]), 0.f), *a);
+            }
+          }
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&bar->d_empty[q]);
+          const float sum = ((acc[0] + acc[1]) + (acc[2] + acc[3])) + ((acc[4] + acc[5]) + (acc[6] + acc[7]));
+          const int64_t sidx = (int64_t)it.j * kKeys + row;
+          if (sidx < V) {
+            const float v = sum * ks;
+            scores[it.b * cap + sidx] = v;
+            hist_add(sHist, u & 1, v);
           }
         }
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&bar->d_empty[q]);
-        const float sum = ((acc[0] + acc[1]) + (acc[2] + acc[3])) + ((acc[4] + acc[5]) + (acc[6] + acc[7]));
-        const int64_t sidx = (int64_t)it.j * kKeys + row;
-        if (sidx < V) scores[it.b * cap + sidx] = sum * ks;
+        alive = ok;
       }
-      if (seq_end) {  // both groups release the sequence's weights once they pass its end
+      if (seq_end) {
+        // both groups release the sequence's weights once they pass its end,
+        // then add its histogram (every score of it in this CTA is counted)
         __syncwarp();
-        if (lane == 0) mbar_arrive(&bar->w_empty[u % kWSlots]);
+        if (lane == 0 && alive) mbar_arrive(&bar->w_empty[u % kWSlots]);
+        alive = !named_bar_or(3, kEpiThreads, !alive);
+        if (alive && ghist != nullptr) flush_hist(sHist, u & 1, ghist, it.b, etid);
       }
     }
   }
@@ -394,12 +445,13 @@ constexpr int kSwKeys = 256;                        // keys per tile (MMA N)
 constexpr int kSwTileBytes = kSwKeys * kCI;         // 32 KB, one ring stage
 constexpr int kSwABytes = 2 * kSwH * 128;           // query operand, 16 KB
 constexpr int kSwRedBytes = 2 * 2 * 4 * kSwKeys * 4;  // [group][buffer][warp][key] fp32
-constexpr int kSwStages =
-    (kSmemLimit - 2048 - kBSlots * kSwABytes - kWSlots * kSwH * 4 - kSwRedBytes) / kSwTileBytes;
+constexpr int kSwStages = (kSmemLimit - 2048 - kBSlots * kSwABytes - kWSlots * kSwH * 4 -
+                           kSwRedBytes - kHistBytes) / kSwTileBytes;
 constexpr int kSwOffA = kSwStages * kSwTileBytes;
 constexpr int kSwOffW = kSwOffA + kBSlots * kSwABytes;
 constexpr int kSwOffRed = kSwOffW + kWSlots * kSwH * 4;
-constexpr int kSwOffBar = kSwOffRed + kSwRedBytes;
+constexpr int kSwOffHist = kSwOffRed + kSwRedBytes;
+constexpr int kSwOffBar = kSwOffHist + kHistBytes;
 constexpr int kSwSmem = kSwOffBar + (int)sizeof(DecIdxBars<kSwStages>) + 1024;
 static_assert(kSwStages >= 4 && kSwSmem <= kSmemLimit, "shared memory budget");
 static_assert(kSwABytes + kSwH * 4 == 64 * (2 * 128 + 4), "query operand record");
@@ -422,7 +474,8 @@ __device__ __forceinline__ void reduce_scatter8(float (&v)[8], int lane) {
 __global__ void __launch_bounds__(kThreads, 1) decode_index_sw_kernel(
     const __grid_constant__ CUtensorMap tm_keys, const float* __restrict__ key_scale,
     const uint8_t* __restrict__ qop, const int64_t* __restrict__ pos, int64_t batch, int64_t cap,
-    int m, float* __restrict__ scores, unsigned int* __restrict__ err) {
+    int m, float* __restrict__ scores, uint32_t* __restrict__ ghist,
+    unsigned int* __restrict__ err) {
   constexpr int S = kSwStages;
   using namespace sm100;
   extern __shared__ uint8_t smem_raw[];
@@ -431,8 +484,10 @@ __global__ void __launch_bounds__(kThreads, 1) decode_index_sw_kernel(
   uint8_t* sA = smem + kSwOffA;
   float* sW = reinterpret_cast<float*>(smem + kSwOffW);
   float* sRed = reinterpret_cast<float*>(smem + kSwOffRed);
+  uint32_t* sHist = reinterpret_cast<uint32_t*>(smem + kSwOffHist);
   DecIdxBars<S>* bar = reinterpret_cast<DecIdxBars<S>*>(smem + kSwOffBar);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  for (int j = threadIdx.x; j < 2 * kHistBins; j += kThreads) sHist[j] = 0u;
 
   if (warp == 0) {
     if (lane == 0) {
@@ -472,6 +527,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_index_sw_kernel(
   // previous kernel
   pdl_wait();
   pdl_trigger();
+  if (threadIdx.x == 0) bar->abort = flag_value(err);
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -479,7 +535,8 @@ __global__ void __launch_bounds__(kThreads, 1) decode_index_sw_kernel(
   const int count = bar->count;
   const int64_t b0 = bar->b0;
   const int j0 = bar->j0;
-  const bool live = count > 0 && flag_value(err) == 0;
+  // the same decision in every thread: the barriers of the epilogue need all
+  const bool live = count > 0 && bar->abort == 0;
 
   if (warp == 0 && live) {
     // ------------------------------- TMA producer --------------------------------
@@ -570,10 +627,14 @@ __global__ void __launch_bounds__(kThreads, 1) decode_index_sw_kernel(
     const int key_in_chunk = 8 * (vk >> 1) + 2 * (lane & 3) + (vk & 1);
     float* red_g = sRed + grp * (2 * 4 * kSwKeys);
     const int p = wq * 32 + lane;  // this thread's key pair in the final sum
+    const int etid = threadIdx.x - 4 * 32;
     TileWalk it;
     it.start(pos, b0, j0, m, cap, kSwKeys);
     int64_t V = 0;
     int u = -1, mine = 0;
+    // false once a wait of this group gave up (the flag is set): from then on
+    // nothing is awaited or written, but every barrier below is still reached
+    bool alive = true;
     for (int i = 0; i < count; ++i, it.next(pos, batch, m, cap)) {
       if (i == 0 || it.j == 0) {
         ++u;
@@ -587,7 +648,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_index_sw_kernel(
         const float ks0 = s0 < V ? __ldcs(ksp) : 0.f;
         const float ks1 = s0 + 1 < V ? __ldcs(ksp + 1) : 0.f;
         const bool ok =
-            mbar_wait(&bar->w_full[u % kWSlots], (uint32_t)((u / kWSlots) & 1), err) &&
+            alive && mbar_wait(&bar->w_full[u % kWSlots], (uint32_t)((u / kWSlots) & 1), err) &&
             mbar_wait(&bar->d_full[grp], (uint32_t)(mine & 1), err);
         float* red = red_g + (mine & 1) * (4 * kSwKeys) + wq * kSwKeys;
         if (ok) {
@@ -623,24 +684,38 @@ __global__ void __launch_bounds__(kThreads, 1) decode_index_sw_kernel(
             }
           }
         }
-        // a failed wait set the error flag; the group leaves together
-        if (named_bar_or(1 + grp, 128, !ok)) break;
-        const float* rs = red_g + (mine & 1) * (4 * kSwKeys) + 2 * p;
-        float2 sum = *reinterpret_cast<const float2*>(rs);
+        // a failed wait set the error flag; the group stops together
+        alive = !named_bar_or(1 + grp, 128, !ok);
+        if (alive) {
+          const float* rs = red_g + (mine & 1) * (4 * kSwKeys) + 2 * p;
+          float2 sum = *reinterpret_cast<const float2*>(rs);
 #pragma unroll
-        for (int w = 1; w < 4; ++w) {
-          const float2 x = *reinterpret_cast<const float2*>(rs + w * kSwKeys);
-          sum.x += x.x;
-          sum.y += x.y;
+          for (int w = 1; w < 4; ++w) {
+            const float2 x = *reinterpret_cast<const float2*>(rs + w * kSwKeys);
+            sum.x += x.x;
+            sum.y += x.y;
+          }
+          float* out = scores + it.b * cap + s0;
+          if (s0 < V) {
+            const float v0 = sum.x * ks0;
+            __stcg(out, v0);
+            hist_add(sHist, u & 1, v0);
+          }
+          if (s0 + 1 < V) {
+            const float v1 = sum.y * ks1;
+            __stcg(out + 1, v1);
+            hist_add(sHist, u & 1, v1);
+          }
         }
-        float* out = scores + it.b * cap + s0;
-        if (s0 < V) __stcg(out, sum.x * ks0);
-        if (s0 + 1 < V) __stcg(out + 1, sum.y * ks1);
         ++mine;
       }
-      if (seq_end) {  // both groups release the sequence's weights once they pass its end
+      if (seq_end) {
+        // both groups release the sequence's weights once they pass its end,
+        // then add its histogram (every score of it in this CTA is counted)
         __syncwarp();
-        if (lane == 0) mbar_arrive(&bar->w_empty[u % kWSlots]);
+        if (lane == 0 && alive) mbar_arrive(&bar->w_empty[u % kWSlots]);
+        alive = !named_bar_or(3, kEpiThreads, !alive);
+        if (alive && ghist != nullptr) flush_hist(sHist, u & 1, ghist, it.b, etid);
       }
     }
   }
@@ -654,7 +729,8 @@ __global__ void __launch_bounds__(kThreads, 1) decode_index_sw_kernel(
 }
 
 cudaError_t launch_sw(const csa_cache_desc& d, const CacheView& cv, const int64_t* pos,
-                      const uint8_t* qop, float* scores, unsigned int* err, cudaStream_t s) {
+                      const uint8_t* qop, float* scores, uint32_t* ghist, unsigned int* err,
+                      cudaStream_t s) {
   CUtensorMap tk;
   if (!make_tmap_3d(&tk, cv.ikey_fp8, 1, kCI, (uint64_t)d.capacity, (uint64_t)d.batch, kCI,
                     (uint64_t)d.capacity * kCI, kCI, kSwKeys))
@@ -666,12 +742,13 @@ cudaError_t launch_sw(const csa_cache_desc& d, const CacheView& cv, const int64_
   const unsigned grid = (unsigned)std::max<int64_t>(1, std::min<int64_t>(sm_count(), max_tiles));
   return launch_pdl(decode_index_sw_kernel, dim3(grid), dim3(kThreads), (size_t)kSwSmem, s, tk,
                     (const float*)cv.ikey_scale, qop, pos, (int64_t)d.batch, (int64_t)d.capacity,
-                    d.m, scores, err);
+                    d.m, scores, ghist, err);
 }
 
 template <int H>
 cudaError_t launch_h(const csa_cache_desc& d, const CacheView& cv, const int64_t* pos,
-                     const uint8_t* qop, float* scores, unsigned int* err, cudaStream_t s) {
+                     const uint8_t* qop, float* scores, uint32_t* ghist, unsigned int* err,
+                     cudaStream_t s) {
   using C = DecIdxCfg<H>;
   CUtensorMap tk;
   if (!make_tmap_3d(&tk, cv.ikey_fp8, 1, kCI, (uint64_t)d.capacity, (uint64_t)d.batch, kCI,
@@ -684,7 +761,7 @@ cudaError_t launch_h(const csa_cache_desc& d, const CacheView& cv, const int64_t
   const unsigned grid = (unsigned)std::max<int64_t>(1, std::min<int64_t>(sm_count(), max_tiles));
   return launch_pdl(kern, dim3(grid), dim3(kThreads), (size_t)C::SMEM, s, tk,
                     (const float*)cv.ikey_scale, qop, pos,
-                    (int64_t)d.batch, (int64_t)d.capacity, d.m, scores, err);
+                    (int64_t)d.batch, (int64_t)d.capacity, d.m, scores, ghist, err);
 }
 
 }  // namespace
@@ -695,10 +772,10 @@ bool decode_index_tc_supported(const csa_cache_desc& d) {
 
 cudaError_t launch_decode_index_tc(const csa_cache_desc& d, const CacheView& cv,
                                    const int64_t* pos, const uint8_t* qop, float* scores,
-                                   unsigned int* err, cudaStream_t s) {
+                                   uint32_t* ghist, unsigned int* err, cudaStream_t s) {
   switch (d.nh_i) {
-    case 64: return launch_sw(d, cv, pos, qop, scores, err, s);
-    case 128: return launch_h<128>(d, cv, pos, qop, scores, err, s);
+    case 64: return launch_sw(d, cv, pos, qop, scores, ghist, err, s);
+    case 128: return launch_h<128>(d, cv, pos, qop, scores, ghist, err, s);
     default: return cudaErrorInvalidValue;
   }
 }

@@ -3,368 +3,333 @@
 // of "DeepSeek-V4: million-token context"; ties to the smaller index, the
 // chosen indices listed ascending; all V entries when V <= k).
 //
-// One thread-block cluster per sequence (up to 16 CTAs); CTA r of the cluster
-// copies the contiguous slice r of the sequence's scores (L2-resident after
-// the indexer) into shared memory as order keys -- unsigned integers whose
-// order is the float order -- so every later pass reads shared memory only.
-// An exact radix refinement then finds the k-th largest key: each pass
-// histograms the keys of the current window into 4096 bins, the bins are
-// summed across the cluster through distributed shared memory (each CTA
-// reduces 4096/CS bins and writes the totals into every peer), and every CTA
-// finds the same bin T where the count from the top reaches what is still
-// needed.  Keys above bin T are chosen.  When bin T holds few keys (the usual
-// case after one pass) they are copied into the first CTA of the cluster,
-// which ranks them by (key descending, index ascending) and publishes the
-// exact cut (key, index) of the k-th choice; otherwise the window narrows to
-// bin T with a 4096x finer bin, until the bin holds one key value or is taken
-// whole (three passes at most for 32-bit keys).  A last pass writes the
-// chosen positions in index order.  Every decision is taken from
-// cluster-wide sums, so all CTAs of a cluster run the same passes and
-// cluster barriers.
-#include <cooperative_groups.h>
-
+// The indexer kernel leaves, next to the scores, a histogram of each
+// sequence's scores over the top 12 bits of their order keys (unsigned
+// integers whose order is the float order).  That fixes, before any score is
+// read again, the bin T where the count from the top reaches k: every score
+// in a higher bin is chosen, none in a lower one, and only the few scores in
+// bin T need ranking.  So the selection is one pass over the scores, spread
+// over many CTAs, plus a small exact step:
+//   * CTA (j, b) takes slice j (4096 scores) of sequence b: it marks the
+//     chosen scores of the slice in a bitmap (one bit per entry) and copies
+//     the slice's bin-T scores, in index order, to the slice's candidate area;
+//   * the last CTA to finish a sequence (an atomic count of finished slices;
+//     no CTA waits for another) gathers the candidates in index order, finds
+//     among them the `need` = k - (count above bin T) largest by the same
+//     order (radix select, ties to the earlier position = the smaller index),
+//     marks them in the bitmap and writes the chosen indices in ascending
+//     order from the bitmap.
 #include "common.cuh"
 #include "launch.h"
 #include "sm100.cuh"
+#include "topk.cuh"
 
 namespace csa {
 
 namespace {
 
-namespace cg = cooperative_groups;
+constexpr int kThreads = 256;
+constexpr int kPer = 16;                   // scores per thread
+constexpr int kSlice = kThreads * kPer;    // 4096 scores per CTA
+constexpr int kBins = kDecHistBins;        // 4096
+constexpr int kBinsPerThread = kBins / kThreads;  // 16
+constexpr int kSmemCand = 2048;            // threshold-bin candidates staged in shared memory
+constexpr int kSmemWords = 2048;           // bitmap words staged in shared memory (65536 entries)
+static_assert(kBins % kThreads == 0 && kSlice % 32 == 0, "shapes");
 
-constexpr int kThreads = 512;
-constexpr int kWarps = kThreads / 32;
-constexpr int kBins = 4096;
-constexpr int kBinBits = 12;
-constexpr int kBinsPerThread = kBins / kThreads;  // 8
-constexpr int kMaxSlice = 45056;                  // keys per CTA (176 KB)
-constexpr int kMaxCluster = 16;                   // above 8: a non-portable cluster size
-constexpr int kSliceTarget = 16384;               // keys per CTA the cluster size aims for
-constexpr int kSmallWin = 512;                    // bin-T keys ranked directly
-
-struct __align__(16) TopkShared {
-  uint32_t hist[kBins];   // this CTA's counts
-  uint32_t ghist[kBins];  // the cluster's counts
-  uint32_t wcnt[kWarps];  // per warp: strict << 16 | window (final pass)
-  uint32_t wred[2][kWarps];
-  uint32_t pub[4];        // read by peers: min, max key; then strict, window counts
-  uint32_t T, G, C;
-  uint32_t cand_key[kSmallWin];  // first CTA: the cluster's bin-T keys and positions
-  int32_t cand_pos[kSmallWin];
-  uint32_t cand_n;
-  uint32_t cut_key;  // written by the first CTA into every CTA
-  int32_t cut_pos;
+struct KeysInGlobal {
+  const uint32_t* k;
+  __device__ __forceinline__ uint32_t key(int64_t i) const { return __ldcg(k + i); }
 };
 
-__device__ __forceinline__ uint32_t bitlen(uint32_t x) { return x == 0 ? 0u : 32u - __clz(x); }
+struct __align__(16) SelShared {
+  SelectShared<kThreads> sel;
+  uint32_t wsum[kThreads / 32];
+  uint32_t T, G, CT;
+  uint32_t last;
+  uint32_t slice_off[kDecMaxSlices + 1];
+};
 
-__global__ void __launch_bounds__(kThreads) decode_topk_kernel(
-    const int64_t* __restrict__ pos, int64_t cap, int m, int k, const float* __restrict__ scores,
-    int32_t* __restrict__ sel, int slice) {
-  cg::cluster_group cl = cg::this_cluster();
-  const int CS = (int)cl.num_blocks(), r = (int)cl.block_rank();
-  extern __shared__ __align__(16) unsigned char smem_raw[];
-  TopkShared& sh = *reinterpret_cast<TopkShared*>(smem_raw);
-  uint32_t* key = reinterpret_cast<uint32_t*>(smem_raw + sizeof(TopkShared));
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int64_t b = blockIdx.y;
-
-  sm100::pdl_wait();  // the scores come from the previous kernel
-  sm100::pdl_trigger();
-  const int64_t t = pos[b];
-  const int64_t V = t < 0 ? 0 : min((t + 1) / m, cap);
-  int32_t* out = sel + b * k;
-  if (V <= k) {  // the same decision in every CTA of the cluster
-    if (r == 0)
-      for (int j = tid; j < k; j += kThreads) out[j] = j < V ? j : -1;
-    return;
+// Block-wide exclusive prefix of v (every thread gets its own and the total).
+__device__ __forceinline__ uint32_t block_excl_scan(uint32_t v, uint32_t* wsum, uint32_t& total) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  uint32_t inc = v;
+#pragma unroll
+  for (int off = 1; off < 32; off <<= 1) {
+    const uint32_t x = __shfl_up_sync(0xffffffffu, inc, off);
+    if (lane >= off) inc += x;
   }
-  const int64_t lo = (int64_t)r * slice;
-  const int n = (int)max((int64_t)0, min((int64_t)slice, V - lo));
-  if (tid == 0) sh.cand_n = 0u;  // peers add to it only after the first cluster barrier
-
-  // 1. slice -> shared memory as order keys; the slice's key range
-  uint32_t mn = 0xffffffffu, mx = 0u;
-  {
-    const float* row = scores + b * cap + lo;
-    constexpr int kBatch = 16;  // loads in flight per thread
-    for (int i0 = tid; i0 < n; i0 += kThreads * kBatch) {
-      float v[kBatch];
-#pragma unroll
-      for (int u = 0; u < kBatch; ++u) {
-        const int i = i0 + u * kThreads;
-        v[u] = i < n ? __ldcg(row + i) : 0.f;
-      }
-#pragma unroll
-      for (int u = 0; u < kBatch; ++u) {
-        const int i = i0 + u * kThreads;
-        if (i < n) {
-          const uint32_t ky = order_key(v[u]);
-          key[i] = ky;
-          mn = min(mn, ky);
-          mx = max(mx, ky);
-        }
-      }
-    }
-#pragma unroll
-    for (int off = 16; off > 0; off >>= 1) {
-      mn = min(mn, __shfl_xor_sync(0xffffffffu, mn, off));
-      mx = max(mx, __shfl_xor_sync(0xffffffffu, mx, off));
-    }
-    if (lane == 0) {
-      sh.wred[0][warp] = mn;
-      sh.wred[1][warp] = mx;
-    }
-    __syncthreads();
-    if (tid == 0) {
-      for (int w = 0; w < kWarps; ++w) {
-        mn = min(mn, sh.wred[0][w]);
-        mx = max(mx, sh.wred[1][w]);
-      }
-      sh.pub[0] = mn;
-      sh.pub[1] = mx;
-    }
-  }
-  cl.sync();
-  uint32_t kmin = 0xffffffffu, kmax = 0u;
-  for (int q = 0; q < CS; ++q) {
-    const uint32_t* p = cl.map_shared_rank(sh.pub, q);
-    kmin = min(kmin, p[0]);
-    kmax = max(kmax, p[1]);
-  }
-
-  // 2. radix refinement of the window [base, base + 4096 << shift)
-  uint32_t base = kmin, need = (uint32_t)k;
-  int shift = (int)bitlen(kmax - kmin) - kBinBits;
-  shift = shift < 0 ? 0 : shift;
-  uint32_t klo, khi, need_w;
-  bool exact = false;  // the cut (cut_key, cut_pos) decides instead of the window
-  uint32_t cut_key = 0u;
-  int32_t cut_pos = 0;
-  for (;;) {
-    for (int i = tid; i < kBins; i += kThreads) sh.hist[i] = 0u;
-    __syncthreads();
-    for (int i = tid; i < n; i += kThreads) {
-      const uint32_t ky = key[i];
-      if (ky >= base) {
-        const uint32_t bin = (ky - base) >> shift;
-        if (bin < (uint32_t)kBins) atomicAdd(&sh.hist[bin], 1u);
-      }
-    }
-    __syncthreads();
-    cl.sync();
-    {  // this CTA's share of the bins, summed over the cluster, into every peer
-      const int per = kBins / CS;
-      for (int bin = r * per + tid; bin < (r + 1) * per; bin += kThreads) {
-        uint32_t s = 0;
-        for (int q = 0; q < CS; ++q) s += cl.map_shared_rank(sh.hist, q)[bin];
-        for (int q = 0; q < CS; ++q) cl.map_shared_rank(sh.ghist, q)[bin] = s;
-      }
-    }
-    cl.sync();
-    {  // the bin where the count from the top reaches `need` (thread tid owns
-       // bins 4095 - 8 tid .. 4088 - 8 tid, descending)
-      uint32_t mine[kBinsPerThread], loc = 0;
-#pragma unroll
-      for (int j = 0; j < kBinsPerThread; ++j) {
-        mine[j] = sh.ghist[kBins - 1 - (tid * kBinsPerThread + j)];
-        loc += mine[j];
-      }
-      uint32_t inc = loc;
-#pragma unroll
-      for (int off = 1; off < 32; off <<= 1) {
-        const uint32_t x = __shfl_up_sync(0xffffffffu, inc, off);
-        if (lane >= off) inc += x;
-      }
-      if (lane == 31) sh.wred[0][warp] = inc;
-      __syncthreads();
-      uint32_t acc = inc - loc;
-      for (int w = 0; w < warp; ++w) acc += sh.wred[0][w];
-#pragma unroll
-      for (int j = 0; j < kBinsPerThread; ++j) {
-        if (acc < need && acc + mine[j] >= need) {
-          sh.T = (uint32_t)(kBins - 1 - (tid * kBinsPerThread + j));
-          sh.G = acc;
-          sh.C = mine[j];
-        }
-        acc += mine[j];
-      }
-      __syncthreads();
-    }
-    const uint32_t T = sh.T, G = sh.G, C = sh.C;
-    klo = base + (T << shift);
-    khi = klo + ((1u << shift) - 1u);
-    need -= G;
-    if (shift == 0 || C == need) {
-      need_w = need;
-      break;
-    }
-    if (C <= (uint32_t)kSmallWin) {
-      // the bin-T keys of the whole cluster into the first CTA, ranked there
-      uint32_t* cnt = cl.map_shared_rank(&sh.cand_n, 0);
-      uint32_t* ck = cl.map_shared_rank(sh.cand_key, 0);
-      int32_t* cp = cl.map_shared_rank(sh.cand_pos, 0);
-      for (int i = tid; i < n; i += kThreads) {
-        const uint32_t ky = key[i];
-        if (ky >= klo && ky <= khi) {
-          const uint32_t slot = atomicAdd(cnt, 1u);
-          if (slot < (uint32_t)kSmallWin) {
-            ck[slot] = ky;
-            cp[slot] = (int32_t)(lo + i);
-          }
-        }
-      }
-      cl.sync();
-      if (r == 0) {
-        const int nc = (int)min(sh.cand_n, (uint32_t)kSmallWin);
-        for (int e = tid; e < nc; e += kThreads) {
-          const uint32_t ke = sh.cand_key[e];
-          const int32_t pe = sh.cand_pos[e];
-          uint32_t rank = 0;
-          for (int f = 0; f < nc; ++f) {
-            const uint32_t kf = sh.cand_key[f];
-            rank += (kf > ke || (kf == ke && sh.cand_pos[f] < pe)) ? 1u : 0u;
-          }
-          if (rank == need - 1) {  // the last choice: publish the cut everywhere
-            for (int q = 0; q < CS; ++q) {
-              *cl.map_shared_rank(&sh.cut_key, q) = ke;
-              *cl.map_shared_rank(&sh.cut_pos, q) = pe;
-            }
-          }
-        }
-      }
-      cl.sync();
-      exact = true;
-      cut_key = sh.cut_key;
-      cut_pos = sh.cut_pos;
-      need_w = 0u;
-      break;
-    }
-    base = klo;
-    shift = shift > kBinBits ? shift - kBinBits : 0;
-    __syncthreads();  // sh.T / G / C are rewritten by the next pass
-  }
-
-  // 3. chosen: key > khi, or klo <= key <= khi among the first need_w of those
-  //    (in index order across the cluster).  Warp w scans a contiguous segment.
-  const int seg = ((n + kWarps - 1) / kWarps + 31) & ~31;
-  const int s0 = min(n, warp * seg), s1 = min(n, s0 + seg);
-  // strict: chosen outright; in window: chosen by index order up to need_w
-  auto strict_of = [&](uint32_t ky, int i) {
-    return exact ? (ky > cut_key || (ky == cut_key && (int32_t)(lo + i) <= cut_pos)) : ky > khi;
-  };
-  auto window_of = [&](uint32_t ky) { return !exact && ky >= klo && ky <= khi; };
-  uint32_t strict = 0, win = 0;
-  for (int i0 = s0; i0 < s1; i0 += 32) {
-    const int i = i0 + lane;
-    const uint32_t ky = i < s1 ? key[i] : 0u;
-    strict += __popc(__ballot_sync(0xffffffffu, i < s1 && strict_of(ky, i)));
-    win += __popc(__ballot_sync(0xffffffffu, i < s1 && window_of(ky)));
-  }
-  if (lane == 0) sh.wcnt[warp] = (strict << 16) | win;  // both < 2^16
+  if (lane == 31) wsum[warp] = inc;
   __syncthreads();
-  if (tid == 0) {
-    uint32_t st = 0, wi = 0;
-    for (int w = 0; w < kWarps; ++w) {
-      st += sh.wcnt[w] >> 16;
-      wi += sh.wcnt[w] & 0xffffu;
-    }
-    sh.pub[2] = st;
-    sh.pub[3] = wi;
+  uint32_t before = 0;
+  total = 0;
+  for (int w = 0; w < kThreads / 32; ++w) {
+    if (w < warp) before += wsum[w];
+    total += wsum[w];
   }
-  cl.sync();
-  uint32_t win_before = 0, out_before = 0;  // over the earlier CTAs of the cluster
-  for (int q = 0; q < r; ++q) {
-    const uint32_t* p = cl.map_shared_rank(sh.pub, q);
-    const uint32_t wq = p[3];
-    const uint32_t take = need_w > win_before ? min(wq, need_w - win_before) : 0u;
-    out_before += p[2] + take;
-    win_before += wq;
-  }
-  cl.sync();  // no CTA leaves while a peer may still read its shared memory
-  for (int w = 0; w < warp; ++w) {
-    const uint32_t st = sh.wcnt[w] >> 16, wi = sh.wcnt[w] & 0xffffu;
-    const uint32_t take = need_w > win_before ? min(wi, need_w - win_before) : 0u;
-    out_before += st + take;
-    win_before += wi;
-  }
-  const uint32_t lt = (1u << lane) - 1u;
-  for (int i0 = s0; i0 < s1; i0 += 32) {
-    const int i = i0 + lane;
-    const uint32_t ky = i < s1 ? key[i] : 0u;
-    const bool is_w = i < s1 && window_of(ky);
-    const uint32_t wm = __ballot_sync(0xffffffffu, is_w);
-    const bool pick = (i < s1 && strict_of(ky, i)) || (is_w && win_before + __popc(wm & lt) < need_w);
-    const uint32_t pm = __ballot_sync(0xffffffffu, pick);
-    const uint32_t o = out_before + __popc(pm & lt);
-    if (pick && o < (uint32_t)k) out[o] = (int32_t)(lo + i);
-    out_before += __popc(pm);
-    win_before += __popc(wm);
-  }
+  __syncthreads();
+  return before + inc - v;
 }
 
-// Cluster size and slice length for a capacity: slices of about
-// kSliceTarget keys, at most kMaxCluster CTAs.
-void topk_shape(int64_t cap, int& cs, int& slice) {
-  cs = 1;
-  while (cs < kMaxCluster && (int64_t)cs * kSliceTarget < cap) cs *= 2;
-  const int64_t s = (cap + cs - 1) / cs;
-  slice = (int)((s + 31) & ~(int64_t)31);
+__global__ void __launch_bounds__(kThreads, 4) decode_topk_hist_kernel(
+    const int64_t* __restrict__ pos, int64_t cap, int m, int k, const float* __restrict__ scores,
+    DecodeSelectWs ws, int32_t* __restrict__ sel) {
+  __shared__ SelShared sh;
+  // [kSmemCand] keys, [kSmemCand] indices, [kSmemWords] bitmap words
+  extern __shared__ __align__(16) uint32_t dyn_smem[];
+  uint32_t* dyn_key = dyn_smem;
+  int32_t* dyn_idx = reinterpret_cast<int32_t*>(dyn_smem + kSmemCand);
+  uint32_t* dyn_bm = dyn_smem + 2 * kSmemCand;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int j = blockIdx.x;
+  const int64_t b = blockIdx.y;
+
+  const int64_t t = pos[b];  // an input of the step: read before the wait
+  sm100::pdl_wait();         // the scores and the histogram come from the indexer
+  sm100::pdl_trigger();
+  const int64_t V = t < 0 ? 0 : min((t + 1) / m, cap);
+  int32_t* out = sel + b * k;
+  if (V <= k) {  // every visible entry
+    if (j == 0)
+      for (int i = tid; i < k; i += kThreads) out[i] = i < V ? i : -1;
+    return;
+  }
+  const int64_t lo = (int64_t)j * kSlice;
+  if (lo >= V) return;  // past the sequence's last slice (not counted below)
+  const int nsl = (int)((V + kSlice - 1) / kSlice);
+
+  // this thread's 16 scores start loading now, under the histogram scan
+  const int64_t s0 = lo + (int64_t)tid * kPer;
+  const float* row = scores + b * cap;
+  uint32_t keys[kPer];  // (rows are `cap` floats apart: no vector loads)
+#pragma unroll
+  for (int i = 0; i < kPer; ++i) keys[i] = s0 + i < V ? order_key(__ldcg(row + s0 + i)) : 0u;
+
+  // 1. the bin T where the count from the top reaches k (thread tid owns
+  //    bins 4095 - 16 tid - i, i = 0 .. 15, i.e. descending)
+  if (tid == 0) {  // (a histogram that cannot reach k leaves a defined, capped result)
+    sh.T = 0u;
+    sh.G = 0u;
+    sh.CT = 0u;
+  }
+  {
+    const uint32_t* gh = ws.ghist + b * kBins;
+    uint32_t c[kBinsPerThread], loc = 0;
+#pragma unroll
+    for (int i = 0; i < kBinsPerThread; ++i) {
+      c[i] = __ldcg(gh + kBins - 1 - (tid * kBinsPerThread + i));
+      loc += c[i];
+    }
+    uint32_t total;
+    uint32_t acc = block_excl_scan(loc, sh.wsum, total);
+#pragma unroll
+    for (int i = 0; i < kBinsPerThread; ++i) {
+      if (acc < (uint32_t)k && acc + c[i] >= (uint32_t)k) {
+        sh.T = (uint32_t)(kBins - 1 - (tid * kBinsPerThread + i));
+        sh.G = acc;
+        sh.CT = c[i];
+      }
+      acc += c[i];
+    }
+    __syncthreads();
+  }
+  const uint32_t T = sh.T, G = sh.G, CT = sh.CT;
+  const uint32_t need = (uint32_t)k - G;
+  const bool all_of_T = CT == need;  // bin T is taken whole: no candidates
+
+  // 2. classify this thread's 16 scores (loaded above): chosen outright, or a
+  //    bin-T candidate
+  uint32_t strict = 0, cand = 0;
+#pragma unroll
+  for (int i = 0; i < kPer; ++i) {
+    if (s0 + i < V) {
+      const uint32_t bin = keys[i] >> kDecHistShift;
+      if (bin > T || (all_of_T && bin == T)) strict |= 1u << i;
+      else if (bin == T) cand |= 1u << i;
+    }
+  }
+  // two threads make one bitmap word (lo half: the even thread)
+  const uint32_t other = __shfl_xor_sync(0xffffffffu, strict, 1);
+  if ((lane & 1) == 0) __stcg(ws.bitmap + b * ws.words + (s0 >> 5), strict | (other << 16));
+  uint32_t ncand = 0;
+  const uint32_t off = block_excl_scan((uint32_t)__popc(cand), sh.wsum, ncand);
+  {
+    uint32_t* ck = ws.cand_key + b * cap + lo;
+    int32_t* ci = ws.cand_idx + b * cap + lo;
+    uint32_t p = off;
+#pragma unroll
+    for (int i = 0; i < kPer; ++i)
+      if (cand & (1u << i)) {
+        __stcg(ck + p, keys[i]);
+        __stcg(ci + p, (int32_t)(s0 + i));
+        ++p;
+      }
+  }
+  if (tid == 0) __stcg(ws.cand_cnt + b * kDecMaxSlices + j, ncand);
+
+  // 3. the last CTA of the sequence finishes it
+  __threadfence();
+  __syncthreads();
+  if (tid == 0) sh.last = atomicAdd(ws.done + b, 1u) == (uint32_t)(nsl - 1) ? 1u : 0u;
+  __syncthreads();
+  if (sh.last == 0u) return;
+  __threadfence();
+
+  // the sequence's bitmap into shared memory when it fits (loads issued now,
+  // under the candidate bookkeeping)
+  const int64_t nwords = (V + 31) / 32;
+  const bool bm_smem = nwords <= kSmemWords;
+  uint32_t* bmg = ws.bitmap + b * ws.words;
+  uint32_t* bm = bm_smem ? dyn_bm : bmg;
+  if (bm_smem)
+    for (int64_t w = tid; w < nwords; w += kThreads) dyn_bm[w] = __ldcg(bmg + w);
+
+  if (!all_of_T) {
+    // the candidates of every slice, in index order, into one array: shared
+    // memory when they fit (the usual case: bin T holds a few hundred to a
+    // couple of thousand scores), else the global gather area
+    if (warp == 0) {  // slice offsets: a shuffle scan, lane l owns slices l, l + 32, ..
+      uint32_t run = 0;
+      for (int q0 = 0; q0 < nsl; q0 += 32) {
+        const int q = q0 + lane;
+        const uint32_t c = q < nsl ? __ldcg(ws.cand_cnt + b * kDecMaxSlices + q) : 0u;
+        uint32_t inc = c;
+#pragma unroll
+        for (int off = 1; off < 32; off <<= 1) {
+          const uint32_t x = __shfl_up_sync(0xffffffffu, inc, off);
+          if (lane >= off) inc += x;
+        }
+        if (q < nsl) sh.slice_off[q] = run + inc - c;
+        run += __shfl_sync(0xffffffffu, inc, 31);
+      }
+      if (lane == 0) sh.slice_off[nsl] = run;
+    }
+    __syncthreads();
+    const uint32_t C = sh.slice_off[nsl];
+    const bool in_smem = C <= (uint32_t)kSmemCand;
+    uint32_t* cck = in_smem ? dyn_key : ws.cc_key + b * cap;
+    int32_t* cci = in_smem ? dyn_idx : ws.cc_idx + b * cap;
+    for (int q = warp; q < nsl; q += kThreads / 32) {
+      const uint32_t base = sh.slice_off[q], n = sh.slice_off[q + 1] - base;
+      const uint32_t* ck = ws.cand_key + b * cap + (int64_t)q * kSlice;
+      const int32_t* ci = ws.cand_idx + b * cap + (int64_t)q * kSlice;
+      for (uint32_t i = lane; i < n; i += 32) {
+        const uint32_t kv = __ldcg(ck + i);
+        const int32_t iv = __ldcg(ci + i);
+        if (in_smem) {
+          cck[base + i] = kv;
+          cci[base + i] = iv;
+        } else {
+          __stcg(cck + base + i, kv);
+          __stcg(cci + base + i, iv);
+        }
+      }
+    }
+    __threadfence_block();
+    __syncthreads();
+    // the need largest of them (ties: the earlier position, i.e. the smaller
+    // index), marked in the bitmap
+    uint32_t Tk = 0u, take_eq = 0u;
+    const bool all = need >= C;
+    if (!all) {
+      if (in_smem)
+        radix_kth<kThreads>(KeysInSmem{cck}, C, (int)need, sh.sel, Tk, take_eq);
+      else
+        radix_kth<kThreads>(KeysInGlobal{cck}, C, (int)need, sh.sel, Tk, take_eq);
+    }
+    auto key_at = [&](int64_t i) { return in_smem ? cck[i] : __ldcg(cck + i); };
+    const int64_t seg = ((C + kThreads / 32 - 1) / (kThreads / 32) + 31) / 32 * 32;
+    const int64_t plo = (int64_t)warp * seg, phi = min((int64_t)C, plo + seg);
+    uint32_t eq = 0;
+    for (int64_t base = plo; base < phi; base += 32) {
+      const int64_t i = base + lane;
+      eq += __popc(__ballot_sync(0xffffffffu, i < phi && !all && key_at(i) == Tk));
+    }
+    if (lane == 0) sh.sel.warp_b[warp] = eq;
+    __syncthreads();
+    uint32_t eq_before = 0;
+    for (int w = 0; w < warp; ++w) eq_before += sh.sel.warp_b[w];
+    const uint32_t lt = (1u << lane) - 1u;
+    for (int64_t base = plo; base < phi; base += 32) {
+      const int64_t i = base + lane;
+      const uint32_t key = i < phi ? key_at(i) : 0u;
+      const bool is_eq = i < phi && !all && key == Tk;
+      const uint32_t em = __ballot_sync(0xffffffffu, is_eq);
+      const bool take = i < phi && (all || key > Tk || (is_eq && eq_before + __popc(em & lt) < take_eq));
+      if (take) {
+        const int32_t s = in_smem ? cci[i] : __ldcg(cci + i);
+        atomicOr(bm + (s >> 5), 1u << (s & 31));
+      }
+      eq_before += __popc(em);
+    }
+    if (!bm_smem) __threadfence();
+  }
+  __syncthreads();
+
+  // 4. the chosen indices in ascending order, from the bitmap
+  const int64_t per = (nwords + kThreads - 1) / kThreads;
+  const int64_t w0 = min(nwords, (int64_t)tid * per), w1 = min(nwords, w0 + per);
+  auto word = [&](int64_t w) { return bm_smem ? dyn_bm[w] : __ldcg(bmg + w); };
+  uint32_t cnt = 0;
+  for (int64_t w = w0; w < w1; ++w) cnt += __popc(word(w));
+  uint32_t total;
+  uint32_t o = block_excl_scan(cnt, sh.wsum, total);
+  for (int64_t w = w0; w < w1; ++w) {
+    uint32_t x = word(w);
+    while (x != 0u) {
+      const int bit = __ffs(x) - 1;
+      x &= x - 1u;
+      if (o < (uint32_t)k) out[o] = (int32_t)(w * 32 + bit);
+      ++o;
+    }
+  }
+  for (uint32_t i = total + tid; i < (uint32_t)k; i += kThreads) out[i] = -1;  // (total == k)
 }
 
 }  // namespace
 
-bool decode_topk_supported(const csa_cache_desc& d) {
-  int cs, slice;
-  topk_shape(d.capacity, cs, slice);
-  return !d.is_hca && slice <= kMaxSlice;
+bool decode_select_supported(const csa_cache_desc& d) {
+  return !d.is_hca && (d.capacity + kSlice - 1) / kSlice <= kDecMaxSlices;
 }
 
-cudaError_t launch_decode_topk(const csa_cache_desc& d, const int64_t* pos, const float* scores,
-                               int32_t* sel, cudaStream_t s) {
-  int cs, slice;
-  topk_shape(d.capacity, cs, slice);
-  if (slice > kMaxSlice) return cudaErrorInvalidValue;
-  cudaLaunchConfig_t cfg = {};
-  cudaLaunchAttribute attr[2];
-  auto configure = [&]() -> cudaError_t {
-    const size_t smem = sizeof(TopkShared) + (size_t)slice * 4;
-    cudaError_t e = cudaFuncSetAttribute(decode_topk_kernel,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (e != cudaSuccess) return e;
-    cfg.gridDim = dim3((unsigned)cs, (unsigned)d.batch);
-    cfg.blockDim = dim3(kThreads);
-    cfg.dynamicSmemBytes = smem;
-    cfg.stream = s;
-    attr[0].id = cudaLaunchAttributeClusterDimension;
-    attr[0].val.clusterDim.x = (unsigned)cs;
-    attr[0].val.clusterDim.y = 1;
-    attr[0].val.clusterDim.z = 1;
-    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-    attr[1].val.programmaticStreamSerializationAllowed = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 2;
-    return cudaSuccess;
+DecodeSelectWs decode_select_ws(const csa_cache_desc& d, uint8_t* base, size_t* bytes) {
+  DecodeSelectWs w = {};
+  const size_t B = (size_t)d.batch, cap = (size_t)d.capacity;
+  w.words = (int64_t)((cap + kSlice - 1) / kSlice * (kSlice / 32));
+  size_t off = 0;
+  auto take = [&](size_t n) {
+    const size_t o = off;
+    off = (off + n + 255) & ~(size_t)255;
+    return o;
   };
-  cudaError_t e = configure();
-  if (e != cudaSuccess) return e;
-  if (cs > 8) {  // a non-portable cluster: use it only where the device can place one
-    int clusters = 0;
-    if (cudaFuncSetAttribute(decode_topk_kernel,
-                             cudaFuncAttributeNonPortableClusterSizeAllowed, 1) != cudaSuccess ||
-        cudaOccupancyMaxActiveClusters(&clusters, decode_topk_kernel, &cfg) != cudaSuccess ||
-        clusters < 1) {
-      cudaGetLastError();  // clear a refusal; fall back to eight CTAs
-      cs = 8;
-      const int64_t sl = (d.capacity + cs - 1) / cs;
-      slice = (int)((sl + 31) & ~(int64_t)31);
-      if (slice > kMaxSlice) return cudaErrorInvalidValue;
-      if ((e = configure()) != cudaSuccess) return e;
-    }
+  const size_t o_gh = take(B * kBins * 4), o_done = take(B * 4), o_bm = take(B * w.words * 4),
+               o_ck = take(B * cap * 4), o_ci = take(B * cap * 4),
+               o_cnt = take(B * kDecMaxSlices * 4), o_cck = take(B * cap * 4),
+               o_cci = take(B * cap * 4);
+  *bytes = off;
+  if (base != nullptr) {
+    w.ghist = reinterpret_cast<uint32_t*>(base + o_gh);
+    w.done = reinterpret_cast<uint32_t*>(base + o_done);
+    w.bitmap = reinterpret_cast<uint32_t*>(base + o_bm);
+    w.cand_key = reinterpret_cast<uint32_t*>(base + o_ck);
+    w.cand_idx = reinterpret_cast<int32_t*>(base + o_ci);
+    w.cand_cnt = reinterpret_cast<uint32_t*>(base + o_cnt);
+    w.cc_key = reinterpret_cast<uint32_t*>(base + o_cck);
+    w.cc_idx = reinterpret_cast<int32_t*>(base + o_cci);
   }
-  return cudaLaunchKernelEx(&cfg, decode_topk_kernel, pos, (int64_t)d.capacity, d.m, d.k,
-                            scores, sel, slice);
+  return w;
+}
+
+cudaError_t launch_decode_select(const csa_cache_desc& d, const int64_t* pos, const float* scores,
+                                 const DecodeSelectWs& ws, int32_t* sel, cudaStream_t s) {
+  const unsigned nsl = (unsigned)((d.capacity + kSlice - 1) / kSlice);
+  if (nsl > (unsigned)kDecMaxSlices) return cudaErrorInvalidValue;
+  constexpr size_t kDyn = (size_t)kSmemCand * 8 + (size_t)kSmemWords * 4;
+  const cudaError_t e = cudaFuncSetAttribute(decode_topk_hist_kernel,
+                                             cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kDyn);
+  if (e != cudaSuccess) return e;
+  return launch_pdl(decode_topk_hist_kernel, dim3(nsl, (unsigned)d.batch), dim3(kThreads), kDyn, s,
+                    pos, (int64_t)d.capacity, d.m, d.k, scores, ws, sel);
 }
 
 }  // namespace csa

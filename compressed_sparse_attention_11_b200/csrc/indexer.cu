@@ -93,7 +93,8 @@ cudaError_t launch_index_scores(const void* q_i, const float* w_i, const void* k
   if (index_scores_tc_supported(nh_i, c_i, dt, q_i, k_i)) {
     unsigned int* err = device_timeout_flag();
     if (err == nullptr) return cudaErrorUnknown;
-    return launch_index_scores_tc(q_i, w_i, k_i, batch, n, nh_i, c_i, m, scores, ld, err, s);
+    return launch_index_scores_tc(q_i, w_i, k_i, batch, n, nh_i, c_i, m, scores, false, ld, err,
+                                  s);
   }
   const int nh_pad = (nh_i + kIdxHG - 1) / kIdxHG * kIdxHG;
   const size_t smem = sizeof(float) * ((size_t)c_i * kIdxKeys + (size_t)c_i * nh_pad);

@@ -50,10 +50,16 @@ struct IdxCfg {
   static_assert(SMEM <= 232448, "shared memory budget");
 };
 
-template <int H, int CI>
+__device__ __forceinline__ void put_score(float* p, float v) { *p = v; }
+__device__ __forceinline__ void put_score(__nv_bfloat16* p, float v) {
+  *p = __float2bfloat16_rn(v);
+}
+
+// ST: the stored score type (fp32, or bf16 for the bf16-score selection).
+template <int H, int CI, typename ST>
 __global__ void __launch_bounds__(kThreads, 1) index_scores_tc_kernel(
     const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
-    const float* __restrict__ w_i, int64_t n, int m, int64_t E, float* __restrict__ scores,
+    const float* __restrict__ w_i, int64_t n, int m, int64_t E, ST* __restrict__ scores,
     int64_t ld, unsigned int* __restrict__ err) {
   using C = IdxCfg<H, CI>;
   using namespace sm100;
@@ -196,7 +202,7 @@ __global__ void __launch_bounds__(kThreads, 1) index_scores_tc_kernel(
 #pragma unroll
         for (int qq = 0; qq < C::QW; ++qq) {
           const int64_t t = t0 + p * C::HQ + colhalf * C::QW + qq;
-          if (t < n && s < min((t + 1) / m, E)) scores[(b * n + t) * ld + s] = acc[qq];
+          if (t < n && s < min((t + 1) / m, E)) put_score(scores + (b * n + t) * ld + s, acc[qq]);
         }
       }
       if (!ok) break;
@@ -211,9 +217,9 @@ __global__ void __launch_bounds__(kThreads, 1) index_scores_tc_kernel(
   }
 }
 
-template <int H, int CI>
+template <int H, int CI, typename ST>
 cudaError_t launch_tc(const void* q_i, const float* w_i, const void* k_i, int64_t batch,
-                      int64_t n, int m, float* scores, int64_t ld, unsigned int* err,
+                      int64_t n, int m, ST* scores, int64_t ld, unsigned int* err,
                       cudaStream_t s) {
   using C = IdxCfg<H, CI>;
   const int64_t E = n / m;
@@ -222,7 +228,7 @@ cudaError_t launch_tc(const void* q_i, const float* w_i, const void* k_i, int64_
                          (uint64_t)n * H * CI * 2, 64, 256) ||
       !make_tmap_bf16_3d(&tk, k_i, CI, E, batch, CI * 2ull, (uint64_t)E * CI * 2, 64, kKT))
     return cudaErrorInvalidValue;
-  auto kern = index_scores_tc_kernel<H, CI>;
+  auto kern = index_scores_tc_kernel<H, CI, ST>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
   if (e != cudaSuccess) return e;
   dim3 grid((unsigned)((n + C::TQ - 1) / C::TQ), (unsigned)batch);
@@ -242,10 +248,14 @@ bool index_scores_tc_supported(int nh_i, int c_i, csa_dtype dt, const void* q_i,
 
 cudaError_t launch_index_scores_tc(const void* q_i, const float* w_i, const void* k_i,
                                    int64_t batch, int64_t n, int nh_i, int c_i, int m,
-                                   float* scores, int64_t ld, unsigned int* err,
+                                   void* scores, bool bf16_scores, int64_t ld, unsigned int* err,
                                    cudaStream_t s) {
-#define CSA_IDX_CASE(HH, CC) \
-  if (nh_i == HH && c_i == CC) return launch_tc<HH, CC>(q_i, w_i, k_i, batch, n, m, scores, ld, err, s);
+#define CSA_IDX_CASE(HH, CC)                                                                   \
+  if (nh_i == HH && c_i == CC)                                                                 \
+    return bf16_scores                                                                         \
+               ? launch_tc<HH, CC, __nv_bfloat16>(q_i, w_i, k_i, batch, n, m,                  \
+                                                  (__nv_bfloat16*)scores, ld, err, s)          \
+               : launch_tc<HH, CC, float>(q_i, w_i, k_i, batch, n, m, (float*)scores, ld, err, s);
   CSA_IDX_CASE(64, 128) CSA_IDX_CASE(64, 64) CSA_IDX_CASE(32, 128) CSA_IDX_CASE(32, 64)
   CSA_IDX_CASE(16, 128) CSA_IDX_CASE(16, 64) CSA_IDX_CASE(128, 128) CSA_IDX_CASE(128, 64)
 #undef CSA_IDX_CASE

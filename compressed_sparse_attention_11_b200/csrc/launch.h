@@ -44,21 +44,45 @@ unsigned int* device_timeout_flag();
 
 // tcgen05 indexer (bf16, c_i in {64, 128}, nh_i in {16, 32, 64, 128}).
 bool index_scores_tc_supported(int nh_i, int c_i, csa_dtype dt, const void* q_i, const void* k_i);
+// scores: fp32, or bf16 when bf16_scores.
 cudaError_t launch_index_scores_tc(const void* q_i, const float* w_i, const void* k_i,
                                    int64_t batch, int64_t n, int nh_i, int c_i, int m,
-                                   float* scores, int64_t ld, unsigned int* err, cudaStream_t s);
+                                   void* scores, bool bf16_scores, int64_t ld, unsigned int* err,
+                                   cudaStream_t s);
+
+// Low-precision indexer: E4M3 codes + fp32 scale of rows of 128 bf16 values,
+// and the FP8 x FP8 tcgen05 scores (c_i = 128, nh_i in {16, 32, 64, 128}).
+bool index_fp8_supported(int nh_i, int c_i);
+cudaError_t launch_quantize_rows_fp8(const void* x, int64_t rows, uint8_t* codes, float* scales,
+                                     cudaStream_t s);
+cudaError_t launch_index_scores_fp8(const uint8_t* q8, const float* qs, const uint8_t* k8,
+                                    const float* ks, const float* w_i, int64_t batch, int64_t n,
+                                    int nh_i, int m, void* scores, bool bf16_scores, int64_t ld,
+                                    unsigned int* err, cudaStream_t s);
+// Top-k rows over bf16 scores (rows of at most 32768 keys).
+cudaError_t launch_topk_rows_bf16(const __nv_bfloat16* scores, int64_t ld, int64_t batch,
+                                  int64_t n, int m, int64_t E, int k, int32_t* idx,
+                                  cudaStream_t s);
 
 // tcgen05 attention (bf16, 64 heads of dim 512, up to 2048 selected entries).
 bool attn_tc_supported(int nh, int c, int k, csa_dtype dt, const void* q, const void* kv_comp,
-                       const void* kv_win);
+                       const void* kv_win, int rope_dims);
 // One warp waits on a barrier that is completed first (arrive) or never; the
 // wait gives up after limit_us and sets *err.
 cudaError_t launch_selftest_wait(uint32_t limit_us, bool arrive, unsigned int* err,
                                  cudaStream_t s);
+// Query RMSNorm + rotation and output rotation of the attention kernels
+// (gamma == NULL: off).
+struct QNormRope {
+  const float* gamma;
+  float eps;
+  int rope_dims;
+  float base;
+};
 cudaError_t launch_attn_tc(const void* q, const void* kv_comp, const int32_t* idx, int k,
                            const void* kv_win, int window, const float* sink, float scale,
-                           int64_t batch, int64_t n, int m, void* out, unsigned int* err,
-                           cudaStream_t s);
+                           int64_t batch, int64_t n, int m, const QNormRope& qn, void* out,
+                           unsigned int* err, cudaStream_t s);
 
 // tcgen05 decode indexer over FP8 keys (c_i = 128, nh_i in {64, 128}), persistent.
 struct CacheView;
@@ -77,16 +101,37 @@ __host__ __device__ inline int decode_qop_row(int h, int part, int H) {
 }
 // qop: [batch] query operands (written by the append step); scores
 // [batch][capacity] fp32, written for s < V of each sequence.
+// ghist [batch][kDecHistBins]: each sequence's score histogram (added to).
 cudaError_t launch_decode_index_tc(const csa_cache_desc& d, const CacheView& cv,
                                    const int64_t* pos, const uint8_t* qop, float* scores,
-                                   unsigned int* err, cudaStream_t s);
+                                   uint32_t* ghist, unsigned int* err, cudaStream_t s);
 
-// Exact top-k over the indexer's scores, one thread-block cluster per
-// sequence with the scores staged in shared memory.  sel [batch][k]: the
-// chosen entry indices ascending, -1 padded when V <= k.
-bool decode_topk_supported(const csa_cache_desc& d);
-cudaError_t launch_decode_topk(const csa_cache_desc& d, const int64_t* pos, const float* scores,
-                               int32_t* sel, cudaStream_t s);
+// Histogram of each sequence's indexer scores over the top kDecHistShift..31
+// bits of their order keys, written by the indexer for the selection step.
+constexpr int kDecHistBins = 4096;
+constexpr int kDecHistShift = 20;
+constexpr int kDecMaxSlices = 512;  // 4096-score slices per sequence (2M entries)
+
+// Selection scratch inside the decode workspace (see decode_select_ws).
+struct DecodeSelectWs {
+  uint32_t* ghist;     // [batch][kDecHistBins]  zeroed by the append step
+  uint32_t* done;      // [batch]                finished slices; zeroed by the append step
+  uint32_t* bitmap;    // [batch][words]         chosen entries, one bit each
+  uint32_t* cand_key;  // [batch][capacity]      threshold-bin candidates, per slice
+  int32_t* cand_idx;
+  uint32_t* cand_cnt;  // [batch][kDecMaxSlices]
+  uint32_t* cc_key;    // [batch][capacity]      the candidates gathered in index order
+  int32_t* cc_idx;
+  int64_t words;
+};
+// Layout of the scratch at `base` (NULL: only the size); *bytes its size.
+DecodeSelectWs decode_select_ws(const csa_cache_desc& d, uint8_t* base, size_t* bytes);
+// Exact top-k from the indexer's scores and histogram: many CTAs per
+// sequence, the last of them writing sel [batch][k] (ascending, -1 padded
+// when V <= k).
+bool decode_select_supported(const csa_cache_desc& d);
+cudaError_t launch_decode_select(const csa_cache_desc& d, const int64_t* pos, const float* scores,
+                                 const DecodeSelectWs& ws, int32_t* sel, cudaStream_t s);
 
 // tcgen05 decode attention (64 heads x 512, FP8/bf16 cache): one 128-entry
 // tile per CTA (ntile = decode_attn_splits), merged by a combine kernel.
@@ -98,9 +143,17 @@ cudaError_t launch_decode_attn_tc(const csa_cache_desc& d, const CacheView& cv,
                                   float* part_o, float* part_ms, unsigned int* err,
                                   cudaStream_t s);
 
+// nr != NULL: each entry i RMSNorm-ed and its trailing dims rotated for
+// position m * i as it is written (or by a second in-place pass).
 cudaError_t launch_compress(const void* ca, const void* cb, const void* za, const void* zb,
                             const float* ba, const float* bb, int64_t batch, int64_t n, int c,
-                            int m, int overlap, csa_dtype dt, void* out, cudaStream_t s);
+                            int m, int overlap, csa_dtype dt, const csa_norm_rope* nr, void* out,
+                            cudaStream_t s);
+// Rows [batch, n, heads, c]: RMSNorm + rotation of the trailing dims for
+// position t * pos_mul (t the row's token); out may equal x.
+cudaError_t launch_norm_rope_rows(const void* x, int64_t batch, int64_t n, int heads, int c,
+                                  int64_t pos_mul, const csa_norm_rope* nr, csa_dtype dt,
+                                  void* out, cudaStream_t s);
 
 // fp32 scores[b][t][s] (row stride `ld`) for s < V(t); entries beyond V(t) untouched.
 cudaError_t launch_index_scores(const void* q_i, const float* w_i, const void* k_i,
@@ -111,10 +164,18 @@ cudaError_t launch_index_scores(const void* q_i, const float* w_i, const void* k
 cudaError_t launch_topk_rows(const float* scores, int64_t ld, int64_t batch, int64_t n,
                              int m, int64_t E, int k, int32_t* idx, cudaStream_t s);
 
+// q_nr != NULL: each query head RMSNorm-ed and rotated for position t before
+// the logits, and the output's trailing dims rotated by -t (the entries are
+// taken as given: already normed and rotated).
 cudaError_t launch_attn(const void* q, const void* kv_comp, const int32_t* idx, int k,
                         const void* kv_win, int window, const float* sink, float scale,
                         int64_t batch, int64_t n, int nh, int c, int m, csa_dtype dt,
-                        void* out, cudaStream_t s);
+                        const csa_norm_rope* q_nr, void* out, cudaStream_t s);
+
+// Grouped output projection: z = grouped o W1^T (bf16 [rows, G dg]), y = z W2^T.
+cudaError_t launch_grouped_out_proj(const void* o, int64_t rows, int nh, int c, int G, int dg,
+                                    int d, const void* w1, const void* w2, void* z, void* y,
+                                    cudaStream_t s);
 
 // ---- decode --------------------------------------------------------------
 struct CacheView {

@@ -72,8 +72,11 @@ struct __align__(16) RowTopkShared {
 
 __device__ __forceinline__ uint32_t bit_length(uint32_t x) { return x == 0 ? 0u : 32u - __clz(x); }
 
+// ST: float, or __nv_bfloat16 for scores stored in bf16 (each widened to fp32
+// exactly, so the order and the ties are those of the bf16 values).
+template <typename ST>
 __global__ void __launch_bounds__(kRowThreads) topk_rows_staged_kernel(
-    const float* __restrict__ scores, int64_t ld, int64_t n, int m, int64_t E, int k,
+    const ST* __restrict__ scores, int64_t ld, int64_t n, int m, int64_t E, int k,
     int32_t* __restrict__ idx) {
   extern __shared__ __align__(16) unsigned char smem_raw[];
   RowTopkShared& sh = *reinterpret_cast<RowTopkShared*>(smem_raw);
@@ -87,9 +90,9 @@ __global__ void __launch_bounds__(kRowThreads) topk_rows_staged_kernel(
     return;
   }
   // 1. the row as order keys, with its key range
-  const float* row = scores + (b * n + t) * ld;
+  const ST* row = scores + (b * n + t) * ld;
   uint32_t mn = 0xffffffffu, mx = 0u;
-  if ((ld & 3) == 0 && (reinterpret_cast<uintptr_t>(scores) & 15) == 0) {
+  if (sizeof(ST) == 4 && (ld & 3) == 0 && (reinterpret_cast<uintptr_t>(scores) & 15) == 0) {
     // 16-byte rows: the whole row lands in shared memory in one round trip
     // (cp.async, zero past V), then becomes order keys in place
     const int nch = (V + 3) >> 2;
@@ -116,7 +119,7 @@ __global__ void __launch_bounds__(kRowThreads) topk_rows_staged_kernel(
 #pragma unroll
       for (int u = 0; u < kBatch; ++u) {
         const int i = i0 + u * kRowThreads;
-        v[u] = i < V ? __ldcs(row + i) : 0.f;
+        v[u] = i < V ? to_f32(__ldcs(row + i)) : 0.f;
       }
 #pragma unroll
       for (int u = 0; u < kBatch; ++u) {
@@ -334,15 +337,28 @@ __global__ void __launch_bounds__(kRowThreads) topk_rows_staged_kernel(
   }
 }
 
+cudaError_t launch_topk_rows_bf16(const __nv_bfloat16* scores, int64_t ld, int64_t batch,
+                                  int64_t n, int m, int64_t E, int k, int32_t* idx,
+                                  cudaStream_t s) {
+  if (E > kRowMaxKeys) return cudaErrorInvalidValue;
+  const size_t smem = sizeof(RowTopkShared) + (size_t)E * sizeof(uint32_t);
+  auto kern = topk_rows_staged_kernel<__nv_bfloat16>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  kern<<<dim3((unsigned)n, (unsigned)batch), kRowThreads, smem, s>>>(scores, ld, n, m, E, k, idx);
+  return cudaGetLastError();
+}
+
 cudaError_t launch_topk_rows(const float* scores, int64_t ld, int64_t batch, int64_t n, int m,
                              int64_t E, int k, int32_t* idx, cudaStream_t s) {
   if (E <= kRowMaxKeys) {
     const size_t smem = sizeof(RowTopkShared) + (size_t)E * sizeof(uint32_t);
-    cudaError_t e = cudaFuncSetAttribute(topk_rows_staged_kernel,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    auto kern = topk_rows_staged_kernel<float>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)smem);
     if (e != cudaSuccess) return e;
-    topk_rows_staged_kernel<<<dim3((unsigned)n, (unsigned)batch), kRowThreads, smem, s>>>(
-        scores, ld, n, m, E, k, idx);
+    kern<<<dim3((unsigned)n, (unsigned)batch), kRowThreads, smem, s>>>(scores, ld, n, m, E, k,
+                                                                     idx);
     return cudaGetLastError();
   }
   const int64_t smem_keys = E <= kSelSmemKeys ? E : 0;

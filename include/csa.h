@@ -60,7 +60,8 @@ typedef enum { CSA_F32 = 0, CSA_BF16 = 1 } csa_dtype;
 const char* csa_status_string(int status);
 /* Reason for the last non-OK status returned on this thread ("" if none). */
 const char* csa_last_error(void);
-/* ABI version, bumped on any signature or layout change. */
+/* ABI version, bumped on any signature or layout change (2: csa_decode_params
+ * gained scores_out; the norm / RoPE calls were added). */
 int csa_abi_version(void);
 /* Synchronises `stream`, then returns CSA_ERR_TIMEOUT if any kernel of this
  * library on the current device gave up a bounded wait since the last check,
@@ -148,6 +149,34 @@ csa_status csa_index_topk_noalloc(const void* q_i, const float* w_i, const void*
                                   csa_dtype dt, int32_t* idx, void* stream);
 
 /* ------------------------------------------------------------------------
+ * csa_index_topk_lowp -- the lightning indexer + top-k in low precision
+ * ([Analysis] "Lightning Indexer": a few heads and FP8 keep the indexer
+ * cheap, the ReLU suits FP8; [Analysis] "FP4 Quantization-Aware Training":
+ * index scores kept in BF16 instead of FP32).  `flags`:
+ *   CSA_INDEX_FP8_QK     every query head q_i[t, h, :] and every key
+ *                        k_i[s, :] is quantised to E4M3 with one fp32 scale
+ *                        (amax / 448; 1 when amax = 0; code = E4M3(x / scale),
+ *                        round to nearest even, saturating) and scored on the
+ *                        FP8 tensor cores: I[t, s] is the indexer formula on
+ *                        the dequantised vectors (fp32 accumulation);
+ *   CSA_INDEX_BF16_SCORES the scores are stored as bf16 (rounded to nearest
+ *                        even) and the top-k is taken over those values
+ *                        (ties: the smaller s).
+ * Either or both.  The selection then approximates csa_index_topk's; its
+ * recall against it is what the two forms trade for speed and traffic.
+ * Arguments as csa_index_topk; dt must be CSA_BF16, the FP8 form needs
+ * c_i = 128 and nh_i in {16, 32, 64, 128}, the bf16-score form n/m <= 32768
+ * (and c_i in {64, 128} with those nh_i when not FP8), else
+ * CSA_ERR_UNSUPPORTED.  ws: csa_index_topk_lowp_workspace(...) bytes.
+ * ------------------------------------------------------------------------ */
+enum { CSA_INDEX_FP8_QK = 1, CSA_INDEX_BF16_SCORES = 2 };
+size_t csa_index_topk_lowp_workspace(int64_t batch, int64_t n, int nh_i, int c_i, int m, int k,
+                                     int flags);
+csa_status csa_index_topk_lowp(const void* q_i, const float* w_i, const void* k_i, int64_t batch,
+                               int64_t n, int nh_i, int c_i, int m, int k, csa_dtype dt,
+                               int flags, int32_t* idx, void* ws, size_t ws_bytes, void* stream);
+
+/* ------------------------------------------------------------------------
  * csa_sparse_attn -- CSA core attention: shared-KV MQA over the selected
  * compressed entries plus the sliding window, with the sink in the same
  * denominator ([Walk-through] 4.3 shared-KV MQA, 4.5 sliding window and
@@ -178,6 +207,82 @@ csa_status csa_sparse_attn(const void* q, const void* kv_comp, const int32_t* id
 csa_status hca_attn(const void* q, const void* kv_comp, const void* kv_win, int window,
                     const float* sink, float scale, int64_t batch, int64_t n, int nh, int c,
                     int m_heavy, csa_dtype dt, void* out, void* stream);
+
+/* ------------------------------------------------------------------------
+ * RMSNorm and partial RoPE around core attention ([Walk-through] 4.5 "other
+ * details": query / KV entry normalisation and partial RoPE; 7.1 Partial
+ * RoPE; 7.4 Query/KV Entry Normalization).  Every query head and every KV
+ * entry is RMSNorm-ed before core attention; the trailing `rope_dims` dims of
+ * queries and entries are rotated for their position; since each entry is
+ * both key and value, the attention output's trailing dims are rotated back
+ * by position -t, so the output depends on relative positions only.
+ *
+ *   RMSNorm(x) = x / sqrt(mean(x^2) + eps) * gamma      (over the c dims)
+ *   RoPE_p(x):   pair j = dims (c - R + 2j, c - R + 2j + 1), j < R/2, turns
+ *                by angle p * rope_base^(-2j/R)
+ * Positions: a query or window row of token t sits at t; compressed entry s
+ * at m * s (its block's first token).  Angles are reduced in double
+ * precision, so positions of millions keep float-accurate rotations.
+ * ------------------------------------------------------------------------ */
+typedef struct {
+  const float* gamma; /* [c] fp32 RMSNorm weight (device, 16-byte aligned)   */
+  float eps;          /* >= 0, finite                                          */
+  int32_t rope_dims;  /* R: 0 <= R <= c, R % 8 == 0 (0: no rotation)          */
+  float rope_base;    /* > 1 and finite                                        */
+} csa_norm_rope;
+
+/* out[b, t, h, :] = RoPE_{t * pos_mul}(RMSNorm(x[b, t, h, :])) for rows
+ * [batch, n, heads, c] of `dt` (queries: heads = nh, pos_mul = 1; window
+ * rows: heads = 1, pos_mul = 1; compressed entries: n = entries, heads = 1,
+ * pos_mul = m).  out may equal x (in place).  c % 8 == 0, c <= 1024. */
+csa_status csa_norm_rope_rows(const void* x, int64_t batch, int64_t n, int heads, int c,
+                              int64_t pos_mul, const csa_norm_rope* nr, csa_dtype dt, void* out,
+                              void* stream);
+
+/* csa_compress followed by RMSNorm + RoPE of each entry i at position m * i
+ * (gamma = the KV entries' weight), done as the entries are written (one
+ * kernel) wherever an entry's dims tile a block, else as a second in-place
+ * pass over the compressed output.  Same arguments and errors as
+ * csa_compress, plus `nr` (required). */
+csa_status csa_compress_norm_rope(const void* ca, const void* cb, const void* za,
+                                  const void* zb, const float* ba, const float* bb,
+                                  int64_t batch, int64_t n, int c, int m, int overlap,
+                                  csa_dtype dt, const csa_norm_rope* nr, void* out, void* stream);
+
+/* csa_sparse_attn / hca_attn with the query RMSNorm + RoPE (nr->gamma = the
+ * query weight) applied in the kernel's prologue and the output's trailing
+ * dims rotated by -t in its epilogue.  The entries (kv_comp, kv_win) are
+ * taken as given: pass them already normed and rotated (csa_compress_norm_rope
+ * and csa_norm_rope_rows).  Same arguments and errors as the plain calls,
+ * plus `nr` (required; the tensor-core path takes rope_dims <= 64). */
+csa_status csa_sparse_attn_norm_rope(const void* q, const void* kv_comp, const int32_t* idx,
+                                     int k, const void* kv_win, int window, const float* sink,
+                                     float scale, int64_t batch, int64_t n, int nh, int c, int m,
+                                     csa_dtype dt, const csa_norm_rope* nr, void* out,
+                                     void* stream);
+csa_status hca_attn_norm_rope(const void* q, const void* kv_comp, const void* kv_win, int window,
+                              const float* sink, float scale, int64_t batch, int64_t n, int nh,
+                              int c, int m_heavy, csa_dtype dt, const csa_norm_rope* nr,
+                              void* out, void* stream);
+
+/* ------------------------------------------------------------------------
+ * csa_grouped_out_proj -- grouped output projection after core attention
+ * ([Walk-through] 4.4: the n_h heads form G groups; each group's
+ * concatenated head outputs are projected to d_g, and the G results,
+ * concatenated, to the model dim d; [Formulas B9] gives V4-Flash n_h = 64,
+ * g = 8, d_g = 1024, d = 4096).  All bf16, fp32 accumulation:
+ *   z[r, g d_g + j] = sum_k o[r, g (nh/G) c + k] w1[g, j, k]   (o as [rows, nh c])
+ *   y[r, j]         = sum_k z[r, k] w2[j, k]
+ *   o : [rows, nh, c]   w1 : [G, d_g, (nh/G) c]   w2 : [d, G d_g]   y : [rows, d]
+ *   ws: the intermediate z, [rows, G d_g] bf16 (csa_grouped_out_proj_workspace
+ *       bytes; rounded to bf16 between the two products).
+ * Needs nh % G == 0, (nh/G) c % 64 == 0, d_g % 256 == 0, d % 256 == 0, else
+ * CSA_ERR_UNSUPPORTED.  Pointers 16-byte aligned.
+ * ------------------------------------------------------------------------ */
+size_t csa_grouped_out_proj_workspace(int64_t rows, int groups, int d_g);
+csa_status csa_grouped_out_proj(const void* o, int64_t rows, int nh, int c, int groups, int d_g,
+                                int d, const void* w1, const void* w2, void* ws,
+                                size_t ws_bytes, void* y, void* stream);
 
 /* ------------------------------------------------------------------------
  * Decode over a persistent cache ([Analysis] "Inference KV Cache": a state
@@ -240,6 +345,12 @@ typedef struct {
                            * receives each sequence's selected entry indices
                            * (ascending, -1 padded when V <= k); NULL keeps
                            * them in the workspace.  Ignored for HCA.        */
+  float* scores_out;      /* CSA, optional: [batch][capacity] fp32 device
+                           * array that receives each sequence's indexer
+                           * scores I[s] for s < V (the rest untouched); NULL
+                           * keeps them in the workspace.  Needs the
+                           * tensor-core indexer shape (c_i = 128, nh_i 64 or
+                           * 128), else CSA_ERR_UNSUPPORTED.  Ignored for HCA. */
 } csa_decode_params;
 
 /* Offsets and total size of a cache for `desc`. Host-only, no launch. */

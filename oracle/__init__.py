@@ -544,8 +544,8 @@ def grouped_output_projection(o, W1, W2) -> np.ndarray:
 def index_scores_row_fp8(q_i_t, w_i_t, K_i, V: int) -> np.ndarray:
     """index_scores_row with q_i_t [H, c_i] and K_i [E, c_i] first put through
     the FP8 E4M3 form (per-row scale amax/448): scores of the V visible keys."""
-    qc, qs, _ = quantize_entries(np.asarray(q_i_t, dtype=np.float32), 0)
-    kc, ks, _ = quantize_entries(np.asarray(f64(K_i)[:V], dtype=np.float32), 0)
+    qc, qs, _ = quantize_entries(f64(q_i_t).astype(np.float32), 0)
+    kc, ks, _ = quantize_entries(f64(K_i)[:V].astype(np.float32), 0)
     q = e4m3_decode(qc) * qs.astype(np.float64)[:, None]
     K = e4m3_decode(kc) * ks.astype(np.float64)[:, None]
     return index_scores_row(q, w_i_t, K, V)

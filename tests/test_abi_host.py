@@ -34,7 +34,7 @@ def test_library_exports_every_declared_function():
     for name in declared:
         assert hasattr(L, name), name
     assert set(declared) == set(csa.EXPORTED)
-    assert L.csa_abi_version() == 1
+    assert L.csa_abi_version() == 2
 
 
 def test_status_strings():

@@ -192,14 +192,16 @@ def _csa_dims(name, seed, k=512):
     return G.Decode(name, 2, 0, 512, 64, 4, 64, 128, False, nh_i=64, c_i=128, k=k, seed=seed)
 
 
-def test_decode_csa_topk_cluster_of_four():
-    """~36000 visible entries: the top-k runs as a 4-CTA cluster per sequence."""
+def test_decode_csa_topk_many_slices():
+    """~36000 visible entries: the selection spreads each sequence over nine
+    4096-score slices, the last of which resolves the threshold bin."""
     _run_and_compare(_csa_dims("csa_decode_cluster", 106), B=2, E=36000, steps=2, seed=13)
 
 
 def test_decode_csa_all_scores_tied():
     """q_i = 0 makes every score 0: the selection is entries 0..k-1 (ties go to
-    the smaller index), across a 2-CTA cluster."""
+    the smaller index): every score falls in the threshold bin, so the exact
+    step ranks all 20000 of them, gathered from five slices."""
     def edit(inp):
         inp["q_i"].zero_()
     _run_and_compare(_csa_dims("csa_decode_ties", 107), B=2, E=20000, steps=2, seed=14, edit=edit,
@@ -210,7 +212,7 @@ def test_decode_csa_topk_integer_scores_with_ties():
     """Scores in {0, 1, 2, 3}, computed exactly on both sides: one index-key dim
     holds the integer, one dim holds 448 (entry scale exactly 1), and one
     query head reads the integer dim with weight 1.  The k-th largest score
-    sits inside a large tied group that spans the cluster's CTAs, so the
+    sits inside a large tied group that spans several slices, so the
     selection is fixed by the smaller-index rule alone."""
     def edit(inp):
         B, E, ci = inp["cache_ikey"].shape
@@ -239,3 +241,40 @@ def test_write_rows_fills_ring_and_state():
         par, row = (u // w.m) % 2, u % w.m
         for si, nm in enumerate(("ca", "cb", "za", "zb")):
             assert torch.equal(host(st)[:, par, si, row], inp["rows_" + nm][:, u - first])
+
+
+def test_decode_index_scores_match_oracle_elementwise():
+    """The decode indexer's scores themselves, element by element.  The GPU
+    feeds the bf16 query to the FP8 tensor-core MMA as hi + lo E4M3 halves
+    times a per-head power of two s_h >= max|q_h| / 448; that pair equals the
+    bf16 value except for elements below 2^-2 s_h, whose error is at most
+    2^-10 s_h.  So |I_gpu[s] - I[s]| <= sum_h w_h 2^-10 s_h sum_d |k_sd|, plus
+    fp32 accumulation, bounded here by 2^-16 sum_h w_h sum_d |q_hd k_sd|."""
+    w = _csa_dims("csa_decode_scores", 110)
+    B, E = 2, 3000
+    inp, cache, t0, first, tail, names = _setup(w, B, E, 1, seed=17)
+    biases = {k: v.to(DEV) for k, v in _biases(inp, w).items()}
+    rows = {nm: inp["rows_" + nm][:, tail].contiguous().to(DEV) for nm in names}
+    pos = torch.full((B,), t0, dtype=torch.int64, device=DEV)
+    scores = torch.full((B, cache.desc.capacity), float("nan"), dtype=torch.float32, device=DEV)
+    cache.decode_step(pos, rows, biases, inp["sink"].to(DEV), w.scale, inp["q"][0].to(DEV),
+                      inp["q_i"][0].to(DEV), inp["w_i"][0].to(DEV), scores_out=scores)
+    csa.csa_check()
+    got = host(scores).double().numpy()
+    for b in range(B):
+        seq = _oracle_sequence(w, inp, b, E, first, tail, names)
+        seq.step(t0, {nm: inp["rows_" + nm][b, tail] for nm in names}, _biases(inp, w),
+                 inp["q"][0, b], inp["q_i"][0, b], inp["w_i"][0, b], inp["sink"], w.scale, w.k)
+        V = O.visible(t0, w.m)
+        K = np.stack([O.dequantize_entry(*e) for e in seq.ikeys[:V]])
+        q = O.f64(inp["q_i"][0, b])
+        wt = O.f64(inp["w_i"][0, b])
+        ref = O.index_scores_row(q, wt, K, V)
+        s_h = 2.0 ** np.ceil(np.log2(np.abs(q).max(axis=1) / 448.0))
+        kabs = np.abs(K).sum(axis=1)                                  # [V]
+        bound = (wt * s_h).sum() * 2.0 ** -10 * kabs + \
+            2.0 ** -16 * (np.abs(K) @ np.abs(q).T @ np.abs(wt))
+        err = np.abs(got[b, :V] - ref)
+        assert np.all(np.isfinite(got[b, :V]))
+        assert np.all(err <= bound), (b, float(err.max()), float((err / bound).max()))
+        assert np.isnan(got[b, V:]).all()             # nothing past the visible entries

@@ -615,6 +615,10 @@ def test_fp8_index_scores_exact_when_inputs_are_e4m3_values():
     K[:, 1] = -448.0
     w = r.uniform(0, 1, H)
     assert np.array_equal(O.index_scores_row_fp8(q, w, K, 40), O.index_scores_row(q, w, K, 40))
+    # the same from bf16 torch tensors (how the GPU tests call it)
+    qt, Kt = torch.tensor(q, dtype=torch.bfloat16), torch.tensor(K, dtype=torch.bfloat16)
+    assert np.array_equal(O.index_scores_row_fp8(qt, torch.tensor(w), Kt, 40),
+                          O.index_scores_row(q, w, K, 40))
 
 
 def test_fp8_index_scores_close_to_plain_on_random_inputs():
