@@ -51,11 +51,12 @@ MEASURED_TRAFFIC = {
         'compressed_sparse_attention_11_b200/csrc/topk.cu': '44874bde73cf3699',
         'compressed_sparse_attention_11_b200/csrc/sm100.cuh': '1863469781a2e737',
         'compressed_sparse_attention_11_b200/csrc/common.cuh': '2c8e048cf6f6eadb'}},
-    # attn_tc_kernel 4572.6 MB read + 4246.8 MB written (n = 65536)
-    "sparse_attn": {"bytes": 8819453440, "sources": {
-        'compressed_sparse_attention_11_b200/csrc/attn_tc.cu': '56c9e75b4031b33f',
+    # attn_tc_kernel 4554.1 MB read + 4247.6 MB written (n = 65536)
+    "sparse_attn": {"bytes": 8801669120, "sources": {
+        'compressed_sparse_attention_11_b200/csrc/attn_tc.cu': '16fc1a623830605f',
         'compressed_sparse_attention_11_b200/csrc/sm100.cuh': '1863469781a2e737',
         'compressed_sparse_attention_11_b200/csrc/common.cuh': '2c8e048cf6f6eadb',
+        'compressed_sparse_attention_11_b200/csrc/rope.cuh': '8af18f1b31f2b303',
         'compressed_sparse_attention_11_b200/csrc/tc_attn_util.cuh': 'fbd5bcb87c834e55'}},
 }
 

@@ -35,6 +35,8 @@ EXPORTED = (
     "csa_norm_rope_rows", "csa_compress_norm_rope", "csa_sparse_attn_norm_rope",
     "hca_attn_norm_rope", "csa_index_topk_lowp_workspace", "csa_index_topk_lowp",
     "csa_grouped_out_proj_workspace", "csa_grouped_out_proj",
+    "csa_paged_cache_layout", "csa_paged_cache_store_entries", "csa_paged_cache_write_rows",
+    "csa_paged_decode_step",
 )
 CSA_INDEX_FP8_QK, CSA_INDEX_BF16_SCORES = 1, 2
 
@@ -67,6 +69,11 @@ class DecodeParams(ctypes.Structure):
     _fields_ = [("ba", ctypes.c_void_p), ("bb", ctypes.c_void_p), ("iba", ctypes.c_void_p),
                 ("ibb", ctypes.c_void_p), ("sink", ctypes.c_void_p), ("scale", ctypes.c_float),
                 ("sel_out", ctypes.c_void_p), ("scores_out", ctypes.c_void_p)]
+
+
+class Paging(ctypes.Structure):
+    _fields_ = [("block_tokens", ctypes.c_int32), ("num_blocks", ctypes.c_int64),
+                ("max_blocks", ctypes.c_int64), ("block_table", ctypes.c_void_p)]
 
 
 class NormRope(ctypes.Structure):
@@ -117,6 +124,15 @@ def lib() -> ctypes.CDLL:
                                             i32, i32, ctypes.POINTER(NormRope), vp, vp]),
         "hca_attn_norm_rope": (i32, [vp, vp, vp, i32, vp, f32, i64, i64, i32, i32, i32, i32,
                                      ctypes.POINTER(NormRope), vp, vp]),
+        "csa_paged_cache_layout": (i32, [ctypes.POINTER(CacheDesc), ctypes.POINTER(Paging),
+                                         ctypes.POINTER(CacheLayout)]),
+        "csa_paged_cache_store_entries": (i32, [ctypes.POINTER(CacheDesc), ctypes.POINTER(Paging),
+                                                vp, i64, i64, vp, vp, i32, vp]),
+        "csa_paged_cache_write_rows": (i32, [ctypes.POINTER(CacheDesc), ctypes.POINTER(Paging), vp,
+                                             i64, i64, ctypes.POINTER(Rows), vp]),
+        "csa_paged_decode_step": (i32, [ctypes.POINTER(CacheDesc), ctypes.POINTER(Paging), vp, vp,
+                                        ctypes.POINTER(Rows), ctypes.POINTER(DecodeParams), vp, vp,
+                                        vp, vp, vp, sz, vp]),
         "csa_grouped_out_proj_workspace": (sz, [i64, i32, i32]),
         "csa_grouped_out_proj": (i32, [vp, i64, i32, i32, i32, i32, i32, vp, vp, vp, sz, vp, vp]),
         "csa_index_topk_lowp_workspace": (sz, [i64, i64, i32, i32, i32, i32, i32]),
@@ -363,15 +379,34 @@ def csa_grouped_out_proj(o, w1, w2, ws: Optional[torch.Tensor] = None,
 # ------------------------------------------------------------------- decode ---
 
 class CsaCache:
-    """A caller-owned decode cache (one layer, ``batch`` sequences)."""
+    """A caller-owned decode cache (one layer, ``batch`` sequences).
+
+    With ``block_table`` (int32 [batch, max_blocks] on the device) the
+    compressed entries live in a paged pool of ``num_blocks`` blocks of
+    ``block_tokens`` raw tokens each (the classical cache; capacity becomes
+    max_blocks * block_tokens // m); the window ring and the compressor tail
+    stay per sequence."""
 
     def __init__(self, batch: int, capacity: int, c: int, rope_dims: int, m: int, window: int,
                  nh: int, is_hca: bool, c_i: int = 0, nh_i: int = 0, k: int = 0,
-                 device="cuda"):
+                 device="cuda", block_table: Optional[torch.Tensor] = None,
+                 block_tokens: int = 128, num_blocks: int = 0):
+        self.paging = None
+        if block_table is not None:
+            if block_table.dtype != torch.int32 or block_table.dim() != 2:
+                raise ValueError("block_table must be an int32 [batch, max_blocks] tensor")
+            self.block_table = block_table
+            capacity = block_table.shape[1] * (block_tokens // m)
+            self.paging = Paging(int(block_tokens), int(num_blocks), int(block_table.shape[1]),
+                                 _ptr(block_table))
         self.desc = CacheDesc(batch, capacity, c, rope_dims, c_i, m, window, nh, nh_i, k,
                               1 if is_hca else 0)
         self.layout = CacheLayout()
-        _check(lib().csa_cache_layout(ctypes.byref(self.desc), ctypes.byref(self.layout)))
+        if self.paging is not None:
+            _check(lib().csa_paged_cache_layout(ctypes.byref(self.desc), ctypes.byref(self.paging),
+                                                ctypes.byref(self.layout)))
+        else:
+            _check(lib().csa_cache_layout(ctypes.byref(self.desc), ctypes.byref(self.layout)))
         self.buffer = torch.zeros(self.layout.total_bytes, dtype=torch.uint8, device=device)
         ws = int(lib().csa_decode_workspace(ctypes.byref(self.desc)))
         self.workspace = torch.empty(max(ws, 16), dtype=torch.uint8, device=device)
@@ -383,18 +418,41 @@ class CsaCache:
         return self.buffer[off:off + nbytes].view(dtype).view(*shape)
 
     def entries(self):
+        """The entry regions as [batch, capacity, ...] (gathered through the
+        block table when paged; absent blocks read as zeros)."""
         d = self.desc
         B, cap = d.batch, d.capacity
-        out = dict(codes=self.region("entry_fp8", torch.uint8, (B, cap, d.c - d.rope_dims)),
-                   scale=self.region("entry_scale", torch.float32, (B, cap)),
-                   rope=self.region("entry_rope", torch.bfloat16, (B, cap, d.rope_dims)))
+        rows = B * cap
+        if self.paging is not None:
+            epb = self.paging.block_tokens // d.m
+            rows = self.paging.num_blocks * epb
+        out = dict(codes=self.region("entry_fp8", torch.uint8, (rows, d.c - d.rope_dims)),
+                   scale=self.region("entry_scale", torch.float32, (rows,)),
+                   rope=self.region("entry_rope", torch.bfloat16, (rows, d.rope_dims)))
         if not d.is_hca:
-            out["icodes"] = self.region("ikey_fp8", torch.uint8, (B, cap, d.c_i))
-            out["iscale"] = self.region("ikey_scale", torch.float32, (B, cap))
-        return out
+            out["icodes"] = self.region("ikey_fp8", torch.uint8, (rows, d.c_i))
+            out["iscale"] = self.region("ikey_scale", torch.float32, (rows,))
+        if self.paging is None:
+            return {k: v.view(B, cap, *v.shape[1:]) for k, v in out.items()}
+        bt = self.block_table.long()
+        s = torch.arange(cap, device=bt.device)
+        blk = bt[:, s // epb]                                       # [B, cap]
+        ok = (blk >= 0) & (blk < self.paging.num_blocks)
+        row = torch.where(ok, blk * epb + (s % epb)[None, :], torch.zeros_like(blk))
+        res = {}
+        for k, v in out.items():
+            g = v[row.reshape(-1)].reshape(B, cap, *v.shape[1:]).clone()
+            g[~ok] = 0
+            res[k] = g
+        return res
 
     def store_entries(self, first: int, kv, ikey=None):
         count = kv.shape[1]
+        if self.paging is not None:
+            _check(lib().csa_paged_cache_store_entries(
+                ctypes.byref(self.desc), ctypes.byref(self.paging), _ptr(self.buffer), first,
+                count, _ptr(kv), _ptr(ikey), _dt(kv), _stream(self.buffer)))
+            return
         _check(lib().csa_cache_store_entries(ctypes.byref(self.desc), _ptr(self.buffer), first,
                                              count, _ptr(kv), _ptr(ikey), _dt(kv),
                                              _stream(self.buffer)))
@@ -412,6 +470,11 @@ class CsaCache:
     def write_rows(self, first_pos: int, rows: dict):
         count = rows["kv_win"].shape[1]
         r = self._rows(rows)
+        if self.paging is not None:
+            _check(lib().csa_paged_cache_write_rows(
+                ctypes.byref(self.desc), ctypes.byref(self.paging), _ptr(self.buffer), first_pos,
+                count, ctypes.byref(r), _stream(self.buffer)))
+            return
         _check(lib().csa_cache_write_rows(ctypes.byref(self.desc), _ptr(self.buffer), first_pos,
                                           count, ctypes.byref(r), _stream(self.buffer)))
 
@@ -440,6 +503,12 @@ class CsaCache:
                          _ptr(scores_out))
         if pos.dtype != torch.int64:
             raise ValueError("pos must be int64")
+        if self.paging is not None:
+            _check(lib().csa_paged_decode_step(
+                ctypes.byref(self.desc), ctypes.byref(self.paging), _ptr(self.buffer), _ptr(pos),
+                ctypes.byref(r), ctypes.byref(p), _ptr(q), _ptr(q_i), _ptr(w_i), _ptr(out),
+                _ptr(self.workspace), self.workspace.numel(), _stream(q)))
+            return out
         _check(lib().csa_decode_step(ctypes.byref(self.desc), _ptr(self.buffer), _ptr(pos),
                                      ctypes.byref(r), ctypes.byref(p), _ptr(q), _ptr(q_i),
                                      _ptr(w_i), _ptr(out), _ptr(self.workspace),

@@ -161,6 +161,10 @@ __device__ __forceinline__ void q_round_rope(uint32_t (&r)[32], bool mine, int r
   }
 }
 
+// kQNorm: the query RMSNorm + rotation in the prologue and the output
+// rotation in the epilogue (a separate instantiation, so that the plain
+// kernel carries none of its registers).
+template <bool kQNorm>
 __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(
     const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ kv_comp,
     const int32_t* __restrict__ idx, int k, const __nv_bfloat16* __restrict__ kv_win,
@@ -177,7 +181,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(
   int* pscan = reinterpret_cast<int*>(smem + OFF_SCAN);
   float* qinv = reinterpret_cast<float*>(smem + OFF_QINV);
   AttnBars* bar = reinterpret_cast<AttnBars*>(smem + OFF_BAR);
-  const bool qnorm = qn.gamma != nullptr;
+  constexpr bool qnorm = kQNorm;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if ((int64_t)blockIdx.x >= total) return;
@@ -691,12 +695,12 @@ cudaError_t launch_attn_tc(const void* q, const void* kv_comp, const int32_t* id
                            const void* kv_win, int window, const float* sink, float scale,
                            int64_t batch, int64_t n, int m, const QNormRope& qn, void* out,
                            unsigned int* err, cudaStream_t s) {
-  cudaError_t e = cudaFuncSetAttribute(attn_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       SMEM);
+  auto kern = qn.gamma != nullptr ? attn_tc_kernel<true> : attn_tc_kernel<false>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM);
   if (e != cudaSuccess) return e;
   const int64_t total = batch * n;
   const int64_t grid = std::min<int64_t>(total, sm_count());
-  attn_tc_kernel<<<(unsigned)grid, kThreads, SMEM, s>>>(
+  kern<<<(unsigned)grid, kThreads, SMEM, s>>>(
       (const __nv_bfloat16*)q, (const __nv_bfloat16*)kv_comp, idx, k,
       (const __nv_bfloat16*)kv_win, window, sink, scale, n, m, n / m, total, qn,
       (__nv_bfloat16*)out, err);

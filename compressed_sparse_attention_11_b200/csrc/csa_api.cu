@@ -470,19 +470,41 @@ csa_status csa_grouped_out_proj(const void* o, int64_t rows, int nh, int c, int 
                      "csa_grouped_out_proj");
 }
 
-csa_status csa_cache_layout(const csa_cache_desc* desc, csa_cache_layout_t* layout) {
-  csa_status st = check_desc(desc);
-  if (st != CSA_OK) return st;
-  REQUIRE(layout != nullptr, "layout is NULL");
-  cache_layout(*desc, layout);
+}  // extern "C"
+
+namespace {
+
+csa_status check_paging(const csa_cache_desc* d, const csa_paging* pg) {
+  if (pg == nullptr) return ok();
+  REQUIRE(pg->block_tokens >= d->m && pg->block_tokens % d->m == 0,
+          "block_tokens must be a positive multiple of m");
+  const int epb = pg->block_tokens / d->m;
+  REQUIRE((epb & (epb - 1)) == 0, "block_tokens / m must be a power of two");
+  REQUIRE(pg->num_blocks >= 1 && pg->max_blocks >= 1, "num_blocks and max_blocks must be >= 1");
+  REQUIRE(d->capacity == pg->max_blocks * epb, "capacity must equal max_blocks * block_tokens / m");
+  REQUIRE(pg->num_blocks * (int64_t)epb < ((int64_t)1 << 31), "the pool must hold < 2^31 entries");
+  REQUIRE_PTR(pg->block_table);
+  if (!d->is_hca && epb < 32)
+    return fail(CSA_ERR_UNSUPPORTED, "a paged CSA layer needs at least 32 entries per block");
   return ok();
 }
 
-csa_status csa_cache_store_entries(const csa_cache_desc* desc, void* cache, int64_t first,
-                                   int64_t count, const void* kv, const void* ikey,
-                                   csa_dtype dt, void* stream) {
+csa_status cache_layout_impl(const csa_cache_desc* desc, const csa_paging* pg,
+                             csa_cache_layout_t* layout) {
   csa_status st = check_desc(desc);
   if (st != CSA_OK) return st;
+  if ((st = check_paging(desc, pg)) != CSA_OK) return st;
+  REQUIRE(layout != nullptr, "layout is NULL");
+  cache_layout(*desc, layout, pg);
+  return ok();
+}
+
+csa_status store_entries_impl(const csa_cache_desc* desc, const csa_paging* pg, void* cache,
+                              int64_t first, int64_t count, const void* kv, const void* ikey,
+                              csa_dtype dt, void* stream) {
+  csa_status st = check_desc(desc);
+  if (st != CSA_OK) return st;
+  if ((st = check_paging(desc, pg)) != CSA_OK) return st;
   REQUIRE(valid_dt(dt), "dt must be CSA_F32 or CSA_BF16");
   REQUIRE(first >= 0 && count >= 0 && first + count <= desc->capacity,
           "entries [first, first+count) must lie within [0, capacity)");
@@ -490,7 +512,7 @@ csa_status csa_cache_store_entries(const csa_cache_desc* desc, void* cache, int6
   REQUIRE_PTR(cache);
   REQUIRE_PTR(kv);
   if (!desc->is_hca) REQUIRE_PTR(ikey);
-  return cuda_status(launch_store_entries(*desc, cache_view(*desc, cache), first, count, kv,
+  return cuda_status(launch_store_entries(*desc, cache_view(*desc, cache, pg), first, count, kv,
                                           ikey, dt, (cudaStream_t)stream),
                      "csa_cache_store_entries");
 }
@@ -511,30 +533,28 @@ static csa_status check_rows(const csa_cache_desc* d, const csa_rows* rows) {
   return ok();
 }
 
-csa_status csa_cache_write_rows(const csa_cache_desc* desc, void* cache, int64_t first_pos,
-                                int64_t count, const csa_rows* rows, void* stream) {
+csa_status write_rows_impl(const csa_cache_desc* desc, const csa_paging* pg, void* cache,
+                           int64_t first_pos, int64_t count, const csa_rows* rows, void* stream) {
   csa_status st = check_desc(desc);
   if (st != CSA_OK) return st;
+  if ((st = check_paging(desc, pg)) != CSA_OK) return st;
   REQUIRE(first_pos >= 0 && count >= 0, "first_pos and count must be >= 0");
   if (count == 0) return ok();
   REQUIRE_PTR(cache);
   if ((st = check_rows(desc, rows)) != CSA_OK) return st;
-  return cuda_status(launch_write_rows(*desc, cache_view(*desc, cache), first_pos, count, *rows,
-                                       (cudaStream_t)stream),
+  return cuda_status(launch_write_rows(*desc, cache_view(*desc, cache, pg), first_pos, count,
+                                       *rows, (cudaStream_t)stream),
                      "csa_cache_write_rows");
 }
 
-size_t csa_decode_workspace(const csa_cache_desc* desc) {
-  if (check_desc(desc) != CSA_OK) return 0;
-  return decode_workspace(*desc);
-}
-
-csa_status csa_decode_step(const csa_cache_desc* desc, void* cache, const int64_t* pos,
-                           const csa_rows* rows, const csa_decode_params* params,
-                           const void* q, const void* q_i, const float* w_i, void* out,
-                           void* ws, size_t ws_bytes, void* stream) {
+csa_status decode_step_impl(const csa_cache_desc* desc, const csa_paging* pg, void* cache,
+                            const int64_t* pos, const csa_rows* rows,
+                            const csa_decode_params* params, const void* q, const void* q_i,
+                            const float* w_i, void* out, void* ws, size_t ws_bytes,
+                            void* stream) {
   csa_status st = check_desc(desc);
   if (st != CSA_OK) return st;
+  if ((st = check_paging(desc, pg)) != CSA_OK) return st;
   REQUIRE_PTR(cache);
   REQUIRE_PTR(pos);
   if ((st = check_rows(desc, rows)) != CSA_OK) return st;
@@ -560,9 +580,68 @@ csa_status csa_decode_step(const csa_cache_desc* desc, void* cache, const int64_
   if (ws == nullptr || ws_bytes < need)
     return fail(CSA_ERR_WORKSPACE, "workspace %zu bytes < required %zu", ws_bytes, need);
   REQUIRE_PTR(ws);
-  return cuda_status(launch_decode_step(*desc, cache_view(*desc, cache), pos, *rows, *params, q,
-                                        q_i, w_i, out, ws, (cudaStream_t)stream),
+  return cuda_status(launch_decode_step(*desc, cache_view(*desc, cache, pg), pos, *rows, *params,
+                                        q, q_i, w_i, out, ws, (cudaStream_t)stream),
                      "csa_decode_step");
+}
+
+}  // namespace
+
+extern "C" {
+
+csa_status csa_cache_layout(const csa_cache_desc* desc, csa_cache_layout_t* layout) {
+  return cache_layout_impl(desc, nullptr, layout);
+}
+csa_status csa_paged_cache_layout(const csa_cache_desc* desc, const csa_paging* paging,
+                                  csa_cache_layout_t* layout) {
+  REQUIRE(paging != nullptr, "paging is NULL");
+  return cache_layout_impl(desc, paging, layout);
+}
+
+csa_status csa_cache_store_entries(const csa_cache_desc* desc, void* cache, int64_t first,
+                                   int64_t count, const void* kv, const void* ikey,
+                                   csa_dtype dt, void* stream) {
+  return store_entries_impl(desc, nullptr, cache, first, count, kv, ikey, dt, stream);
+}
+csa_status csa_paged_cache_store_entries(const csa_cache_desc* desc, const csa_paging* paging,
+                                         void* cache, int64_t first, int64_t count,
+                                         const void* kv, const void* ikey, csa_dtype dt,
+                                         void* stream) {
+  REQUIRE(paging != nullptr, "paging is NULL");
+  return store_entries_impl(desc, paging, cache, first, count, kv, ikey, dt, stream);
+}
+
+csa_status csa_cache_write_rows(const csa_cache_desc* desc, void* cache, int64_t first_pos,
+                                int64_t count, const csa_rows* rows, void* stream) {
+  return write_rows_impl(desc, nullptr, cache, first_pos, count, rows, stream);
+}
+csa_status csa_paged_cache_write_rows(const csa_cache_desc* desc, const csa_paging* paging,
+                                      void* cache, int64_t first_pos, int64_t count,
+                                      const csa_rows* rows, void* stream) {
+  REQUIRE(paging != nullptr, "paging is NULL");
+  return write_rows_impl(desc, paging, cache, first_pos, count, rows, stream);
+}
+
+size_t csa_decode_workspace(const csa_cache_desc* desc) {
+  if (check_desc(desc) != CSA_OK) return 0;
+  return decode_workspace(*desc);
+}
+
+csa_status csa_decode_step(const csa_cache_desc* desc, void* cache, const int64_t* pos,
+                           const csa_rows* rows, const csa_decode_params* params,
+                           const void* q, const void* q_i, const float* w_i, void* out,
+                           void* ws, size_t ws_bytes, void* stream) {
+  return decode_step_impl(desc, nullptr, cache, pos, rows, params, q, q_i, w_i, out, ws,
+                          ws_bytes, stream);
+}
+csa_status csa_paged_decode_step(const csa_cache_desc* desc, const csa_paging* paging,
+                                 void* cache, const int64_t* pos, const csa_rows* rows,
+                                 const csa_decode_params* params, const void* q,
+                                 const void* q_i, const float* w_i, void* out, void* ws,
+                                 size_t ws_bytes, void* stream) {
+  REQUIRE(paging != nullptr, "paging is NULL");
+  return decode_step_impl(desc, paging, cache, pos, rows, params, q, q_i, w_i, out, ws, ws_bytes,
+                          stream);
 }
 
 }  // extern "C"

@@ -33,15 +33,18 @@ constexpr int kDecSelThreads = 1024;      // one selection block per sequence
 
 static inline size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
 
-void cache_layout(const csa_cache_desc& d, csa_cache_layout_t* L) {
+void cache_layout(const csa_cache_desc& d, csa_cache_layout_t* L, const csa_paging* pg) {
   const size_t B = (size_t)d.batch, cap = (size_t)d.capacity;
   const size_t body = (size_t)(d.c - d.rope_dims);
+  // entry rows: batch x capacity, or the paged pool's blocks x entries per block
+  const size_t rows = pg != nullptr ? (size_t)pg->num_blocks * (size_t)(pg->block_tokens / d.m)
+                                    : B * cap;
   size_t off = 0;
-  L->entry_fp8 = off;   off = align256(off + B * cap * body);
-  L->entry_scale = off; off = align256(off + B * cap * 4);
-  L->entry_rope = off;  off = align256(off + B * cap * (size_t)d.rope_dims * 2);
-  L->ikey_fp8 = off;    if (!d.is_hca) off = align256(off + B * cap * (size_t)d.c_i);
-  L->ikey_scale = off;  if (!d.is_hca) off = align256(off + B * cap * 4);
+  L->entry_fp8 = off;   off = align256(off + rows * body);
+  L->entry_scale = off; off = align256(off + rows * 4);
+  L->entry_rope = off;  off = align256(off + rows * (size_t)d.rope_dims * 2);
+  L->ikey_fp8 = off;    if (!d.is_hca) off = align256(off + rows * (size_t)d.c_i);
+  L->ikey_scale = off;  if (!d.is_hca) off = align256(off + rows * 4);
   L->window = off;      off = align256(off + B * (size_t)d.window * d.c * 2);
   L->state = off;
   off = align256(off + B * 2 * (d.is_hca ? 1 : 4) * (size_t)d.m * d.c * 2);
@@ -50,9 +53,9 @@ void cache_layout(const csa_cache_desc& d, csa_cache_layout_t* L) {
   L->total_bytes = off;
 }
 
-CacheView cache_view(const csa_cache_desc& d, void* cache) {
+CacheView cache_view(const csa_cache_desc& d, void* cache, const csa_paging* pg) {
   csa_cache_layout_t L;
-  cache_layout(d, &L);
+  cache_layout(d, &L, pg);
   uint8_t* base = static_cast<uint8_t*>(cache);
   CacheView v;
   v.entry_fp8 = base + L.entry_fp8;
@@ -63,6 +66,13 @@ CacheView cache_view(const csa_cache_desc& d, void* cache) {
   v.window = reinterpret_cast<__nv_bfloat16*>(base + L.window);
   v.state = reinterpret_cast<__nv_bfloat16*>(base + L.state);
   v.istate = reinterpret_cast<__nv_bfloat16*>(base + L.istate);
+  v.btab = pg != nullptr ? pg->block_table : nullptr;
+  v.bt_stride = pg != nullptr ? pg->max_blocks : 0;
+  v.nblocks = pg != nullptr ? pg->num_blocks : 0;
+  int sh = 0;
+  if (pg != nullptr)
+    while ((1 << sh) < pg->block_tokens / d.m) ++sh;
+  v.epb_shift = sh;
   return v;
 }
 
@@ -104,7 +114,8 @@ __global__ void __launch_bounds__(256) store_entries_kernel(
     for (int e = threadIdx.x; e < d.c_i; e += blockDim.x)
       sx[d.c + e] = to_f32(ikey[(b * count + j) * d.c_i + e]);
   __syncthreads();
-  const int64_t es = b * d.capacity + slot;
+  const int64_t es = entry_row(cv, b, slot, d.capacity);
+  if (es < 0) return;  // no block for this entry (uniform over the block)
   quantize_store(sx, d.c, d.rope_dims, cv.entry_fp8 + es * (d.c - d.rope_dims),
                  cv.entry_scale + es, cv.entry_rope + es * d.rope_dims, red);
   if (!d.is_hca)
@@ -394,7 +405,8 @@ __global__ void __launch_bounds__(1024) append_emit_kernel(csa_cache_desc d, Cac
       sx[d.c + e] = emit_dim(cv.istate, b, i, d.m, d.c_i, e, p.iba, p.ibb, false);
   __syncthreads();
   float* red = sx + d.c + (d.is_hca ? 0 : d.c_i);
-  const int64_t es = b * d.capacity + i;
+  const int64_t es = entry_row(cv, b, i, d.capacity);
+  if (es < 0) return;  // no block for the emitted entry (uniform over the block)
   quantize_store(sx, d.c, d.rope_dims, cv.entry_fp8 + es * (d.c - d.rope_dims),
                  cv.entry_scale + es, cv.entry_rope + es * d.rope_dims, red);
   if (!d.is_hca)
@@ -439,8 +451,14 @@ __global__ void __launch_bounds__(kSelThreads) index_chunk_kernel(
   __syncthreads();
   for (int64_t e = threadIdx.x; e < Vc; e += blockDim.x) {
     const int64_t s = c0 + e;
-    const uint8_t* kr = cv.ikey_fp8 + (b * d.capacity + s) * ci;
-    const float ks = cv.ikey_scale[b * d.capacity + s];
+    const int64_t er = entry_row(cv, b, s, d.capacity);
+    if (er < 0) {  // no block: the entry scores 0
+      sc[e] = 0.f;
+      keys[e] = order_key(0.f);
+      continue;
+    }
+    const uint8_t* kr = cv.ikey_fp8 + er * ci;
+    const float ks = cv.ikey_scale[er];
     float score = 0.f;
     for (int hg = 0; hg < H; hg += 32) {
       float acc[32];
@@ -578,8 +596,11 @@ __global__ void __launch_bounds__(256) attn_split_kernel(
 #pragma unroll
         for (int u = 0; u < 8; ++u) v[u] = 0.f;
       } else if (row < d.capacity) {
-        const int64_t es = b * d.capacity + row;
-        if (dd < body) {
+        const int64_t es = entry_row(cv, b, row, d.capacity);
+        if (es < 0) {
+#pragma unroll
+          for (int u = 0; u < 8; ++u) v[u] = 0.f;
+        } else if (dd < body) {
           const float sc = cv.entry_scale[es];
           const uint2 raw = *reinterpret_cast<const uint2*>(cv.entry_fp8 + es * body + dd);
           const uint8_t* by = reinterpret_cast<const uint8_t*>(&raw);
@@ -677,7 +698,7 @@ __global__ void __launch_bounds__(256) attn_combine_kernel(
 // ---------------------------------------------------------------------------
 struct DecodeWs {
   int nchunks, nsplit;
-  bool tc_index, tc_attn, hist_select;
+  bool tc_index, tc_attn, hist_select, attn_select;
   size_t cand_score, cand_idx, scores, qop, sel, part_o, part_ms, select, total;
 };
 
@@ -699,6 +720,9 @@ static DecodeWs decode_ws_layout(const csa_cache_desc& d) {
   w.part_o = off;     off = align256(off + B * w.nsplit * d.nh * (size_t)d.c * 4);
   w.part_ms = off;    off = align256(off + B * w.nsplit * d.nh * 2 * 4);
   w.hist_select = w.tc_index && decode_select_supported(d);
+  // the attention kernel takes the top-k itself where the scores fit its
+  // shared memory; the selection kernel otherwise
+  w.attn_select = w.hist_select && w.tc_attn && decode_attn_selects(d);
   size_t sel_bytes = 0;
   if (w.hist_select) decode_select_ws(d, nullptr, &sel_bytes);
   w.select = off;     off = align256(off + sel_bytes);
@@ -744,7 +768,9 @@ cudaError_t launch_decode_step(const csa_cache_desc& d, const CacheView& cv, con
     // indexer then keeps no histogram)
     err = launch_decode_index_tc(d, cv, pos, qop, scores, sws.ghist, flag, s);
     if (err != cudaSuccess) return err;
-    if (w.hist_select) {
+    if (w.attn_select) {
+      err = cudaSuccess;  // the attention kernel selects
+    } else if (w.hist_select) {
       err = launch_decode_select(d, pos, scores, sws, sel, s);
     } else {
       decode_select_kernel<<<(unsigned)d.batch, kDecSelThreads, 0, s>>>(d, pos, scores, sel);
@@ -768,8 +794,13 @@ cudaError_t launch_decode_step(const csa_cache_desc& d, const CacheView& cv, con
   if (w.tc_attn) {
     unsigned int* flag = device_timeout_flag();
     if (flag == nullptr) return cudaErrorUnknown;
-    return launch_decode_attn_tc(d, cv, pos, q, sel, p.sink, p.scale, w.nsplit, out, part_o,
-                                 part_ms, flag, s);
+    const float* ascores = nullptr;
+    if (w.attn_select)
+      ascores = p.scores_out != nullptr ? p.scores_out : reinterpret_cast<float*>(wb + w.scores);
+    return launch_decode_attn_tc(d, cv, pos, q, w.attn_select ? nullptr : sel, p.sink, p.scale,
+                                 w.nsplit, out, part_o, part_ms, ascores,
+                                 w.attn_select ? sws.ghist : nullptr,
+                                 w.attn_select ? p.sel_out : nullptr, flag, s);
   }
   const size_t asmem = sizeof(float) * ((size_t)kDecTE * (d.c + 1) + (size_t)kDecHG * d.c +
                                         kDecHG * kDecTE) + sizeof(int64_t) * kDecTE;

@@ -86,12 +86,154 @@ __device__ __forceinline__ void dequant16(const uint4 c8, float sc, uint4& lo, u
   hi = make_uint4(o[4], o[5], o[6], o[7]);
 }
 
+// ---------------------------------------------------------------------------
+// The selection step inside the attention kernel (the top-k of section 4.2 of
+// "DeepSeek-V4: million-token context"; larger score first, ties to the
+// smaller index): the indexer left a histogram of the sequence's scores over
+// the top 12 bits of their order keys, which fixes the first radix digit
+// without a pass; the scores then land in shared memory as order keys (one
+// pass from L2) and two more digits (bits 19..8, then 7..0) are refined over
+// the keys of the threshold bin only, when its count does not settle the cut.
+// The chosen indices are emitted in ascending order by contiguous per-thread
+// segments.  Every thread of the CTA calls it; returns min(k, V).
+// ---------------------------------------------------------------------------
+constexpr int kSelStage = 49152;  // keys staged in shared memory (192 KB)
+constexpr int kSelBins = 4096;
+
+struct SelState {
+  uint32_t T, G, C;
+};
+
+// The bin T (among `nbins`, counts in h, bin nbins - 1 highest) where the
+// count from the top reaches `need`, with the count above it (G) and in it.
+__device__ __forceinline__ void sel_find_bin(const uint32_t* h, int nbins, uint32_t need,
+                                             int* wsum, SelState* st) {
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int per = (nbins + kThreads - 1) / kThreads;
+  uint32_t c[(kSelBins + kThreads - 1) / kThreads], loc = 0;
+#pragma unroll
+  for (int j = 0; j < (kSelBins + kThreads - 1) / kThreads; ++j) {
+    const int bin = nbins - 1 - (tid * per + j);
+    c[j] = (j < per && bin >= 0) ? h[bin] : 0u;
+    loc += c[j];
+  }
+  uint32_t inc = loc;
+#pragma unroll
+  for (int off = 1; off < 32; off <<= 1) {
+    const uint32_t x = __shfl_up_sync(0xffffffffu, inc, off);
+    if (lane >= off) inc += x;
+  }
+  if (lane == 31) wsum[warp] = (int)inc;
+  __syncthreads();
+  uint32_t acc = inc - loc;
+  for (int w = 0; w < warp; ++w) acc += (uint32_t)wsum[w];
+#pragma unroll
+  for (int j = 0; j < (kSelBins + kThreads - 1) / kThreads; ++j) {
+    const int bin = nbins - 1 - (tid * per + j);
+    if (j < per && bin >= 0 && acc < need && acc + c[j] >= need) {
+      st->T = (uint32_t)bin;
+      st->G = acc;
+      st->C = c[j];
+    }
+    acc += c[j];
+  }
+  __syncthreads();
+}
+
+__device__ int fused_select(const float* __restrict__ row, const uint32_t* __restrict__ gh,
+                            int V, int k, uint32_t* skey, uint32_t* hist, int32_t* list,
+                            int* wsum, SelState* st) {
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  if (V <= k) {
+    for (int i = tid; i < V; i += kThreads) list[i] = i;
+    __syncthreads();
+    return V;
+  }
+  // the row into shared memory in one round trip (4-byte cp.async: rows are
+  // `capacity` floats apart, so not 16-byte aligned in general), then as
+  // order keys in place
+  for (int i = tid; i < V; i += kThreads)
+    asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(
+                     (uint32_t)__cvta_generic_to_shared(skey + i)),
+                 "l"(row + i)
+                 : "memory");
+  asm volatile("cp.async.commit_group;\n\tcp.async.wait_all;" ::: "memory");
+  __syncthreads();
+  for (int i = tid; i < V; i += kThreads) skey[i] = order_key(__uint_as_float(skey[i]));
+  // digit 1 (bits 31..20) from the indexer's histogram
+  for (int j = tid; j < kSelBins; j += kThreads) hist[j] = __ldcg(gh + j);
+  if (tid == 0) *st = SelState{0u, 0u, 0u};  // (a histogram short of k: a capped result)
+  __syncthreads();
+  sel_find_bin(hist, kSelBins, (uint32_t)k, wsum, st);
+  uint32_t need = (uint32_t)k - st->G;
+  uint32_t prefix = st->T << 20, mask = 0xfff00000u;
+  bool all_eq = st->C == need;
+  // digits 2 (bits 19..8, 4096 bins) and 3 (bits 7..0, 256 bins), over the
+  // keys that share the prefix, while the threshold bin does not settle it
+  for (int lvl = 0; lvl < 2 && !all_eq; ++lvl) {
+    const int shift = lvl == 0 ? 8 : 0;
+    const int nb = lvl == 0 ? 4096 : 256;
+    for (int j = tid; j < nb; j += kThreads) hist[j] = 0u;
+    __syncthreads();
+    for (int i = tid; i < V; i += kThreads) {
+      const uint32_t ky = skey[i];
+      if ((ky & mask) == prefix) atomicAdd(&hist[(ky >> shift) & (uint32_t)(nb - 1)], 1u);
+    }
+    __syncthreads();
+    sel_find_bin(hist, nb, need, wsum, st);
+    need -= st->G;
+    prefix |= st->T << shift;
+    mask |= (uint32_t)(nb - 1) << shift;
+    all_eq = st->C == need;
+  }
+  // emit: key above the prefix, or equal to it (all of them, or the first
+  // `need` in index order); contiguous segments per thread keep the order
+  const int per = (V + kThreads - 1) / kThreads;
+  const int lo = min(V, tid * per), hi = min(V, lo + per);
+  uint32_t gt = 0, eq = 0;
+  for (int i = lo; i < hi; ++i) {
+    const uint32_t km = skey[i] & mask;
+    gt += km > prefix ? 1u : 0u;
+    eq += km == prefix ? 1u : 0u;
+  }
+  // exclusive prefix of eq, then of the taken counts
+  auto excl = [&](uint32_t v) -> uint32_t {
+    uint32_t inc = v;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+      const uint32_t x = __shfl_up_sync(0xffffffffu, inc, off);
+      if (lane >= off) inc += x;
+    }
+    if (lane == 31) wsum[warp] = (int)inc;
+    __syncthreads();
+    uint32_t a = inc - v;
+    for (int w = 0; w < warp; ++w) a += (uint32_t)wsum[w];
+    __syncthreads();
+    return a;
+  };
+  const uint32_t eq_before = excl(eq);
+  const uint32_t take_eq = all_eq ? eq : (eq_before >= need ? 0u : min(eq, need - eq_before));
+  uint32_t o = excl(gt + take_eq);
+  uint32_t eq_seen = 0;
+  for (int i = lo; i < hi; ++i) {
+    const uint32_t km = skey[i] & mask;
+    const bool is_eq = km == prefix;
+    const bool take = km > prefix || (is_eq && eq_seen < take_eq);
+    eq_seen += is_eq ? 1u : 0u;
+    if (take && o < (uint32_t)k) list[o] = i;
+    o += take ? 1u : 0u;
+  }
+  __syncthreads();
+  return k;
+}
+
 __global__ void __launch_bounds__(kThreads, 1) decode_attn_tc_kernel(
     const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CacheView cv,
     const int64_t* __restrict__ pos, const int32_t* __restrict__ sel, int k, int window, int m,
     int64_t cap, const float* __restrict__ sink, float scale, int nsplit,
     float* __restrict__ part_o, float* __restrict__ part_ms, __nv_bfloat16* __restrict__ out,
-    unsigned int* __restrict__ err) {
+    const float* __restrict__ scores, const uint32_t* __restrict__ ghist,
+    int32_t* __restrict__ sel_out, unsigned int* __restrict__ err) {
   using namespace sm100;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = smem_raw + ((1024 - (smem_u32(smem_raw) & 1023)) & 1023);
@@ -138,8 +280,18 @@ __global__ void __launch_bounds__(kThreads, 1) decode_attn_tc_kernel(
   const int nwin = t < 0 ? 0 : (int)(t - w0 + 1);
 
   // -------- the entry list: valid selections in order (CSA) or 0..V-1 (HCA) ----
+  // (scores != NULL: the CSA selection itself runs here, from the indexer's
+  // scores and histogram)
+  const bool csa = sel != nullptr || scores != nullptr;
   int nsel;
-  if (sel != nullptr) {
+  if (scores != nullptr) {
+    SelState* st = reinterpret_cast<SelState*>(red);
+    nsel = fused_select(scores + b * cap, ghist + b * kSelBins, (int)V, k,
+                        reinterpret_cast<uint32_t*>(sQ), reinterpret_cast<uint32_t*>(sP), list,
+                        wcount, st);
+    if (sel_out != nullptr && split == 0)
+      for (int j = tid; j < k; j += kThreads) sel_out[b * k + j] = j < nsel ? list[j] : -1;
+  } else if (sel != nullptr) {
     const int32_t* row = sel + b * k;
     const int per = (k + kThreads - 1) / kThreads;
     const int lo = min(k, tid * per), hi = min(k, lo + per);
@@ -196,8 +348,10 @@ __global__ void __launch_bounds__(kThreads, 1) decode_attn_tc_kernel(
       if (r >= kTE) continue;
       const int slot = tile * kTE + r;
       if (slot < nsel) {
-        const int64_t es = b * cap + (sel != nullptr ? (int64_t)list[slot] : (int64_t)slot);
-        if (body) {
+        const int64_t es = entry_row(cv, b, csa ? (int64_t)list[slot] : (int64_t)slot, cap);
+        if (es < 0) {
+          // no block for this entry: zeros
+        } else if (body) {
           lo[i] = __ldcs(reinterpret_cast<const uint4*>(cv.entry_fp8 + es * kBody + s_me * 64 +
                                                          q_me * 16));
           hi[i].x = __float_as_uint(__ldcs(cv.entry_scale + es));
@@ -495,10 +649,15 @@ int decode_attn_splits(const csa_cache_desc& d) {
   return (int)std::max<int64_t>(1, std::min<int64_t>(tmax, per_sm));
 }
 
+bool decode_attn_selects(const csa_cache_desc& d) {
+  return !d.is_hca && d.capacity <= kSelStage && d.k <= kMaxSelDec;
+}
+
 cudaError_t launch_decode_attn_tc(const csa_cache_desc& d, const CacheView& cv,
                                   const int64_t* pos, const void* q, const int32_t* sel,
                                   const float* sink, float scale, int nsplit, void* out,
-                                  float* part_o, float* part_ms, unsigned int* err,
+                                  float* part_o, float* part_ms, const float* scores,
+                                  const uint32_t* ghist, int32_t* sel_out, unsigned int* err,
                                   cudaStream_t s) {
   CUtensorMap tq;
   if (!make_tmap_bf16_3d(&tq, q, kC, kNH, d.batch, kC * 2ull, (uint64_t)kNH * kC * 2, 64, kNH))
@@ -509,7 +668,7 @@ cudaError_t launch_decode_attn_tc(const csa_cache_desc& d, const CacheView& cv,
   e = launch_pdl(decode_attn_tc_kernel, dim3((unsigned)nsplit, (unsigned)d.batch), dim3(kThreads),
                  (size_t)SMEM, s, tq, cv, pos, d.is_hca ? nullptr : sel, (int)d.k, (int)d.window,
                  (int)d.m, (int64_t)d.capacity, sink, scale, nsplit, part_o, part_ms,
-                 (__nv_bfloat16*)out, err);
+                 (__nv_bfloat16*)out, scores, ghist, sel_out, err);
   if (e != cudaSuccess || nsplit == 1) return e;
   return launch_pdl(decode_combine_kernel, dim3(kNH, (unsigned)d.batch), dim3(kC / 4), 0, s,
                     (const float*)part_o, (const float*)part_ms, sink, nsplit,

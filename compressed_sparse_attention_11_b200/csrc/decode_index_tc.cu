@@ -102,6 +102,47 @@ __device__ __forceinline__ void hist_add(uint32_t* hist, int slot, float score) 
   atomicAdd(hist + slot * kHistBins + (order_key(score) >> kHistShift), 1u);
 }
 
+// Paged classical cache: entry s of sequence b in block btab[b][s >> shift]
+// of the pool (btab == NULL: the contiguous [batch][capacity] form).  A key
+// tile is then brought in as boxes of `box` rows, one per block piece.
+struct PagedKeys {
+  const int32_t* btab;
+  int64_t stride, nblocks;
+  int shift, box;
+};
+
+__device__ __forceinline__ int64_t paged_row(const PagedKeys& pk, int64_t b, int64_t s,
+                                             int64_t cap) {
+  if (pk.btab == nullptr) return b * cap + s;
+  const int64_t blk = pk.btab[b * pk.stride + (s >> pk.shift)];
+  if (blk < 0 || blk >= pk.nblocks) return -1;
+  return (blk << pk.shift) + (s & ((int64_t(1) << pk.shift) - 1));
+}
+
+// Rows (or -1) of the boxes of keys s0 .. s0 + tk - 1 below V; returns the
+// bytes the present ones bring.
+__device__ __forceinline__ uint32_t paged_tile_rows(const PagedKeys& pk, int64_t b, int64_t s0,
+                                                    int tk, int64_t V, int64_t cap,
+                                                    int64_t (&rows)[8]) {
+  uint32_t bytes = 0;
+#pragma unroll
+  for (int q = 0; q < 8; ++q) {
+    rows[q] = -1;
+    const int64_t sq = s0 + (int64_t)q * pk.box;
+    if (q * pk.box < tk && sq < V) rows[q] = paged_row(pk, b, sq, cap);
+    if (rows[q] >= 0) bytes += (uint32_t)pk.box * 128u;
+  }
+  return bytes;
+}
+
+__device__ __forceinline__ void paged_tile_load(const CUtensorMap* tm, uint64_t* bar,
+                                                uint8_t* dst, const PagedKeys& pk,
+                                                const int64_t (&rows)[8]) {
+#pragma unroll
+  for (int q = 0; q < 8; ++q)
+    if (rows[q] >= 0) sm100::tma_load_3d(dst + q * pk.box * 128, tm, bar, 0, (int)rows[q], 0);
+}
+
 // Tiles of tk keys of sequence b.
 __device__ __forceinline__ int tiles_of(const int64_t* pos, int64_t b, int m, int64_t cap,
                                         int tk) {
@@ -171,8 +212,9 @@ __device__ void locate_range(const int64_t* pos, int64_t batch, int m, int64_t c
 template <int H>
 __global__ void __launch_bounds__(kThreads, 1) decode_index_tc_kernel(
     const __grid_constant__ CUtensorMap tm_keys, const float* __restrict__ key_scale,
-    const uint8_t* __restrict__ qop, const int64_t* __restrict__ pos, int64_t batch, int64_t cap, int m,
-    float* __restrict__ scores, uint32_t* __restrict__ ghist, unsigned int* __restrict__ err) {
+    PagedKeys pk, const uint8_t* __restrict__ qop, const int64_t* __restrict__ pos, int64_t batch,
+    int64_t cap, int m, float* __restrict__ scores, uint32_t* __restrict__ ghist,
+    unsigned int* __restrict__ err) {
   using C = DecIdxCfg<H>;
   constexpr int S = C::STAGES;
   using namespace sm100;
@@ -246,11 +288,25 @@ __global__ void __launch_bounds__(kThreads, 1) decode_index_tc_kernel(
       const int s = k % S;
       if (k >= S && !mbar_wait(&bar->empty[s], (uint32_t)(((k / S) - 1) & 1), err)) break;
       const int here = min(TPP, count - k * TPP);
-      if (lane == 0) mbar_arrive_expect_tx(&bar->full[s], here * kTileBytes);
-      for (int r = 0; r < here; ++r, it.next(pos, batch, m, cap))
-        if (lane == 0)
-          tma_load_3d(sRaw + s * C::STAGE_BYTES + r * kTileBytes, &tm_keys, &bar->full[s], 0,
-                      it.j * kKeys, (int)it.b);
+      if (pk.btab == nullptr) {
+        if (lane == 0) mbar_arrive_expect_tx(&bar->full[s], here * kTileBytes);
+        for (int r = 0; r < here; ++r, it.next(pos, batch, m, cap))
+          if (lane == 0)
+            tma_load_3d(sRaw + s * C::STAGE_BYTES + r * kTileBytes, &tm_keys, &bar->full[s], 0,
+                        it.j * kKeys, (int)it.b);
+      } else {  // paged: per-block boxes of each tile of the stage, one barrier arm
+        int64_t rows[TPP][8];
+        uint32_t bytes = 0;
+        TileWalk w2 = it;
+        for (int r = 0; r < here; ++r, w2.next(pos, batch, m, cap))
+          bytes += paged_tile_rows(pk, w2.b, (int64_t)w2.j * kKeys, kKeys,
+                                   min((pos[w2.b] + 1) / m, cap), cap, rows[r]);
+        if (lane == 0) mbar_arrive_expect_tx(&bar->full[s], bytes);
+        for (int r = 0; r < here; ++r, it.next(pos, batch, m, cap))
+          if (lane == 0)
+            paged_tile_load(&tm_keys, &bar->full[s], sRaw + s * C::STAGE_BYTES + r * kTileBytes,
+                            pk, rows[r]);
+      }
       __syncwarp();
     }
     // every issued stage has landed before the CTA exits
@@ -340,7 +396,8 @@ __global__ void __launch_bounds__(kThreads, 1) decode_index_tc_kernel(
     auto scale_of = [&](const TileWalk& w) -> float {
       const int64_t sidx = (int64_t)w.j * kKeys + row;
       const int64_t Vw = min((pos[w.b] + 1) / m, cap);
-      return sidx < Vw ? __ldcs(key_scale + w.b * cap + sidx) : 0.f;
+      const int64_t kr = sidx < Vw ? paged_row(pk, w.b, sidx, cap) : -1;
+      return kr >= 0 ? __ldcs(key_scale + kr) : 0.f;
     };
     TileWalk ahead = it;
     int first = 0;  // this group's first tile
@@ -473,8 +530,8 @@ __device__ __forceinline__ void reduce_scatter8(float (&v)[8], int lane) {
 
 __global__ void __launch_bounds__(kThreads, 1) decode_index_sw_kernel(
     const __grid_constant__ CUtensorMap tm_keys, const float* __restrict__ key_scale,
-    const uint8_t* __restrict__ qop, const int64_t* __restrict__ pos, int64_t batch, int64_t cap,
-    int m, float* __restrict__ scores, uint32_t* __restrict__ ghist,
+    PagedKeys pk, const uint8_t* __restrict__ qop, const int64_t* __restrict__ pos, int64_t batch,
+    int64_t cap, int m, float* __restrict__ scores, uint32_t* __restrict__ ghist,
     unsigned int* __restrict__ err) {
   constexpr int S = kSwStages;
   using namespace sm100;
@@ -546,10 +603,20 @@ __global__ void __launch_bounds__(kThreads, 1) decode_index_sw_kernel(
     for (; i < count; ++i, it.next(pos, batch, m, cap)) {
       const int s = i % S;
       if (i >= S && !mbar_wait(&bar->empty[s], (uint32_t)(((i / S) - 1) & 1), err)) break;
-      if (lane == 0) {
-        mbar_arrive_expect_tx(&bar->full[s], kSwTileBytes);
-        tma_load_3d(sRaw + s * kSwTileBytes, &tm_keys, &bar->full[s], 0, it.j * kSwKeys,
-                    (int)it.b);
+      if (pk.btab == nullptr) {
+        if (lane == 0) {
+          mbar_arrive_expect_tx(&bar->full[s], kSwTileBytes);
+          tma_load_3d(sRaw + s * kSwTileBytes, &tm_keys, &bar->full[s], 0, it.j * kSwKeys,
+                      (int)it.b);
+        }
+      } else {  // paged: one box per block piece of the tile
+        int64_t rows[8];
+        const uint32_t bytes = paged_tile_rows(pk, it.b, (int64_t)it.j * kSwKeys, kSwKeys,
+                                               min((pos[it.b] + 1) / m, cap), cap, rows);
+        if (lane == 0) {
+          mbar_arrive_expect_tx(&bar->full[s], bytes);
+          paged_tile_load(&tm_keys, &bar->full[s], sRaw + s * kSwTileBytes, pk, rows);
+        }
       }
       __syncwarp();
     }
@@ -644,9 +711,9 @@ __global__ void __launch_bounds__(kThreads, 1) decode_index_sw_kernel(
       if ((i & 1) == grp) {
         // key scales of this thread's two keys, ahead of the accumulator
         const int64_t s0 = (int64_t)it.j * kSwKeys + 2 * p;
-        const float* ksp = key_scale + it.b * cap + s0;
-        const float ks0 = s0 < V ? __ldcs(ksp) : 0.f;
-        const float ks1 = s0 + 1 < V ? __ldcs(ksp + 1) : 0.f;
+        const int64_t kr0 = s0 < V ? paged_row(pk, it.b, s0, cap) : -1;  // s0 even: one block
+        const float ks0 = kr0 >= 0 ? __ldcs(key_scale + kr0) : 0.f;
+        const float ks1 = kr0 >= 0 && s0 + 1 < V ? __ldcs(key_scale + kr0 + 1) : 0.f;
         const bool ok =
             alive && mbar_wait(&bar->w_full[u % kWSlots], (uint32_t)((u / kWSlots) & 1), err) &&
             mbar_wait(&bar->d_full[grp], (uint32_t)(mine & 1), err);
@@ -728,21 +795,37 @@ __global__ void __launch_bounds__(kThreads, 1) decode_index_sw_kernel(
   }
 }
 
+// The key tensor map: [batch][capacity][128] with boxes of `tk` keys, or
+// (paged) the pool's [blocks * entries-per-block][128] rows with boxes of one
+// block piece; the matching PagedKeys.
+bool key_map(const csa_cache_desc& d, const CacheView& cv, int tk, CUtensorMap* tm,
+             PagedKeys* pk) {
+  if (cv.btab == nullptr) {
+    *pk = PagedKeys{nullptr, 0, 0, 0, tk};
+    return make_tmap_3d(tm, cv.ikey_fp8, 1, kCI, (uint64_t)d.capacity, (uint64_t)d.batch, kCI,
+                        (uint64_t)d.capacity * kCI, kCI, (uint32_t)tk);
+  }
+  const int epb = 1 << cv.epb_shift;
+  const int box = std::min(epb, tk);
+  *pk = PagedKeys{cv.btab, cv.bt_stride, cv.nblocks, cv.epb_shift, box};
+  const uint64_t rows = (uint64_t)cv.nblocks << cv.epb_shift;
+  return make_tmap_3d(tm, cv.ikey_fp8, 1, kCI, rows, 1, kCI, rows * kCI, kCI, (uint32_t)box);
+}
+
 cudaError_t launch_sw(const csa_cache_desc& d, const CacheView& cv, const int64_t* pos,
                       const uint8_t* qop, float* scores, uint32_t* ghist, unsigned int* err,
                       cudaStream_t s) {
   CUtensorMap tk;
-  if (!make_tmap_3d(&tk, cv.ikey_fp8, 1, kCI, (uint64_t)d.capacity, (uint64_t)d.batch, kCI,
-                    (uint64_t)d.capacity * kCI, kCI, kSwKeys))
-    return cudaErrorInvalidValue;
+  PagedKeys pk;
+  if (!key_map(d, cv, kSwKeys, &tk, &pk)) return cudaErrorInvalidValue;
   cudaError_t e = cudaFuncSetAttribute(decode_index_sw_kernel,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, kSwSmem);
   if (e != cudaSuccess) return e;
   const int64_t max_tiles = d.batch * ((d.capacity + kSwKeys - 1) / kSwKeys);
   const unsigned grid = (unsigned)std::max<int64_t>(1, std::min<int64_t>(sm_count(), max_tiles));
   return launch_pdl(decode_index_sw_kernel, dim3(grid), dim3(kThreads), (size_t)kSwSmem, s, tk,
-                    (const float*)cv.ikey_scale, qop, pos, (int64_t)d.batch, (int64_t)d.capacity,
-                    d.m, scores, ghist, err);
+                    (const float*)cv.ikey_scale, pk, qop, pos, (int64_t)d.batch,
+                    (int64_t)d.capacity, d.m, scores, ghist, err);
 }
 
 template <int H>
@@ -751,16 +834,15 @@ cudaError_t launch_h(const csa_cache_desc& d, const CacheView& cv, const int64_t
                      cudaStream_t s) {
   using C = DecIdxCfg<H>;
   CUtensorMap tk;
-  if (!make_tmap_3d(&tk, cv.ikey_fp8, 1, kCI, (uint64_t)d.capacity, (uint64_t)d.batch, kCI,
-                    (uint64_t)d.capacity * kCI, kCI, kKeys))
-    return cudaErrorInvalidValue;
+  PagedKeys pk;
+  if (!key_map(d, cv, kKeys, &tk, &pk)) return cudaErrorInvalidValue;
   auto kern = decode_index_tc_kernel<H>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
   if (e != cudaSuccess) return e;
   const int64_t max_tiles = d.batch * ((d.capacity + kKeys - 1) / kKeys);
   const unsigned grid = (unsigned)std::max<int64_t>(1, std::min<int64_t>(sm_count(), max_tiles));
   return launch_pdl(kern, dim3(grid), dim3(kThreads), (size_t)C::SMEM, s, tk,
-                    (const float*)cv.ikey_scale, qop, pos,
+                    (const float*)cv.ikey_scale, pk, qop, pos,
                     (int64_t)d.batch, (int64_t)d.capacity, d.m, scores, ghist, err);
 }
 

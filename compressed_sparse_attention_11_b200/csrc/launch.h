@@ -137,10 +137,15 @@ cudaError_t launch_decode_select(const csa_cache_desc& d, const int64_t* pos, co
 // tile per CTA (ntile = decode_attn_splits), merged by a combine kernel.
 bool decode_attn_tc_supported(const csa_cache_desc& d);
 int decode_attn_splits(const csa_cache_desc& d);
+// With scores != NULL (CSA, decode_attn_selects(d)) the kernel takes the
+// top-k itself from the indexer's scores and histogram (sel unused) and, if
+// sel_out != NULL, writes the selection there.
+bool decode_attn_selects(const csa_cache_desc& d);
 cudaError_t launch_decode_attn_tc(const csa_cache_desc& d, const CacheView& cv,
                                   const int64_t* pos, const void* q, const int32_t* sel,
                                   const float* sink, float scale, int nsplit, void* out,
-                                  float* part_o, float* part_ms, unsigned int* err,
+                                  float* part_o, float* part_ms, const float* scores,
+                                  const uint32_t* ghist, int32_t* sel_out, unsigned int* err,
                                   cudaStream_t s);
 
 // nr != NULL: each entry i RMSNorm-ed and its trailing dims rotated for
@@ -187,10 +192,28 @@ struct CacheView {
   __nv_bfloat16* window;
   __nv_bfloat16* state;
   __nv_bfloat16* istate;
+  // paged classical cache: entry s of sequence b sits in physical block
+  // btab[b][s >> epb_shift] of the pool, row s & (epb - 1); NULL btab: the
+  // contiguous [batch][capacity] form
+  const int32_t* btab;
+  int64_t bt_stride;   // block-table row length
+  int64_t nblocks;     // blocks in the pool
+  int epb_shift;       // log2(entries per block)
 };
 
-CacheView cache_view(const csa_cache_desc& d, void* cache);
-void cache_layout(const csa_cache_desc& d, csa_cache_layout_t* L);
+// Row of entry s of sequence b in the entry regions, or -1 when its block is
+// absent from the pool (such entries read as zero and are not written).
+__host__ __device__ __forceinline__ int64_t entry_row(const CacheView& cv, int64_t b, int64_t s,
+                                                      int64_t cap) {
+  if (cv.btab == nullptr) return b * cap + s;
+  const int64_t blk = cv.btab[b * cv.bt_stride + (s >> cv.epb_shift)];
+  if (blk < 0 || blk >= cv.nblocks) return -1;
+  return (blk << cv.epb_shift) + (s & ((int64_t(1) << cv.epb_shift) - 1));
+}
+
+// Paging of the classical cache (NULL: contiguous).
+CacheView cache_view(const csa_cache_desc& d, void* cache, const csa_paging* pg = nullptr);
+void cache_layout(const csa_cache_desc& d, csa_cache_layout_t* L, const csa_paging* pg = nullptr);
 
 cudaError_t launch_store_entries(const csa_cache_desc& d, const CacheView& cv, int64_t first,
                                  int64_t count, const void* kv, const void* ikey, csa_dtype dt,

@@ -388,6 +388,49 @@ csa_status csa_decode_step(const csa_cache_desc* desc, void* cache, const int64_
                            const void* q, const void* q_i, const float* w_i, void* out,
                            void* ws, size_t ws_bytes, void* stream);
 
+/* ------------------------------------------------------------------------
+ * Paged classical cache ([Analysis] "Inference KV Cache": the compressed
+ * entries live in a classical cache of blocks allocated per request, each
+ * block covering lcm(m, m') raw tokens -- 128 for V4's m = 4 and m' = 128,
+ * i.e. 32 CSA entries or 1 HCA entry per block -- so CSA and HCA layers of a
+ * sequence share one block table; the state cache (window ring and
+ * compressor tail) stays per sequence).  DSA is the special case m = 1 (one
+ * entry per token, 128 per block).
+ *
+ * The entry regions (entry_fp8, entry_scale, entry_rope, ikey_fp8,
+ * ikey_scale) then hold num_blocks * (block_tokens / m) rows instead of
+ * batch * capacity: entry s of sequence b is row
+ *   block_table[b][s / epb] * epb + s % epb,   epb = block_tokens / m.
+ * Entries whose block is absent (-1 or >= num_blocks) read as zero and are
+ * not written; the caller allocates a sequence's blocks before it reaches
+ * them.  desc->capacity must equal max_blocks * epb.  epb must be a power of
+ * two, and at least 32 for CSA layers.
+ * ------------------------------------------------------------------------ */
+typedef struct {
+  int32_t block_tokens;        /* raw tokens per block (a multiple of m)          */
+  int64_t num_blocks;          /* blocks in the pool                              */
+  int64_t max_blocks;          /* block-table row length                          */
+  const int32_t* block_table;  /* device [batch][max_blocks] int32 (-1: absent)    */
+} csa_paging;
+
+/* The paged forms of csa_cache_layout, csa_cache_store_entries,
+ * csa_cache_write_rows and csa_decode_step: same arguments and results,
+ * plus the paging; csa_decode_workspace applies unchanged. */
+csa_status csa_paged_cache_layout(const csa_cache_desc* desc, const csa_paging* paging,
+                                  csa_cache_layout_t* layout);
+csa_status csa_paged_cache_store_entries(const csa_cache_desc* desc, const csa_paging* paging,
+                                         void* cache, int64_t first, int64_t count,
+                                         const void* kv, const void* ikey, csa_dtype dt,
+                                         void* stream);
+csa_status csa_paged_cache_write_rows(const csa_cache_desc* desc, const csa_paging* paging,
+                                      void* cache, int64_t first_pos, int64_t count,
+                                      const csa_rows* rows, void* stream);
+csa_status csa_paged_decode_step(const csa_cache_desc* desc, const csa_paging* paging,
+                                 void* cache, const int64_t* pos, const csa_rows* rows,
+                                 const csa_decode_params* params, const void* q,
+                                 const void* q_i, const float* w_i, void* out, void* ws,
+                                 size_t ws_bytes, void* stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -54,17 +54,34 @@ def test_store_entries_bit_exact(dt):
             assert got["iscale"][b, 2 + e].item() == iscale
 
 
-def _setup(w, B, E, steps, seed, edit=None):
+def _block_table(B, cap, epb, seed):
+    """A block table covering `cap` entries per sequence in a pool with a few
+    spare blocks, the physical blocks in a random order."""
+    nb = (cap + epb - 1) // epb
+    pool = B * nb + 7
+    perm = np.random.default_rng(seed).permutation(pool)[:B * nb]
+    return torch.tensor(perm.reshape(B, nb), dtype=torch.int32, device=DEV), pool
+
+
+def _setup(w, B, E, steps, seed, edit=None, paged=False):
     """Cache with E stored entries and raw rows up to position t0-1 (t0 = m*E).
-    ``edit(inp)`` may change the host inputs in place before anything uses them."""
+    ``edit(inp)`` may change the host inputs in place before anything uses them.
+    ``paged``: the entries in a pool of 128-token blocks behind a block table."""
     t0 = w.m * E
     inp = G.decode_inputs(w, entries=E, batch=B, t=t0, steps=steps, seed=seed)
     if edit is not None:
         edit(inp)
     first = int(inp["first_pos"])
     cap = E + steps // w.m + 2
-    cache = csa.CsaCache(B, cap, w.c, w.rope_dims, w.m, w.window, w.nh, w.is_hca, c_i=w.c_i,
-                         nh_i=w.nh_i, k=w.k)
+    if paged:
+        epb = 128 // w.m
+        bt, pool = _block_table(B, cap, epb, seed)
+        cache = csa.CsaCache(B, cap, w.c, w.rope_dims, w.m, w.window, w.nh, w.is_hca,
+                             c_i=w.c_i, nh_i=w.nh_i, k=w.k, block_table=bt, block_tokens=128,
+                             num_blocks=pool)
+    else:
+        cache = csa.CsaCache(B, cap, w.c, w.rope_dims, w.m, w.window, w.nh, w.is_hca,
+                             c_i=w.c_i, nh_i=w.nh_i, k=w.k)
     cache.store_entries(0, inp["cache_kv"].to(DEV),
                         None if w.is_hca else inp["cache_ikey"].to(DEV))
     tail = w.window + 2 * w.m
@@ -91,8 +108,9 @@ def _biases(inp, w):
     return {k: inp[k] for k in keys}
 
 
-def _run_and_compare(w, B, E, steps, seed, check_seqs=None, edit=None, sel_exact=False):
-    inp, cache, t0, first, tail, names = _setup(w, B, E, steps, seed, edit)
+def _run_and_compare(w, B, E, steps, seed, check_seqs=None, edit=None, sel_exact=False,
+                     paged=False):
+    inp, cache, t0, first, tail, names = _setup(w, B, E, steps, seed, edit, paged)
     biases = _biases(inp, w)
     dbias = {k: v.to(DEV) for k, v in biases.items()}
     sink = inp["sink"].to(DEV)
@@ -278,3 +296,60 @@ def test_decode_index_scores_match_oracle_elementwise():
         assert np.all(np.isfinite(got[b, :V]))
         assert np.all(err <= bound), (b, float(err.max()), float((err / bound).max()))
         assert np.isnan(got[b, V:]).all()             # nothing past the visible entries
+
+
+# ----------------------------------------------------------- paged cache ---
+# The classical cache in 128-token blocks behind a block table ([Analysis]
+# "Inference KV Cache"): 32 CSA entries or 1 HCA entry per block (m = 4, 128).
+
+def test_paged_decode_csa_realistic_dims():
+    w = G.Decode("csa_decode_paged", 2, 0, 512, 64, 4, 64, 128, False, nh_i=64, c_i=128, k=512,
+                 seed=111)
+    _run_and_compare(w, B=2, E=2500, steps=4, seed=18, paged=True)
+
+
+def test_paged_decode_csa_128_index_heads():
+    w = G.Decode("csa_decode_paged_h128", 2, 0, 512, 64, 4, 64, 128, False, nh_i=128, c_i=128,
+                 k=256, seed=112)
+    _run_and_compare(w, B=2, E=1300, steps=3, seed=19, paged=True)
+
+
+def test_paged_decode_hca_split_k():
+    w = G.Decode("hca_decode_paged", 2, 0, 512, 64, 128, 64, 128, True, seed=113)
+    _run_and_compare(w, B=2, E=300, steps=2, seed=20, paged=True)
+
+
+def test_dsa_decode_is_csa_with_m1():
+    """m = 1: every token is an entry and the indexer picks the top k among all
+    of them (the fine-grained token selection of DSA), here in 128-entry
+    blocks of the paged cache and in the contiguous cache."""
+    w = G.Decode("dsa_decode", 2, 0, 512, 64, 1, 64, 128, False, nh_i=64, c_i=128, k=256,
+                 seed=114)
+    _run_and_compare(w, B=2, E=3000, steps=3, seed=21, paged=True)
+    _run_and_compare(w, B=2, E=700, steps=2, seed=22)
+
+
+def test_paged_decode_bit_identical_to_contiguous():
+    """Same inputs through the contiguous and the paged cache: the same
+    arithmetic on the same values, only the entry addresses differ."""
+    w = G.Decode("csa_decode_pair", 3, 0, 512, 64, 4, 64, 128, False, nh_i=64, c_i=128, k=512,
+                 seed=115)
+    B, E, steps = 3, 2300, 5
+    outs = []
+    for paged in (False, True):
+        inp, cache, t0, first, tail, names = _setup(w, B, E, steps, 23, paged=paged)
+        biases = {k: v.to(DEV) for k, v in _biases(inp, w).items()}
+        res = []
+        for s_ in range(steps):
+            rows = {nm: inp["rows_" + nm][:, tail + s_].contiguous().to(DEV) for nm in names}
+            pos = torch.full((B,), t0 + s_, dtype=torch.int64, device=DEV)
+            sel = torch.empty((B, w.k), dtype=torch.int32, device=DEV)
+            o = cache.decode_step(pos, rows, biases, inp["sink"].to(DEV), w.scale,
+                                  inp["q"][s_].to(DEV), inp["q_i"][s_].to(DEV),
+                                  inp["w_i"][s_].to(DEV), sel_out=sel)
+            res.append((host(o), host(sel)))
+        csa.csa_check()
+        outs.append(res)
+    for (o1, s1), (o2, s2) in zip(*outs):
+        assert torch.equal(s1, s2)
+        assert torch.equal(o1, o2)
