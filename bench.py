@@ -391,7 +391,7 @@ def bench_prefill_extras(L, dev, K, W, peaks):
     return out
 
 
-# ------------------------------------------------------------ other layers ---# ------------------------------------------------------------ other layers ---
+# ------------------------------------------------------------ other layers ---
 
 def bench_hca_prefill(dev, K, W, peaks):
     import compressed_sparse_attention_11_b200 as csa
@@ -631,13 +631,37 @@ def run_profile_case(args):
     import dataclasses
     import compressed_sparse_attention_11_b200 as csa
     dev = torch.device("cuda", 0)
-    if args.profile in ("prefill", "hca"):
-        base = G.CSA_PREFILL if args.profile == "prefill" else G.HCA_PREFILL
+    if args.profile in ("prefill", "hca", "next"):
+        base = G.HCA_PREFILL if args.profile == "hca" else G.CSA_PREFILL
         w = dataclasses.replace(base, n=args.n) if args.n else base
         if args.profile == "prefill":
             L = CsaPrefill(w, dev)
             for _ in range(args.steps):
                 L.step()
+        elif args.profile == "next":
+            # the 'next' rows once per step: norm + RoPE layer, FP8 / bf16-score
+            # indexer, grouped output projection (V4-Flash shapes)
+            L = CsaPrefill(w, dev)
+            d = L.d
+            g = torch.Generator(device="cpu").manual_seed(7)
+            gam = (1.0 + 0.25 * torch.randn(w.c, generator=g)).to(dev)
+            win_n = torch.empty_like(d["kv_win"])
+            idx = torch.empty_like(L.idx)
+            kin = w.nh // 8 * w.c
+            w1 = (torch.randn(8, 1024, kin, generator=g) * kin ** -0.5).to(torch.bfloat16).to(dev)
+            w2 = (torch.randn(4096, 8192, generator=g) * 8192 ** -0.5).to(torch.bfloat16).to(dev)
+            y = torch.empty((1, w.n, 4096), dtype=torch.bfloat16, device=dev)
+            for _ in range(args.steps):
+                csa.csa_compress_norm_rope(d["ca"], d["cb"], d["za"], d["zb"], d["ba"], d["bb"],
+                                           w.m, gam, out=L.kv)
+                csa.csa_compress(d["ica"], d["icb"], d["iza"], d["izb"], d["iba"], d["ibb"], w.m,
+                                 out=L.ki)
+                csa.csa_index_topk_lowp(d["q_i"], d["w_i"], L.ki, w.m, w.k, fp8_qk=True,
+                                        bf16_scores=True, out=idx)
+                csa.csa_norm_rope_rows(d["kv_win"], gam, out=win_n)
+                csa.csa_sparse_attn_norm_rope(d["q"], L.kv, idx, win_n, w.window, d["sink"],
+                                              w.scale, w.m, gam, out=L.out)
+                csa.csa_grouped_out_proj(L.out, w1, w2, out=y)
         else:
             d = {k: v.to(dev) for k, v in G.prefill_inputs(w).items()}
             for _ in range(args.steps):
@@ -668,9 +692,9 @@ def main():
     ap.add_argument("--impl", default="ours", choices=("ours", "reference"))
     ap.add_argument("--skip-extras", action="store_true", help="headline workload only")
     ap.add_argument("--skip-cpu", action="store_true", help="no oracle timing")
-    ap.add_argument("--profile", choices=("prefill", "hca", "decode_csa", "decode_mixed"),
+    ap.add_argument("--profile", choices=("prefill", "hca", "next", "decode_csa", "decode_mixed"),
                     help="run --steps steps of one workload (for a profiler) and exit")
-    ap.add_argument("--n", type=int, default=None, help="--profile prefill/hca: tokens")
+    ap.add_argument("--n", type=int, default=None, help="--profile prefill/hca/next: tokens")
     ap.add_argument("--batch", type=int, default=None, help="--profile decode_*: sequences")
     args = ap.parse_args()
     if args.impl == "reference":

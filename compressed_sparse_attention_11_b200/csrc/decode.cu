@@ -81,8 +81,9 @@ CacheView cache_view(const csa_cache_desc& d, void* cache, const csa_paging* pg)
 // code = E4M3(x / scale), round to nearest even, saturating; trailing
 // rope_dims dims as bf16.  `x` is in shared memory; called by all threads.
 // ---------------------------------------------------------------------------
-__device__ void quantize_store(const float* x, int c, int rope, uint8_t* codes, float* scale_out,
-                               __nv_bfloat16* rope_out, float* red) {
+__device__ __noinline__ void quantize_store(const float* x, int c, int rope, uint8_t* codes,
+                                            float* scale_out, __nv_bfloat16* rope_out,
+                                            float* red) {
   const int body = c - rope;
   float amax = 0.f;
   for (int d = threadIdx.x; d < body; d += blockDim.x) amax = fmaxf(amax, fabsf(x[d]));
@@ -196,49 +197,30 @@ cudaError_t launch_write_rows(const csa_cache_desc& d, const CacheView& cv, int6
 // Per-dim softmax over the state rows of entry i (dims d of a `dim`-wide
 // stream set).  CSA: own block (parity i%2, streams ca/za) and, for i > 0, the
 // previous block (parity (i-1)%2, streams cb/zb).  HCA: streams C/Z.  The
-// rows are loaded sixteen at a time (CSA: all 2m at once) before they are
-// folded in, so a block of rows costs one memory latency, not one per row.
-__device__ float emit_dim(const __nv_bfloat16* st, int64_t b, int64_t i, int m, int dim, int d,
-                          const float* ba, const float* bb, bool hca) {
+// rows are loaded eight at a time before they are folded in, so a block of
+// rows costs one memory latency, not one per row.  (Out of line and rolled,
+// like quantize_store: the emission runs once per entry, so its code is
+// fetched about once per launch and its size is what it costs.)
+__device__ __noinline__ float emit_dim(const __nv_bfloat16* st, int64_t b, int64_t i, int m,
+                                       int dim, int d, const float* ba, const float* bb,
+                                       bool hca) {
   float M = kNegInf, S = 0.f, A = 0.f;
-  if (!hca && m <= 8) {  // CSA: both blocks' 2m rows and biases in flight at once
-    const int64_t pa = i & 1, pb = (i - 1) & 1;
-    auto blk = [&](int64_t par, int s) { return st + ((b * 2 + par) * 4 + s) * (int64_t)m * dim; };
-    const __nv_bfloat16 *ca = blk(pa, 0), *za = blk(pa, 2), *cb = blk(pb, 1), *zb = blk(pb, 3);
-    float cv[16], zv[16];
+  auto fold = [&](const __nv_bfloat16* cp, const __nv_bfloat16* zp, const float* bias) {
+#pragma unroll 1
+    for (int j0 = 0; j0 < m; j0 += 8) {
+      float cval[8], zval[8];
 #pragma unroll
-    for (int j = 0; j < 8; ++j) {
-      cv[j] = cv[8 + j] = 0.f;
-      zv[j] = zv[8 + j] = kNegInf;
-      if (j < m) {
-        cv[j] = __bfloat162float(ca[(int64_t)j * dim + d]);
-        zv[j] = __bfloat162float(za[(int64_t)j * dim + d]) + ba[(int64_t)j * dim + d];
-        if (i > 0) {
-          cv[8 + j] = __bfloat162float(cb[(int64_t)j * dim + d]);
-          zv[8 + j] = __bfloat162float(zb[(int64_t)j * dim + d]) + bb[(int64_t)j * dim + d];
-        }
-      }
-    }
-#pragma unroll
-    for (int j = 0; j < 16; ++j)
-      if ((j & 7) < m && (j < 8 || i > 0)) osm_update(M, S, A, zv[j], cv[j]);
-    return A / S;
-  }
-  auto fold = [&](const __nv_bfloat16* cb, const __nv_bfloat16* zb, const float* bias) {
-    for (int j0 = 0; j0 < m; j0 += 16) {
-      float cval[16], zval[16];
-#pragma unroll
-      for (int q = 0; q < 16; ++q) {
-        const int64_t j = j0 + q;
+      for (int q = 0; q < 8; ++q) {
         cval[q] = 0.f;
         zval[q] = kNegInf;
-        if (j < m) {
-          cval[q] = __bfloat162float(cb[j * dim + d]);
-          zval[q] = __bfloat162float(zb[j * dim + d]) + bias[j * dim + d];
+        if (j0 + q < m) {
+          const int64_t o = (int64_t)(j0 + q) * dim + d;
+          cval[q] = __bfloat162float(cp[o]);
+          zval[q] = __bfloat162float(zp[o]) + bias[o];
         }
       }
 #pragma unroll
-      for (int q = 0; q < 16; ++q)
+      for (int q = 0; q < 8; ++q)
         if (j0 + q < m) osm_update(M, S, A, zval[q], cval[q]);
     }
   };
@@ -246,10 +228,9 @@ __device__ float emit_dim(const __nv_bfloat16* st, int64_t b, int64_t i, int m, 
     const __nv_bfloat16* base = st + b * 2 * (int64_t)m * dim;
     fold(base, base + (int64_t)m * dim, ba);
   } else {
-    const int64_t pa = i & 1, pb = (i - 1) & 1;
     auto blk = [&](int64_t par, int s) { return st + ((b * 2 + par) * 4 + s) * (int64_t)m * dim; };
-    fold(blk(pa, 0), blk(pa, 2), ba);
-    if (i > 0) fold(blk(pb, 1), blk(pb, 3), bb);
+    fold(blk(i & 1, 0), blk(i & 1, 2), ba);
+    if (i > 0) fold(blk((i - 1) & 1, 1), blk((i - 1) & 1, 3), bb);
   }
   return A / S;
 }
@@ -398,11 +379,14 @@ __global__ void __launch_bounds__(1024) append_emit_kernel(csa_cache_desc d, Cac
   __syncthreads();                 // the rows just written are read back below
   const int64_t i = t / d.m;
   if (i >= d.capacity) return;
-  for (int e = threadIdx.x; e < d.c; e += blockDim.x)
-    sx[e] = emit_dim(cv.state, b, i, d.m, d.c, e, p.ba, p.bb, d.is_hca);
-  if (!d.is_hca)
-    for (int e = threadIdx.x; e < d.c_i; e += blockDim.x)
-      sx[d.c + e] = emit_dim(cv.istate, b, i, d.m, d.c_i, e, p.iba, p.ibb, false);
+  // one dim of the entry, or of the index key after it, per thread and round
+  const int ndim = d.c + (d.is_hca ? 0 : d.c_i);
+#pragma unroll 1
+  for (int e = threadIdx.x; e < ndim; e += blockDim.x) {
+    const bool key = e >= d.c;
+    sx[e] = emit_dim(key ? cv.istate : cv.state, b, i, d.m, key ? d.c_i : d.c, key ? e - d.c : e,
+                     key ? p.iba : p.ba, key ? p.ibb : p.bb, d.is_hca);
+  }
   __syncthreads();
   float* red = sx + d.c + (d.is_hca ? 0 : d.c_i);
   const int64_t es = entry_row(cv, b, i, d.capacity);

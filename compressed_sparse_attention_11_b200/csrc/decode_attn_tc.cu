@@ -10,12 +10,12 @@
 // E_t is cut into 128-entry tiles and each sequence's tiles into `nsplit`
 // contiguous ranges, one CTA per range (about one CTA per SM over the
 // batch).  In a CTA:
-//   * every warp but the MMA warp gathers: each thread owns one 16-dim
-//     quarter of one 64-dim slab for up to 12 rows of the tile, issues all of
-//     its loads at once (the FP8 codes of a row are 448 contiguous bytes, the
-//     RoPE dims and window rows 1 KB of bf16), then dequantises (code * scale)
-//     into the 128-byte-swizzled bf16 slab once the previous tile's P.V has
-//     released that slab;
+//   * the eight softmax warps also gather: each thread owns one 16-dim
+//     quarter of one 64-dim slab for 16 rows of the tile; once the
+//     previous tile's P.V has released that slab it copies the rows' bytes
+//     there by cp.async (the FP8 codes of a row are 448 contiguous bytes, the
+//     RoPE dims and window rows 1 KB of bf16) and widens the FP8 quarters in
+//     place (code * scale -> bf16, 128-byte swizzle);
 //   * S^T = K Q^T (M = 128 entries, N = 64 heads), the eight softmax warps
 //     keep a running max per head (moved, with O^T rescaled in TMEM, only
 //     when a tile's max exceeds it by more than 2^8) and write P^T in bf16;
@@ -41,10 +41,10 @@ constexpr int kSlabs = kC / 64;                // 64-dim slabs; slab 7 holds the
 constexpr int kSlabBytes = kTE * 128;          // 16 KB
 constexpr int kQSlabBytes = kNH * 128;         // 8 KB
 constexpr int kSoftWarps = 8;
-constexpr int kMmaWarp = 11;
-constexpr int kThreads = (kMmaWarp + 1) * 32;  // 384
-constexpr int kGatherThreads = kMmaWarp * 32;  // 352: every warp but the MMA warp
-constexpr int kRowsPerThread = (kTE + kMmaWarp - 1) / kMmaWarp;  // 12
+constexpr int kMmaWarp = 8;
+constexpr int kThreads = (kMmaWarp + 1) * 32;  // 288
+constexpr int kGatherThreads = kMmaWarp * 32;  // 256: the softmax warps gather too
+constexpr int kRowsPerThread = (kTE + kMmaWarp - 1) / kMmaWarp;  // 16
 constexpr int kMaxSelDec = 1024;
 constexpr float kRescaleLog2 = 8.f;
 static_assert(kGatherThreads % 32 == 0, "a thread keeps one slab quarter for every row");
@@ -64,7 +64,14 @@ constexpr int OFF_P = OFF_KV + kSlabs * kSlabBytes;     // 196608
 constexpr int OFF_LIST = OFF_P + kTE * 128;             // 212992
 constexpr int OFF_RED = OFF_LIST + kMaxSelDec * 4;      // [2 (max,sum)][2 hh][4 quad][32]
 constexpr int OFF_SCAN = OFF_RED + 2 * 2 * 4 * 32 * 4;  // [12] warp counts
-constexpr int OFF_BAR = OFF_SCAN + 64;
+constexpr int OFF_BM = OFF_SCAN + 64;                   // selection bitmap, 1 bit per entry
+// The selection stages the scores in the Q and KV slabs (192 KB): kSelScores
+// floats, then the bitmap of the threshold bin's entries (kSelWords words).
+constexpr int kSelStage = 49152;
+constexpr int kSelWords = kSelStage / 32;
+constexpr int kSelScores = kSelStage - kSelWords;
+constexpr int OFF_SCALE = OFF_BM + kSelWords * 4;        // [128] FP8 scales of a tile's rows
+constexpr int OFF_BAR = OFF_SCALE + kTE * 4;
 constexpr int SMEM = OFF_BAR + (int)sizeof(DecAttnBars) + 1024;
 static_assert(SMEM <= 232448, "shared memory budget");
 
@@ -90,14 +97,15 @@ __device__ __forceinline__ void dequant16(const uint4 c8, float sc, uint4& lo, u
 // The selection step inside the attention kernel (the top-k of section 4.2 of
 // "DeepSeek-V4: million-token context"; larger score first, ties to the
 // smaller index): the indexer left a histogram of the sequence's scores over
-// the top 12 bits of their order keys, which fixes the first radix digit
-// without a pass; the scores then land in shared memory as order keys (one
-// pass from L2) and two more digits (bits 19..8, then 7..0) are refined over
-// the keys of the threshold bin only, when its count does not settle the cut.
-// The chosen indices are emitted in ascending order by contiguous per-thread
-// segments.  Every thread of the CTA calls it; returns min(k, V).
+// the top 12 bits of their order keys, which gives the bin T holding the k-th
+// largest score, the count G above it and the count C in it.  The scores land
+// in shared memory by cp.async; one pass then marks, by warp ballots (one
+// 32-entry word each), the scores above bin T in the selection bitmap and
+// those in bin T in a candidate bitmap; the need = k - G largest candidates
+// (two more radix digits of the key, then the smaller indices among equal
+// keys) join the selection, and the chosen indices are emitted in ascending
+// order from the bitmap.  Every thread of the CTA calls it; returns min(k, V).
 // ---------------------------------------------------------------------------
-constexpr int kSelStage = 49152;  // keys staged in shared memory (192 KB)
 constexpr int kSelBins = 4096;
 
 struct SelState {
@@ -106,13 +114,14 @@ struct SelState {
 
 // The bin T (among `nbins`, counts in h, bin nbins - 1 highest) where the
 // count from the top reaches `need`, with the count above it (G) and in it.
-__device__ __forceinline__ void sel_find_bin(const uint32_t* h, int nbins, uint32_t need,
-                                             int* wsum, SelState* st) {
+__device__ __noinline__ void sel_find_bin(const uint32_t* h, int nbins, uint32_t need,
+                                          int* wsum, SelState* st) {
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  constexpr int kPerMax = (kSelBins + kThreads - 1) / kThreads;
   const int per = (nbins + kThreads - 1) / kThreads;
-  uint32_t c[(kSelBins + kThreads - 1) / kThreads], loc = 0;
+  uint32_t c[kPerMax], loc = 0;
 #pragma unroll
-  for (int j = 0; j < (kSelBins + kThreads - 1) / kThreads; ++j) {
+  for (int j = 0; j < kPerMax; ++j) {
     const int bin = nbins - 1 - (tid * per + j);
     c[j] = (j < per && bin >= 0) ? h[bin] : 0u;
     loc += c[j];
@@ -128,7 +137,7 @@ __device__ __forceinline__ void sel_find_bin(const uint32_t* h, int nbins, uint3
   uint32_t acc = inc - loc;
   for (int w = 0; w < warp; ++w) acc += (uint32_t)wsum[w];
 #pragma unroll
-  for (int j = 0; j < (kSelBins + kThreads - 1) / kThreads; ++j) {
+  for (int j = 0; j < kPerMax; ++j) {
     const int bin = nbins - 1 - (tid * per + j);
     if (j < per && bin >= 0 && acc < need && acc + c[j] >= need) {
       st->T = (uint32_t)bin;
@@ -140,89 +149,135 @@ __device__ __forceinline__ void sel_find_bin(const uint32_t* h, int nbins, uint3
   __syncthreads();
 }
 
+// Block-wide exclusive prefix of v.
+__device__ __forceinline__ uint32_t sel_excl(uint32_t v, int* wsum) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  uint32_t inc = v;
+#pragma unroll
+  for (int off = 1; off < 32; off <<= 1) {
+    const uint32_t x = __shfl_up_sync(0xffffffffu, inc, off);
+    if (lane >= off) inc += x;
+  }
+  if (lane == 31) wsum[warp] = (int)inc;
+  __syncthreads();
+  uint32_t a = inc - v;
+  for (int w = 0; w < warp; ++w) a += (uint32_t)wsum[w];
+  __syncthreads();
+  return a;
+}
+
 __device__ int fused_select(const float* __restrict__ row, const uint32_t* __restrict__ gh,
-                            int V, int k, uint32_t* skey, uint32_t* hist, int32_t* list,
-                            int* wsum, SelState* st) {
+                            int V, int k, float* stage, uint32_t* hist, uint32_t* bm,
+                            int32_t* list, int* wsum, SelState* st) {
+  using namespace sm100;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   if (V <= k) {
+#pragma unroll 1
     for (int i = tid; i < V; i += kThreads) list[i] = i;
     __syncthreads();
     return V;
   }
-  // the row into shared memory in one round trip (4-byte cp.async: rows are
-  // `capacity` floats apart, so not 16-byte aligned in general), then as
-  // order keys in place
-  for (int i = tid; i < V; i += kThreads)
-    asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(
-                     (uint32_t)__cvta_generic_to_shared(skey + i)),
-                 "l"(row + i)
-                 : "memory");
-  asm volatile("cp.async.commit_group;\n\tcp.async.wait_all;" ::: "memory");
-  __syncthreads();
-  for (int i = tid; i < V; i += kThreads) skey[i] = order_key(__uint_as_float(skey[i]));
-  // digit 1 (bits 31..20) from the indexer's histogram
-  for (int j = tid; j < kSelBins; j += kThreads) hist[j] = __ldcg(gh + j);
+  // the scores (as 16-byte chunks from the row's 16-byte-aligned start: a
+  // chunk holding any score of the row never crosses a page) and the
+  // histogram, in one round trip
+  const int r0 = (int)((reinterpret_cast<uintptr_t>(row) >> 2) & 3);
+  const float* abase = row - r0;
+  const int nchunk = (V + r0 + 3) >> 2;
+  const uint32_t sk = smem_u32(stage), sh = smem_u32(hist);
+#pragma unroll 1
+  for (int c = tid; c < nchunk; c += kThreads) cp_async_16(sk + 16u * c, abase + 4 * c);
+#pragma unroll 1
+  for (int c = tid; c < kSelBins / 4; c += kThreads) cp_async_16(sh + 16u * c, gh + 4 * c);
+  cp_async_wait_all();
   if (tid == 0) *st = SelState{0u, 0u, 0u};  // (a histogram short of k: a capped result)
   __syncthreads();
   sel_find_bin(hist, kSelBins, (uint32_t)k, wsum, st);
+  const uint32_t T = st->T;
   uint32_t need = (uint32_t)k - st->G;
-  uint32_t prefix = st->T << 20, mask = 0xfff00000u;
-  bool all_eq = st->C == need;
-  // digits 2 (bits 19..8, 4096 bins) and 3 (bits 7..0, 256 bins), over the
-  // keys that share the prefix, while the threshold bin does not settle it
-  for (int lvl = 0; lvl < 2 && !all_eq; ++lvl) {
-    const int shift = lvl == 0 ? 8 : 0;
-    const int nb = lvl == 0 ? 4096 : 256;
-    for (int j = tid; j < nb; j += kThreads) hist[j] = 0u;
-    __syncthreads();
-    for (int i = tid; i < V; i += kThreads) {
-      const uint32_t ky = skey[i];
-      if ((ky & mask) == prefix) atomicAdd(&hist[(ky >> shift) & (uint32_t)(nb - 1)], 1u);
+  const bool all_of_T = st->C == need;
+  const float* sc = stage + r0;  // score i at sc[i]
+  uint32_t* cbm = reinterpret_cast<uint32_t*>(stage + kSelScores);
+  const int nwords = (V + 31) >> 5;
+  // one pass: "above bin T" (or "in or above" when bin T is taken whole) and
+  // "in bin T", one word per warp ballot
+#pragma unroll 1
+  for (int w = warp; w < nwords; w += kThreads / 32) {
+    const int i = w * 32 + lane;
+    const uint32_t bin = i < V ? order_key(sc[i]) >> 20 : 0u;
+    const bool in = i < V && bin == T;
+    const uint32_t above = __ballot_sync(0xffffffffu, i < V && (bin > T || (all_of_T && in)));
+    const uint32_t cand = __ballot_sync(0xffffffffu, in && !all_of_T);
+    if (lane == 0) {
+      bm[w] = above;
+      cbm[w] = cand;
     }
-    __syncthreads();
-    sel_find_bin(hist, nb, need, wsum, st);
-    need -= st->G;
-    prefix |= st->T << shift;
-    mask |= (uint32_t)(nb - 1) << shift;
-    all_eq = st->C == need;
   }
-  // emit: key above the prefix, or equal to it (all of them, or the first
-  // `need` in index order); contiguous segments per thread keep the order
-  const int per = (V + kThreads - 1) / kThreads;
-  const int lo = min(V, tid * per), hi = min(V, lo + per);
-  uint32_t gt = 0, eq = 0;
-  for (int i = lo; i < hi; ++i) {
-    const uint32_t km = skey[i] & mask;
-    gt += km > prefix ? 1u : 0u;
-    eq += km == prefix ? 1u : 0u;
-  }
-  // exclusive prefix of eq, then of the taken counts
-  auto excl = [&](uint32_t v) -> uint32_t {
-    uint32_t inc = v;
-#pragma unroll
-    for (int off = 1; off < 32; off <<= 1) {
-      const uint32_t x = __shfl_up_sync(0xffffffffu, inc, off);
-      if (lane >= off) inc += x;
+  __syncthreads();
+  // thread tid owns words [w0, w1) from here on
+  const int per = (nwords + kThreads - 1) / kThreads;
+  const int w0 = min(nwords, tid * per), w1 = min(nwords, w0 + per);
+  if (!all_of_T) {
+    // the need largest candidates by the value (key bits 19..0, then
+    // 65535 - index): radix digits of 11, 9, 8 and 8 bits until a digit's
+    // bin is taken whole (the values are unique, so the last one is)
+    auto val = [&](int i) -> uint64_t {
+      return ((uint64_t)(order_key(sc[i]) & 0xfffffu) << 16) | (uint64_t)(0xffffu - (uint32_t)i);
+    };
+    uint64_t pfx = 0, msk = 0;
+    bool settled = false;
+    constexpr int kShift[4] = {25, 16, 8, 0};
+    constexpr int kWidth[4] = {11, 9, 8, 8};
+#pragma unroll 1
+    for (int lvl = 0; lvl < 4 && !settled; ++lvl) {
+      const int shf = kShift[lvl], nb = 1 << kWidth[lvl];
+#pragma unroll 1
+      for (int j = tid; j < nb; j += kThreads) hist[j] = 0u;
+      __syncthreads();
+#pragma unroll 1
+      for (int w = w0; w < w1; ++w) {
+        uint32_t x = cbm[w];
+        while (x != 0u) {
+          const int i = w * 32 + __ffs(x) - 1;
+          x &= x - 1u;
+          const uint64_t v = val(i);
+          if ((v & msk) == pfx) atomicAdd(&hist[(uint32_t)(v >> shf) & (uint32_t)(nb - 1)], 1u);
+        }
+      }
+      __syncthreads();
+      sel_find_bin(hist, nb, need, wsum, st);
+      need -= st->G;
+      pfx |= (uint64_t)st->T << shf;
+      msk |= (uint64_t)(nb - 1) << shf;
+      settled = st->C == need;
     }
-    if (lane == 31) wsum[warp] = (int)inc;
-    __syncthreads();
-    uint32_t a = inc - v;
-    for (int w = 0; w < warp; ++w) a += (uint32_t)wsum[w];
-    __syncthreads();
-    return a;
-  };
-  const uint32_t eq_before = excl(eq);
-  const uint32_t take_eq = all_eq ? eq : (eq_before >= need ? 0u : min(eq, need - eq_before));
-  uint32_t o = excl(gt + take_eq);
-  uint32_t eq_seen = 0;
-  for (int i = lo; i < hi; ++i) {
-    const uint32_t km = skey[i] & mask;
-    const bool is_eq = km == prefix;
-    const bool take = km > prefix || (is_eq && eq_seen < take_eq);
-    eq_seen += is_eq ? 1u : 0u;
-    if (take && o < (uint32_t)k) list[o] = i;
-    o += take ? 1u : 0u;
+    // chosen candidates: above the prefix on the ranked bits, or equal to it
+#pragma unroll 1
+    for (int w = w0; w < w1; ++w) {
+      uint32_t x = cbm[w], take = 0u;
+      while (x != 0u) {
+        const int bit = __ffs(x) - 1;
+        x &= x - 1u;
+        if ((val(w * 32 + bit) & msk) >= pfx) take |= 1u << bit;
+      }
+      bm[w] |= take;
+    }
   }
+  // emit: the marked indices in ascending order
+  uint32_t cnt = 0;
+#pragma unroll 1
+  for (int w = w0; w < w1; ++w) cnt += (uint32_t)__popc(bm[w]);
+  uint32_t o = sel_excl(cnt, wsum);
+#pragma unroll 1
+  for (int w = w0; w < w1; ++w) {
+    uint32_t x = bm[w];
+    while (x != 0u) {
+      const int bit = __ffs(x) - 1;
+      x &= x - 1u;
+      if (o < (uint32_t)k) list[o] = w * 32 + bit;
+      ++o;
+    }
+  }
+  fence_proxy_async();  // the staged scores are overwritten by TMA next
   __syncthreads();
   return k;
 }
@@ -243,6 +298,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_attn_tc_kernel(
   int32_t* list = reinterpret_cast<int32_t*>(smem + OFF_LIST);
   float* red = reinterpret_cast<float*>(smem + OFF_RED);
   int* wcount = reinterpret_cast<int*>(smem + OFF_SCAN);
+  float* sScale = reinterpret_cast<float*>(smem + OFF_SCALE);
   DecAttnBars* bar = reinterpret_cast<DecAttnBars*>(smem + OFF_BAR);
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -252,6 +308,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_attn_tc_kernel(
   const int64_t pbase = (b * nsplit + split) * kNH;
 
   if (tid == 0) {
+#pragma unroll 1
     for (int s = 0; s < kSlabs; ++s) {
       mbar_init(&bar->slab_full[s], kGatherThreads / 8);  // 4 lanes per slab in each warp
       mbar_init(&bar->slab_empty[s], 1);
@@ -287,15 +344,17 @@ __global__ void __launch_bounds__(kThreads, 1) decode_attn_tc_kernel(
   if (scores != nullptr) {
     SelState* st = reinterpret_cast<SelState*>(red);
     nsel = fused_select(scores + b * cap, ghist + b * kSelBins, (int)V, k,
-                        reinterpret_cast<uint32_t*>(sQ), reinterpret_cast<uint32_t*>(sP), list,
-                        wcount, st);
+                        reinterpret_cast<float*>(sQ), reinterpret_cast<uint32_t*>(sP),
+                        reinterpret_cast<uint32_t*>(smem + OFF_BM), list, wcount, st);
     if (sel_out != nullptr && split == 0)
+#pragma unroll 1
       for (int j = tid; j < k; j += kThreads) sel_out[b * k + j] = j < nsel ? list[j] : -1;
   } else if (sel != nullptr) {
     const int32_t* row = sel + b * k;
     const int per = (k + kThreads - 1) / kThreads;
     const int lo = min(k, tid * per), hi = min(k, lo + per);
     int cnt = 0;
+#pragma unroll 1
     for (int j = lo; j < hi; ++j) cnt += (row[j] >= 0 && row[j] < V) ? 1 : 0;
     int inc = cnt;
 #pragma unroll
@@ -312,6 +371,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_attn_tc_kernel(
       nsel += wcount[w];
     }
     int p = base + inc - cnt;
+#pragma unroll 1
     for (int j = lo; j < hi; ++j)
       if (row[j] >= 0 && row[j] < V) list[p++] = row[j];
   } else {
@@ -333,52 +393,71 @@ __global__ void __launch_bounds__(kThreads, 1) decode_attn_tc_kernel(
   }
 
   // -------- gather of tile jt of the range by one thread -------------------------
-  // Thread tid owns 16-dim quarter q_me of slab s_me for rows warp + 11 i.
+  // Thread tid owns 16-dim quarter q_me of slab s_me for rows warp + 8 i.
+  // The bytes travel by cp.async straight into the slab (no registers held
+  // across the copy): a bf16 quarter (RoPE dims, window rows) lands in its two
+  // final 16-byte chunks; an FP8 quarter (16 codes) lands in the second of
+  // them and is widened in place once it has arrived (code * scale -> bf16
+  // into both chunks; only this thread touches them).
   const int s_me = (tid & 31) >> 2, q_me = tid & 3;
   auto gather_tile = [&](int jt) -> bool {
     const int tile = tile0 + jt;
-    // an FP8 row (a selected entry, body slab) keeps its scale in hi.x
     const bool body = s_me < kBody / 64;
-    uint4 lo[kRowsPerThread], hi[kRowsPerThread];
-#pragma unroll
-    for (int i = 0; i < kRowsPerThread; ++i) {  // every load in flight before any use
-      const int r = warp + kMmaWarp * i;
-      lo[i] = make_uint4(0, 0, 0, 0);
-      hi[i] = lo[i];
-      if (r >= kTE) continue;
-      const int slot = tile * kTE + r;
-      if (slot < nsel) {
-        const int64_t es = entry_row(cv, b, csa ? (int64_t)list[slot] : (int64_t)slot, cap);
-        if (es < 0) {
-          // no block for this entry: zeros
-        } else if (body) {
-          lo[i] = __ldcs(reinterpret_cast<const uint4*>(cv.entry_fp8 + es * kBody + s_me * 64 +
-                                                         q_me * 16));
-          hi[i].x = __float_as_uint(__ldcs(cv.entry_scale + es));
-        } else {
-          const uint4* p = reinterpret_cast<const uint4*>(cv.entry_rope + es * kRope + q_me * 16);
-          lo[i] = __ldcs(p);
-          hi[i] = __ldcs(p + 1);
+    // the slab is free once the previous tile's P.V chunk that reads it is done
+    const bool free_ok =
+        jt == 0 || mbar_wait_small(&bar->slab_empty[s_me], (uint32_t)((jt - 1) & 1), err);
+    const uint32_t dst = smem_u32(sKV) + (uint32_t)(s_me * kSlabBytes);
+    if (free_ok) {
+#pragma unroll 2
+      for (int i = 0; i < kRowsPerThread; ++i) {
+        const int r = warp + kMmaWarp * i;
+        const int slot = tile * kTE + r;
+        const uint32_t d0 = dst + (uint32_t)(r * 128 + (((2 * q_me) ^ (r & 7)) * 16));
+        const uint32_t d1 = d0 ^ 16u;  // chunks 2 q and 2 q + 1 differ in bit 4 only
+        const int64_t es =
+            slot < nsel ? entry_row(cv, b, csa ? (int64_t)list[slot] : (int64_t)slot, cap) : -1;
+        if (es >= 0) {
+          if (body) {
+            cp_async_16(d1, cv.entry_fp8 + es * kBody + s_me * 64 + q_me * 16);
+            if (lane == 0)  // the row's scale, for every thread of the row
+              asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(
+                               smem_u32(sScale + r)),
+                           "l"(cv.entry_scale + es)
+                           : "memory");
+          } else {
+            const __nv_bfloat16* p = cv.entry_rope + es * kRope + q_me * 16;
+            cp_async_16(d0, p);
+            cp_async_16(d1, p + 8);
+          }
+        } else if (slot >= nsel && slot < N) {
+          const int64_t u = w0 + (slot - nsel);
+          const __nv_bfloat16* p =
+              cv.window + (b * window + u % window) * kC + s_me * 64 + q_me * 16;
+          cp_async_16(d0, p);
+          cp_async_16(d1, p + 8);
+        } else {  // past the end, or an entry without a block: zeros
+          st_shared_v4(d0, make_uint4(0, 0, 0, 0));
+          st_shared_v4(d1, make_uint4(0, 0, 0, 0));
+          if (lane == 0) sScale[r] = 0.f;
         }
-      } else if (slot < N) {
-        const int64_t u = w0 + (slot - nsel);
-        const uint4* p = reinterpret_cast<const uint4*>(
-            cv.window + (b * window + u % window) * kC + s_me * 64 + q_me * 16);
-        lo[i] = __ldcs(p);
-        hi[i] = __ldcs(p + 1);
       }
     }
-    // the slab is free once the previous tile's P.V chunk that reads it is done
-    if (jt >= 1 && !mbar_wait(&bar->slab_empty[s_me], (uint32_t)((jt - 1) & 1), err)) return false;
-    uint8_t* dst = sKV + s_me * kSlabBytes;
-#pragma unroll
-    for (int i = 0; i < kRowsPerThread; ++i) {
-      const int r = warp + kMmaWarp * i;
-      if (r >= kTE) continue;
-      uint4 a = lo[i], c = hi[i];
-      if (body && tile * kTE + r < nsel) dequant16(lo[i], __uint_as_float(hi[i].x), a, c);
-      *reinterpret_cast<uint4*>(dst + r * 128 + (((2 * q_me) ^ (r & 7)) * 16)) = a;
-      *reinterpret_cast<uint4*>(dst + r * 128 + (((2 * q_me + 1) ^ (r & 7)) * 16)) = c;
+    cp_async_wait_all();
+    // every gather thread's copies (the scales included) have landed; a
+    // failed wait anywhere stops them all here
+    if (named_bar_or(1, kGatherThreads, !free_ok)) return false;
+    if (body) {
+#pragma unroll 2
+      for (int i = 0; i < kRowsPerThread; ++i) {
+        const int r = warp + kMmaWarp * i;
+        if (tile * kTE + r >= nsel) continue;
+        const uint32_t d0 = dst + (uint32_t)(r * 128 + (((2 * q_me) ^ (r & 7)) * 16));
+        const uint32_t d1 = d0 ^ 16u;
+        uint4 a, c;
+        dequant16(ld_shared_v4(d1), sScale[r], a, c);
+        st_shared_v4(d0, a);
+        st_shared_v4(d1, c);
+      }
     }
     fence_proxy_async();  // generic-proxy writes before the tensor core reads them
     mbar_arrive(&bar->slab_full[s_me]);
@@ -397,14 +476,15 @@ __global__ void __launch_bounds__(kThreads, 1) decode_attn_tc_kernel(
           tma_load_3d(sQ + s * kQSlabBytes, &tm_q, &bar->q_full, s * 64, 0, (int)b);
       }
       __syncwarp();
-      bool ok = mbar_wait(&bar->q_full, 0, err);
+      bool ok = mbar_wait_small(&bar->q_full, 0, err);
       int issued = 0;  // tiles whose P.V was issued
       for (int jt = 0; jt < ntile && ok; ++jt) {
         for (int s = 0; s < kSlabs && ok; ++s)
-          ok = mbar_wait(&bar->slab_full[s], (uint32_t)(jt & 1), err);
+          ok = mbar_wait_small(&bar->slab_full[s], (uint32_t)(jt & 1), err);
         if (!ok) break;
         tc_fence_after();
         if (lane == 0) {
+#pragma unroll 1
           for (int s = 0; s < kSlabs; ++s)
 #pragma unroll
             for (int kk = 0; kk < 4; ++kk)
@@ -413,9 +493,10 @@ __global__ void __launch_bounds__(kThreads, 1) decode_attn_tc_kernel(
           mma_commit(&bar->s_full);
         }
         __syncwarp();
-        if (!(ok = mbar_wait(&bar->p_full, (uint32_t)(jt & 1), err))) break;
+        if (!(ok = mbar_wait_small(&bar->p_full, (uint32_t)(jt & 1), err))) break;
         tc_fence_after();
         if (lane == 0) {
+#pragma unroll 1
           for (int c = 0; c < 4; ++c) {
 #pragma unroll
             for (int kk = 0; kk < kTE / 16; ++kk)
@@ -433,12 +514,11 @@ __global__ void __launch_bounds__(kThreads, 1) decode_attn_tc_kernel(
       }
       if (lane == 0) mma_commit(&bar->o_full);
       __syncwarp();
-      mbar_wait(&bar->o_full, 0, err, false);  // every MMA done before TMEM is released
-      if (!ok && issued == 0) mbar_wait(&bar->q_full, 0, err, false);  // the Q load has landed
+      mbar_wait_small(&bar->o_full, 0, err, false);  // every MMA done before TMEM is released
+      if (!ok && issued == 0) mbar_wait_small(&bar->q_full, 0, err, false);  // the Q load has landed
     }
   } else if (live) {
-    // -------- gather (every warp here), softmax and epilogue (warps 0-7) ----------
-    const bool soft = warp < kSoftWarps;
+    // -------- gather, softmax and epilogue (warps 0-7) ------------------------------
     const int quad = warp & 3, hh = (warp >> 2) & 1;
     const int row = quad * 32 + lane;  // entry row within a tile / dim within a chunk
     const uint32_t lane_base = tmem + ((uint32_t)(quad * 32) << 16);
@@ -446,14 +526,11 @@ __global__ void __launch_bounds__(kThreads, 1) decode_attn_tc_kernel(
     const float qscale = scale * kLog2e;
     uint32_t gphase = 0;
     float m_run = kNegInf;  // lane i: running max (log2 units) of head hh*32+i
-    float psum[32];
-#pragma unroll
-    for (int i = 0; i < 32; ++i) psum[i] = 0.f;
+    float lsum = 0.f;       // lane i: its head's sum of P over this warp's rows
     bool ok = true;
     for (int jt = 0; jt < ntile && ok; ++jt) {
       if (!(ok = gather_tile(jt))) break;
-      if (!soft) continue;
-      if (!(ok = mbar_wait(&bar->s_full, (uint32_t)(jt & 1), err))) break;
+      if (!(ok = mbar_wait_small(&bar->s_full, (uint32_t)(jt & 1), err))) break;
       tc_fence_after();
       const bool valid = (tile0 + jt) * kTE + row < N;
       float v[32];
@@ -481,15 +558,16 @@ __global__ void __launch_bounds__(kThreads, 1) decode_attn_tc_kernel(
       // rmax is rewritten next tile only after every warp of the group has read it
       if (!(ok = group_sync(&bar->grp[hh], gphase, err))) break;
       // P^T (and, for a rescale, O^T) is free once the previous P.V is done
-      if (jt >= 1 && !(ok = mbar_wait(&bar->p_empty, (uint32_t)((jt - 1) & 1), err))) break;
+      if (jt >= 1 && !(ok = mbar_wait_small(&bar->p_empty, (uint32_t)((jt - 1) & 1), err))) break;
       tc_fence_after();
       if (__any_sync(0xffffffffu, resc)) {
         float f[32];
 #pragma unroll
         for (int i = 0; i < 32; ++i) {
           f[i] = __shfl_sync(0xffffffffu, f_lane, i);
-          psum[i] *= f[i];
         }
+        lsum *= f_lane;
+#pragma unroll 1
         for (int c = 0; c < 4; ++c) {
           uint32_t o[32];
           tmem_ld32(lane_base + kColO + c * kNH + hh * 32, o);
@@ -504,6 +582,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_attn_tc_kernel(
       tmem_ld32(s_addr, r);
       tmem_ld_wait();
       uint32_t pk[16];
+      float ps[32];  // this tile's P of the thread's entry row, per head
 #pragma unroll
       for (int i = 0; i < 32; i += 2) {
         float ma = __shfl_sync(0xffffffffu, m_run, i);
@@ -513,8 +592,8 @@ __global__ void __launch_bounds__(kThreads, 1) decode_attn_tc_kernel(
         const float la = valid ? __uint_as_float(r[i]) * qscale : kNegInf;
         const float lb = valid ? __uint_as_float(r[i + 1]) * qscale : kNegInf;
         const float pa = ex2(la - ma), pb = ex2(lb - mb);
-        psum[i] += pa;
-        psum[i + 1] += pb;
+        ps[i] = pa;
+        ps[i + 1] = pb;
         pk[i >> 1] = pack_bf16x2(pa, pb);
       }
       uint8_t* prow = sP + row * 128;
@@ -526,14 +605,14 @@ __global__ void __launch_bounds__(kThreads, 1) decode_attn_tc_kernel(
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&bar->p_full);
+      lsum += transpose_reduce<false>(ps);  // (after P is handed over)
     }
     // ---- epilogue: this range's O^T, max and sum (or, alone, the output) ----------
-    if (!soft) ok = false;
-    if (ok) ok = mbar_wait(&bar->o_full, 0, err);
+    if (ok) ok = mbar_wait_small(&bar->o_full, 0, err);
     if (ok) {
       tc_fence_after();
       float* rsum = red + (2 * 4 + hh * 4) * 32;
-      rsum[quad * 32 + lane] = transpose_reduce<false>(psum);
+      rsum[quad * 32 + lane] = lsum;
       ok = group_sync(&bar->grp[hh], gphase, err);
     }
     if (ok) {
@@ -549,6 +628,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_attn_tc_kernel(
         part_ms[(pbase + h) * 2 + 0] = m_run;
         part_ms[(pbase + h) * 2 + 1] = tot;
       }
+#pragma unroll 1
       for (int c = 0; c < 4; ++c) {
         uint32_t o[32];
         tmem_ld32(lane_base + kColO + c * kNH + hh * 32, o);
@@ -650,7 +730,7 @@ int decode_attn_splits(const csa_cache_desc& d) {
 }
 
 bool decode_attn_selects(const csa_cache_desc& d) {
-  return !d.is_hca && d.capacity <= kSelStage && d.k <= kMaxSelDec;
+  return !d.is_hca && d.capacity + 8 <= kSelScores && d.k <= kMaxSelDec;
 }
 
 cudaError_t launch_decode_attn_tc(const csa_cache_desc& d, const CacheView& cv,

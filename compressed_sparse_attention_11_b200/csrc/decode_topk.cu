@@ -34,7 +34,7 @@ constexpr int kSlice = kThreads * kPer;    // 4096 scores per CTA
 constexpr int kBins = kDecHistBins;        // 4096
 constexpr int kBinsPerThread = kBins / kThreads;  // 16
 constexpr int kSmemCand = 2048;            // threshold-bin candidates staged in shared memory
-constexpr int kSmemWords = 2048;           // bitmap words staged in shared memory (65536 entries)
+constexpr int kSmemWords = 8192;           // bitmap words staged in shared memory (262144 entries)
 static_assert(kBins % kThreads == 0 && kSlice % 32 == 0, "shapes");
 
 struct KeysInGlobal {
@@ -181,8 +181,11 @@ __global__ void __launch_bounds__(kThreads, 4) decode_topk_hist_kernel(
   const bool bm_smem = nwords <= kSmemWords;
   uint32_t* bmg = ws.bitmap + b * ws.words;
   uint32_t* bm = bm_smem ? dyn_bm : bmg;
-  if (bm_smem)
-    for (int64_t w = tid; w < nwords; w += kThreads) dyn_bm[w] = __ldcg(bmg + w);
+  if (bm_smem) {  // every load in flight at once (rows of words are 512-byte aligned)
+    const int nchunk = (int)((nwords + 3) / 4);
+    for (int c = tid; c < nchunk; c += kThreads)
+      sm100::cp_async_16(sm100::smem_u32(dyn_bm) + 16u * c, bmg + 4 * c);
+  }
 
   if (!all_of_T) {
     // the candidates of every slice, in index order, into one array: shared
@@ -214,17 +217,20 @@ __global__ void __launch_bounds__(kThreads, 4) decode_topk_hist_kernel(
       const uint32_t* ck = ws.cand_key + b * cap + (int64_t)q * kSlice;
       const int32_t* ci = ws.cand_idx + b * cap + (int64_t)q * kSlice;
       for (uint32_t i = lane; i < n; i += 32) {
-        const uint32_t kv = __ldcg(ck + i);
-        const int32_t iv = __ldcg(ci + i);
-        if (in_smem) {
-          cck[base + i] = kv;
-          cci[base + i] = iv;
+        if (in_smem) {  // 4-byte copies, all in flight
+          asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(sm100::smem_u32(cck + base + i)),
+                       "l"(ck + i)
+                       : "memory");
+          asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(sm100::smem_u32(cci + base + i)),
+                       "l"(ci + i)
+                       : "memory");
         } else {
-          __stcg(cck + base + i, kv);
-          __stcg(cci + base + i, iv);
+          __stcg(cck + base + i, __ldcg(ck + i));
+          __stcg(cci + base + i, __ldcg(ci + i));
         }
       }
     }
+    sm100::cp_async_wait_all();  // (the bitmap's copies too)
     __threadfence_block();
     __syncthreads();
     // the need largest of them (ties: the earlier position, i.e. the smaller
@@ -264,6 +270,7 @@ __global__ void __launch_bounds__(kThreads, 4) decode_topk_hist_kernel(
     }
     if (!bm_smem) __threadfence();
   }
+  sm100::cp_async_wait_all();
   __syncthreads();
 
   // 4. the chosen indices in ascending order, from the bitmap

@@ -77,6 +77,17 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, unsign
   }
   return true;
 }
+// The same wait with its spinning part out of line, for kernels that run
+// through their code about once per launch (their size is paid for in
+// instruction fetches; the call's register saves happen only when it spins).
+static __device__ __noinline__ bool mbar_wait_spin(uint64_t* bar, uint32_t parity,
+                                                   unsigned int* flag, bool abort_on_flag) {
+  return mbar_wait(bar, parity, flag, abort_on_flag);
+}
+__device__ __forceinline__ bool mbar_wait_small(uint64_t* bar, uint32_t parity,
+                                                unsigned int* flag, bool abort_on_flag = true) {
+  return mbar_try_wait(bar, parity) || mbar_wait_spin(bar, parity, flag, abort_on_flag);
+}
 
 // mbar_wait with an explicit limit (ns) and no early exit on the flag.
 __device__ __forceinline__ bool mbar_wait_limit(uint64_t* bar, uint32_t parity,
@@ -174,6 +185,28 @@ __device__ __forceinline__ void cp_async_16_hint(void* dst, const void* src, uin
                    smem_u32(dst)),
                "l"(src), "r"(bytes), "l"(policy)
                : "memory");
+}
+// Copies 16 bytes from global to shared address `dst` (L2 only, default
+// cache policy).
+__device__ __forceinline__ void cp_async_16(uint32_t dst, const void* src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
+}
+__device__ __forceinline__ void st_shared_v4(uint32_t a, uint4 v) {
+  asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(a), "r"(v.x), "r"(v.y), "r"(v.z),
+               "r"(v.w)
+               : "memory");
+}
+__device__ __forceinline__ uint4 ld_shared_v4(uint32_t a) {
+  uint4 v;
+  asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
+               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+               : "r"(a)
+               : "memory");
+  return v;
+}
+// Waits until every cp.async issued so far by this thread has landed.
+__device__ __forceinline__ void cp_async_wait_all() {
+  asm volatile("cp.async.commit_group;\n\tcp.async.wait_all;" ::: "memory");
 }
 // Arrives on `bar` (without raising its expected count) once every cp.async
 // issued so far by this thread has completed.

@@ -353,3 +353,42 @@ def test_paged_decode_bit_identical_to_contiguous():
     for (o1, s1), (o2, s2) in zip(*outs):
         assert torch.equal(s1, s2)
         assert torch.equal(o1, o2)
+
+
+@pytest.mark.parametrize("is_hca", [False, True])
+def test_decode_step_replays_in_a_cuda_graph(is_hca):
+    """A decode step captured in a CUDA graph (the launches of every kernel of
+    the step, with their programmatic dependencies) replays bit-identically
+    to the same step launched directly; the step is idempotent at a fixed
+    position, so the replay recomputes exactly what was computed."""
+    w = G.Decode("graph_decode", 2, 0, 512, 64, 128 if is_hca else 4, 64, 128, is_hca, nh_i=64,
+                 c_i=128, k=512, seed=117)
+    B, E, steps = 2, 40 if is_hca else 2100, 1
+    inp, cache, t0, first, tail, names = _setup(w, B, E, steps, 29)
+    biases = {k: v.to(DEV) for k, v in _biases(inp, w).items()}
+    rows = {nm: inp["rows_" + nm][:, tail].contiguous().to(DEV) for nm in names}
+    pos = torch.full((B,), t0, dtype=torch.int64, device=DEV)
+    sink, q = inp["sink"].to(DEV), inp["q"][0].to(DEV)
+    qi = None if is_hca else inp["q_i"][0].to(DEV)
+    wi = None if is_hca else inp["w_i"][0].to(DEV)
+    out = torch.empty_like(q)
+
+    def step():
+        cache.decode_step(pos, rows, biases, sink, w.scale, q, qi, wi, out=out)
+
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(side):
+        step()
+    torch.cuda.current_stream().wait_stream(side)
+    eager = host(out)
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        step()
+    out.zero_()
+    for _ in range(3):
+        g.replay()
+    torch.cuda.synchronize()
+    csa.csa_check()
+    assert torch.equal(host(out), eager)
+    del g
