@@ -194,45 +194,52 @@ cudaError_t launch_write_rows(const csa_cache_desc& d, const CacheView& cv, int6
 // ---------------------------------------------------------------------------
 // Step 1: append the token's rows and emit a finished entry.
 // ---------------------------------------------------------------------------
+// One block's rows of dim d folded into the online softmax state (M, S, A).
+__device__ __noinline__ void emit_fold(const __nv_bfloat16* cp, const __nv_bfloat16* zp,
+                                       const float* bias, int m, int dim, int d, float* state) {
+  float M = state[0], S = state[1], A = state[2];
+#pragma unroll 1
+  for (int j0 = 0; j0 < m; j0 += 4) {
+    float cval[4], zval[4];
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      cval[q] = 0.f;
+      zval[q] = kNegInf;
+      if (j0 + q < m) {
+        const int64_t o = (int64_t)(j0 + q) * dim + d;
+        cval[q] = __bfloat162float(cp[o]);
+        zval[q] = __bfloat162float(zp[o]) + bias[o];
+      }
+    }
+#pragma unroll
+    for (int q = 0; q < 4; ++q)
+      if (j0 + q < m) osm_update(M, S, A, zval[q], cval[q]);
+  }
+  state[0] = M;
+  state[1] = S;
+  state[2] = A;
+}
+
 // Per-dim softmax over the state rows of entry i (dims d of a `dim`-wide
 // stream set).  CSA: own block (parity i%2, streams ca/za) and, for i > 0, the
 // previous block (parity (i-1)%2, streams cb/zb).  HCA: streams C/Z.  The
-// rows are loaded eight at a time before they are folded in, so a block of
-// rows costs one memory latency, not one per row.  (Out of line and rolled,
+// rows are loaded four at a time before they are folded in, so a CSA block
+// of rows costs one memory latency, not one per row.  (Out of line and rolled,
 // like quantize_store: the emission runs once per entry, so its code is
 // fetched about once per launch and its size is what it costs.)
 __device__ __noinline__ float emit_dim(const __nv_bfloat16* st, int64_t b, int64_t i, int m,
                                        int dim, int d, const float* ba, const float* bb,
                                        bool hca) {
-  float M = kNegInf, S = 0.f, A = 0.f;
-  auto fold = [&](const __nv_bfloat16* cp, const __nv_bfloat16* zp, const float* bias) {
-#pragma unroll 1
-    for (int j0 = 0; j0 < m; j0 += 8) {
-      float cval[8], zval[8];
-#pragma unroll
-      for (int q = 0; q < 8; ++q) {
-        cval[q] = 0.f;
-        zval[q] = kNegInf;
-        if (j0 + q < m) {
-          const int64_t o = (int64_t)(j0 + q) * dim + d;
-          cval[q] = __bfloat162float(cp[o]);
-          zval[q] = __bfloat162float(zp[o]) + bias[o];
-        }
-      }
-#pragma unroll
-      for (int q = 0; q < 8; ++q)
-        if (j0 + q < m) osm_update(M, S, A, zval[q], cval[q]);
-    }
-  };
+  float state[3] = {kNegInf, 0.f, 0.f};
   if (hca) {
     const __nv_bfloat16* base = st + b * 2 * (int64_t)m * dim;
-    fold(base, base + (int64_t)m * dim, ba);
+    emit_fold(base, base + (int64_t)m * dim, ba, m, dim, d, state);
   } else {
     auto blk = [&](int64_t par, int s) { return st + ((b * 2 + par) * 4 + s) * (int64_t)m * dim; };
-    fold(blk(i & 1, 0), blk(i & 1, 2), ba);
-    if (i > 0) fold(blk((i - 1) & 1, 1), blk((i - 1) & 1, 3), bb);
+    emit_fold(blk(i & 1, 0), blk(i & 1, 2), ba, m, dim, d, state);
+    if (i > 0) emit_fold(blk((i - 1) & 1, 1), blk((i - 1) & 1, 3), bb, m, dim, d, state);
   }
-  return A / S;
+  return state[2] / state[1];
 }
 
 // The token's rows -- the window row and the compressor-state rows -- copied
@@ -354,7 +361,8 @@ __global__ void __launch_bounds__(1024) append_emit_kernel(csa_cache_desc d, Cac
                                                           const float* __restrict__ w_i,
                                                           uint8_t* __restrict__ qop,
                                                           uint32_t* __restrict__ ghist,
-                                                          uint32_t* __restrict__ sel_done) {
+                                                          uint32_t* __restrict__ sel_done,
+                                                          uint32_t* __restrict__ idx_done) {
   extern __shared__ float sx[];  // [c + c_i] + 32
   const int64_t b = blockIdx.x;
   // the previous step's kernels read the window slot this token overwrites
@@ -368,7 +376,10 @@ __global__ void __launch_bounds__(1024) append_emit_kernel(csa_cache_desc d, Cac
     if (ghist != nullptr) {
       uint4* gh = reinterpret_cast<uint4*>(ghist + b * kDecHistBins);
       for (int e = threadIdx.x; e < kDecHistBins / 4; e += blockDim.x) gh[e] = make_uint4(0, 0, 0, 0);
-      if (threadIdx.x == 0) sel_done[b] = 0u;
+      if (threadIdx.x == 0) {
+        sel_done[b] = 0u;
+        idx_done[b] = 0u;
+      }
     }
     return;
   }
@@ -742,7 +753,8 @@ cudaError_t launch_decode_step(const csa_cache_desc& d, const CacheView& cv, con
   cudaError_t err = launch_pdl(append_emit_kernel,
                                dim3((unsigned)d.batch, qop != nullptr ? 2u : 1u),
                                dim3(emit_threads), emit_smem, s, d, cv, pos, rows, p,
-                               (const __nv_bfloat16*)q_i, w_i, qop, sws.ghist, sws.done);
+                               (const __nv_bfloat16*)q_i, w_i, qop, sws.ghist, sws.done,
+                               sws.idx_done);
   if (err != cudaSuccess) return err;
   if (!d.is_hca && w.tc_index) {
     float* scores = p.scores_out != nullptr ? p.scores_out : reinterpret_cast<float*>(wb + w.scores);
@@ -750,7 +762,8 @@ cudaError_t launch_decode_step(const csa_cache_desc& d, const CacheView& cv, con
     if (flag == nullptr) return cudaErrorUnknown;
     // (sws.ghist is NULL when the selection below does not use it: the
     // indexer then keeps no histogram)
-    err = launch_decode_index_tc(d, cv, pos, qop, scores, sws.ghist, flag, s);
+    err = launch_decode_index_tc(d, cv, pos, qop, scores, sws.ghist,
+                                 w.attn_select ? sws.idx_done : nullptr, flag, s);
     if (err != cudaSuccess) return err;
     if (w.attn_select) {
       err = cudaSuccess;  // the attention kernel selects
@@ -784,7 +797,9 @@ cudaError_t launch_decode_step(const csa_cache_desc& d, const CacheView& cv, con
     return launch_decode_attn_tc(d, cv, pos, q, w.attn_select ? nullptr : sel, p.sink, p.scale,
                                  w.nsplit, out, part_o, part_ms, ascores,
                                  w.attn_select ? sws.ghist : nullptr,
-                                 w.attn_select ? p.sel_out : nullptr, flag, s);
+                                 w.attn_select ? p.sel_out : nullptr,
+                                 w.attn_select ? sws.idx_done : nullptr,
+                                 decode_index_tile_keys(d), flag, s);
   }
   const size_t asmem = sizeof(float) * ((size_t)kDecTE * (d.c + 1) + (size_t)kDecHG * d.c +
                                         kDecHG * kDecTE) + sizeof(int64_t) * kDecTE;

@@ -199,17 +199,32 @@ __device__ int fused_select(const float* __restrict__ row, const uint32_t* __res
   uint32_t* cbm = reinterpret_cast<uint32_t*>(stage + kSelScores);
   const int nwords = (V + 31) >> 5;
   // one pass: "above bin T" (or "in or above" when bin T is taken whole) and
-  // "in bin T", one word per warp ballot
+  // "in bin T".  A warp takes 128 scores a step, four per lane; each lane's
+  // four bits are OR-reduced over the eight lanes of a 32-score word.
+  const int nblk = (nwords + 3) >> 2;
 #pragma unroll 1
-  for (int w = warp; w < nwords; w += kThreads / 32) {
-    const int i = w * 32 + lane;
-    const uint32_t bin = i < V ? order_key(sc[i]) >> 20 : 0u;
-    const bool in = i < V && bin == T;
-    const uint32_t above = __ballot_sync(0xffffffffu, i < V && (bin > T || (all_of_T && in)));
-    const uint32_t cand = __ballot_sync(0xffffffffu, in && !all_of_T);
-    if (lane == 0) {
-      bm[w] = above;
-      cbm[w] = cand;
+  for (int q = warp; q < nblk; q += kThreads / 32) {
+    const int i0 = q * 128 + 4 * lane;
+    uint32_t ab = 0u, cd = 0u;
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const int i = i0 + e;
+      const uint32_t bin = i < V ? order_key(sc[i]) >> 20 : 0u;
+      const bool in = i < V && bin == T;
+      ab |= (i < V && (bin > T || (all_of_T && in)) ? 1u : 0u) << e;
+      cd |= (in && !all_of_T ? 1u : 0u) << e;
+    }
+    ab <<= 4 * (lane & 7);
+    cd <<= 4 * (lane & 7);
+#pragma unroll
+    for (int off = 1; off < 8; off <<= 1) {
+      ab |= __shfl_xor_sync(0xffffffffu, ab, off);
+      cd |= __shfl_xor_sync(0xffffffffu, cd, off);
+    }
+    const int w = q * 4 + (lane >> 3);
+    if ((lane & 7) == 0 && w < nwords) {
+      bm[w] = ab;
+      cbm[w] = cd;
     }
   }
   __syncthreads();
@@ -288,7 +303,8 @@ __global__ void __launch_bounds__(kThreads, 1) decode_attn_tc_kernel(
     int64_t cap, const float* __restrict__ sink, float scale, int nsplit,
     float* __restrict__ part_o, float* __restrict__ part_ms, __nv_bfloat16* __restrict__ out,
     const float* __restrict__ scores, const uint32_t* __restrict__ ghist,
-    int32_t* __restrict__ sel_out, unsigned int* __restrict__ err) {
+    int32_t* __restrict__ sel_out, const uint32_t* __restrict__ idx_done, int idx_tile,
+    unsigned int* __restrict__ err) {
   using namespace sm100;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = smem_raw + ((1024 - (smem_u32(smem_raw) & 1023)) & 1023);
@@ -327,10 +343,29 @@ __global__ void __launch_bounds__(kThreads, 1) decode_attn_tc_kernel(
     tmem_alloc(&bar->tmem_base, 512);
     tmem_relinquish();
   }
-  // set-up above; the selection and the cache are written by earlier kernels
-  pdl_wait();
+  // the window ring of the sequence (the rows of the range's last tile)
+  // starts moving into L2 under the wait: a prefetch changes no data
+  if (split == nsplit - 1 && tid == 0 && window <= 4096)
+    bulk_prefetch_l2(cv.window + b * window * kC, (uint32_t)window * kC * 2);
+  // set-up above; the selection and the cache are written by earlier kernels.
+  // Selecting here from the indexer's scores, the sequence's own tile count
+  // is awaited rather than the end of the indexer's grid, so a sequence
+  // starts as soon as its keys are scored (the cache itself was written
+  // before the indexer started)
+  if (scores != nullptr && idx_done != nullptr) {
+    if (tid == 0) {
+      const int64_t tp = pos[b];
+      const int64_t Vp = tp < 0 ? 0 : min((tp + 1) / m, cap);
+      const uint32_t want = (uint32_t)((Vp + idx_tile - 1) / idx_tile);
+      const bool ok = want == 0 || wait_count(idx_done + b, want, err);
+      bar->abort = ok ? flag_value(err) : 1u;
+    }
+    __syncthreads();  // nothing indexer-written is read before the count is complete
+  } else {
+    pdl_wait();
+    if (tid == 0) bar->abort = flag_value(err);
+  }
   pdl_trigger();
-  if (tid == 0) bar->abort = flag_value(err);
   const int64_t t = pos[b];
   const int64_t V = t < 0 ? 0 : min((t + 1) / m, cap);
   const int64_t w0 = max((int64_t)0, t - window + 1);
@@ -519,6 +554,23 @@ __global__ void __launch_bounds__(kThreads, 1) decode_attn_tc_kernel(
     }
   } else if (live) {
     // -------- gather, softmax and epilogue (warps 0-7) ------------------------------
+    // the rows of the range's later tiles start moving into L2 now (one bulk
+    // prefetch per piece), so that their gathers, which wait for the slabs,
+    // read L2 rather than HBM
+#pragma unroll 1
+    for (int slot = (tile0 + 1) * kTE + tid; slot < min(N, tile1 * kTE); slot += kGatherThreads) {
+      if (slot < nsel) {
+        const int64_t es = entry_row(cv, b, csa ? (int64_t)list[slot] : (int64_t)slot, cap);
+        if (es >= 0) {
+          bulk_prefetch_l2(cv.entry_fp8 + es * kBody, kBody);
+          bulk_prefetch_l2(cv.entry_rope + es * kRope, kRope * 2);
+          bulk_prefetch_l2(cv.entry_scale + (es & ~(int64_t)3), 16);
+        }
+      } else {
+        const int64_t u = w0 + (slot - nsel);
+        bulk_prefetch_l2(cv.window + (b * window + u % window) * kC, kC * 2);
+      }
+    }
     const int quad = warp & 3, hh = (warp >> 2) & 1;
     const int row = quad * 32 + lane;  // entry row within a tile / dim within a chunk
     const uint32_t lane_base = tmem + ((uint32_t)(quad * 32) << 16);
@@ -737,7 +789,8 @@ cudaError_t launch_decode_attn_tc(const csa_cache_desc& d, const CacheView& cv,
                                   const int64_t* pos, const void* q, const int32_t* sel,
                                   const float* sink, float scale, int nsplit, void* out,
                                   float* part_o, float* part_ms, const float* scores,
-                                  const uint32_t* ghist, int32_t* sel_out, unsigned int* err,
+                                  const uint32_t* ghist, int32_t* sel_out,
+                                  const uint32_t* idx_done, int idx_tile, unsigned int* err,
                                   cudaStream_t s) {
   CUtensorMap tq;
   if (!make_tmap_bf16_3d(&tq, q, kC, kNH, d.batch, kC * 2ull, (uint64_t)kNH * kC * 2, 64, kNH))
@@ -748,7 +801,7 @@ cudaError_t launch_decode_attn_tc(const csa_cache_desc& d, const CacheView& cv,
   e = launch_pdl(decode_attn_tc_kernel, dim3((unsigned)nsplit, (unsigned)d.batch), dim3(kThreads),
                  (size_t)SMEM, s, tq, cv, pos, d.is_hca ? nullptr : sel, (int)d.k, (int)d.window,
                  (int)d.m, (int64_t)d.capacity, sink, scale, nsplit, part_o, part_ms,
-                 (__nv_bfloat16*)out, scores, ghist, sel_out, err);
+                 (__nv_bfloat16*)out, scores, ghist, sel_out, idx_done, idx_tile, err);
   if (e != cudaSuccess || nsplit == 1) return e;
   return launch_pdl(decode_combine_kernel, dim3(kNH, (unsigned)d.batch), dim3(kC / 4), 0, s,
                     (const float*)part_o, (const float*)part_ms, sink, nsplit,

@@ -214,6 +214,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_index_tc_kernel(
     const __grid_constant__ CUtensorMap tm_keys, const float* __restrict__ key_scale,
     PagedKeys pk, const uint8_t* __restrict__ qop, const int64_t* __restrict__ pos, int64_t batch,
     int64_t cap, int m, float* __restrict__ scores, uint32_t* __restrict__ ghist,
+    uint32_t* __restrict__ idx_done,
     unsigned int* __restrict__ err) {
   using C = DecIdxCfg<H>;
   constexpr int S = C::STAGES;
@@ -411,11 +412,14 @@ __global__ void __launch_bounds__(kThreads, 1) decode_index_tc_kernel(
     // false once a wait of this warp gave up (the flag is set): from then on
     // nothing is awaited or written, but every barrier below is still reached
     bool alive = true;
+    int seq_tiles = 0;  // tiles of the current sequence in this CTA's range so far
     for (int i = 0; i < count; ++i, it.next(pos, batch, m, cap)) {
       if (i == 0 || it.j == 0) {
         ++u;
         V = min((pos[it.b] + 1) / m, cap);
+        seq_tiles = 0;
       }
+      ++seq_tiles;
       const bool seq_end = i + 1 == count || it.j + 1 == it.nt;
       if (mine_of(i)) {
         const float ks = ks_next;
@@ -473,6 +477,13 @@ __global__ void __launch_bounds__(kThreads, 1) decode_index_tc_kernel(
         if (lane == 0 && alive) mbar_arrive(&bar->w_empty[u % kWSlots]);
         alive = !named_bar_or(3, kEpiThreads, !alive);
         if (alive && ghist != nullptr) flush_hist(sHist, u & 1, ghist, it.b, etid);
+        if (idx_done != nullptr) {
+          // every score and histogram count of the sequence from this CTA is
+          // written and fenced before the CTA's tile count is published
+          __threadfence();
+          alive = !named_bar_or(3, kEpiThreads, !alive);
+          if (etid == 0 && alive) atomicAdd(idx_done + it.b, (uint32_t)seq_tiles);
+        }
       }
     }
   }
@@ -532,6 +543,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_index_sw_kernel(
     const __grid_constant__ CUtensorMap tm_keys, const float* __restrict__ key_scale,
     PagedKeys pk, const uint8_t* __restrict__ qop, const int64_t* __restrict__ pos, int64_t batch,
     int64_t cap, int m, float* __restrict__ scores, uint32_t* __restrict__ ghist,
+    uint32_t* __restrict__ idx_done,
     unsigned int* __restrict__ err) {
   constexpr int S = kSwStages;
   using namespace sm100;
@@ -702,11 +714,14 @@ __global__ void __launch_bounds__(kThreads, 1) decode_index_sw_kernel(
     // false once a wait of this group gave up (the flag is set): from then on
     // nothing is awaited or written, but every barrier below is still reached
     bool alive = true;
+    int seq_tiles = 0;  // tiles of the current sequence in this CTA's range so far
     for (int i = 0; i < count; ++i, it.next(pos, batch, m, cap)) {
       if (i == 0 || it.j == 0) {
         ++u;
         V = min((pos[it.b] + 1) / m, cap);
+        seq_tiles = 0;
       }
+      ++seq_tiles;
       const bool seq_end = i + 1 == count || it.j + 1 == it.nt;
       if ((i & 1) == grp) {
         // key scales of this thread's two keys, ahead of the accumulator
@@ -783,6 +798,13 @@ __global__ void __launch_bounds__(kThreads, 1) decode_index_sw_kernel(
         if (lane == 0 && alive) mbar_arrive(&bar->w_empty[u % kWSlots]);
         alive = !named_bar_or(3, kEpiThreads, !alive);
         if (alive && ghist != nullptr) flush_hist(sHist, u & 1, ghist, it.b, etid);
+        if (idx_done != nullptr) {
+          // every score and histogram count of the sequence from this CTA is
+          // written and fenced before the CTA's tile count is published
+          __threadfence();
+          alive = !named_bar_or(3, kEpiThreads, !alive);
+          if (etid == 0 && alive) atomicAdd(idx_done + it.b, (uint32_t)seq_tiles);
+        }
       }
     }
   }
@@ -813,8 +835,8 @@ bool key_map(const csa_cache_desc& d, const CacheView& cv, int tk, CUtensorMap* 
 }
 
 cudaError_t launch_sw(const csa_cache_desc& d, const CacheView& cv, const int64_t* pos,
-                      const uint8_t* qop, float* scores, uint32_t* ghist, unsigned int* err,
-                      cudaStream_t s) {
+                      const uint8_t* qop, float* scores, uint32_t* ghist, uint32_t* idx_done,
+                      unsigned int* err, cudaStream_t s) {
   CUtensorMap tk;
   PagedKeys pk;
   if (!key_map(d, cv, kSwKeys, &tk, &pk)) return cudaErrorInvalidValue;
@@ -825,13 +847,13 @@ cudaError_t launch_sw(const csa_cache_desc& d, const CacheView& cv, const int64_
   const unsigned grid = (unsigned)std::max<int64_t>(1, std::min<int64_t>(sm_count(), max_tiles));
   return launch_pdl(decode_index_sw_kernel, dim3(grid), dim3(kThreads), (size_t)kSwSmem, s, tk,
                     (const float*)cv.ikey_scale, pk, qop, pos, (int64_t)d.batch,
-                    (int64_t)d.capacity, d.m, scores, ghist, err);
+                    (int64_t)d.capacity, d.m, scores, ghist, idx_done, err);
 }
 
 template <int H>
 cudaError_t launch_h(const csa_cache_desc& d, const CacheView& cv, const int64_t* pos,
-                     const uint8_t* qop, float* scores, uint32_t* ghist, unsigned int* err,
-                     cudaStream_t s) {
+                     const uint8_t* qop, float* scores, uint32_t* ghist, uint32_t* idx_done,
+                     unsigned int* err, cudaStream_t s) {
   using C = DecIdxCfg<H>;
   CUtensorMap tk;
   PagedKeys pk;
@@ -843,7 +865,7 @@ cudaError_t launch_h(const csa_cache_desc& d, const CacheView& cv, const int64_t
   const unsigned grid = (unsigned)std::max<int64_t>(1, std::min<int64_t>(sm_count(), max_tiles));
   return launch_pdl(kern, dim3(grid), dim3(kThreads), (size_t)C::SMEM, s, tk,
                     (const float*)cv.ikey_scale, pk, qop, pos,
-                    (int64_t)d.batch, (int64_t)d.capacity, d.m, scores, ghist, err);
+                    (int64_t)d.batch, (int64_t)d.capacity, d.m, scores, ghist, idx_done, err);
 }
 
 }  // namespace
@@ -852,12 +874,15 @@ bool decode_index_tc_supported(const csa_cache_desc& d) {
   return !d.is_hca && d.c_i == kCI && (d.nh_i == 64 || d.nh_i == 128);
 }
 
+int decode_index_tile_keys(const csa_cache_desc& d) { return d.nh_i == 64 ? kSwKeys : kKeys; }
+
 cudaError_t launch_decode_index_tc(const csa_cache_desc& d, const CacheView& cv,
                                    const int64_t* pos, const uint8_t* qop, float* scores,
-                                   uint32_t* ghist, unsigned int* err, cudaStream_t s) {
+                                   uint32_t* ghist, uint32_t* idx_done, unsigned int* err,
+                                   cudaStream_t s) {
   switch (d.nh_i) {
-    case 64: return launch_sw(d, cv, pos, qop, scores, ghist, err, s);
-    case 128: return launch_h<128>(d, cv, pos, qop, scores, ghist, err, s);
+    case 64: return launch_sw(d, cv, pos, qop, scores, ghist, idx_done, err, s);
+    case 128: return launch_h<128>(d, cv, pos, qop, scores, ghist, idx_done, err, s);
     default: return cudaErrorInvalidValue;
   }
 }

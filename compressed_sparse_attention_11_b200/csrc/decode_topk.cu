@@ -34,7 +34,7 @@ constexpr int kSlice = kThreads * kPer;    // 4096 scores per CTA
 constexpr int kBins = kDecHistBins;        // 4096
 constexpr int kBinsPerThread = kBins / kThreads;  // 16
 constexpr int kSmemCand = 2048;            // threshold-bin candidates staged in shared memory
-constexpr int kSmemWords = 8192;           // bitmap words staged in shared memory (262144 entries)
+constexpr int kMaxSmemWords = 45056;       // bitmap words stageable in shared memory (1,441,792 entries)
 static_assert(kBins % kThreads == 0 && kSlice % 32 == 0, "shapes");
 
 struct KeysInGlobal {
@@ -73,9 +73,9 @@ __device__ __forceinline__ uint32_t block_excl_scan(uint32_t v, uint32_t* wsum, 
 
 __global__ void __launch_bounds__(kThreads, 4) decode_topk_hist_kernel(
     const int64_t* __restrict__ pos, int64_t cap, int m, int k, const float* __restrict__ scores,
-    DecodeSelectWs ws, int32_t* __restrict__ sel) {
+    DecodeSelectWs ws, int32_t* __restrict__ sel, int smem_words) {
   __shared__ SelShared sh;
-  // [kSmemCand] keys, [kSmemCand] indices, [kSmemWords] bitmap words
+  // [kSmemCand] keys, [kSmemCand] indices, [smem_words] bitmap words
   extern __shared__ __align__(16) uint32_t dyn_smem[];
   uint32_t* dyn_key = dyn_smem;
   int32_t* dyn_idx = reinterpret_cast<int32_t*>(dyn_smem + kSmemCand);
@@ -178,7 +178,7 @@ __global__ void __launch_bounds__(kThreads, 4) decode_topk_hist_kernel(
   // the sequence's bitmap into shared memory when it fits (loads issued now,
   // under the candidate bookkeeping)
   const int64_t nwords = (V + 31) / 32;
-  const bool bm_smem = nwords <= kSmemWords;
+  const bool bm_smem = nwords <= smem_words;
   uint32_t* bmg = ws.bitmap + b * ws.words;
   uint32_t* bm = bm_smem ? dyn_bm : bmg;
   if (bm_smem) {  // every load in flight at once (rows of words are 512-byte aligned)
@@ -243,7 +243,9 @@ __global__ void __launch_bounds__(kThreads, 4) decode_topk_hist_kernel(
       else
         radix_kth<kThreads>(KeysInGlobal{cck}, C, (int)need, sh.sel, Tk, take_eq);
     }
-    auto key_at = [&](int64_t i) { return in_smem ? cck[i] : __ldcg(cck + i); };
+    // (plain loads through the chosen pointer: a select between a shared and
+    // an L2 load would issue both, and wait for the L2 one, every time)
+    auto key_at = [&](int64_t i) { return cck[i]; };
     const int64_t seg = ((C + kThreads / 32 - 1) / (kThreads / 32) + 31) / 32 * 32;
     const int64_t plo = (int64_t)warp * seg, phi = min((int64_t)C, plo + seg);
     uint32_t eq = 0;
@@ -263,7 +265,7 @@ __global__ void __launch_bounds__(kThreads, 4) decode_topk_hist_kernel(
       const uint32_t em = __ballot_sync(0xffffffffu, is_eq);
       const bool take = i < phi && (all || key > Tk || (is_eq && eq_before + __popc(em & lt) < take_eq));
       if (take) {
-        const int32_t s = in_smem ? cci[i] : __ldcg(cci + i);
+        const int32_t s = cci[i];
         atomicOr(bm + (s >> 5), 1u << (s & 31));
       }
       eq_before += __popc(em);
@@ -273,22 +275,44 @@ __global__ void __launch_bounds__(kThreads, 4) decode_topk_hist_kernel(
   sm100::cp_async_wait_all();
   __syncthreads();
 
-  // 4. the chosen indices in ascending order, from the bitmap
-  const int64_t per = (nwords + kThreads - 1) / kThreads;
-  const int64_t w0 = min(nwords, (int64_t)tid * per), w1 = min(nwords, w0 + per);
-  auto word = [&](int64_t w) { return bm_smem ? dyn_bm[w] : __ldcg(bmg + w); };
+  // 4. the chosen indices in ascending order, from the bitmap: warp w takes
+  //    a contiguous run of words, 32 words a step with lane l on word l (a
+  //    bank each); counts first, then, from the warps' offsets, the indices
+  constexpr int kWarps = kThreads / 32;
+  auto word = [&](int64_t w) { return bm[w]; };
+  const int64_t seg = ((nwords + kWarps - 1) / kWarps + 31) / 32 * 32;
+  const int64_t ws0 = min(nwords, (int64_t)warp * seg), ws1 = min(nwords, ws0 + seg);
   uint32_t cnt = 0;
-  for (int64_t w = w0; w < w1; ++w) cnt += __popc(word(w));
-  uint32_t total;
-  uint32_t o = block_excl_scan(cnt, sh.wsum, total);
-  for (int64_t w = w0; w < w1; ++w) {
-    uint32_t x = word(w);
+#pragma unroll 4
+  for (int64_t w = ws0 + lane; w < ws1; w += 32) cnt += __popc(word(w));
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) cnt += __shfl_xor_sync(0xffffffffu, cnt, off);
+  if (lane == 0) sh.wsum[warp] = cnt;
+  __syncthreads();
+  uint32_t o = 0, total = 0;
+  for (int w = 0; w < kWarps; ++w) {
+    if (w < warp) o += sh.wsum[w];
+    total += sh.wsum[w];
+  }
+#pragma unroll 1
+  for (int64_t base = ws0; base < ws1; base += 32) {
+    const int64_t w = base + lane;
+    uint32_t x = w < ws1 ? word(w) : 0u;
+    const uint32_t c = (uint32_t)__popc(x);
+    uint32_t inc = c;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+      const uint32_t y = __shfl_up_sync(0xffffffffu, inc, off);
+      if (lane >= off) inc += y;
+    }
+    uint32_t p = o + inc - c;
     while (x != 0u) {
       const int bit = __ffs(x) - 1;
       x &= x - 1u;
-      if (o < (uint32_t)k) out[o] = (int32_t)(w * 32 + bit);
-      ++o;
+      if (p < (uint32_t)k) out[p] = (int32_t)(w * 32 + bit);
+      ++p;
     }
+    o += __shfl_sync(0xffffffffu, inc, 31);
   }
   for (uint32_t i = total + tid; i < (uint32_t)k; i += kThreads) out[i] = -1;  // (total == k)
 }
@@ -309,7 +333,8 @@ DecodeSelectWs decode_select_ws(const csa_cache_desc& d, uint8_t* base, size_t* 
     off = (off + n + 255) & ~(size_t)255;
     return o;
   };
-  const size_t o_gh = take(B * kBins * 4), o_done = take(B * 4), o_bm = take(B * w.words * 4),
+  const size_t o_gh = take(B * kBins * 4), o_done = take(B * 4), o_idone = take(B * 4),
+               o_bm = take(B * w.words * 4),
                o_ck = take(B * cap * 4), o_ci = take(B * cap * 4),
                o_cnt = take(B * kDecMaxSlices * 4), o_cck = take(B * cap * 4),
                o_cci = take(B * cap * 4);
@@ -317,6 +342,7 @@ DecodeSelectWs decode_select_ws(const csa_cache_desc& d, uint8_t* base, size_t* 
   if (base != nullptr) {
     w.ghist = reinterpret_cast<uint32_t*>(base + o_gh);
     w.done = reinterpret_cast<uint32_t*>(base + o_done);
+    w.idx_done = reinterpret_cast<uint32_t*>(base + o_idone);
     w.bitmap = reinterpret_cast<uint32_t*>(base + o_bm);
     w.cand_key = reinterpret_cast<uint32_t*>(base + o_ck);
     w.cand_idx = reinterpret_cast<int32_t*>(base + o_ci);
@@ -331,12 +357,15 @@ cudaError_t launch_decode_select(const csa_cache_desc& d, const int64_t* pos, co
                                  const DecodeSelectWs& ws, int32_t* sel, cudaStream_t s) {
   const unsigned nsl = (unsigned)((d.capacity + kSlice - 1) / kSlice);
   if (nsl > (unsigned)kDecMaxSlices) return cudaErrorInvalidValue;
-  constexpr size_t kDyn = (size_t)kSmemCand * 8 + (size_t)kSmemWords * 4;
+  // the bitmap of a whole sequence in shared memory when it fits the limit
+  const int64_t words = ((d.capacity + 31) / 32 + 3) / 4 * 4;
+  const int smem_words = (int)std::min<int64_t>(words, kMaxSmemWords);
+  const size_t kDyn = (size_t)kSmemCand * 8 + (size_t)smem_words * 4;
   const cudaError_t e = cudaFuncSetAttribute(decode_topk_hist_kernel,
                                              cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kDyn);
   if (e != cudaSuccess) return e;
   return launch_pdl(decode_topk_hist_kernel, dim3(nsl, (unsigned)d.batch), dim3(kThreads), kDyn, s,
-                    pos, (int64_t)d.capacity, d.m, d.k, scores, ws, sel);
+                    pos, (int64_t)d.capacity, d.m, d.k, scores, ws, sel, smem_words);
 }
 
 }  // namespace csa

@@ -102,9 +102,16 @@ __host__ __device__ inline int decode_qop_row(int h, int part, int H) {
 // qop: [batch] query operands (written by the append step); scores
 // [batch][capacity] fp32, written for s < V of each sequence.
 // ghist [batch][kDecHistBins]: each sequence's score histogram (added to).
+// idx_done [batch] (optional): each CTA adds, once its scores and histogram
+// counts of a sequence are written (fenced), the number of the sequence's
+// key tiles it scored, so a later kernel can start on a sequence as soon as
+// the count reaches decode_index_tiles(d, pos) without waiting for the grid.
 cudaError_t launch_decode_index_tc(const csa_cache_desc& d, const CacheView& cv,
                                    const int64_t* pos, const uint8_t* qop, float* scores,
-                                   uint32_t* ghist, unsigned int* err, cudaStream_t s);
+                                   uint32_t* ghist, uint32_t* idx_done, unsigned int* err,
+                                   cudaStream_t s);
+// Keys per indexer tile of launch_decode_index_tc for this cache.
+int decode_index_tile_keys(const csa_cache_desc& d);
 
 // Histogram of each sequence's indexer scores over the top kDecHistShift..31
 // bits of their order keys, written by the indexer for the selection step.
@@ -116,6 +123,8 @@ constexpr int kDecMaxSlices = 512;  // 4096-score slices per sequence (2M entrie
 struct DecodeSelectWs {
   uint32_t* ghist;     // [batch][kDecHistBins]  zeroed by the append step
   uint32_t* done;      // [batch]                finished slices; zeroed by the append step
+  uint32_t* idx_done;  // [batch]                key tiles the indexer has scored and counted
+                       //                        in ghist (released); zeroed by the append step
   uint32_t* bitmap;    // [batch][words]         chosen entries, one bit each
   uint32_t* cand_key;  // [batch][capacity]      threshold-bin candidates, per slice
   int32_t* cand_idx;
@@ -139,13 +148,16 @@ bool decode_attn_tc_supported(const csa_cache_desc& d);
 int decode_attn_splits(const csa_cache_desc& d);
 // With scores != NULL (CSA, decode_attn_selects(d)) the kernel takes the
 // top-k itself from the indexer's scores and histogram (sel unused) and, if
-// sel_out != NULL, writes the selection there.
+// sel_out != NULL, writes the selection there; with idx_done != NULL it
+// starts on a sequence once the indexer's tile count for it is complete
+// (tiles of idx_tile keys) instead of waiting for the indexer's whole grid.
 bool decode_attn_selects(const csa_cache_desc& d);
 cudaError_t launch_decode_attn_tc(const csa_cache_desc& d, const CacheView& cv,
                                   const int64_t* pos, const void* q, const int32_t* sel,
                                   const float* sink, float scale, int nsplit, void* out,
                                   float* part_o, float* part_ms, const float* scores,
-                                  const uint32_t* ghist, int32_t* sel_out, unsigned int* err,
+                                  const uint32_t* ghist, int32_t* sel_out,
+                                  const uint32_t* idx_done, int idx_tile, unsigned int* err,
                                   cudaStream_t s);
 
 // nr != NULL: each entry i RMSNorm-ed and its trailing dims rotated for

@@ -89,6 +89,25 @@ __device__ __forceinline__ bool mbar_wait_small(uint64_t* bar, uint32_t parity,
   return mbar_try_wait(bar, parity) || mbar_wait_spin(bar, parity, flag, abort_on_flag);
 }
 
+// Waits until the counter in global memory reaches `target` (an acquire
+// load: what its writers released before adding is visible afterwards);
+// bounded like mbar_wait, and given up as soon as *flag is set.
+static __device__ __noinline__ bool wait_count(const uint32_t* counter, uint32_t target,
+                                               unsigned int* flag) {
+  const uint64_t t0 = globaltimer();
+  while (true) {
+    uint32_t v;
+    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(counter) : "memory");
+    if (v >= target) return true;
+    if (flag_value(flag) != 0) return false;
+    if (globaltimer() - t0 > kWaitLimitNs) {
+      atomicOr(flag, 1u);
+      return false;
+    }
+    __nanosleep(200);
+  }
+}
+
 // mbar_wait with an explicit limit (ns) and no early exit on the flag.
 __device__ __forceinline__ bool mbar_wait_limit(uint64_t* bar, uint32_t parity,
                                                 unsigned int* flag, uint64_t limit_ns) {
