@@ -362,7 +362,8 @@ __global__ void __launch_bounds__(1024) append_emit_kernel(csa_cache_desc d, Cac
                                                           uint8_t* __restrict__ qop,
                                                           uint32_t* __restrict__ ghist,
                                                           uint32_t* __restrict__ sel_done,
-                                                          uint32_t* __restrict__ idx_done) {
+                                                          uint32_t* __restrict__ idx_done,
+                                                          uint32_t* __restrict__ list_ready) {
   extern __shared__ float sx[];  // [c + c_i] + 32
   const int64_t b = blockIdx.x;
   // the previous step's kernels read the window slot this token overwrites
@@ -379,6 +380,7 @@ __global__ void __launch_bounds__(1024) append_emit_kernel(csa_cache_desc d, Cac
       if (threadIdx.x == 0) {
         sel_done[b] = 0u;
         idx_done[b] = 0u;
+        list_ready[b] = 0u;
       }
     }
     return;
@@ -754,7 +756,7 @@ cudaError_t launch_decode_step(const csa_cache_desc& d, const CacheView& cv, con
                                dim3((unsigned)d.batch, qop != nullptr ? 2u : 1u),
                                dim3(emit_threads), emit_smem, s, d, cv, pos, rows, p,
                                (const __nv_bfloat16*)q_i, w_i, qop, sws.ghist, sws.done,
-                               sws.idx_done);
+                               sws.idx_done, sws.list_ready);
   if (err != cudaSuccess) return err;
   if (!d.is_hca && w.tc_index) {
     float* scores = p.scores_out != nullptr ? p.scores_out : reinterpret_cast<float*>(wb + w.scores);
@@ -799,7 +801,9 @@ cudaError_t launch_decode_step(const csa_cache_desc& d, const CacheView& cv, con
                                  w.attn_select ? sws.ghist : nullptr,
                                  w.attn_select ? p.sel_out : nullptr,
                                  w.attn_select ? sws.idx_done : nullptr,
-                                 decode_index_tile_keys(d), flag, s);
+                                 decode_index_tile_keys(d),
+                                 w.attn_select ? reinterpret_cast<int32_t*>(wb + w.sel) : nullptr,
+                                 w.attn_select ? sws.list_ready : nullptr, flag, s);
   }
   const size_t asmem = sizeof(float) * ((size_t)kDecTE * (d.c + 1) + (size_t)kDecHG * d.c +
                                         kDecHG * kDecTE) + sizeof(int64_t) * kDecTE;

@@ -297,6 +297,24 @@ __device__ int fused_select(const float* __restrict__ row, const uint32_t* __res
   return k;
 }
 
+// Split s > 0 of a selecting launch, before its first tile that needs the
+// selection: waits (thread 0) for split 0 to publish it, then the gather
+// threads copy slots [lo, hi) of it into shared memory.  False if the wait
+// gave up (in every gather thread).
+__device__ __noinline__ bool fetch_list(const uint32_t* ready, const int32_t* src, int32_t* list,
+                                        int lo, int hi, unsigned int* err) {
+  using namespace sm100;
+  const int tid = threadIdx.x;
+  const bool got = tid != 0 || wait_count(ready, 1u, err);
+  if (named_bar_or(2, kGatherThreads, !got)) return false;
+  for (int sl = lo + tid; sl < hi; sl += kGatherThreads) list[sl] = __ldcg(src + sl);
+  named_bar_or(2, kGatherThreads, false);
+  return true;
+}
+
+// kSelect: the launch selects (scores != NULL); the other instance (HCA, or
+// a selection given in sel) holds none of the selection code.
+template <bool kSelect>
 __global__ void __launch_bounds__(kThreads, 1) decode_attn_tc_kernel(
     const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CacheView cv,
     const int64_t* __restrict__ pos, const int32_t* __restrict__ sel, int k, int window, int m,
@@ -304,6 +322,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_attn_tc_kernel(
     float* __restrict__ part_o, float* __restrict__ part_ms, __nv_bfloat16* __restrict__ out,
     const float* __restrict__ scores, const uint32_t* __restrict__ ghist,
     int32_t* __restrict__ sel_out, const uint32_t* __restrict__ idx_done, int idx_tile,
+    int32_t* __restrict__ xlist, uint32_t* __restrict__ list_ready,
     unsigned int* __restrict__ err) {
   using namespace sm100;
   extern __shared__ uint8_t smem_raw[];
@@ -352,14 +371,16 @@ __global__ void __launch_bounds__(kThreads, 1) decode_attn_tc_kernel(
   // is awaited rather than the end of the indexer's grid, so a sequence
   // starts as soon as its keys are scored (the cache itself was written
   // before the indexer started)
-  if (scores != nullptr && idx_done != nullptr) {
-    if (tid == 0) {
+  if (kSelect && idx_done != nullptr) {
+    // (only the selecting CTA of a sequence reads what the indexer wrote)
+    if (tid == 0 && split == 0) {
       const int64_t tp = pos[b];
       const int64_t Vp = tp < 0 ? 0 : min((tp + 1) / m, cap);
       const uint32_t want = (uint32_t)((Vp + idx_tile - 1) / idx_tile);
       const bool ok = want == 0 || wait_count(idx_done + b, want, err);
       bar->abort = ok ? flag_value(err) : 1u;
     }
+    if (tid == 0 && split != 0) bar->abort = flag_value(err);
     __syncthreads();  // nothing indexer-written is read before the count is complete
   } else {
     pdl_wait();
@@ -374,16 +395,36 @@ __global__ void __launch_bounds__(kThreads, 1) decode_attn_tc_kernel(
   // -------- the entry list: valid selections in order (CSA) or 0..V-1 (HCA) ----
   // (scores != NULL: the CSA selection itself runs here, from the indexer's
   // scores and histogram)
-  const bool csa = sel != nullptr || scores != nullptr;
+  const bool csa = sel != nullptr || kSelect;
   int nsel;
-  if (scores != nullptr) {
+  // (split > 0 of a selecting launch: the selection comes from split 0 of the
+  // same sequence through xlist; the range's window-only tiles go first)
+  bool xfetch = false;
+  if (kSelect && split == 0) {
     SelState* st = reinterpret_cast<SelState*>(red);
     nsel = fused_select(scores + b * cap, ghist + b * kSelBins, (int)V, k,
                         reinterpret_cast<float*>(sQ), reinterpret_cast<uint32_t*>(sP),
                         reinterpret_cast<uint32_t*>(smem + OFF_BM), list, wcount, st);
-    if (sel_out != nullptr && split == 0)
+    if (nsplit > 1 && V > k && xlist != nullptr) {
+#pragma unroll 1
+      for (int j = tid; j < nsel; j += kThreads) xlist[b * k + j] = list[j];
+      __threadfence();
+      __syncthreads();
+      if (tid == 0)
+        asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(list_ready + b), "r"(1u)
+                     : "memory");
+    }
+    if (sel_out != nullptr)
 #pragma unroll 1
       for (int j = tid; j < k; j += kThreads) sel_out[b * k + j] = j < nsel ? list[j] : -1;
+  } else if (kSelect) {
+    nsel = (int)min(V, (int64_t)k);
+    if (V <= k) {
+#pragma unroll 1
+      for (int i = tid; i < nsel; i += kThreads) list[i] = i;
+    } else {
+      xfetch = true;
+    }
   } else if (sel != nullptr) {
     const int32_t* row = sel + b * k;
     const int per = (k + kThreads - 1) / kThreads;
@@ -417,6 +458,11 @@ __global__ void __launch_bounds__(kThreads, 1) decode_attn_tc_kernel(
   const int tile0 = (int)((int64_t)T * split / nsplit);
   const int tile1 = (int)((int64_t)T * (split + 1) / nsplit);
   const int ntile = tile1 - tile0;
+  // tiles of the range in processing order: with xfetch, the tiles holding
+  // only window rows (slots >= nsel) first, while split 0 selects
+  const int wtile = max(tile0, (nsel + kTE - 1) / kTE);
+  const int nw = xfetch ? max(0, tile1 - wtile) : 0;
+  auto tile_at = [&](int jt) { return jt < nw ? wtile + jt : tile0 + (jt - nw); };
   tc_fence_before();
   __syncthreads();  // the list, the barriers and the TMEM address
   tc_fence_after();
@@ -436,7 +482,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_attn_tc_kernel(
   // into both chunks; only this thread touches them).
   const int s_me = (tid & 31) >> 2, q_me = tid & 3;
   auto gather_tile = [&](int jt) -> bool {
-    const int tile = tile0 + jt;
+    const int tile = tile_at(jt);
     const bool body = s_me < kBody / 64;
     // the slab is free once the previous tile's P.V chunk that reads it is done
     const bool free_ok =
@@ -560,6 +606,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_attn_tc_kernel(
 #pragma unroll 1
     for (int slot = (tile0 + 1) * kTE + tid; slot < min(N, tile1 * kTE); slot += kGatherThreads) {
       if (slot < nsel) {
+        if (xfetch) continue;  // (the selection is not known yet)
         const int64_t es = entry_row(cv, b, csa ? (int64_t)list[slot] : (int64_t)slot, cap);
         if (es >= 0) {
           bulk_prefetch_l2(cv.entry_fp8 + es * kBody, kBody);
@@ -581,10 +628,14 @@ __global__ void __launch_bounds__(kThreads, 1) decode_attn_tc_kernel(
     float lsum = 0.f;       // lane i: its head's sum of P over this warp's rows
     bool ok = true;
     for (int jt = 0; jt < ntile && ok; ++jt) {
+      if (xfetch && jt == nw &&
+          !(ok = fetch_list(list_ready + b, xlist + b * k, list, tile0 * kTE,
+                            min(tile1 * kTE, nsel), err)))
+        break;
       if (!(ok = gather_tile(jt))) break;
       if (!(ok = mbar_wait_small(&bar->s_full, (uint32_t)(jt & 1), err))) break;
       tc_fence_after();
-      const bool valid = (tile0 + jt) * kTE + row < N;
+      const bool valid = tile_at(jt) * kTE + row < N;
       float v[32];
       {
         uint32_t r[32];
@@ -790,18 +841,20 @@ cudaError_t launch_decode_attn_tc(const csa_cache_desc& d, const CacheView& cv,
                                   const float* sink, float scale, int nsplit, void* out,
                                   float* part_o, float* part_ms, const float* scores,
                                   const uint32_t* ghist, int32_t* sel_out,
-                                  const uint32_t* idx_done, int idx_tile, unsigned int* err,
-                                  cudaStream_t s) {
+                                  const uint32_t* idx_done, int idx_tile, int32_t* xlist,
+                                  uint32_t* list_ready, unsigned int* err, cudaStream_t s) {
   CUtensorMap tq;
   if (!make_tmap_bf16_3d(&tq, q, kC, kNH, d.batch, kC * 2ull, (uint64_t)kNH * kC * 2, 64, kNH))
     return cudaErrorInvalidValue;
-  cudaError_t e = cudaFuncSetAttribute(decode_attn_tc_kernel,
+  auto kern = scores != nullptr ? decode_attn_tc_kernel<true> : decode_attn_tc_kernel<false>;
+  cudaError_t e = cudaFuncSetAttribute(kern,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM);
   if (e != cudaSuccess) return e;
-  e = launch_pdl(decode_attn_tc_kernel, dim3((unsigned)nsplit, (unsigned)d.batch), dim3(kThreads),
+  e = launch_pdl(kern, dim3((unsigned)nsplit, (unsigned)d.batch), dim3(kThreads),
                  (size_t)SMEM, s, tq, cv, pos, d.is_hca ? nullptr : sel, (int)d.k, (int)d.window,
                  (int)d.m, (int64_t)d.capacity, sink, scale, nsplit, part_o, part_ms,
-                 (__nv_bfloat16*)out, scores, ghist, sel_out, idx_done, idx_tile, err);
+                 (__nv_bfloat16*)out, scores, ghist, sel_out, idx_done, idx_tile, xlist,
+                 list_ready, err);
   if (e != cudaSuccess || nsplit == 1) return e;
   return launch_pdl(decode_combine_kernel, dim3(kNH, (unsigned)d.batch), dim3(kC / 4), 0, s,
                     (const float*)part_o, (const float*)part_ms, sink, nsplit,

@@ -334,6 +334,7 @@ DecodeSelectWs decode_select_ws(const csa_cache_desc& d, uint8_t* base, size_t* 
     return o;
   };
   const size_t o_gh = take(B * kBins * 4), o_done = take(B * 4), o_idone = take(B * 4),
+               o_lready = take(B * 4),
                o_bm = take(B * w.words * 4),
                o_ck = take(B * cap * 4), o_ci = take(B * cap * 4),
                o_cnt = take(B * kDecMaxSlices * 4), o_cck = take(B * cap * 4),
@@ -343,6 +344,7 @@ DecodeSelectWs decode_select_ws(const csa_cache_desc& d, uint8_t* base, size_t* 
     w.ghist = reinterpret_cast<uint32_t*>(base + o_gh);
     w.done = reinterpret_cast<uint32_t*>(base + o_done);
     w.idx_done = reinterpret_cast<uint32_t*>(base + o_idone);
+    w.list_ready = reinterpret_cast<uint32_t*>(base + o_lready);
     w.bitmap = reinterpret_cast<uint32_t*>(base + o_bm);
     w.cand_key = reinterpret_cast<uint32_t*>(base + o_ck);
     w.cand_idx = reinterpret_cast<int32_t*>(base + o_ci);

@@ -125,6 +125,8 @@ struct DecodeSelectWs {
   uint32_t* done;      // [batch]                finished slices; zeroed by the append step
   uint32_t* idx_done;  // [batch]                key tiles the indexer has scored and counted
                        //                        in ghist (released); zeroed by the append step
+  uint32_t* list_ready;  // [batch]              the attention's selection is published;
+                         //                      zeroed by the append step
   uint32_t* bitmap;    // [batch][words]         chosen entries, one bit each
   uint32_t* cand_key;  // [batch][capacity]      threshold-bin candidates, per slice
   int32_t* cand_idx;
@@ -151,14 +153,17 @@ int decode_attn_splits(const csa_cache_desc& d);
 // sel_out != NULL, writes the selection there; with idx_done != NULL it
 // starts on a sequence once the indexer's tile count for it is complete
 // (tiles of idx_tile keys) instead of waiting for the indexer's whole grid.
+// With several CTAs per sequence only split 0 selects: it publishes the
+// selection in xlist [batch][k] and sets list_ready[b] (zeroed by the append
+// step); the others process their window-only tiles meanwhile.
 bool decode_attn_selects(const csa_cache_desc& d);
 cudaError_t launch_decode_attn_tc(const csa_cache_desc& d, const CacheView& cv,
                                   const int64_t* pos, const void* q, const int32_t* sel,
                                   const float* sink, float scale, int nsplit, void* out,
                                   float* part_o, float* part_ms, const float* scores,
                                   const uint32_t* ghist, int32_t* sel_out,
-                                  const uint32_t* idx_done, int idx_tile, unsigned int* err,
-                                  cudaStream_t s);
+                                  const uint32_t* idx_done, int idx_tile, int32_t* xlist,
+                                  uint32_t* list_ready, unsigned int* err, cudaStream_t s);
 
 // nr != NULL: each entry i RMSNorm-ed and its trailing dims rotated for
 // position m * i as it is written (or by a second in-place pass).
