@@ -276,15 +276,26 @@ __global__ void __launch_bounds__(kThreads, 4) decode_topk_hist_kernel(
   __syncthreads();
 
   // 4. the chosen indices in ascending order, from the bitmap: warp w takes
-  //    a contiguous run of words, 32 words a step with lane l on word l (a
-  //    bank each); counts first, then, from the warps' offsets, the indices
+  //    a contiguous run of words, 128 words a step with lane l on words
+  //    4l .. 4l+3 (one 16-byte access per lane); counts first, then, from
+  //    the warps' offsets, the indices
   constexpr int kWarps = kThreads / 32;
-  auto word = [&](int64_t w) { return bm[w]; };
-  const int64_t seg = ((nwords + kWarps - 1) / kWarps + 31) / 32 * 32;
+  const int64_t seg = ((nwords + kWarps - 1) / kWarps + 127) / 128 * 128;
   const int64_t ws0 = min(nwords, (int64_t)warp * seg), ws1 = min(nwords, ws0 + seg);
+  auto quad = [&](int64_t w) -> uint4 {  // words w .. w+3 (w a multiple of 4), zero past ws1
+    if (w + 4 <= ws1) return *reinterpret_cast<const uint4*>(bm + w);
+    uint4 q = make_uint4(0u, 0u, 0u, 0u);
+    if (w < ws1) q.x = bm[w];
+    if (w + 1 < ws1) q.y = bm[w + 1];
+    if (w + 2 < ws1) q.z = bm[w + 2];
+    return q;
+  };
   uint32_t cnt = 0;
-#pragma unroll 4
-  for (int64_t w = ws0 + lane; w < ws1; w += 32) cnt += __popc(word(w));
+#pragma unroll 2
+  for (int64_t w = ws0 + 4 * lane; w < ws1; w += 128) {
+    const uint4 q = quad(w);
+    cnt += __popc(q.x) + __popc(q.y) + __popc(q.z) + __popc(q.w);
+  }
 #pragma unroll
   for (int off = 16; off > 0; off >>= 1) cnt += __shfl_xor_sync(0xffffffffu, cnt, off);
   if (lane == 0) sh.wsum[warp] = cnt;
@@ -295,10 +306,11 @@ __global__ void __launch_bounds__(kThreads, 4) decode_topk_hist_kernel(
     total += sh.wsum[w];
   }
 #pragma unroll 1
-  for (int64_t base = ws0; base < ws1; base += 32) {
-    const int64_t w = base + lane;
-    uint32_t x = w < ws1 ? word(w) : 0u;
-    const uint32_t c = (uint32_t)__popc(x);
+  for (int64_t base = ws0; base < ws1; base += 128) {
+    const int64_t w = base + 4 * lane;
+    const uint4 q = quad(w);
+    const uint32_t wd[4] = {q.x, q.y, q.z, q.w};
+    const uint32_t c = __popc(q.x) + __popc(q.y) + __popc(q.z) + __popc(q.w);
     uint32_t inc = c;
 #pragma unroll
     for (int off = 1; off < 32; off <<= 1) {
@@ -306,11 +318,15 @@ __global__ void __launch_bounds__(kThreads, 4) decode_topk_hist_kernel(
       if (lane >= off) inc += y;
     }
     uint32_t p = o + inc - c;
-    while (x != 0u) {
-      const int bit = __ffs(x) - 1;
-      x &= x - 1u;
-      if (p < (uint32_t)k) out[p] = (int32_t)(w * 32 + bit);
-      ++p;
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      uint32_t x = wd[e];
+      while (x != 0u) {
+        const int bit = __ffs(x) - 1;
+        x &= x - 1u;
+        if (p < (uint32_t)k) out[p] = (int32_t)((w + e) * 32 + bit);
+        ++p;
+      }
     }
     o += __shfl_sync(0xffffffffu, inc, 31);
   }
