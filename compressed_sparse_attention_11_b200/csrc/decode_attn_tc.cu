@@ -391,6 +391,10 @@ __global__ void __launch_bounds__(kThreads, 1) decode_attn_tc_kernel(
   const int64_t V = t < 0 ? 0 : min((t + 1) / m, cap);
   const int64_t w0 = max((int64_t)0, t - window + 1);
   const int nwin = t < 0 ? 0 : (int)(t - w0 + 1);
+  // ring slot of window row w0 (row w0 + i sits at slot w0m + i, wrapped
+  // once: i < window), so no 64-bit remainder per row
+  const int w0m = (int)(w0 % window);
+  const __nv_bfloat16* const ring = cv.window + b * window * kC;
 
   // -------- the entry list: valid selections in order (CSA) or 0..V-1 (HCA) ----
   // (scores != NULL: the CSA selection itself runs here, from the indexer's
@@ -511,9 +515,9 @@ __global__ void __launch_bounds__(kThreads, 1) decode_attn_tc_kernel(
             cp_async_16(d1, p + 8);
           }
         } else if (slot >= nsel && slot < N) {
-          const int64_t u = w0 + (slot - nsel);
-          const __nv_bfloat16* p =
-              cv.window + (b * window + u % window) * kC + s_me * 64 + q_me * 16;
+          int u = w0m + (slot - nsel);
+          u -= u >= window ? window : 0;
+          const __nv_bfloat16* p = ring + (int64_t)u * kC + s_me * 64 + q_me * 16;
           cp_async_16(d0, p);
           cp_async_16(d1, p + 8);
         } else {  // past the end, or an entry without a block: zeros
@@ -614,8 +618,9 @@ __global__ void __launch_bounds__(kThreads, 1) decode_attn_tc_kernel(
           bulk_prefetch_l2(cv.entry_scale + (es & ~(int64_t)3), 16);
         }
       } else {
-        const int64_t u = w0 + (slot - nsel);
-        bulk_prefetch_l2(cv.window + (b * window + u % window) * kC, kC * 2);
+        int u = w0m + (slot - nsel);
+        u -= u >= window ? window : 0;
+        bulk_prefetch_l2(ring + (int64_t)u * kC, kC * 2);
       }
     }
     const int quad = warp & 3, hh = (warp >> 2) & 1;
