@@ -44,17 +44,17 @@ UNIT = "tokens/s"
 # profiles/).  A figure is reported only while the kernel sources it was
 # measured on are unchanged (sha256 prefix per file), else null.
 MEASURED_TRAFFIC = {
-    # index_scores_tc_kernel 1133.3 MB read + 2136.3 MB written, topk_rows_staged_kernel
-    # 2149.4 MB read + 131.0 MB written (n = 65536; ncu dram__bytes_read/write.sum)
-    "index_topk": {"bytes": 5550000640, "sources": {
-        'compressed_sparse_attention_11_b200/csrc/indexer_tc.cu': '7f5543f1ca4e8e9e',
-        'compressed_sparse_attention_11_b200/csrc/topk.cu': '44874bde73cf3699',
-        'compressed_sparse_attention_11_b200/csrc/sm100.cuh': '1863469781a2e737',
+    # index_scores_tc_kernel 1126.2 MB read + 2136.1 MB written, topk_rows_staged_kernel
+    # 2149.4 MB read + 131.3 MB written (n = 65536; ncu dram__bytes_read/write.sum)
+    "index_topk": {"bytes": 5543051520, "sources": {
+        'compressed_sparse_attention_11_b200/csrc/indexer_tc.cu': 'e3d3bdb783809238',
+        'compressed_sparse_attention_11_b200/csrc/topk.cu': '7d7a94f9ad3e7624',
+        'compressed_sparse_attention_11_b200/csrc/sm100.cuh': 'efc54e296506e512',
         'compressed_sparse_attention_11_b200/csrc/common.cuh': '2c8e048cf6f6eadb'}},
-    # attn_tc_kernel 4554.1 MB read + 4247.6 MB written (n = 65536)
-    "sparse_attn": {"bytes": 8801669120, "sources": {
-        'compressed_sparse_attention_11_b200/csrc/attn_tc.cu': '16fc1a623830605f',
-        'compressed_sparse_attention_11_b200/csrc/sm100.cuh': '1863469781a2e737',
+    # attn_tc_kernel 4571.7 MB read + 4242.5 MB written (n = 65536)
+    "sparse_attn": {"bytes": 8814228992, "sources": {
+        'compressed_sparse_attention_11_b200/csrc/attn_tc.cu': '9eaa94c3e12544ce',
+        'compressed_sparse_attention_11_b200/csrc/sm100.cuh': 'efc54e296506e512',
         'compressed_sparse_attention_11_b200/csrc/common.cuh': '2c8e048cf6f6eadb',
         'compressed_sparse_attention_11_b200/csrc/rope.cuh': '8af18f1b31f2b303',
         'compressed_sparse_attention_11_b200/csrc/tc_attn_util.cuh': 'fbd5bcb87c834e55'}},
