@@ -258,6 +258,9 @@ def time_steps(step_fn, ncalls, K, world, dev):
     evs = [[torch.cuda.Event(enable_timing=True) for _ in range(ncalls + 1)] for _ in range(K)]
     start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     barrier(world)
+    # keep the device busy while the host enqueues the first step, so that the
+    # timed region holds device time only (no wait for the first launch)
+    torch.cuda._sleep(2_000_000)
     start.record()
     for i in range(K):
         step_fn(evs[i])

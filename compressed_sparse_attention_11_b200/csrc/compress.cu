@@ -6,16 +6,19 @@
 // (CSA: m own-block rows of Za/Ca and m previous-block rows of Zb/Cb; the
 // first entry has no previous block), applied as Hadamard weights to C.
 //
-// HBM-streaming kernels: every input row is read exactly once, 16 bytes per
-// thread per row (8 dims), lanes along the dims so that each load
-// instruction of a warp reads 512 contiguous bytes of one row.  Entries of
-// at most eight rows (CSA m <= 4) take one thread per (entry, 8-dim chunk)
-// with the softmax kept online in registers over its rows.  Larger row sets
-// are split over R warps of one block; a thread's rows are read in rounds of
-// four with all loads of a round issued before its arithmetic (a two-pass
-// softmax over registers), and the R partial states are merged through
-// shared memory.  A row whose logit equals the running maximum gets weight 1
-// exactly, so a single +inf logit selects its row.
+// HBM-streaming kernels: every input row is read exactly once, lanes along
+// the dims so that each load instruction of a warp reads contiguous bytes of
+// one row.  Entries of at most eight rows (CSA m <= 4) take one thread per
+// (entry, 4-dim chunk): all of its rows are loaded at once (8 bytes of a
+// bf16 row per lane), then each dim takes a two-pass softmax over them in
+// registers with no data-dependent branch; 64 registers keep four blocks of
+// 256 threads per SM, and with them enough loads in flight to stream.
+// Larger row sets are split over R warps of one block, one thread per
+// (entry, 8-dim chunk, row group); a thread's rows are read in rounds of
+// four with all loads of a round issued before its arithmetic, and the R
+// partial states are merged through shared memory.  A
+// row whose logit equals the maximum gets weight 1 exactly, so a single +inf
+// logit selects its row.
 #include "common.cuh"
 #include "launch.h"
 #include "rope.cuh"
@@ -162,62 +165,154 @@ struct EntryNormRope {
   float base;
 };
 
-// Entries with at most eight rows: one thread per (entry, 8-dim chunk).  With
-// the norm, an entry's c / 8 threads (a power of two dividing the block) sum
-// their squares by shuffles, and across warps through shared memory.
+// Four elements of one row, raw.
+template <typename T>
+struct Raw4;
+template <>
+struct Raw4<__nv_bfloat16> {
+  uint2 u;
+  __device__ __forceinline__ void load(const __nv_bfloat16* p) {
+    u = __ldcs(reinterpret_cast<const uint2*>(p));
+  }
+  __device__ __forceinline__ float get(int q) const {
+    const uint32_t w = q < 2 ? u.x : u.y;
+    return __uint_as_float((q & 1) ? (w & 0xffff0000u) : (w << 16));
+  }
+};
+template <>
+struct Raw4<float> {
+  float4 a;
+  __device__ __forceinline__ void load(const float* p) {
+    a = __ldcs(reinterpret_cast<const float4*>(p));
+  }
+  __device__ __forceinline__ float get(int q) const {
+    return q == 0 ? a.x : q == 1 ? a.y : q == 2 ? a.z : a.w;
+  }
+};
+
+// Four consecutive dims d0 .. d0 + 3 (d0 a multiple of 4) of an entry whose
+// reciprocal RMS is `inv`: scaled by inv * gamma[d], and turned pairwise for
+// position `pos` where they lie in the trailing rope_dims dims.
+__device__ __forceinline__ void norm_rope4(float v[4], int d0, int c, float inv,
+                                           const float* __restrict__ gamma, int64_t pos,
+                                           int rope_dims, float base) {
+#pragma unroll
+  for (int q = 0; q < 4; ++q) v[q] = v[q] * inv * __ldg(gamma + d0 + q);
+  if (d0 >= c - rope_dims) {
+    const int j0 = (d0 - (c - rope_dims)) >> 1;
+#pragma unroll
+    for (int p = 0; p < 2; ++p) {
+      float cs, sn;
+      rope_cos_sin(pos, j0 + p, rope_dims, base, cs, sn);
+      rope_turn(v[2 * p], v[2 * p + 1], cs, sn);
+    }
+  }
+}
+
+// Softmax over the live rows of four dims: o[q] = sum_j w_j C_j[q] / sum_j w_j
+// with w_j = exp(l_j - max l), l_j = Z_j[q] + bias_j[q].  The logits are kept
+// in base-2 units; a row at the maximum weighs 1 exactly, which the plain
+// form gets from ex2(0) when every maximum is finite, and the guarded form
+// keeps for an infinite maximum (a +inf logit selects its row, all -inf
+// logits weigh alike).
+template <int kMaxRows, typename T, typename Bias>
+__device__ __forceinline__ void fold_rows4(const Raw4<T> (&cr)[kMaxRows],
+                                           const Raw4<T> (&zr)[kMaxRows],
+                                           const bool (&live)[kMaxRows], const Bias& bias,
+                                           float o[4]) {
+  float lg[kMaxRows][4], mx[4], sum[4], acc[4];
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    mx[q] = kNegInf;
+    sum[q] = 0.f;
+    acc[q] = 0.f;
+  }
+#pragma unroll
+  for (int j = 0; j < kMaxRows; ++j) {
+    if (!live[j]) continue;
+    const float4 bj = bias(j);
+    const float b4[4] = {bj.x, bj.y, bj.z, bj.w};
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      lg[j][q] = (zr[j].get(q) + b4[q]) * kLog2e;
+      mx[q] = fmaxf(mx[q], lg[j][q]);
+    }
+  }
+  const float kInf = -kNegInf;
+  const bool finite = fabsf(mx[0]) < kInf && fabsf(mx[1]) < kInf &&
+                      fabsf(mx[2]) < kInf && fabsf(mx[3]) < kInf;
+  if (finite) {
+#pragma unroll
+    for (int j = 0; j < kMaxRows; ++j) {
+      if (!live[j]) continue;
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        const float w = ex2(lg[j][q] - mx[q]);
+        sum[q] += w;
+        acc[q] = fmaf(w, cr[j].get(q), acc[q]);
+      }
+    }
+  } else {
+#pragma unroll
+    for (int j = 0; j < kMaxRows; ++j) {
+      if (!live[j]) continue;
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        const float w = lg[j][q] >= mx[q] ? 1.f : ex2(lg[j][q] - mx[q]);
+        sum[q] += w;
+        acc[q] = fmaf(w, cr[j].get(q), acc[q]);
+      }
+    }
+  }
+#pragma unroll
+  for (int q = 0; q < 4; ++q) o[q] = acc[q] / sum[q];
+}
+
+// Entries with at most eight rows, one thread per (entry, 4-dim chunk): all
+// rows of the thread are loaded at once (8 bytes of a bf16 row per lane, so a
+// warp reads 256 contiguous bytes of it), then each dim takes a two-pass
+// softmax over its rows in registers, with no data-dependent branch.
 template <typename T, bool kNorm>
-__global__ void __launch_bounds__(256) compress_rows_kernel(
+__global__ void __launch_bounds__(256, sizeof(T) == 2 ? 4 : 2) compress_rows_kernel(
     const T* __restrict__ ca, const T* __restrict__ cb, const T* __restrict__ za,
     const T* __restrict__ zb, const float* __restrict__ ba, const float* __restrict__ bb,
     int64_t n, int c, int m, int rows, int64_t E, int64_t items, EntryNormRope nr,
     T* __restrict__ out) {
+  constexpr int kMaxRows = 8;
   const int64_t g0 = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
   if (!kNorm && g0 >= items) return;
   const bool act = g0 < items;  // (with the norm every thread reaches the block barrier)
   const int64_t g = act ? g0 : items - 1;
-  const int chunks = c >> 3;
-  const int d0 = (int)(g % chunks) * 8;
+  const int chunks = c >> 2;
+  const int d0 = (int)(g % chunks) * 4;
   const int64_t rest = g / chunks;
   const int64_t i = rest % E, b = rest / E;
-  float M[8], S[8], A[8];
+  Raw4<T> cr[kMaxRows], zr[kMaxRows];
+  bool live[kMaxRows];
 #pragma unroll
-  for (int q = 0; q < 8; ++q) {
-    M[q] = kNegInf;
-    S[q] = 0.f;
-    A[q] = 0.f;
-  }
-  for (int j = 0; j < rows; ++j) {
-    const T* cp;
-    const T* zp;
-    const float* bp;
-    if (!row_ptrs(ca, cb, za, zb, ba, bb, b * n, i, j, m, c, d0, cp, zp, bp)) continue;
-    float cv[8], zv[8], bv[8];
-    load8(cp, cv);
-    load8(zp, zv);
-    load8(bp, bv);
-#pragma unroll
-    for (int q = 0; q < 8; ++q) {
-      const float l = zv[q] + bv[q];
-      if (l >= M[q]) {  // new maximum (or equal to it): weight 1 for this row
-        const float f = M[q] == l ? 1.f : ex2((M[q] - l) * kLog2e);
-        S[q] = S[q] * f + 1.f;
-        A[q] = A[q] * f + cv[q];
-        M[q] = l;
-      } else {
-        const float w = ex2((l - M[q]) * kLog2e);
-        S[q] += w;
-        A[q] = fmaf(w, cv[q], A[q]);
-      }
+  for (int j = 0; j < kMaxRows; ++j) {
+    const T* cp = nullptr;
+    const T* zp = nullptr;
+    const float* bp = nullptr;
+    live[j] = j < rows && row_ptrs(ca, cb, za, zb, ba, bb, b * n, i, j, m, c, d0, cp, zp, bp);
+    if (live[j]) {
+      cr[j].load(cp);
+      zr[j].load(zp);
     }
   }
-  float o[8];
-#pragma unroll
-  for (int q = 0; q < 8; ++q) o[q] = A[q] / S[q];
+  // the positional bias of row j (a few KB shared by all entries: L1 hits),
+  // read once per pass rather than held in registers
+  const auto bias = [&](int j) {
+    return __ldg(reinterpret_cast<const float4*>((j < m ? ba + (int64_t)j * c
+                                                        : bb + (int64_t)(j - m) * c) + d0));
+  };
+  float o[4];
+  fold_rows4(cr, zr, live, bias, o);
   if constexpr (kNorm) {
     __shared__ float wsum[8];
     float ss = 0.f;
 #pragma unroll
-    for (int q = 0; q < 8; ++q) ss = fmaf(o[q], o[q], ss);
+    for (int q = 0; q < 4; ++q) ss = fmaf(o[q], o[q], ss);
     const int seg = chunks < 32 ? chunks : 32;
     for (int off = seg >> 1; off > 0; off >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, off);
     if (chunks > 32) {  // the entry spans chunks / 32 warps of the block
@@ -229,9 +324,16 @@ __global__ void __launch_bounds__(256) compress_rows_kernel(
       for (int w = 0; w < chunks / 32; ++w) ss += wsum[w0 + w];
     }
     const float inv = 1.f / sqrtf(ss / (float)c + nr.eps);
-    norm_rope8(o, d0, c, inv, nr.gamma, (int64_t)m * i, nr.rope_dims, nr.base);
+    norm_rope4(o, d0, c, inv, nr.gamma, (int64_t)m * i, nr.rope_dims, nr.base);
   }
-  if (act) store8(out + (b * E + i) * c + d0, o);
+  if (act) {
+    T* dst = out + (b * E + i) * c + d0;
+    if constexpr (sizeof(T) == 2) {
+      *reinterpret_cast<uint2*>(dst) = make_uint2(pack_bf16x2(o[0], o[1]), pack_bf16x2(o[2], o[3]));
+    } else {
+      *reinterpret_cast<float4*>(dst) = make_float4(o[0], o[1], o[2], o[3]);
+    }
+  }
 }
 
 // Entries with more rows: block (CX chunks) x (R row groups); thread (x, r)
@@ -323,11 +425,12 @@ cudaError_t launch_compress_t(const void* ca, const void* cb, const void* za, co
   const int rows = overlap ? 2 * m : m;
   if (batch * E == 0) return cudaSuccess;
   const int chunks = c / 8;
-  const bool fused = nr != nullptr && chunks <= 256 && 256 % chunks == 0;
   if (rows <= 8) {
-    const int64_t items = batch * E * chunks;
+    const int chunks4 = c / 4;
+    const bool fused4 = nr != nullptr && chunks4 <= 256 && 256 % chunks4 == 0;
+    const int64_t items = batch * E * chunks4;
     const unsigned grid = (unsigned)((items + 255) / 256);
-    if (fused) {
+    if (fused4) {
       const EntryNormRope enr{nr->gamma, nr->eps, nr->rope_dims, nr->rope_base};
       compress_rows_kernel<T, true><<<grid, 256, 0, s>>>(
           (const T*)ca, (const T*)cb, (const T*)za, (const T*)zb, ba, bb, n, c, m, rows, E,

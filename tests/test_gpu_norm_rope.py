@@ -49,10 +49,10 @@ def test_norm_rope_rows_in_place():
 
 
 @pytest.mark.parametrize("dt,n,c,m,overlap", [
-    (torch.bfloat16, 1024, 512, 4, True),     # fused: an entry's 64 threads span two warps
-    (torch.float32, 512, 128, 4, True),       # fused: 16 threads per entry
+    (torch.bfloat16, 1024, 512, 4, True),     # fused: an entry's 128 threads span four warps
+    (torch.float32, 512, 128, 4, True),       # fused: 32 threads per entry, one warp
     (torch.bfloat16, 2048, 512, 128, False),  # HCA split kernel + in-place second pass
-    (torch.float32, 96, 40, 4, True),         # 5 chunks per entry: second pass
+    (torch.float32, 96, 40, 4, True),         # 10 chunks per entry: second pass
 ])
 def test_compress_norm_rope(dt, n, c, m, overlap):
     B, R = 2, 64 if c >= 64 else 8

@@ -37,11 +37,11 @@ def _streams(B, n, c, m, dt, seed, overlap=True):
     (1, 1030, 136, 8, torch.bfloat16),    # 16 rows per entry: rows split over thread groups
     (2, 2048 + 64, 512, 64, torch.bfloat16),  # 128 rows: two rounds per thread
     (1, 512, 40, 16, torch.float32),      # fp32, 32 rows, 5 chunks
-    # bf16, c a multiple of 64: entry groups streamed by bulk copies
-    (2, 1030, 128, 4, torch.bfloat16),    # 16 entries a group, ragged last group
-    (3, 200, 64, 2, torch.bfloat16),      # 32 entries a group, three sequences
+    # bf16, one thread per (entry, 4 dims): entries across warps and blocks
+    (2, 1030, 128, 4, torch.bfloat16),    # 32 threads an entry, ragged tail rows
+    (3, 200, 64, 2, torch.bfloat16),      # 16 threads an entry, three sequences
     (1, 777, 256, 1, torch.bfloat16),     # m = 1 (DSA), two rows per entry
-    (2, 12, 512, 4, torch.bfloat16),      # fewer entries than a group
+    (2, 12, 512, 4, torch.bfloat16),      # fewer entries than a block holds
 ])
 def test_csa_compress_parity(B, n, c, m, dt):
     s = _streams(B, n, c, m, dt, seed=11)
@@ -61,8 +61,8 @@ def test_csa_compress_parity(B, n, c, m, dt):
     (1, 96, 16, 32, torch.bfloat16),
     (1, 2048 + 5, 264, 512, torch.bfloat16),  # 512 rows: eight rounds per thread, 33 chunks
     (2, 40, 24, 5, torch.bfloat16),       # odd m within one round
-    (2, 1000, 128, 8, torch.bfloat16),    # bulk-copied groups, eight rows per entry
-    (1, 130, 64, 1, torch.bfloat16),      # m = 1 through the bulk-copied groups: identity
+    (2, 1000, 128, 8, torch.bfloat16),    # eight own rows per entry, one thread each
+    (1, 130, 64, 1, torch.bfloat16),      # m = 1 through the per-thread rows: identity
 ])
 def test_hca_compress_parity(B, n, c, m, dt):
     s = _streams(B, n, c, m, dt, seed=12, overlap=False)
