@@ -11,13 +11,13 @@
 // one row.  Entries of at most eight rows (CSA m <= 4) take one thread per
 // (entry, 4-dim chunk): all of its rows are loaded at once (8 bytes of a
 // bf16 row per lane), then each dim takes a two-pass softmax over them in
-// registers with no data-dependent branch; 64 registers keep four blocks of
-// 256 threads per SM, and with them enough loads in flight to stream.
-// Larger row sets are split over R warps of one block, one thread per
-// (entry, 8-dim chunk, row group); a thread's rows are read in rounds of
-// four with all loads of a round issued before its arithmetic, and the R
-// partial states are merged through shared memory.  A
-// row whose logit equals the maximum gets weight 1 exactly, so a single +inf
+// registers, branch-free unless a maximum is infinite; 64 registers keep
+// four blocks of 256 threads per SM, and with them enough loads in flight
+// to stream.  Larger row sets are split over R warps of one block, one
+// thread per (entry, 8-dim chunk, row group); a thread's rows are read in
+// rounds of four with all loads of a round issued before its arithmetic,
+// and the R partial states are merged through shared memory.  A row whose
+// logit equals an infinite maximum gets weight 1 exactly, so a single +inf
 // logit selects its row.
 #include "common.cuh"
 #include "launch.h"
@@ -211,10 +211,10 @@ __device__ __forceinline__ void norm_rope4(float v[4], int d0, int c, float inv,
 
 // Softmax over the live rows of four dims: o[q] = sum_j w_j C_j[q] / sum_j w_j
 // with w_j = exp(l_j - max l), l_j = Z_j[q] + bias_j[q].  The logits are kept
-// in base-2 units; a row at the maximum weighs 1 exactly, which the plain
-// form gets from ex2(0) when every maximum is finite, and the guarded form
-// keeps for an infinite maximum (a +inf logit selects its row, all -inf
-// logits weigh alike).
+// in base-2 units.  When every maximum is finite the weights are ex2(l - max)
+// throughout; otherwise the guarded form gives the row at the maximum weight
+// 1 exactly (a +inf logit selects its row, all -inf logits weigh alike),
+// where l - max would be inf - inf.
 template <int kMaxRows, typename T, typename Bias>
 __device__ __forceinline__ void fold_rows4(const Raw4<T> (&cr)[kMaxRows],
                                            const Raw4<T> (&zr)[kMaxRows],
@@ -271,7 +271,8 @@ __device__ __forceinline__ void fold_rows4(const Raw4<T> (&cr)[kMaxRows],
 // Entries with at most eight rows, one thread per (entry, 4-dim chunk): all
 // rows of the thread are loaded at once (8 bytes of a bf16 row per lane, so a
 // warp reads 256 contiguous bytes of it), then each dim takes a two-pass
-// softmax over its rows in registers, with no data-dependent branch.
+// softmax over its rows in registers (branch-free unless a maximum is
+// infinite).
 template <typename T, bool kNorm>
 __global__ void __launch_bounds__(256, sizeof(T) == 2 ? 4 : 2) compress_rows_kernel(
     const T* __restrict__ ca, const T* __restrict__ cb, const T* __restrict__ za,
