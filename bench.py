@@ -425,12 +425,26 @@ def bench_hca_prefill(dev, K, W, peaks):
                          "hca_attn": roofline("flops", attn_flops, per[1], peaks)}}
 
 
-def _decode_layer(w: G.Decode, dev, steps):
+def _decode_layer(w: G.Decode, dev, steps, paged: bool = False):
+    """One decode layer's cache and per-step inputs.  ``paged``: the entries in
+    a pool of 128-token blocks behind a block table whose physical blocks are
+    in a seeded random order (the classical paged cache)."""
     import compressed_sparse_attention_11_b200 as csa
     inp = G.decode_inputs(w, steps=steps)
     E = w.t // w.m
-    cache = csa.CsaCache(w.batch, E + steps // w.m + 2, w.c, w.rope_dims, w.m, w.window, w.nh,
-                         w.is_hca, c_i=w.c_i, nh_i=w.nh_i, k=w.k, device=dev)
+    cap = E + steps // w.m + 2
+    if paged:
+        epb = 128 // w.m
+        nb = (cap + epb - 1) // epb
+        pool = w.batch * nb + 7
+        perm = torch.randperm(pool, generator=torch.Generator().manual_seed(17))[:w.batch * nb]
+        bt = perm.view(w.batch, nb).to(torch.int32).to(dev)
+        cache = csa.CsaCache(w.batch, cap, w.c, w.rope_dims, w.m, w.window, w.nh, w.is_hca,
+                             c_i=w.c_i, nh_i=w.nh_i, k=w.k, device=dev, block_table=bt,
+                             block_tokens=128, num_blocks=pool)
+    else:
+        cache = csa.CsaCache(w.batch, cap, w.c, w.rope_dims, w.m, w.window, w.nh, w.is_hca,
+                             c_i=w.c_i, nh_i=w.nh_i, k=w.k, device=dev)
     cache.store_entries(0, inp["cache_kv"].to(dev),
                         None if w.is_hca else inp["cache_ikey"].to(dev))
     names = ("ca", "za", "kv_win") if w.is_hca else \
@@ -469,10 +483,10 @@ def decode_bytes(w: G.Decode, t: int):
                 + 4 * w.c_i * 2)
 
 
-def bench_decode(layers, dev, K, W, peaks, name):
+def bench_decode(layers, dev, K, W, peaks, name, paged: bool = False):
     """Times `steps` consecutive decode positions (the last one emits), L2 flushed."""
     steps = 4
-    built = [_decode_layer(w, dev, steps) for w in layers]
+    built = [_decode_layer(w, dev, steps, paged) for w in layers]
     flush = torch.empty(512 << 20, dtype=torch.uint8, device=dev)
     times = []
     for it in range(W + K):
@@ -804,6 +818,10 @@ def main():
         torch.cuda.empty_cache()
         workloads["csa_decode"] = bench_decode([G.CSA_DECODE], dev, max(2, args.steps // 2),
                                                1, peaks, G.CSA_DECODE.name)
+        torch.cuda.empty_cache()
+        workloads["csa_decode_paged"] = bench_decode([G.CSA_DECODE], dev,
+                                                     max(2, args.steps // 2), 1, peaks,
+                                                     G.CSA_DECODE.name + "_paged128", paged=True)
         torch.cuda.empty_cache()
         workloads["mixed_decode"] = bench_decode([G.MIXED_DECODE_CSA, G.MIXED_DECODE_HCA], dev,
                                                  max(2, args.steps // 2), 1, peaks,
