@@ -425,6 +425,19 @@ def bench_hca_prefill(dev, K, W, peaks):
                          "hca_attn": roofline("flops", attn_flops, per[1], peaks)}}
 
 
+def paged_block_table(batch: int, capacity: int, m: int, block_tokens: int = 128,
+                      spare: int = 7, seed: int = 17):
+    """A block table (int32 [batch, blocks per sequence], on the host) over a
+    pool of batch * blocks + spare blocks of block_tokens tokens, enough for
+    `capacity` entries per sequence, the physical blocks in a seeded random
+    order (no two table slots share a block).  Returns (table, pool size)."""
+    epb = block_tokens // m
+    nb = (capacity + epb - 1) // epb
+    pool = batch * nb + spare
+    perm = torch.randperm(pool, generator=torch.Generator().manual_seed(seed))[:batch * nb]
+    return perm.view(batch, nb).to(torch.int32), pool
+
+
 def _decode_layer(w: G.Decode, dev, steps, paged: bool = False):
     """One decode layer's cache and per-step inputs.  ``paged``: the entries in
     a pool of 128-token blocks behind a block table whose physical blocks are
@@ -434,11 +447,8 @@ def _decode_layer(w: G.Decode, dev, steps, paged: bool = False):
     E = w.t // w.m
     cap = E + steps // w.m + 2
     if paged:
-        epb = 128 // w.m
-        nb = (cap + epb - 1) // epb
-        pool = w.batch * nb + 7
-        perm = torch.randperm(pool, generator=torch.Generator().manual_seed(17))[:w.batch * nb]
-        bt = perm.view(w.batch, nb).to(torch.int32).to(dev)
+        bt, pool = paged_block_table(w.batch, cap, w.m)
+        bt = bt.to(dev)
         cache = csa.CsaCache(w.batch, cap, w.c, w.rope_dims, w.m, w.window, w.nh, w.is_hca,
                              c_i=w.c_i, nh_i=w.nh_i, k=w.k, device=dev, block_table=bt,
                              block_tokens=128, num_blocks=pool)

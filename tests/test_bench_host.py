@@ -12,6 +12,7 @@ import os
 
 import numpy as np
 import pytest
+import torch
 
 import bench
 import oracle
@@ -89,3 +90,16 @@ def test_measured_traffic_follows_sources(monkeypatch):
     stale = dict(entry, sources=dict(entry["sources"], **{path: "0" * 16}))
     monkeypatch.setitem(bench.MEASURED_TRAFFIC, call, stale)
     assert bench.measured_traffic(call) is None
+
+
+@pytest.mark.parametrize("batch,cap,m", [(64, 32770, 4), (3, 1, 4), (2, 300, 128), (5, 97, 1)])
+def test_paged_block_table_is_a_partial_permutation(batch, cap, m):
+    """The paged decode workload's table: enough blocks per sequence for the
+    capacity, every physical block inside the pool and used at most once."""
+    bt, pool = bench.paged_block_table(batch, cap, m)
+    assert bt.dtype == torch.int32 and bt.shape[0] == batch
+    assert bt.shape[1] * (128 // m) >= cap > (bt.shape[1] - 1) * (128 // m)
+    flat = bt.flatten().tolist()
+    assert len(set(flat)) == len(flat)
+    assert min(flat) >= 0 and max(flat) < pool
+    assert pool == batch * bt.shape[1] + 7
