@@ -32,7 +32,7 @@ def _rank_main(rank, world, port, times, out):
 
 def test_two_gloo_ranks_take_the_slowest_time():
     world, times = 2, [12.5, 20.0]
-    with mp.Manager() as mgr:
+    with mp.get_context("spawn").Manager() as mgr:
         out = mgr.dict()
         mp.start_processes(_rank_main, args=(world, _free_port(), times, out), nprocs=world,
                            join=True, start_method="spawn")
