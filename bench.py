@@ -699,7 +699,7 @@ def run_profile_case(args):
             [G.MIXED_DECODE_CSA, G.MIXED_DECODE_HCA]
         if args.batch:
             layers = [dataclasses.replace(x, batch=args.batch) for x in layers]
-        built = [_decode_layer(x, dev, 4) for x in layers]
+        built = [_decode_layer(x, dev, 4, args.paged) for x in layers]
         for it in range(args.steps):
             for x, (cache, ps, biases, sink, out) in zip(layers, built):
                 st = ps[it % 4]
@@ -708,7 +708,7 @@ def run_profile_case(args):
     torch.cuda.synchronize()
     csa.csa_check()
     print(json.dumps({"profile": args.profile, "steps": args.steps, "n": args.n,
-                      "batch": args.batch, "ok": True}), flush=True)
+                      "batch": args.batch, "paged": args.paged, "ok": True}), flush=True)
 
 
 def main():
@@ -723,6 +723,8 @@ def main():
                     help="run --steps steps of one workload (for a profiler) and exit")
     ap.add_argument("--n", type=int, default=None, help="--profile prefill/hca/next: tokens")
     ap.add_argument("--batch", type=int, default=None, help="--profile decode_*: sequences")
+    ap.add_argument("--paged", action="store_true",
+                    help="--profile decode_*: entries in the paged 128-token-block cache")
     args = ap.parse_args()
     if args.impl == "reference":
         run_reference(args)
